@@ -1,0 +1,494 @@
+#!/usr/bin/env python
+"""Benchmark: KDA prefill tokens/s and decode tokens/s on one B200 (replicas for N > 1).
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill leg: kda_chunk_fwd over B=2 sequences x T=2048 tokens, H=32 heads,
+    dk = dv = 128, chunk 64, bf16 q/k/v/o, fp32 g/beta/state (steps a1-a4);
+  * decode leg: kda_decode_step for N=256 sequences x H=32 heads, 128 x 128 fp32
+    state updated in place (step a5); the 8 pre-drawn input sets are cycled.
+Each leg is timed with CUDA events on the stream it is launched on.  `value` is
+the prefill leg's tokens/s (sum of sequence lengths, not x heads); the decode
+leg's tokens/s (sequences x steps) is reported in `decode`.  L2 is flushed
+(a 256 MiB write) before each leg of each step, outside the leg's events.
+
+Multi-GPU: every rank runs an independent replica (no data-path collective;
+the path shards by sequence and head).  value = sum over ranks of the tokens
+divided by the max over ranks of the time.
+
+`--impl reference` times the fp64 CPU oracle (the correctness reference; there
+is no other implementation of this method to run) on the host cores, on a
+bounded sample of the same prefill workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s and decode tokens/s; % of tensor / HBM roofline (1 B200)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return d, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------- algorithmic cost
+
+def prefill_bytes(tokens_x_heads: int, n_seq_heads: int, dk=128, dv=128, in_bytes=2) -> int:
+    """q, k (dk) and v (dv) in the input dtype, g fp32 (dk), beta fp32, o (dv);
+    plus the initial and final state (fp32) once per (sequence, head)."""
+    per = in_bytes * (2 * dk + dv) + 4 * dk + 4 + in_bytes * dv
+    return tokens_x_heads * per + n_seq_heads * 2 * 4 * dk * dv
+
+
+def prefill_flops(tokens_x_heads: int, d=128, C=64) -> int:
+    """Per head and token: 6 d^2 + 3 C d + C^2 (Kimi Linear, aiwiki.ai, 'The
+    constrained DPLR form and the chunkwise algorithm', training cost)."""
+    return tokens_x_heads * (6 * d * d + 3 * C * d + C * C)
+
+
+def decode_bytes(units: int, dk=128, dv=128, in_bytes=2) -> int:
+    """State read + write (fp32) + q, k, v, o (input dtype) + g fp32 + beta."""
+    return units * (2 * 4 * dk * dv + in_bytes * (2 * dk + 2 * dv) + 4 * dk + 4)
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ ours
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_124_b200 as kda
+    from gated_delta_rule_124_b200 import workloads as wl
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    kda.load()
+
+    # ---- inputs (resident in HBM before timing)
+    pc = wl.prefill_config(1)
+    P = pc.to(dev)
+    dcase = wl.decode_config()
+    D = [{k: v.to(dev) for k, v in s.items()} for s in dcase.steps]
+    state = dcase.state0.to(dev)
+    Np, H, dk, dv, C = P.N, P.H, P.dk, P.dv, P.chunk
+    total = P.total
+    ws = kda.alloc_workspace(total, Np, H, dk, dv, C, "bf16", dev)
+    o = torch.empty_like(P.v)
+    hN = torch.empty(Np, H, dk, dv, dtype=torch.float32, device=dev)
+    Nd = dcase.N
+    od = torch.empty(Nd, H, dv, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def prefill():
+        kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, None, P.B, P.T, Np, H,
+                          dk, dv, C, "bf16", o, hN, ws)
+
+    def decode(i):
+        s = D[i % len(D)]
+        kda.kda_decode_step(s["q"], s["k"], s["v"], s["g"], s["beta"], state, od, Nd, H, dk,
+                            dv, "bf16")
+
+    def step(i, ev=None):
+        flush.zero_()
+        if ev: ev[0].record(stream)
+        prefill()
+        if ev: ev[1].record(stream)
+        flush.zero_()
+        if ev: ev[2].record(stream)
+        decode(i)
+        if ev: ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    pre_sum, dec_sum = sum(pre_ms), sum(dec_ms)
+
+    # ---- max over ranks (device time)
+    if world > 1:
+        t = torch.tensor([total_ms, pre_sum, dec_sum], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, pre_sum, dec_sum = t.tolist()
+
+    pre_tokens = total * world * args.steps
+    dec_tokens = Nd * world * args.steps
+    value = pre_tokens / (pre_sum / 1e3)
+    dec_value = dec_tokens / (dec_sum / 1e3)
+
+    # ---- per-kernel times of the prefill (dominant kernel) with the step calls
+    kern = prefill_kernel_times(kda, P, ws, dev, stream, reps=max(5, min(50, args.steps)))
+
+    # ---- end to end through host buffers (pinned), copies inside the region
+    e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=max(3, min(args.steps, 50)))
+
+    peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tx = total * H
+    pb = prefill_bytes(tx, Np * H)
+    pf = prefill_flops(tx)
+    pre_avg = pre_sum / args.steps / 1e3  # s
+    dom_name, dom_s = kern["dominant"]
+    # roofline of the dominant prefill kernel: its share of the algorithmic bytes
+    dom_bytes = kern["bytes"][dom_name]
+    roof = {"kernel": dom_name, "bound": "hbm", "achieved": dom_bytes / dom_s / 1e9,
+            "peak": hbm, "unit": "GB/s", "frac": dom_bytes / dom_s / 1e9 / hbm,
+            "traffic": None, "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+            "per_launch_us": dom_s * 1e6, "algorithmic_bytes_per_launch": dom_bytes}
+    dec_avg = dec_sum / args.steps / 1e3
+    db = decode_bytes(Nd * H)
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; distributions of the pages' configurations)",
+        "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": H, "dk": dk, "dv": dv,
+                   "chunk": C, "decode_workload": dcase.name,
+                   "l2": "flushed (256 MiB write) before each leg",
+                   "parallelism": f"replicas x{world}"},
+        "prefill": {"value": value, "unit": "tokens/s", "ms_per_call": pre_avg * 1e3,
+                    "hbm_frac": pb / pre_avg / 1e9 / hbm,
+                    "tensor_frac": pf / pre_avg / 1e12 / peaks["bf16_tflops"],
+                    "algorithmic_bytes": pb, "paper_flops": pf,
+                    "kernels_us": {k: v * 1e6 for k, v in kern["times"].items()}},
+        "decode": {"value": dec_value, "unit": "tokens/s", "ms_per_step": dec_avg * 1e3,
+                   "roofline": {"bound": "hbm", "achieved": db / dec_avg / 1e9, "peak": hbm,
+                                "unit": "GB/s", "frac": db / dec_avg / 1e9 / hbm,
+                                "traffic": None, "algorithmic_bytes_per_launch": db}},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": args.steps * (kern["launches_per_call"] + 1),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(pc, seconds=args.cpu_seconds)
+    return res
+
+
+def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
+    """Times of the prefill kernels.  For the CUDA-core path: each step call
+    (a1..a4) on its own; for the tensor-core path: the single fused kernel is
+    the whole call."""
+    import torch
+    Np, H, dk, dv, C, total = P.N, P.H, P.dk, P.dv, P.chunk, P.total
+    tc = kda.kda_chunk_fwd_workspace_size(total, Np, H, dk, dv, C, "bf16") < \
+        kda.kda_chunk_fwd_workspace_size(total, Np, H, dk, dv, C, "f32")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    in_b = 2
+    if tc:
+        o = torch.empty_like(P.v)
+        hN = torch.empty(Np, H, dk, dv, device=dev)
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, None, P.B, P.T, Np,
+                              H, dk, dv, C, "bf16", o, hN, ws)
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        t = statistics.median(a.elapsed_time(b) for a, b in ts) / 1e3
+        nb = prefill_bytes(total * H, Np * H)
+        return {"times": {"chunk_fwd_tc": t}, "bytes": {"chunk_fwd_tc": nb},
+                "dominant": ("chunk_fwd_tc", t), "launches_per_call": 2}
+    G = torch.empty(total, H, dk, device=dev)
+    W = torch.empty(total, H, dk, device=dev)
+    U = torch.empty(total, H, dv, device=dev)
+    maxc = kda.kda_num_chunks_upper_bound(total, Np, C)
+    S = torch.empty(maxc, H, dk, dv, device=dev)
+    hN = torch.empty(Np, H, dk, dv, device=dev)
+    o = torch.empty_like(P.v)
+    a = (None, P.B, P.T, Np, H)
+    calls = {
+        "a1_gate_cumsum": lambda: kda.kda_chunk_gate_cumsum(P.g, *a, dk, C, G, ws),
+        "a2_intra": lambda: kda.kda_chunk_intra(P.k, P.v, G, P.beta, *a, dk, dv, C, "bf16", W,
+                                                U, ws),
+        "a3_inter": lambda: kda.kda_chunk_inter(P.k, G, W, U, P.initial_state, *a, dk, dv, C,
+                                                "bf16", S, hN, ws),
+        "a4_output": lambda: kda.kda_chunk_output(P.q, P.k, G, U, S, *a, dk, dv, C, "bf16", o,
+                                                  ws),
+    }
+    tx = total * H
+    nbytes = {
+        "a1_gate_cumsum": tx * dk * 8,
+        "a2_intra": tx * (in_b * (dk + dv) + 4 * dk + 4 + 4 * (dk + dv)),
+        "a3_inter": tx * (in_b * dk + 4 * dk + 4 * dk + 8 * dv) + maxc * H * dk * dv * 4,
+        "a4_output": tx * (in_b * 2 * dk + 4 * dk + 4 * dv + in_b * dv) + maxc * H * dk * dv * 4,
+    }
+    times = {}
+    for name in calls:
+        ts = []
+        for _ in range(reps):
+            for n2, f in calls.items():  # run the whole sequence so inputs are valid
+                if n2 == name:
+                    flush.zero_()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    f()
+                    e1.record(stream)
+                    ts.append((e0, e1))
+                else:
+                    f()
+        torch.cuda.synchronize()
+        # each step call also launches the chunk-table kernel; it is included
+        times[name] = statistics.median(x.elapsed_time(y) for x, y in ts) / 1e3
+    dom = max(times, key=times.get)
+    return {"times": times, "bytes": nbytes, "dominant": (dom, times[dom]),
+            "launches_per_call": 5}
+
+
+def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
+    """Prefill through the public call with pinned host buffers: H2D of the
+    inputs, kda_chunk_fwd, D2H of o and the final state -- all inside the
+    events; the same for one decode step (state resident on the device)."""
+    pin = lambda t: None if t is None else t.pin_memory()
+    hq, hk, hv, hg, hb, h0 = map(pin, (pc.q, pc.k, pc.v, pc.g, pc.beta, pc.initial_state))
+    dq, dk_, dv_, dg, db, d0 = (torch.empty_like(x, device=dev) for x in (hq, hk, hv, hg, hb, h0))
+    H, dk, dv, C, N, total = pc.H, pc.dk, pc.dv, pc.chunk, pc.N, pc.total
+    o = torch.empty_like(dv_)
+    hN = torch.empty(N, H, dk, dv, device=dev)
+    ho = torch.empty_like(hv).pin_memory()
+    hhN = torch.empty(N, H, dk, dv).pin_memory()
+    ws = kda.alloc_workspace(total, N, H, dk, dv, C, "bf16", dev)
+
+    def one():
+        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (d0, h0)):
+            d.copy_(h, non_blocking=True)
+        kda.kda_chunk_fwd(dq, dk_, dv_, dg, db, d0, None, pc.B, pc.T, N, H, dk, dv, C, "bf16",
+                          o, hN, ws)
+        ho.copy_(o, non_blocking=True)
+        hhN.copy_(hN, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3 / steps
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb, h0))
+    d2h = ho.numel() * ho.element_size() + hhN.numel() * hhN.element_size()
+
+    # decode: per step the token's inputs go up and o comes back
+    s0 = dcase.steps[0]
+    hs = {k: v.pin_memory() for k, v in s0.items()}
+    ds = {k: torch.empty_like(v, device=dev) for k, v in hs.items()}
+    state = dcase.state0.to(dev)
+    od = torch.empty(dcase.N, H, dv, dtype=torch.bfloat16, device=dev)
+    hod = torch.empty_like(od, device="cpu").pin_memory()
+
+    def dec():
+        for kname in ds:
+            ds[kname].copy_(hs[kname], non_blocking=True)
+        kda.kda_decode_step(ds["q"], ds["k"], ds["v"], ds["g"], ds["beta"], state, od, dcase.N,
+                            H, dk, dv, "bf16")
+        hod.copy_(od, non_blocking=True)
+
+    for _ in range(2):
+        dec()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        dec()
+    b.record(stream)
+    torch.cuda.synchronize()
+    td = a.elapsed_time(b) / 1e3 / steps
+    dh2d = sum(x.numel() * x.element_size() for x in hs.values())
+    return {"value": total / t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "decode": {"value": dcase.N / td, "unit": "tokens/s", "h2d_bytes_per_step": dh2d,
+                       "d2h_bytes_per_step": hod.numel() * hod.element_size()}}
+
+
+# ------------------------------------------------------------- cpu baseline
+
+def cpu_baseline(pc, seconds=15.0, heads=None):
+    """The fp64 oracle (as it stands) on the host cores, on a bounded sample of
+    the prefill workload.  With `heads` given: the first sequence, first
+    `heads` heads, once.  Otherwise the whole workload (all sequences and
+    heads), repeated until about `seconds` of CPU time have run.  Reported as
+    tokens/s of the full workload (head-tokens/s / H)."""
+    import oracle
+    cores = oracle.max_threads()
+    H = pc.H
+    if heads is not None:
+        T = pc.T
+        t = time.perf_counter()
+        oracle.forward(pc.q[:T, :heads], pc.k[:T, :heads], pc.v[:T, :heads], pc.g[:T, :heads],
+                       pc.beta[:T, :heads], pc.initial_state[:1, :heads], num_threads=cores)
+        el = time.perf_counter() - t
+        return {"value": T * heads / el / H, "unit": "tokens/s", "cores": cores,
+                "kind": "oracle", "sample": f"1 sequence x {T} tokens x {heads} of {H} heads, "
+                                            f"fp64 token recurrence, {el:.1f} s"}
+    cu = pc.cu_host()
+    reps, el = 0, 0.0
+    while el < seconds:
+        t = time.perf_counter()
+        oracle.forward(pc.q, pc.k, pc.v, pc.g, pc.beta, pc.initial_state, cu_seqlens=cu,
+                       num_threads=cores)
+        el += time.perf_counter() - t
+        reps += 1
+    return {"value": pc.total * reps / el, "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"whole prefill workload ({pc.N} x {pc.T} tokens x {H} heads) x {reps} "
+                      f"repetitions, fp64 token recurrence, {el:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from gated_delta_rule_124_b200 import workloads as wl
+    pc = wl.prefill_config(1)
+    for _ in range(args.warmup):
+        cpu_baseline(pc, heads=1)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_baseline(pc, heads=max(1, min(pc.H, args.ref_heads)))
+        vals.append(r["value"])
+    el = time.perf_counter() - t0
+    v = statistics.median(vals)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": pc.H, "dk": pc.dk,
+                       "dv": pc.dv, "chunk": pc.chunk},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"],
+                             "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-heads", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world, local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

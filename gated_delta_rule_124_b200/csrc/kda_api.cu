@@ -1,0 +1,254 @@
+// C ABI of libkda: argument validation, workspace layout and launch order.
+// Everything here runs on the host and only enqueues work; see include/kda.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <initializer_list>
+
+#include "kda.h"
+#include "kda_common.cuh"
+#include "kda_chunk_tc.cuh"
+
+namespace {
+
+using kda::Workspace;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
+bool dtype_ok(kda_dtype_t t) { return t == KDA_DTYPE_F32 || t == KDA_DTYPE_BF16; }
+
+// Shapes and sequence description shared by every prefill entry point.
+struct Prefill {
+    int total, N;
+};
+
+kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, int H, int dk,
+                                  int dv, int chunk, kda_dtype_t dt, Prefill* out) {
+    if (B < 1 || T < 0 || num_seqs < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return KDA_ERR_INVALID_ARG;
+    if (cu) {
+        if (B != 1) return KDA_ERR_INVALID_ARG;
+        if (!aligned16(cu)) return KDA_ERR_INVALID_ARG;
+        out->total = T;
+        out->N = num_seqs;
+    } else {
+        if (num_seqs != B) return KDA_ERR_INVALID_ARG;
+        if ((long long)B * T > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+        out->total = B * T;
+        out->N = B;
+    }
+    if (!dim_ok(dk) || !dim_ok(dv) || !chunk_ok(chunk)) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+bool use_tc_path(int dk, int dv, int chunk, kda_dtype_t dt) {
+    return kda::tc_path_available() && dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 &&
+           chunk == 64;
+}
+
+size_t workspace_bytes_for(int total, int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
+    const bool inter = !use_tc_path(dk, dv, chunk, dt);
+    Workspace w = kda::carve(nullptr, total, N, H, dk, dv, chunk, inter);
+    return w.total_bytes;
+}
+
+kda_status_t check_ws(void* ws, size_t bytes, const Prefill& p, int H, int dk, int dv,
+                      int chunk, kda_dtype_t dt, Workspace* out, bool need_intermediates) {
+    if (!ws) return KDA_ERR_WORKSPACE;
+    if (!aligned256(ws)) return KDA_ERR_INVALID_ARG;
+    Workspace w = kda::carve(ws, p.total, p.N, H, dk, dv, chunk, need_intermediates);
+    if (bytes < w.total_bytes) return KDA_ERR_WORKSPACE;
+    *out = w;
+    return KDA_OK;
+}
+
+kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Reset the status word and build the chunk table (two stream operations).
+kda_status_t begin_prefill(const Workspace& w, const int32_t* cu, int B, int T, int N, int chunk,
+                           int maxc, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    e = kda::launch_build_chunk_table(cu, B, T, N, chunk, maxc, w.status, w.chunk_start,
+                                      w.chunk_info, st);
+    return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status_t s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: shape or dtype not supported";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+        case KDA_ERR_BAD_SEQLENS:
+            return "KDA_ERR_BAD_SEQLENS: cu_seqlens is not 0..T non-decreasing";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int kda_num_chunks_upper_bound(int total_tokens, int num_seqs, int chunk) {
+    if (total_tokens < 0 || num_seqs < 1 || chunk < 1) return 0;
+    return kda::max_chunks(total_tokens, num_seqs, chunk);
+}
+
+size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
+                                    int chunk, kda_dtype_t dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
+        !chunk_ok(chunk) || !dtype_ok(dtype))
+        return 0;
+    return workspace_bytes_for(total_tokens, num_seqs, H, dk, dv, chunk, dtype);
+}
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                           int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                           float* final_state, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    Prefill p;
+    kda_status_t s =
+        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);
+    if (s != KDA_OK) return s;
+    if (!q || !k || !v || !g || !beta || !o) return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : {q, k, v, (const void*)g, (const void*)beta, (const void*)o})
+        if (!aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    const bool tc = use_tc_path(dk, dv, chunk, dtype);
+    Workspace w;
+    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, dtype, &w, !tc);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int maxc = kda::max_chunks(p.total, p.N, chunk);
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);
+    if (s != KDA_OK) return s;
+    if (p.total == 0 && !final_state) return KDA_OK;
+    if (tc) {
+        return from_cuda(kda::launch_chunk_fwd_tc(q, k, v, g, beta, initial_state, cu_seqlens,
+                                                  T, p.N, H, w.chunk_start, w.status, o,
+                                                  final_state, st));
+    }
+    cudaError_t e = kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
+    if (e == cudaSuccess)
+        e = kda::launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, chunk, dtype,
+                              w.status, w.W, w.U, st);
+    if (e == cudaSuccess)
+        e = kda::launch_inter(k, w.G, w.W, w.U, initial_state, cu_seqlens, B, T, p.N,
+                              w.chunk_start, H, dk, dv, chunk, dtype, w.status, w.states,
+                              final_state, st);
+    if (e == cudaSuccess)
+        e = kda::launch_output(q, k, w.G, w.U, w.states, w.chunk_info, maxc, H, dk, dv, chunk,
+                               dtype, w.status, o, st);
+    return from_cuda(e);
+}
+
+// ------------------------------------------------- one step per call (a1-a4)
+
+#define KDA_PREFILL_PROLOGUE(...)                                                   \
+    Prefill p;                                                                            \
+    kda_status_t s =                                                                      \
+        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);     \
+    if (s != KDA_OK) return s;                                                            \
+    for (const void* ptr : std::initializer_list<const void*>{__VA_ARGS__})              \
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;                          \
+    Workspace w;                                                                          \
+    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, dtype, &w, false);      \
+    if (s != KDA_OK) return s;                                                            \
+    cudaStream_t st = static_cast<cudaStream_t>(stream);                                  \
+    const int maxc = kda::max_chunks(p.total, p.N, chunk);
+
+// First enqueue of a step call; every argument check must come before it.
+#define KDA_PREFILL_BEGIN()                                                               \
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);                         \
+    if (s != KDA_OK) return s;
+
+kda_status_t kda_chunk_gate_cumsum(const float* g, const int32_t* cu_seqlens, int B, int T,
+                                   int num_seqs, int H, int dk, int chunk, float* G,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    const int dv = dk;
+    const kda_dtype_t dtype = KDA_DTYPE_F32;
+    KDA_PREFILL_PROLOGUE((const void*)g, (const void*)G)
+    KDA_PREFILL_BEGIN()
+    return from_cuda(kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, G, st));
+}
+
+kda_status_t kda_chunk_intra(const void* k, const void* v, const float* G, const float* beta,
+                             const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                             int dk, int dv, int chunk, kda_dtype_t dtype, float* W, float* Ut,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    KDA_PREFILL_PROLOGUE(k, v, (const void*)G, (const void*)beta, (const void*)W,
+                         (const void*)Ut)
+    KDA_PREFILL_BEGIN()
+    return from_cuda(kda::launch_intra(k, v, G, beta, w.chunk_info, maxc, H, dk, dv, chunk,
+                                       dtype, w.status, W, Ut, st));
+}
+
+kda_status_t kda_chunk_inter(const void* k, const float* G, const float* W, float* U,
+                             const float* initial_state, const int32_t* cu_seqlens, int B,
+                             int T, int num_seqs, int H, int dk, int dv, int chunk,
+                             kda_dtype_t dtype, float* chunk_states, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    KDA_PREFILL_PROLOGUE(k, (const void*)G, (const void*)W, (const void*)U,
+                         (const void*)chunk_states)
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    KDA_PREFILL_BEGIN()
+    return from_cuda(kda::launch_inter(k, G, W, U, initial_state, cu_seqlens, B, T, p.N,
+                                       w.chunk_start, H, dk, dv, chunk, dtype, w.status,
+                                       chunk_states, final_state, st));
+}
+
+kda_status_t kda_chunk_output(const void* q, const void* k, const float* G, const float* U,
+                              const float* chunk_states, const int32_t* cu_seqlens, int B,
+                              int T, int num_seqs, int H, int dk, int dv, int chunk,
+                              kda_dtype_t dtype, void* o, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    KDA_PREFILL_PROLOGUE(q, k, (const void*)G, (const void*)U, (const void*)chunk_states,
+                         (const void*)o)
+    KDA_PREFILL_BEGIN()
+    return from_cuda(kda::launch_output(q, k, G, U, chunk_states, w.chunk_info, maxc, H, dk, dv,
+                                        chunk, dtype, w.status, o, st));
+}
+
+#undef KDA_PREFILL_PROLOGUE
+#undef KDA_PREFILL_BEGIN
+
+// ----------------------------------------------------------------- decode
+
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, float* state, void* o, int N, int H, int dk,
+                             int dv, kda_dtype_t dtype, void* stream) {
+    if (N < 0 || H < 1 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    for (const void* ptr : {q, k, v, (const void*)g, (const void*)beta, (const void*)state,
+                            (const void*)o})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_decode(q, k, v, g, beta, state, o, N, H, dk, dv, dtype,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+// ----------------------------------------------------------------- status
+
+kda_status_t kda_get_device_status(void* workspace, void* stream) {
+    if (!workspace || !aligned256(workspace)) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    if (word & kda::STATUS_BAD_SEQLENS) return KDA_ERR_BAD_SEQLENS;
+    if (word & kda::STATUS_TIMEOUT) return KDA_ERR_TIMEOUT;
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,18 @@
+// Tensor-core (tcgen05 / TMEM / TMA) chunkwise prefill for bf16, dk = dv = 128,
+// chunk = 64.  Internal to libkda.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+// True when the tensor-core prefill kernel is compiled into this library.
+bool tc_path_available();
+
+cudaError_t launch_chunk_fwd_tc(const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, const float* h0, const int32_t* cu_seqlens,
+                                int T, int N, int H, const int* chunk_start,
+                                uint32_t* status, void* o, float* hN, cudaStream_t st);
+
+}  // namespace kda

@@ -1,0 +1,121 @@
+// Shared device helpers of libkda (not part of the public ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// ---------------------------------------------------------------- workspace
+// Layout of the caller's workspace (all offsets 256-byte aligned):
+//   [0, 256)              status word (uint32 at offset 0) + padding
+//   chunk_start[N + 1]    int32: global index of each sequence's first chunk
+//   chunk_info[maxc]      int4 {seq, first token, rows, chunk-in-sequence};
+//                         unused slots hold seq = -1, rows = 0
+//   then, for the CUDA-core path only: G, W, U (token-major fp32) and the
+//   per-chunk states [maxc, H, dk, dv] fp32.
+constexpr size_t kAlign = 256;
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a = kAlign) {
+    return (x + a - 1) / a * a;
+}
+
+// Device status bits (OR-ed by kernels; the first error wins on the host).
+enum : uint32_t { STATUS_BAD_SEQLENS = 1u, STATUS_TIMEOUT = 2u };
+
+struct Workspace {
+    uint32_t* status;
+    int* chunk_start;
+    int4* chunk_info;
+    float* G;
+    float* W;
+    float* U;
+    float* states;
+    size_t header_bytes;  // status + tables
+    size_t total_bytes;   // header + CUDA-core path intermediates
+};
+
+inline int max_chunks(int total_tokens, int num_seqs, int chunk) {
+    // sum_s ceil(len_s / C) <= (total + N (C - 1)) / C
+    return (int)(((long long)total_tokens + (long long)num_seqs * (chunk - 1)) / chunk);
+}
+
+inline Workspace carve(void* base, int total, int N, int H, int dk, int dv, int chunk,
+                       bool with_intermediates) {
+    Workspace w{};
+    const int maxc = max_chunks(total, N, chunk);
+    char* p = static_cast<char*>(base);
+    size_t off = 0;
+    w.status = reinterpret_cast<uint32_t*>(p + off);
+    off += kAlign;
+    w.chunk_start = reinterpret_cast<int*>(p + off);
+    off = align_up(off + sizeof(int) * (size_t)(N + 1));
+    w.chunk_info = reinterpret_cast<int4*>(p + off);
+    off = align_up(off + sizeof(int4) * (size_t)maxc);
+    w.header_bytes = off;
+    if (with_intermediates) {
+        w.G = reinterpret_cast<float*>(p + off);
+        off = align_up(off + sizeof(float) * (size_t)total * H * dk);
+        w.W = reinterpret_cast<float*>(p + off);
+        off = align_up(off + sizeof(float) * (size_t)total * H * dk);
+        w.U = reinterpret_cast<float*>(p + off);
+        off = align_up(off + sizeof(float) * (size_t)total * H * dv);
+        w.states = reinterpret_cast<float*>(p + off);
+        off = align_up(off + sizeof(float) * (size_t)maxc * H * dk * dv);
+    }
+    w.total_bytes = off;
+    return w;
+}
+
+// ------------------------------------------------------------- conversions
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ bool status_bad(const uint32_t* status) {
+    return *reinterpret_cast<const volatile uint32_t*>(status) != 0u;
+}
+
+}  // namespace kda
+
+// Launchers implemented in the .cu files (host side, return cudaError_t).
+namespace kda {
+cudaError_t launch_build_chunk_table(const int32_t* cu_seqlens, int B, int T, int N, int chunk,
+                                     int maxc, uint32_t* status, int* chunk_start,
+                                     int4* chunk_info, cudaStream_t st);
+cudaError_t launch_gate_cumsum(const float* g, const int4* info, int maxc, int H, int dk,
+                               const uint32_t* status, float* G, cudaStream_t st);
+cudaError_t launch_intra(const void* k, const void* v, const float* G, const float* beta,
+                         const int4* info, int maxc, int H, int dk, int dv, int chunk,
+                         kda_dtype_t dt, const uint32_t* status, float* W, float* U,
+                         cudaStream_t st);
+cudaError_t launch_inter(const void* k, const float* G, const float* W, float* U,
+                         const float* h0, const int32_t* cu_seqlens, int B, int T, int N,
+                         const int* chunk_start, int H, int dk, int dv, int chunk,
+                         kda_dtype_t dt, const uint32_t* status, float* states, float* hN,
+                         cudaStream_t st);
+cudaError_t launch_output(const void* q, const void* k, const float* G, const float* U,
+                          const float* states, const int4* info, int maxc, int H, int dk,
+                          int dv, int chunk, kda_dtype_t dt, const uint32_t* status, void* o,
+                          cudaStream_t st);
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, float* state, void* o, int N, int H, int dk,
+                          int dv, kda_dtype_t dt, cudaStream_t st);
+}  // namespace kda

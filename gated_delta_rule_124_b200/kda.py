@@ -1,0 +1,245 @@
+"""Thin ctypes binding of libkda.so (see include/kda.h).
+
+Argument marshalling only: every function here passes device pointers, sizes
+and the current CUDA stream to the C ABI, and every step of the computation
+runs in the library's CUDA kernels.  There is no CPU fallback: if libkda.so
+cannot be loaded, every call raises :class:`KdaError`.
+
+Functions with the C names take tensors that are already allocated (device
+tensors from PyTorch) and return the status code, raising :class:`KdaError`
+on anything but ``KDA_OK`` unless ``check=False``.  :func:`chunk_fwd` and
+:func:`decode_step` are convenience wrappers that allocate outputs and the
+workspace with PyTorch and then make the same calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = 1
+KDA_ERR_UNSUPPORTED = 2
+KDA_ERR_CUDA = 3
+KDA_ERR_TIMEOUT = 4
+KDA_ERR_WORKSPACE = 5
+KDA_ERR_BAD_SEQLENS = 6
+
+KDA_DTYPE_F32 = 0
+KDA_DTYPE_BF16 = 1
+
+# Every symbol include/kda.h declares.
+EXPORTS = (
+    "kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
+    "kda_num_chunks_upper_bound", "kda_chunk_gate_cumsum", "kda_chunk_intra",
+    "kda_chunk_inter", "kda_chunk_output", "kda_decode_step", "kda_get_device_status",
+)
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        super().__init__(f"{what}: {status_string(status)}" if what else status_string(status))
+
+
+_lib = None
+_lock = threading.Lock()
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "kda_status_string": ([_i], ctypes.c_char_p),
+    "kda_chunk_fwd_workspace_size": ([_i, _i, _i, _i, _i, _i, _i], _sz),
+    "kda_num_chunks_upper_bound": ([_i, _i, _i], _i),
+    "kda_chunk_fwd": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_chunk_gate_cumsum": ([_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _sz, _vp], _i),
+    "kda_chunk_intra": ([_vp] * 5 + [_i] * 8 + [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_chunk_inter": ([_vp] * 6 + [_i] * 8 + [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_chunk_output": ([_vp] * 6 + [_i] * 8 + [_vp, _vp, _sz, _vp], _i),
+    "kda_decode_step": ([_vp] * 7 + [_i] * 5 + [_vp], _i),
+    "kda_get_device_status": ([_vp, _vp], _i),
+}
+
+
+def load(path: str = LIB_PATH):
+    """Load libkda.so (once).  Raises KdaError if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise KdaError(KDA_ERR_CUDA, f"libkda.so not found at {path}; run "
+                               "`python -m gated_delta_rule_124_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (args, res) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load().kda_status_string(int(status)).decode()
+    except KdaError:
+        return f"status {status}"
+
+
+def _p(t) -> int | None:
+    """Device pointer of a tensor (or None for NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        if not torch.cuda.is_available():
+            return None
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def dtype_code(dtype) -> int:
+    if dtype in (torch.bfloat16, "bf16", KDA_DTYPE_BF16):
+        return KDA_DTYPE_BF16
+    if dtype in (torch.float32, "f32", KDA_DTYPE_F32):
+        return KDA_DTYPE_F32
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def _ret(st: int, what: str, check: bool) -> int:
+    if check and st != KDA_OK:
+        raise KdaError(st, what)
+    return st
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+# ------------------------------------------------------------- C-named calls
+
+def kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype) -> int:
+    return int(load().kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk,
+                                                   dtype_code(dtype)))
+
+
+def kda_num_chunks_upper_bound(total_tokens, num_seqs, chunk) -> int:
+    return int(load().kda_num_chunks_upper_bound(total_tokens, num_seqs, chunk))
+
+
+def kda_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H, dk, dv,
+                  chunk, dtype, o, final_state, workspace, workspace_bytes=None, stream=None,
+                  check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
+                              _p(cu_seqlens), B, T, num_seqs, H, dk, dv, chunk,
+                              dtype_code(dtype), _p(o), _p(final_state), _p(workspace), wb,
+                              _stream(stream))
+    return _ret(st, "kda_chunk_fwd", check)
+
+
+def kda_chunk_gate_cumsum(g, cu_seqlens, B, T, num_seqs, H, dk, chunk, G, workspace,
+                          workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_gate_cumsum(_p(g), _p(cu_seqlens), B, T, num_seqs, H, dk, chunk,
+                                      _p(G), _p(workspace), wb, _stream(stream))
+    return _ret(st, "kda_chunk_gate_cumsum", check)
+
+
+def kda_chunk_intra(k, v, G, beta, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, W, Ut,
+                    workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_intra(_p(k), _p(v), _p(G), _p(beta), _p(cu_seqlens), B, T, num_seqs,
+                                H, dk, dv, chunk, dtype_code(dtype), _p(W), _p(Ut),
+                                _p(workspace), wb, _stream(stream))
+    return _ret(st, "kda_chunk_intra", check)
+
+
+def kda_chunk_inter(k, G, W, U, initial_state, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk,
+                    dtype, chunk_states, final_state, workspace, workspace_bytes=None,
+                    stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_inter(_p(k), _p(G), _p(W), _p(U), _p(initial_state), _p(cu_seqlens),
+                                B, T, num_seqs, H, dk, dv, chunk, dtype_code(dtype),
+                                _p(chunk_states), _p(final_state), _p(workspace), wb,
+                                _stream(stream))
+    return _ret(st, "kda_chunk_inter", check)
+
+
+def kda_chunk_output(q, k, G, U, chunk_states, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk,
+                     dtype, o, workspace, workspace_bytes=None, stream=None,
+                     check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_output(_p(q), _p(k), _p(G), _p(U), _p(chunk_states), _p(cu_seqlens),
+                                 B, T, num_seqs, H, dk, dv, chunk, dtype_code(dtype), _p(o),
+                                 _p(workspace), wb, _stream(stream))
+    return _ret(st, "kda_chunk_output", check)
+
+
+def kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,
+                    check=True) -> int:
+    st = load().kda_decode_step(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state), _p(o), N, H,
+                                dk, dv, dtype_code(dtype), _stream(stream))
+    return _ret(st, "kda_decode_step", check)
+
+
+def kda_get_device_status(workspace, stream=None) -> int:
+    return int(load().kda_get_device_status(_p(workspace), _stream(stream)))
+
+
+# ------------------------------------------------------- allocating wrappers
+
+def alloc_workspace(total_tokens, num_seqs, H, dk, dv, chunk, dtype, device="cuda"):
+    n = kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype)
+    if n == 0:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
+              output_final_state=True, workspace=None, stream=None):
+    """KDA chunkwise forward.  q, k [B, T, H, dk] or [T_total, H, dk] (packed with
+    cu_seqlens); v likewise with dv; g like q (fp32); beta [.., H] (fp32).
+    Returns (o, final_state or None).  All tensors on the current CUDA device."""
+    packed = q.dim() == 3
+    if packed:
+        total, H, dk = q.shape
+        B, T = 1, total
+        N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+        if cu_seqlens is None:
+            B, T = 1, total
+    else:
+        B, T, H, dk = q.shape
+        total, N = B * T, B
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens needs packed [T_total, H, d] inputs")
+    dv = v.shape[-1]
+    o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    hN = (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+          if output_final_state else None)
+    if workspace is None:
+        workspace = alloc_workspace(total, N, H, dk, dv, chunk, q.dtype, q.device)
+    kda_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, N, H, dk, dv, chunk,
+                  q.dtype, o, hN, workspace, stream=stream)
+    return o, hN
+
+
+def decode_step(q, k, v, g, beta, state, o=None, stream=None):
+    """One recurrent step.  q, k, g [N, H, dk]; v [N, H, dv]; beta [N, H];
+    state [N, H, dk, dv] fp32, updated in place.  Returns o [N, H, dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=v.dtype, device=v.device)
+    kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, q.dtype, stream=stream)
+    return o

@@ -1,0 +1,192 @@
+/*
+ * kda.h -- C ABI of libkda.so: Kimi Delta Attention (KDA) on one NVIDIA B200.
+ *
+ * KDA (Kimi Linear, aiwiki.ai, section "Kimi Delta Attention") is the gated
+ * delta rule with the scalar forget gate replaced by a diagonal, per-channel
+ * gate.  Per (sequence, head) it carries a state S of dk x dv floats and, for
+ * each token t,
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t,            alpha_t = exp(g_t) per key channel.
+ *
+ * In the diagonal-plus-low-rank reading (section "The constrained DPLR form
+ * and the chunkwise algorithm") the transition is Diag(alpha) - a b^T with
+ * a = beta k and b = alpha * k.  Prefill evaluates this chunk by chunk (WY
+ * representation + UT transform inside a chunk, a carried state between
+ * chunks); decode applies one token to a resident state.
+ *
+ * ---------------------------------------------------------------- conventions
+ * Pointers:   every tensor pointer is a DEVICE pointer unless stated, must be
+ *             16-byte aligned, and is owned by the caller.  The library never
+ *             allocates, frees or keeps memory, never synchronises a stream
+ *             (except kda_get_device_status) and keeps no global state.
+ * Streams:    `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *             stream).  All work is enqueued asynchronously on it.
+ * Layouts:    row-major (C order), token-major:
+ *               q, k, g     [total_tokens, H, dk]
+ *               v, o        [total_tokens, H, dv]
+ *               beta        [total_tokens, H]
+ *               states      [num_seqs, H, dk, dv]  -- S[c][j] is key channel c,
+ *                           value channel j (dv contiguous); this one layout is
+ *                           used by prefill, decode and every state argument.
+ * Sequences:  cu_seqlens == NULL: B sequences of T tokens each, total = B*T,
+ *             num_seqs must equal B.  cu_seqlens != NULL: int32 device array
+ *             [num_seqs + 1] of packed-sequence offsets (cu[0] = 0,
+ *             non-decreasing, cu[num_seqs] = T); B must be 1 and T is the
+ *             total token count.  Chunks start at each sequence's first token
+ *             and never straddle sequences; a sequence's last chunk may be
+ *             short.  A zero-length sequence passes its initial state through.
+ * Gates:      g = log(alpha) in fp32, any finite value; beta in fp32.
+ * dtype:      the type of q, k, v and o (KDA_DTYPE_F32 or KDA_DTYPE_BF16).
+ *             g, beta and every state are always fp32; arithmetic is fp32.
+ * Errors:     a return other than KDA_OK means nothing was enqueued.  Checks
+ *             that need device data (cu_seqlens contents) run on the device
+ *             and are reported by kda_get_device_status().
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* NULL / misaligned pointer, bad size or shape combination */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid arguments, but no kernel for this shape / dtype */
+    KDA_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch error, ...) */
+    KDA_ERR_TIMEOUT = 4,      /* device side: a bounded wait gave up (set in the status word) */
+    KDA_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than *_workspace_size() */
+    KDA_ERR_BAD_SEQLENS = 6   /* device side: cu_seqlens not 0 .. T non-decreasing */
+} kda_status_t;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype_t;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* kda_status_string(kda_status_t status);
+
+/* ------------------------------------------------------------------ prefill
+ * kda_chunk_fwd: chunkwise KDA forward over B x T tokens or packed sequences.
+ *   Defining passage: Kimi Linear (aiwiki.ai), "The constrained DPLR form and
+ *   the chunkwise algorithm" (chunks of C tokens, WY representation, UT
+ *   transform, recurrent between chunks, parallel inside a chunk).
+ * In:  q, k [total, H, dk], v [total, H, dv] (dtype); g [total, H, dk] fp32;
+ *      beta [total, H] fp32; initial_state [num_seqs, H, dk, dv] fp32 or NULL
+ *      (zeros); cu_seqlens as above or NULL.
+ * Out: o [total, H, dv] (dtype), every token written; final_state
+ *      [num_seqs, H, dk, dv] fp32 or NULL (not written).  initial_state and
+ *      final_state may be the same buffer.
+ * Workspace: device scratch of at least kda_chunk_fwd_workspace_size() bytes,
+ *      256-byte aligned, owned by the caller, reusable across calls on the same
+ *      stream; it also holds the device status word.
+ * Shapes: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}.  bf16 with
+ *      dk = dv = 128 and chunk = 64 runs the tensor-core (tcgen05) kernel;
+ *      other supported shapes run the CUDA-core kernels.  Otherwise
+ *      KDA_ERR_UNSUPPORTED.
+ */
+size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
+                                    int chunk, kda_dtype_t dtype);
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                           int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                           float* final_state, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* --------------------------------------------- prefill, one step per call
+ * The four steps of the chunkwise form as separate calls, with the
+ * intermediates in caller-owned buffers.  kda_chunk_fwd computes the same
+ * result; these exist so that each step can be checked and timed on its own.
+ * Notation, per (sequence, head, chunk) with rows r, i of the chunk:
+ *   G_r = sum_{j <= r in chunk} g_j (inclusive, per channel), Gam = exp(G);
+ *   A[r,i] = beta_r sum_c k[r,c] k[i,c] exp(G[r,c] - G[i,c])   (i < r);
+ *   Tm = (I + A)^{-1};  W = Tm diag(beta) (K * Gam);  Ut = Tm diag(beta) V;
+ *   S_n = state at the start of chunk n;  U_n = Ut - W S_n;
+ *   S_{n+1} = Diag(Gam_last) S_n + (K * exp(G_last - G))^T U_n;
+ *   O_n = (Q * Gam) S_n + (P masked to i <= r) U_n,
+ *         P[r,i] = sum_c q[r,c] k[i,c] exp(G[r,c] - G[i,c]).
+ * (Derived from the recurrence above: one step is S_r = Diag(alpha_r)
+ * S_{r-1} + k_r u_r^T with u_r = beta_r (v_r - (Diag(alpha_r) S_{r-1})^T k_r),
+ * unrolled inside a chunk.)
+ * All intermediates are fp32 and token-major where they have one row per
+ * token.  Chunk states are numbered by global chunk index: sequences in
+ * order, chunks in order within a sequence; there are
+ * kda_num_chunks_upper_bound() slots, of which sum_s ceil(len_s / chunk) are
+ * used.  Workspace: kda_chunk_fwd_workspace_size() bytes, as for
+ * kda_chunk_fwd.  Any dtype / shape that kda_chunk_fwd accepts.
+ */
+int kda_num_chunks_upper_bound(int total_tokens, int num_seqs, int chunk);
+
+/* a1: cumulative log-gate.  G [total, H, dk] fp32 = per-chunk inclusive
+ * cumulative sum of g over tokens, per (head, channel): the logarithm of the
+ * running decay product that section "The constrained DPLR form and the
+ * chunkwise algorithm" identifies as the unstable divisor of general DPLR. */
+kda_status_t kda_chunk_gate_cumsum(const float* g, const int32_t* cu_seqlens, int B, int T,
+                                   int num_seqs, int H, int dk, int chunk, float* G,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* a2: intra-chunk WY / UT factors.  From k, v (dtype), G, beta: builds A,
+ * solves the unit-lower-triangular system (UT transform) and writes
+ * W [total, H, dk] fp32 and Ut [total, H, dv] fp32 (row r of a chunk at the
+ * chunk's r-th token). */
+kda_status_t kda_chunk_intra(const void* k, const void* v, const float* G, const float* beta,
+                             const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                             int dk, int dv, int chunk, kda_dtype_t dtype, float* W, float* Ut,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* a3: inter-chunk state propagation, serial over the chunks of each
+ * sequence, state carried in fp32.  In: k (dtype), G, W, U (holding Ut on
+ * entry; overwritten in place with U_n = Ut - W S_n), initial_state or NULL.
+ * Out: chunk_states [num_chunks_upper_bound, H, dk, dv] fp32 (S_n per
+ * chunk), final_state [num_seqs, H, dk, dv] or NULL. */
+kda_status_t kda_chunk_inter(const void* k, const float* G, const float* W, float* U,
+                             const float* initial_state, const int32_t* cu_seqlens, int B,
+                             int T, int num_seqs, int H, int dk, int dv, int chunk,
+                             kda_dtype_t dtype, float* chunk_states, float* final_state,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* a4: output.  O_n = (Q * Gam) S_n + (P masked) U_n for every chunk.
+ * In: q, k (dtype), G, U (as left by kda_chunk_inter), chunk_states.
+ * Out: o [total, H, dv] (dtype). */
+kda_status_t kda_chunk_output(const void* q, const void* k, const float* G, const float* U,
+                              const float* chunk_states, const int32_t* cu_seqlens, int B,
+                              int T, int num_seqs, int H, int dk, int dv, int chunk,
+                              kda_dtype_t dtype, void* o, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------- decode
+ * kda_decode_step: one token per (sequence, head), state updated in place.
+ *   Defining passages: Kimi Linear (aiwiki.ai), "Why linear attention exists"
+ *   (decoding is a recurrent update whose cost per token does not depend on
+ *   the context read so far) and "The constrained DPLR form and the chunkwise
+ *   algorithm" (a fixed 128 x 128 state per head).
+ * In:  q, k [N, H, dk], v [N, H, dv] (dtype); g [N, H, dk] fp32; beta [N, H]
+ *      fp32.  In/out: state [N, H, dk, dv] fp32 (the prefill state layout).
+ * Out: o [N, H, dv] (dtype) = S_new^T q.
+ * One read and one write of every state element.  No workspace.
+ * Shapes: dk, dv in {32, 64, 128}; N >= 0 (N = 0 enqueues nothing).
+ */
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, float* state, void* o, int N, int H, int dk,
+                             int dv, kda_dtype_t dtype, void* stream);
+
+/* ------------------------------------------------------------------ status
+ * Synchronises `stream`, then reads the device status word kept at the start
+ * of `workspace`.  Every prefill call (kda_chunk_fwd and the step calls)
+ * clears that word on entry, so it describes the LAST prefill call enqueued
+ * with this workspace.  Returns KDA_OK, the device-side error it recorded
+ * (KDA_ERR_BAD_SEQLENS, KDA_ERR_TIMEOUT), or KDA_ERR_CUDA if the copy or the
+ * stream reports an error.  The only blocking call in the library.  After a
+ * device-side error the call's kernels skipped their work: outputs are
+ * unspecified.
+ */
+kda_status_t kda_get_device_status(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H_ */

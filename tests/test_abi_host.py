@@ -1,0 +1,127 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports
+every function include/kda.h declares, and rejects bad arguments before
+enqueuing anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_124_b200 as kda
+from gated_delta_rule_124_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_binding_exports():
+    assert sorted(kda.EXPORTS) == declared_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = kda.status_string(code)
+        assert s.startswith("KDA_"), s
+    assert "UNKNOWN" in kda.status_string(99)
+
+
+def test_workspace_size_rules(lib):
+    f = kda.kda_chunk_fwd_workspace_size
+    assert f(4096, 2, 32, 128, 128, 64, "bf16") > 0
+    assert f(64, 1, 1, 32, 32, 16, "f32") > 0
+    assert f(64, 1, 1, 48, 32, 16, "f32") == 0   # unsupported dk
+    assert f(64, 1, 1, 32, 32, 8, "f32") == 0    # unsupported chunk
+    assert f(64, 0, 1, 32, 32, 16, "f32") == 0   # no sequences
+    # grows with tokens
+    assert f(8192, 2, 32, 64, 64, 64, "f32") > f(4096, 2, 32, 64, 64, 64, "f32")
+
+
+def test_chunk_upper_bound(lib):
+    assert kda.kda_num_chunks_upper_bound(4096, 2, 64) == 64 + 1  # (4096 + 2*63) // 64
+    assert kda.kda_num_chunks_upper_bound(0, 3, 16) == 2
+    # bound covers any split of 100 tokens into 3 sequences
+    for a in range(0, 101, 7):
+        for b in range(0, 101 - a, 11):
+            c = 100 - a - b
+            used = sum((x + 15) // 16 for x in (a, b, c))
+            assert used <= kda.kda_num_chunks_upper_bound(100, 3, 16)
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-NULL address; never dereferenced on these paths
+
+
+def _fwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, initial_state=None, cu_seqlens=None,
+                B=1, T=64, num_seqs=1, H=1, dk=32, dv=32, chunk=16, dtype="f32", o=FAKE,
+                final_state=None, workspace=FAKE * 2, workspace_bytes=1 << 40, stream=0,
+                check=False)
+    args.update(kw)
+    return kda.kda_chunk_fwd(**args)
+
+
+def test_chunk_fwd_rejects_bad_arguments(lib):
+    assert _fwd(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _fwd(o=None) == kda.KDA_ERR_INVALID_ARG
+    assert _fwd(k=FAKE + 4) == kda.KDA_ERR_INVALID_ARG          # misaligned
+    assert _fwd(B=0) == kda.KDA_ERR_INVALID_ARG
+    assert _fwd(T=-1) == kda.KDA_ERR_INVALID_ARG
+    assert _fwd(num_seqs=2) == kda.KDA_ERR_INVALID_ARG          # != B without cu_seqlens
+    assert _fwd(cu_seqlens=FAKE, B=2, num_seqs=2) == kda.KDA_ERR_INVALID_ARG
+    assert _fwd(dk=48) == kda.KDA_ERR_UNSUPPORTED
+    assert _fwd(chunk=128) == kda.KDA_ERR_UNSUPPORTED
+    assert _fwd(dtype=kda.KDA_DTYPE_F32, workspace=None) == kda.KDA_ERR_WORKSPACE
+    assert _fwd(workspace_bytes=16) == kda.KDA_ERR_WORKSPACE
+    assert _fwd(workspace=FAKE + 16) == kda.KDA_ERR_INVALID_ARG  # not 256-aligned
+    assert _fwd(final_state=FAKE + 8) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments(lib):
+    def dec(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, state=FAKE, o=FAKE, N=4, H=2,
+                 dk=128, dv=128, dtype="bf16", stream=0, check=False)
+        a.update(kw)
+        return kda.kda_decode_step(**a)
+    assert dec(state=None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(q=FAKE + 2) == kda.KDA_ERR_INVALID_ARG
+    assert dec(N=-1) == kda.KDA_ERR_INVALID_ARG
+    assert dec(H=0) == kda.KDA_ERR_INVALID_ARG
+    assert dec(dk=96) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(N=0) == kda.KDA_OK                                 # nothing to do
+    assert dec(N=0, q=None) == kda.KDA_OK
+
+
+def test_step_calls_reject_bad_arguments(lib):
+    common = dict(cu_seqlens=None, B=1, T=64, num_seqs=1, H=1, chunk=16, workspace=FAKE * 2,
+                  workspace_bytes=1 << 40, stream=0, check=False)
+    assert kda.kda_chunk_gate_cumsum(g=None, dk=32, G=FAKE, **common) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_intra(k=FAKE, v=FAKE, G=FAKE, beta=FAKE, dk=32, dv=32, dtype="f32",
+                               W=None, Ut=FAKE, **common) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_inter(k=FAKE, G=FAKE, W=FAKE, U=FAKE, initial_state=FAKE + 4, dk=32,
+                               dv=32, dtype="f32", chunk_states=FAKE, final_state=None,
+                               **common) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_output(q=FAKE, k=FAKE, G=FAKE, U=FAKE, chunk_states=FAKE, dk=32,
+                                dv=96, dtype="f32", o=FAKE, **common) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_get_device_status_rejects_bad_workspace(lib):
+    assert kda.kda_get_device_status(None, 0) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_get_device_status(FAKE + 16, 0) == kda.KDA_ERR_INVALID_ARG

@@ -1,0 +1,213 @@
+"""GPU parity of the chunkwise prefill (kda_chunk_fwd and the per-step calls)
+against the fp64 oracle (token recurrence) and its chunkwise restatement."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_124_b200 as kda
+from gated_delta_rule_124_b200 import workloads as wl
+from oracle import chunkwise
+from tests.helpers import oracle_prefill, rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd(case, final=True):
+    c = case.to("cuda")
+    packed = c.cu_seqlens is not None
+    B, T = (1, c.total) if packed else (c.B, c.T)
+    ws = kda.alloc_workspace(c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype)
+    o = torch.full_like(c.v, float("nan"))
+    hN = torch.full((c.N, c.H, c.dk, c.dv), float("nan"), device="cuda") if final else None
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, B, T, c.N,
+                      c.H, c.dk, c.dv, c.chunk, c.dtype, o, hN, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    return o, hN
+
+
+def check_case(case, heads=None):
+    o, hN = run_fwd(case)
+    ro, rh = oracle_prefill(case, heads)
+    sl = slice(None) if heads is None else list(heads)
+    tol = tol_for(case.dtype)
+    eo = rel_err(o[:, sl], ro)
+    eh = rel_err(hN[:, sl], rh)
+    assert eo <= tol and eh <= tol, (case.name, eo, eh)
+    return eo, eh
+
+
+# ---------------------------------------------------------------- configs
+
+def test_config0_tiny_fp32():
+    case = wl.prefill_config(0)
+    check_case(case)
+
+
+def test_config1_all_heads():
+    case = wl.prefill_config(1)
+    check_case(case)
+
+
+def test_config2_long_sampled_heads():
+    """T = 65536: all tokens of three heads (first, middle, last) against the
+    oracle; the chunk chain is 1024 chunks long."""
+    case = wl.prefill_config(2)
+    check_case(case, heads=[0, 17, 31])
+
+
+def test_config3_varlen_sampled_heads():
+    case = wl.prefill_config(3)
+    check_case(case, heads=[0, 31])
+
+
+# ----------------------------------------------------- shapes and edge cases
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv,C", [(32, 32, 16), (64, 32, 32), (32, 128, 64), (128, 64, 16),
+                                     (128, 128, 64), (64, 64, 64)])
+def test_ragged_lengths(dtype, dk, dv, C):
+    """Lengths that are not multiples of the chunk, shorter than one chunk,
+    exactly one chunk, and length 1, packed with cu_seqlens."""
+    lens = [C * 3 + 5, C - 1, 1, C, 2 * C + 1]
+    case = wl.make_prefill(100 + dk + dv + C, lens, H=3, dk=dk, dv=dv, chunk=C, dtype=dtype,
+                           varlen=True)
+    check_case(case)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_batched_equal_lengths_with_tail(dtype):
+    case = wl.make_prefill(5, [200] * 3, H=4, dk=128, dv=128, chunk=64, dtype=dtype)
+    check_case(case)
+
+
+def test_zero_length_sequences_pass_state_through():
+    lens = [0, 70, 0, 3, 0]
+    case = wl.make_prefill(8, lens, H=2, dk=64, dv=64, chunk=32, dtype="f32", varlen=True)
+    o, hN = run_fwd(case)
+    ro, rh = oracle_prefill(case)
+    assert rel_err(o, ro) <= 1e-4
+    assert rel_err(hN, rh) <= 1e-4
+    assert torch.equal(hN[0].cpu(), case.initial_state[0])
+    assert torch.equal(hN[4].cpu(), case.initial_state[4])
+
+
+def test_null_initial_state_means_zeros():
+    case = wl.make_prefill(9, [150], H=2, dk=128, dv=128, chunk=64, dtype="bf16", init_std=None)
+    check_case(case)
+
+
+def test_strong_decay_is_finite():
+    """Gates far below zero (sum of g over a chunk near -300) stay finite."""
+    case = wl.make_prefill(10, [256], H=2, dk=128, dv=128, chunk=64, dtype="bf16", g_mu=4.0)
+    check_case(case)
+
+
+def test_split_prefill_composes():
+    """Prefill in three calls chained through initial/final state equals one
+    call: the state layout is the same on input and output."""
+    case = wl.make_prefill(12, [64 * 5 + 17], H=4, dk=128, dv=128, chunk=64, dtype="f32")
+    o_full, h_full = run_fwd(case)
+    c = case.to("cuda")
+    cuts = [0, 64, 64 * 3 + 7, c.total]
+    h = c.initial_state
+    outs = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, h = kda.chunk_fwd(c.q[None, a:b], c.k[None, a:b], c.v[None, a:b], c.g[None, a:b],
+                             c.beta[None, a:b], h, chunk=64)
+        outs.append(o[0])
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat(outs), o_full.double().cpu().numpy()) <= 1e-5
+    assert rel_err(h, h_full.double().cpu().numpy()) <= 1e-5
+
+
+def test_final_state_optional_and_in_place():
+    case = wl.make_prefill(13, [100, 100], H=2, dk=64, dv=64, chunk=32, dtype="f32")
+    c = case.to("cuda")
+    ws = kda.alloc_workspace(c.total, 2, 2, 64, 64, 32, "f32")
+    o1 = torch.empty_like(c.v)
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, c.initial_state, None, 2, 100, 2, 2, 64, 64, 32,
+                      "f32", o1, None, ws)
+    st = c.initial_state.clone()
+    o2 = torch.empty_like(c.v)
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, st, None, 2, 100, 2, 2, 64, 64, 32, "f32", o2,
+                      st, ws)
+    torch.cuda.synchronize()
+    ro, rh = oracle_prefill(case)
+    assert rel_err(o1, ro) <= 1e-4 and rel_err(o2, ro) <= 1e-4
+    assert rel_err(st, rh) <= 1e-4
+
+
+def test_bad_cu_seqlens_reported_on_device():
+    case = wl.make_prefill(14, [40, 40], H=1, dk=32, dv=32, chunk=16, dtype="f32", varlen=True)
+    c = case.to("cuda")
+    bad = torch.tensor([0, 50, 40], dtype=torch.int32, device="cuda")  # ends right, not monotone
+    ws = kda.alloc_workspace(80, 2, 1, 32, 32, 16, "f32")
+    o = torch.empty_like(c.v)
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, None, bad, 1, 80, 2, 1, 32, 32, 16, "f32", o,
+                      None, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
+    bad2 = torch.tensor([0, 30, 70], dtype=torch.int32, device="cuda")  # wrong total
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, None, bad2, 1, 80, 2, 1, 32, 32, 16, "f32", o,
+                      None, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
+    # a good call on the same workspace clears the word
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, None, c.cu_seqlens, 1, 80, 2, 1, 32, 32, 16,
+                      "f32", o, None, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+
+
+def test_deterministic():
+    case = wl.make_prefill(15, [300, 77], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    o1, h1 = run_fwd(case)
+    o2, h2 = run_fwd(case)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+# ------------------------------------------------- one step per call (a1-a4)
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_calls_match_chunkwise_intermediates(dtype):
+    lens = [64 * 2 + 9, 30]
+    case = wl.make_prefill(16, lens, H=2, dk=128, dv=64, chunk=64, dtype=dtype, varlen=True)
+    c = case.to("cuda")
+    N, H, dk, dv, C = c.N, c.H, c.dk, c.dv, c.chunk
+    tot = c.total
+    ws = kda.alloc_workspace(tot, N, H, dk, dv, C, dtype)
+    G = torch.empty(tot, H, dk, device="cuda")
+    W = torch.empty(tot, H, dk, device="cuda")
+    U = torch.empty(tot, H, dv, device="cuda")
+    maxc = kda.kda_num_chunks_upper_bound(tot, N, C)
+    S = torch.full((maxc, H, dk, dv), float("nan"), device="cuda")
+    hN = torch.empty(N, H, dk, dv, device="cuda")
+    o = torch.empty_like(c.v)
+    args = (c.cu_seqlens, 1, tot, N, H)
+    kda.kda_chunk_gate_cumsum(c.g, *args, dk, C, G, ws)
+    kda.kda_chunk_intra(c.k, c.v, G, c.beta, *args, dk, dv, C, dtype, W, U, ws)
+    Ut = U.clone()
+    kda.kda_chunk_inter(c.k, G, W, U, c.initial_state, *args, dk, dv, C, dtype, S, hN, ws)
+    kda.kda_chunk_output(c.q, c.k, G, U, S, *args, dk, dv, C, dtype, o, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    f64 = lambda t: t.detach().cpu().double().numpy()
+    _, _, inter = chunkwise.forward(f64(case.q), f64(case.k), f64(case.v), f64(case.g),
+                                    f64(case.beta), f64(case.initial_state), case.cu_host(),
+                                    chunk=C, keep=True)
+    cu = case.cu_host()
+    gidx = 0
+    for s in range(N):
+        nch = (lens[s] + C - 1) // C
+        for n in range(nch):
+            t0 = cu[s] + n * C
+            t1 = min(t0 + C, cu[s + 1])
+            for h in range(H):
+                r = inter[(s, h, n)]
+                assert rel_err(G[t0:t1, h], r["G"]) <= 1e-6
+                assert rel_err(W[t0:t1, h], r["W"]) <= 1e-4
+                assert rel_err(Ut[t0:t1, h], r["Ut"]) <= 1e-4
+                assert rel_err(U[t0:t1, h], r["U"]) <= 1e-4
+                assert rel_err(S[gidx + n, h], r["S_in"]) <= 1e-5
+                assert rel_err(o[t0:t1, h], r["O"]) <= tol_for(dtype)
+        gidx += nch
+    ro, rh = oracle_prefill(case)
+    assert rel_err(o, ro) <= tol_for(dtype)
+    assert rel_err(hN, rh) <= 1e-4
