@@ -4,10 +4,10 @@ The compute lives in libkda.so (CUDA, C ABI in include/kda.h); :mod:`.kda` is
 its ctypes binding and :mod:`.workloads` draws seeded synthetic inputs.
 """
 from .kda import (  # noqa: F401
-    EXPORTS, KDA_DTYPE_BF16, KDA_DTYPE_F32, KDA_ERR_BAD_SEQLENS, KDA_ERR_CUDA,
+    EXPORTS, KDA_DTYPE_BF16, KDA_DTYPE_F32, KDA_NOALLOC_SCRATCH_BYTES, KDA_ERR_BAD_SEQLENS, KDA_ERR_CUDA,
     KDA_ERR_INVALID_ARG, KDA_ERR_TIMEOUT, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_OK,
     KdaError, alloc_workspace, chunk_fwd, decode_step, kda_chunk_fwd,
     kda_chunk_fwd_workspace_size, kda_chunk_gate_cumsum, kda_chunk_inter, kda_chunk_intra,
-    kda_chunk_output, kda_decode_step, kda_get_device_status, kda_num_chunks_upper_bound,
+    kda_chunk_output, kda_chunk_fwd_noalloc, kda_decode_step, kda_get_device_status, kda_num_chunks_upper_bound,
     load, status_string,
 )

@@ -38,6 +38,7 @@ EXPORTS = (
     "kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
     "kda_num_chunks_upper_bound", "kda_chunk_gate_cumsum", "kda_chunk_intra",
     "kda_chunk_inter", "kda_chunk_output", "kda_decode_step", "kda_get_device_status",
+    "kda_chunk_fwd_noalloc",
 )
 
 
@@ -62,7 +63,11 @@ _SIGS = {
     "kda_chunk_output": ([_vp] * 6 + [_i] * 8 + [_vp, _vp, _sz, _vp], _i),
     "kda_decode_step": ([_vp] * 7 + [_i] * 5 + [_vp], _i),
     "kda_get_device_status": ([_vp, _vp], _i),
+    "kda_chunk_fwd_noalloc": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp], _i),
 }
+
+# Size of the library's built-in scratch used by kda_chunk_fwd_noalloc.
+KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 def load(path: str = LIB_PATH):
@@ -191,6 +196,18 @@ def kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None
     st = load().kda_decode_step(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state), _p(o), N, H,
                                 dk, dv, dtype_code(dtype), _stream(stream))
     return _ret(st, "kda_decode_step", check)
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H, dk,
+                          dv, chunk, dtype, o, final_state, stream=None, check=True) -> int:
+    """kda_chunk_fwd without a workspace: for callers that may not allocate
+    device memory.  The library's own static scratch array is used instead;
+    see include/kda.h for its size limit and sharing rules."""
+    st = load().kda_chunk_fwd_noalloc(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
+                                      _p(cu_seqlens), B, T, num_seqs, H, dk, dv, chunk,
+                                      dtype_code(dtype), _p(o), _p(final_state),
+                                      _stream(stream))
+    return _ret(st, "kda_chunk_fwd_noalloc", check)
 
 
 def kda_get_device_status(workspace, stream=None) -> int:

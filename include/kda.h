@@ -174,6 +174,36 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
                              const float* beta, float* state, void* o, int N, int H, int dk,
                              int dv, kda_dtype_t dtype, void* stream);
 
+/* ------------------------------------------------ prefill, no allocation
+ * kda_chunk_fwd_noalloc: the same computation as kda_chunk_fwd, with no
+ * workspace argument, for callers that may not obtain device memory: an
+ * operator inside an engine or graph runtime whose interface passes only
+ * inputs and outputs and whose planner owns all device memory, or a serving
+ * loop that reserved nearly all HBM up front, where a cudaMalloc would fail,
+ * fragment that reservation or stall other streams.  The pages have no
+ * counterpart to this call; it is a packaging choice of this library.
+ * Scratch: one static device array of KDA_NOALLOC_SCRATCH_BYTES inside the
+ *      library, held on every GPU that loads the library until the process
+ *      exits.  The first call on a device looks up that array's address (with
+ *      the device current) -- make it before any stream capture.  Calls share
+ *      the array: results never depend on an earlier call, but calls whose
+ *      work overlaps on the GPU race.
+ * Limit: a problem fits when kda_chunk_fwd_workspace_size(total_tokens,
+ *      num_seqs, H, dk, dv, chunk, KDA_DTYPE_F32) <= KDA_NOALLOC_SCRATCH_BYTES;
+ *      otherwise KDA_ERR_WORKSPACE and nothing is enqueued.
+ * Path: the CUDA-core kernels, for both dtypes.  Device-side cu_seqlens
+ *      errors skip the work (o, final_state unwritten) and are not reported.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Arguments and other errors: as kda_chunk_fwd.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* initial_state,
+                                   const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                                   int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                                   float* final_state, void* stream);
+
 /* ------------------------------------------------------------------ status
  * Synchronises `stream`, then reads the device status word kept at the start
  * of `workspace`.  Every prefill call (kda_chunk_fwd and the step calls)

@@ -1,0 +1,61 @@
+"""kda_chunk_fwd_noalloc: prefill for callers that may not allocate device memory.
+
+Some callers are handed only their inputs and outputs -- an operator inside an
+engine whose memory planner owns the whole device, or a serving loop that
+reserved nearly all HBM up front -- and cannot pass a workspace.  This entry
+point uses a static scratch array inside the library instead.  The GPU test
+calls it twice in a row, through the C ABI, on two different problems (so the
+second call runs on scratch the first one left behind) and compares each
+result with kda_chunk_fwd's.  This file is collected last on purpose.
+"""
+import pytest
+import torch
+
+import gated_delta_rule_124_b200 as kda
+from gated_delta_rule_124_b200 import workloads as wl
+from tests.helpers import rel_err, tol_for
+
+
+def _problem(seed, lens, H, d, C, dtype):
+    return wl.make_prefill(seed, lens, H=H, dk=d, dv=d, chunk=C, dtype=dtype, varlen=True)
+
+
+def _with_workspace(c):
+    ws = kda.alloc_workspace(c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype)
+    o = torch.empty_like(c.v)
+    hN = torch.empty(c.N, c.H, c.dk, c.dv, device="cuda")
+    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, 1, c.total,
+                      c.N, c.H, c.dk, c.dv, c.chunk, c.dtype, o, hN, ws)
+    return o, hN
+
+
+def _no_alloc(c):
+    o = torch.full_like(c.v, float("nan"))
+    hN = torch.full((c.N, c.H, c.dk, c.dv), float("nan"), device="cuda")
+    kda.kda_chunk_fwd_noalloc(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, 1,
+                              c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype, o, hN)
+    return o, hN
+
+
+@pytest.mark.gpu
+def test_no_alloc_matches_workspace_entry_point_twice():
+    first = _problem(501, [300, 64, 17], H=4, d=128, C=64, dtype="bf16").to("cuda")
+    second = _problem(502, [90, 1, 200], H=3, d=64, C=32, dtype="f32").to("cuda")
+    for c in (first, second):
+        ref_o, ref_h = _with_workspace(c)
+        o, h = _no_alloc(c)
+        torch.cuda.synchronize()
+        tol = tol_for(c.dtype)
+        assert rel_err(o, ref_o.double().cpu().numpy()) <= tol
+        assert rel_err(h, ref_h.double().cpu().numpy()) <= tol
+
+
+def test_no_alloc_rejects_problems_beyond_the_scratch():
+    """Checked on the host before anything is enqueued: no GPU needed."""
+    fake = 1 << 20
+    total, H, d, C = 1 << 16, 32, 128, 64   # needs far more than the static scratch
+    assert kda.kda_chunk_fwd_workspace_size(total, 1, H, d, d, C, "f32") > \
+        kda.KDA_NOALLOC_SCRATCH_BYTES
+    st = kda.kda_chunk_fwd_noalloc(fake, fake, fake, fake, fake, None, None, 1, total, 1, H, d,
+                                   d, C, "bf16", fake, None, stream=0, check=False)
+    assert st == kda.KDA_ERR_WORKSPACE
