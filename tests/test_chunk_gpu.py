@@ -211,3 +211,22 @@ def test_step_calls_match_chunkwise_intermediates(dtype):
     ro, rh = oracle_prefill(case)
     assert rel_err(o, ro) <= tol_for(dtype)
     assert rel_err(hN, rh) <= 1e-4
+
+
+def test_mixed_fast_and_exact_chunks():
+    """One chunk with extreme decay (its per-channel log-decay range exceeds
+    the tensor-core factorisation's headroom, so it is evaluated exactly)
+    between ordinary chunks: the state must carry across both kinds."""
+    case = wl.make_prefill(17, [64 * 4 + 10], H=2, dk=128, dv=128, chunk=64, dtype="bf16")
+    case.g[64:128] *= 6.0
+    check_case(case)
+
+
+@pytest.mark.parametrize("lens", [[1], [63], [65], [1, 1, 1], [0, 64, 0, 129, 7],
+                                  [300, 2, 700, 64, 63]])
+def test_varlen_edge_lengths_bf16_d128(lens):
+    """Packed sequences with lengths around the chunk size, including empty
+    and single-token sequences, on the bf16 d = 128 chunk-64 path."""
+    case = wl.make_prefill(200 + sum(lens), lens, H=3, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    check_case(case)
