@@ -37,6 +37,32 @@ METRIC = "KDA prefill tokens/s and decode tokens/s; % of tensor / HBM roofline (
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
+# ncu capture of each kernel (summaries in profiles/).  Reported only while the
+# kernel's source still matches the capture; null once it has changed.
+MEASURED_TRAFFIC = {
+    "chunk_fwd_tc": ("gated_delta_rule_124_b200/csrc/kda_chunk_tc.cu",
+                     "4231175dcf260063f6cc2aa1e8befdeb56dac955", 195476992),
+    "decode": ("gated_delta_rule_124_b200/csrc/kda_decode.cu",
+               "0055ed0bdb7266f6b3dd4c18570118f7bd32fa1c", 1027668224),
+}
+
+
+def measured_traffic(name):
+    import hashlib
+    entry = MEASURED_TRAFFIC.get(name)
+    if entry is None:
+        return None
+    path, sha, nbytes = entry
+    try:
+        with open(os.path.join(ROOT, path), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != sha:
+                return None
+    except OSError:
+        return None
+    return nbytes
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -85,7 +111,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -223,7 +249,8 @@ def run_ours(args, rank, world, local_rank):
     dom_bytes = kern["bytes"][dom_name]
     roof = {"kernel": dom_name, "bound": "hbm", "achieved": dom_bytes / dom_s / 1e9,
             "peak": hbm, "unit": "GB/s", "frac": dom_bytes / dom_s / 1e9 / hbm,
-            "traffic": None, "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+            "traffic": measured_traffic(dom_name),
+            "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
             "per_launch_us": dom_s * 1e6, "algorithmic_bytes_per_launch": dom_bytes}
     dec_avg = dec_sum / args.steps / 1e3
     db = decode_bytes(Nd * H)
@@ -244,7 +271,8 @@ def run_ours(args, rank, world, local_rank):
         "decode": {"value": dec_value, "unit": "tokens/s", "ms_per_step": dec_avg * 1e3,
                    "roofline": {"bound": "hbm", "achieved": db / dec_avg / 1e9, "peak": hbm,
                                 "unit": "GB/s", "frac": db / dec_avg / 1e9 / hbm,
-                                "traffic": None, "algorithmic_bytes_per_launch": db}},
+                                "traffic": measured_traffic("decode"),
+                                "algorithmic_bytes_per_launch": db}},
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": args.steps * (kern["launches_per_call"] + 1),
@@ -458,7 +486,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

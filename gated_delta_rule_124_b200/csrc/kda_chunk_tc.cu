@@ -88,10 +88,10 @@ constexpr uint32_t TM_S = 384;    // fp32 state
 
 constexpr uint32_t TX_BYTES = 3 * 16384 + 32768;
 
-// fp32 64 x 64 matrices: A with an XOR swizzle that spreads a column over the
-// banks (written one row per lane); T with 4-float groups permuted per row so
-// that row vectors stay contiguous and 8 rows of one column group differ in bank.
-__device__ __forceinline__ int a_idx(int r, int c) { return r * C + (c ^ (r & 31)); }
+// fp32 64 x 64 matrices A and T: 4-float groups permuted per row, so that row
+// vectors stay contiguous and 8 consecutive rows of one column group fall in
+// different banks.
+__device__ __forceinline__ int a_idx(int r, int c) { return r * C + (c ^ ((r & 7) << 2)); }
 __device__ __forceinline__ int t_idx(int r, int c) { return r * C + (c ^ ((r & 7) << 2)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -484,10 +484,15 @@ __global__ void __launch_bounds__(NT, 1)
                     if (m < C) {
                         const float b = sbeta[m];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int col = cq * 32 + i;
-                            Af[a_idx(m, col)] =
-                                (m < L && col < m) ? b * __uint_as_float(v[i]) : 0.f;
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const int col = cq * 32 + 4 * i4;
+                            float y[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                y[i] = (m < L && col + i < m) ? b * __uint_as_float(v[4 * i4 + i])
+                                                              : 0.f;
+                            *reinterpret_cast<float4*>(Af + a_idx(m, col)) =
+                                make_float4(y[0], y[1], y[2], y[3]);
                         }
                     } else {
                         const int r = m - C;
