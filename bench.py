@@ -92,6 +92,24 @@ def decode_bytes(units: int, dk=128, dv=128, in_bytes=2) -> int:
     return units * (2 * 4 * dk * dv + in_bytes * (2 * dk + 2 * dv) + 4 * dk + 4)
 
 
+# ------------------------------------------------------------- multi-rank
+
+def max_over_ranks(vals, world, device="cpu"):
+    """Element-wise max of per-rank device times over all ranks (replicas)."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank_step, world, steps, time_ms):
+    """Whole-job units/s: every rank's units over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (time_ms / 1e3)
+
+
 # ------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -221,16 +239,10 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
     pre_sum, dec_sum = sum(pre_ms), sum(dec_ms)
 
-    # ---- max over ranks (device time)
-    if world > 1:
-        t = torch.tensor([total_ms, pre_sum, dec_sum], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, pre_sum, dec_sum = t.tolist()
-
-    pre_tokens = total * world * args.steps
-    dec_tokens = Nd * world * args.steps
-    value = pre_tokens / (pre_sum / 1e3)
-    dec_value = dec_tokens / (dec_sum / 1e3)
+    # ---- max over ranks (device time), whole-job throughput
+    total_ms, pre_sum, dec_sum = max_over_ranks([total_ms, pre_sum, dec_sum], world, dev)
+    value = job_throughput(total, world, args.steps, pre_sum)
+    dec_value = job_throughput(Nd, world, args.steps, dec_sum)
 
     # ---- per-kernel times of the prefill (dominant kernel) with the step calls
     kern = prefill_kernel_times(kda, P, ws, dev, stream, reps=max(5, min(50, args.steps)))
