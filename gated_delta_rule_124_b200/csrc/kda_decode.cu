@@ -12,12 +12,15 @@
 //
 // The state is the only large operand (64 KiB per head at 128 x 128, fp32);
 // the kernel reads and writes it exactly once, so the step is bound by HBM
-// bandwidth.  One CTA of 256 threads owns one (sequence, head): lane l of
-// warp w holds columns [4 c4, 4 c4 + 4) of rows {w RPW + rw + 8 RPW p}, so
-// every warp-wide load or store is a run of whole 512-byte rows (16-byte
-// vectors).  Both column reductions (Sbar^T k and Sbar^T q) are a shuffle
-// inside the warp (when a warp spans several rows) and one shared-memory pass
-// across the 8 warps.
+// bandwidth.  Both column reductions (Sbar^T k, Sbar^T q) run over dk only, so
+// the dv columns of one (sequence, head) are independent: a CTA of 256 threads
+// owns one (sequence, head) and a slice of DVS value columns (DVS = 64 for
+// dv = 128: two CTAs per head, 32 state floats per thread, 4 CTAs per SM).
+// Lane l of warp w holds columns [4 c4, 4 c4 + 4) of the slice in rows
+// {w RPW + rw + 8 RPW p}, so every warp-wide load or store covers whole row
+// slices with 16-byte vectors.  The column reductions are a shuffle inside the
+// warp (when a warp spans several rows) and one shared-memory pass across the
+// 8 warps.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -25,13 +28,13 @@
 
 namespace kda {
 
-template <int DK, int DV, typename TIn>
-__global__ void __launch_bounds__(256, 2) decode_kernel(
+template <int DK, int DV, int DVS, typename TIn>
+__global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2) decode_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
     const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
     TIn* __restrict__ o) {
     constexpr int NW = 8;              // warps per CTA
-    constexpr int LPR = DV / 4;        // lanes per row (float4 each)
+    constexpr int LPR = DVS / 4;       // lanes per row slice (float4 each)
     constexpr int RPW = 32 / LPR;      // rows per warp per pass
     constexpr int RP = NW * RPW;       // rows per pass
     constexpr int NP = DK / RP;        // passes (float4 registers per thread)
@@ -42,16 +45,18 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(
     __shared__ float s_kq;
 
     const int unit = blockIdx.x;  // (sequence, head)
+    const int j0 = blockIdx.y * DVS;  // first value column of this slice
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int rw = lane / LPR, c4 = lane % LPR;
-    float4* S = reinterpret_cast<float4*>(state + (size_t)unit * DK * DV);
+    // row r of the slice starts at float4 index r * (DV / 4) + j0 / 4
+    float4* S = reinterpret_cast<float4*>(state + (size_t)unit * DK * DV + j0);
 
     // 1. stream the state in (independent of everything else: issue first)
     float4 x[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const int row = p * RP + w * RPW + rw;
-        x[p] = __ldcs(S + row * LPR + c4);
+        x[p] = __ldcs(S + row * (DV / 4) + c4);
     }
     // 2. the token's vectors into shared memory
     for (int c = tid; c < DK; c += blockDim.x) {
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(
     }
     // 4. u = beta (v - Sbar^T k) for this thread's four columns
     const float b = beta[unit];
-    const size_t vo = (size_t)unit * DV + 4 * c4;
+    const size_t vo = (size_t)unit * DV + j0 + 4 * c4;
     float4 u;
     u.x = b * (to_f32(v[vo + 0]) - sk.x);
     u.y = b * (to_f32(v[vo + 1]) - sk.y);
@@ -117,7 +122,7 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(
         const float kc = s_k[row];
         float4 y = x[p];
         y.x += kc * u.x; y.y += kc * u.y; y.z += kc * u.z; y.w += kc * u.w;
-        __stcs(S + row * LPR + c4, y);
+        __stcs(S + row * (DV / 4) + c4, y);
     }
     // 6. o = Sbar^T q + u (k^T q)
     if (w == 0 && rw == 0) {
@@ -137,10 +142,12 @@ static cudaError_t decode_dispatch(const void* q, const void* k, const void* v, 
     const TIn* K = (const TIn*)k;
     const TIn* V = (const TIn*)v;
     TIn* O = (TIn*)o;
-#define KDA_DECODE_CASE(A, B)                                                          \
-    if (dk == A && dv == B) {                                                          \
-        decode_kernel<A, B, TIn><<<units, 256, 0, st>>>(Q, K, V, g, beta, state, O); \
-        return cudaGetLastError();                                                     \
+#define KDA_DECODE_CASE(A, B)                                                           \
+    if (dk == A && dv == B) {                                                           \
+        constexpr int DVS = (B == 128) ? 64 : B;                                        \
+        const dim3 grid(units, B / DVS);                                                \
+        decode_kernel<A, B, DVS, TIn><<<grid, 256, 0, st>>>(Q, K, V, g, beta, state, O); \
+        return cudaGetLastError();                                                      \
     }
     KDA_DECODE_CASE(128, 128)
     KDA_DECODE_CASE(128, 64)
