@@ -181,7 +181,7 @@ def run_ours(args, rank, world, local_rank):
     kda.load()
 
     # ---- inputs (resident in HBM before timing)
-    pc = wl.prefill_config(1)
+    pc = wl.prefill_config(args.prefill_config)
     P = pc.to(dev)
     dcase = wl.decode_config()
     D = [{k: v.to(dev) for k, v in s.items()} for s in dcase.steps]
@@ -195,9 +195,11 @@ def run_ours(args, rank, world, local_rank):
     od = torch.empty(Nd, H, dv, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
+
     def prefill():
-        kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, None, P.B, P.T, Np, H,
-                          dk, dv, C, "bf16", o, hN, ws)
+        kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc, Tc, Np,
+                          H, dk, dv, C, "bf16", o, hN, ws)
 
     def decode(i):
         s = D[i % len(D)]
@@ -272,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; distributions of the pages' configurations)",
         "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": H, "dk": dk, "dv": dv,
-                   "chunk": C, "decode_workload": dcase.name,
+                   "chunk": C, "prefill_path": kern["path"], "decode_workload": dcase.name,
                    "l2": "flushed (256 MiB write) before each leg",
                    "parallelism": f"replicas x{world}"},
         "prefill": {"value": value, "unit": "tokens/s", "ms_per_call": pre_avg * 1e3,
@@ -295,17 +297,32 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
+def prefill_path(Np, H, dk, dv, C, dtype="bf16"):
+    """Which prefill kernels kda_chunk_fwd runs (the library's rule, see
+    include/kda.h): 'fused' (one tensor-core kernel), 'split' (chunk-parallel
+    intra kernel + per-chain kernel) or 'simt' (CUDA-core kernels)."""
+    import torch
+    env = os.environ.get("KDA_CHUNK_PATH")
+    if env == "simt" or not (dtype == "bf16" and dk == dv == 128 and C == 64):
+        return "simt"
+    if env in ("fused", "split"):
+        return env
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return "split" if Np * H < 2 * sms else "fused"
+
+
 def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     """Times of the prefill kernels.  For the CUDA-core path: each step call
-    (a1..a4) on its own; for the tensor-core path: the single fused kernel is
-    the whole call."""
+    (a1..a4) on its own; for the tensor-core paths: the whole call (one fused
+    kernel, or the intra + chain pair of the split path)."""
     import torch
     Np, H, dk, dv, C, total = P.N, P.H, P.dk, P.dv, P.chunk, P.total
-    tc = kda.kda_chunk_fwd_workspace_size(total, Np, H, dk, dv, C, "bf16") < \
-        kda.kda_chunk_fwd_workspace_size(total, Np, H, dk, dv, C, "f32")
+    path = prefill_path(Np, H, dk, dv, C)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     in_b = 2
-    if tc:
+    Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
+    if path != "simt":
+        name = "chunk_fwd_tc" if path == "fused" else "chunk_fwd_split(intra+chain)"
         o = torch.empty_like(P.v)
         hN = torch.empty(Np, H, dk, dv, device=dev)
         ts = []
@@ -313,15 +330,15 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, None, P.B, P.T, Np,
-                              H, dk, dv, C, "bf16", o, hN, ws)
+            kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc,
+                              Tc, Np, H, dk, dv, C, "bf16", o, hN, ws)
             b.record(stream)
             ts.append((a, b))
         torch.cuda.synchronize()
         t = statistics.median(a.elapsed_time(b) for a, b in ts) / 1e3
         nb = prefill_bytes(total * H, Np * H)
-        return {"times": {"chunk_fwd_tc": t}, "bytes": {"chunk_fwd_tc": nb},
-                "dominant": ("chunk_fwd_tc", t), "launches_per_call": 2}
+        return {"times": {name: t}, "bytes": {name: nb}, "dominant": (name, t),
+                "launches_per_call": 2 if path == "fused" else 3, "path": path}
     G = torch.empty(total, H, dk, device=dev)
     W = torch.empty(total, H, dk, device=dev)
     U = torch.empty(total, H, dv, device=dev)
@@ -329,7 +346,7 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     S = torch.empty(maxc, H, dk, dv, device=dev)
     hN = torch.empty(Np, H, dk, dv, device=dev)
     o = torch.empty_like(P.v)
-    a = (None, P.B, P.T, Np, H)
+    a = (P.cu_seqlens, Bc, Tc, Np, H)
     calls = {
         "a1_gate_cumsum": lambda: kda.kda_chunk_gate_cumsum(P.g, *a, dk, C, G, ws),
         "a2_intra": lambda: kda.kda_chunk_intra(P.k, P.v, G, P.beta, *a, dk, dv, C, "bf16", W,
@@ -366,7 +383,7 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
         times[name] = statistics.median(x.elapsed_time(y) for x, y in ts) / 1e3
     dom = max(times, key=times.get)
     return {"times": times, "bytes": nbytes, "dominant": (dom, times[dom]),
-            "launches_per_call": 5}
+            "launches_per_call": 5, "path": path}
 
 
 def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
@@ -383,10 +400,15 @@ def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
     hhN = torch.empty(N, H, dk, dv).pin_memory()
     ws = kda.alloc_workspace(total, N, H, dk, dv, C, "bf16", dev)
 
+    hcu = None if pc.cu_seqlens is None else pc.cu_seqlens.pin_memory()
+    dcu = None if hcu is None else torch.empty_like(hcu, device=dev)
+    Bc, Tc = (1, total) if hcu is not None else (pc.B, pc.T)
+
     def one():
-        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (d0, h0)):
-            d.copy_(h, non_blocking=True)
-        kda.kda_chunk_fwd(dq, dk_, dv_, dg, db, d0, None, pc.B, pc.T, N, H, dk, dv, C, "bf16",
+        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (d0, h0), (dcu, hcu)):
+            if d is not None:
+                d.copy_(h, non_blocking=True)
+        kda.kda_chunk_fwd(dq, dk_, dv_, dg, db, d0, dcu, Bc, Tc, N, H, dk, dv, C, "bf16",
                           o, hN, ws)
         ho.copy_(o, non_blocking=True)
         hhN.copy_(hN, non_blocking=True)
@@ -401,7 +423,8 @@ def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
     b.record(stream)
     torch.cuda.synchronize()
     t = a.elapsed_time(b) / 1e3 / steps
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb, h0))
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb, h0, hcu)
+              if x is not None)
     d2h = ho.numel() * ho.element_size() + hhN.numel() * hhN.element_size()
 
     # decode: per step the token's inputs go up and o comes back
@@ -504,6 +527,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-config", type=int, default=1, choices=[1, 2, 3],
+                    help="prefill workload: 1 = B=2 x T=2048 (default), 2 = B=1 x T=65536, "
+                         "3 = 16 packed sequences of U[1024,16384] tokens")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

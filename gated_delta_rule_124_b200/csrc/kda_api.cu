@@ -3,6 +3,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <stdlib.h>
+#include <string.h>
+
 #include <initializer_list>
 
 #include "kda.h"
@@ -43,22 +46,50 @@ kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, 
     return KDA_OK;
 }
 
-bool use_tc_path(int dk, int dv, int chunk, kda_dtype_t dt) {
-    return kda::tc_path_available() && dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 &&
-           chunk == 64;
+// Which kernels kda_chunk_fwd runs.
+enum class Path { Simt, Fused, Split };
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+// bf16, dk = dv = 128, chunk 64 runs on the tensor cores: one kernel with one
+// CTA per (sequence, head) when there are enough of them to fill the GPU,
+// otherwise the two-kernel split (chunk-parallel intra-chunk kernel + per-chain
+// kernel).  KDA_CHUNK_PATH = fused | split | simt forces a path (testing).
+Path select_path(int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
+    const bool tc_shape = dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
+                          kda::tc_path_available();
+    const char* env = getenv("KDA_CHUNK_PATH");
+    if (env && !strcmp(env, "simt")) return Path::Simt;
+    if (!tc_shape) return Path::Simt;
+    if (env && !strcmp(env, "fused")) return Path::Fused;
+    if (env && !strcmp(env, "split")) return Path::Split;
+    return ((long long)N * H < 2LL * sm_count()) ? Path::Split : Path::Fused;
+}
+
+Workspace carve_for(void* base, const Prefill& p, int H, int dk, int dv, int chunk, Path path) {
+    return kda::carve(base, p.total, p.N, H, dk, dv, chunk, path == Path::Simt,
+                      path == Path::Split ? kda::split_blob_bytes() : 0);
 }
 
 size_t workspace_bytes_for(int total, int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
-    const bool inter = !use_tc_path(dk, dv, chunk, dt);
-    Workspace w = kda::carve(nullptr, total, N, H, dk, dv, chunk, inter);
-    return w.total_bytes;
+    const Prefill p{total, N};
+    return carve_for(nullptr, p, H, dk, dv, chunk, select_path(N, H, dk, dv, chunk, dt))
+        .total_bytes;
 }
 
 kda_status_t check_ws(void* ws, size_t bytes, const Prefill& p, int H, int dk, int dv,
-                      int chunk, kda_dtype_t dt, Workspace* out, bool need_intermediates) {
+                      int chunk, Path path, Workspace* out) {
     if (!ws) return KDA_ERR_WORKSPACE;
     if (!aligned256(ws)) return KDA_ERR_INVALID_ARG;
-    Workspace w = kda::carve(ws, p.total, p.N, H, dk, dv, chunk, need_intermediates);
+    Workspace w = carve_for(ws, p, H, dk, dv, chunk, path);
     if (bytes < w.total_bytes) return KDA_ERR_WORKSPACE;
     *out = w;
     return KDA_OK;
@@ -122,19 +153,25 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
         if (!aligned16(ptr)) return KDA_ERR_INVALID_ARG;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_INVALID_ARG;
-    const bool tc = use_tc_path(dk, dv, chunk, dtype);
+    const Path path = select_path(p.N, H, dk, dv, chunk, dtype);
     Workspace w;
-    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, dtype, &w, !tc);
+    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, path, &w);
     if (s != KDA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int maxc = kda::max_chunks(p.total, p.N, chunk);
     s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);
     if (s != KDA_OK) return s;
     if (p.total == 0 && !final_state) return KDA_OK;
-    if (tc) {
+    if (path == Path::Fused) {
         return from_cuda(kda::launch_chunk_fwd_tc(q, k, v, g, beta, initial_state, cu_seqlens,
                                                   T, p.N, H, w.chunk_start, w.status, o,
                                                   final_state, st));
+    }
+    if (path == Path::Split) {
+        return from_cuda(kda::launch_chunk_fwd_split(q, k, v, g, beta, initial_state,
+                                                     cu_seqlens, T, p.N, H, w.chunk_info, maxc,
+                                                     w.chunk_start, w.status, w.blobs, o,
+                                                     final_state, st));
     }
     cudaError_t e = kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
     if (e == cudaSuccess)
@@ -160,7 +197,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
     for (const void* ptr : std::initializer_list<const void*>{__VA_ARGS__})              \
         if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;                          \
     Workspace w;                                                                          \
-    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, dtype, &w, false);      \
+    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, Path::Fused, &w);       \
     if (s != KDA_OK) return s;                                                            \
     cudaStream_t st = static_cast<cudaStream_t>(stream);                                  \
     const int maxc = kda::max_chunks(p.total, p.N, chunk);

@@ -1,0 +1,831 @@
+// KDA chunkwise prefill, split into two tensor-core kernels (bf16, dk = dv =
+// 128, chunk 64) for problems with few (sequence, head) chains, where one CTA
+// per chain would leave most SMs idle:
+//
+//   chunk_intra_kernel  one CTA per (chunk, head), all chunks in parallel: the
+//                       in-chunk cumulative log-gate, the operand tiles, A and
+//                       P, the UT transform T = (I + A)^{-1} and
+//                       W = T diag(b) (K * Gam); it writes the chain's operands
+//                       for that chunk to the workspace as one blob laid out
+//                       exactly as the chain kernel's shared memory wants it.
+//   chunk_chain_kernel  one CTA per (sequence, head), chunks in order: bulk
+//                       copies of each chunk's blob (double-buffered) and V,
+//                       then Ut = Tb V, X = [W ; Q*Gam] S, U = Ut - W S,
+//                       O = X + [. ; P] U and S <- Gam_last S + K~^T U, with
+//                       S carried in fp32 in tensor memory.
+//
+// The arithmetic of each step is the same code as the single-kernel path in
+// kda_chunk_tc.cu (same operand layouts and factorisation of the gate; see
+// there); only where each step runs, and the hand-off through the workspace,
+// differ.  Kimi Linear (aiwiki.ai), "The constrained DPLR form and the
+// chunkwise algorithm": parallel inside a chunk, recurrent between chunks --
+// this split runs the first part on every SM and keeps only the second on the
+// per-chain critical path.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include "kda_chunk_tc.cuh"
+#include "kda_common.cuh"
+#include "kda_sm100.cuh"
+#include "kda_tc_util.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int NT = 512;
+constexpr float kRef = 80.f;
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+// ---- per (chunk, head) blob in the workspace (each part 1024-byte aligned)
+constexpr uint32_t BL_WQ = 0;        // [W kb0 | Q*Gam kb0 | W kb1 | Q*Gam kb1]   32 KB
+constexpr uint32_t BL_RAP = 32768;   // K * E^-1 (or K * exp(G_last - G))         16 KB
+constexpr uint32_t BL_PM = 49152;    // P (masked), rows 64-127 of its operand      8 KB
+constexpr uint32_t BL_TB = 57344;    // T diag(b), rows 0-63 of its operand         8 KB
+constexpr uint32_t BL_SC = 65536;    // exp(G_last)[128], row scale of K~^T U [128]  1 KB
+constexpr uint32_t BLOB = 66560;
+
+}  // namespace
+
+size_t split_blob_bytes() { return BLOB; }
+
+namespace {
+
+// ===================================================================== intra
+namespace intra {
+constexpr uint32_t OFF_K = 0;          // K (TMA); exact path: K * Gam in place
+constexpr uint32_t OFF_RAP = 16384;    // K * E^-1
+constexpr uint32_t OFF_WQ = 32768;     // [W kb0 | Q kb0 | W kb1 | Q kb1]
+constexpr uint32_t OFF_G = 65536;      // g (TMA) -> G -> A fp32 | T fp32
+constexpr uint32_t OFF_LAP = 98304;    // [K * E ; Q * E]; exact path: A | P fp32
+constexpr uint32_t OFF_TB = 131072;    // T diag(b) rows 0-63
+constexpr uint32_t OFF_MID = 139264;   // scratch; garbage rows of the Tb and P operands
+constexpr uint32_t OFF_PM = 147456;    // P rows 64-127
+constexpr uint32_t OFF_BETA = 155648;
+constexpr uint32_t OFF_GM = OFF_BETA + 256;
+constexpr uint32_t OFF_EGM = OFF_GM + 512;
+constexpr uint32_t OFF_GC = OFF_EGM + 512;
+constexpr uint32_t OFF_GL = OFF_GC + 512;
+constexpr uint32_t OFF_WSC = OFF_GL + 512;
+constexpr uint32_t OFF_KSC = OFF_WSC + 512;
+constexpr uint32_t OFF_BAR = OFF_KSC + 512;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+static_assert(OFF_PM == OFF_MID + 8192, "P rows follow the garbage rows");
+constexpr uint32_t TM_X = 0;     // A|P
+constexpr uint32_t TM_W = 128;   // W
+constexpr uint32_t TX_BYTES = 2 * 16384 + 32768;
+
+struct Params {
+    const float* beta;
+    const int4* info;
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    uint8_t* blobs;
+};
+
+__global__ void __launch_bounds__(NT, 1)
+    chunk_intra_kernel(const __grid_constant__ CUtensorMap tmq,
+                       const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmg, const Params p) {
+    if (status_bad(p.status)) return;
+    const int4 ci = p.info[blockIdx.x];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int h = blockIdx.y, t0 = ci.y;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* sbeta = reinterpret_cast<float*>(sm + OFF_BETA);
+    float* sGm = reinterpret_cast<float*>(sm + OFF_GM);
+    float* seGm = reinterpret_cast<float*>(sm + OFF_EGM);
+    float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
+    float* sGL = reinterpret_cast<float*>(sm + OFF_GL);
+    float* sWsc = reinterpret_cast<float*>(sm + OFF_WSC);
+    float* sKsc = reinterpret_cast<float*>(sm + OFF_KSC);
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_mma = bar_tma + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int quarter = warp & 3, cq = warp >> 2, lane = tid & 31;
+    const int trow = 32 * quarter + (tid & 31);
+    const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
+    uint8_t* blob = p.blobs + ((size_t)blockIdx.x * p.H + h) * BLOB;
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    bool failed = false;
+    uint32_t mma_phase = 0;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_tma, TX_BYTES);
+        tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, h, t0);
+        tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, h, t0);
+        tma_load_3d(sm + OFF_WQ + 8192, &tmq, bar_tma, 0, h, t0);
+        tma_load_3d(sm + OFF_WQ + 16384 + 8192, &tmq, bar_tma, 64, h, t0);
+        tma_load_3d(sm + OFF_G, &tmg, bar_tma, 0, h, t0);
+    }
+    if (tid < C) sbeta[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * p.H + h] : 0.f;
+    do {
+        bool ok = mbar_wait(bar_tma, 0, kWaitNs);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        // -------------------- E1: in-chunk cumulative log-gate, per channel
+        bool slow_local = false;
+        if (tid < D) {
+            float* g = reinterpret_cast<float*>(sm + OFF_G);
+            const int c = tid;
+            float x[C];
+#pragma unroll
+            for (int r = 0; r < C; ++r) x[r] = g[r * D + c];
+            float G = 0.f, gmax = -INFINITY, gmin = INFINITY;
+#pragma unroll
+            for (int r = 0; r < C; ++r) {
+                if (r < L) {
+                    G += x[r];
+                    gmax = fmaxf(gmax, G);
+                    gmin = fminf(gmin, G);
+                }
+                x[r] = G;
+            }
+#pragma unroll
+            for (int r = 0; r < C; ++r) g[r * D + c] = x[r];
+            const float Gm = gmax - kRef;
+            sGm[c] = Gm;
+            seGm[c] = expf(Gm);
+            sGC[c] = expf(G);
+            sGL[c] = G;
+            slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
+        }
+        const bool slow = __syncthreads_or(slow_local);
+        if (tid < D) {
+            sWsc[tid] = slow ? 1.f : seGm[tid];
+            sKsc[tid] = slow ? 1.f : expf(sGL[tid] - sGm[tid]);
+        }
+        // ---------------- exact A and P on CUDA cores (rare: extreme decay)
+        if (slow) {
+            const float* G = reinterpret_cast<const float*>(sm + OFF_G);
+            float* Af = reinterpret_cast<float*>(sm + OFF_LAP);
+            float* Pf = Af + C * C;
+            for (int idx = tid; idx < C * C; idx += NT) {
+                const int r = idx >> 6, i = idx & 63;
+                float a = 0.f, pp = 0.f;
+                if (r < L && i <= r) {
+                    for (int c = 0; c < D; ++c) {
+                        const float e = expf(G[r * D + c] - G[i * D + c]);
+                        const float ki = tile_elem(sm + OFF_K, 8192, i, c);
+                        a += tile_elem(sm + OFF_K, 8192, r, c) * ki * e;
+                        pp += tile_elem(sm + OFF_WQ + 8192, 16384, r, c) * ki * e;
+                    }
+                }
+                Af[a_idx(r, i)] = (i < r) ? sbeta[r] * a : 0.f;
+                Pf[idx] = pp;
+            }
+            __syncthreads();
+        }
+        // ------------------------------ E2: operand tiles, row-parallel
+        {
+            const float* G = reinterpret_cast<const float*>(sm + OFF_G);
+#pragma unroll
+            for (int s = 0; s < (C * 16) / NT; ++s) {
+                const int it = tid + NT * s;
+                const int r = it >> 4, j = it & 15, kb = j >> 3, ch = j & 7, c0 = 8 * j;
+                const uint32_t o64 = sw128_off(r, ch);
+                uint8_t* pk = sm + OFF_K + kb * 8192 + o64;
+                uint8_t* pq = sm + OFF_WQ + kb * 16384 + 8192 + o64;
+                uint8_t* pr = sm + OFF_RAP + kb * 8192 + o64;
+                float lk[8], lq[8], rk[8], qg[8];
+                if (r < L) {
+                    float k8[8], q8[8], g8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(pk), k8);
+                    unpack8(*reinterpret_cast<const uint4*>(pq), q8);
+                    load8(G + r * D + c0, g8);
+                    if (!slow) {
+                        float m8[8], e8[8];
+                        load8(sGm + c0, m8);
+                        load8(seGm + c0, e8);
+                        // factors within exp(+-80), rounded to bf16 right after
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float x = g8[i] - m8[i];
+                            const float E = __expf(x), Ei = __expf(-x);
+                            lk[i] = k8[i] * E;
+                            lq[i] = q8[i] * E;
+                            rk[i] = k8[i] * Ei;
+                            qg[i] = lq[i] * e8[i];
+                        }
+                    } else {
+                        float l8[8];
+                        load8(sGL + c0, l8);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float gam = expf(g8[i]);
+                            lk[i] = k8[i] * gam;  // K * Gam, in place of K
+                            lq[i] = 0.f;
+                            rk[i] = k8[i] * expf(l8[i] - g8[i]);
+                            qg[i] = q8[i] * gam;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) lk[i] = lq[i] = rk[i] = qg[i] = 0.f;
+                }
+                if (!slow) {
+                    *reinterpret_cast<uint4*>(sm + OFF_LAP + kb * 16384 + o64) = pack8(lk);
+                    *reinterpret_cast<uint4*>(sm + OFF_LAP + kb * 16384 + 8192 + o64) =
+                        pack8(lq);
+                } else {
+                    *reinterpret_cast<uint4*>(pk) = pack8(lk);
+                }
+                *reinterpret_cast<uint4*>(pr) = pack8(rk);
+                *reinterpret_cast<uint4*>(pq) = pack8(qg);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ------------------------------------------------ A, P (M=128, N=64)
+        if (!slow) {
+            if (tid == 0) {
+                constexpr uint32_t id = idesc_bf16_f32(128, 64, false, false);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int kb = ks >> 2, kk = ks & 3;
+                    mma_bf16(tbase + TM_X,
+                             sdesc_sw128(sbase + OFF_LAP + kb * 16384 + kk * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_RAP + kb * 8192 + kk * 32, 16, 1024), id,
+                             ks > 0);
+                }
+                mma_commit(bar_mma);
+            }
+            ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+            ++mma_phase;
+            if (__syncthreads_or(!ok)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+        }
+        // ----- A -> fp32 (swizzled, in the G region), P -> bf16 PM rows 64-127
+        {
+            float* Af = reinterpret_cast<float*>(sm + OFF_G);
+            const int m = trow;  // TMEM lane == row of the 128-row result
+            if (!slow) {
+                if (cq < 2) {
+                    uint32_t v[32];
+                    tmem_ld32(tbase + tlane + TM_X + cq * 32, v);
+                    tmem_wait_ld();
+                    if (m < C) {
+                        const float b = sbeta[m];
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const int col = cq * 32 + 4 * i4;
+                            float y[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                y[i] = (m < L && col + i < m) ? b * __uint_as_float(v[4 * i4 + i])
+                                                              : 0.f;
+                            *reinterpret_cast<float4*>(Af + a_idx(m, col)) =
+                                make_float4(y[0], y[1], y[2], y[3]);
+                        }
+                    } else {
+                        const int r = m - C;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            float y[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int col = cq * 32 + q4 * 8 + i;
+                                y[i] = (r < L && col <= r) ? __uint_as_float(v[q4 * 8 + i]) : 0.f;
+                            }
+                            *reinterpret_cast<uint4*>(sm + OFF_MID +
+                                                      sw128_off(m, (cq * 32 + q4 * 8) >> 3)) =
+                                pack8(y);
+                        }
+                    }
+                }
+            } else {
+                const float4* srcA = reinterpret_cast<const float4*>(sm + OFF_LAP);
+                float4* dstA = reinterpret_cast<float4*>(Af);
+                for (int i = tid; i < C * C / 4; i += NT) dstA[i] = srcA[i];
+                if (m >= C && cq < 2) {
+                    const float* Pf = reinterpret_cast<const float*>(sm + OFF_LAP) + C * C;
+                    const int r = m - C;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float y[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int col = cq * 32 + q4 * 8 + i;
+                            y[i] = (r < L && col <= r) ? Pf[r * C + col] : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(sm + OFF_MID +
+                                                  sw128_off(m, (cq * 32 + q4 * 8) >> 3)) =
+                            pack8(y);
+                    }
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ------------------ UT transform: T = (I + A)^{-1}, blocked 16 x 16
+        {
+            const float* Af = reinterpret_cast<const float*>(sm + OFF_G);
+            float* Tf = reinterpret_cast<float*>(sm + OFF_G + 16384);
+            float* Mf = reinterpret_cast<float*>(sm + OFF_MID);
+            if (tid < C) {
+                // diagonal blocks, right-looking forward substitution: one
+                // column of one block per thread
+                const int I = tid >> 4, jj = tid & 15, col = 16 * I + jj;
+                float pv[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) pv[rr] = (rr == jj) ? 1.f : 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const float x = pv[rr];
+                    Tf[t_idx(16 * I + rr, col)] = x;
+#pragma unroll
+                    for (int r2 = rr + 1; r2 < 16; ++r2)
+                        pv[r2] -= Af[a_idx(16 * I + r2, 16 * I + rr)] * x;
+                }
+            }
+            __syncthreads();
+            offdiag_level<1>(Af, Tf, Mf, warp, lane);
+            offdiag_level<2>(Af, Tf, Mf, warp, lane);
+            offdiag_level<3>(Af, Tf, Mf, warp, lane);
+            // Tb = T diag(b) -> bf16, K-major rows of 64 (rows 0-63)
+            for (int e = tid; e < C * 8; e += NT) {
+                const int r = e >> 3, ch = e & 7;
+                const float4 t0v = *reinterpret_cast<const float4*>(Tf + t_idx(r, 8 * ch));
+                const float4 t1v = *reinterpret_cast<const float4*>(Tf + t_idx(r, 8 * ch + 4));
+                const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int col = 8 * ch + i;
+                    y[i] = (col <= r) ? tv[i] * sbeta[col] : 0.f;
+                }
+                *reinterpret_cast<uint4*>(sm + OFF_TB + sw128_off(r, ch)) = pack8(y);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ---------------------------------- W = Tb (K*E) [*exp(Gm)]  (N=128)
+        if (tid == 0) {
+            constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
+            const uint32_t bW = slow ? OFF_K : OFF_LAP;
+            const uint32_t lboW = slow ? 8192u : 16384u;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tbase + TM_W, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
+                         sdesc_sw128(sbase + bW + ks * 2048, lboW, 1024), id, ks > 0);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ++mma_phase;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        // W (rows 0-63), column-scaled -> bf16 into the W rows of [W ; Q*Gam]
+        if (quarter < 2) {
+            const int r = trow;
+            uint32_t v[32];
+            tmem_ld32(tbase + tlane + TM_W + cq * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int col = cq * 32 + q4 * 8;
+                float sc[8], y[8];
+                load8(sWsc + col, sc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]) * sc[i];
+                *reinterpret_cast<uint4*>(sm + OFF_WQ + (col >> 6) * 16384 +
+                                          sw128_off(r, (col & 63) >> 3)) = pack8(y);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ---- hand the chain's operands to the workspace
+        if (tid == 0) {
+            bulk_s2g(blob + BL_WQ, sm + OFF_WQ, 32768);
+            bulk_s2g(blob + BL_RAP, sm + OFF_RAP, 16384);
+            bulk_s2g(blob + BL_PM, sm + OFF_PM, 8192);
+            bulk_s2g(blob + BL_TB, sm + OFF_TB, 8192);
+            bulk_commit();
+        }
+        if (tid < D) {
+            float* sc = reinterpret_cast<float*>(blob + BL_SC);
+            sc[tid] = sGC[tid];
+            sc[D + tid] = sKsc[tid];
+        }
+        if (tid == 0) bulk_wait_all();
+    } while (false);
+    if (failed && tid == 0) {
+        if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
+        mbar_wait(bar_tma, 0, kWaitNs);
+        atomicOr(p.status_out, STATUS_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+}
+}  // namespace intra
+
+// ===================================================================== chain
+namespace chain {
+constexpr uint32_t OFF_WQ = 0;         // [W | Q*Gam] blob part
+constexpr uint32_t OFF_RAP0 = 32768;   // K E^-1, two buffers
+constexpr uint32_t OFF_RAP1 = 49152;
+constexpr uint32_t OFF_PM0 = 65536;    // P rows 64-127, two buffers; the operand starts
+constexpr uint32_t OFF_PM1 = 73728;    //   8 KB earlier (rows 0-63: whatever is there)
+constexpr uint32_t OFF_TB = 81920;     // Tb rows 0-63; its rows 64-127 are the V tile
+constexpr uint32_t OFF_V = 90112;      // V (TMA)
+constexpr uint32_t OFF_SB = 106496;    // S bf16 [dk][dv]
+constexpr uint32_t OFF_UB = 139264;    // U bf16 [token][dv]
+constexpr uint32_t OFF_SC0 = 155648;   // exp(G_last), row scale: two buffers of 1 KB
+constexpr uint32_t OFF_SC1 = 156672;
+constexpr uint32_t OFF_BAR = 157696;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+static_assert(OFF_V == OFF_TB + 8192, "Tb garbage rows");
+constexpr uint32_t TM_W = 0;     // (K E^-1)^T U
+constexpr uint32_t TM_UT = 128;  // Ut
+constexpr uint32_t TM_X = 256;   // [W;QGam] S, then O
+constexpr uint32_t TM_S = 384;   // fp32 state
+constexpr uint32_t TX_BYTES = 32768 + 16384 + 8192 + 8192 + 16384 + 1024;
+
+struct Params {
+    const float* h0;
+    const int32_t* cu;
+    int T;
+    int H;
+    const int* chunk_start;
+    const uint32_t* status;
+    uint32_t* status_out;
+    const uint8_t* blobs;
+    __nv_bfloat16* o;
+    float* hN;
+};
+
+__global__ void __launch_bounds__(NT, 1)
+    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
+    if (status_bad(p.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_mma = bar_ld + 1;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int quarter = warp & 3, cq = warp >> 2;
+    const int trow = 32 * quarter + (tid & 31);
+    const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
+    const int seq = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int t_begin = p.cu ? p.cu[seq] : seq * p.T;
+    const int t_end = p.cu ? p.cu[seq + 1] : (seq + 1) * p.T;
+    const int cbase = p.chunk_start[seq];
+    auto blob = [&](int n) { return p.blobs + ((size_t)(cbase + n) * p.H + h) * BLOB; };
+
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    bool failed = false;
+    uint32_t mma_phase = 0;
+
+    if (tid == 0 && t_begin < t_end) {
+        const uint8_t* b0 = blob(0);
+        mbar_arrive_expect_tx(bar_ld, TX_BYTES);
+        bulk_g2s(sm + OFF_RAP0, b0 + BL_RAP, 16384, bar_ld);
+        bulk_g2s(sm + OFF_PM0, b0 + BL_PM, 8192, bar_ld);
+        bulk_g2s(sm + OFF_SC0, b0 + BL_SC, 1024, bar_ld);
+        bulk_g2s(sm + OFF_TB, b0 + BL_TB, 8192, bar_ld);
+        bulk_g2s(sm + OFF_WQ, b0 + BL_WQ, 32768, bar_ld);
+        tma_load_3d(sm + OFF_V, &tmv, bar_ld, 0, h, t_begin);
+        tma_load_3d(sm + OFF_V + 8192, &tmv, bar_ld, 64, h, t_begin);
+    }
+
+    // ---- initial state: fp32 into TMEM (row c = lane c), bf16 copy into Sb
+    {
+        const int c = trow;
+        const float* src = p.h0 ? p.h0 + (((size_t)seq * p.H + h) * D + c) * D : nullptr;
+        {
+            const int piece = cq;
+            uint32_t r[32];
+            float x[32];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                float4 v = src ? *reinterpret_cast<const float4*>(src + piece * 32 + i)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
+            tmem_st32(tbase + tlane + TM_S + piece * 32, r);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = x[q4 * 8 + i];
+                const int col = piece * 32 + q4 * 8;
+                *reinterpret_cast<uint4*>(sm + OFF_SB + (col >> 6) * 16384 +
+                                          sw128_off(c, (col & 63) >> 3)) = pack8(y);
+            }
+        }
+        tmem_wait_st();
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    int n = 0;
+    for (int t0 = t_begin; t0 < t_end && !failed; t0 += C, ++n) {
+        const int L = min(C, t_end - t0);
+        const int tn = t0 + C;
+        const bool has_next = tn < t_end;
+        const uint32_t pm_op = ((n & 1) ? OFF_PM1 : OFF_PM0) - 8192;
+        const uint32_t rap_op = (n & 1) ? OFF_RAP1 : OFF_RAP0;
+        const float* ssc = reinterpret_cast<const float*>(sm + ((n & 1) ? OFF_SC1 : OFF_SC0));
+        bool ok = mbar_wait(bar_ld, n & 1, kWaitNs);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        if (has_next && tid == 0) {  // double-buffered parts of the next chunk
+            const uint8_t* bn = blob(n + 1);
+            mbar_arrive_expect_tx(bar_ld, TX_BYTES);
+            bulk_g2s(sm + ((n & 1) ? OFF_RAP0 : OFF_RAP1), bn + BL_RAP, 16384, bar_ld);
+            bulk_g2s(sm + ((n & 1) ? OFF_PM0 : OFF_PM1), bn + BL_PM, 8192, bar_ld);
+            bulk_g2s(sm + ((n & 1) ? OFF_SC0 : OFF_SC1), bn + BL_SC, 1024, bar_ld);
+        }
+        // -------------------------------------------------- Ut = Tb V  (N=128)
+        if (tid == 0) {
+            constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tbase + TM_UT, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
+                         sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id, ks > 0);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ++mma_phase;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        if (has_next && tid == 0) {  // V and Tb regions are free
+            bulk_g2s(sm + OFF_TB, blob(n + 1) + BL_TB, 8192, bar_ld);
+            tma_load_3d(sm + OFF_V, &tmv, bar_ld, 0, h, tn);
+            tma_load_3d(sm + OFF_V + 8192, &tmv, bar_ld, 64, h, tn);
+        }
+        // ------------------------------- X = [W ; Q*Gam] S   (M=128, N=128)
+        if (tid == 0) {
+            constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int kb = ks >> 2, kk = ks & 3;
+                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
+                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ++mma_phase;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        if (has_next && tid == 0)  // the [W ; Q*Gam] region is free
+            bulk_g2s(sm + OFF_WQ, blob(n + 1) + BL_WQ, 32768, bar_ld);
+        // U = Ut - W S  (rows 0-63) -> bf16 Ub
+        if (quarter < 2) {
+            const int r = trow;
+            uint32_t a[32], b[32];
+            tmem_ld32(tbase + tlane + TM_UT + cq * 32, a);
+            tmem_ld32(tbase + tlane + TM_X + cq * 32, b);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int col = cq * 32 + q4 * 8;
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    y[i] = __uint_as_float(a[q4 * 8 + i]) - __uint_as_float(b[q4 * 8 + i]);
+                *reinterpret_cast<uint4*>(sm + OFF_UB + (col >> 6) * 8192 +
+                                          sw128_off(r, (col & 63) >> 3)) = pack8(y);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ---- O = X[64:] + [. ; P] U  (accumulate);  (K E^-1)^T U -> TM_W
+        if (tid == 0) {
+            constexpr uint32_t idP = idesc_bf16_f32(128, 128, false, true);
+            constexpr uint32_t idK = idesc_bf16_f32(128, 128, true, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + pm_op + ks * 32, 16, 1024),
+                         sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idP, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tbase + TM_W, sdesc_sw128(sbase + rap_op + ks * 2048, 8192, 1024),
+                         sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idK, ks > 0);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ++mma_phase;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        // S <- Gam_last * S + ksc * (K E^-1)^T U   (lane = state row c); O rows out
+        {
+            const int c = trow;
+            const float gc = ssc[c], ks = ssc[D + c];
+            uint32_t a[32], sv[32];
+            tmem_ld32(tbase + tlane + TM_W + cq * 32, a);
+            tmem_ld32(tbase + tlane + TM_S + cq * 32, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                sv[i] = __float_as_uint(fmaf(gc, __uint_as_float(sv[i]), ks * __uint_as_float(a[i])));
+            tmem_st32(tbase + tlane + TM_S + cq * 32, sv);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int col = cq * 32 + q4 * 8;
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(sv[q4 * 8 + i]);
+                *reinterpret_cast<uint4*>(sm + OFF_SB + (col >> 6) * 16384 +
+                                          sw128_off(c, (col & 63) >> 3)) = pack8(y);
+            }
+            if (quarter >= 2) {
+                const int r = trow - C;
+                uint32_t v[32];
+                tmem_ld32(tbase + tlane + TM_X + cq * 32, v);
+                tmem_wait_ld();
+                if (r < L) {
+                    __nv_bfloat16* dst = p.o + ((size_t)(t0 + r) * p.H + h) * D + cq * 32;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float y[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]);
+                        *reinterpret_cast<uint4*>(dst + q4 * 8) = pack8(y);
+                    }
+                }
+            }
+            tmem_wait_st();
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (!failed && p.hN) {
+        const int c = trow;
+        float* dst = p.hN + (((size_t)seq * p.H + h) * D + c) * D;
+        {
+            const int piece = cq;
+            uint32_t s[32];
+            tmem_ld32(tbase + tlane + TM_S + piece * 32, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(dst + piece * 32 + i) =
+                    make_float4(__uint_as_float(s[i]), __uint_as_float(s[i + 1]),
+                                __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+        }
+    }
+    if (failed && tid == 0) {
+        if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
+        mbar_wait(bar_ld, n & 1, kWaitNs);
+        atomicOr(p.status_out, STATUS_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+}  // namespace chain
+
+PFN_cuTensorMapEncodeTiled_v12000 split_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
+}
+
+bool split_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int total,
+               int H, int box0, CUtensorMapSwizzle sw) {
+    auto fn = split_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total};
+    cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)D * esize * H};
+    cuuint32_t box[3] = {(cuuint32_t)box0, 1, (cuuint32_t)C};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* h0,
+                                   const int32_t* cu_seqlens, int T, int N, int H,
+                                   const int4* chunk_info, int maxc, const int* chunk_start,
+                                   uint32_t* status, void* blobs, void* o, float* hN,
+                                   cudaStream_t st) {
+    const int total = cu_seqlens ? T : N * T;
+    if (total == 0) {
+        if (hN) {
+            if (h0) return cudaMemcpyAsync(hN, h0, sizeof(float) * (size_t)N * H * D * D,
+                                           cudaMemcpyDeviceToDevice, st);
+            return cudaMemsetAsync(hN, 0, sizeof(float) * (size_t)N * H * D * D, st);
+        }
+        return cudaSuccess;
+    }
+    CUtensorMap mq, mk, mv, mg;
+    if (!split_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)intra::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chain::chunk_chain_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)chain::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    uint8_t* bl = static_cast<uint8_t*>(blobs);
+    if (maxc > 0) {
+        intra::Params pa{beta, chunk_info, H, status, status, bl};
+        intra::chunk_intra_kernel<<<dim3(maxc, H), NT, intra::SMEM_BYTES, st>>>(mq, mk, mg, pa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    chain::Params pb{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
+                     (__nv_bfloat16*)o, hN};
+    chain::chunk_chain_kernel<<<N * H, NT, chain::SMEM_BYTES, st>>>(mv, pb);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -15,4 +15,15 @@ cudaError_t launch_chunk_fwd_tc(const void* q, const void* k, const void* v, con
                                 int T, int N, int H, const int* chunk_start,
                                 uint32_t* status, void* o, float* hN, cudaStream_t st);
 
+// Two-kernel split of the same computation for problems with few (sequence,
+// head) chains: chunk-parallel intra-chunk kernel + per-chain kernel, handing
+// over through `blobs` (split_blob_bytes() per (chunk slot, head)).
+size_t split_blob_bytes();
+cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* h0,
+                                   const int32_t* cu_seqlens, int T, int N, int H,
+                                   const int4* chunk_info, int maxc, const int* chunk_start,
+                                   uint32_t* status, void* blobs, void* o, float* hN,
+                                   cudaStream_t st);
+
 }  // namespace kda

@@ -16,7 +16,8 @@ namespace kda {
 //   chunk_info[maxc]      int4 {seq, first token, rows, chunk-in-sequence};
 //                         unused slots hold seq = -1, rows = 0
 //   then, for the CUDA-core path only: G, W, U (token-major fp32) and the
-//   per-chunk states [maxc, H, dk, dv] fp32.
+//   per-chunk states [maxc, H, dk, dv] fp32; for the split tensor-core path
+//   only: one operand blob per (chunk slot, head).
 constexpr size_t kAlign = 256;
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a = kAlign) {
@@ -34,6 +35,7 @@ struct Workspace {
     float* W;
     float* U;
     float* states;
+    uint8_t* blobs;
     size_t header_bytes;  // status + tables
     size_t total_bytes;   // header + CUDA-core path intermediates
 };
@@ -44,7 +46,7 @@ inline int max_chunks(int total_tokens, int num_seqs, int chunk) {
 }
 
 inline Workspace carve(void* base, int total, int N, int H, int dk, int dv, int chunk,
-                       bool with_intermediates) {
+                       bool with_intermediates, size_t blob_bytes = 0) {
     Workspace w{};
     const int maxc = max_chunks(total, N, chunk);
     char* p = static_cast<char*>(base);
@@ -65,6 +67,11 @@ inline Workspace carve(void* base, int total, int N, int H, int dk, int dv, int 
         off = align_up(off + sizeof(float) * (size_t)total * H * dv);
         w.states = reinterpret_cast<float*>(p + off);
         off = align_up(off + sizeof(float) * (size_t)maxc * H * dk * dv);
+    }
+    if (blob_bytes) {
+        off = align_up(off, 1024);
+        w.blobs = reinterpret_cast<uint8_t*>(p + off);
+        off = align_up(off + blob_bytes * (size_t)maxc * H);
     }
     w.total_bytes = off;
     return w;

@@ -230,3 +230,56 @@ def test_varlen_edge_lengths_bf16_d128(lens):
     case = wl.make_prefill(200 + sum(lens), lens, H=3, dk=128, dv=128, chunk=64, dtype="bf16",
                            varlen=True)
     check_case(case)
+
+
+# ----------------------------- every prefill path on the same problems
+# bf16, d = 128, chunk 64 can run as one tensor-core kernel per (sequence, head)
+# ("fused"), as the chunk-parallel + per-chain pair ("split"), or on the
+# CUDA-core kernels ("simt"); KDA_CHUNK_PATH forces the choice.
+
+PATH_CASES = {
+    "varlen": lambda: wl.make_prefill(301, [300, 77, 1, 128], H=4, dk=128, dv=128, chunk=64,
+                                      dtype="bf16", varlen=True),
+    "empty_seqs": lambda: wl.make_prefill(302, [0, 64, 0, 129, 7], H=3, dk=128, dv=128,
+                                          chunk=64, dtype="bf16", varlen=True),
+    "batched_tail": lambda: wl.make_prefill(303, [200] * 3, H=4, dk=128, dv=128, chunk=64,
+                                            dtype="bf16"),
+    "no_initial_state": lambda: wl.make_prefill(304, [150, 70], H=2, dk=128, dv=128, chunk=64,
+                                                dtype="bf16", varlen=True, init_std=None),
+    "strong_decay": lambda: wl.make_prefill(305, [256], H=2, dk=128, dv=128, chunk=64,
+                                            dtype="bf16", g_mu=4.0),
+}
+
+
+@pytest.fixture
+def chunk_path(request, monkeypatch):
+    monkeypatch.setenv("KDA_CHUNK_PATH", request.param)
+    return request.param
+
+
+@pytest.mark.parametrize("chunk_path", ["fused", "split", "simt"], indirect=True)
+@pytest.mark.parametrize("name", sorted(PATH_CASES))
+def test_every_path_matches_oracle(chunk_path, name):
+    case = PATH_CASES[name]()
+    check_case(case)
+
+
+@pytest.mark.parametrize("chunk_path", ["fused", "split"], indirect=True)
+def test_tc_paths_mixed_fast_and_exact_chunks(chunk_path):
+    case = wl.make_prefill(306, [64 * 4 + 10], H=2, dk=128, dv=128, chunk=64, dtype="bf16")
+    case.g[64:128] *= 6.0
+    check_case(case)
+
+
+def test_split_and_fused_agree_closely(monkeypatch):
+    """The two tensor-core paths run the same arithmetic in the same order:
+    their results agree to a few bf16 ulps of o."""
+    case = wl.make_prefill(307, [640, 333], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    monkeypatch.setenv("KDA_CHUNK_PATH", "fused")
+    o1, h1 = run_fwd(case)
+    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
+    o2, h2 = run_fwd(case)
+    torch.cuda.synchronize()
+    assert rel_err(o2, o1.double().cpu().numpy()) <= 1e-2
+    assert rel_err(h2, h1.double().cpu().numpy()) <= 1e-5
