@@ -8,8 +8,9 @@
 //                       W = T diag(b) (K * Gam); it writes the chain's operands
 //                       for that chunk to the workspace as one blob laid out
 //                       exactly as the chain kernel's shared memory wants it.
-//   chunk_chain_kernel  one CTA per (sequence, head), chunks in order: bulk
-//                       copies of each chunk's blob (double-buffered) and V,
+//   chunk_chain_kernel  two CTAs per (sequence, head) -- one per half of the
+//                       value columns -- chunks in order: bulk copies of each
+//                       chunk's blob and that half of V,
 //                       then Ut = Tb V, X = [W ; Q*Gam] S, U = Ut - W S,
 //                       O = X + [. ; P] U and S <- Gam_last S + K~^T U, with
 //                       S carried in fp32 in tensor memory.
@@ -463,26 +464,30 @@ __global__ void __launch_bounds__(NT, 1)
 }  // namespace intra
 
 // ===================================================================== chain
+// One CTA per (sequence, head, half of the value columns): the two halves of a
+// state evolve independently (the transition acts on the key side only), so a
+// chain runs on two SMs with N = 64 products, and two such CTAs fit on one SM.
 namespace chain {
-constexpr uint32_t OFF_WQ = 0;         // [W | Q*Gam] blob part
-constexpr uint32_t OFF_RAP0 = 32768;   // K E^-1, two buffers
-constexpr uint32_t OFF_RAP1 = 49152;
-constexpr uint32_t OFF_PM0 = 65536;    // P rows 64-127, two buffers; the operand starts
-constexpr uint32_t OFF_PM1 = 73728;    //   8 KB earlier (rows 0-63: whatever is there)
-constexpr uint32_t OFF_TB = 81920;     // Tb rows 0-63; its rows 64-127 are the V tile
-constexpr uint32_t OFF_V = 90112;      // V (TMA)
-constexpr uint32_t OFF_SB = 106496;    // S bf16 [dk][dv]
-constexpr uint32_t OFF_UB = 139264;    // U bf16 [token][dv]
-constexpr uint32_t OFF_SC0 = 155648;   // exp(G_last), row scale: two buffers of 1 KB
-constexpr uint32_t OFF_SC1 = 156672;
-constexpr uint32_t OFF_BAR = 157696;
+constexpr int NTC = 256;         // threads (8 warps: 4 lane quarters x 2 column pieces)
+constexpr int DVS = 64;          // value columns per CTA
+constexpr uint32_t OFF_WQ = 0;         // [W | Q*Gam] (blob part)
+constexpr uint32_t OFF_RAP = 32768;    // K E^-1
+constexpr uint32_t OFF_PM = 49152;     // P rows 64-127; operand starts 8 KB earlier (RAP tail)
+constexpr uint32_t OFF_TB = 57344;     // Tb rows 0-63; its rows 64-127 are the V tile
+constexpr uint32_t OFF_V = 65536;      // V [64 tokens][64 columns of this half] (TMA)
+constexpr uint32_t OFF_SB = 73728;     // S bf16 [dk][64], MN-major
+constexpr uint32_t OFF_UB = 90112;     // U bf16 [token][64], MN-major
+constexpr uint32_t OFF_SC0 = 98304;    // exp(G_last), row scale: two buffers of 1 KB
+constexpr uint32_t OFF_SC1 = 99328;
+constexpr uint32_t OFF_BAR = 100352;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_V == OFF_TB + 8192, "Tb garbage rows");
-constexpr uint32_t TM_W = 0;     // (K E^-1)^T U
-constexpr uint32_t TM_UT = 128;  // Ut
-constexpr uint32_t TM_X = 256;   // [W;QGam] S, then O
-constexpr uint32_t TM_S = 384;   // fp32 state
-constexpr uint32_t TX_BYTES = 32768 + 16384 + 8192 + 8192 + 16384 + 1024;
+static_assert(OFF_PM == OFF_RAP + 16384, "P garbage rows");
+constexpr uint32_t TM_W = 0;     // (K E^-1)^T U   [128 x 64]
+constexpr uint32_t TM_UT = 64;   // Ut
+constexpr uint32_t TM_X = 128;   // [W;QGam] S, then O
+constexpr uint32_t TM_S = 192;   // fp32 state [128 x 64]
+constexpr uint32_t TX_BYTES = 1024 + 8192 + 8192 + 32768 + 16384 + 8192;
 
 struct Params {
     const float* h0;
@@ -497,7 +502,7 @@ struct Params {
     float* hN;
 };
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTC, 2)
     chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
     if (status_bad(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
@@ -508,10 +513,11 @@ __global__ void __launch_bounds__(NT, 1)
     uint64_t* bar_mma = bar_ld + 1;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int quarter = warp & 3, cq = warp >> 2;
+    const int quarter = warp & 3, cq = warp >> 2;  // rows 32 quarter + lane, columns 32 cq ..
     const int trow = 32 * quarter + (tid & 31);
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
-    const int seq = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int chain_id = blockIdx.x >> 1, half = blockIdx.x & 1, j0 = DVS * half;
+    const int seq = chain_id / p.H, h = chain_id % p.H;
     const int t_begin = p.cu ? p.cu[seq] : seq * p.T;
     const int t_end = p.cu ? p.cu[seq + 1] : (seq + 1) * p.T;
     const int cbase = p.chunk_start[seq];
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(NT, 1)
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(s_tmem, 512);
+        tmem_alloc(s_tmem, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -536,41 +542,35 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0 && t_begin < t_end) {
         const uint8_t* b0 = blob(0);
         mbar_arrive_expect_tx(bar_ld, TX_BYTES);
-        bulk_g2s(sm + OFF_RAP0, b0 + BL_RAP, 16384, bar_ld);
-        bulk_g2s(sm + OFF_PM0, b0 + BL_PM, 8192, bar_ld);
         bulk_g2s(sm + OFF_SC0, b0 + BL_SC, 1024, bar_ld);
         bulk_g2s(sm + OFF_TB, b0 + BL_TB, 8192, bar_ld);
+        tma_load_3d(sm + OFF_V, &tmv, bar_ld, j0, h, t_begin);
         bulk_g2s(sm + OFF_WQ, b0 + BL_WQ, 32768, bar_ld);
-        tma_load_3d(sm + OFF_V, &tmv, bar_ld, 0, h, t_begin);
-        tma_load_3d(sm + OFF_V + 8192, &tmv, bar_ld, 64, h, t_begin);
+        bulk_g2s(sm + OFF_RAP, b0 + BL_RAP, 16384, bar_ld);
+        bulk_g2s(sm + OFF_PM, b0 + BL_PM, 8192, bar_ld);
     }
-
-    // ---- initial state: fp32 into TMEM (row c = lane c), bf16 copy into Sb
+    // ---- initial state (this half): fp32 into TMEM (row c = lane), bf16 into Sb
     {
         const int c = trow;
-        const float* src = p.h0 ? p.h0 + (((size_t)seq * p.H + h) * D + c) * D : nullptr;
-        {
-            const int piece = cq;
-            uint32_t r[32];
-            float x[32];
+        const float* src =
+            p.h0 ? p.h0 + (((size_t)seq * p.H + h) * D + c) * D + j0 + cq * 32 : nullptr;
+        uint32_t r[32];
+        float x[32];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                float4 v = src ? *reinterpret_cast<const float4*>(src + piece * 32 + i)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
-            }
+        for (int i = 0; i < 32; i += 4) {
+            float4 v = src ? *reinterpret_cast<const float4*>(src + i)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+        }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
-            tmem_st32(tbase + tlane + TM_S + piece * 32, r);
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
+        tmem_st32(tbase + tlane + TM_S + cq * 32, r);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                float y[8];
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float y[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = x[q4 * 8 + i];
-                const int col = piece * 32 + q4 * 8;
-                *reinterpret_cast<uint4*>(sm + OFF_SB + (col >> 6) * 16384 +
-                                          sw128_off(c, (col & 63) >> 3)) = pack8(y);
-            }
+            for (int i = 0; i < 8; ++i) y[i] = x[q4 * 8 + i];
+            *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_off(c, cq * 4 + q4)) = pack8(y);
         }
         tmem_wait_st();
     }
@@ -584,24 +584,19 @@ __global__ void __launch_bounds__(NT, 1)
         const int L = min(C, t_end - t0);
         const int tn = t0 + C;
         const bool has_next = tn < t_end;
-        const uint32_t pm_op = ((n & 1) ? OFF_PM1 : OFF_PM0) - 8192;
-        const uint32_t rap_op = (n & 1) ? OFF_RAP1 : OFF_RAP0;
         const float* ssc = reinterpret_cast<const float*>(sm + ((n & 1) ? OFF_SC1 : OFF_SC0));
         bool ok = mbar_wait(bar_ld, n & 1, kWaitNs);
         if (__syncthreads_or(!ok)) {
             failed = true;
             break;
         }
-        if (has_next && tid == 0) {  // double-buffered parts of the next chunk
-            const uint8_t* bn = blob(n + 1);
+        if (has_next && tid == 0) {
             mbar_arrive_expect_tx(bar_ld, TX_BYTES);
-            bulk_g2s(sm + ((n & 1) ? OFF_RAP0 : OFF_RAP1), bn + BL_RAP, 16384, bar_ld);
-            bulk_g2s(sm + ((n & 1) ? OFF_PM0 : OFF_PM1), bn + BL_PM, 8192, bar_ld);
-            bulk_g2s(sm + ((n & 1) ? OFF_SC0 : OFF_SC1), bn + BL_SC, 1024, bar_ld);
+            bulk_g2s(sm + ((n & 1) ? OFF_SC0 : OFF_SC1), blob(n + 1) + BL_SC, 1024, bar_ld);
         }
-        // -------------------------------------------------- Ut = Tb V  (N=128)
+        // ---------------------------------------------------- Ut = Tb V  (N=64)
         if (tid == 0) {
-            constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
+            constexpr uint32_t id = idesc_bf16_f32(128, DVS, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tbase + TM_UT, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
@@ -617,12 +612,11 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_after();
         if (has_next && tid == 0) {  // V and Tb regions are free
             bulk_g2s(sm + OFF_TB, blob(n + 1) + BL_TB, 8192, bar_ld);
-            tma_load_3d(sm + OFF_V, &tmv, bar_ld, 0, h, tn);
-            tma_load_3d(sm + OFF_V + 8192, &tmv, bar_ld, 64, h, tn);
+            tma_load_3d(sm + OFF_V, &tmv, bar_ld, j0, h, tn);
         }
-        // ------------------------------- X = [W ; Q*Gam] S   (M=128, N=128)
+        // ------------------------------------- X = [W ; Q*Gam] S   (N=64)
         if (tid == 0) {
-            constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
+            constexpr uint32_t id = idesc_bf16_f32(128, DVS, false, true);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int kb = ks >> 2, kk = ks & 3;
@@ -649,30 +643,28 @@ __global__ void __launch_bounds__(NT, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                const int col = cq * 32 + q4 * 8;
                 float y[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     y[i] = __uint_as_float(a[q4 * 8 + i]) - __uint_as_float(b[q4 * 8 + i]);
-                *reinterpret_cast<uint4*>(sm + OFF_UB + (col >> 6) * 8192 +
-                                          sw128_off(r, (col & 63) >> 3)) = pack8(y);
+                *reinterpret_cast<uint4*>(sm + OFF_UB + sw128_off(r, cq * 4 + q4)) = pack8(y);
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ---- O = X[64:] + [. ; P] U  (accumulate);  (K E^-1)^T U -> TM_W
+        // ---- O = X[64:] + [. ; P] U  (accumulate);  (K E^-1)^T U -> TM_W   (N=64)
         if (tid == 0) {
-            constexpr uint32_t idP = idesc_bf16_f32(128, 128, false, true);
-            constexpr uint32_t idK = idesc_bf16_f32(128, 128, true, true);
+            constexpr uint32_t idP = idesc_bf16_f32(128, DVS, false, true);
+            constexpr uint32_t idK = idesc_bf16_f32(128, DVS, true, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + pm_op + ks * 32, 16, 1024),
+                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_PM - 8192 + ks * 32, 16, 1024),
                          sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idP, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tbase + TM_W, sdesc_sw128(sbase + rap_op + ks * 2048, 8192, 1024),
+                mma_bf16(tbase + TM_W, sdesc_sw128(sbase + OFF_RAP + ks * 2048, 8192, 1024),
                          sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idK, ks > 0);
             mma_commit(bar_mma);
         }
@@ -683,6 +675,10 @@ __global__ void __launch_bounds__(NT, 1)
             break;
         }
         tc_fence_after();
+        if (has_next && tid == 0) {  // K E^-1 and P regions are free
+            bulk_g2s(sm + OFF_RAP, blob(n + 1) + BL_RAP, 16384, bar_ld);
+            bulk_g2s(sm + OFF_PM, blob(n + 1) + BL_PM, 8192, bar_ld);
+        }
         // S <- Gam_last * S + ksc * (K E^-1)^T U   (lane = state row c); O rows out
         {
             const int c = trow;
@@ -697,12 +693,10 @@ __global__ void __launch_bounds__(NT, 1)
             tmem_st32(tbase + tlane + TM_S + cq * 32, sv);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                const int col = cq * 32 + q4 * 8;
                 float y[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(sv[q4 * 8 + i]);
-                *reinterpret_cast<uint4*>(sm + OFF_SB + (col >> 6) * 16384 +
-                                          sw128_off(c, (col & 63) >> 3)) = pack8(y);
+                *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_off(c, cq * 4 + q4)) = pack8(y);
             }
             if (quarter >= 2) {
                 const int r = trow - C;
@@ -710,7 +704,8 @@ __global__ void __launch_bounds__(NT, 1)
                 tmem_ld32(tbase + tlane + TM_X + cq * 32, v);
                 tmem_wait_ld();
                 if (r < L) {
-                    __nv_bfloat16* dst = p.o + ((size_t)(t0 + r) * p.H + h) * D + cq * 32;
+                    __nv_bfloat16* dst =
+                        p.o + ((size_t)(t0 + r) * p.H + h) * D + j0 + cq * 32;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         float y[8];
@@ -730,18 +725,15 @@ __global__ void __launch_bounds__(NT, 1)
 
     if (!failed && p.hN) {
         const int c = trow;
-        float* dst = p.hN + (((size_t)seq * p.H + h) * D + c) * D;
-        {
-            const int piece = cq;
-            uint32_t s[32];
-            tmem_ld32(tbase + tlane + TM_S + piece * 32, s);
-            tmem_wait_ld();
+        float* dst = p.hN + (((size_t)seq * p.H + h) * D + c) * D + j0 + cq * 32;
+        uint32_t s[32];
+        tmem_ld32(tbase + tlane + TM_S + cq * 32, s);
+        tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(dst + piece * 32 + i) =
-                    make_float4(__uint_as_float(s[i]), __uint_as_float(s[i + 1]),
-                                __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
-        }
+        for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(__uint_as_float(s[i]), __uint_as_float(s[i + 1]),
+                            __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
     }
     if (failed && tid == 0) {
         if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
@@ -750,7 +742,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 512);
+    if (warp == 0) tmem_dealloc(tbase, 256);
 }
 }  // namespace chain
 
@@ -824,7 +816,7 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
     }
     chain::Params pb{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
                      (__nv_bfloat16*)o, hN};
-    chain::chunk_chain_kernel<<<N * H, NT, chain::SMEM_BYTES, st>>>(mv, pb);
+    chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
     return cudaGetLastError();
 }
 
