@@ -58,16 +58,20 @@ size_t split_blob_bytes() { return BLOB; }
 namespace {
 
 // ===================================================================== intra
+// Persistent: one CTA per SM walks the (chunk slot, head) items with a stride
+// of the grid, fetching the next item's inputs while the current one is
+// computed and writing each item's blob while the next one starts.
 namespace intra {
 constexpr uint32_t OFF_K = 0;          // K (TMA); exact path: K * Gam in place
-constexpr uint32_t OFF_RAP = 16384;    // K * E^-1
-constexpr uint32_t OFF_WQ = 32768;     // [W kb0 | Q kb0 | W kb1 | Q kb1]
-constexpr uint32_t OFF_G = 65536;      // g (TMA) -> G -> A fp32 | T fp32
-constexpr uint32_t OFF_LAP = 98304;    // [K * E ; Q * E]; exact path: A | P fp32
-constexpr uint32_t OFF_TB = 131072;    // T diag(b) rows 0-63
-constexpr uint32_t OFF_MID = 139264;   // scratch; garbage rows of the Tb and P operands
-constexpr uint32_t OFF_PM = 147456;    // P rows 64-127
-constexpr uint32_t OFF_BETA = 155648;
+constexpr uint32_t OFF_Q = 16384;      // Q (TMA)
+constexpr uint32_t OFF_RAP = 32768;    // K * E^-1
+constexpr uint32_t OFF_WQ = 49152;     // [W kb0 | Q*Gam kb0 | W kb1 | Q*Gam kb1]
+constexpr uint32_t OFF_G = 81920;      // g (TMA) -> G -> A fp32 | T fp32
+constexpr uint32_t OFF_LAP = 114688;   // [K * E ; Q * E]; exact path: A | P fp32
+constexpr uint32_t OFF_TB = 147456;    // T diag(b) rows 0-63
+constexpr uint32_t OFF_MID = 155648;   // scratch; garbage rows of the Tb and P operands
+constexpr uint32_t OFF_PM = 163840;    // P rows 64-127
+constexpr uint32_t OFF_BETA = 172032;
 constexpr uint32_t OFF_GM = OFF_BETA + 256;
 constexpr uint32_t OFF_EGM = OFF_GM + 512;
 constexpr uint32_t OFF_GC = OFF_EGM + 512;
@@ -77,6 +81,7 @@ constexpr uint32_t OFF_KSC = OFF_WSC + 512;
 constexpr uint32_t OFF_BAR = OFF_KSC + 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_PM == OFF_MID + 8192, "P rows follow the garbage rows");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 constexpr uint32_t TM_X = 0;     // A|P
 constexpr uint32_t TM_W = 128;   // W
 constexpr uint32_t TX_BYTES = 2 * 16384 + 32768;
@@ -84,6 +89,7 @@ constexpr uint32_t TX_BYTES = 2 * 16384 + 32768;
 struct Params {
     const float* beta;
     const int4* info;
+    int maxc;
     int H;
     const uint32_t* status;
     uint32_t* status_out;
@@ -95,10 +101,7 @@ __global__ void __launch_bounds__(NT, 1)
                        const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmg, const Params p) {
     if (status_bad(p.status)) return;
-    const int4 ci = p.info[blockIdx.x];
-    const int L = ci.z;
-    if (L <= 0) return;
-    const int h = blockIdx.y, t0 = ci.y;
+    const int maxc = p.maxc, nitems = maxc * p.H;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -117,7 +120,11 @@ __global__ void __launch_bounds__(NT, 1)
     const int quarter = warp & 3, cq = warp >> 2, lane = tid & 31;
     const int trow = 32 * quarter + (tid & 31);
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
-    uint8_t* blob = p.blobs + ((size_t)blockIdx.x * p.H + h) * BLOB;
+    // items whose chunk slot is empty (varlen upper bound) are skipped
+    auto advance = [&](int it) {
+        while (it < nitems && p.info[it % maxc].z <= 0) it += gridDim.x;
+        return it;
+    };
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
@@ -134,17 +141,30 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t tbase = *s_tmem;
     bool failed = false;
     uint32_t mma_phase = 0;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_tma, TX_BYTES);
-        tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, h, t0);
-        tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, h, t0);
-        tma_load_3d(sm + OFF_WQ + 8192, &tmq, bar_tma, 0, h, t0);
-        tma_load_3d(sm + OFF_WQ + 16384 + 8192, &tmq, bar_tma, 64, h, t0);
-        tma_load_3d(sm + OFF_G, &tmg, bar_tma, 0, h, t0);
+    int item = advance(blockIdx.x);
+    float beta_next = 0.f;
+    if (item < nitems) {
+        const int4 c0i = p.info[item % maxc];
+        const int h0i = item / maxc;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_tma, TX_BYTES);
+            tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, h0i, c0i.y);
+            tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, h0i, c0i.y);
+            tma_load_3d(sm + OFF_Q, &tmq, bar_tma, 0, h0i, c0i.y);
+            tma_load_3d(sm + OFF_Q + 8192, &tmq, bar_tma, 64, h0i, c0i.y);
+            tma_load_3d(sm + OFF_G, &tmg, bar_tma, 0, h0i, c0i.y);
+        }
+        if (tid < C) beta_next = tid < c0i.z ? p.beta[(size_t)(c0i.y + tid) * p.H + h0i] : 0.f;
     }
-    if (tid < C) sbeta[tid] = tid < L ? p.beta[(size_t)(t0 + tid) * p.H + h] : 0.f;
-    do {
-        bool ok = mbar_wait(bar_tma, 0, kWaitNs);
+    int n = 0;
+    for (; item < nitems && !failed; ++n) {
+        const int4 ci = p.info[item % maxc];
+        const int L = ci.z, h = item / maxc;
+        const int nxt = advance(item + gridDim.x);
+        uint8_t* blob = p.blobs + ((size_t)(item % maxc) * p.H + h) * BLOB;
+        bool armed = false;  // (thread 0) next item's transaction count registered
+        if (tid < C) sbeta[tid] = beta_next;
+        bool ok = mbar_wait(bar_tma, n & 1, kWaitNs);
         if (__syncthreads_or(!ok)) {
             failed = true;
             break;
@@ -176,6 +196,7 @@ __global__ void __launch_bounds__(NT, 1)
             sGL[c] = G;
             slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
         }
+        if (tid == 0) bulk_wait_read();  // previous item's write-out has read its tiles
         const bool slow = __syncthreads_or(slow_local);
         if (tid < D) {
             sWsc[tid] = slow ? 1.f : seGm[tid];
@@ -194,7 +215,7 @@ __global__ void __launch_bounds__(NT, 1)
                         const float e = expf(G[r * D + c] - G[i * D + c]);
                         const float ki = tile_elem(sm + OFF_K, 8192, i, c);
                         a += tile_elem(sm + OFF_K, 8192, r, c) * ki * e;
-                        pp += tile_elem(sm + OFF_WQ + 8192, 16384, r, c) * ki * e;
+                        pp += tile_elem(sm + OFF_Q, 8192, r, c) * ki * e;
                     }
                 }
                 Af[a_idx(r, i)] = (i < r) ? sbeta[r] * a : 0.f;
@@ -211,7 +232,8 @@ __global__ void __launch_bounds__(NT, 1)
                 const int r = it >> 4, j = it & 15, kb = j >> 3, ch = j & 7, c0 = 8 * j;
                 const uint32_t o64 = sw128_off(r, ch);
                 uint8_t* pk = sm + OFF_K + kb * 8192 + o64;
-                uint8_t* pq = sm + OFF_WQ + kb * 16384 + 8192 + o64;
+                const uint8_t* pq = sm + OFF_Q + kb * 8192 + o64;
+                uint8_t* pqg = sm + OFF_WQ + kb * 16384 + 8192 + o64;
                 uint8_t* pr = sm + OFF_RAP + kb * 8192 + o64;
                 float lk[8], lq[8], rk[8], qg[8];
                 if (r < L) {
@@ -257,13 +279,27 @@ __global__ void __launch_bounds__(NT, 1)
                     *reinterpret_cast<uint4*>(pk) = pack8(lk);
                 }
                 *reinterpret_cast<uint4*>(pr) = pack8(rk);
-                *reinterpret_cast<uint4*>(pq) = pack8(qg);
+                *reinterpret_cast<uint4*>(pqg) = pack8(qg);
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid < C && nxt < nitems) {
+            const int4 cn = p.info[nxt % maxc];
+            beta_next = tid < cn.z ? p.beta[(size_t)(cn.y + tid) * p.H + nxt / maxc] : 0.f;
+        }
+        if (!slow && nxt < nitems && tid == 0) {  // K and Q are consumed: prefetch
+            const int4 cn = p.info[nxt % maxc];
+            const int hn = nxt / maxc;
+            mbar_arrive_expect_tx(bar_tma, TX_BYTES);
+            armed = true;
+            tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, hn, cn.y);
+            tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, hn, cn.y);
+            tma_load_3d(sm + OFF_Q, &tmq, bar_tma, 0, hn, cn.y);
+            tma_load_3d(sm + OFF_Q + 8192, &tmq, bar_tma, 64, hn, cn.y);
+        }
         // ------------------------------------------------ A, P (M=128, N=64)
         if (!slow) {
             if (tid == 0) {
@@ -394,6 +430,15 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (nxt < nitems && tid == 0) {  // G region is free: prefetch g (and K, Q)
+            const int4 cn = p.info[nxt % maxc];
+            const int hn = nxt / maxc;
+            if (!armed) {
+                mbar_arrive_expect_tx(bar_tma, TX_BYTES);
+                armed = true;
+            }
+            tma_load_3d(sm + OFF_G, &tmg, bar_tma, 0, hn, cn.y);
+        }
         // ---------------------------------- W = Tb (K*E) [*exp(Gm)]  (N=128)
         if (tid == 0) {
             constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
@@ -412,6 +457,14 @@ __global__ void __launch_bounds__(NT, 1)
             break;
         }
         tc_fence_after();
+        if (slow && nxt < nitems && tid == 0) {  // exact path: K region free only now
+            const int4 cn = p.info[nxt % maxc];
+            const int hn = nxt / maxc;
+            tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, hn, cn.y);
+            tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, hn, cn.y);
+            tma_load_3d(sm + OFF_Q, &tmq, bar_tma, 0, hn, cn.y);
+            tma_load_3d(sm + OFF_Q + 8192, &tmq, bar_tma, 64, hn, cn.y);
+        }
         // W (rows 0-63), column-scaled -> bf16 into the W rows of [W ; Q*Gam]
         if (quarter < 2) {
             const int r = trow;
@@ -437,7 +490,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ---- hand the chain's operands to the workspace
+        // ---- hand the chain's operands to the workspace (asynchronously)
         if (tid == 0) {
             bulk_s2g(blob + BL_WQ, sm + OFF_WQ, 32768);
             bulk_s2g(blob + BL_RAP, sm + OFF_RAP, 16384);
@@ -450,11 +503,12 @@ __global__ void __launch_bounds__(NT, 1)
             sc[tid] = sGC[tid];
             sc[D + tid] = sKsc[tid];
         }
-        if (tid == 0) bulk_wait_all();
-    } while (false);
+        item = nxt;
+    }
+    if (tid == 0) bulk_wait_all();
     if (failed && tid == 0) {
         if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
-        mbar_wait(bar_tma, 0, kWaitNs);
+        mbar_wait(bar_tma, n & 1, kWaitNs);
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
@@ -809,8 +863,13 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
     if (e != cudaSuccess) return e;
     uint8_t* bl = static_cast<uint8_t*>(blobs);
     if (maxc > 0) {
-        intra::Params pa{beta, chunk_info, H, status, status, bl};
-        intra::chunk_intra_kernel<<<dim3(maxc, H), NT, intra::SMEM_BYTES, st>>>(mq, mk, mg, pa);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long items = (long long)maxc * H;
+        const int grid = (int)(items < sms ? items : sms);
+        intra::Params pa{beta, chunk_info, maxc, H, status, status, bl};
+        intra::chunk_intra_kernel<<<grid, NT, intra::SMEM_BYTES, st>>>(mq, mk, mg, pa);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
