@@ -44,7 +44,7 @@ constexpr float kRef = 80.f;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // ---- per (chunk, head) blob in the workspace (each part 1024-byte aligned)
-constexpr uint32_t BL_WQ = 0;        // [W kb0 | Q*Gam kb0 | W kb1 | Q*Gam kb1]   32 KB
+constexpr uint32_t BL_WQ = 0;        // [-W kb0 | Q*Gam kb0 | -W kb1 | Q*Gam kb1] 32 KB
 constexpr uint32_t BL_RAP = 32768;   // K * E^-1 (or K * exp(G_last - G))         16 KB
 constexpr uint32_t BL_PM = 49152;    // P (masked), rows 64-127 of its operand      8 KB
 constexpr uint32_t BL_TB = 57344;    // T diag(b), rows 0-63 of its operand         8 KB
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (tid == 0) bulk_wait_read();  // previous item's write-out has read its tiles
         const bool slow = __syncthreads_or(slow_local);
         if (tid < D) {
-            sWsc[tid] = slow ? 1.f : seGm[tid];
+            sWsc[tid] = slow ? -1.f : -seGm[tid];  // the blob holds -W
             sKsc[tid] = slow ? 1.f : expf(sGL[tid] - sGm[tid]);
         }
         // ---------------- exact A and P on CUDA cores (rare: extreme decay)
@@ -486,10 +486,6 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
         // ---- hand the chain's operands to the workspace (asynchronously)
         if (tid == 0) {
             bulk_s2g(blob + BL_WQ, sm + OFF_WQ, 32768);
@@ -527,20 +523,21 @@ constexpr int DVS = 64;          // value columns per CTA
 constexpr uint32_t OFF_WQ = 0;         // [W | Q*Gam] (blob part)
 constexpr uint32_t OFF_RAP = 32768;    // K E^-1
 constexpr uint32_t OFF_PM = 49152;     // P rows 64-127; operand starts 8 KB earlier (RAP tail)
-constexpr uint32_t OFF_TB = 57344;     // Tb rows 0-63; its rows 64-127 are the V tile
-constexpr uint32_t OFF_V = 65536;      // V [64 tokens][64 columns of this half] (TMA)
-constexpr uint32_t OFF_SB = 73728;     // S bf16 [dk][64], MN-major
-constexpr uint32_t OFF_UB = 90112;     // U bf16 [token][64], MN-major
-constexpr uint32_t OFF_SC0 = 98304;    // exp(G_last), row scale: two buffers of 1 KB
-constexpr uint32_t OFF_SC1 = 99328;
-constexpr uint32_t OFF_BAR = 100352;
+constexpr uint32_t OFF_TB = 57344;     // Tb rows 0-63 of a 128-row operand ...
+constexpr uint32_t OFF_ZERO = 65536;   // ... whose rows 64-127 are zeros (set once)
+constexpr uint32_t OFF_V = 73728;      // V [64 tokens][64 columns of this half] (TMA)
+constexpr uint32_t OFF_SB = 81920;     // S bf16 [dk][64], MN-major
+constexpr uint32_t OFF_UB = 98304;     // U bf16 [token][64], MN-major
+constexpr uint32_t OFF_SC0 = 106496;   // exp(G_last), row scale: two buffers of 1 KB
+constexpr uint32_t OFF_SC1 = 107520;
+constexpr uint32_t OFF_BAR = 108544;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
-static_assert(OFF_V == OFF_TB + 8192, "Tb garbage rows");
+static_assert(OFF_ZERO == OFF_TB + 8192, "Tb zero rows");
 static_assert(OFF_PM == OFF_RAP + 16384, "P garbage rows");
+static_assert(2 * SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
 constexpr uint32_t TM_W = 0;     // (K E^-1)^T U   [128 x 64]
-constexpr uint32_t TM_UT = 64;   // Ut
-constexpr uint32_t TM_X = 128;   // [W;QGam] S, then O
-constexpr uint32_t TM_S = 192;   // fp32 state [128 x 64]
+constexpr uint32_t TM_X = 64;    // [Ut ; 0] + [-W ; Q*Gam] S = [U ; Q*Gam S], then O
+constexpr uint32_t TM_S = 128;   // fp32 state [128 x 64]
 constexpr uint32_t TX_BYTES = 1024 + 8192 + 8192 + 32768 + 16384 + 8192;
 
 struct Params {
@@ -628,6 +625,8 @@ __global__ void __launch_bounds__(NTC, 2)
         }
         tmem_wait_st();
     }
+    for (int i = tid; i < 8192 / 16; i += NTC)
+        reinterpret_cast<uint4*>(sm + OFF_ZERO)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -648,34 +647,18 @@ __global__ void __launch_bounds__(NTC, 2)
             mbar_arrive_expect_tx(bar_ld, TX_BYTES);
             bulk_g2s(sm + ((n & 1) ? OFF_SC0 : OFF_SC1), blob(n + 1) + BL_SC, 1024, bar_ld);
         }
-        // ---------------------------------------------------- Ut = Tb V  (N=64)
+        // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
         if (tid == 0) {
             constexpr uint32_t id = idesc_bf16_f32(128, DVS, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tbase + TM_UT, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
+                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
                          sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id, ks > 0);
-            mma_commit(bar_mma);
-        }
-        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
-        ++mma_phase;
-        if (__syncthreads_or(!ok)) {
-            failed = true;
-            break;
-        }
-        tc_fence_after();
-        if (has_next && tid == 0) {  // V and Tb regions are free
-            bulk_g2s(sm + OFF_TB, blob(n + 1) + BL_TB, 8192, bar_ld);
-            tma_load_3d(sm + OFF_V, &tmv, bar_ld, j0, h, tn);
-        }
-        // ------------------------------------- X = [W ; Q*Gam] S   (N=64)
-        if (tid == 0) {
-            constexpr uint32_t id = idesc_bf16_f32(128, DVS, false, true);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int kb = ks >> 2, kk = ks & 3;
                 mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
-                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id, ks > 0);
+                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id, 1);
             }
             mma_commit(bar_mma);
         }
@@ -686,21 +669,22 @@ __global__ void __launch_bounds__(NTC, 2)
             break;
         }
         tc_fence_after();
-        if (has_next && tid == 0)  // the [W ; Q*Gam] region is free
+        if (has_next && tid == 0) {  // V, Tb and [-W ; Q*Gam] regions are free
+            bulk_g2s(sm + OFF_TB, blob(n + 1) + BL_TB, 8192, bar_ld);
+            tma_load_3d(sm + OFF_V, &tmv, bar_ld, j0, h, tn);
             bulk_g2s(sm + OFF_WQ, blob(n + 1) + BL_WQ, 32768, bar_ld);
-        // U = Ut - W S  (rows 0-63) -> bf16 Ub
+        }
+        // U (rows 0-63 of the accumulator) -> bf16 Ub
         if (quarter < 2) {
             const int r = trow;
-            uint32_t a[32], b[32];
-            tmem_ld32(tbase + tlane + TM_UT + cq * 32, a);
-            tmem_ld32(tbase + tlane + TM_X + cq * 32, b);
+            uint32_t a[32];
+            tmem_ld32(tbase + tlane + TM_X + cq * 32, a);
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 float y[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    y[i] = __uint_as_float(a[q4 * 8 + i]) - __uint_as_float(b[q4 * 8 + i]);
+                for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(a[q4 * 8 + i]);
                 *reinterpret_cast<uint4*>(sm + OFF_UB + sw128_off(r, cq * 4 + q4)) = pack8(y);
             }
         }
