@@ -312,33 +312,65 @@ def prefill_path(Np, H, dk, dv, C, dtype="bf16"):
 
 
 def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
-    """Times of the prefill kernels.  For the CUDA-core path: each step call
-    (a1..a4) on its own; for the tensor-core paths: the whole call (one fused
-    kernel, or the intra + chain pair of the split path)."""
+    """Device times of the prefill kernels, each from CUDA events around its own
+    call on the launching stream, L2 flushed before each.  CUDA-core path: the
+    four step calls (a1..a4); split plan: kda_chunk_split_intra and
+    kda_chunk_split_chain; fused plan: the one kernel (the whole call).  Each
+    call's time includes the chunk-table kernel that starts it, where it has
+    one.  Algorithmic bytes are the pages' inputs and outputs that each kernel
+    must move; the split plan's hand-over through the workspace is overhead."""
     import torch
     Np, H, dk, dv, C, total = P.N, P.H, P.dk, P.dv, P.chunk, P.total
     path = prefill_path(Np, H, dk, dv, C)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     in_b = 2
+    tx = total * H
     Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
+
+    def timed(calls):
+        times = {}
+        for name in calls:
+            ts = []
+            for _ in range(reps):
+                for n2, f in calls.items():  # the whole sequence, so inputs are valid
+                    if n2 == name:
+                        flush.zero_()
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record(stream)
+                        f()
+                        e1.record(stream)
+                        ts.append((e0, e1))
+                    else:
+                        f()
+            torch.cuda.synchronize()
+            times[name] = statistics.median(x.elapsed_time(y) for x, y in ts) / 1e3
+        return times
+
     if path != "simt":
-        name = "chunk_fwd_tc" if path == "fused" else "chunk_fwd_split(intra+chain)"
         o = torch.empty_like(P.v)
         hN = torch.empty(Np, H, dk, dv, device=dev)
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc,
-                              Tc, Np, H, dk, dv, C, "bf16", o, hN, ws)
-            b.record(stream)
-            ts.append((a, b))
-        torch.cuda.synchronize()
-        t = statistics.median(a.elapsed_time(b) for a, b in ts) / 1e3
-        nb = prefill_bytes(total * H, Np * H)
-        return {"times": {name: t}, "bytes": {name: nb}, "dominant": (name, t),
-                "launches_per_call": 2 if path == "fused" else 3, "path": path}
+        if path == "fused":
+            name = "chunk_fwd_tc"
+            calls = {name: lambda: kda.kda_chunk_fwd(
+                P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc, Tc, Np, H, dk,
+                dv, C, "bf16", o, hN, ws)}
+            nbytes = {name: prefill_bytes(tx, Np * H)}
+            launches = 2
+        else:
+            a = (P.cu_seqlens, Bc, Tc, Np, H)
+            calls = {
+                "split_intra": lambda: kda.kda_chunk_split_intra(P.q, P.k, P.g, P.beta, *a, ws),
+                "split_chain": lambda: kda.kda_chunk_split_chain(P.v, P.initial_state, *a, o,
+                                                                 hN, ws),
+            }
+            nbytes = {"split_intra": tx * (in_b * 2 * dk + 4 * dk + 4),
+                      "split_chain": tx * in_b * 2 * dv + Np * H * 2 * 4 * dk * dv}
+            launches = 3
+        times = timed(calls)
+        dom = max(times, key=times.get)
+        return {"times": times, "bytes": nbytes, "dominant": (dom, times[dom]),
+                "launches_per_call": launches, "path": path}
     G = torch.empty(total, H, dk, device=dev)
     W = torch.empty(total, H, dk, device=dev)
     U = torch.empty(total, H, dv, device=dev)
@@ -363,24 +395,7 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
         "a3_inter": tx * (in_b * dk + 4 * dk + 4 * dk + 8 * dv) + maxc * H * dk * dv * 4,
         "a4_output": tx * (in_b * 2 * dk + 4 * dk + 4 * dv + in_b * dv) + maxc * H * dk * dv * 4,
     }
-    times = {}
-    for name in calls:
-        ts = []
-        for _ in range(reps):
-            for n2, f in calls.items():  # run the whole sequence so inputs are valid
-                if n2 == name:
-                    flush.zero_()
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    f()
-                    e1.record(stream)
-                    ts.append((e0, e1))
-                else:
-                    f()
-        torch.cuda.synchronize()
-        # each step call also launches the chunk-table kernel; it is included
-        times[name] = statistics.median(x.elapsed_time(y) for x, y in ts) / 1e3
+    times = timed(calls)
     dom = max(times, key=times.get)
     return {"times": times, "bytes": nbytes, "dominant": (dom, times[dom]),
             "launches_per_call": 5, "path": path}

@@ -258,6 +258,64 @@ kda_status_t kda_chunk_output(const void* q, const void* k, const float* G, cons
 #undef KDA_PREFILL_PROLOGUE
 #undef KDA_PREFILL_BEGIN
 
+// ------------------------------- tensor-core split path, one kernel per call
+
+namespace {
+constexpr int kTcD = 128, kTcC = 64;
+
+kda_status_t split_prologue(const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                            std::initializer_list<const void*> ptrs, void* workspace,
+                            size_t workspace_bytes, Prefill* p, Workspace* w) {
+    kda_status_t s = check_prefill_shape(cu_seqlens, B, T, num_seqs, H, kTcD, kTcD, kTcC,
+                                         KDA_DTYPE_BF16, p);
+    if (s != KDA_OK) return s;
+    for (const void* ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    if (!kda::tc_path_available()) return KDA_ERR_UNSUPPORTED;
+    return check_ws(workspace, workspace_bytes, *p, H, kTcD, kTcD, kTcC, Path::Split, w);
+}
+}  // namespace
+
+size_t kda_chunk_split_workspace_size(int total_tokens, int num_seqs, int H) {
+    if (total_tokens < 0 || num_seqs < 1 || H < 1) return 0;
+    const Prefill p{total_tokens, num_seqs};
+    return carve_for(nullptr, p, H, kTcD, kTcD, kTcC, Path::Split).total_bytes;
+}
+
+kda_status_t kda_chunk_split_intra(const void* q, const void* k, const float* g,
+                                   const float* beta, const int32_t* cu_seqlens, int B, int T,
+                                   int num_seqs, int H, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+    Prefill p;
+    Workspace w;
+    kda_status_t s = split_prologue(cu_seqlens, B, T, num_seqs, H,
+                                    {q, k, (const void*)g, (const void*)beta}, workspace,
+                                    workspace_bytes, &p, &w);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int maxc = kda::max_chunks(p.total, p.N, kTcC);
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, kTcC, maxc, st);
+    if (s != KDA_OK) return s;
+    return from_cuda(kda::launch_split_intra(q, k, g, beta, p.total, H, w.chunk_info, maxc,
+                                             w.status, w.blobs, st));
+}
+
+kda_status_t kda_chunk_split_chain(const void* v, const float* initial_state,
+                                   const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                                   void* o, float* final_state, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    Prefill p;
+    Workspace w;
+    kda_status_t s = split_prologue(cu_seqlens, B, T, num_seqs, H, {v, (const void*)o},
+                                    workspace, workspace_bytes, &p, &w);
+    if (s != KDA_OK) return s;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_split_chain(v, initial_state, cu_seqlens, T, p.N, H,
+                                             w.chunk_start, w.status, w.blobs, o, final_state,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 // ----------------------------------------------------------------- decode
 
 kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const float* g,

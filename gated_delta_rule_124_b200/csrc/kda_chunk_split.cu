@@ -39,7 +39,6 @@ namespace {
 using namespace sm100;
 using namespace tc;
 
-constexpr int NT = 512;
 constexpr float kRef = 80.f;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -58,33 +57,34 @@ size_t split_blob_bytes() { return BLOB; }
 namespace {
 
 // ===================================================================== intra
-// Persistent: one CTA per SM walks the (chunk slot, head) items with a stride
-// of the grid, fetching the next item's inputs while the current one is
-// computed and writing each item's blob while the next one starts.
+// Persistent, two CTAs of 256 threads per SM (about 100 KB of shared memory
+// each): every CTA walks the (chunk slot, head) items with a stride of the
+// grid.  Operand tiles are built in place over the loaded K and Q; everything
+// that only the chain kernel needs (Q * Gam, P, Tb, -W, the row scales) goes
+// straight from registers to the item's blob in the workspace.  The next
+// item's inputs are fetched as soon as their shared-memory regions are free;
+// the other CTA on the SM covers the wait.
 namespace intra {
-constexpr uint32_t OFF_K = 0;          // K (TMA); exact path: K * Gam in place
-constexpr uint32_t OFF_Q = 16384;      // Q (TMA)
-constexpr uint32_t OFF_RAP = 32768;    // K * E^-1
-constexpr uint32_t OFF_WQ = 49152;     // [W kb0 | Q*Gam kb0 | W kb1 | Q*Gam kb1]
-constexpr uint32_t OFF_G = 81920;      // g (TMA) -> G -> A fp32 | T fp32
-constexpr uint32_t OFF_LAP = 114688;   // [K * E ; Q * E]; exact path: A | P fp32
-constexpr uint32_t OFF_TB = 147456;    // T diag(b) rows 0-63
-constexpr uint32_t OFF_MID = 155648;   // scratch; garbage rows of the Tb and P operands
-constexpr uint32_t OFF_PM = 163840;    // P rows 64-127
-constexpr uint32_t OFF_BETA = 172032;
+constexpr int NTI = 256;
+// [K kb0 | Q kb0 | K kb1 | Q kb1] as loaded; E2 turns it in place into the
+// 128-row operand [K * E ; Q * E] (exact path: K * Gam in the K rows).
+constexpr uint32_t OFF_KQ = 0;
+constexpr uint32_t OFF_G = 32768;      // g (TMA) -> G -> A fp32 | T fp32
+constexpr uint32_t OFF_RAP = 65536;    // K * E^-1 (exact path: K * exp(G_last - G))
+constexpr uint32_t OFF_TB = 81920;     // T diag(b) rows 0-63; exact path: A fp32 (16 KB)
+constexpr uint32_t OFF_MID = 90112;    // garbage rows of the Tb operand; inverse scratch
+constexpr uint32_t OFF_BETA = 98304;
 constexpr uint32_t OFF_GM = OFF_BETA + 256;
 constexpr uint32_t OFF_EGM = OFF_GM + 512;
-constexpr uint32_t OFF_GC = OFF_EGM + 512;
-constexpr uint32_t OFF_GL = OFF_GC + 512;
+constexpr uint32_t OFF_GL = OFF_EGM + 512;
 constexpr uint32_t OFF_WSC = OFF_GL + 512;
-constexpr uint32_t OFF_KSC = OFF_WSC + 512;
-constexpr uint32_t OFF_BAR = OFF_KSC + 512;
+constexpr uint32_t OFF_BAR = OFF_WSC + 512;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
-static_assert(OFF_PM == OFF_MID + 8192, "P rows follow the garbage rows");
-static_assert(SMEM_BYTES <= 232448, "shared memory");
-constexpr uint32_t TM_X = 0;     // A|P
-constexpr uint32_t TM_W = 128;   // W
-constexpr uint32_t TX_BYTES = 2 * 16384 + 32768;
+static_assert(OFF_MID == OFF_TB + 8192, "Tb garbage rows follow Tb");
+static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
+constexpr uint32_t TM_X = 0;     // [A ; P] accumulator, 64 columns
+constexpr uint32_t TM_W = 128;   // W accumulator, 128 columns
+constexpr uint32_t TX_KQ = 32768, TX_G = 32768;
 
 struct Params {
     const float* beta;
@@ -96,7 +96,7 @@ struct Params {
     uint8_t* blobs;
 };
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTI, 2)
     chunk_intra_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmg, const Params p) {
@@ -109,25 +109,39 @@ __global__ void __launch_bounds__(NT, 1)
     float* sbeta = reinterpret_cast<float*>(sm + OFF_BETA);
     float* sGm = reinterpret_cast<float*>(sm + OFF_GM);
     float* seGm = reinterpret_cast<float*>(sm + OFF_EGM);
-    float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
     float* sGL = reinterpret_cast<float*>(sm + OFF_GL);
     float* sWsc = reinterpret_cast<float*>(sm + OFF_WSC);
-    float* sKsc = reinterpret_cast<float*>(sm + OFF_KSC);
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    uint64_t* bar_mma = bar_tma + 1;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int quarter = warp & 3, cq = warp >> 2, lane = tid & 31;
-    const int trow = 32 * quarter + (tid & 31);
+    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_g = bar_kq + 1;
+    uint64_t* bar_mma = bar_kq + 2;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 32);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, cq = warp >> 2;  // TMEM lanes 32 quarter.., columns 32 cq..
+    const int trow = 32 * quarter + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
     // items whose chunk slot is empty (varlen upper bound) are skipped
     auto advance = [&](int it) {
         while (it < nitems && p.info[it % maxc].z <= 0) it += gridDim.x;
         return it;
     };
+    auto load_kq = [&](int it) {  // thread 0
+        const int4 c = p.info[it % maxc];
+        const int hh = it / maxc;
+        mbar_arrive_expect_tx(bar_kq, TX_KQ);
+        tma_load_3d(sm + OFF_KQ, &tmk, bar_kq, 0, hh, c.y);
+        tma_load_3d(sm + OFF_KQ + 8192, &tmq, bar_kq, 0, hh, c.y);
+        tma_load_3d(sm + OFF_KQ + 16384, &tmk, bar_kq, 64, hh, c.y);
+        tma_load_3d(sm + OFF_KQ + 24576, &tmq, bar_kq, 64, hh, c.y);
+    };
+    auto load_g = [&](int it) {  // thread 0
+        const int4 c = p.info[it % maxc];
+        mbar_arrive_expect_tx(bar_g, TX_G);
+        tma_load_3d(sm + OFF_G, &tmg, bar_g, 0, it / maxc, c.y);
+    };
 
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
+        mbar_init(bar_kq, 1);
+        mbar_init(bar_g, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
@@ -141,20 +155,21 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t tbase = *s_tmem;
     bool failed = false;
     uint32_t mma_phase = 0;
+    // loads issued and not yet waited for (thread 0's view; for the exit path)
+    int kq_issued = 0, g_issued = 0;
     int item = advance(blockIdx.x);
-    float beta_next = 0.f;
+    float beta_next = 0.f;  // (tid < C) this thread's beta of the next item
+    auto fetch_beta = [&](int it) {
+        const int4 c = p.info[it % maxc];
+        return tid < c.z ? p.beta[(size_t)(c.y + tid) * p.H + it / maxc] : 0.f;
+    };
     if (item < nitems) {
-        const int4 c0i = p.info[item % maxc];
-        const int h0i = item / maxc;
         if (tid == 0) {
-            mbar_arrive_expect_tx(bar_tma, TX_BYTES);
-            tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, h0i, c0i.y);
-            tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, h0i, c0i.y);
-            tma_load_3d(sm + OFF_Q, &tmq, bar_tma, 0, h0i, c0i.y);
-            tma_load_3d(sm + OFF_Q + 8192, &tmq, bar_tma, 64, h0i, c0i.y);
-            tma_load_3d(sm + OFF_G, &tmg, bar_tma, 0, h0i, c0i.y);
+            load_kq(item);
+            load_g(item);
+            kq_issued = g_issued = 1;
         }
-        if (tid < C) beta_next = tid < c0i.z ? p.beta[(size_t)(c0i.y + tid) * p.H + h0i] : 0.f;
+        if (tid < C) beta_next = fetch_beta(item);
     }
     int n = 0;
     for (; item < nitems && !failed; ++n) {
@@ -162,9 +177,8 @@ __global__ void __launch_bounds__(NT, 1)
         const int L = ci.z, h = item / maxc;
         const int nxt = advance(item + gridDim.x);
         uint8_t* blob = p.blobs + ((size_t)(item % maxc) * p.H + h) * BLOB;
-        bool armed = false;  // (thread 0) next item's transaction count registered
         if (tid < C) sbeta[tid] = beta_next;
-        bool ok = mbar_wait(bar_tma, n & 1, kWaitNs);
+        bool ok = mbar_wait(bar_g, n & 1, kWaitNs) && mbar_wait(bar_kq, n & 1, kWaitNs);
         if (__syncthreads_or(!ok)) {
             failed = true;
             break;
@@ -192,34 +206,51 @@ __global__ void __launch_bounds__(NT, 1)
             const float Gm = gmax - kRef;
             sGm[c] = Gm;
             seGm[c] = expf(Gm);
-            sGC[c] = expf(G);
             sGL[c] = G;
             slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
         }
-        if (tid == 0) bulk_wait_read();  // previous item's write-out has read its tiles
         const bool slow = __syncthreads_or(slow_local);
-        if (tid < D) {
-            sWsc[tid] = slow ? -1.f : -seGm[tid];  // the blob holds -W
-            sKsc[tid] = slow ? 1.f : expf(sGL[tid] - sGm[tid]);
+        if (tid < D) {  // row scales of the chain kernel; -W column scale
+            const float gl = sGL[tid];
+            sWsc[tid] = slow ? -1.f : -seGm[tid];
+            float* sc = reinterpret_cast<float*>(blob + BL_SC);
+            sc[tid] = expf(gl);
+            sc[D + tid] = slow ? 1.f : expf(gl - sGm[tid]);
         }
-        // ---------------- exact A and P on CUDA cores (rare: extreme decay)
+        // -------- exact A (fp32, into the Tb region) and P (straight to the
+        // blob) on CUDA cores (rare: extreme decay)
         if (slow) {
             const float* G = reinterpret_cast<const float*>(sm + OFF_G);
-            float* Af = reinterpret_cast<float*>(sm + OFF_LAP);
-            float* Pf = Af + C * C;
-            for (int idx = tid; idx < C * C; idx += NT) {
-                const int r = idx >> 6, i = idx & 63;
-                float a = 0.f, pp = 0.f;
-                if (r < L && i <= r) {
+            float* Af = reinterpret_cast<float*>(sm + OFF_TB);
+            for (int task = tid; task < C * 8; task += NTI) {
+                const int r = task >> 3, i0 = 8 * (task & 7);
+                float a[8], pp[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a[j] = pp[j] = 0.f;
+                if (r < L) {
                     for (int c = 0; c < D; ++c) {
-                        const float e = expf(G[r * D + c] - G[i * D + c]);
-                        const float ki = tile_elem(sm + OFF_K, 8192, i, c);
-                        a += tile_elem(sm + OFF_K, 8192, r, c) * ki * e;
-                        pp += tile_elem(sm + OFF_Q, 8192, r, c) * ki * e;
+                        const float kr = tile_elem(sm + OFF_KQ, 16384, r, c);
+                        const float qr = tile_elem(sm + OFF_KQ + 8192, 16384, r, c);
+                        const float gr = G[r * D + c];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int i = i0 + j;
+                            if (i <= r) {
+                                const float e = expf(gr - G[i * D + c]);
+                                const float ki = tile_elem(sm + OFF_KQ, 16384, i, c) * e;
+                                a[j] += kr * ki;
+                                pp[j] += qr * ki;
+                            }
+                        }
                     }
                 }
-                Af[a_idx(r, i)] = (i < r) ? sbeta[r] * a : 0.f;
-                Pf[idx] = pp;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = i0 + j;
+                    Af[a_idx(r, i)] = (i < r) ? sbeta[r] * a[j] : 0.f;
+                    if (i > r) pp[j] = 0.f;
+                }
+                *reinterpret_cast<uint4*>(blob + BL_PM + sw128_off(r, task & 7)) = pack8(pp);
             }
             __syncthreads();
         }
@@ -227,14 +258,12 @@ __global__ void __launch_bounds__(NT, 1)
         {
             const float* G = reinterpret_cast<const float*>(sm + OFF_G);
 #pragma unroll
-            for (int s = 0; s < (C * 16) / NT; ++s) {
-                const int it = tid + NT * s;
+            for (int s = 0; s < (C * 16) / NTI; ++s) {
+                const int it = tid + NTI * s;
                 const int r = it >> 4, j = it & 15, kb = j >> 3, ch = j & 7, c0 = 8 * j;
                 const uint32_t o64 = sw128_off(r, ch);
-                uint8_t* pk = sm + OFF_K + kb * 8192 + o64;
-                const uint8_t* pq = sm + OFF_Q + kb * 8192 + o64;
-                uint8_t* pqg = sm + OFF_WQ + kb * 16384 + 8192 + o64;
-                uint8_t* pr = sm + OFF_RAP + kb * 8192 + o64;
+                uint8_t* pk = sm + OFF_KQ + kb * 16384 + o64;
+                uint8_t* pq = pk + 8192;
                 float lk[8], lq[8], rk[8], qg[8];
                 if (r < L) {
                     float k8[8], q8[8], g8[8];
@@ -271,35 +300,18 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i) lk[i] = lq[i] = rk[i] = qg[i] = 0.f;
                 }
-                if (!slow) {
-                    *reinterpret_cast<uint4*>(sm + OFF_LAP + kb * 16384 + o64) = pack8(lk);
-                    *reinterpret_cast<uint4*>(sm + OFF_LAP + kb * 16384 + 8192 + o64) =
-                        pack8(lq);
-                } else {
-                    *reinterpret_cast<uint4*>(pk) = pack8(lk);
-                }
-                *reinterpret_cast<uint4*>(pr) = pack8(rk);
-                *reinterpret_cast<uint4*>(pqg) = pack8(qg);
+                *reinterpret_cast<uint4*>(pk) = pack8(lk);
+                *reinterpret_cast<uint4*>(pq) = pack8(lq);
+                *reinterpret_cast<uint4*>(sm + OFF_RAP + kb * 8192 + o64) = pack8(rk);
+                *reinterpret_cast<uint4*>(blob + BL_WQ + kb * 16384 + 8192 + o64) = pack8(qg);
+                *reinterpret_cast<uint4*>(blob + BL_RAP + kb * 8192 + o64) = pack8(rk);
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid < C && nxt < nitems) {
-            const int4 cn = p.info[nxt % maxc];
-            beta_next = tid < cn.z ? p.beta[(size_t)(cn.y + tid) * p.H + nxt / maxc] : 0.f;
-        }
-        if (!slow && nxt < nitems && tid == 0) {  // K and Q are consumed: prefetch
-            const int4 cn = p.info[nxt % maxc];
-            const int hn = nxt / maxc;
-            mbar_arrive_expect_tx(bar_tma, TX_BYTES);
-            armed = true;
-            tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, hn, cn.y);
-            tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, hn, cn.y);
-            tma_load_3d(sm + OFF_Q, &tmq, bar_tma, 0, hn, cn.y);
-            tma_load_3d(sm + OFF_Q + 8192, &tmq, bar_tma, 64, hn, cn.y);
-        }
+        if (tid < C && nxt < nitems) beta_next = fetch_beta(nxt);
         // ------------------------------------------------ A, P (M=128, N=64)
         if (!slow) {
             if (tid == 0) {
@@ -308,7 +320,7 @@ __global__ void __launch_bounds__(NT, 1)
                 for (int ks = 0; ks < 8; ++ks) {
                     const int kb = ks >> 2, kk = ks & 3;
                     mma_bf16(tbase + TM_X,
-                             sdesc_sw128(sbase + OFF_LAP + kb * 16384 + kk * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_KQ + kb * 16384 + kk * 32, 16, 1024),
                              sdesc_sw128(sbase + OFF_RAP + kb * 8192 + kk * 32, 16, 1024), id,
                              ks > 0);
                 }
@@ -322,50 +334,28 @@ __global__ void __launch_bounds__(NT, 1)
             }
             tc_fence_after();
         }
-        // ----- A -> fp32 (swizzled, in the G region), P -> bf16 PM rows 64-127
+        // ------ A -> fp32 (swizzled, in the G region); P -> bf16, to the blob
         {
             float* Af = reinterpret_cast<float*>(sm + OFF_G);
             const int m = trow;  // TMEM lane == row of the 128-row result
             if (!slow) {
-                if (cq < 2) {
-                    uint32_t v[32];
-                    tmem_ld32(tbase + tlane + TM_X + cq * 32, v);
-                    tmem_wait_ld();
-                    if (m < C) {
-                        const float b = sbeta[m];
+                uint32_t v[32];
+                tmem_ld32(tbase + tlane + TM_X + cq * 32, v);
+                tmem_wait_ld();
+                if (m < C) {
+                    const float b = sbeta[m];
 #pragma unroll
-                        for (int i4 = 0; i4 < 8; ++i4) {
-                            const int col = cq * 32 + 4 * i4;
-                            float y[4];
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const int col = cq * 32 + 4 * i4;
+                        float y[4];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                y[i] = (m < L && col + i < m) ? b * __uint_as_float(v[4 * i4 + i])
-                                                              : 0.f;
-                            *reinterpret_cast<float4*>(Af + a_idx(m, col)) =
-                                make_float4(y[0], y[1], y[2], y[3]);
-                        }
-                    } else {
-                        const int r = m - C;
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            float y[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int col = cq * 32 + q4 * 8 + i;
-                                y[i] = (r < L && col <= r) ? __uint_as_float(v[q4 * 8 + i]) : 0.f;
-                            }
-                            *reinterpret_cast<uint4*>(sm + OFF_MID +
-                                                      sw128_off(m, (cq * 32 + q4 * 8) >> 3)) =
-                                pack8(y);
-                        }
+                        for (int i = 0; i < 4; ++i)
+                            y[i] = (m < L && col + i < m) ? b * __uint_as_float(v[4 * i4 + i])
+                                                          : 0.f;
+                        *reinterpret_cast<float4*>(Af + a_idx(m, col)) =
+                            make_float4(y[0], y[1], y[2], y[3]);
                     }
-                }
-            } else {
-                const float4* srcA = reinterpret_cast<const float4*>(sm + OFF_LAP);
-                float4* dstA = reinterpret_cast<float4*>(Af);
-                for (int i = tid; i < C * C / 4; i += NT) dstA[i] = srcA[i];
-                if (m >= C && cq < 2) {
-                    const float* Pf = reinterpret_cast<const float*>(sm + OFF_LAP) + C * C;
+                } else {
                     const int r = m - C;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
@@ -373,19 +363,20 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int col = cq * 32 + q4 * 8 + i;
-                            y[i] = (r < L && col <= r) ? Pf[r * C + col] : 0.f;
+                            y[i] = (r < L && col <= r) ? __uint_as_float(v[q4 * 8 + i]) : 0.f;
                         }
-                        *reinterpret_cast<uint4*>(sm + OFF_MID +
-                                                  sw128_off(m, (cq * 32 + q4 * 8) >> 3)) =
+                        *reinterpret_cast<uint4*>(blob + BL_PM +
+                                                  sw128_off(r, (cq * 32 + q4 * 8) >> 3)) =
                             pack8(y);
                     }
                 }
+            } else {
+                const float4* srcA = reinterpret_cast<const float4*>(sm + OFF_TB);
+                float4* dstA = reinterpret_cast<float4*>(Af);
+                for (int i = tid; i < C * C / 4; i += NTI) dstA[i] = srcA[i];
             }
         }
-        fence_async_smem();
-        tc_fence_before();
         __syncthreads();
-        tc_fence_after();
         // ------------------ UT transform: T = (I + A)^{-1}, blocked 16 x 16
         {
             const float* Af = reinterpret_cast<const float*>(sm + OFF_G);
@@ -411,8 +402,9 @@ __global__ void __launch_bounds__(NT, 1)
             offdiag_level<1>(Af, Tf, Mf, warp, lane);
             offdiag_level<2>(Af, Tf, Mf, warp, lane);
             offdiag_level<3>(Af, Tf, Mf, warp, lane);
-            // Tb = T diag(b) -> bf16, K-major rows of 64 (rows 0-63)
-            for (int e = tid; e < C * 8; e += NT) {
+            // Tb = T diag(b) -> bf16, K-major rows of 64 (rows 0-63), in
+            // shared memory for the W product and in the blob for the chain
+            for (int e = tid; e < C * 8; e += NTI) {
                 const int r = e >> 3, ch = e & 7;
                 const float4 t0v = *reinterpret_cast<const float4*>(Tf + t_idx(r, 8 * ch));
                 const float4 t1v = *reinterpret_cast<const float4*>(Tf + t_idx(r, 8 * ch + 4));
@@ -423,31 +415,26 @@ __global__ void __launch_bounds__(NT, 1)
                     const int col = 8 * ch + i;
                     y[i] = (col <= r) ? tv[i] * sbeta[col] : 0.f;
                 }
-                *reinterpret_cast<uint4*>(sm + OFF_TB + sw128_off(r, ch)) = pack8(y);
+                const uint4 u = pack8(y);
+                *reinterpret_cast<uint4*>(sm + OFF_TB + sw128_off(r, ch)) = u;
+                *reinterpret_cast<uint4*>(blob + BL_TB + sw128_off(r, ch)) = u;
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (nxt < nitems && tid == 0) {  // G region is free: prefetch g (and K, Q)
-            const int4 cn = p.info[nxt % maxc];
-            const int hn = nxt / maxc;
-            if (!armed) {
-                mbar_arrive_expect_tx(bar_tma, TX_BYTES);
-                armed = true;
-            }
-            tma_load_3d(sm + OFF_G, &tmg, bar_tma, 0, hn, cn.y);
-        }
         // ---------------------------------- W = Tb (K*E) [*exp(Gm)]  (N=128)
         if (tid == 0) {
+            if (nxt < nitems) {  // the G region is free: fetch the next g
+                load_g(nxt);
+                ++g_issued;
+            }
             constexpr uint32_t id = idesc_bf16_f32(128, 128, false, true);
-            const uint32_t bW = slow ? OFF_K : OFF_LAP;
-            const uint32_t lboW = slow ? 8192u : 16384u;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tbase + TM_W, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
-                         sdesc_sw128(sbase + bW + ks * 2048, lboW, 1024), id, ks > 0);
+                         sdesc_sw128(sbase + OFF_KQ + ks * 2048, 16384, 1024), id, ks > 0);
             mma_commit(bar_mma);
         }
         ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
@@ -457,54 +444,39 @@ __global__ void __launch_bounds__(NT, 1)
             break;
         }
         tc_fence_after();
-        if (slow && nxt < nitems && tid == 0) {  // exact path: K region free only now
-            const int4 cn = p.info[nxt % maxc];
-            const int hn = nxt / maxc;
-            tma_load_3d(sm + OFF_K, &tmk, bar_tma, 0, hn, cn.y);
-            tma_load_3d(sm + OFF_K + 8192, &tmk, bar_tma, 64, hn, cn.y);
-            tma_load_3d(sm + OFF_Q, &tmq, bar_tma, 0, hn, cn.y);
-            tma_load_3d(sm + OFF_Q + 8192, &tmq, bar_tma, 64, hn, cn.y);
+        if (tid == 0 && nxt < nitems) {  // K, Q region is free: fetch the next K, Q
+            load_kq(nxt);
+            ++kq_issued;
         }
-        // W (rows 0-63), column-scaled -> bf16 into the W rows of [W ; Q*Gam]
+        // -W (rows 0-63), column-scaled -> bf16, to the blob's [-W ; Q*Gam]
         if (quarter < 2) {
             const int r = trow;
-            uint32_t v[32];
-            tmem_ld32(tbase + tlane + TM_W + cq * 32, v);
-            tmem_wait_ld();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int col = cq * 32 + q4 * 8;
-                float sc[8], y[8];
-                load8(sWsc + col, sc);
+            for (int hcol = 0; hcol < 2; ++hcol) {
+                const int cbase = 64 * cq + 32 * hcol;
+                uint32_t v[32];
+                tmem_ld32(tbase + tlane + TM_W + cbase, v);
+                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]) * sc[i];
-                *reinterpret_cast<uint4*>(sm + OFF_WQ + (col >> 6) * 16384 +
-                                          sw128_off(r, (col & 63) >> 3)) = pack8(y);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int col = cbase + q4 * 8;
+                    float sc[8], y[8];
+                    load8(sWsc + col, sc);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]) * sc[i];
+                    *reinterpret_cast<uint4*>(blob + BL_WQ + (col >> 6) * 16384 +
+                                              sw128_off(r, (col & 63) >> 3)) = pack8(y);
+                }
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ---- hand the chain's operands to the workspace (asynchronously)
-        if (tid == 0) {
-            bulk_s2g(blob + BL_WQ, sm + OFF_WQ, 32768);
-            bulk_s2g(blob + BL_RAP, sm + OFF_RAP, 16384);
-            bulk_s2g(blob + BL_PM, sm + OFF_PM, 8192);
-            bulk_s2g(blob + BL_TB, sm + OFF_TB, 8192);
-            bulk_commit();
-        }
-        if (tid < D) {
-            float* sc = reinterpret_cast<float*>(blob + BL_SC);
-            sc[tid] = sGC[tid];
-            sc[D + tid] = sKsc[tid];
         }
         item = nxt;
     }
-    if (tid == 0) bulk_wait_all();
     if (failed && tid == 0) {
+        // wait (bounded) for this CTA's copies and products still in flight
         if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
-        mbar_wait(bar_tma, n & 1, kWaitNs);
+        // (a wait on a phase that has already completed returns at once)
+        if (kq_issued > 0) mbar_wait(bar_kq, (kq_issued - 1) & 1, kWaitNs);
+        if (g_issued > 0) mbar_wait(bar_g, (g_issued - 1) & 1, kWaitNs);
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
@@ -812,12 +784,35 @@ bool split_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
 
 }  // namespace
 
-cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,
-                                   const float* beta, const float* h0,
-                                   const int32_t* cu_seqlens, int T, int N, int H,
-                                   const int4* chunk_info, int maxc, const int* chunk_start,
-                                   uint32_t* status, void* blobs, void* o, float* hN,
-                                   cudaStream_t st) {
+cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
+                               int total, int H, const int4* chunk_info, int maxc,
+                               uint32_t* status, void* blobs, cudaStream_t st) {
+    if (total == 0 || maxc == 0) return cudaSuccess;
+    CUtensorMap mq, mk, mg;
+    if (!split_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)intra::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long items = (long long)maxc * H;
+    const int grid = (int)(items < 2 * sms ? items : 2 * sms);
+    intra::Params pa{beta, chunk_info, maxc, H, status, status, static_cast<uint8_t*>(blobs)};
+    intra::chunk_intra_kernel<<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(mq, mk, mg, pa);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
+                               int N, int H, const int* chunk_start, uint32_t* status,
+                               const void* blobs, void* o, float* hN, cudaStream_t st) {
     const int total = cu_seqlens ? T : N * T;
     if (total == 0) {
         if (hN) {
@@ -827,40 +822,31 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
         }
         return cudaSuccess;
     }
-    CUtensorMap mq, mk, mv, mg;
-    if (!split_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    CUtensorMap mv;
+    if (!split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel,
+    cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)intra::SMEM_BYTES);
+                                         (int)chain::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chain::chunk_chain_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)chain::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    uint8_t* bl = static_cast<uint8_t*>(blobs);
-    if (maxc > 0) {
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const long long items = (long long)maxc * H;
-        const int grid = (int)(items < sms ? items : sms);
-        intra::Params pa{beta, chunk_info, maxc, H, status, status, bl};
-        intra::chunk_intra_kernel<<<grid, NT, intra::SMEM_BYTES, st>>>(mq, mk, mg, pa);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    chain::Params pb{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
-                     (__nv_bfloat16*)o, hN};
+    chain::Params pb{h0, cu_seqlens, T, H, chunk_start, status, status,
+                     static_cast<const uint8_t*>(blobs), (__nv_bfloat16*)o, hN};
     chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
     return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* h0,
+                                   const int32_t* cu_seqlens, int T, int N, int H,
+                                   const int4* chunk_info, int maxc, const int* chunk_start,
+                                   uint32_t* status, void* blobs, void* o, float* hN,
+                                   cudaStream_t st) {
+    const int total = cu_seqlens ? T : N * T;
+    cudaError_t e =
+        launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs, st);
+    if (e != cudaSuccess) return e;
+    return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN, st);
 }
 
 }  // namespace kda

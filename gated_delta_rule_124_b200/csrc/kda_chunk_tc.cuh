@@ -25,5 +25,13 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
                                    const int4* chunk_info, int maxc, const int* chunk_start,
                                    uint32_t* status, void* blobs, void* o, float* hN,
                                    cudaStream_t st);
+// Its two kernels one at a time (the chain kernel reads what the intra kernel
+// wrote, on the same stream).
+cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
+                               int total, int H, const int4* chunk_info, int maxc,
+                               uint32_t* status, void* blobs, cudaStream_t st);
+cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
+                               int N, int H, const int* chunk_start, uint32_t* status,
+                               const void* blobs, void* o, float* hN, cudaStream_t st);
 
 }  // namespace kda

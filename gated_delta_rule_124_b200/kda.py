@@ -38,7 +38,8 @@ EXPORTS = (
     "kda_status_string", "kda_chunk_fwd_workspace_size", "kda_chunk_fwd",
     "kda_num_chunks_upper_bound", "kda_chunk_gate_cumsum", "kda_chunk_intra",
     "kda_chunk_inter", "kda_chunk_output", "kda_decode_step", "kda_get_device_status",
-    "kda_chunk_fwd_noalloc",
+    "kda_chunk_fwd_noalloc", "kda_chunk_split_workspace_size", "kda_chunk_split_intra",
+    "kda_chunk_split_chain",
 )
 
 
@@ -64,6 +65,9 @@ _SIGS = {
     "kda_decode_step": ([_vp] * 7 + [_i] * 5 + [_vp], _i),
     "kda_get_device_status": ([_vp, _vp], _i),
     "kda_chunk_fwd_noalloc": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp], _i),
+    "kda_chunk_split_workspace_size": ([_i, _i, _i], _sz),
+    "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
+    "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
 
 # Size of the library's built-in scratch used by kda_chunk_fwd_noalloc.
@@ -189,6 +193,27 @@ def kda_chunk_output(q, k, G, U, chunk_states, cu_seqlens, B, T, num_seqs, H, dk
                                  B, T, num_seqs, H, dk, dv, chunk, dtype_code(dtype), _p(o),
                                  _p(workspace), wb, _stream(stream))
     return _ret(st, "kda_chunk_output", check)
+
+
+def kda_chunk_split_workspace_size(total_tokens, num_seqs, H) -> int:
+    return int(load().kda_chunk_split_workspace_size(total_tokens, num_seqs, H))
+
+
+def kda_chunk_split_intra(q, k, g, beta, cu_seqlens, B, T, num_seqs, H, workspace,
+                          workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_split_intra(_p(q), _p(k), _p(g), _p(beta), _p(cu_seqlens), B, T,
+                                      num_seqs, H, _p(workspace), wb, _stream(stream))
+    return _ret(st, "kda_chunk_split_intra", check)
+
+
+def kda_chunk_split_chain(v, initial_state, cu_seqlens, B, T, num_seqs, H, o, final_state,
+                          workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_split_chain(_p(v), _p(initial_state), _p(cu_seqlens), B, T,
+                                      num_seqs, H, _p(o), _p(final_state), _p(workspace), wb,
+                                      _stream(stream))
+    return _ret(st, "kda_chunk_split_chain", check)
 
 
 def kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,

@@ -82,10 +82,20 @@ const char* kda_status_string(kda_status_t status);
  * Workspace: device scratch of at least kda_chunk_fwd_workspace_size() bytes,
  *      256-byte aligned, owned by the caller, reusable across calls on the same
  *      stream; it also holds the device status word.
- * Shapes: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}.  bf16 with
- *      dk = dv = 128 and chunk = 64 runs the tensor-core (tcgen05) kernel;
- *      other supported shapes run the CUDA-core kernels.  Otherwise
- *      KDA_ERR_UNSUPPORTED.
+ * Shapes: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}; anything else is
+ *      KDA_ERR_UNSUPPORTED.  bf16 with dk = dv = 128 and chunk = 64 runs on the
+ *      tensor cores (tcgen05 / TMEM / TMA), in one of two plans:
+ *        fused -- one kernel, one CTA per (sequence, head) walking its chunks;
+ *        split -- kda_chunk_split_intra then kda_chunk_split_chain (below),
+ *                 for problems with too few (sequence, head) pairs to fill
+ *                 the GPU.
+ *      split is taken when num_seqs * H < 2 * (number of SMs), fused
+ *      otherwise.  Other supported shapes run the CUDA-core kernels (the four
+ *      step calls below, in order).  The environment variable KDA_CHUNK_PATH =
+ *      fused | split | simt forces one plan (testing; shapes without the
+ *      tensor-core plans always run the CUDA-core kernels).
+ *      kda_chunk_fwd_workspace_size() follows the same choice, so read the
+ *      environment before sizing the workspace, not between the two calls.
  */
 size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
                                     int chunk, kda_dtype_t dtype);
@@ -157,6 +167,43 @@ kda_status_t kda_chunk_output(const void* q, const void* k, const float* G, cons
                               int T, int num_seqs, int H, int dk, int dv, int chunk,
                               kda_dtype_t dtype, void* o, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* --------------------------------- tensor-core split plan, one kernel per call
+ * The two kernels of the split plan (see kda_chunk_fwd), callable one at a
+ * time so that each can be checked and timed on its own.  q, k, v, o bf16;
+ * dk = dv = 128; chunk = 64 (no other shape: the call returns
+ * KDA_ERR_UNSUPPORTED when the tensor-core kernels are not in the library).
+ *   kda_chunk_split_intra: chunk-parallel over (chunk, head).  Builds the
+ *     chunk table, then per chunk computes G (a1), A, the UT-transform
+ *     inverse and W (a2), and the chunk-local operands of a4 (Q * Gam, the
+ *     masked P), and stores them, in bf16 tensor-core tile layout, in the
+ *     workspace (an opaque format of this library version).
+ *   kda_chunk_split_chain: two CTAs per (sequence, head), one per half of
+ *     the value columns (the transition acts on the key side only, so the
+ *     columns of S evolve independently).  Serial over the chunks of the
+ *     sequence: Ut = Tm diag(beta) V, U_n = Ut - W S_n, O_n, S_{n+1} (a3, a4),
+ *     S carried in fp32 in tensor memory.  Writes o and final_state (NULL:
+ *     not written).  It must follow kda_chunk_split_intra on the same
+ *     stream, with the same workspace, cu_seqlens and shapes; it does not
+ *     reset the device status word, so a failure of either kernel is
+ *     reported by kda_get_device_status().
+ * Workspace: at least kda_chunk_split_workspace_size() bytes, 256-byte
+ *   aligned (it is kda_chunk_fwd_workspace_size() when kda_chunk_fwd takes
+ *   the split plan).  Defining passage: Kimi Linear (aiwiki.ai), "The
+ *   constrained DPLR form and the chunkwise algorithm" (the intra-chunk part
+ *   is parallel across chunks; only the state passes from chunk to chunk).
+ */
+size_t kda_chunk_split_workspace_size(int total_tokens, int num_seqs, int H);
+
+kda_status_t kda_chunk_split_intra(const void* q, const void* k, const float* g,
+                                   const float* beta, const int32_t* cu_seqlens, int B, int T,
+                                   int num_seqs, int H, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+kda_status_t kda_chunk_split_chain(const void* v, const float* initial_state,
+                                   const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                                   void* o, float* final_state, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------- decode
  * kda_decode_step: one token per (sequence, head), state updated in place.

@@ -122,6 +122,24 @@ def test_step_calls_reject_bad_arguments(lib):
                                 dv=96, dtype="f32", o=FAKE, **common) == kda.KDA_ERR_UNSUPPORTED
 
 
+def test_split_calls_reject_bad_arguments(lib):
+    f = kda.kda_chunk_split_workspace_size
+    assert f(4096, 2, 32) > 0
+    assert f(8192, 2, 32) > f(4096, 2, 32)
+    assert f(4096, 0, 32) == 0 and f(-1, 1, 32) == 0 and f(64, 1, 0) == 0
+    common = dict(cu_seqlens=None, B=1, T=64, num_seqs=1, H=1, workspace=FAKE * 2,
+                  workspace_bytes=1 << 40, stream=0, check=False)
+    intra = dict(q=FAKE, k=FAKE, g=FAKE, beta=FAKE, **common)
+    chain = dict(v=FAKE, initial_state=None, o=FAKE, final_state=None, **common)
+    assert kda.kda_chunk_split_intra(**{**intra, "q": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_split_intra(**{**intra, "g": FAKE + 4}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_split_intra(**{**intra, "B": 0}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_split_intra(**{**intra, "num_seqs": 2}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_split_chain(**{**chain, "o": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_split_chain(**{**chain, "v": FAKE + 2}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_chunk_split_chain(**{**chain, "H": 0}) == kda.KDA_ERR_INVALID_ARG
+
+
 def test_get_device_status_rejects_bad_workspace(lib):
     assert kda.kda_get_device_status(None, 0) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_get_device_status(FAKE + 16, 0) == kda.KDA_ERR_INVALID_ARG

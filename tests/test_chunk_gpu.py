@@ -283,3 +283,41 @@ def test_split_and_fused_agree_closely(monkeypatch):
     torch.cuda.synchronize()
     assert rel_err(o2, o1.double().cpu().numpy()) <= 1e-2
     assert rel_err(h2, h1.double().cpu().numpy()) <= 1e-5
+
+
+def test_split_step_calls_compose(monkeypatch):
+    """kda_chunk_split_intra then kda_chunk_split_chain is the split plan of
+    kda_chunk_fwd: identical bits, and within tolerance of the oracle."""
+    case = wl.make_prefill(308, [333, 64, 0, 700], H=3, dk=128, dv=128, chunk=64,
+                           dtype="bf16", varlen=True)
+    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
+    o1, h1 = run_fwd(case)
+    c = case.to("cuda")
+    n = kda.kda_chunk_split_workspace_size(c.total, c.N, c.H)
+    assert n == kda.kda_chunk_fwd_workspace_size(c.total, c.N, c.H, 128, 128, 64, "bf16")
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    o = torch.full_like(c.v, float("nan"))
+    hN = torch.full((c.N, c.H, 128, 128), float("nan"), device="cuda")
+    args = (c.cu_seqlens, 1, c.total, c.N, c.H)
+    kda.kda_chunk_split_intra(c.q, c.k, c.g, c.beta, *args, ws)
+    kda.kda_chunk_split_chain(c.v, c.initial_state, *args, o, hN, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    assert torch.equal(o, o1) and torch.equal(hN, h1)
+    ro, rh = oracle_prefill(case)
+    assert rel_err(o, ro) <= tol_for("bf16") and rel_err(hN, rh) <= tol_for("bf16")
+
+
+def test_split_chain_keeps_the_intra_status():
+    """A bad cu_seqlens seen by the intra call stays reported after the chain
+    call (the chain call does not reset the status word)."""
+    case = wl.make_prefill(309, [128, 64], H=2, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    c = case.to("cuda")
+    bad = torch.tensor([0, 150, 140], dtype=torch.int32, device="cuda")  # decreasing
+    ws = torch.empty(kda.kda_chunk_split_workspace_size(c.total, c.N, c.H), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.zeros_like(c.v)
+    args = (bad, 1, c.total, c.N, c.H)
+    kda.kda_chunk_split_intra(c.q, c.k, c.g, c.beta, *args, ws)
+    kda.kda_chunk_split_chain(c.v, None, *args, o, None, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
