@@ -300,7 +300,8 @@ def run_ours(args, rank, world, local_rank):
 def prefill_path(Np, H, dk, dv, C, dtype="bf16"):
     """Which prefill kernels kda_chunk_fwd runs (the library's rule, see
     include/kda.h): 'fused' (one tensor-core kernel), 'split' (chunk-parallel
-    intra kernel + per-chain kernel) or 'simt' (CUDA-core kernels)."""
+    intra kernel + per-chain kernel), 'overlap' (the two co-scheduled in one
+    launch) or 'simt' (CUDA-core kernels)."""
     import torch
     env = os.environ.get("KDA_CHUNK_PATH")
     if env == "simt" or not (dtype == "bf16" and dk == dv == 128 and C == 64):
@@ -308,6 +309,10 @@ def prefill_path(Np, H, dk, dv, C, dtype="bf16"):
     if env in ("fused", "split"):
         return env
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    if 2 * Np * H <= sms:
+        return "overlap"
+    if env == "overlap":
+        return "split"
     return "split" if Np * H < 2 * sms else "fused"
 
 
@@ -350,8 +355,8 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     if path != "simt":
         o = torch.empty_like(P.v)
         hN = torch.empty(Np, H, dk, dv, device=dev)
-        if path == "fused":
-            name = "chunk_fwd_tc"
+        if path in ("fused", "overlap"):
+            name = "chunk_fwd_tc" if path == "fused" else "chunk_fwd_overlap"
             calls = {name: lambda: kda.kda_chunk_fwd(
                 P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc, Tc, Np, H, dk,
                 dv, C, "bf16", o, hN, ws)}

@@ -47,7 +47,7 @@ kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, 
 }
 
 // Which kernels kda_chunk_fwd runs.
-enum class Path { Simt, Fused, Split };
+enum class Path { Simt, Fused, Split, Overlap };
 
 int sm_count() {
     int dev = 0, n = 0;
@@ -59,10 +59,12 @@ int sm_count() {
     return n;
 }
 
-// bf16, dk = dv = 128, chunk 64 runs on the tensor cores: one kernel with one
-// CTA per (sequence, head) when there are enough of them to fill the GPU,
-// otherwise the two-kernel split (chunk-parallel intra-chunk kernel + per-chain
-// kernel).  KDA_CHUNK_PATH = fused | split | simt forces a path (testing).
+// bf16, dk = dv = 128, chunk 64 runs on the tensor cores.  With few (sequence,
+// head) chains (2 N H <= SMs) the chunk-parallel intra-chunk kernel and the
+// per-chain kernel run co-scheduled in one launch; with somewhat more
+// (N H < 2 SMs) as two launches; otherwise one kernel with one CTA per
+// (sequence, head).  KDA_CHUNK_PATH = fused | split | overlap | simt forces a
+// path (testing); overlap falls back to split where it does not apply.
 Path select_path(int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
     const bool tc_shape = dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
                           kda::tc_path_available();
@@ -71,12 +73,16 @@ Path select_path(int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
     if (!tc_shape) return Path::Simt;
     if (env && !strcmp(env, "fused")) return Path::Fused;
     if (env && !strcmp(env, "split")) return Path::Split;
+    const bool overlap = kda::overlap_grid(N, H) > 0;
+    if (env && !strcmp(env, "overlap")) return overlap ? Path::Overlap : Path::Split;
+    if (overlap) return Path::Overlap;
     return ((long long)N * H < 2LL * sm_count()) ? Path::Split : Path::Fused;
 }
 
 Workspace carve_for(void* base, const Prefill& p, int H, int dk, int dv, int chunk, Path path) {
     return kda::carve(base, p.total, p.N, H, dk, dv, chunk, path == Path::Simt,
-                      path == Path::Split ? kda::split_blob_bytes() : 0);
+                      (path == Path::Split || path == Path::Overlap) ? kda::split_blob_bytes()
+                                                                     : 0);
 }
 
 size_t workspace_bytes_for(int total, int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
@@ -166,6 +172,12 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
         return from_cuda(kda::launch_chunk_fwd_tc(q, k, v, g, beta, initial_state, cu_seqlens,
                                                   T, p.N, H, w.chunk_start, w.status, o,
                                                   final_state, st));
+    }
+    if (path == Path::Overlap) {
+        return from_cuda(kda::launch_chunk_fwd_overlap(q, k, v, g, beta, initial_state,
+                                                       cu_seqlens, T, p.N, H, w.chunk_info,
+                                                       maxc, w.chunk_start, w.status, w.blobs,
+                                                       w.flags, o, final_state, st));
     }
     if (path == Path::Split) {
         return from_cuda(kda::launch_chunk_fwd_split(q, k, v, g, beta, initial_state,

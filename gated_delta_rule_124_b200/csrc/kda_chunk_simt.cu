@@ -29,9 +29,9 @@ __global__ void build_chunk_table_kernel(const int32_t* __restrict__ cu, int B, 
                                          int* __restrict__ chunk_start,
                                          int4* __restrict__ info) {
     __shared__ int warp_sums[32];
-    __shared__ int bad;
+    __shared__ int bad, most;
     const int tid = threadIdx.x, nt = blockDim.x;
-    if (tid == 0) bad = 0;
+    if (tid == 0) bad = most = 0;
     __syncthreads();
     auto seq_lo = [&](int s) -> int { return cu ? cu[s] : s * T; };
     const int total = cu ? T : B * T;
@@ -51,8 +51,13 @@ __global__ void build_chunk_table_kernel(const int32_t* __restrict__ cu, int B, 
     // contiguous run of sequences
     const int per = (N + nt - 1) / nt;
     const int s0 = min(N, tid * per), s1 = min(N, s0 + per);
-    int local = 0;
-    for (int s = s0; s < s1; ++s) local += (seq_lo(s + 1) - seq_lo(s) + chunk - 1) / chunk;
+    int local = 0, lmax = 0;
+    for (int s = s0; s < s1; ++s) {
+        const int c = (seq_lo(s + 1) - seq_lo(s) + chunk - 1) / chunk;
+        local += c;
+        lmax = max(lmax, c);
+    }
+    if (lmax > 0) atomicMax(&most, lmax);
     // block exclusive scan of `local`
     const int lane = tid & 31, wid = tid >> 5;
     int x = local;
@@ -86,6 +91,8 @@ __global__ void build_chunk_table_kernel(const int32_t* __restrict__ cu, int B, 
         // nothing: chunk_start[N] written by the owner of the last run
     }
     __syncthreads();
+    // status word 1: the largest number of chunks of one sequence
+    if (tid == 0) status[1] = static_cast<uint32_t>(most);
     const int used = chunk_start[N];
     for (int c = tid; c < maxc; c += nt) {
         if (c >= used) {

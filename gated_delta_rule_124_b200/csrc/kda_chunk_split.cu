@@ -56,6 +56,11 @@ size_t split_blob_bytes() { return BLOB; }
 
 namespace {
 
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) &
+                                      ~static_cast<uintptr_t>(1023));
+}
+
 // ===================================================================== intra
 // Persistent, two CTAs of 256 threads per SM (about 100 KB of shared memory
 // each): every CTA walks the (chunk slot, head) items with a stride of the
@@ -71,8 +76,11 @@ constexpr int NTI = 256;
 constexpr uint32_t OFF_KQ = 0;
 constexpr uint32_t OFF_G = 32768;      // g (TMA) -> G -> A fp32 | T fp32
 constexpr uint32_t OFF_RAP = 65536;    // K * E^-1 (exact path: K * exp(G_last - G))
-constexpr uint32_t OFF_TB = 81920;     // T diag(b) rows 0-63; exact path: A fp32 (16 KB)
-constexpr uint32_t OFF_MID = 90112;    // garbage rows of the Tb operand; inverse scratch
+// T diag(b) rows 0-63, then the garbage rows of its 128-row operand (also the
+// inverse's scratch); before that: the scan's partial results (E1) and, on
+// the exact path, A in fp32 (16 KB).
+constexpr uint32_t OFF_TB = 81920;
+constexpr uint32_t OFF_MID = 90112;
 constexpr uint32_t OFF_BETA = 98304;
 constexpr uint32_t OFF_GM = OFF_BETA + 256;
 constexpr uint32_t OFF_EGM = OFF_GM + 512;
@@ -84,7 +92,7 @@ static_assert(OFF_MID == OFF_TB + 8192, "Tb garbage rows follow Tb");
 static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 constexpr uint32_t TM_X = 0;     // [A ; P] accumulator, 64 columns
 constexpr uint32_t TM_W = 128;   // W accumulator, 128 columns
-constexpr uint32_t TX_KQ = 32768, TX_G = 32768;
+constexpr uint32_t TX_K = 16384, TX_Q = 16384, TX_G = 32768;
 
 struct Params {
     const float* beta;
@@ -94,53 +102,74 @@ struct Params {
     const uint32_t* status;
     uint32_t* status_out;
     uint8_t* blobs;
+    // co-scheduled with the chain kernel only:
+    int N;
+    const int* chunk_start;
+    const uint32_t* rounds;  // largest number of chunks of one sequence
+    uint32_t* flags;         // [slot, head]: set once that blob is complete
 };
 
-__global__ void __launch_bounds__(NTI, 2)
-    chunk_intra_kernel(const __grid_constant__ CUtensorMap tmq,
-                       const __grid_constant__ CUtensorMap tmk,
-                       const __grid_constant__ CUtensorMap tmg, const Params p) {
-    if (status_bad(p.status)) return;
-    const int maxc = p.maxc, nitems = maxc * p.H;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+// One worker (CTA) of the intra-chunk kernel.  Items are (chunk slot, head)
+// pairs taken with a stride of `nworkers`: alone, in slot order; co-scheduled
+// with the chains (kOverlap), round by round -- chunk n of every (sequence,
+// head) before chunk n + 1 of any -- and each finished blob is flagged.
+template <bool kOverlap>
+__device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* tmk,
+                                    const CUtensorMap* tmg, const Params& p, uint8_t* sm,
+                                    int worker, int nworkers) {
+    const int maxc = p.maxc, NH = kOverlap ? p.N * p.H : 1;
+    const int nitems = kOverlap ? static_cast<int>(*p.rounds) * NH : maxc * p.H;
     const uint32_t sbase = smem_u32(sm);
     float* sbeta = reinterpret_cast<float*>(sm + OFF_BETA);
     float* sGm = reinterpret_cast<float*>(sm + OFF_GM);
     float* seGm = reinterpret_cast<float*>(sm + OFF_EGM);
     float* sGL = reinterpret_cast<float*>(sm + OFF_GL);
     float* sWsc = reinterpret_cast<float*>(sm + OFF_WSC);
-    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    uint64_t* bar_g = bar_kq + 1;
-    uint64_t* bar_mma = bar_kq + 2;
+    uint64_t* bar_k = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_q = bar_k + 1;
+    uint64_t* bar_g = bar_k + 2;
+    uint64_t* bar_mma = bar_k + 3;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 32);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, cq = warp >> 2;  // TMEM lanes 32 quarter.., columns 32 cq..
     const int trow = 32 * quarter + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
-    // items whose chunk slot is empty (varlen upper bound) are skipped
+    // item -> (chunk slot, head); items of empty slots (varlen upper bound)
+    // or past the end of a sequence are skipped
+    auto slot_of = [&](int it) {
+        return kOverlap ? p.chunk_start[(it % NH) / p.H] + it / NH : it % maxc;
+    };
+    auto head_of = [&](int it) { return kOverlap ? (it % NH) % p.H : it / maxc; };
+    auto valid = [&](int it) {
+        if (!kOverlap) return p.info[it % maxc].z > 0;
+        const int s = (it % NH) / p.H;
+        return p.chunk_start[s] + it / NH < p.chunk_start[s + 1];
+    };
     auto advance = [&](int it) {
-        while (it < nitems && p.info[it % maxc].z <= 0) it += gridDim.x;
+        while (it < nitems && !valid(it)) it += nworkers;
         return it;
     };
-    auto load_kq = [&](int it) {  // thread 0
-        const int4 c = p.info[it % maxc];
-        const int hh = it / maxc;
-        mbar_arrive_expect_tx(bar_kq, TX_KQ);
-        tma_load_3d(sm + OFF_KQ, &tmk, bar_kq, 0, hh, c.y);
-        tma_load_3d(sm + OFF_KQ + 8192, &tmq, bar_kq, 0, hh, c.y);
-        tma_load_3d(sm + OFF_KQ + 16384, &tmk, bar_kq, 64, hh, c.y);
-        tma_load_3d(sm + OFF_KQ + 24576, &tmq, bar_kq, 64, hh, c.y);
+    // loads of an item's inputs (thread 0), each on its own barrier
+    auto load_k = [&](int it) {
+        const int t0 = p.info[slot_of(it)].y, hh = head_of(it);
+        mbar_arrive_expect_tx(bar_k, TX_K);
+        tma_load_3d(sm + OFF_KQ, tmk, bar_k, 0, hh, t0);
+        tma_load_3d(sm + OFF_KQ + 16384, tmk, bar_k, 64, hh, t0);
     };
-    auto load_g = [&](int it) {  // thread 0
-        const int4 c = p.info[it % maxc];
+    auto load_q = [&](int it) {
+        const int t0 = p.info[slot_of(it)].y, hh = head_of(it);
+        mbar_arrive_expect_tx(bar_q, TX_Q);
+        tma_load_3d(sm + OFF_KQ + 8192, tmq, bar_q, 0, hh, t0);
+        tma_load_3d(sm + OFF_KQ + 24576, tmq, bar_q, 64, hh, t0);
+    };
+    auto load_g = [&](int it) {
         mbar_arrive_expect_tx(bar_g, TX_G);
-        tma_load_3d(sm + OFF_G, &tmg, bar_g, 0, it / maxc, c.y);
+        tma_load_3d(sm + OFF_G, tmg, bar_g, 0, head_of(it), p.info[slot_of(it)].y);
     };
 
     if (tid == 0) {
-        mbar_init(bar_kq, 1);
+        mbar_init(bar_k, 1);
+        mbar_init(bar_q, 1);
         mbar_init(bar_g, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
@@ -155,59 +184,112 @@ __global__ void __launch_bounds__(NTI, 2)
     const uint32_t tbase = *s_tmem;
     bool failed = false;
     uint32_t mma_phase = 0;
-    // loads issued and not yet waited for (thread 0's view; for the exit path)
-    int kq_issued = 0, g_issued = 0;
-    int item = advance(blockIdx.x);
+    // loads issued (thread 0's count; for the exit path)
+    int k_issued = 0, q_issued = 0, g_issued = 0;
+    int item = advance(worker);
+    long long flag_pending = -1;  // (kOverlap) finished blob not yet released
     float beta_next = 0.f;  // (tid < C) this thread's beta of the next item
     auto fetch_beta = [&](int it) {
-        const int4 c = p.info[it % maxc];
-        return tid < c.z ? p.beta[(size_t)(c.y + tid) * p.H + it / maxc] : 0.f;
+        const int4 c = p.info[slot_of(it)];
+        return tid < c.z ? p.beta[(size_t)(c.y + tid) * p.H + head_of(it)] : 0.f;
     };
     if (item < nitems) {
         if (tid == 0) {
-            load_kq(item);
+            load_k(item);
+            load_q(item);
             load_g(item);
-            kq_issued = g_issued = 1;
+            k_issued = q_issued = g_issued = 1;
         }
         if (tid < C) beta_next = fetch_beta(item);
     }
     int n = 0;
     for (; item < nitems && !failed; ++n) {
-        const int4 ci = p.info[item % maxc];
-        const int L = ci.z, h = item / maxc;
-        const int nxt = advance(item + gridDim.x);
-        uint8_t* blob = p.blobs + ((size_t)(item % maxc) * p.H + h) * BLOB;
+        const int slot = slot_of(item), h = head_of(item);
+        const int L = p.info[slot].z;
+        const int nxt = advance(item + nworkers);
+        uint8_t* blob = p.blobs + ((size_t)slot * p.H + h) * BLOB;
         if (tid < C) sbeta[tid] = beta_next;
-        bool ok = mbar_wait(bar_g, n & 1, kWaitNs) && mbar_wait(bar_kq, n & 1, kWaitNs);
+        if (tid == 0) {
+            // the previous item's bulk write-out has read its tiles (and, when
+            // a chain waits for it, has completed)
+            if (kOverlap)
+                bulk_wait_all();
+            else
+                bulk_wait_read();
+        }
+        bool ok = mbar_wait(bar_g, n & 1, kWaitNs) && mbar_wait(bar_k, n & 1, kWaitNs) &&
+                  mbar_wait(bar_q, n & 1, kWaitNs);
         if (__syncthreads_or(!ok)) {
             failed = true;
             break;
         }
-        // -------------------- E1: in-chunk cumulative log-gate, per channel
+        // the previous item's blob is complete (every write of it precedes the
+        // barrier above): release it to its chain.  The last thread does it.
+        if (kOverlap && flag_pending >= 0 && tid == NTI - 1) {
+            fence_proxy_async_global();
+            flag_release(p.flags + flag_pending, 1u);
+        }
+        flag_pending = -1;
+        // ------------- E1: in-chunk cumulative log-gate, per channel.  Thread
+        // (row group grp = 8 rows, channels 4 c4 ..): scan of its 8 rows, then
+        // the totals of the groups above it added; per-channel max / min.
         bool slow_local = false;
-        if (tid < D) {
+        {
             float* g = reinterpret_cast<float*>(sm + OFF_G);
-            const int c = tid;
-            float x[C];
+            float4* tot = reinterpret_cast<float4*>(sm + OFF_TB);           // [8][32]
+            float4* gmx = reinterpret_cast<float4*>(sm + OFF_TB + 4096);    // [8][32]
+            float4* gmn = reinterpret_cast<float4*>(sm + OFF_TB + 8192);    // [8][32]
+            const int c4 = tid & 31, grp = tid >> 5, r0 = 8 * grp;
+            float4 x[8];
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int r = 0; r < C; ++r) x[r] = g[r * D + c];
-            float G = 0.f, gmax = -INFINITY, gmin = INFINITY;
-#pragma unroll
-            for (int r = 0; r < C; ++r) {
-                if (r < L) {
-                    G += x[r];
-                    gmax = fmaxf(gmax, G);
-                    gmin = fminf(gmin, G);
-                }
-                x[r] = G;
+            for (int i = 0; i < 8; ++i) {
+                float4 v = *reinterpret_cast<const float4*>(g + (r0 + i) * D + 4 * c4);
+                if (r0 + i >= L) v = make_float4(0.f, 0.f, 0.f, 0.f);
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                x[i] = acc;
             }
+            tot[grp * 32 + c4] = acc;
+            __syncthreads();
+            float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < grp; ++j) {
+                const float4 t = tot[j * 32 + c4];
+                off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w;
+            }
+            float4 mx = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            float4 mn = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
 #pragma unroll
-            for (int r = 0; r < C; ++r) g[r * D + c] = x[r];
-            const float Gm = gmax - kRef;
-            sGm[c] = Gm;
-            seGm[c] = expf(Gm);
-            sGL[c] = G;
-            slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
+            for (int i = 0; i < 8; ++i) {
+                float4 v = x[i];
+                v.x += off.x; v.y += off.y; v.z += off.z; v.w += off.w;
+                *reinterpret_cast<float4*>(g + (r0 + i) * D + 4 * c4) = v;
+                if (r0 + i < L) {
+                    mx.x = fmaxf(mx.x, v.x); mx.y = fmaxf(mx.y, v.y);
+                    mx.z = fmaxf(mx.z, v.z); mx.w = fmaxf(mx.w, v.w);
+                    mn.x = fminf(mn.x, v.x); mn.y = fminf(mn.y, v.y);
+                    mn.z = fminf(mn.z, v.z); mn.w = fminf(mn.w, v.w);
+                }
+            }
+            gmx[grp * 32 + c4] = mx;
+            gmn[grp * 32 + c4] = mn;
+            __syncthreads();
+            if (tid < D) {
+                const int c = tid;
+                const float* fx = reinterpret_cast<const float*>(gmx);
+                const float* fn = reinterpret_cast<const float*>(gmn);
+                float gmax = -INFINITY, gmin = INFINITY;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    gmax = fmaxf(gmax, fx[j * D + c]);
+                    gmin = fminf(gmin, fn[j * D + c]);
+                }
+                const float Gm = gmax - kRef;
+                const float gl = g[(L - 1) * D + c];
+                sGm[c] = Gm;
+                seGm[c] = expf(Gm);
+                sGL[c] = gl;
+                slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
+            }
         }
         const bool slow = __syncthreads_or(slow_local);
         if (tid < D) {  // row scales of the chain kernel; -W column scale
@@ -254,13 +336,17 @@ __global__ void __launch_bounds__(NTI, 2)
             }
             __syncthreads();
         }
-        // ------------------------------ E2: operand tiles, row-parallel
+        // ------------------------------ E2: operand tiles, row-parallel; each
+        // thread keeps one 8-channel group (j = tid & 15) for all its rows
         {
             const float* G = reinterpret_cast<const float*>(sm + OFF_G);
+            const int j = tid & 15, kb = j >> 3, ch = j & 7, c0 = 8 * j;
+            float m8[8], e8[8];
+            load8(slow ? sGL + c0 : sGm + c0, m8);
+            load8(seGm + c0, e8);
 #pragma unroll
             for (int s = 0; s < (C * 16) / NTI; ++s) {
-                const int it = tid + NTI * s;
-                const int r = it >> 4, j = it & 15, kb = j >> 3, ch = j & 7, c0 = 8 * j;
+                const int r = (tid + NTI * s) >> 4;
                 const uint32_t o64 = sw128_off(r, ch);
                 uint8_t* pk = sm + OFF_KQ + kb * 16384 + o64;
                 uint8_t* pq = pk + 8192;
@@ -271,9 +357,6 @@ __global__ void __launch_bounds__(NTI, 2)
                     unpack8(*reinterpret_cast<const uint4*>(pq), q8);
                     load8(G + r * D + c0, g8);
                     if (!slow) {
-                        float m8[8], e8[8];
-                        load8(sGm + c0, m8);
-                        load8(seGm + c0, e8);
                         // factors within exp(+-80), rounded to bf16 right after
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -284,15 +367,13 @@ __global__ void __launch_bounds__(NTI, 2)
                             rk[i] = k8[i] * Ei;
                             qg[i] = lq[i] * e8[i];
                         }
-                    } else {
-                        float l8[8];
-                        load8(sGL + c0, l8);
+                    } else {  // m8 holds G_last here
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const float gam = expf(g8[i]);
                             lk[i] = k8[i] * gam;  // K * Gam, in place of K
                             lq[i] = 0.f;
-                            rk[i] = k8[i] * expf(l8[i] - g8[i]);
+                            rk[i] = k8[i] * expf(m8[i] - g8[i]);
                             qg[i] = q8[i] * gam;
                         }
                     }
@@ -304,7 +385,6 @@ __global__ void __launch_bounds__(NTI, 2)
                 *reinterpret_cast<uint4*>(pq) = pack8(lq);
                 *reinterpret_cast<uint4*>(sm + OFF_RAP + kb * 8192 + o64) = pack8(rk);
                 *reinterpret_cast<uint4*>(blob + BL_WQ + kb * 16384 + 8192 + o64) = pack8(qg);
-                *reinterpret_cast<uint4*>(blob + BL_RAP + kb * 8192 + o64) = pack8(rk);
             }
         }
         fence_async_smem();
@@ -312,6 +392,14 @@ __global__ void __launch_bounds__(NTI, 2)
         __syncthreads();
         tc_fence_after();
         if (tid < C && nxt < nitems) beta_next = fetch_beta(nxt);
+        if (tid == 0) {
+            bulk_s2g(blob + BL_RAP, sm + OFF_RAP, 16384);  // the chain's K E^-1
+            bulk_commit();
+            if (slow && nxt < nitems) {  // exact path: Q is consumed already
+                load_q(nxt);
+                ++q_issued;
+            }
+        }
         // ------------------------------------------------ A, P (M=128, N=64)
         if (!slow) {
             if (tid == 0) {
@@ -333,6 +421,10 @@ __global__ void __launch_bounds__(NTI, 2)
                 break;
             }
             tc_fence_after();
+            if (tid == 0 && nxt < nitems) {  // the Q * E rows are consumed
+                load_q(nxt);
+                ++q_issued;
+            }
         }
         // ------ A -> fp32 (swizzled, in the G region); P -> bf16, to the blob
         {
@@ -379,12 +471,12 @@ __global__ void __launch_bounds__(NTI, 2)
         __syncthreads();
         // ------------------ UT transform: T = (I + A)^{-1}, blocked 16 x 16
         {
-            const float* Af = reinterpret_cast<const float*>(sm + OFF_G);
+            const float* __restrict__ Af = reinterpret_cast<const float*>(sm + OFF_G);
             float* Tf = reinterpret_cast<float*>(sm + OFF_G + 16384);
             float* Mf = reinterpret_cast<float*>(sm + OFF_MID);
             if (tid < C) {
-                // diagonal blocks, right-looking forward substitution: one
-                // column of one block per thread
+                // diagonal blocks, right-looking forward substitution in
+                // registers: one column of one block per thread
                 const int I = tid >> 4, jj = tid & 15, col = 16 * I + jj;
                 float pv[16];
 #pragma unroll
@@ -392,32 +484,28 @@ __global__ void __launch_bounds__(NTI, 2)
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
                     const float x = pv[rr];
-                    Tf[t_idx(16 * I + rr, col)] = x;
 #pragma unroll
                     for (int r2 = rr + 1; r2 < 16; ++r2)
                         pv[r2] -= Af[a_idx(16 * I + r2, 16 * I + rr)] * x;
                 }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) Tf[t_idx(16 * I + rr, col)] = pv[rr];
             }
             __syncthreads();
             offdiag_level<1>(Af, Tf, Mf, warp, lane);
             offdiag_level<2>(Af, Tf, Mf, warp, lane);
             offdiag_level<3>(Af, Tf, Mf, warp, lane);
-            // Tb = T diag(b) -> bf16, K-major rows of 64 (rows 0-63), in
-            // shared memory for the W product and in the blob for the chain
+            // Tb = T diag(b) -> bf16, K-major rows of 64 (rows 0-63)
             for (int e = tid; e < C * 8; e += NTI) {
                 const int r = e >> 3, ch = e & 7;
                 const float4 t0v = *reinterpret_cast<const float4*>(Tf + t_idx(r, 8 * ch));
                 const float4 t1v = *reinterpret_cast<const float4*>(Tf + t_idx(r, 8 * ch + 4));
                 const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-                float y[8];
+                float b8[8], y[8];
+                load8(sbeta + 8 * ch, b8);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int col = 8 * ch + i;
-                    y[i] = (col <= r) ? tv[i] * sbeta[col] : 0.f;
-                }
-                const uint4 u = pack8(y);
-                *reinterpret_cast<uint4*>(sm + OFF_TB + sw128_off(r, ch)) = u;
-                *reinterpret_cast<uint4*>(blob + BL_TB + sw128_off(r, ch)) = u;
+                for (int i = 0; i < 8; ++i) y[i] = (8 * ch + i <= r) ? tv[i] * b8[i] : 0.f;
+                *reinterpret_cast<uint4*>(sm + OFF_TB + sw128_off(r, ch)) = pack8(y);
             }
         }
         fence_async_smem();
@@ -426,6 +514,8 @@ __global__ void __launch_bounds__(NTI, 2)
         tc_fence_after();
         // ---------------------------------- W = Tb (K*E) [*exp(Gm)]  (N=128)
         if (tid == 0) {
+            bulk_s2g(blob + BL_TB, sm + OFF_TB, 8192);  // the chain's Tb
+            bulk_commit();
             if (nxt < nitems) {  // the G region is free: fetch the next g
                 load_g(nxt);
                 ++g_issued;
@@ -444,9 +534,9 @@ __global__ void __launch_bounds__(NTI, 2)
             break;
         }
         tc_fence_after();
-        if (tid == 0 && nxt < nitems) {  // K, Q region is free: fetch the next K, Q
-            load_kq(nxt);
-            ++kq_issued;
+        if (tid == 0 && nxt < nitems) {  // the K rows are consumed: fetch the next K
+            load_k(nxt);
+            ++k_issued;
         }
         // -W (rows 0-63), column-scaled -> bf16, to the blob's [-W ; Q*Gam]
         if (quarter < 2) {
@@ -469,19 +559,35 @@ __global__ void __launch_bounds__(NTI, 2)
                 }
             }
         }
+        if (kOverlap) flag_pending = static_cast<long long>(slot) * p.H + h;
         item = nxt;
     }
+    if (tid == 0) bulk_wait_all();
     if (failed && tid == 0) {
         // wait (bounded) for this CTA's copies and products still in flight
-        if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
         // (a wait on a phase that has already completed returns at once)
-        if (kq_issued > 0) mbar_wait(bar_kq, (kq_issued - 1) & 1, kWaitNs);
+        if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
+        if (k_issued > 0) mbar_wait(bar_k, (k_issued - 1) & 1, kWaitNs);
+        if (q_issued > 0) mbar_wait(bar_q, (q_issued - 1) & 1, kWaitNs);
         if (g_issued > 0) mbar_wait(bar_g, (g_issued - 1) & 1, kWaitNs);
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
     __syncthreads();
+    if (kOverlap && flag_pending >= 0 && tid == NTI - 1) {
+        fence_proxy_async_global();
+        flag_release(p.flags + flag_pending, 1u);
+    }
     if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
+__global__ void __launch_bounds__(NTI, 2)
+    chunk_intra_kernel(const __grid_constant__ CUtensorMap tmq,
+                       const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmg, const Params p) {
+    if (status_bad(p.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    run<false>(&tmq, &tmk, &tmg, p, align1024(smem_raw), blockIdx.x, gridDim.x);
 }
 }  // namespace intra
 
@@ -523,14 +629,18 @@ struct Params {
     const uint8_t* blobs;
     __nv_bfloat16* o;
     float* hN;
+    const uint32_t* flags;  // co-scheduled with the intra kernel: blob ready flags
 };
 
-__global__ void __launch_bounds__(NTC, 2)
-    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
-    if (status_bad(p.status)) return;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+// One chain CTA: (sequence, head) `chain_id`, value columns [64 half, +64).
+// Each chunk's loads come in three groups, issued as soon as their regions
+// are free (1: row scales; 2: Tb, V, [-W ; Q*Gam]; 3: K E^-1, P).  When
+// co-scheduled with the intra kernel (kOverlap) a chunk's groups wait for its
+// blob's flag: polled at each issue point, waited for (bounded) only when the
+// chunk is next.
+template <bool kOverlap>
+__device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uint8_t* sm,
+                                    int chain_id, int half) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_ld + 1;
@@ -539,7 +649,7 @@ __global__ void __launch_bounds__(NTC, 2)
     const int quarter = warp & 3, cq = warp >> 2;  // rows 32 quarter + lane, columns 32 cq ..
     const int trow = 32 * quarter + (tid & 31);
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
-    const int chain_id = blockIdx.x >> 1, half = blockIdx.x & 1, j0 = DVS * half;
+    const int j0 = DVS * half;
     const int seq = chain_id / p.H, h = chain_id % p.H;
     const int t_begin = p.cu ? p.cu[seq] : seq * p.T;
     const int t_end = p.cu ? p.cu[seq + 1] : (seq + 1) * p.T;
@@ -561,16 +671,72 @@ __global__ void __launch_bounds__(NTC, 2)
     const uint32_t tbase = *s_tmem;
     bool failed = false;
     uint32_t mma_phase = 0;
+    // thread 0: load groups of the coming chunk not issued yet, whether its
+    // transaction count is registered, whether its blob was seen ready
+    int pend = 0, coming = 0;
+    bool armed = false, rdy = false;
+    uint32_t polled = 0;  // value of the last flag poll (issued, used one gate later)
+    const uint32_t* flag0 = kOverlap ? p.flags + (size_t)cbase * p.H + h : nullptr;
+    auto issue = [&](int n, int groups) {
+        const uint8_t* b = blob(n);
+        if (groups & 1) bulk_g2s(sm + ((n & 1) ? OFF_SC1 : OFF_SC0), b + BL_SC, 1024, bar_ld);
+        if (groups & 2) {
+            bulk_g2s(sm + OFF_TB, b + BL_TB, 8192, bar_ld);
+            tma_load_3d(sm + OFF_V, tmv, bar_ld, j0, h, t_begin + n * C);
+            bulk_g2s(sm + OFF_WQ, b + BL_WQ, 32768, bar_ld);
+        }
+        if (groups & 4) {
+            bulk_g2s(sm + OFF_RAP, b + BL_RAP, 16384, bar_ld);
+            bulk_g2s(sm + OFF_PM, b + BL_PM, 8192, bar_ld);
+        }
+    };
+    auto issue_ready = [&](int n, int groups) {  // thread 0
+        groups &= pend;
+        if (!groups) return;
+        if (!armed) {
+            mbar_arrive_expect_tx(bar_ld, TX_BYTES);
+            armed = true;
+        }
+        issue(n, groups);
+        pend &= ~groups;
+    };
+    // gate(): check the poll issued at the previous gate (its value has
+    // arrived by now), issue another if the blob is not ready yet
+    auto gate = [&](int n, int groups) {  // thread 0: non-blocking
+        if (kOverlap && !rdy) {
+            if (polled == 0u) {
+                polled = flag_poll(flag0 + (size_t)n * p.H);
+                return;
+            }
+            rdy = true;
+            flag_acquire_fence();
+            fence_proxy_async_global();
+        }
+        issue_ready(n, groups);
+    };
+    auto gate_wait = [&](int n) -> bool {  // thread 0: bounded wait, then all groups
+        if (kOverlap && !rdy) {
+            const uint64_t t0 = global_timer_ns();
+            while (polled == 0u) {
+                polled = flag_poll(flag0 + (size_t)n * p.H);
+                if (polled != 0u) break;
+                if (status_bad(p.status) || global_timer_ns() - t0 > kWaitNs) return false;
+                __nanosleep(128);
+            }
+            rdy = true;
+            flag_acquire_fence();
+            fence_proxy_async_global();
+        }
+        issue_ready(n, 7);
+        return true;
+    };
 
     if (tid == 0 && t_begin < t_end) {
-        const uint8_t* b0 = blob(0);
-        mbar_arrive_expect_tx(bar_ld, TX_BYTES);
-        bulk_g2s(sm + OFF_SC0, b0 + BL_SC, 1024, bar_ld);
-        bulk_g2s(sm + OFF_TB, b0 + BL_TB, 8192, bar_ld);
-        tma_load_3d(sm + OFF_V, &tmv, bar_ld, j0, h, t_begin);
-        bulk_g2s(sm + OFF_WQ, b0 + BL_WQ, 32768, bar_ld);
-        bulk_g2s(sm + OFF_RAP, b0 + BL_RAP, 16384, bar_ld);
-        bulk_g2s(sm + OFF_PM, b0 + BL_PM, 8192, bar_ld);
+        pend = 7;
+        if (kOverlap)
+            polled = flag_poll(flag0);
+        else
+            gate(0, 7);
     }
     // ---- initial state (this half): fp32 into TMEM (row c = lane), bf16 into Sb
     {
@@ -610,14 +776,21 @@ __global__ void __launch_bounds__(NTC, 2)
         const int tn = t0 + C;
         const bool has_next = tn < t_end;
         const float* ssc = reinterpret_cast<const float*>(sm + ((n & 1) ? OFF_SC1 : OFF_SC0));
-        bool ok = mbar_wait(bar_ld, n & 1, kWaitNs);
+        bool ok = true;
+        if (tid == 0 && pend) ok = gate_wait(n);
+        ok = ok && mbar_wait(bar_ld, n & 1, kWaitNs);
         if (__syncthreads_or(!ok)) {
             failed = true;
             break;
         }
-        if (has_next && tid == 0) {
-            mbar_arrive_expect_tx(bar_ld, TX_BYTES);
-            bulk_g2s(sm + ((n & 1) ? OFF_SC0 : OFF_SC1), blob(n + 1) + BL_SC, 1024, bar_ld);
+        if (has_next && tid == 0) {  // the other row-scale buffer is free
+            pend = 7;
+            coming = n + 1;
+            armed = rdy = false;
+            if (kOverlap)
+                polled = flag_poll(flag0 + (size_t)(n + 1) * p.H);  // checked at the next gate
+            else
+                gate(n + 1, 1);
         }
         // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
         if (tid == 0) {
@@ -641,11 +814,7 @@ __global__ void __launch_bounds__(NTC, 2)
             break;
         }
         tc_fence_after();
-        if (has_next && tid == 0) {  // V, Tb and [-W ; Q*Gam] regions are free
-            bulk_g2s(sm + OFF_TB, blob(n + 1) + BL_TB, 8192, bar_ld);
-            tma_load_3d(sm + OFF_V, &tmv, bar_ld, j0, h, tn);
-            bulk_g2s(sm + OFF_WQ, blob(n + 1) + BL_WQ, 32768, bar_ld);
-        }
+        if (has_next && tid == 0) gate(n + 1, 3);  // V, Tb, [-W ; Q*Gam] regions free
         // U (rows 0-63 of the accumulator) -> bf16 Ub
         if (quarter < 2) {
             const int r = trow;
@@ -685,10 +854,7 @@ __global__ void __launch_bounds__(NTC, 2)
             break;
         }
         tc_fence_after();
-        if (has_next && tid == 0) {  // K E^-1 and P regions are free
-            bulk_g2s(sm + OFF_RAP, blob(n + 1) + BL_RAP, 16384, bar_ld);
-            bulk_g2s(sm + OFF_PM, blob(n + 1) + BL_PM, 8192, bar_ld);
-        }
+        if (has_next && tid == 0) gate(n + 1, 7);  // K E^-1 and P regions free
         // S <- Gam_last * S + ksc * (K E^-1)^T U   (lane = state row c); O rows out
         {
             const int c = trow;
@@ -746,15 +912,48 @@ __global__ void __launch_bounds__(NTC, 2)
                             __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
     }
     if (failed && tid == 0) {
+        // wait (bounded) for products and copies still in flight
         if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
-        mbar_wait(bar_ld, n & 1, kWaitNs);
+        if (armed) mbar_wait(bar_ld, coming & 1, kWaitNs);  // at once if complete
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 256);
 }
+
+__global__ void __launch_bounds__(NTC, 2)
+    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
+    if (status_bad(p.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    run<false>(&tmv, p, align1024(smem_raw), blockIdx.x >> 1, blockIdx.x & 1);
+}
 }  // namespace chain
+
+// =================================================================== overlap
+// Both kernels in one cooperative launch (every CTA resident, two per SM): the
+// first 2 N H CTAs run the chains, the others the intra-chunk work round by
+// round.  A chain waits only for the blobs of its own chunks and an intra
+// worker never waits for a chain, so every wait ends (each is also bounded).
+static_assert(intra::NTI == chain::NTC, "one block size");
+constexpr uint32_t OVERLAP_SMEM =
+    intra::SMEM_BYTES > chain::SMEM_BYTES ? intra::SMEM_BYTES : chain::SMEM_BYTES;
+
+__global__ void __launch_bounds__(intra::NTI, 2)
+    chunk_overlap_kernel(const __grid_constant__ CUtensorMap tmq,
+                         const __grid_constant__ CUtensorMap tmk,
+                         const __grid_constant__ CUtensorMap tmg,
+                         const __grid_constant__ CUtensorMap tmv, const intra::Params pi,
+                         const chain::Params pc, int nchain) {
+    if (status_bad(pi.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    const int b = static_cast<int>(blockIdx.x);
+    if (b < nchain)
+        chain::run<true>(&tmv, pc, sm, b >> 1, b & 1);
+    else
+        intra::run<true>(&tmq, &tmk, &tmg, pi, sm, b - nchain, static_cast<int>(gridDim.x) - nchain);
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 split_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -834,6 +1033,68 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
                      static_cast<const uint8_t*>(blobs), (__nv_bfloat16*)o, hN};
     chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
     return cudaGetLastError();
+}
+
+// Grid of the co-scheduled launch, or 0 when it does not apply: the device
+// must keep two such CTAs per SM resident and support cooperative launches,
+// and the chains may take at most half of the CTAs.
+int overlap_grid(int N, int H) {
+    int dev = 0, sms = 0, nb = 0, coop = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(chunk_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)OVERLAP_SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, chunk_overlap_kernel, intra::NTI,
+                                                      OVERLAP_SMEM) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (!coop || nb < 2 || sms <= 0) return 0;
+    if (2LL * N * H > sms) return 0;
+    return 2 * sms;
+}
+
+cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v, const float* g,
+                                     const float* beta, const float* h0,
+                                     const int32_t* cu_seqlens, int T, int N, int H,
+                                     const int4* chunk_info, int maxc, const int* chunk_start,
+                                     uint32_t* status, void* blobs, uint32_t* flags, void* o,
+                                     float* hN, cudaStream_t st) {
+    const int total = cu_seqlens ? T : N * T;
+    if (total == 0)
+        return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN,
+                                  st);
+    const int grid = overlap_grid(N, H);
+    if (grid == 0) return cudaErrorInvalidConfiguration;
+    CUtensorMap mq, mk, mg, mv;
+    if (!split_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(flags, 0, sizeof(uint32_t) * (size_t)maxc * H, st);
+    if (e != cudaSuccess) return e;
+    uint8_t* bl = static_cast<uint8_t*>(blobs);
+    const intra::Params pi{beta, chunk_info, maxc, H, status, status, bl,
+                           N, chunk_start, status + 1, flags};
+    const chain::Params pc{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
+                           (__nv_bfloat16*)o, hN, flags};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(intra::NTI);
+    cfg.dynamicSmemBytes = OVERLAP_SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chunk_overlap_kernel, mq, mk, mg, mv, pi, pc, 2 * N * H);
 }
 
 cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,

@@ -33,5 +33,15 @@ cudaError_t launch_split_intra(const void* q, const void* k, const float* g, con
 cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
                                int N, int H, const int* chunk_start, uint32_t* status,
                                const void* blobs, void* o, float* hN, cudaStream_t st);
+// The two kernels co-scheduled in one cooperative launch (chains wait for the
+// blobs of their chunks through `flags`, one uint32 per (chunk slot, head)).
+// overlap_grid() is its grid size, or 0 when the launch does not apply.
+int overlap_grid(int N, int H);
+cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v, const float* g,
+                                     const float* beta, const float* h0,
+                                     const int32_t* cu_seqlens, int T, int N, int H,
+                                     const int4* chunk_info, int maxc, const int* chunk_start,
+                                     uint32_t* status, void* blobs, uint32_t* flags, void* o,
+                                     float* hN, cudaStream_t st);
 
 }  // namespace kda

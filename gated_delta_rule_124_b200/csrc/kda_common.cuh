@@ -11,13 +11,16 @@ namespace kda {
 
 // ---------------------------------------------------------------- workspace
 // Layout of the caller's workspace (all offsets 256-byte aligned):
-//   [0, 256)              status word (uint32 at offset 0) + padding
+//   [0, 256)              status word (uint32 at offset 0); at offset 4 the
+//                         largest number of chunks of one sequence (written
+//                         by the chunk-table kernel); padding
 //   chunk_start[N + 1]    int32: global index of each sequence's first chunk
 //   chunk_info[maxc]      int4 {seq, first token, rows, chunk-in-sequence};
 //                         unused slots hold seq = -1, rows = 0
 //   then, for the CUDA-core path only: G, W, U (token-major fp32) and the
 //   per-chunk states [maxc, H, dk, dv] fp32; for the split tensor-core path
-//   only: one operand blob per (chunk slot, head).
+//   only: one operand blob per (chunk slot, head), then one uint32 ready flag
+//   per (chunk slot, head).
 constexpr size_t kAlign = 256;
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a = kAlign) {
@@ -36,6 +39,7 @@ struct Workspace {
     float* U;
     float* states;
     uint8_t* blobs;
+    uint32_t* flags;
     size_t header_bytes;  // status + tables
     size_t total_bytes;   // header + CUDA-core path intermediates
 };
@@ -72,6 +76,8 @@ inline Workspace carve(void* base, int total, int N, int H, int dk, int dv, int 
         off = align_up(off, 1024);
         w.blobs = reinterpret_cast<uint8_t*>(p + off);
         off = align_up(off + blob_bytes * (size_t)maxc * H);
+        w.flags = reinterpret_cast<uint32_t*>(p + off);
+        off = align_up(off + sizeof(uint32_t) * (size_t)maxc * H);
     }
     w.total_bytes = off;
     return w;

@@ -103,6 +103,32 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's generic-proxy global accesses with its async-proxy
+// (bulk copy / TMA) accesses to global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------------- flags between CTAs (gpu scope)
+// Publish: every earlier write of this thread, and the writes of the threads
+// of its CTA that reached a __syncthreads() before this call, become visible
+// at gpu scope before the flag does.
+__device__ __forceinline__ void flag_release(uint32_t* flag, uint32_t v) {
+    asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(v)
+                 : "memory");
+}
+// Poll without ordering (the thread stalls only where it uses the value);
+// after seeing the flag set, flag_acquire_fence() orders every later read of
+// this thread after the writes the flag published.
+__device__ __forceinline__ uint32_t flag_poll(const uint32_t* flag) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v;
+}
+__device__ __forceinline__ void flag_acquire_fence() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // -------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

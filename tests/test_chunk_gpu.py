@@ -257,23 +257,61 @@ def chunk_path(request, monkeypatch):
     return request.param
 
 
-@pytest.mark.parametrize("chunk_path", ["fused", "split", "simt"], indirect=True)
+@pytest.mark.parametrize("chunk_path", ["fused", "split", "overlap", "simt"], indirect=True)
 @pytest.mark.parametrize("name", sorted(PATH_CASES))
 def test_every_path_matches_oracle(chunk_path, name):
     case = PATH_CASES[name]()
     check_case(case)
 
 
-@pytest.mark.parametrize("chunk_path", ["fused", "split"], indirect=True)
+@pytest.mark.parametrize("chunk_path", ["fused", "split", "overlap"], indirect=True)
 def test_tc_paths_mixed_fast_and_exact_chunks(chunk_path):
     case = wl.make_prefill(306, [64 * 4 + 10], H=2, dk=128, dv=128, chunk=64, dtype="bf16")
     case.g[64:128] *= 6.0
     check_case(case)
 
 
+@pytest.mark.parametrize("lengths", [[640, 333], [64 * 40, 1, 64 * 7 + 5, 0, 200]])
+def test_overlap_and_split_identical(monkeypatch, lengths):
+    """The co-scheduled launch runs the same device code as the two-launch
+    split, only interleaved: identical bits."""
+    case = wl.make_prefill(310, lengths, H=3, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
+    o1, h1 = run_fwd(case)
+    monkeypatch.setenv("KDA_CHUNK_PATH", "overlap")
+    o2, h2 = run_fwd(case)
+    assert torch.equal(o1, o2) and torch.equal(h1, h2)
+
+
+def test_overlap_repeated_calls_same_workspace(monkeypatch):
+    """Ready flags are reset by every call: back-to-back calls on one
+    workspace give identical results."""
+    monkeypatch.setenv("KDA_CHUNK_PATH", "overlap")
+    case = wl.make_prefill(311, [500, 64 * 9], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    c = case.to("cuda")
+    ws = kda.alloc_workspace(c.total, c.N, c.H, 128, 128, 64, "bf16")
+    outs = []
+    for _ in range(3):
+        o = torch.empty_like(c.v)
+        hN = torch.empty(c.N, c.H, 128, 128, device="cuda")
+        kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, 1,
+                          c.total, c.N, c.H, 128, 128, 64, "bf16", o, hN, ws)
+        outs.append((o, hN))
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    for o, hN in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(hN, outs[0][1])
+    ro, rh = oracle_prefill(case)
+    assert rel_err(outs[0][0], ro) <= tol_for("bf16")
+
+
 def test_split_and_fused_agree_closely(monkeypatch):
-    """The two tensor-core paths run the same arithmetic in the same order:
-    their results agree to a few bf16 ulps of o."""
+    """The two tensor-core paths use the same factorisation and operand
+    layouts; only the in-chunk cumulative sum of g is taken in a different
+    order (sequential in the fused kernel, two-level in the split one), so an
+    operand can round to the neighbouring bf16 value.  Their results agree far
+    inside the oracle tolerance."""
     case = wl.make_prefill(307, [640, 333], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
                            varlen=True)
     monkeypatch.setenv("KDA_CHUNK_PATH", "fused")
@@ -282,7 +320,7 @@ def test_split_and_fused_agree_closely(monkeypatch):
     o2, h2 = run_fwd(case)
     torch.cuda.synchronize()
     assert rel_err(o2, o1.double().cpu().numpy()) <= 1e-2
-    assert rel_err(h2, h1.double().cpu().numpy()) <= 1e-5
+    assert rel_err(h2, h1.double().cpu().numpy()) <= 2e-3
 
 
 def test_split_step_calls_compose(monkeypatch):
