@@ -297,23 +297,10 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
-def prefill_path(Np, H, dk, dv, C, dtype="bf16"):
-    """Which prefill kernels kda_chunk_fwd runs (the library's rule, see
-    include/kda.h): 'fused' (one tensor-core kernel), 'split' (chunk-parallel
-    intra kernel + per-chain kernel), 'overlap' (the two co-scheduled in one
-    launch) or 'simt' (CUDA-core kernels)."""
-    import torch
-    env = os.environ.get("KDA_CHUNK_PATH")
-    if env == "simt" or not (dtype == "bf16" and dk == dv == 128 and C == 64):
-        return "simt"
-    if env in ("fused", "split"):
-        return env
-    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    if 2 * Np * H <= sms:
-        return "overlap"
-    if env == "overlap":
-        return "split"
-    return "split" if Np * H < 2 * sms else "fused"
+def prefill_path(kda, total, Np, H, dk, dv, C, packed, dtype="bf16"):
+    """The plan kda_chunk_fwd runs for this problem (the library's own answer):
+    'simt', 'fused', 'split' or 'overlap' (see include/kda.h)."""
+    return kda.PLAN_NAMES[kda.kda_chunk_fwd_plan(total, Np, H, dk, dv, C, dtype, packed)]
 
 
 def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
@@ -326,7 +313,7 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     must move; the split plan's hand-over through the workspace is overhead."""
     import torch
     Np, H, dk, dv, C, total = P.N, P.H, P.dk, P.dv, P.chunk, P.total
-    path = prefill_path(Np, H, dk, dv, C)
+    path = prefill_path(kda, total, Np, H, dk, dv, C, P.cu_seqlens is not None)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     in_b = 2
     tx = total * H

@@ -49,23 +49,29 @@ kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, 
 // Which kernels kda_chunk_fwd runs.
 enum class Path { Simt, Fused, Split, Overlap };
 
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        return 148;
-    }
-    return n;
+// Whether co-scheduling the two split kernels pays: the chains get one SM per
+// unit (2 N H SMs) and the intra-chunk items the rest, against the two kernels
+// back to back on every SM.  Cost model in units of one chain step, from
+// B200 measurements: an intra-chunk item costs about 4.8 chain steps of one
+// unit, and two intra units share an SM.  Needs the chain length, so only
+// when every sequence has the same length (B x T, or one packed sequence).
+bool overlap_pays(long long items, long long rounds, long long NH, int sms) {
+    const double rho = 4.8;
+    const double intra_split = items * rho / (2.0 * sms);
+    const double intra_ov = items * rho / (2.0 * (sms - 2 * NH));
+    const double chain = static_cast<double>(rounds);
+    return (intra_ov > chain ? intra_ov : chain) <= 0.85 * (intra_split + chain);
 }
 
-// bf16, dk = dv = 128, chunk 64 runs on the tensor cores.  With few (sequence,
-// head) chains (2 N H <= SMs) the chunk-parallel intra-chunk kernel and the
-// per-chain kernel run co-scheduled in one launch; with somewhat more
-// (N H < 2 SMs) as two launches; otherwise one kernel with one CTA per
-// (sequence, head).  KDA_CHUNK_PATH = fused | split | overlap | simt forces a
-// path (testing); overlap falls back to split where it does not apply.
-Path select_path(int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
+// bf16, dk = dv = 128, chunk 64 runs on the tensor cores as the split plan:
+// the chunk-parallel intra-chunk kernel and the per-chain kernel, co-scheduled
+// in one launch on disjoint SMs where overlap_pays(), else as two launches.
+// The single fused kernel (one CTA per (sequence, head)) is slower on every
+// measured shape and runs only when forced.  KDA_CHUNK_PATH = fused | split |
+// overlap | simt forces a plan (testing); overlap falls back to split where
+// the launch does not apply.
+Path select_path(int total, int N, bool packed, int H, int dk, int dv, int chunk,
+                 kda_dtype_t dt) {
     const bool tc_shape = dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
                           kda::tc_path_available();
     const char* env = getenv("KDA_CHUNK_PATH");
@@ -73,10 +79,13 @@ Path select_path(int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
     if (!tc_shape) return Path::Simt;
     if (env && !strcmp(env, "fused")) return Path::Fused;
     if (env && !strcmp(env, "split")) return Path::Split;
-    const bool overlap = kda::overlap_grid(N, H) > 0;
-    if (env && !strcmp(env, "overlap")) return overlap ? Path::Overlap : Path::Split;
-    if (overlap) return Path::Overlap;
-    return ((long long)N * H < 2LL * sm_count()) ? Path::Split : Path::Fused;
+    const int sms = kda::overlap_grid(N, H);
+    if (sms == 0) return Path::Split;
+    if (env && !strcmp(env, "overlap")) return Path::Overlap;
+    if (packed && N > 1) return Path::Split;
+    const long long rounds = ((long long)total / N + chunk - 1) / chunk;
+    const long long items = rounds * N * H;
+    return overlap_pays(items, rounds, (long long)N * H, sms) ? Path::Overlap : Path::Split;
 }
 
 Workspace carve_for(void* base, const Prefill& p, int H, int dk, int dv, int chunk, Path path) {
@@ -86,8 +95,10 @@ Workspace carve_for(void* base, const Prefill& p, int H, int dk, int dv, int chu
 }
 
 size_t workspace_bytes_for(int total, int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
+    // the split and co-scheduled plans share one layout, so packing does not matter
     const Prefill p{total, N};
-    return carve_for(nullptr, p, H, dk, dv, chunk, select_path(N, H, dk, dv, chunk, dt))
+    return carve_for(nullptr, p, H, dk, dv, chunk,
+                     select_path(total, N, false, H, dk, dv, chunk, dt))
         .total_bytes;
 }
 
@@ -136,6 +147,20 @@ int kda_num_chunks_upper_bound(int total_tokens, int num_seqs, int chunk) {
     return kda::max_chunks(total_tokens, num_seqs, chunk);
 }
 
+int kda_chunk_fwd_plan(int total_tokens, int num_seqs, int packed, int H, int dk, int dv,
+                       int chunk, kda_dtype_t dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
+        !chunk_ok(chunk) || !dtype_ok(dtype))
+        return -1;
+    switch (select_path(total_tokens, num_seqs, packed != 0, H, dk, dv, chunk, dtype)) {
+        case Path::Simt: return KDA_PLAN_SIMT;
+        case Path::Fused: return KDA_PLAN_FUSED;
+        case Path::Split: return KDA_PLAN_SPLIT;
+        case Path::Overlap: return KDA_PLAN_OVERLAP;
+    }
+    return -1;
+}
+
 size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
                                     int chunk, kda_dtype_t dtype) {
     if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
@@ -159,7 +184,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
         if (!aligned16(ptr)) return KDA_ERR_INVALID_ARG;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_INVALID_ARG;
-    const Path path = select_path(p.N, H, dk, dv, chunk, dtype);
+    const Path path = select_path(p.total, p.N, cu_seqlens != nullptr, H, dk, dv, chunk, dtype);
     Workspace w;
     s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, path, &w);
     if (s != KDA_OK) return s;

@@ -113,10 +113,12 @@ struct Params {
 // pairs taken with a stride of `nworkers`: alone, in slot order; co-scheduled
 // with the chains (kOverlap), round by round -- chunk n of every (sequence,
 // head) before chunk n + 1 of any -- and each finished blob is flagged.
+// The unit is a group of NTI threads (a whole CTA, or half of one) that
+// synchronises on named barrier `bar`; `tbase` is its 256 TMEM columns.
 template <bool kOverlap>
 __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* tmk,
                                     const CUtensorMap* tmg, const Params& p, uint8_t* sm,
-                                    int worker, int nworkers) {
+                                    uint32_t tbase, uint32_t bar, int worker, int nworkers) {
     const int maxc = p.maxc, NH = kOverlap ? p.N * p.H : 1;
     const int nitems = kOverlap ? static_cast<int>(*p.rounds) * NH : maxc * p.H;
     const uint32_t sbase = smem_u32(sm);
@@ -129,8 +131,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     uint64_t* bar_q = bar_k + 1;
     uint64_t* bar_g = bar_k + 2;
     uint64_t* bar_mma = bar_k + 3;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 32);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x & (NTI - 1), warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, cq = warp >> 2;  // TMEM lanes 32 quarter.., columns 32 cq..
     const int trow = 32 * quarter + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
@@ -149,22 +150,37 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         while (it < nitems && !valid(it)) it += nworkers;
         return it;
     };
+    // everything the loop needs of an item, fetched (global loads) one item
+    // ahead of its use: {item, chunk slot, head, rows, first token}
+    struct Item {
+        int it, slot, h, L, t0;
+    };
+    auto describe = [&](int it) {
+        Item d{it, 0, 0, 0, 0};
+        if (it < nitems) {
+            d.slot = slot_of(it);
+            d.h = head_of(it);
+            const int4 c = p.info[d.slot];
+            d.L = c.z;
+            d.t0 = c.y;
+        }
+        return d;
+    };
+    int* s_ahead = reinterpret_cast<int*>(sm + OFF_BAR + 32);  // the item after the next
     // loads of an item's inputs (thread 0), each on its own barrier
-    auto load_k = [&](int it) {
-        const int t0 = p.info[slot_of(it)].y, hh = head_of(it);
+    auto load_k = [&](const Item& d) {
         mbar_arrive_expect_tx(bar_k, TX_K);
-        tma_load_3d(sm + OFF_KQ, tmk, bar_k, 0, hh, t0);
-        tma_load_3d(sm + OFF_KQ + 16384, tmk, bar_k, 64, hh, t0);
+        tma_load_3d(sm + OFF_KQ, tmk, bar_k, 0, d.h, d.t0);
+        tma_load_3d(sm + OFF_KQ + 16384, tmk, bar_k, 64, d.h, d.t0);
     };
-    auto load_q = [&](int it) {
-        const int t0 = p.info[slot_of(it)].y, hh = head_of(it);
+    auto load_q = [&](const Item& d) {
         mbar_arrive_expect_tx(bar_q, TX_Q);
-        tma_load_3d(sm + OFF_KQ + 8192, tmq, bar_q, 0, hh, t0);
-        tma_load_3d(sm + OFF_KQ + 24576, tmq, bar_q, 64, hh, t0);
+        tma_load_3d(sm + OFF_KQ + 8192, tmq, bar_q, 0, d.h, d.t0);
+        tma_load_3d(sm + OFF_KQ + 24576, tmq, bar_q, 64, d.h, d.t0);
     };
-    auto load_g = [&](int it) {
+    auto load_g = [&](const Item& d) {
         mbar_arrive_expect_tx(bar_g, TX_G);
-        tma_load_3d(sm + OFF_G, tmg, bar_g, 0, head_of(it), p.info[slot_of(it)].y);
+        tma_load_3d(sm + OFF_G, tmg, bar_g, 0, d.h, d.t0);
     };
 
     if (tid == 0) {
@@ -174,39 +190,33 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
-    if (warp == 0) {
-        tmem_alloc(s_tmem, 256);
-        tmem_relinquish();
-    }
     tc_fence_before();
-    __syncthreads();
+    group_sync(bar, NTI);
     tc_fence_after();
-    const uint32_t tbase = *s_tmem;
     bool failed = false;
     uint32_t mma_phase = 0;
     // loads issued (thread 0's count; for the exit path)
     int k_issued = 0, q_issued = 0, g_issued = 0;
-    int item = advance(worker);
+    Item cur = describe(advance(worker));
+    Item nxt = describe(cur.it < nitems ? advance(cur.it + nworkers) : nitems);
     long long flag_pending = -1;  // (kOverlap) finished blob not yet released
     float beta_next = 0.f;  // (tid < C) this thread's beta of the next item
-    auto fetch_beta = [&](int it) {
-        const int4 c = p.info[slot_of(it)];
-        return tid < c.z ? p.beta[(size_t)(c.y + tid) * p.H + head_of(it)] : 0.f;
+    auto fetch_beta = [&](const Item& d) {
+        return tid < d.L ? p.beta[(size_t)(d.t0 + tid) * p.H + d.h] : 0.f;
     };
-    if (item < nitems) {
+    if (cur.it < nitems) {
         if (tid == 0) {
-            load_k(item);
-            load_q(item);
-            load_g(item);
+            load_k(cur);
+            load_q(cur);
+            load_g(cur);
             k_issued = q_issued = g_issued = 1;
         }
-        if (tid < C) beta_next = fetch_beta(item);
+        if (tid < C) beta_next = fetch_beta(cur);
     }
     int n = 0;
-    for (; item < nitems && !failed; ++n) {
-        const int slot = slot_of(item), h = head_of(item);
-        const int L = p.info[slot].z;
-        const int nxt = advance(item + nworkers);
+    for (; cur.it < nitems && !failed; ++n) {
+        const int slot = cur.slot, h = cur.h, L = cur.L;
+        const bool more = nxt.it < nitems;
         uint8_t* blob = p.blobs + ((size_t)slot * p.H + h) * BLOB;
         if (tid < C) sbeta[tid] = beta_next;
         if (tid == 0) {
@@ -219,7 +229,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         }
         bool ok = mbar_wait(bar_g, n & 1, kWaitNs) && mbar_wait(bar_k, n & 1, kWaitNs) &&
                   mbar_wait(bar_q, n & 1, kWaitNs);
-        if (__syncthreads_or(!ok)) {
+        if (group_sync_or(bar, NTI, !ok)) {
             failed = true;
             break;
         }
@@ -250,7 +260,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 x[i] = acc;
             }
             tot[grp * 32 + c4] = acc;
-            __syncthreads();
+            group_sync(bar, NTI);
             float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < grp; ++j) {
                 const float4 t = tot[j * 32 + c4];
@@ -272,7 +282,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             }
             gmx[grp * 32 + c4] = mx;
             gmn[grp * 32 + c4] = mn;
-            __syncthreads();
+            group_sync(bar, NTI);
             if (tid < D) {
                 const int c = tid;
                 const float* fx = reinterpret_cast<const float*>(gmx);
@@ -291,7 +301,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
             }
         }
-        const bool slow = __syncthreads_or(slow_local);
+        const bool slow = group_sync_or(bar, NTI, slow_local);
         if (tid < D) {  // row scales of the chain kernel; -W column scale
             const float gl = sGL[tid];
             sWsc[tid] = slow ? -1.f : -seGm[tid];
@@ -334,7 +344,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 }
                 *reinterpret_cast<uint4*>(blob + BL_PM + sw128_off(r, task & 7)) = pack8(pp);
             }
-            __syncthreads();
+            group_sync(bar, NTI);
         }
         // ------------------------------ E2: operand tiles, row-parallel; each
         // thread keeps one 8-channel group (j = tid & 15) for all its rows
@@ -389,13 +399,13 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        group_sync(bar, NTI);
         tc_fence_after();
-        if (tid < C && nxt < nitems) beta_next = fetch_beta(nxt);
+        if (tid < C && more) beta_next = fetch_beta(nxt);
         if (tid == 0) {
             bulk_s2g(blob + BL_RAP, sm + OFF_RAP, 16384);  // the chain's K E^-1
             bulk_commit();
-            if (slow && nxt < nitems) {  // exact path: Q is consumed already
+            if (slow && more) {  // exact path: Q is consumed already
                 load_q(nxt);
                 ++q_issued;
             }
@@ -416,12 +426,12 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             }
             ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
             ++mma_phase;
-            if (__syncthreads_or(!ok)) {
+            if (group_sync_or(bar, NTI, !ok)) {
                 failed = true;
                 break;
             }
             tc_fence_after();
-            if (tid == 0 && nxt < nitems) {  // the Q * E rows are consumed
+            if (tid == 0 && more) {  // the Q * E rows are consumed
                 load_q(nxt);
                 ++q_issued;
             }
@@ -468,12 +478,20 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 for (int i = tid; i < C * C / 4; i += NTI) dstA[i] = srcA[i];
             }
         }
-        __syncthreads();
+        group_sync(bar, NTI);
         // ------------------ UT transform: T = (I + A)^{-1}, blocked 16 x 16
         {
             const float* __restrict__ Af = reinterpret_cast<const float*>(sm + OFF_G);
             float* Tf = reinterpret_cast<float*>(sm + OFF_G + 16384);
             float* Mf = reinterpret_cast<float*>(sm + OFF_MID);
+            if (tid == NTI - 32) {  // idle here: look up the item after the next
+                const Item d = describe(more ? advance(nxt.it + nworkers) : nitems);
+                s_ahead[0] = d.it;
+                s_ahead[1] = d.slot;
+                s_ahead[2] = d.h;
+                s_ahead[3] = d.L;
+                s_ahead[4] = d.t0;
+            }
             if (tid < C) {
                 // diagonal blocks, right-looking forward substitution in
                 // registers: one column of one block per thread
@@ -491,10 +509,10 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) Tf[t_idx(16 * I + rr, col)] = pv[rr];
             }
-            __syncthreads();
-            offdiag_level<1>(Af, Tf, Mf, warp, lane);
-            offdiag_level<2>(Af, Tf, Mf, warp, lane);
-            offdiag_level<3>(Af, Tf, Mf, warp, lane);
+            group_sync(bar, NTI);
+            offdiag_level<1>(Af, Tf, Mf, warp, lane, bar, NTI);
+            offdiag_level<2>(Af, Tf, Mf, warp, lane, bar, NTI);
+            offdiag_level<3>(Af, Tf, Mf, warp, lane, bar, NTI);
             // Tb = T diag(b) -> bf16, K-major rows of 64 (rows 0-63)
             for (int e = tid; e < C * 8; e += NTI) {
                 const int r = e >> 3, ch = e & 7;
@@ -510,13 +528,13 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        group_sync(bar, NTI);
         tc_fence_after();
         // ---------------------------------- W = Tb (K*E) [*exp(Gm)]  (N=128)
         if (tid == 0) {
             bulk_s2g(blob + BL_TB, sm + OFF_TB, 8192);  // the chain's Tb
             bulk_commit();
-            if (nxt < nitems) {  // the G region is free: fetch the next g
+            if (more) {  // the G region is free: fetch the next g
                 load_g(nxt);
                 ++g_issued;
             }
@@ -529,12 +547,12 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         }
         ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
         ++mma_phase;
-        if (__syncthreads_or(!ok)) {
+        if (group_sync_or(bar, NTI, !ok)) {
             failed = true;
             break;
         }
         tc_fence_after();
-        if (tid == 0 && nxt < nitems) {  // the K rows are consumed: fetch the next K
+        if (tid == 0 && more) {  // the K rows are consumed: fetch the next K
             load_k(nxt);
             ++k_issued;
         }
@@ -560,7 +578,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             }
         }
         if (kOverlap) flag_pending = static_cast<long long>(slot) * p.H + h;
-        item = nxt;
+        cur = nxt;
+        nxt = Item{s_ahead[0], s_ahead[1], s_ahead[2], s_ahead[3], s_ahead[4]};
     }
     if (tid == 0) bulk_wait_all();
     if (failed && tid == 0) {
@@ -573,12 +592,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
-    __syncthreads();
+    group_sync(bar, NTI);
     if (kOverlap && flag_pending >= 0 && tid == NTI - 1) {
         fence_proxy_async_global();
         flag_release(p.flags + flag_pending, 1u);
     }
-    if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
 __global__ void __launch_bounds__(NTI, 2)
@@ -587,7 +605,18 @@ __global__ void __launch_bounds__(NTI, 2)
                        const __grid_constant__ CUtensorMap tmg, const Params p) {
     if (status_bad(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
-    run<false>(&tmq, &tmk, &tmg, p, align1024(smem_raw), blockIdx.x, gridDim.x);
+    __shared__ uint32_t s_tmem;
+    if (threadIdx.x < 32) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    run<false>(&tmq, &tmk, &tmg, p, align1024(smem_raw), s_tmem, 1, blockIdx.x, gridDim.x);
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
 }
 }  // namespace intra
 
@@ -636,16 +665,18 @@ struct Params {
 // Each chunk's loads come in three groups, issued as soon as their regions
 // are free (1: row scales; 2: Tb, V, [-W ; Q*Gam]; 3: K E^-1, P).  When
 // co-scheduled with the intra kernel (kOverlap) a chunk's groups wait for its
-// blob's flag: polled at each issue point, waited for (bounded) only when the
-// chunk is next.
+// blob's flag: read (acquire) while the products of the current chunk run,
+// checked at each issue point, waited for (bounded) only when the chunk is
+// next.
+// The unit is a group of NTC threads synchronising on named barrier `bar`;
+// `tbase` is its 256 TMEM columns.
 template <bool kOverlap>
 __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uint8_t* sm,
-                                    int chain_id, int half) {
+                                    uint32_t tbase, uint32_t bar, int chain_id, int half) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_ld + 1;
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 16);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x & (NTC - 1), warp = tid >> 5;
     const int quarter = warp & 3, cq = warp >> 2;  // rows 32 quarter + lane, columns 32 cq ..
     const int trow = 32 * quarter + (tid & 31);
     const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
@@ -661,21 +692,16 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
-    if (warp == 0) {
-        tmem_alloc(s_tmem, 256);
-        tmem_relinquish();
-    }
     tc_fence_before();
-    __syncthreads();
+    group_sync(bar, NTC);
     tc_fence_after();
-    const uint32_t tbase = *s_tmem;
     bool failed = false;
     uint32_t mma_phase = 0;
     // thread 0: load groups of the coming chunk not issued yet, whether its
     // transaction count is registered, whether its blob was seen ready
     int pend = 0, coming = 0;
     bool armed = false, rdy = false;
-    uint32_t polled = 0;  // value of the last flag poll (issued, used one gate later)
+    uint32_t polled = 0;  // value of the last flag read (issued before an MMA wait)
     const uint32_t* flag0 = kOverlap ? p.flags + (size_t)cbase * p.H + h : nullptr;
     auto issue = [&](int n, int groups) {
         const uint8_t* b = blob(n);
@@ -700,16 +726,16 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         issue(n, groups);
         pend &= ~groups;
     };
-    // gate(): check the poll issued at the previous gate (its value has
-    // arrived by now), issue another if the blob is not ready yet
+    // read the coming chunk's flag (thread 0, just before an MMA wait, which
+    // hides the read's latency)
+    auto poll = [&](int n) {
+        if (kOverlap && !rdy) polled = flag_acquire(flag0 + (size_t)n * p.H);
+    };
+    // gate(): issue `groups` of chunk n if the last read saw its blob ready
     auto gate = [&](int n, int groups) {  // thread 0: non-blocking
         if (kOverlap && !rdy) {
-            if (polled == 0u) {
-                polled = flag_poll(flag0 + (size_t)n * p.H);
-                return;
-            }
+            if (polled == 0u) return;
             rdy = true;
-            flag_acquire_fence();
             fence_proxy_async_global();
         }
         issue_ready(n, groups);
@@ -718,13 +744,12 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         if (kOverlap && !rdy) {
             const uint64_t t0 = global_timer_ns();
             while (polled == 0u) {
-                polled = flag_poll(flag0 + (size_t)n * p.H);
+                polled = flag_acquire(flag0 + (size_t)n * p.H);
                 if (polled != 0u) break;
                 if (status_bad(p.status) || global_timer_ns() - t0 > kWaitNs) return false;
                 __nanosleep(128);
             }
             rdy = true;
-            flag_acquire_fence();
             fence_proxy_async_global();
         }
         issue_ready(n, 7);
@@ -734,7 +759,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     if (tid == 0 && t_begin < t_end) {
         pend = 7;
         if (kOverlap)
-            polled = flag_poll(flag0);
+            polled = flag_acquire(flag0);
         else
             gate(0, 7);
     }
@@ -767,7 +792,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         reinterpret_cast<uint4*>(sm + OFF_ZERO)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    group_sync(bar, NTC);
     tc_fence_after();
 
     int n = 0;
@@ -779,7 +804,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         bool ok = true;
         if (tid == 0 && pend) ok = gate_wait(n);
         ok = ok && mbar_wait(bar_ld, n & 1, kWaitNs);
-        if (__syncthreads_or(!ok)) {
+        if (group_sync_or(bar, NTC, !ok)) {
             failed = true;
             break;
         }
@@ -787,10 +812,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
             pend = 7;
             coming = n + 1;
             armed = rdy = false;
-            if (kOverlap)
-                polled = flag_poll(flag0 + (size_t)(n + 1) * p.H);  // checked at the next gate
-            else
-                gate(n + 1, 1);
+            polled = 0u;
+            gate(n + 1, 1);  // (co-scheduled: not yet read; issued at a later gate)
         }
         // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
         if (tid == 0) {
@@ -806,10 +829,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
                          sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id, 1);
             }
             mma_commit(bar_mma);
+            if (has_next) poll(n + 1);
         }
         ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
         ++mma_phase;
-        if (__syncthreads_or(!ok)) {
+        if (group_sync_or(bar, NTC, !ok)) {
             failed = true;
             break;
         }
@@ -831,7 +855,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        group_sync(bar, NTC);
         tc_fence_after();
         // ---- O = X[64:] + [. ; P] U  (accumulate);  (K E^-1)^T U -> TM_W   (N=64)
         if (tid == 0) {
@@ -846,10 +870,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
                 mma_bf16(tbase + TM_W, sdesc_sw128(sbase + OFF_RAP + ks * 2048, 8192, 1024),
                          sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idK, ks > 0);
             mma_commit(bar_mma);
+            if (has_next) poll(n + 1);
         }
         ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
         ++mma_phase;
-        if (__syncthreads_or(!ok)) {
+        if (group_sync_or(bar, NTC, !ok)) {
             failed = true;
             break;
         }
@@ -895,7 +920,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        group_sync(bar, NTC);
         tc_fence_after();
     }
 
@@ -918,28 +943,50 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 256);
+    group_sync(bar, NTC);
 }
 
 __global__ void __launch_bounds__(NTC, 2)
     chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
     if (status_bad(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
-    run<false>(&tmv, p, align1024(smem_raw), blockIdx.x >> 1, blockIdx.x & 1);
+    __shared__ uint32_t s_tmem;
+    if (threadIdx.x < 32) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    run<false>(&tmv, p, align1024(smem_raw), s_tmem, 1, blockIdx.x >> 1, blockIdx.x & 1);
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
 }
 }  // namespace chain
 
 // =================================================================== overlap
-// Both kernels in one cooperative launch (every CTA resident, two per SM): the
-// first 2 N H CTAs run the chains, the others the intra-chunk work round by
-// round.  A chain waits only for the blobs of its own chunks and an intra
-// worker never waits for a chain, so every wait ends (each is also bounded).
-static_assert(intra::NTI == chain::NTC, "one block size");
-constexpr uint32_t OVERLAP_SMEM =
-    intra::SMEM_BYTES > chain::SMEM_BYTES ? intra::SMEM_BYTES : chain::SMEM_BYTES;
+// Both kernels in one cooperative launch of one 512-thread CTA per SM; each
+// CTA is two independent 256-thread units (named barriers 1 and 2, 256 TMEM
+// columns and one shared-memory region each).  The first 2 N H CTAs run one
+// chain unit each (one value-column half of one (sequence, head)) with the
+// SM to itself -- a chain step is a short dependent sequence of products and
+// epilogues that slows down by more than half when another unit shares its
+// SM -- and the others run two intra-chunk units each, round by round.  A
+// chain waits only for the blobs of its own chunks and an intra unit never
+// waits for a chain; every CTA is resident (cooperative launch), so every
+// wait ends (each is also bounded).
+constexpr int NTO = 512;
+static_assert(intra::NTI == 256 && chain::NTC == 256, "two 256-thread units per CTA");
+constexpr uint32_t unit_bytes() {
+    const uint32_t a = intra::OFF_BAR + 64, b = chain::OFF_BAR + 64;
+    return ((a > b ? a : b) + 1023) / 1024 * 1024;
+}
+constexpr uint32_t UNIT_BYTES = unit_bytes();
+constexpr uint32_t OVERLAP_SMEM = 2 * UNIT_BYTES + 1024;
+static_assert(OVERLAP_SMEM + 1024 <= 232448, "one CTA per SM");
 
-__global__ void __launch_bounds__(intra::NTI, 2)
+__global__ void __launch_bounds__(NTO, 1)
     chunk_overlap_kernel(const __grid_constant__ CUtensorMap tmq,
                          const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmg,
@@ -947,12 +994,26 @@ __global__ void __launch_bounds__(intra::NTI, 2)
                          const chain::Params pc, int nchain) {
     if (status_bad(pi.status)) return;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = align1024(smem_raw);
+    __shared__ uint32_t s_tmem;
+    if (threadIdx.x < 32) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int unit = static_cast<int>(threadIdx.x) >> 8;
+    uint8_t* sm = align1024(smem_raw) + unit * UNIT_BYTES;
+    const uint32_t tb = s_tmem + 256u * unit;
     const int b = static_cast<int>(blockIdx.x);
-    if (b < nchain)
-        chain::run<true>(&tmv, pc, sm, b >> 1, b & 1);
-    else
-        intra::run<true>(&tmq, &tmk, &tmg, pi, sm, b - nchain, static_cast<int>(gridDim.x) - nchain);
+    if (b < nchain) {
+        if (unit == 0) chain::run<true>(&tmv, pc, sm, tb, 1, b >> 1, b & 1);
+    } else
+        intra::run<true>(&tmq, &tmk, &tmg, pi, sm, tb, 1 + unit, 2 * (b - nchain) + unit,
+                         2 * (static_cast<int>(gridDim.x) - nchain));
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(s_tmem, 512);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 split_encode_fn() {
@@ -1035,9 +1096,10 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
     return cudaGetLastError();
 }
 
-// Grid of the co-scheduled launch, or 0 when it does not apply: the device
-// must keep two such CTAs per SM resident and support cooperative launches,
-// and the chains may take at most half of the CTAs.
+// Grid of the co-scheduled launch (one CTA per SM), or 0 when it does not
+// apply: the device must support cooperative launches and keep one such CTA
+// per SM resident, and at least one SM must be left for the intra-chunk work
+// after one SM per chain unit.
 int overlap_grid(int N, int H) {
     int dev = 0, sms = 0, nb = 0, coop = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -1045,14 +1107,17 @@ int overlap_grid(int N, int H) {
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
         cudaFuncSetAttribute(chunk_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)OVERLAP_SMEM) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, chunk_overlap_kernel, intra::NTI,
+        cudaFuncSetAttribute(chunk_overlap_kernel,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, chunk_overlap_kernel, NTO,
                                                       OVERLAP_SMEM) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
-    if (!coop || nb < 2 || sms <= 0) return 0;
-    if (2LL * N * H > sms) return 0;
-    return 2 * sms;
+    if (!coop || nb < 1 || sms <= 0) return 0;
+    if (2LL * N * H >= sms) return 0;
+    return sms;
 }
 
 cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v, const float* g,
@@ -1086,7 +1151,7 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
                            (__nv_bfloat16*)o, hN, flags};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(intra::NTI);
+    cfg.blockDim = dim3(NTO);
     cfg.dynamicSmemBytes = OVERLAP_SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

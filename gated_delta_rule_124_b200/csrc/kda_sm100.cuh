@@ -109,6 +109,26 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// -------------------------------------------- named barriers (thread groups)
+// A CTA may run independent groups of `n` threads (warps [first, first + n/32)),
+// each synchronising on its own barrier `id` (1..15; 0 is __syncthreads).
+__device__ __forceinline__ void group_sync(uint32_t id, uint32_t n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Barrier over the group that also returns whether `pred` held in any thread.
+__device__ __forceinline__ bool group_sync_or(uint32_t id, uint32_t n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------- flags between CTAs (gpu scope)
 // Publish: every earlier write of this thread, and the writes of the threads
 // of its CTA that reached a __syncthreads() before this call, become visible
@@ -117,16 +137,12 @@ __device__ __forceinline__ void flag_release(uint32_t* flag, uint32_t v) {
     asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(v)
                  : "memory");
 }
-// Poll without ordering (the thread stalls only where it uses the value);
-// after seeing the flag set, flag_acquire_fence() orders every later read of
-// this thread after the writes the flag published.
-__device__ __forceinline__ uint32_t flag_poll(const uint32_t* flag) {
+// Acquire read: every later memory access of this thread is ordered after
+// the writes that the flag published (and waits for this load to complete).
+__device__ __forceinline__ uint32_t flag_acquire(const uint32_t* flag) {
     uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     return v;
-}
-__device__ __forceinline__ void flag_acquire_fence() {
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
 // -------------------------------------------------------------------- tcgen05

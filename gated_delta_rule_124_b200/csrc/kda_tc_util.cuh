@@ -73,9 +73,12 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
 // one warp per block J.  Fragments (m16n8k8, tf32): lane = 4 g + t;
 // A: (g, t), (g+8, t), (g, t+4), (g+8, t+4); B: (t, g), (t+4, g);
 // C: (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+// Ends with a barrier over the thread group: `bar_id` 0 = the whole CTA,
+// otherwise named barrier `bar_id` over `nthreads` threads.
 template <int DIST>
 __device__ __forceinline__ void offdiag_level(const float* Af, float* Tf, float* Ms, int warp,
-                                              int lane) {
+                                              int lane, uint32_t bar_id = 0,
+                                              uint32_t nthreads = 0) {
     constexpr int NB = 4 - DIST;
     if (warp < NB) {
         const int J = warp, I = J + DIST, g = lane >> 2, t = lane & 3;
@@ -132,7 +135,10 @@ __device__ __forceinline__ void offdiag_level(const float* Af, float* Tf, float*
             Tf[t_idx(16 * I + g + 8, col + 1)] = -out[nt][3];
         }
     }
-    __syncthreads();
+    if (bar_id == 0)
+        __syncthreads();
+    else
+        sm100::group_sync(bar_id, nthreads);
 }
 
 }  // namespace tc

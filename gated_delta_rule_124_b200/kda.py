@@ -39,7 +39,7 @@ EXPORTS = (
     "kda_num_chunks_upper_bound", "kda_chunk_gate_cumsum", "kda_chunk_intra",
     "kda_chunk_inter", "kda_chunk_output", "kda_decode_step", "kda_get_device_status",
     "kda_chunk_fwd_noalloc", "kda_chunk_split_workspace_size", "kda_chunk_split_intra",
-    "kda_chunk_split_chain",
+    "kda_chunk_split_chain", "kda_chunk_fwd_plan",
 )
 
 
@@ -66,6 +66,7 @@ _SIGS = {
     "kda_get_device_status": ([_vp, _vp], _i),
     "kda_chunk_fwd_noalloc": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp], _i),
     "kda_chunk_split_workspace_size": ([_i, _i, _i], _sz),
+    "kda_chunk_fwd_plan": ([_i] * 8, _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
@@ -140,6 +141,16 @@ def _nbytes(t) -> int:
 def kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype) -> int:
     return int(load().kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk,
                                                    dtype_code(dtype)))
+
+
+KDA_PLAN_SIMT, KDA_PLAN_FUSED, KDA_PLAN_SPLIT, KDA_PLAN_OVERLAP = 0, 1, 2, 3
+PLAN_NAMES = {KDA_PLAN_SIMT: "simt", KDA_PLAN_FUSED: "fused", KDA_PLAN_SPLIT: "split",
+              KDA_PLAN_OVERLAP: "overlap"}
+
+
+def kda_chunk_fwd_plan(total_tokens, num_seqs, H, dk, dv, chunk, dtype, packed=False) -> int:
+    return int(load().kda_chunk_fwd_plan(total_tokens, num_seqs, int(bool(packed)), H, dk, dv,
+                                         chunk, dtype_code(dtype)))
 
 
 def kda_num_chunks_upper_bound(total_tokens, num_seqs, chunk) -> int:

@@ -83,22 +83,45 @@ const char* kda_status_string(kda_status_t status);
  *      256-byte aligned, owned by the caller, reusable across calls on the same
  *      stream; it also holds the device status word.
  * Shapes: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}; anything else is
- *      KDA_ERR_UNSUPPORTED.  bf16 with dk = dv = 128 and chunk = 64 runs on the
- *      tensor cores (tcgen05 / TMEM / TMA), in one of two plans:
- *        fused -- one kernel, one CTA per (sequence, head) walking its chunks;
- *        split -- kda_chunk_split_intra then kda_chunk_split_chain (below),
- *                 for problems with too few (sequence, head) pairs to fill
- *                 the GPU.
- *      split is taken when num_seqs * H < 2 * (number of SMs), fused
- *      otherwise.  Other supported shapes run the CUDA-core kernels (the four
- *      step calls below, in order).  The environment variable KDA_CHUNK_PATH =
- *      fused | split | simt forces one plan (testing; shapes without the
- *      tensor-core plans always run the CUDA-core kernels).
- *      kda_chunk_fwd_workspace_size() follows the same choice, so read the
- *      environment before sizing the workspace, not between the two calls.
+ *      KDA_ERR_UNSUPPORTED.  Which kernels run is the call's plan (see
+ *      kda_chunk_fwd_plan below): bf16 with dk = dv = 128 and chunk = 64 runs
+ *      on the tensor cores (tcgen05 / TMEM / TMA) as the split plan, other
+ *      supported shapes on the CUDA-core kernels (the four step calls below,
+ *      in order).  kda_chunk_fwd_workspace_size() follows the plan.
  */
 size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
                                     int chunk, kda_dtype_t dtype);
+
+/* Plans of kda_chunk_fwd (which kernels one call runs):
+ *   KDA_PLAN_SIMT     the CUDA-core kernels: gate cumsum, intra, inter, output;
+ *   KDA_PLAN_FUSED    one tensor-core kernel, one CTA per (sequence, head)
+ *                     walking its chunks (runs only when forced, see below);
+ *   KDA_PLAN_SPLIT    kda_chunk_split_intra then kda_chunk_split_chain (below):
+ *                     the chunk-parallel part on every SM, then the chains;
+ *   KDA_PLAN_OVERLAP  the same two kernels co-scheduled in one cooperative
+ *                     launch, chains and intra-chunk work on disjoint SMs,
+ *                     each chain starting on a chunk as soon as that chunk's
+ *                     operands are ready.  Taken when the chain length is known
+ *                     on the host (no cu_seqlens, or a single packed sequence),
+ *                     2 * num_seqs * H is below the number of SMs, and a cost
+ *                     model says that the chains, not the intra-chunk work,
+ *                     are the longer part (long sequences, few heads).
+ * kda_chunk_fwd_plan returns the plan for these arguments on the current
+ * device (`packed` != 0: the call passes cu_seqlens), or -1 for arguments
+ * kda_chunk_fwd_workspace_size() rejects.  The split and overlap plans share
+ * one workspace layout.  The environment variable KDA_CHUNK_PATH = fused |
+ * split | overlap | simt forces a plan (testing; shapes without the
+ * tensor-core plans always run SIMT, and overlap falls back to split where the
+ * launch does not apply); it is read by every call, so set it before sizing
+ * the workspace, not between the two calls. */
+enum {
+    KDA_PLAN_SIMT = 0,
+    KDA_PLAN_FUSED = 1,
+    KDA_PLAN_SPLIT = 2,
+    KDA_PLAN_OVERLAP = 3
+};
+int kda_chunk_fwd_plan(int total_tokens, int num_seqs, int packed, int H, int dk, int dv,
+                       int chunk, kda_dtype_t dtype);
 
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, const float* initial_state,

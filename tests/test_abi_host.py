@@ -122,6 +122,17 @@ def test_step_calls_reject_bad_arguments(lib):
                                 dv=96, dtype="f32", o=FAKE, **common) == kda.KDA_ERR_UNSUPPORTED
 
 
+def test_plan_query(lib):
+    f = kda.kda_chunk_fwd_plan
+    assert f(4096, 2, 32, 128, 128, 64, "bf16") in (kda.KDA_PLAN_SIMT, kda.KDA_PLAN_SPLIT,
+                                                   kda.KDA_PLAN_OVERLAP)
+    assert f(64, 1, 1, 32, 32, 16, "f32") == kda.KDA_PLAN_SIMT   # no tensor-core plan
+    assert f(64, 3, 1, 32, 32, 16, "f32", packed=True) == kda.KDA_PLAN_SIMT
+    assert f(64, 1, 1, 48, 32, 16, "f32") == -1
+    assert f(64, 0, 1, 32, 32, 16, "f32") == -1
+    assert f(-1, 1, 1, 32, 32, 16, "f32") == -1
+
+
 def test_split_calls_reject_bad_arguments(lib):
     f = kda.kda_chunk_split_workspace_size
     assert f(4096, 2, 32) > 0

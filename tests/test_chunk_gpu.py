@@ -257,10 +257,18 @@ def chunk_path(request, monkeypatch):
     return request.param
 
 
+def assert_plan(case, name):
+    """The forced plan is the one the library reports for this problem."""
+    plan = kda.kda_chunk_fwd_plan(case.total, case.N, case.H, case.dk, case.dv, case.chunk,
+                                  case.dtype, packed=case.cu_seqlens is not None)
+    assert kda.PLAN_NAMES[plan] == name, (kda.PLAN_NAMES[plan], name)
+
+
 @pytest.mark.parametrize("chunk_path", ["fused", "split", "overlap", "simt"], indirect=True)
 @pytest.mark.parametrize("name", sorted(PATH_CASES))
 def test_every_path_matches_oracle(chunk_path, name):
     case = PATH_CASES[name]()
+    assert_plan(case, chunk_path)
     check_case(case)
 
 
@@ -268,6 +276,7 @@ def test_every_path_matches_oracle(chunk_path, name):
 def test_tc_paths_mixed_fast_and_exact_chunks(chunk_path):
     case = wl.make_prefill(306, [64 * 4 + 10], H=2, dk=128, dv=128, chunk=64, dtype="bf16")
     case.g[64:128] *= 6.0
+    assert_plan(case, chunk_path)
     check_case(case)
 
 
@@ -280,6 +289,7 @@ def test_overlap_and_split_identical(monkeypatch, lengths):
     monkeypatch.setenv("KDA_CHUNK_PATH", "split")
     o1, h1 = run_fwd(case)
     monkeypatch.setenv("KDA_CHUNK_PATH", "overlap")
+    assert_plan(case, "overlap")
     o2, h2 = run_fwd(case)
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
 
@@ -290,6 +300,7 @@ def test_overlap_repeated_calls_same_workspace(monkeypatch):
     monkeypatch.setenv("KDA_CHUNK_PATH", "overlap")
     case = wl.make_prefill(311, [500, 64 * 9], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
                            varlen=True)
+    assert_plan(case, "overlap")
     c = case.to("cuda")
     ws = kda.alloc_workspace(c.total, c.N, c.H, 128, 128, 64, "bf16")
     outs = []
@@ -304,6 +315,20 @@ def test_overlap_repeated_calls_same_workspace(monkeypatch):
         assert torch.equal(o, outs[0][0]) and torch.equal(hN, outs[0][1])
     ro, rh = oracle_prefill(case)
     assert rel_err(outs[0][0], ro) <= tol_for("bf16")
+
+
+def test_default_plans(monkeypatch):
+    """Without an override: long chains over few heads -> overlap; short
+    chains, many chains, or packed sequences of unknown length -> split."""
+    monkeypatch.delenv("KDA_CHUNK_PATH", raising=False)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    f = kda.kda_chunk_fwd_plan
+    assert f(65536, 1, 32, 128, 128, 64, "bf16") == kda.KDA_PLAN_OVERLAP
+    assert f(65536, 1, 32, 128, 128, 64, "bf16", packed=True) == kda.KDA_PLAN_OVERLAP
+    assert f(65536, 2, 16, 128, 128, 64, "bf16", packed=True) == kda.KDA_PLAN_SPLIT
+    assert f(4096, 2, 32, 128, 128, 64, "bf16") == kda.KDA_PLAN_SPLIT
+    assert f(4096 * sms, sms, 32, 128, 128, 64, "bf16") == kda.KDA_PLAN_SPLIT
+    assert f(4096, 2, 32, 128, 128, 64, "f32") == kda.KDA_PLAN_SIMT
 
 
 def test_split_and_fused_agree_closely(monkeypatch):
