@@ -227,19 +227,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             else
                 bulk_wait_read();
         }
-        bool ok = mbar_wait(bar_g, n & 1, kWaitNs) && mbar_wait(bar_k, n & 1, kWaitNs) &&
-                  mbar_wait(bar_q, n & 1, kWaitNs);
+        bool ok = mbar_wait(bar_g, n & 1, kWaitNs);  // K, Q: after E1
         if (group_sync_or(bar, NTI, !ok)) {
             failed = true;
             break;
         }
-        // the previous item's blob is complete (every write of it precedes the
-        // barrier above): release it to its chain.  The last thread does it.
-        if (kOverlap && flag_pending >= 0 && tid == NTI - 1) {
-            fence_proxy_async_global();
-            flag_release(p.flags + flag_pending, 1u);
-        }
-        flag_pending = -1;
         // ------------- E1: in-chunk cumulative log-gate, per channel.  Thread
         // (row group grp = 8 rows, channels 4 c4 ..): scan of its 8 rows, then
         // the totals of the groups above it added; per-channel max / min.
@@ -300,6 +292,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 sGL[c] = gl;
                 slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
             }
+        }
+        ok = mbar_wait(bar_k, n & 1, kWaitNs) && mbar_wait(bar_q, n & 1, kWaitNs);
+        if (group_sync_or(bar, NTI, !ok)) {
+            failed = true;
+            break;
         }
         const bool slow = group_sync_or(bar, NTI, slow_local);
         if (tid < D) {  // row scales of the chain kernel; -W column scale
@@ -484,7 +481,14 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             const float* __restrict__ Af = reinterpret_cast<const float*>(sm + OFF_G);
             float* Tf = reinterpret_cast<float*>(sm + OFF_G + 16384);
             float* Mf = reinterpret_cast<float*>(sm + OFF_MID);
-            if (tid == NTI - 32) {  // idle here: look up the item after the next
+            if (tid == NTI - 32) {  // idle in this phase
+                // the previous item's blob is complete (all of its writes came
+                // before this item's first barrier): release it to its chain
+                if (kOverlap && flag_pending >= 0) {
+                    fence_proxy_async_global();
+                    flag_release(p.flags + flag_pending, 1u);
+                }
+                // look up the item after the next
                 const Item d = describe(more ? advance(nxt.it + nworkers) : nitems);
                 s_ahead[0] = d.it;
                 s_ahead[1] = d.slot;
@@ -593,7 +597,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     }
     tc_fence_before();
     group_sync(bar, NTI);
-    if (kOverlap && flag_pending >= 0 && tid == NTI - 1) {
+    if (kOverlap && flag_pending >= 0 && tid == NTI - 32) {
         fence_proxy_async_global();
         flag_release(p.flags + flag_pending, 1u);
     }
@@ -638,14 +642,23 @@ constexpr uint32_t OFF_UB = 98304;     // U bf16 [token][64], MN-major
 constexpr uint32_t OFF_SC0 = 106496;   // exp(G_last), row scale: two buffers of 1 KB
 constexpr uint32_t OFF_SC1 = 107520;
 constexpr uint32_t OFF_BAR = 108544;
+// (co-scheduled) number of leading chunks whose blobs are ready, or -1 if the
+// wait for one gave up; written by the watcher thread, read by thread 0
+constexpr uint32_t OFF_RDY = OFF_BAR + 32;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_ZERO == OFF_TB + 8192, "Tb zero rows");
 static_assert(OFF_PM == OFF_RAP + 16384, "P garbage rows");
 static_assert(2 * SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
 constexpr uint32_t TM_W = 0;     // (K E^-1)^T U   [128 x 64]
-constexpr uint32_t TM_X = 64;    // [Ut ; 0] + [-W ; Q*Gam] S = [U ; Q*Gam S], then O
+// [Ut ; 0] + [-W ; Q*Gam] S = [U ; Q*Gam S], then O in rows 64-127; two
+// buffers (even / odd chunks), so that a chunk's O is read out while the next
+// chunk's first products run
+constexpr uint32_t TM_X = 64;
 constexpr uint32_t TM_S = 128;   // fp32 state [128 x 64]
-constexpr uint32_t TX_BYTES = 1024 + 8192 + 8192 + 32768 + 16384 + 8192;
+constexpr uint32_t TM_X1 = 192;
+// loads of one chunk: groups 1 and 2 on one barrier, group 3 (needed only by
+// the second round of products) on another
+constexpr uint32_t TX_A = 1024 + 8192 + 8192 + 32768, TX_B = 16384 + 8192;
 
 struct Params {
     const float* h0;
@@ -664,10 +677,10 @@ struct Params {
 // One chain CTA: (sequence, head) `chain_id`, value columns [64 half, +64).
 // Each chunk's loads come in three groups, issued as soon as their regions
 // are free (1: row scales; 2: Tb, V, [-W ; Q*Gam]; 3: K E^-1, P).  When
-// co-scheduled with the intra kernel (kOverlap) a chunk's groups wait for its
-// blob's flag: read (acquire) while the products of the current chunk run,
-// checked at each issue point, waited for (bounded) only when the chunk is
-// next.
+// co-scheduled with the intra kernel (kOverlap) a chunk's groups wait until
+// the watcher (another thread of the CTA, below) has seen that chunk's blob
+// flag: checked at each issue point, waited for (bounded) only when the chunk
+// is next.
 // The unit is a group of NTC threads synchronising on named barrier `bar`;
 // `tbase` is its 256 TMEM columns.
 template <bool kOverlap>
@@ -676,6 +689,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_ld + 1;
+    uint64_t* bar_ld3 = bar_ld + 2;
     const int tid = threadIdx.x & (NTC - 1), warp = tid >> 5;
     const int quarter = warp & 3, cq = warp >> 2;  // rows 32 quarter + lane, columns 32 cq ..
     const int trow = 32 * quarter + (tid & 31);
@@ -686,9 +700,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     const int t_end = p.cu ? p.cu[seq + 1] : (seq + 1) * p.T;
     const int cbase = p.chunk_start[seq];
     auto blob = [&](int n) { return p.blobs + ((size_t)(cbase + n) * p.H + h) * BLOB; };
+    auto tx = [](int n) { return (n & 1) ? TM_X1 : TM_X; };
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
+        mbar_init(bar_ld3, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
@@ -700,9 +716,9 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     // thread 0: load groups of the coming chunk not issued yet, whether its
     // transaction count is registered, whether its blob was seen ready
     int pend = 0, coming = 0;
-    bool armed = false, rdy = false;
-    uint32_t polled = 0;  // value of the last flag read (issued before an MMA wait)
-    const uint32_t* flag0 = kOverlap ? p.flags + (size_t)cbase * p.H + h : nullptr;
+    int ld3_chunk = -1;  // chunk whose group 3 is in flight and not yet waited for
+    bool armed = false, armed3 = false, rdy = false;
+    const int* s_rdy = reinterpret_cast<const int*>(sm + OFF_RDY);
     auto issue = [&](int n, int groups) {
         const uint8_t* b = blob(n);
         if (groups & 1) bulk_g2s(sm + ((n & 1) ? OFF_SC1 : OFF_SC0), b + BL_SC, 1024, bar_ld);
@@ -712,29 +728,29 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
             bulk_g2s(sm + OFF_WQ, b + BL_WQ, 32768, bar_ld);
         }
         if (groups & 4) {
-            bulk_g2s(sm + OFF_RAP, b + BL_RAP, 16384, bar_ld);
-            bulk_g2s(sm + OFF_PM, b + BL_PM, 8192, bar_ld);
+            bulk_g2s(sm + OFF_RAP, b + BL_RAP, 16384, bar_ld3);
+            bulk_g2s(sm + OFF_PM, b + BL_PM, 8192, bar_ld3);
+            ld3_chunk = n;
         }
     };
     auto issue_ready = [&](int n, int groups) {  // thread 0
         groups &= pend;
         if (!groups) return;
-        if (!armed) {
-            mbar_arrive_expect_tx(bar_ld, TX_BYTES);
+        if ((groups & 3) && !armed) {
+            mbar_arrive_expect_tx(bar_ld, TX_A);
             armed = true;
+        }
+        if ((groups & 4) && !armed3) {
+            mbar_arrive_expect_tx(bar_ld3, TX_B);
+            armed3 = true;
         }
         issue(n, groups);
         pend &= ~groups;
     };
-    // read the coming chunk's flag (thread 0, just before an MMA wait, which
-    // hides the read's latency)
-    auto poll = [&](int n) {
-        if (kOverlap && !rdy) polled = flag_acquire(flag0 + (size_t)n * p.H);
-    };
-    // gate(): issue `groups` of chunk n if the last read saw its blob ready
+    // gate(): issue `groups` of chunk n if the watcher has seen its blob ready
     auto gate = [&](int n, int groups) {  // thread 0: non-blocking
         if (kOverlap && !rdy) {
-            if (polled == 0u) return;
+            if (smem_acquire(s_rdy) <= n) return;
             rdy = true;
             fence_proxy_async_global();
         }
@@ -743,11 +759,11 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     auto gate_wait = [&](int n) -> bool {  // thread 0: bounded wait, then all groups
         if (kOverlap && !rdy) {
             const uint64_t t0 = global_timer_ns();
-            while (polled == 0u) {
-                polled = flag_acquire(flag0 + (size_t)n * p.H);
-                if (polled != 0u) break;
-                if (status_bad(p.status) || global_timer_ns() - t0 > kWaitNs) return false;
-                __nanosleep(128);
+            while (true) {
+                const int r = smem_acquire(s_rdy);
+                if (r > n) break;
+                if (r < 0 || global_timer_ns() - t0 > kWaitNs) return false;
+                __nanosleep(32);
             }
             rdy = true;
             fence_proxy_async_global();
@@ -758,10 +774,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
 
     if (tid == 0 && t_begin < t_end) {
         pend = 7;
-        if (kOverlap)
-            polled = flag_acquire(flag0);
-        else
-            gate(0, 7);
+        gate(0, 7);
     }
     // ---- initial state (this half): fp32 into TMEM (row c = lane), bf16 into Sb
     {
@@ -795,6 +808,24 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     group_sync(bar, NTC);
     tc_fence_after();
 
+    // O rows of chunk m (rows 64-127 of its X buffer; warps of lane quarters 2, 3)
+    auto o_out = [&](int m, int tt0, int LL) {
+        const int r = trow - C;
+        uint32_t v[32];
+        tmem_ld32(tbase + tlane + tx(m) + cq * 32, v);
+        tmem_wait_ld();
+        if (r < LL) {
+            __nv_bfloat16* dst = p.o + ((size_t)(tt0 + r) * p.H + h) * D + j0 + cq * 32;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]);
+                *reinterpret_cast<uint4*>(dst + q4 * 8) = pack8(y);
+            }
+        }
+    };
+    int prev_t0 = 0, prev_L = 0;
     int n = 0;
     for (int t0 = t_begin; t0 < t_end && !failed; t0 += C, ++n) {
         const int L = min(C, t_end - t0);
@@ -811,26 +842,26 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         if (has_next && tid == 0) {  // the other row-scale buffer is free
             pend = 7;
             coming = n + 1;
-            armed = rdy = false;
-            polled = 0u;
-            gate(n + 1, 1);  // (co-scheduled: not yet read; issued at a later gate)
+            armed = armed3 = rdy = false;
+            gate(n + 1, 1);
         }
         // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
         if (tid == 0) {
             constexpr uint32_t id = idesc_bf16_f32(128, DVS, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
+                mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
                          sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int kb = ks >> 2, kk = ks & 3;
-                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
+                mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
                          sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id, 1);
             }
             mma_commit(bar_mma);
-            if (has_next) poll(n + 1);
         }
+        // the previous chunk's O rows, read out while these products run
+        if (n > 0 && quarter >= 2) o_out(n - 1, prev_t0, prev_L);
         ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
         ++mma_phase;
         if (group_sync_or(bar, NTC, !ok)) {
@@ -843,7 +874,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         if (quarter < 2) {
             const int r = trow;
             uint32_t a[32];
-            tmem_ld32(tbase + tlane + TM_X + cq * 32, a);
+            tmem_ld32(tbase + tlane + tx(n) + cq * 32, a);
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -858,21 +889,25 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         group_sync(bar, NTC);
         tc_fence_after();
         // ---- O = X[64:] + [. ; P] U  (accumulate);  (K E^-1)^T U -> TM_W   (N=64)
-        if (tid == 0) {
+        bool ok3 = true;
+        if (tid == 0) {  // K E^-1, P of this chunk
+            ok3 = mbar_wait(bar_ld3, n & 1, kWaitNs);
+            if (ok3) ld3_chunk = -1;
+        }
+        if (tid == 0 && ok3) {
             constexpr uint32_t idP = idesc_bf16_f32(128, DVS, false, true);
             constexpr uint32_t idK = idesc_bf16_f32(128, DVS, true, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tbase + TM_X, sdesc_sw128(sbase + OFF_PM - 8192 + ks * 32, 16, 1024),
+                mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_PM - 8192 + ks * 32, 16, 1024),
                          sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idP, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tbase + TM_W, sdesc_sw128(sbase + OFF_RAP + ks * 2048, 8192, 1024),
                          sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idK, ks > 0);
             mma_commit(bar_mma);
-            if (has_next) poll(n + 1);
         }
-        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ok = ok3 && mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
         ++mma_phase;
         if (group_sync_or(bar, NTC, !ok)) {
             failed = true;
@@ -880,7 +915,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         }
         tc_fence_after();
         if (has_next && tid == 0) gate(n + 1, 7);  // K E^-1 and P regions free
-        // S <- Gam_last * S + ksc * (K E^-1)^T U   (lane = state row c); O rows out
+        // S <- Gam_last * S + ksc * (K E^-1)^T U   (lane = state row c)
         {
             const int c = trow;
             const float gc = ssc[c], ks = ssc[D + c];
@@ -899,30 +934,16 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
                 for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(sv[q4 * 8 + i]);
                 *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_off(c, cq * 4 + q4)) = pack8(y);
             }
-            if (quarter >= 2) {
-                const int r = trow - C;
-                uint32_t v[32];
-                tmem_ld32(tbase + tlane + TM_X + cq * 32, v);
-                tmem_wait_ld();
-                if (r < L) {
-                    __nv_bfloat16* dst =
-                        p.o + ((size_t)(t0 + r) * p.H + h) * D + j0 + cq * 32;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        float y[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]);
-                        *reinterpret_cast<uint4*>(dst + q4 * 8) = pack8(y);
-                    }
-                }
-            }
             tmem_wait_st();
         }
         fence_async_smem();
         tc_fence_before();
         group_sync(bar, NTC);
         tc_fence_after();
+        prev_t0 = t0;
+        prev_L = L;
     }
+    if (!failed && n > 0 && quarter >= 2) o_out(n - 1, prev_t0, prev_L);
 
     if (!failed && p.hN) {
         const int c = trow;
@@ -940,10 +961,33 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         // wait (bounded) for products and copies still in flight
         if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
         if (armed) mbar_wait(bar_ld, coming & 1, kWaitNs);  // at once if complete
+        if (ld3_chunk >= 0) mbar_wait(bar_ld3, ld3_chunk & 1, kWaitNs);
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
     group_sync(bar, NTC);
+}
+
+// The watcher of a co-scheduled chain CTA (one thread of its other unit):
+// follows the blob flags of the chain's chunks in order (acquire, bounded
+// waits) and publishes how many are ready in the chain unit's shared memory,
+// so that the chain's issuing thread never waits on a global read.
+__device__ __forceinline__ void watch(const Params& p, uint8_t* sm_chain, int chain_id) {
+    const int seq = chain_id / p.H, h = chain_id % p.H;
+    const int cbase = p.chunk_start[seq], nch = p.chunk_start[seq + 1] - cbase;
+    int* s_rdy = reinterpret_cast<int*>(sm_chain + OFF_RDY);
+    const uint32_t* f = p.flags + (size_t)cbase * p.H + h;
+    for (int n = 0; n < nch; ++n) {
+        const uint64_t t0 = global_timer_ns();
+        while (flag_acquire(f + (size_t)n * p.H) == 0u) {
+            if (status_bad(p.status) || global_timer_ns() - t0 > kWaitNs) {
+                smem_release(s_rdy, -1);
+                return;
+            }
+            __nanosleep(64);
+        }
+        smem_release(s_rdy, n + 1);
+    }
 }
 
 __global__ void __launch_bounds__(NTC, 2)
@@ -972,7 +1016,8 @@ __global__ void __launch_bounds__(NTC, 2)
 // chain unit each (one value-column half of one (sequence, head)) with the
 // SM to itself -- a chain step is a short dependent sequence of products and
 // epilogues that slows down by more than half when another unit shares its
-// SM -- and the others run two intra-chunk units each, round by round.  A
+// SM; one thread of the idle unit watches the chain's blob flags -- and the
+// others run two intra-chunk units each, round by round.  A
 // chain waits only for the blobs of its own chunks and an intra unit never
 // waits for a chain; every CTA is resident (cooperative launch), so every
 // wait ends (each is also bounded).
@@ -995,19 +1040,24 @@ __global__ void __launch_bounds__(NTO, 1)
     if (status_bad(pi.status)) return;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t s_tmem;
+    const int b = static_cast<int>(blockIdx.x);
     if (threadIdx.x < 32) {
         tmem_alloc(&s_tmem, 512);
         tmem_relinquish();
     }
+    if (b < nchain && threadIdx.x == 0)
+        *reinterpret_cast<int*>(align1024(smem_raw) + chain::OFF_RDY) = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const int unit = static_cast<int>(threadIdx.x) >> 8;
     uint8_t* sm = align1024(smem_raw) + unit * UNIT_BYTES;
     const uint32_t tb = s_tmem + 256u * unit;
-    const int b = static_cast<int>(blockIdx.x);
     if (b < nchain) {
-        if (unit == 0) chain::run<true>(&tmv, pc, sm, tb, 1, b >> 1, b & 1);
+        if (unit == 0)
+            chain::run<true>(&tmv, pc, sm, tb, 1, b >> 1, b & 1);
+        else if (threadIdx.x == 256)
+            chain::watch(pc, align1024(smem_raw), b >> 1);
     } else
         intra::run<true>(&tmq, &tmk, &tmg, pi, sm, tb, 1 + unit, 2 * (b - nchain) + unit,
                          2 * (static_cast<int>(gridDim.x) - nchain));

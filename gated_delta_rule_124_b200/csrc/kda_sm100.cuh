@@ -137,6 +137,18 @@ __device__ __forceinline__ void flag_release(uint32_t* flag, uint32_t v) {
     asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(v)
                  : "memory");
 }
+// Shared-memory word published by one thread of the CTA and read by another.
+__device__ __forceinline__ void smem_release(int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v)
+                 : "memory");
+}
+__device__ __forceinline__ int smem_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p))
+                 : "memory");
+    return v;
+}
+
 // Acquire read: every later memory access of this thread is ordered after
 // the writes that the flag published (and waits for this load to complete).
 __device__ __forceinline__ uint32_t flag_acquire(const uint32_t* flag) {
