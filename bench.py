@@ -38,19 +38,15 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one
-# ncu capture of each kernel (summaries in profiles/).  Reported only while the
-# kernel's source still matches the capture; null once it has changed.
-MEASURED_TRAFFIC = {
-    "chunk_fwd_tc": ("gated_delta_rule_124_b200/csrc/kda_chunk_tc.cu",
-                     "4231175dcf260063f6cc2aa1e8befdeb56dac955", 195476992),
-    "decode": ("gated_delta_rule_124_b200/csrc/kda_decode.cu",
-               "0055ed0bdb7266f6b3dd4c18570118f7bd32fa1c", 1027668224),
-}
+# ncu capture of each kernel on a workload (summaries in profiles/), keyed by
+# (kernel, workload).  Reported only while the kernel's source still matches the
+# capture; null once it has changed, or for a workload never captured.
+MEASURED_TRAFFIC = {}
 
 
-def measured_traffic(name):
+def measured_traffic(name, workload):
     import hashlib
-    entry = MEASURED_TRAFFIC.get(name)
+    entry = MEASURED_TRAFFIC.get((name, workload))
     if entry is None:
         return None
     path, sha, nbytes = entry
@@ -168,6 +164,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ ours
 
+def prefill_case(wl, args):
+    """The prefill workload of this run (a named configuration, or --prefill-shape)."""
+    if args.prefill_shape:
+        B, T, H = (int(x) for x in args.prefill_shape.split(","))
+        return wl.make_prefill(1100, [T] * B, H=H, dk=128, dv=128, chunk=64, dtype="bf16",
+                               name=f"prefill: B={B} H={H} T={T} d=128 C=64 bf16")
+    return wl.prefill_config(args.prefill_config)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -181,7 +186,7 @@ def run_ours(args, rank, world, local_rank):
     kda.load()
 
     # ---- inputs (resident in HBM before timing)
-    pc = wl.prefill_config(args.prefill_config)
+    pc = prefill_case(wl, args)
     P = pc.to(dev)
     dcase = wl.decode_config()
     D = [{k: v.to(dev) for k, v in s.items()} for s in dcase.steps]
@@ -263,7 +268,7 @@ def run_ours(args, rank, world, local_rank):
     dom_bytes = kern["bytes"][dom_name]
     roof = {"kernel": dom_name, "bound": "hbm", "achieved": dom_bytes / dom_s / 1e9,
             "peak": hbm, "unit": "GB/s", "frac": dom_bytes / dom_s / 1e9 / hbm,
-            "traffic": measured_traffic(dom_name),
+            "traffic": measured_traffic(dom_name, pc.name),
             "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
             "per_launch_us": dom_s * 1e6, "algorithmic_bytes_per_launch": dom_bytes}
     dec_avg = dec_sum / args.steps / 1e3
@@ -285,7 +290,7 @@ def run_ours(args, rank, world, local_rank):
         "decode": {"value": dec_value, "unit": "tokens/s", "ms_per_step": dec_avg * 1e3,
                    "roofline": {"bound": "hbm", "achieved": db / dec_avg / 1e9, "peak": hbm,
                                 "unit": "GB/s", "frac": db / dec_avg / 1e9 / hbm,
-                                "traffic": measured_traffic("decode"),
+                                "traffic": measured_traffic("decode", dcase.name),
                                 "algorithmic_bytes_per_launch": db}},
         "roofline": roof,
         "e2e": e2e,
@@ -537,6 +542,9 @@ def main():
     ap.add_argument("--prefill-config", type=int, default=1, choices=[1, 2, 3],
                     help="prefill workload: 1 = B=2 x T=2048 (default), 2 = B=1 x T=65536, "
                          "3 = 16 packed sequences of U[1024,16384] tokens")
+    ap.add_argument("--prefill-shape", default=None, metavar="B,T,H",
+                    help="instead of --prefill-config: B sequences of T tokens, H heads "
+                         "(d = 128, chunk 64, bf16, the default configuration's distributions)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
