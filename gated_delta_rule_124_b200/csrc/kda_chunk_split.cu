@@ -1,27 +1,31 @@
-// KDA chunkwise prefill, split into two tensor-core kernels (bf16, dk = dv =
-// 128, chunk 64) for problems with few (sequence, head) chains, where one CTA
-// per chain would leave most SMs idle:
+// KDA chunkwise prefill as two tensor-core kernels (bf16, dk = dv = 128,
+// chunk 64) -- the default plan of kda_chunk_fwd for these shapes:
 //
-//   chunk_intra_kernel  one CTA per (chunk, head), all chunks in parallel: the
-//                       in-chunk cumulative log-gate, the operand tiles, A and
-//                       P, the UT transform T = (I + A)^{-1} and
-//                       W = T diag(b) (K * Gam); it writes the chain's operands
-//                       for that chunk to the workspace as one blob laid out
-//                       exactly as the chain kernel's shared memory wants it.
+//   chunk_intra_kernel  persistent, two 256-thread CTAs per SM over all
+//                       (chunk, head) items: the in-chunk cumulative
+//                       log-gate, the operand tiles, A and P, the UT transform
+//                       T = (I + A)^{-1} and W = T diag(b) (K * Gam); it writes
+//                       the chain's operands for that chunk to the workspace
+//                       as one blob laid out exactly as the chain kernel's
+//                       shared memory wants it.
 //   chunk_chain_kernel  two CTAs per (sequence, head) -- one per half of the
 //                       value columns -- chunks in order: bulk copies of each
-//                       chunk's blob and that half of V,
-//                       then Ut = Tb V, X = [W ; Q*Gam] S, U = Ut - W S,
-//                       O = X + [. ; P] U and S <- Gam_last S + K~^T U, with
-//                       S carried in fp32 in tensor memory.
+//                       chunk's blob and that half of V, then
+//                       X = [Tb ; 0] V + [-W ; Q*Gam] S = [U ; Q*Gam S],
+//                       O = X[64:] + P U and S <- Gam_last S + K~^T U, with S
+//                       carried in fp32 in tensor memory.
+//   chunk_overlap_kernel the same two bodies co-scheduled in one cooperative
+//                       launch (one 512-thread CTA of two units per SM; chain
+//                       units alone on their SMs), chains waiting on per-blob
+//                       ready flags.
 //
-// The arithmetic of each step is the same code as the single-kernel path in
-// kda_chunk_tc.cu (same operand layouts and factorisation of the gate; see
-// there); only where each step runs, and the hand-off through the workspace,
-// differ.  Kimi Linear (aiwiki.ai), "The constrained DPLR form and the
-// chunkwise algorithm": parallel inside a chunk, recurrent between chunks --
-// this split runs the first part on every SM and keeps only the second on the
-// per-chain critical path.
+// The factorisation of the gate and the operand layouts are those of the
+// single-kernel plan in kda_chunk_tc.cu (see there); only where each step
+// runs, and the hand-off through the workspace, differ.  Kimi Linear
+// (aiwiki.ai), "The constrained DPLR form and the chunkwise algorithm":
+// parallel inside a chunk, recurrent between chunks -- this split runs the
+// first part on every SM and keeps only the second on the per-chain critical
+// path.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
