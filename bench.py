@@ -509,10 +509,19 @@ def cpu_baseline(pc, seconds=15.0, heads=None):
                        num_threads=cores)
         el += time.perf_counter() - t
         reps += 1
+    # one thread, on the first sequence's first two heads
+    T1, h1 = int(cu[1]) - int(cu[0]), min(2, H)
+    t = time.perf_counter()
+    oracle.forward(pc.q[:T1, :h1], pc.k[:T1, :h1], pc.v[:T1, :h1], pc.g[:T1, :h1],
+                   pc.beta[:T1, :h1], pc.initial_state[:1, :h1], num_threads=1)
+    el1 = time.perf_counter() - t
     return {"value": pc.total * reps / el, "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
             "sample": f"whole prefill workload ({pc.N} x {pc.T} tokens x {H} heads) x {reps} "
-                      f"repetitions, fp64 token recurrence, {el:.1f} s"}
+                      f"repetitions, fp64 token recurrence, {el:.1f} s",
+            "single_thread": {"value": T1 * h1 / el1 / H, "unit": "tokens/s",
+                              "sample": f"1 sequence x {T1} tokens x {h1} of {H} heads, "
+                                        f"1 thread, {el1:.2f} s"}}
 
 
 def run_reference(args, rank, world):

@@ -66,3 +66,28 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["higher_is_better"] is True and line["unit"] == "tokens/s"
+
+
+def test_prefill_shape_option():
+    import argparse
+    from gated_delta_rule_124_b200 import workloads as wl
+    args = argparse.Namespace(prefill_shape="2,128,3", prefill_config=1)
+    pc = bench.prefill_case(wl, args)
+    assert (pc.B, pc.T, pc.H, pc.dk, pc.dv, pc.chunk, pc.dtype) == (2, 128, 3, 128, 128, 64,
+                                                                     "bf16")
+    assert pc.cu_seqlens is None and pc.name == "prefill: B=2 H=3 T=128 d=128 C=64 bf16"
+    args = argparse.Namespace(prefill_shape=None, prefill_config=1)
+    assert bench.prefill_case(wl, args).name == wl.prefill_config(1).name
+
+
+def test_measured_traffic_is_hash_guarded(tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    import hashlib
+    sha = hashlib.sha1(b"kernel v1").hexdigest()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {("kern", "wl"): ("k.cu", sha, 123)})
+    assert bench.measured_traffic("kern", "wl") == 123
+    assert bench.measured_traffic("kern", "other workload") is None
+    src.write_text("kernel v2")  # the kernel changed since the capture
+    assert bench.measured_traffic("kern", "wl") is None
