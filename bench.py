@@ -265,6 +265,10 @@ def run_ours(args, rank, world, local_rank):
     # ---- per-kernel times of the prefill (dominant kernel) with the step calls
     kern = prefill_kernel_times(kda, P, ws, dev, stream, reps=max(5, min(50, args.steps)))
 
+    # ---- the steps around the operator (conv/Swish/L2-norm before, RMSNorm and
+    # output gate after), on this workload's tensors, each timed alone
+    layer = layer_times(kda, torch, P, dev, stream, reps=max(5, min(50, args.steps)))
+
     # ---- end to end through host buffers (pinned), copies inside the region
     e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=max(3, min(args.steps, 50)))
 
@@ -304,6 +308,7 @@ def run_ours(args, rank, world, local_rank):
                                 "traffic": measured_traffic("decode", dcase.name),
                                 "algorithmic_bytes_per_launch": db}},
         "roofline": roof,
+        "layer_steps": layer,
         "e2e": e2e,
         "gpu_launches": args.steps * (kern["launches_per_call"] + 1),
         "clocks": clk,
@@ -407,6 +412,48 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     dom = max(times, key=times.get)
     return {"times": times, "bytes": nbytes, "dominant": (dom, times[dom]),
             "launches_per_call": 5, "path": path}
+
+
+def layer_times(kda, torch, P, dev, stream, reps=20):
+    """CUDA-event times of kda_qkv_conv_norm and kda_output_norm_gate on the
+    prefill workload's shapes (bf16), L2 flushed before each, with their HBM
+    fraction (bytes: every tensor read or written once; conv weights excluded)."""
+    total, H, dk, dv = P.total, P.H, P.dk, P.dv
+    Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
+    g = torch.Generator(device=dev).manual_seed(7)
+    xs = [torch.randn(total, H, d, device=dev, generator=g).to(torch.bfloat16)
+          for d in (dk, dk, dv)]
+    ws = [torch.randn(H * d, 4, device=dev, generator=g) for d in (dk, dk, dv)]
+    outs = [torch.empty_like(x) for x in xs]
+    gate = torch.randn(total, H, dv, device=dev, generator=g).to(torch.bfloat16)
+    wn = torch.ones(dv, device=dev)
+    y = torch.empty_like(gate)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = {
+        "qkv_conv_norm": (lambda: kda.kda_qkv_conv_norm(*xs, *ws, P.cu_seqlens, Bc, Tc, P.N, H,
+                                                        dk, dv, "bf16", 1e-6, *outs),
+                          2 * 2 * total * H * (2 * dk + dv)),
+        "output_norm_gate": (lambda: kda.kda_output_norm_gate(outs[2], gate, wn, total, H, dv,
+                                                              "bf16", 1e-6, y),
+                             2 * 3 * total * H * dv),
+    }
+    peaks, _ = load_peaks()
+    res = {}
+    for name, (f, nbytes) in calls.items():
+        f()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            f()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        t = statistics.median(x.elapsed_time(z) for x, z in ts) / 1e3
+        res[name] = {"us": t * 1e6, "bytes": nbytes, "gbs": nbytes / t / 1e9,
+                     "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+    return res
 
 
 def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):

@@ -369,6 +369,41 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
                                         static_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------ layer steps (NEXT-2)
+
+kda_status_t kda_qkv_conv_norm(const void* xq, const void* xk, const void* xv, const float* wq,
+                               const float* wk, const float* wv, const int32_t* cu_seqlens,
+                               int B, int T, int num_seqs, int H, int dk, int dv,
+                               kda_dtype_t dtype, float eps, void* q, void* k, void* v,
+                               void* stream) {
+    Prefill p;
+    kda_status_t s = check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, 64, dtype, &p);
+    if (s != KDA_OK) return s;
+    if (!(eps > 0.f) || !(eps < 1e30f)) return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : std::initializer_list<const void*>{
+             xq, xk, xv, (const void*)wq, (const void*)wk, (const void*)wv, q, k, v})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    const void* const x[3] = {xq, xk, xv};
+    const float* const w[3] = {wq, wk, wv};
+    void* const y[3] = {q, k, v};
+    return from_cuda(kda::launch_qkv_conv(x, w, y, dk, dv, cu_seqlens, p.N,
+                                          cu_seqlens ? 0 : T, p.total, H, eps, dtype,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* w,
+                                  int total_tokens, int H, int dv, kda_dtype_t dtype, float eps,
+                                  void* y, void* stream) {
+    if (total_tokens < 0 || H < 1 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if ((long long)total_tokens * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!(eps > 0.f) || !(eps < 1e30f)) return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : std::initializer_list<const void*>{o, gate, (const void*)w, y})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_norm_gate(o, gate, w, total_tokens, H, dv, eps, dtype, y,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 // ----------------------------------------------------------------- status
 
 kda_status_t kda_get_device_status(void* workspace, void* stream) {

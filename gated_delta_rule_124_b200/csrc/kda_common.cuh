@@ -128,6 +128,11 @@ cudaError_t launch_output(const void* q, const void* k, const float* G, const fl
                           const float* states, const int4* info, int maxc, int H, int dk,
                           int dv, int chunk, kda_dtype_t dt, const uint32_t* status, void* o,
                           cudaStream_t st);
+cudaError_t launch_qkv_conv(const void* const x[3], const float* const w[3], void* const y[3],
+                            int dk, int dv, const int32_t* cu, int N, int T, int total, int H,
+                            float eps, kda_dtype_t dt, cudaStream_t st);
+cudaError_t launch_norm_gate(const void* o, const void* gate, const float* w, int total, int H,
+                             int d, float eps, kda_dtype_t dt, void* y, cudaStream_t st);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* o, int N, int H, int dk,
                           int dv, kda_dtype_t dt, cudaStream_t st);

@@ -39,7 +39,8 @@ EXPORTS = (
     "kda_num_chunks_upper_bound", "kda_chunk_gate_cumsum", "kda_chunk_intra",
     "kda_chunk_inter", "kda_chunk_output", "kda_decode_step", "kda_get_device_status",
     "kda_chunk_fwd_noalloc", "kda_chunk_split_workspace_size", "kda_chunk_split_intra",
-    "kda_chunk_split_chain", "kda_chunk_fwd_plan",
+    "kda_chunk_split_chain", "kda_chunk_fwd_plan", "kda_qkv_conv_norm",
+    "kda_output_norm_gate",
 )
 
 
@@ -67,6 +68,8 @@ _SIGS = {
     "kda_chunk_fwd_noalloc": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp], _i),
     "kda_chunk_split_workspace_size": ([_i, _i, _i], _sz),
     "kda_chunk_fwd_plan": ([_i] * 8, _i),
+    "kda_qkv_conv_norm": ([_vp] * 7 + [_i] * 7 + [ctypes.c_float] + [_vp] * 4, _i),
+    "kda_output_norm_gate": ([_vp] * 3 + [_i] * 4 + [ctypes.c_float] + [_vp] * 2, _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
@@ -225,6 +228,21 @@ def kda_chunk_split_chain(v, initial_state, cu_seqlens, B, T, num_seqs, H, o, fi
                                       num_seqs, H, _p(o), _p(final_state), _p(workspace), wb,
                                       _stream(stream))
     return _ret(st, "kda_chunk_split_chain", check)
+
+
+def kda_qkv_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens, B, T, num_seqs, H, dk, dv, dtype,
+                      eps, q, k, v, stream=None, check=True) -> int:
+    st = load().kda_qkv_conv_norm(_p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
+                                  _p(cu_seqlens), B, T, num_seqs, H, dk, dv, dtype_code(dtype),
+                                  float(eps), _p(q), _p(k), _p(v), _stream(stream))
+    return _ret(st, "kda_qkv_conv_norm", check)
+
+
+def kda_output_norm_gate(o, gate, w, total_tokens, H, dv, dtype, eps, y, stream=None,
+                         check=True) -> int:
+    st = load().kda_output_norm_gate(_p(o), _p(gate), _p(w), total_tokens, H, dv,
+                                     dtype_code(dtype), float(eps), _p(y), _stream(stream))
+    return _ret(st, "kda_output_norm_gate", check)
 
 
 def kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,

@@ -244,6 +244,43 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
                              const float* beta, float* state, void* o, int N, int H, int dk,
                              int dv, kda_dtype_t dtype, void* stream);
 
+/* ---------------------------------------- the steps around the operator
+ * Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
+ * algorithm" (the paragraph on what each KDA head applies): a short depthwise
+ * convolution (kernel 4) with a Swish activation on q, k and v and the L2
+ * normalisation of q and k before the operator; a head-wise RMSNorm and a
+ * sigmoid output gate after it.  Arithmetic in fp32; both calls read and write
+ * each tensor once.
+ *
+ * kda_qkv_conv_norm: for each of q, k, v: y[t, h, c] = Swish(sum_{i=0..3}
+ * w[h*d + c][i] * x[t - 3 + i, h, c]) with Swish(x) = x * sigmoid(x), no bias,
+ * tap 3 on the current token and tokens before the first token of t's
+ * sequence counting as zero (a packed batch never convolves across
+ * sequences); then q and k are scaled per (token, head) by
+ * 1 / sqrt(sum_c y^2 + eps).
+ * In:  xq, xk [total, H, dk], xv [total, H, dv] (dtype); wq, wk [H*dk, 4] and
+ *      wv [H*dv, 4] fp32; cu_seqlens / B / T / num_seqs as for kda_chunk_fwd
+ *      (cu_seqlens contents are not checked here; a malformed array cannot
+ *      make a read leave the tensors); eps > 0.
+ * Out: q, k [total, H, dk], v [total, H, dv] (dtype), not aliasing the inputs.
+ * Shapes: dk, dv in {32, 64, 128}.
+ */
+kda_status_t kda_qkv_conv_norm(const void* xq, const void* xk, const void* xv, const float* wq,
+                               const float* wk, const float* wv, const int32_t* cu_seqlens,
+                               int B, int T, int num_seqs, int H, int dk, int dv,
+                               kda_dtype_t dtype, float eps, void* q, void* k, void* v,
+                               void* stream);
+
+/* kda_output_norm_gate: y[t, h, :] = o[t, h, :] / sqrt(mean_j o[t, h, j]^2 +
+ * eps) * w * sigmoid(gate[t, h, :]).
+ * In:  o, gate [total_tokens, H, dv] (dtype); w [dv] fp32 (shared by the
+ *      heads); eps > 0.  Out: y [total_tokens, H, dv] (dtype); y may be o.
+ * Shapes: dv in {32, 64, 128}.
+ */
+kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* w,
+                                  int total_tokens, int H, int dv, kda_dtype_t dtype, float eps,
+                                  void* y, void* stream);
+
 /* ------------------------------------------------ prefill, no allocation
  * kda_chunk_fwd_noalloc: the same computation as kda_chunk_fwd, with no
  * workspace argument, for callers that may not obtain device memory: an

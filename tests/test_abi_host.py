@@ -154,3 +154,21 @@ def test_split_calls_reject_bad_arguments(lib):
 def test_get_device_status_rejects_bad_workspace(lib):
     assert kda.kda_get_device_status(None, 0) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_get_device_status(FAKE + 16, 0) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_layer_calls_reject_bad_arguments(lib):
+    conv = dict(xq=FAKE, xk=FAKE, xv=FAKE, wq=FAKE, wk=FAKE, wv=FAKE, cu_seqlens=None, B=1,
+                T=64, num_seqs=1, H=2, dk=128, dv=128, dtype="bf16", eps=1e-6, q=FAKE, k=FAKE,
+                v=FAKE, stream=0, check=False)
+    assert kda.kda_qkv_conv_norm(**{**conv, "xq": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm(**{**conv, "wk": FAKE + 4}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm(**{**conv, "eps": 0.0}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm(**{**conv, "eps": float("nan")}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm(**{**conv, "dk": 96}) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_qkv_conv_norm(**{**conv, "num_seqs": 2}) == kda.KDA_ERR_INVALID_ARG
+    gate = dict(o=FAKE, gate=FAKE, w=FAKE, total_tokens=64, H=2, dv=64, dtype="f32", eps=1e-6,
+                y=FAKE, stream=0, check=False)
+    assert kda.kda_output_norm_gate(**{**gate, "y": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_output_norm_gate(**{**gate, "total_tokens": -1}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_output_norm_gate(**{**gate, "dv": 48}) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_output_norm_gate(**{**gate, "eps": -1.0}) == kda.KDA_ERR_INVALID_ARG
