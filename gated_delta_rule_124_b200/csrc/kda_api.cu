@@ -124,6 +124,45 @@ kda_status_t begin_prefill(const Workspace& w, const int32_t* cu, int B, int T, 
     return from_cuda(e);
 }
 
+// The CUDA-core plan after the chunk table: a1 .. a4 as four kernels.
+kda_status_t run_simt(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                      int B, int T, const Prefill& p, int H, int dk, int dv, int chunk,
+                      kda_dtype_t dtype, void* o, float* final_state, const Workspace& w,
+                      int maxc, cudaStream_t st) {
+    cudaError_t e = kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
+    if (e == cudaSuccess)
+        e = kda::launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, chunk, dtype,
+                              w.status, w.W, w.U, st);
+    if (e == cudaSuccess)
+        e = kda::launch_inter(k, w.G, w.W, w.U, initial_state, cu_seqlens, B, T, p.N,
+                              w.chunk_start, H, dk, dv, chunk, dtype, w.status, w.states,
+                              final_state, st);
+    if (e == cudaSuccess)
+        e = kda::launch_output(q, k, w.G, w.U, w.states, w.chunk_info, maxc, H, dk, dv, chunk,
+                               dtype, w.status, o, st);
+    return from_cuda(e);
+}
+
+// Gated DeltaNet (head-uniform gate): the split plan reads the gate per
+// (token, head) directly; every other shape spreads it over the dk channels
+// into the workspace, after the CUDA-core plan's own part, and runs that plan.
+Path gdn_path(int dk, int dv, int chunk, kda_dtype_t dt) {
+    const bool tc_shape = dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
+                          kda::tc_path_available();
+    const char* env = getenv("KDA_CHUNK_PATH");
+    if (env && !strcmp(env, "simt")) return Path::Simt;
+    return tc_shape ? Path::Split : Path::Simt;
+}
+
+size_t gdn_workspace_bytes(const Prefill& p, int H, int dk, int dv, int chunk, Path path,
+                           size_t* spread_offset) {
+    const size_t base = carve_for(nullptr, p, H, dk, dv, chunk, path).total_bytes;
+    *spread_offset = base;
+    if (path != Path::Simt) return base;
+    return kda::align_up(base + sizeof(float) * (size_t)p.total * H * dk);
+}
+
 }  // namespace
 
 extern "C" {
@@ -210,18 +249,8 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
                                                      w.chunk_start, w.status, w.blobs, o,
                                                      final_state, st));
     }
-    cudaError_t e = kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
-    if (e == cudaSuccess)
-        e = kda::launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, chunk, dtype,
-                              w.status, w.W, w.U, st);
-    if (e == cudaSuccess)
-        e = kda::launch_inter(k, w.G, w.W, w.U, initial_state, cu_seqlens, B, T, p.N,
-                              w.chunk_start, H, dk, dv, chunk, dtype, w.status, w.states,
-                              final_state, st);
-    if (e == cudaSuccess)
-        e = kda::launch_output(q, k, w.G, w.U, w.states, w.chunk_info, maxc, H, dk, dv, chunk,
-                               dtype, w.status, o, st);
-    return from_cuda(e);
+    return run_simt(q, k, v, g, beta, initial_state, cu_seqlens, B, T, p, H, dk, dv, chunk,
+                    dtype, o, final_state, w, maxc, st);
 }
 
 // ------------------------------------------------- one step per call (a1-a4)
@@ -367,6 +396,71 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
         if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
     return from_cuda(kda::launch_decode(q, k, v, g, beta, state, o, N, H, dk, dv, dtype,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------- Gated DeltaNet (head-uniform gate)
+
+size_t kda_gdn_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
+                                        int chunk, kda_dtype_t dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
+        !chunk_ok(chunk) || !dtype_ok(dtype))
+        return 0;
+    const Prefill p{total_tokens, num_seqs};
+    size_t off;
+    return gdn_workspace_bytes(p, H, dk, dv, chunk, gdn_path(dk, dv, chunk, dtype), &off);
+}
+
+kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* initial_state,
+                               const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                               int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                               float* final_state, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+    Prefill p;
+    kda_status_t s =
+        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);
+    if (s != KDA_OK) return s;
+    if (!q || !k || !v || !g || !beta || !o) return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : {q, k, v, (const void*)g, (const void*)beta, (const void*)o})
+        if (!aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    const Path path = gdn_path(dk, dv, chunk, dtype);
+    size_t spread_off = 0;
+    const size_t need = gdn_workspace_bytes(p, H, dk, dv, chunk, path, &spread_off);
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return KDA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    const Workspace w = carve_for(workspace, p, H, dk, dv, chunk, path);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int maxc = kda::max_chunks(p.total, p.N, chunk);
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);
+    if (s != KDA_OK) return s;
+    if (p.total == 0 && !final_state) return KDA_OK;
+    if (path == Path::Split)
+        return from_cuda(kda::launch_chunk_fwd_split(q, k, v, nullptr, beta, initial_state,
+                                                     cu_seqlens, T, p.N, H, w.chunk_info, maxc,
+                                                     w.chunk_start, w.status, w.blobs, o,
+                                                     final_state, st, g));
+    float* gfull = reinterpret_cast<float*>(static_cast<char*>(workspace) + spread_off);
+    const cudaError_t e = kda::launch_spread_gate(g, p.total, H, dk, gfull, st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    return run_simt(q, k, v, gfull, beta, initial_state, cu_seqlens, B, T, p, H, dk, dv, chunk,
+                    dtype, o, final_state, w, maxc, st);
+}
+
+kda_status_t kda_gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float* state, void* o, int N, int H, int dk,
+                                 int dv, kda_dtype_t dtype, void* stream) {
+    if (N < 0 || H < 1 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return KDA_OK;
+    for (const void* ptr : {q, k, v, (const void*)g, (const void*)beta, (const void*)state,
+                            (const void*)o})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_decode(q, k, v, g, beta, state, o, N, H, dk, dv, dtype,
+                                        static_cast<cudaStream_t>(stream), true));
 }
 
 // ------------------------------------------------------ layer steps (NEXT-2)

@@ -90,7 +90,11 @@ constexpr uint32_t OFF_GM = OFF_BETA + 256;
 constexpr uint32_t OFF_EGM = OFF_GM + 512;
 constexpr uint32_t OFF_GL = OFF_EGM + 512;
 constexpr uint32_t OFF_WSC = OFF_GL + 512;
-constexpr uint32_t OFF_BAR = OFF_WSC + 512;
+// head-uniform gate: g of the chunk's rows -> their G (64 floats), then
+// {Gm, exp(Gm), G_last}
+constexpr uint32_t OFF_GS = OFF_WSC + 512;
+constexpr uint32_t OFF_GSC = OFF_GS + 256;
+constexpr uint32_t OFF_BAR = OFF_GSC + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 static_assert(OFF_MID == OFF_TB + 8192, "Tb garbage rows follow Tb");
 static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
@@ -111,6 +115,7 @@ struct Params {
     const int* chunk_start;
     const uint32_t* rounds;  // largest number of chunks of one sequence
     uint32_t* flags;         // [slot, head]: set once that blob is complete
+    const float* gh;         // head-uniform gate [total, H] (kScalar)
 };
 
 // One worker (CTA) of the intra-chunk kernel.  Items are (chunk slot, head)
@@ -119,7 +124,11 @@ struct Params {
 // head) before chunk n + 1 of any -- and each finished blob is flagged.
 // The unit is a group of NTI threads (a whole CTA, or half of one) that
 // synchronises on named barrier `bar`; `tbase` is its 256 TMEM columns.
-template <bool kOverlap>
+// kScalar: the gate is one value per (token, head) (Gated DeltaNet; Kimi
+// Linear (aiwiki.ai), "Background: from the delta rule to gated DeltaNet"):
+// read from p.gh by plain loads, scanned by one warp, and every per-channel
+// factor of a row is that row's one factor.
+template <bool kOverlap, bool kScalar = false>
 __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* tmk,
                                     const CUtensorMap* tmg, const Params& p, uint8_t* sm,
                                     uint32_t tbase, uint32_t bar, int worker, int nworkers) {
@@ -208,14 +217,22 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     auto fetch_beta = [&](const Item& d) {
         return tid < d.L ? p.beta[(size_t)(d.t0 + tid) * p.H + d.h] : 0.f;
     };
+    float* sGs = reinterpret_cast<float*>(sm + OFF_GS);
+    float* sGsc = reinterpret_cast<float*>(sm + OFF_GSC);
+    float gs_next = 0.f;  // (kScalar, tid < C) this thread's g of the next item
+    auto fetch_gs = [&](const Item& d) {
+        return tid < d.L ? p.gh[(size_t)(d.t0 + tid) * p.H + d.h] : 0.f;
+    };
     if (cur.it < nitems) {
         if (tid == 0) {
             load_k(cur);
             load_q(cur);
-            load_g(cur);
-            k_issued = q_issued = g_issued = 1;
+            if (!kScalar) load_g(cur);
+            k_issued = q_issued = 1;
+            g_issued = kScalar ? 0 : 1;
         }
         if (tid < C) beta_next = fetch_beta(cur);
+        if (kScalar && tid < C) gs_next = fetch_gs(cur);
     }
     int n = 0;
     for (; cur.it < nitems && !failed; ++n) {
@@ -223,6 +240,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         const bool more = nxt.it < nitems;
         uint8_t* blob = p.blobs + ((size_t)slot * p.H + h) * BLOB;
         if (tid < C) sbeta[tid] = beta_next;
+        if (kScalar && tid < C) sGs[tid] = gs_next;
         if (tid == 0) {
             // the previous item's bulk write-out has read its tiles (and, when
             // a chain waits for it, has completed)
@@ -231,7 +249,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             else
                 bulk_wait_read();
         }
-        bool ok = mbar_wait(bar_g, n & 1, kWaitNs);  // K, Q: after E1
+        bool ok = kScalar || mbar_wait(bar_g, n & 1, kWaitNs);  // K, Q: after E1
         if (group_sync_or(bar, NTI, !ok)) {
             failed = true;
             break;
@@ -240,7 +258,45 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         // (row group grp = 8 rows, channels 4 c4 ..): scan of its 8 rows, then
         // the totals of the groups above it added; per-channel max / min.
         bool slow_local = false;
-        {
+        if (kScalar) {
+            // one warp: lane l holds rows 2l, 2l + 1; inclusive scan by shuffles
+            if (warp == 0) {
+                const int r0 = 2 * lane;
+                const float v0 = r0 < L ? sGs[r0] : 0.f, v1 = r0 + 1 < L ? sGs[r0 + 1] : 0.f;
+                float pre = v0 + v1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, pre, o);
+                    if (lane >= o) pre += y;
+                }
+                const float G0 = pre - v1, G1 = pre;
+                float mx = -INFINITY, mn = INFINITY;
+                if (r0 < L) { mx = G0; mn = G0; }
+                if (r0 + 1 < L) { mx = fmaxf(mx, G1); mn = fminf(mn, G1); }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                }
+                __syncwarp();
+                sGs[r0] = G0;
+                sGs[r0 + 1] = G1;
+                __syncwarp();
+                if (lane == 0) {
+                    const float Gm = mx - kRef;
+                    sGsc[0] = Gm;
+                    sGsc[1] = expf(Gm);
+                    sGsc[2] = sGs[L - 1];
+                }
+                slow_local = !(mx - mn <= 2.f * kRef) || !(mx <= 60.f);
+            }
+            group_sync(bar, NTI);
+            if (tid < D) {  // the per-channel arrays all hold the row-uniform values
+                sGm[tid] = sGsc[0];
+                seGm[tid] = sGsc[1];
+                sGL[tid] = sGsc[2];
+            }
+        } else {
             float* g = reinterpret_cast<float*>(sm + OFF_G);
             float4* tot = reinterpret_cast<float4*>(sm + OFF_TB);           // [8][32]
             float4* gmx = reinterpret_cast<float4*>(sm + OFF_TB + 4096);    // [8][32]
@@ -320,7 +376,25 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 float a[8], pp[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) a[j] = pp[j] = 0.f;
-                if (r < L) {
+                if (r < L && kScalar) {  // one factor per pair, outside the dot products
+                    for (int c = 0; c < D; ++c) {
+                        const float kr = tile_elem(sm + OFF_KQ, 16384, r, c);
+                        const float qr = tile_elem(sm + OFF_KQ + 8192, 16384, r, c);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float ki = tile_elem(sm + OFF_KQ, 16384, i0 + j, c);
+                            a[j] += kr * ki;
+                            pp[j] += qr * ki;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int i = i0 + j;
+                        const float e = i <= r ? expf(sGs[r] - sGs[i]) : 0.f;
+                        a[j] *= e;
+                        pp[j] *= e;
+                    }
+                } else if (r < L) {
                     for (int c = 0; c < D; ++c) {
                         const float kr = tile_elem(sm + OFF_KQ, 16384, r, c);
                         const float qr = tile_elem(sm + OFF_KQ + 8192, 16384, r, c);
@@ -362,7 +436,32 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 uint8_t* pk = sm + OFF_KQ + kb * 16384 + o64;
                 uint8_t* pq = pk + 8192;
                 float lk[8], lq[8], rk[8], qg[8];
-                if (r < L) {
+                if (r < L && kScalar) {  // the row's factors, once
+                    float k8[8], q8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(pk), k8);
+                    unpack8(*reinterpret_cast<const uint4*>(pq), q8);
+                    const float gr = sGs[r];
+                    if (!slow) {
+                        const float x = gr - m8[0];
+                        const float E = __expf(x), Ei = __expf(-x), eg = e8[0];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            lk[i] = k8[i] * E;
+                            lq[i] = q8[i] * E;
+                            rk[i] = k8[i] * Ei;
+                            qg[i] = lq[i] * eg;
+                        }
+                    } else {  // m8 holds G_last here
+                        const float gam = expf(gr), back = expf(m8[0] - gr);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            lk[i] = k8[i] * gam;
+                            lq[i] = 0.f;
+                            rk[i] = k8[i] * back;
+                            qg[i] = q8[i] * gam;
+                        }
+                    }
+                } else if (r < L) {
                     float k8[8], q8[8], g8[8];
                     unpack8(*reinterpret_cast<const uint4*>(pk), k8);
                     unpack8(*reinterpret_cast<const uint4*>(pq), q8);
@@ -402,7 +501,10 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         tc_fence_before();
         group_sync(bar, NTI);
         tc_fence_after();
-        if (tid < C && more) beta_next = fetch_beta(nxt);
+        if (tid < C && more) {
+            beta_next = fetch_beta(nxt);
+            if (kScalar) gs_next = fetch_gs(nxt);
+        }
         if (tid == 0) {
             bulk_s2g(blob + BL_RAP, sm + OFF_RAP, 16384);  // the chain's K E^-1
             bulk_commit();
@@ -542,7 +644,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         if (tid == 0) {
             bulk_s2g(blob + BL_TB, sm + OFF_TB, 8192);  // the chain's Tb
             bulk_commit();
-            if (more) {  // the G region is free: fetch the next g
+            if (more && !kScalar) {  // the G region is free: fetch the next g
                 load_g(nxt);
                 ++g_issued;
             }
@@ -607,6 +709,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     }
 }
 
+template <bool kScalar>
 __global__ void __launch_bounds__(NTI, 2)
     chunk_intra_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
@@ -621,7 +724,8 @@ __global__ void __launch_bounds__(NTI, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    run<false>(&tmq, &tmk, &tmg, p, align1024(smem_raw), s_tmem, 1, blockIdx.x, gridDim.x);
+    run<false, kScalar>(&tmq, &tmk, &tmg, p, align1024(smem_raw), s_tmem, 1, blockIdx.x,
+                        gridDim.x);
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
@@ -1100,19 +1204,27 @@ bool split_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
 
 cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
                                int total, int H, const int4* chunk_info, int maxc,
-                               uint32_t* status, void* blobs, cudaStream_t st) {
+                               uint32_t* status, void* blobs, cudaStream_t st, const float* gh) {
     if (total == 0 || maxc == 0) return cudaSuccess;
     CUtensorMap mq, mk, mg;
     if (!split_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+                   CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel,
+    if (gh) {
+        mg = mq;  // not read: the head-uniform gate comes by plain loads
+    } else if (!split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)intra::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(intra::chunk_intra_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)intra::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -1120,7 +1232,13 @@ cudaError_t launch_split_intra(const void* q, const void* k, const float* g, con
     const long long items = (long long)maxc * H;
     const int grid = (int)(items < 2 * sms ? items : 2 * sms);
     intra::Params pa{beta, chunk_info, maxc, H, status, status, static_cast<uint8_t*>(blobs)};
-    intra::chunk_intra_kernel<<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(mq, mk, mg, pa);
+    pa.gh = gh;
+    if (gh)
+        intra::chunk_intra_kernel<true><<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(mq, mk, mg,
+                                                                                    pa);
+    else
+        intra::chunk_intra_kernel<false><<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(mq, mk, mg,
+                                                                                     pa);
     return cudaGetLastError();
 }
 
@@ -1221,10 +1339,10 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
                                    const int32_t* cu_seqlens, int T, int N, int H,
                                    const int4* chunk_info, int maxc, const int* chunk_start,
                                    uint32_t* status, void* blobs, void* o, float* hN,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, const float* gh) {
     const int total = cu_seqlens ? T : N * T;
     cudaError_t e =
-        launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs, st);
+        launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs, st, gh);
     if (e != cudaSuccess) return e;
     return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN, st);
 }

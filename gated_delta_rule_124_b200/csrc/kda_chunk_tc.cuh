@@ -19,17 +19,19 @@ cudaError_t launch_chunk_fwd_tc(const void* q, const void* k, const void* v, con
 // head) chains: chunk-parallel intra-chunk kernel + per-chain kernel, handing
 // over through `blobs` (split_blob_bytes() per (chunk slot, head)).
 size_t split_blob_bytes();
+// gh != NULL: the gate is head-uniform, gh [total, H] (g is then unused).
 cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,
                                    const float* beta, const float* h0,
                                    const int32_t* cu_seqlens, int T, int N, int H,
                                    const int4* chunk_info, int maxc, const int* chunk_start,
                                    uint32_t* status, void* blobs, void* o, float* hN,
-                                   cudaStream_t st);
+                                   cudaStream_t st, const float* gh = nullptr);
 // Its two kernels one at a time (the chain kernel reads what the intra kernel
 // wrote, on the same stream).
 cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
                                int total, int H, const int4* chunk_info, int maxc,
-                               uint32_t* status, void* blobs, cudaStream_t st);
+                               uint32_t* status, void* blobs, cudaStream_t st,
+                               const float* gh = nullptr);
 cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
                                int N, int H, const int* chunk_start, uint32_t* status,
                                const void* blobs, void* o, float* hN, cudaStream_t st);

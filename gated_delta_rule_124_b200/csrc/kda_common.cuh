@@ -135,5 +135,8 @@ cudaError_t launch_norm_gate(const void* o, const void* gate, const float* w, in
                              int d, float eps, kda_dtype_t dt, void* y, cudaStream_t st);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* o, int N, int H, int dk,
-                          int dv, kda_dtype_t dt, cudaStream_t st);
+                          int dv, kda_dtype_t dt, cudaStream_t st, bool head_gate = false);
+// G_full[t, h, c] = g[t, h] (a head-uniform gate spread over dk channels)
+cudaError_t launch_spread_gate(const float* g, int total, int H, int dk, float* out,
+                               cudaStream_t st);
 }  // namespace kda

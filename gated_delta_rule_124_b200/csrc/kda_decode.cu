@@ -28,7 +28,9 @@
 
 namespace kda {
 
-template <int DK, int DV, int DVS, typename TIn>
+// kHeadGate: g is one value per (sequence, head) [units] (Gated DeltaNet)
+// instead of one per key channel.
+template <int DK, int DV, int DVS, typename TIn, bool kHeadGate>
 __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2) decode_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
     const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2) decode_kernel
         const size_t i = (size_t)unit * DK + c;
         s_k[c] = to_f32(k[i]);
         s_q[c] = to_f32(q[i]);
-        s_a[c] = expf(g[i]);
+        s_a[c] = expf(kHeadGate ? g[unit] : g[i]);
     }
     __syncthreads();
     if (w == 0) {
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2) decode_kernel
 template <typename TIn>
 static cudaError_t decode_dispatch(const void* q, const void* k, const void* v, const float* g,
                                    const float* beta, float* state, void* o, int units, int dk,
-                                   int dv, cudaStream_t st) {
+                                   int dv, bool head_gate, cudaStream_t st) {
     const TIn* Q = (const TIn*)q;
     const TIn* K = (const TIn*)k;
     const TIn* V = (const TIn*)v;
@@ -146,7 +148,10 @@ static cudaError_t decode_dispatch(const void* q, const void* k, const void* v, 
     if (dk == A && dv == B) {                                                           \
         constexpr int DVS = (B == 128) ? 64 : B;                                        \
         const dim3 grid(units, B / DVS);                                                \
-        decode_kernel<A, B, DVS, TIn><<<grid, 256, 0, st>>>(Q, K, V, g, beta, state, O); \
+        if (head_gate)                                                                  \
+            decode_kernel<A, B, DVS, TIn, true><<<grid, 256, 0, st>>>(Q, K, V, g, beta, state, O); \
+        else                                                                            \
+            decode_kernel<A, B, DVS, TIn, false><<<grid, 256, 0, st>>>(Q, K, V, g, beta, state, O); \
         return cudaGetLastError();                                                      \
     }
     KDA_DECODE_CASE(128, 128)
@@ -164,12 +169,13 @@ static cudaError_t decode_dispatch(const void* q, const void* k, const void* v, 
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* o, int N, int H, int dk,
-                          int dv, kda_dtype_t dt, cudaStream_t st) {
+                          int dv, kda_dtype_t dt, cudaStream_t st, bool head_gate) {
     const int units = N * H;
     if (units == 0) return cudaSuccess;
     if (dt == KDA_DTYPE_BF16)
-        return decode_dispatch<__nv_bfloat16>(q, k, v, g, beta, state, o, units, dk, dv, st);
-    return decode_dispatch<float>(q, k, v, g, beta, state, o, units, dk, dv, st);
+        return decode_dispatch<__nv_bfloat16>(q, k, v, g, beta, state, o, units, dk, dv,
+                                              head_gate, st);
+    return decode_dispatch<float>(q, k, v, g, beta, state, o, units, dk, dv, head_gate, st);
 }
 
 }  // namespace kda

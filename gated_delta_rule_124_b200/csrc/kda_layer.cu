@@ -258,7 +258,21 @@ cudaError_t gate_dispatch(const void* o, const void* gate, const float* w, int t
     return cudaGetLastError();
 }
 
+__global__ void spread_gate_kernel(const float* __restrict__ g, long long n, int dk,
+                                   float* __restrict__ out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = g[i / dk];
+}
+
 }  // namespace
+
+cudaError_t launch_spread_gate(const float* g, int total, int H, int dk, float* out,
+                               cudaStream_t st) {
+    const long long n = (long long)total * H * dk;
+    if (n == 0) return cudaSuccess;
+    spread_gate_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(g, n, dk, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_qkv_conv(const void* const x[3], const float* const w[3], void* const y[3],
                             int dk, int dv, const int32_t* cu, int N, int T, int total, int H,

@@ -40,7 +40,8 @@ EXPORTS = (
     "kda_chunk_inter", "kda_chunk_output", "kda_decode_step", "kda_get_device_status",
     "kda_chunk_fwd_noalloc", "kda_chunk_split_workspace_size", "kda_chunk_split_intra",
     "kda_chunk_split_chain", "kda_chunk_fwd_plan", "kda_qkv_conv_norm",
-    "kda_output_norm_gate",
+    "kda_output_norm_gate", "kda_gdn_chunk_fwd_workspace_size", "kda_gdn_chunk_fwd",
+    "kda_gdn_decode_step",
 )
 
 
@@ -70,6 +71,9 @@ _SIGS = {
     "kda_chunk_fwd_plan": ([_i] * 8, _i),
     "kda_qkv_conv_norm": ([_vp] * 7 + [_i] * 7 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_output_norm_gate": ([_vp] * 3 + [_i] * 4 + [ctypes.c_float] + [_vp] * 2, _i),
+    "kda_gdn_chunk_fwd_workspace_size": ([_i] * 7, _sz),
+    "kda_gdn_chunk_fwd": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_gdn_decode_step": ([_vp] * 7 + [_i] * 5 + [_vp], _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
@@ -228,6 +232,29 @@ def kda_chunk_split_chain(v, initial_state, cu_seqlens, B, T, num_seqs, H, o, fi
                                       num_seqs, H, _p(o), _p(final_state), _p(workspace), wb,
                                       _stream(stream))
     return _ret(st, "kda_chunk_split_chain", check)
+
+
+def kda_gdn_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype) -> int:
+    return int(load().kda_gdn_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk,
+                                                       dtype_code(dtype)))
+
+
+def kda_gdn_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H, dk, dv,
+                      chunk, dtype, o, final_state, workspace, workspace_bytes=None, stream=None,
+                      check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
+                                  _p(cu_seqlens), B, T, num_seqs, H, dk, dv, chunk,
+                                  dtype_code(dtype), _p(o), _p(final_state), _p(workspace), wb,
+                                  _stream(stream))
+    return _ret(st, "kda_gdn_chunk_fwd", check)
+
+
+def kda_gdn_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,
+                        check=True) -> int:
+    st = load().kda_gdn_decode_step(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state), _p(o), N,
+                                    H, dk, dv, dtype_code(dtype), _stream(stream))
+    return _ret(st, "kda_gdn_decode_step", check)
 
 
 def kda_qkv_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens, B, T, num_seqs, H, dk, dv, dtype,

@@ -244,6 +244,33 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
                              const float* beta, float* state, void* o, int N, int H, int dk,
                              int dv, kda_dtype_t dtype, void* stream);
 
+/* ------------------------------- Gated DeltaNet: one gate value per head
+ * Kimi Linear (aiwiki.ai), "Background: from the delta rule to gated
+ * DeltaNet": the recurrence with a head-uniform gate alpha_t (one value per
+ * (token, head)) instead of KDA's per-channel one; DeltaNet is the case
+ * g = 0.  Same arguments, layouts, plans' kernels and error behaviour as
+ * kda_chunk_fwd / kda_decode_step, except:
+ *   g [total, H] fp32 (prefill), [N, H] fp32 (decode) -- log alpha per (token,
+ *   head); the workspace is kda_gdn_chunk_fwd_workspace_size() bytes.
+ * bf16, dk = dv = 128, chunk 64 runs the split tensor-core plan with the gate
+ * read per (token, head) (one exponential per row instead of per element);
+ * other shapes spread g over the dk channels in the workspace and run the
+ * CUDA-core plan.  KDA_CHUNK_PATH=simt forces the latter.
+ */
+size_t kda_gdn_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
+                                        int chunk, kda_dtype_t dtype);
+
+kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* initial_state,
+                               const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                               int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                               float* final_state, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+kda_status_t kda_gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, float* state, void* o, int N, int H, int dk,
+                                 int dv, kda_dtype_t dtype, void* stream);
+
 /* ---------------------------------------- the steps around the operator
  * Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
  * algorithm" (the paragraph on what each KDA head applies): a short depthwise

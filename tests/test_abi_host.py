@@ -172,3 +172,22 @@ def test_layer_calls_reject_bad_arguments(lib):
     assert kda.kda_output_norm_gate(**{**gate, "total_tokens": -1}) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_output_norm_gate(**{**gate, "dv": 48}) == kda.KDA_ERR_UNSUPPORTED
     assert kda.kda_output_norm_gate(**{**gate, "eps": -1.0}) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_gdn_calls_reject_bad_arguments(lib):
+    f = kda.kda_gdn_chunk_fwd_workspace_size
+    assert f(4096, 2, 32, 128, 128, 64, "bf16") >= kda.kda_chunk_fwd_workspace_size(
+        4096, 2, 32, 128, 128, 64, "bf16")
+    assert f(64, 1, 1, 48, 32, 16, "f32") == 0
+    args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, initial_state=None, cu_seqlens=None,
+                B=1, T=64, num_seqs=1, H=1, dk=32, dv=32, chunk=16, dtype="f32", o=FAKE,
+                final_state=None, workspace=FAKE * 2, workspace_bytes=16, stream=0, check=False)
+    assert kda.kda_gdn_chunk_fwd(**{**args, "g": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_gdn_chunk_fwd(**{**args, "beta": FAKE + 4}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_gdn_chunk_fwd(**{**args, "dk": 96}) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_gdn_chunk_fwd(**args) == kda.KDA_ERR_WORKSPACE       # 16 bytes
+    dec = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, state=FAKE, o=FAKE, N=2, H=2, dk=128,
+               dv=128, dtype="bf16", stream=0, check=False)
+    assert kda.kda_gdn_decode_step(**{**dec, "state": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_gdn_decode_step(**{**dec, "dv": 40}) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_gdn_decode_step(**{**dec, "N": 0}) == kda.KDA_OK
