@@ -1,0 +1,136 @@
+"""Context-parallel prefill (gated_delta_rule_124_b200.context_parallel): the
+exchange and the affine fold, with 2 gloo ranks on the CPU and the fp64 oracle
+as each rank's local prefill; on the GPU (marked) the same fold with the
+library's kernels over simulated ranks, and the chunked-prefill -> decode
+state hand-off."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from gated_delta_rule_124_b200 import context_parallel as cp
+from gated_delta_rule_124_b200 import workloads as wl
+from tests.helpers import rel_err
+
+
+def _oracle_prefill(q, k, v, g, beta, initial_state):
+    """fp64 oracle as the per-rank prefill (CPU tensors in, float32 out)."""
+    o, hN = oracle.forward(q, k, v, g, beta, initial_state)
+    return torch.from_numpy(o).float(), torch.from_numpy(hN).float()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _case(T=96, B=2, H=2, d=16, seed=21):
+    c = wl.make_prefill(seed, [T] * B, H=H, dk=d, dv=d, chunk=16, dtype="f32")
+    sh = lambda x, last: x.reshape(B, T, H, *last)  # noqa: E731
+    return (c, sh(c.q, (d,)), sh(c.k, (d,)), sh(c.v, (d,)), sh(c.g, (d,)), sh(c.beta, ()),
+            c.initial_state)
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        c, q, k, v, g, beta, h0 = _case()
+        T = q.shape[1]
+        a, b = rank * T // world, (rank + 1) * T // world
+        o, hN = cp.context_parallel_prefill(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b],
+                                            beta[:, a:b], h0, prefill=_oracle_prefill)
+        out[rank] = (o.numpy(), hN.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_gloo_match_the_whole_sequence():
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_worker, args=(2, _free_port(), out), nprocs=2, join=True)
+    c, q, k, v, g, beta, h0 = _case()
+    ro, rh = oracle.forward(q, k, v, g, beta, h0)
+    o = np.concatenate([out[0][0], out[1][0]], axis=1)
+    assert rel_err(o, ro) <= 1e-5
+    for r in range(2):
+        assert rel_err(out[r][1], rh) <= 1e-5
+
+
+def test_fold_of_segment_maps_is_the_recurrence():
+    """entry_states over oracle-computed maps reproduces the states at the
+    segment boundaries (pure host arithmetic)."""
+    c, q, k, v, g, beta, h0 = _case(T=60)
+    cuts = [0, 13, 40, 60]
+    maps = [cp.segment_maps(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b], beta[:, a:b],
+                            _oracle_prefill) for a, b in zip(cuts, cuts[1:])]
+    entries, final = cp.entry_states(maps, h0)
+    for i, a in enumerate(cuts[:-1]):
+        if a == 0:
+            ref = h0.numpy()
+        else:
+            _, ref = oracle.forward(q[:, :a], k[:, :a], v[:, :a], g[:, :a], beta[:, :a], h0)
+        assert rel_err(entries[i], ref) <= 1e-5
+    _, rh = oracle.forward(q, k, v, g, beta, h0)
+    assert rel_err(final, rh) <= 1e-5
+
+
+@pytest.mark.gpu
+def test_simulated_ranks_on_the_gpu():
+    """Four segments of one 1024-token sequence through the library's kernels:
+    maps, fold, finishing prefills."""
+    c = wl.make_prefill(22, [1024, 1024], H=4, dk=128, dv=128, chunk=64, dtype="bf16")
+    B, T, H, d = 2, 1024, 4, 128
+    sh = lambda x, last: x.reshape(B, T, H, *last).cuda()  # noqa: E731
+    q, k, v, g = (sh(x, (d,)) for x in (c.q, c.k, c.v, c.g))
+    beta, h0 = sh(c.beta, ()), c.initial_state.cuda()
+    cuts = [0, 320, 512, 900, 1024]
+    segs = list(zip(cuts, cuts[1:]))
+    maps = [cp.segment_maps(q[:, a:b].contiguous(), k[:, a:b].contiguous(),
+                            v[:, a:b].contiguous(), g[:, a:b].contiguous(),
+                            beta[:, a:b].contiguous()) for a, b in segs]
+    entries, final = cp.entry_states(maps, h0)
+    outs = []
+    for (a, b), s_in in zip(segs, entries):
+        o, _ = cp._library_prefill(q[:, a:b].contiguous(), k[:, a:b].contiguous(),
+                                   v[:, a:b].contiguous(), g[:, a:b].contiguous(),
+                                   beta[:, a:b].contiguous(), s_in.contiguous())
+        outs.append(o)
+    o = torch.cat(outs, dim=1)
+    ro, rh = oracle.forward(c.q.reshape(B, T, H, d), c.k.reshape(B, T, H, d),
+                            c.v.reshape(B, T, H, d), c.g.reshape(B, T, H, d),
+                            c.beta.reshape(B, T, H), c.initial_state)
+    assert rel_err(o, ro) <= 2e-2 and rel_err(final, rh) <= 2e-2
+
+
+@pytest.mark.gpu
+def test_chunked_prefill_then_decode_hands_the_state_over():
+    """Prefill in three pieces (each from the previous piece's final state),
+    then decode steps on that state: the same as the oracle's one pass."""
+    import gated_delta_rule_124_b200 as kda
+    T, H, d = 300, 2, 128
+    c = wl.make_prefill(23, [T + 5], H=H, dk=d, dv=d, chunk=64, dtype="bf16")
+    cd = c.to("cuda")
+    state = cd.initial_state
+    outs = []
+    for a, b in ((0, 77), (77, 200), (200, T)):
+        sl = lambda x: x[a:b].unsqueeze(0).clone()  # noqa: E731  (16-byte aligned copies)
+        o, state = kda.chunk_fwd(sl(cd.q), sl(cd.k), sl(cd.v), sl(cd.g), sl(cd.beta),
+                                 initial_state=state)
+        outs.append(o[0])
+    dec = []
+    for t in range(T, T + 5):
+        one = lambda x: x[t:t + 1].clone()  # noqa: E731
+        dec.append(kda.decode_step(one(cd.q), one(cd.k), one(cd.v), one(cd.g), one(cd.beta),
+                                   state)[0])
+    torch.cuda.synchronize()
+    ro, rh = oracle.forward(c.q, c.k, c.v, c.g, c.beta, c.initial_state)
+    assert rel_err(torch.cat(outs), ro[:T]) <= 2e-2
+    assert rel_err(torch.stack(dec), ro[T:]) <= 2e-2
+    assert rel_err(state[0], rh[0]) <= 2e-2
