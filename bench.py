@@ -42,16 +42,13 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (kernel, workload).  Reported only while the kernel's source still matches the
 # capture; null once it has changed, or for a workload never captured.
 _SPLIT = "gated_delta_rule_124_b200/csrc/kda_chunk_split.cu"
-_DECODE = "gated_delta_rule_124_b200/csrc/kda_decode.cu"
 _CFG1 = "prefill: B=2 H=32 T=2048 d=128 C=64 bf16"
 _CFG2 = "long prefill: B=1 H=32 T=65536 d=128 C=64 bf16 slow decay"
 MEASURED_TRAFFIC = {
-    ("split_intra", _CFG1): (_SPLIT, "fccfa1570cf3f515e90f73c0520ccbc607782efd", 222402304),
-    ("split_chain", _CFG1): (_SPLIT, "fccfa1570cf3f515e90f73c0520ccbc607782efd", 196509184),
+    ("split_intra", _CFG1): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 222362880),
+    ("split_chain", _CFG1): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 195830272),
     # captured on B=1 x T=16384 (a quarter of the tokens) and scaled by 4
-    ("chunk_fwd_overlap", _CFG2): (_SPLIT, "fccfa1570cf3f515e90f73c0520ccbc607782efd", 5244939264),
-    ("decode", "decode: N=256 H=32 d=128 bf16, fp32 state, 8 input sets cycled"):
-        (_DECODE, "74d4998613be6f444437ae56cfccf2e33f395ce8", 1028657152),
+    ("chunk_fwd_overlap", _CFG2): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 5597298688),
 }
 
 
