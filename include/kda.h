@@ -271,6 +271,36 @@ kda_status_t kda_gdn_decode_step(const void* q, const void* k, const void* v, co
                                  const float* beta, float* state, void* o, int N, int H, int dk,
                                  int dv, kda_dtype_t dtype, void* stream);
 
+/* ----------------------------------------------------------------- backward
+ * kda_chunk_bwd: gradients of L = sum(o * dout) + sum(final_state *
+ * dfinal_state) for the forward kda_chunk_fwd computes (same inputs, shapes
+ * and sequence description), with respect to q, k, v, g, beta and the
+ * initial state.  The pages give no backward equations; they are derived from
+ * the token recurrence (Kimi Linear (aiwiki.ai), "Kimi Delta Attention") and
+ * evaluated recurrently, token by token, one CTA per (sequence, head, 32 value
+ * columns), with the states rebuilt from checkpoints every 8 tokens kept in
+ * the workspace: correct, and much slower than the forward.
+ * In:  q, k [total, H, dk], v [total, H, dv], dout [total, H, dv] (dtype);
+ *      g [total, H, dk], beta [total, H] fp32; initial_state [num_seqs, H, dk,
+ *      dv] fp32 or NULL (zeros); dfinal_state likewise or NULL (zeros).
+ * Out: dq, dk [total, H, dk], dv [total, H, dv], dg [total, H, dk], dbeta
+ *      [total, H] -- all fp32; dinitial_state [num_seqs, H, dk, dv] fp32 or
+ *      NULL (not written).
+ * Workspace: kda_chunk_bwd_workspace_size() bytes, 256-byte aligned (the
+ *      checkpoints: about total * H * dk * dv / 2 bytes, plus per-slice
+ *      partial sums).  Shapes: dk, dv in {32, 64, 128}.  cu_seqlens must be
+ *      valid (0 .. T, non-decreasing): it is not checked on the device here.
+ */
+size_t kda_chunk_bwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv);
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* initial_state, const void* dout,
+                           const float* dfinal_state, const int32_t* cu_seqlens, int B, int T,
+                           int num_seqs, int H, int dk, int dv, kda_dtype_t dtype, float* dq,
+                           float* dk_out, float* dv_out, float* dg, float* dbeta,
+                           float* dinitial_state, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* ---------------------------------------- the steps around the operator
  * Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
  * algorithm" (the paragraph on what each KDA head applies): a short depthwise
