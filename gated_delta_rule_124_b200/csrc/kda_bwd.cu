@@ -1,25 +1,28 @@
-// KDA backward (gradients of the chunkwise forward's outputs), recurrent form.
+// KDA backward (gradients of the chunkwise prefill), chunked form on CUDA cores.
 //
-// The pages give no backward equations; these are derived from the forward
-// step (Kimi Linear (aiwiki.ai), "Kimi Delta Attention"):
-//   S_bar = Diag(alpha) S_prev,  w = S_bar^T k,  u = beta (v - w),
-//   S = S_bar + k u^T,  o = S^T q,  alpha = exp(g).
-// Going backwards over the tokens with dS the gradient of the state after the
-// token:
-//   dS += q do^T;  dq = S do;  du = dS^T k;  dk = dS u + S_bar dw;
-//   dv = beta du;  dbeta = du . (v - w);  dw = -beta du;
-//   dS_bar = dS + k dw^T;  dg = alpha * rowsum(dS_bar * S_prev);
-//   dS <- Diag(alpha) dS_bar;  after the first token dS is d initial_state.
-//
-// One CTA of 256 threads per (sequence, head, 32 value columns): the columns
-// of a state evolve independently, so a slice needs only its own columns,
-// while dq, dk, dg and dbeta sum over all columns -- each slice writes its
-// partial sums and a second kernel adds the slices.  The states the backward
-// sweep needs (S before each token) are rebuilt: a forward sweep stores the
-// state every 8 tokens in the workspace, and each 8-token block is rebuilt
-// from its checkpoint into shared memory before it is walked backwards.  This
-// is the plain recurrent form: correct, and far slower than the forward's
-// chunked tensor-core form.
+// The pages give no backward equations; these follow from the chunk form of
+// Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
+// algorithm".  Per (sequence, head) and chunk of C tokens with entry state S,
+// G the inclusive cumulative sum of g inside the chunk and Gam = exp(G_last):
+//   A[r][i] = b_r sum_c k_rc k_ic exp(G_rc - G_ic)   (i < r),  T = (I + A)^-1
+//   P[r][i] = sum_c q_rc k_ic exp(G_rc - G_ic)       (i <= r)
+//   W = T diag(b) (K * exp(G)),  Ut = T diag(b) V,  U = Ut - W S
+//   O = (Q * exp(G)) S + P U,    S' = Diag(Gam) S + (K * exp(G_last - G))^T U
+// Going backwards with dS' the gradient of the exit state and dO of the
+// chunk's outputs (Qt = Q * exp(G), Kt = K * exp(G), Kb = K * exp(G_last - G)):
+//   E  = P^T dO,  F = Qt^T dO - W^T E                              (b1 prep)
+//   X  = Kb dS',  dU = E + X,  dS = Diag(Gam) dS' - W^T X + F      (b2 chain)
+//   Y  = T^T dU (back substitution),  dv = b Y,
+//   dA = -strict_lower(Y U^T),  dP = lower(dO U^T)                 (b3 solve)
+//   dQt = dO S^T,  dKt = -b (Y S^T),  dKb = U dS'^T,
+//   dbeta = Y.V + sum_i dA[r][i] A[r][i] / b_r - Kt.(Y S^T)         (b4 dense)
+//   then the pair sums over (r, i, c) of A and P give dq, dk and dG, and
+//   dg is the reverse cumulative sum of dG inside the chunk          (b5 pairs)
+// The gradient of T = (I + A)^-1 never appears on its own: T^T dT T^T reduces
+// to Y U^T because the gradient reaching W is -dU S^T.  The forward half (G,
+// W, U and the entry state of every chunk) is the CUDA-core prefill's own
+// a1 .. a3.  Every exponent is a difference exp(G_r - G_i) with i <= r, so
+// never positive for g <= 0; all arithmetic is fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -29,317 +32,615 @@
 namespace kda {
 namespace {
 
-constexpr int NTB = 256;  // threads
-constexpr int DVS = 32;   // value columns per CTA
-constexpr int SB = 8;     // tokens per checkpoint block
+constexpr int CB = 64;   // chunk length of the backward
+constexpr int DVS = 32;  // value columns per slice
 
-// Thread (warp w, lane l) holds float4 column group c4 = l & 7 of rows
-// p * 32 + w * 4 + (l >> 3), p < DK / 32.
-template <int DK>
-struct Layout {
-    static constexpr int NP = DK / 32;
-    __device__ static int row(int p, int warp, int lane) { return p * 32 + warp * 4 + (lane >> 3); }
+struct BwdBufs {
+    Workspace w;
+    float* E;     // [total, H, dv]
+    float* dU;    // [total, H, dv]
+    float* Y;     // [total, H, dv]
+    float* F;     // [maxc, H, dk, dv]
+    float* dSx;   // [maxc, H, dk, dv]   gradient of each chunk's exit state
+    float* dAr;   // [maxc, H, C, C]     b_r dA[r][i]
+    float* dP;    // [maxc, H, C, C]
+    float* dQt;   // [total, H, dk]
+    float* dKt;   // [total, H, dk]
+    float* dKb;   // [total, H, dk]
+    float* dGam;  // [maxc, H, dk]
+    float* dbB;   // [total, H]
+    size_t bytes;
 };
 
-__device__ __forceinline__ float4 f4(float a) { return make_float4(a, a, a, a); }
-__device__ __forceinline__ float dot4(float4 a, float4 b) {
-    return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
-}
-// sum over the 8 lanes that hold one row (lanes of equal l >> 3)
-__device__ __forceinline__ float row_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    return x;
+BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
+    BwdBufs b{};
+    b.w = carve(base, total, N, H, dk, dv, CB, true);
+    const size_t maxc = (size_t)max_chunks(total, N, CB);
+    char* p = static_cast<char*>(base);
+    size_t off = b.w.total_bytes;
+    auto take = [&](size_t floats) {
+        float* r = reinterpret_cast<float*>(p + off);
+        off = align_up(off + floats * sizeof(float));
+        return r;
+    };
+    const size_t tv = (size_t)total * H * dv, tk = (size_t)total * H * dk;
+    const size_t cs = maxc * H * dk * dv, cc = maxc * H * CB * CB;
+    b.E = take(tv);
+    b.dU = take(tv);
+    b.Y = take(tv);
+    b.F = take(cs);
+    b.dSx = take(cs);
+    b.dAr = take(cc);
+    b.dP = take(cc);
+    b.dQt = take(tk);
+    b.dKt = take(tk);
+    b.dKb = take(tk);
+    b.dGam = take(maxc * H * dk);
+    b.dbB = take((size_t)total * H);
+    b.bytes = off;
+    return b;
 }
 
-struct BwdParams {
-    const void* q;
-    const void* k;
-    const void* v;
-    const float* g;
-    const float* beta;
-    const float* h0;
-    const void* dout;
-    const float* dhT;
-    const int32_t* cu;
-    int T, N, H, DV, total;
-    float* ckpt;   // [total / SB + N + 1][H][DK][DV]
-    float* dq_p;   // [slices][total][H][DK]
-    float* dk_p;
-    float* dg_p;
-    float* db_p;   // [slices][total][H]
-    float* dv;     // [total][H][DV]
-    float* dh0;    // [N][H][DK][DV] (may be NULL)
-};
-
+// ------------------------------------------------------------ b1: prep
+// One block per (chunk, head).  Shared: Qt, K, G, W [C][dk+1], P [C][C+1],
+// dO and E slices [C][DVS+1].
 template <typename TIn>
-__device__ __forceinline__ float ld(const TIn* p, size_t i) {
-    return to_f32(p[i]);
-}
-
-template <int DK, typename TIn>
-__global__ void __launch_bounds__(NTB, 1) bwd_kernel(const BwdParams p) {
-    using Lo = Layout<DK>;
-    constexpr int NP = Lo::NP;
-    extern __shared__ float4 smem_f4[];
-    float4* sbuf = smem_f4;  // [SB][DK][8] float4: the state before each token of a block
-    __shared__ float s_q[DK], s_k[DK], s_a[DK];
-    __shared__ float s_v[DVS], s_do[DVS], s_col[DVS], s_du[DVS];
-    __shared__ float4 s_red[8][8];
-    __shared__ float s_beta;
-
-    const int unit = blockIdx.x, slice = blockIdx.y;
-    const int seq = unit / p.H, h = unit % p.H;
-    const int j0 = slice * DVS;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, c4 = lane & 7;
-    const int t_begin = p.cu ? p.cu[seq] : seq * p.T;
-    const int t_end = p.cu ? p.cu[seq + 1] : (seq + 1) * p.T;
-    const int nslice = p.DV / DVS;
-    const TIn* Q = static_cast<const TIn*>(p.q);
-    const TIn* K = static_cast<const TIn*>(p.k);
-    const TIn* V = static_cast<const TIn*>(p.v);
-    const TIn* DO = static_cast<const TIn*>(p.dout);
-
-    auto state_ptr = [&](float* base, size_t block) {  // float4 row starts of this slice
-        return reinterpret_cast<float4*>(base + ((block * p.H + h) * DK) * p.DV + j0);
-    };
-    // token t's vectors into shared memory (q, k, alpha over DK; v, do over the slice)
-    auto load_token = [&](int t, bool with_do) {
-        const size_t bk = ((size_t)t * p.H + h) * DK;
-        for (int c = tid; c < DK; c += NTB) {
-            s_q[c] = ld(Q, bk + c);
-            s_k[c] = ld(K, bk + c);
-            s_a[c] = expf(p.g[bk + c]);
-        }
-        if (tid < DVS) {
-            const size_t bv = ((size_t)t * p.H + h) * p.DV + j0 + tid;
-            s_v[tid] = ld(V, bv);
-            s_do[tid] = with_do ? ld(DO, bv) : 0.f;
-        }
-        if (tid == 0) s_beta = p.beta[(size_t)t * p.H + h];
-        __syncthreads();
-    };
-    // column sums over the DK rows of x (one value per row of this thread's
-    // float4 group, weighted by wrow[p]) -> s_out[32]
-    auto col_sum = [&](const float4 (&x)[NP], const float (&wrow)[NP], float* s_out) {
-        float4 acc = f4(0.f);
-#pragma unroll
-        for (int i = 0; i < NP; ++i) {
-            acc.x += x[i].x * wrow[i]; acc.y += x[i].y * wrow[i];
-            acc.z += x[i].z * wrow[i]; acc.w += x[i].w * wrow[i];
-        }
-#pragma unroll
-        for (int o = 8; o < 32; o <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
-        }
-        if (lane < 8) s_red[warp][c4] = acc;
-        __syncthreads();
-        if (tid < 8) {
-            float4 s = f4(0.f);
-#pragma unroll
-            for (int w2 = 0; w2 < 8; ++w2) {
-                const float4 y = s_red[w2][tid];
-                s.x += y.x; s.y += y.y; s.z += y.z; s.w += y.w;
-            }
-            s_out[4 * tid] = s.x; s_out[4 * tid + 1] = s.y;
-            s_out[4 * tid + 2] = s.z; s_out[4 * tid + 3] = s.w;
-        }
-        __syncthreads();
-    };
-    // one forward step on S (registers): S <- Diag(a) S + k (beta (v - S_bar^T k))^T
-    auto forward_step = [&](float4 (&S)[NP]) {
-        float kr[NP];
-#pragma unroll
-        for (int i = 0; i < NP; ++i) {
-            const int r = Lo::row(i, warp, lane);
-            const float a = s_a[r];
-            S[i].x *= a; S[i].y *= a; S[i].z *= a; S[i].w *= a;
-            kr[i] = s_k[r];
-        }
-        col_sum(S, kr, s_col);  // w
-        const float b = s_beta;
-        const float4 u = make_float4(b * (s_v[4 * c4] - s_col[4 * c4]),
-                                     b * (s_v[4 * c4 + 1] - s_col[4 * c4 + 1]),
-                                     b * (s_v[4 * c4 + 2] - s_col[4 * c4 + 2]),
-                                     b * (s_v[4 * c4 + 3] - s_col[4 * c4 + 3]));
-#pragma unroll
-        for (int i = 0; i < NP; ++i) {
-            S[i].x += kr[i] * u.x; S[i].y += kr[i] * u.y;
-            S[i].z += kr[i] * u.z; S[i].w += kr[i] * u.w;
-        }
-    };
-
-    // ---------------- forward sweep: a checkpoint every SB tokens
-    float4 S[NP];
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-        const int r = Lo::row(i, warp, lane);
-        S[i] = p.h0 ? reinterpret_cast<const float4*>(
-                          p.h0 + (((size_t)seq * p.H + h) * DK + r) * p.DV + j0)[c4]
-                    : f4(0.f);
-    }
-    const size_t blk0 = (size_t)(t_begin / SB) + seq;
-    for (int t = t_begin; t < t_end; ++t) {
-        if ((t - t_begin) % SB == 0) {
-            float4* dst = state_ptr(p.ckpt, blk0 + (t - t_begin) / SB);
-#pragma unroll
-            for (int i = 0; i < NP; ++i)
-                dst[(size_t)Lo::row(i, warp, lane) * (p.DV / 4) + c4] = S[i];
-        }
-        load_token(t, false);
-        forward_step(S);
-        __syncthreads();
+__global__ void __launch_bounds__(256) bwd_prep_kernel(
+    const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ dout,
+    const float* __restrict__ G, const float* __restrict__ W, const int4* __restrict__ info,
+    int H, int dk, int dv, const uint32_t* status, float* __restrict__ E,
+    float* __restrict__ F) {
+    if (status_bad(status)) return;
+    const int cidx = blockIdx.x, h = blockIdx.y;
+    const int4 ci = info[cidx];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    extern __shared__ float sm[];
+    const int ldk = dk + 1, lda = CB + 1, lds = DVS + 1;
+    float* Qs = sm;
+    float* Ks = Qs + CB * ldk;
+    float* Gs = Ks + CB * ldk;
+    float* Ws = Gs + CB * ldk;
+    float* Ps = Ws + CB * ldk;
+    float* Ds = Ps + CB * lda;
+    float* Es = Ds + CB * lds;
+    for (int idx = tid; idx < L * dk; idx += nt) {
+        const int r = idx / dk, c = idx % dk;
+        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
+        Qs[r * ldk + c] = to_f32(q[gi]);
+        Ks[r * ldk + c] = to_f32(k[gi]);
+        Gs[r * ldk + c] = G[gi];
+        Ws[r * ldk + c] = W[gi];
     }
     __syncthreads();
-
-    // ---------------- backward sweep, block by block
-    float4 dS[NP];
-#pragma unroll
-    for (int i = 0; i < NP; ++i) {
-        const int r = Lo::row(i, warp, lane);
-        dS[i] = p.dhT ? reinterpret_cast<const float4*>(
-                            p.dhT + (((size_t)seq * p.H + h) * DK + r) * p.DV + j0)[c4]
-                      : f4(0.f);
-    }
-    const int nblk = (t_end - t_begin + SB - 1) / SB;
-    for (int bi = nblk - 1; bi >= 0; --bi) {
-        const int t0 = t_begin + bi * SB, cnt = min(SB, t_end - t0);
-        // rebuild the block's states from its checkpoint
-        const float4* src = state_ptr(p.ckpt, blk0 + bi);
-#pragma unroll
-        for (int i = 0; i < NP; ++i) S[i] = src[(size_t)Lo::row(i, warp, lane) * (p.DV / 4) + c4];
-        for (int i = 0; i < cnt; ++i) {
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp)
-                sbuf[((size_t)i * DK + Lo::row(pp, warp, lane)) * 8 + c4] = S[pp];
-            if (i + 1 < cnt) {
-                load_token(t0 + i, false);
-                forward_step(S);
-                __syncthreads();
-            }
+    for (int idx = tid; idx < L * L; idx += nt) {
+        const int r = idx / L, i = idx % L;
+        float acc = 0.f;
+        if (i <= r) {
+            const float* qr = Qs + r * ldk;
+            const float* ki = Ks + i * ldk;
+            const float* gr = Gs + r * ldk;
+            const float* gi = Gs + i * ldk;
+            for (int c = 0; c < dk; ++c) acc += qr[c] * ki[c] * expf(gr[c] - gi[c]);
         }
-        // walk it backwards
-        for (int i = cnt - 1; i >= 0; --i) {
-            const int t = t0 + i;
-            load_token(t, true);
-            float4 Sp[NP], Sb[NP], St[NP];
-            float kr[NP], qr[NP], ar[NP];
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp) {
-                const int r = Lo::row(pp, warp, lane);
-                Sp[pp] = sbuf[((size_t)i * DK + r) * 8 + c4];
-                ar[pp] = s_a[r];
-                kr[pp] = s_k[r];
-                qr[pp] = s_q[r];
-                Sb[pp] = make_float4(Sp[pp].x * ar[pp], Sp[pp].y * ar[pp], Sp[pp].z * ar[pp],
-                                     Sp[pp].w * ar[pp]);
-            }
-            col_sum(Sb, kr, s_col);  // w
-            const float b = s_beta;
-            const float4 w = make_float4(s_col[4 * c4], s_col[4 * c4 + 1], s_col[4 * c4 + 2],
-                                         s_col[4 * c4 + 3]);
-            const float4 vv = make_float4(s_v[4 * c4], s_v[4 * c4 + 1], s_v[4 * c4 + 2],
-                                          s_v[4 * c4 + 3]);
-            const float4 u = make_float4(b * (vv.x - w.x), b * (vv.y - w.y), b * (vv.z - w.z),
-                                         b * (vv.w - w.w));
-            const float4 dov = make_float4(s_do[4 * c4], s_do[4 * c4 + 1], s_do[4 * c4 + 2],
-                                           s_do[4 * c4 + 3]);
-            const size_t part = ((size_t)slice * p.total + t) * p.H + h;
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp) {
-                St[pp] = make_float4(Sb[pp].x + kr[pp] * u.x, Sb[pp].y + kr[pp] * u.y,
-                                     Sb[pp].z + kr[pp] * u.z, Sb[pp].w + kr[pp] * u.w);
-                dS[pp].x += qr[pp] * dov.x; dS[pp].y += qr[pp] * dov.y;
-                dS[pp].z += qr[pp] * dov.z; dS[pp].w += qr[pp] * dov.w;
-                const float dq = row_sum(dot4(St[pp], dov));
-                if (c4 == 0) p.dq_p[part * DK + Lo::row(pp, warp, lane)] = dq;
-            }
-            col_sum(dS, kr, s_du);  // du
-            const float4 du = make_float4(s_du[4 * c4], s_du[4 * c4 + 1], s_du[4 * c4 + 2],
-                                          s_du[4 * c4 + 3]);
-            if (tid < DVS)
-                p.dv[((size_t)t * p.H + h) * p.DV + j0 + tid] = b * s_du[tid];
-            if (warp == 0) {  // this slice's part of dbeta
-                float x = lane < DVS ? s_du[lane] * (s_v[lane] - s_col[lane]) : 0.f;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                if (lane == 0) p.db_p[part] = x;
-            }
-            const float4 dw = make_float4(-b * du.x, -b * du.y, -b * du.z, -b * du.w);
-#pragma unroll
-            for (int pp = 0; pp < NP; ++pp) {
-                const int r = Lo::row(pp, warp, lane);
-                const float dk = row_sum(dot4(dS[pp], u) + dot4(Sb[pp], dw));
-                const float4 dSb = make_float4(dS[pp].x + kr[pp] * dw.x, dS[pp].y + kr[pp] * dw.y,
-                                               dS[pp].z + kr[pp] * dw.z, dS[pp].w + kr[pp] * dw.w);
-                const float da = row_sum(dot4(dSb, Sp[pp]));
-                if (c4 == 0) {
-                    p.dk_p[part * DK + r] = dk;
-                    p.dg_p[part * DK + r] = ar[pp] * da;
-                }
-                dS[pp] = make_float4(ar[pp] * dSb.x, ar[pp] * dSb.y, ar[pp] * dSb.z,
-                                     ar[pp] * dSb.w);
-            }
-            __syncthreads();
+        Ps[r * lda + i] = acc;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < L * dk; idx += nt) {
+        const int r = idx / dk, c = idx % dk;
+        Qs[r * ldk + c] *= expf(Gs[r * ldk + c]);
+    }
+    float* Fc = F + ((size_t)cidx * H + h) * dk * dv;
+    for (int j0 = 0; j0 < dv; j0 += DVS) {
+        __syncthreads();
+        for (int idx = tid; idx < L * DVS; idx += nt) {
+            const int r = idx / DVS, j = idx % DVS;
+            Ds[r * lds + j] = to_f32(dout[((size_t)(ci.y + r) * H + h) * dv + j0 + j]);
+        }
+        __syncthreads();
+        // E[i][j] = sum_{r >= i} P[r][i] dO[r][j]
+        for (int idx = tid; idx < L * DVS; idx += nt) {
+            const int i = idx / DVS, j = idx % DVS;
+            float acc = 0.f;
+            for (int r = i; r < L; ++r) acc += Ps[r * lda + i] * Ds[r * lds + j];
+            Es[i * lds + j] = acc;
+            E[((size_t)(ci.y + i) * H + h) * dv + j0 + j] = acc;
+        }
+        __syncthreads();
+        // F[c][j] = sum_r Qt[r][c] dO[r][j] - W[r][c] E[r][j]
+        for (int idx = tid; idx < dk * DVS; idx += nt) {
+            const int c = idx / DVS, j = idx % DVS;
+            float acc = 0.f;
+            for (int r = 0; r < L; ++r)
+                acc += Qs[r * ldk + c] * Ds[r * lds + j] - Ws[r * ldk + c] * Es[r * lds + j];
+            Fc[(size_t)c * dv + j0 + j] = acc;
         }
     }
-    if (p.dh0) {
-#pragma unroll
-        for (int i = 0; i < NP; ++i) {
-            const int r = Lo::row(i, warp, lane);
-            reinterpret_cast<float4*>(p.dh0 + (((size_t)seq * p.H + h) * DK + r) * p.DV + j0)[c4] =
-                dS[i];
-        }
-    }
-    (void)nslice;
 }
 
-// dq, dk, dg [total, H, DK] and dbeta [total, H]: the slices' partial sums added.
-__global__ void bwd_reduce_kernel(const float* __restrict__ dq_p, const float* __restrict__ dk_p,
-                                  const float* __restrict__ dg_p, const float* __restrict__ db_p,
-                                  int nslice, long long rows, int DK, float* dq, float* dk,
-                                  float* dg, float* db) {
-    const long long n = rows * DK;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (long long)gridDim.x * blockDim.x) {
-        float a = 0.f, b = 0.f, c = 0.f;
-        for (int s = 0; s < nslice; ++s) {
-            a += dq_p[s * n + i];
-            b += dk_p[s * n + i];
-            c += dg_p[s * n + i];
+size_t prep_smem(int dk) {
+    return sizeof(float) * ((size_t)4 * CB * (dk + 1) + (size_t)CB * (CB + 1) +
+                            (size_t)2 * CB * (DVS + 1));
+}
+
+// ------------------------------------------------------------ b2: chain
+// One block per (sequence, head, dv slice), serial over the chunks from the
+// last.  Shared: dS [dk][DVS], W and Kb [C][dk+1], X [C][DVS+1], Gam [dk].
+template <typename TIn>
+__global__ void __launch_bounds__(256) bwd_chain_kernel(
+    const TIn* __restrict__ k, const float* __restrict__ G, const float* __restrict__ W,
+    const float* __restrict__ E, const float* __restrict__ F, const float* __restrict__ dhT,
+    const int32_t* __restrict__ cu, int T, const int* __restrict__ chunk_start, int H, int dk,
+    int dv, const uint32_t* status, float* __restrict__ dU, float* __restrict__ dSx,
+    float* __restrict__ dh0) {
+    if (status_bad(status)) return;
+    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVS;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int t_begin = cu ? cu[s] : s * T;
+    const int t_end = cu ? cu[s + 1] : (s + 1) * T;
+    extern __shared__ float sm[];
+    const int ldk = dk + 1, ldx = DVS + 1;
+    float* dS = sm;                // [dk][DVS]
+    float* Ws = dS + dk * DVS;     // [C][ldk]
+    float* Kb = Ws + CB * ldk;     // [C][ldk]
+    float* Xs = Kb + CB * ldk;     // [C][ldx]
+    float* eGl = Xs + CB * ldx;    // [dk]
+    const size_t st_base = ((size_t)s * H + h) * dk * dv;
+    for (int idx = tid; idx < dk * DVS; idx += nt) {
+        const int c = idx / DVS, j = idx % DVS;
+        dS[idx] = dhT ? dhT[st_base + (size_t)c * dv + j0 + j] : 0.f;
+    }
+    const int nch = (t_end - t_begin + CB - 1) / CB;
+    for (int n = nch - 1; n >= 0; --n) {
+        const int t0 = t_begin + n * CB;
+        const int L = min(CB, t_end - t0);
+        const size_t cs = (size_t)chunk_start[s] + n;
+        const size_t cbase = (cs * H + h) * dk * dv;
+        __syncthreads();
+        for (int idx = tid; idx < dk * DVS; idx += nt) {
+            const int c = idx / DVS, j = idx % DVS;
+            dSx[cbase + (size_t)c * dv + j0 + j] = dS[idx];
         }
-        dq[i] = a;
-        dk[i] = b;
-        dg[i] = c;
-        if (i < rows) {
-            float d = 0.f;
-            for (int s = 0; s < nslice; ++s) d += db_p[s * rows + i];
-            db[i] = d;
+        const float* Glast = G + ((size_t)(t0 + L - 1) * H + h) * dk;
+        for (int c = tid; c < dk; c += nt) eGl[c] = expf(Glast[c]);
+        for (int idx = tid; idx < L * dk; idx += nt) {
+            const int r = idx / dk, c = idx % dk;
+            const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
+            Ws[r * ldk + c] = W[gi];
+            Kb[r * ldk + c] = to_f32(k[gi]) * expf(Glast[c] - G[gi]);
+        }
+        __syncthreads();
+        // X = Kb dS',  dU = E + X
+        for (int idx = tid; idx < L * DVS; idx += nt) {
+            const int r = idx / DVS, j = idx % DVS;
+            float acc = 0.f;
+            const float* kr = Kb + r * ldk;
+            for (int c = 0; c < dk; ++c) acc += kr[c] * dS[c * DVS + j];
+            Xs[r * ldx + j] = acc;
+            const size_t vi = ((size_t)(t0 + r) * H + h) * dv + j0 + j;
+            dU[vi] = E[vi] + acc;
+        }
+        __syncthreads();
+        // dS <- Diag(Gam) dS' - W^T X + F
+        for (int idx = tid; idx < dk * DVS; idx += nt) {
+            const int c = idx / DVS, j = idx % DVS;
+            float acc = eGl[c] * dS[idx] + F[cbase + (size_t)c * dv + j0 + j];
+            for (int r = 0; r < L; ++r) acc -= Ws[r * ldk + c] * Xs[r * ldx + j];
+            dS[idx] = acc;
         }
     }
+    __syncthreads();
+    if (dh0) {
+        for (int idx = tid; idx < dk * DVS; idx += nt) {
+            const int c = idx / DVS, j = idx % DVS;
+            dh0[st_base + (size_t)c * dv + j0 + j] = dS[idx];
+        }
+    }
+}
+
+size_t chain_smem(int dk) {
+    return sizeof(float) * ((size_t)dk * DVS + (size_t)2 * CB * (dk + 1) +
+                            (size_t)CB * (DVS + 1) + dk);
+}
+
+// ------------------------------------------------------------ b3: solve
+// One block per (chunk, head).  Shared: K, G [C][dk+1], A without b [C][C+1],
+// b [C], Y [C][dv+1], then U, dO, V slices [C][DVS+1].
+template <typename TIn>
+__global__ void __launch_bounds__(256) bwd_solve_kernel(
+    const TIn* __restrict__ k, const TIn* __restrict__ v, const TIn* __restrict__ dout,
+    const float* __restrict__ G, const float* __restrict__ beta, const float* __restrict__ U,
+    const float* __restrict__ dU, const int4* __restrict__ info, int H, int dk, int dv,
+    const uint32_t* status, float* __restrict__ Y, float* __restrict__ dv_out,
+    float* __restrict__ dAr, float* __restrict__ dP, float* __restrict__ dbB) {
+    if (status_bad(status)) return;
+    const int cidx = blockIdx.x, h = blockIdx.y;
+    const int4 ci = info[cidx];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    extern __shared__ float sm[];
+    const int ldk = dk + 1, lda = CB + 1, ldy = dv + 1, lds = DVS + 1;
+    float* Ks = sm;
+    float* Gs = Ks + CB * ldk;
+    float* Ar = Gs + CB * ldk;
+    float* bs = Ar + CB * lda;
+    float* Ys = bs + CB;
+    float* Us = Ys + CB * ldy;
+    float* Ds = Us + CB * lds;
+    float* Vs = Ds + CB * lds;
+    for (int idx = tid; idx < L * dk; idx += nt) {
+        const int r = idx / dk, c = idx % dk;
+        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
+        Ks[r * ldk + c] = to_f32(k[gi]);
+        Gs[r * ldk + c] = G[gi];
+    }
+    for (int r = tid; r < L; r += nt) bs[r] = beta[(size_t)(ci.y + r) * H + h];
+    for (int idx = tid; idx < L * dv; idx += nt) {
+        const int r = idx / dv, j = idx % dv;
+        Ys[r * ldy + j] = dU[((size_t)(ci.y + r) * H + h) * dv + j];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < L * L; idx += nt) {
+        const int r = idx / L, i = idx % L;
+        float acc = 0.f;
+        if (i < r) {
+            const float* kr = Ks + r * ldk;
+            const float* ki = Ks + i * ldk;
+            const float* gr = Gs + r * ldk;
+            const float* gi = Gs + i * ldk;
+            for (int c = 0; c < dk; ++c) acc += kr[c] * ki[c] * expf(gr[c] - gi[c]);
+        }
+        Ar[r * lda + i] = acc;
+    }
+    __syncthreads();
+    // (I + A)^T Y = dU by back substitution, one column per thread:
+    // Y_r = dU_r - sum_{i > r} b_i A[i][r] Y_i
+    for (int col = tid; col < dv; col += nt) {
+        for (int r = L - 2; r >= 0; --r) {
+            float acc = Ys[r * ldy + col];
+            for (int i = r + 1; i < L; ++i) acc -= bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
+            Ys[r * ldy + col] = acc;
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < L * dv; idx += nt) {
+        const int r = idx / dv, j = idx % dv;
+        const size_t vi = ((size_t)(ci.y + r) * H + h) * dv + j;
+        Y[vi] = Ys[r * ldy + j];
+        dv_out[vi] = bs[r] * Ys[r * ldy + j];
+    }
+    // dA[i][j] = -(Y U^T)[i][j] (j < i), dP[i][j] = (dO U^T)[i][j] (j <= i):
+    // thread (i = tid / 4, jl = tid % 4) takes j = jl + 4 m
+    const int i = tid >> 2, jl = tid & 3;
+    float accA[CB / 4], accP[CB / 4];
+#pragma unroll
+    for (int m = 0; m < CB / 4; ++m) accA[m] = accP[m] = 0.f;
+    float yv = 0.f;
+    for (int j0 = 0; j0 < dv; j0 += DVS) {
+        __syncthreads();
+        for (int idx = tid; idx < CB * DVS; idx += nt) {
+            const int r = idx / DVS, j = idx % DVS;
+            const bool in = r < L;
+            const size_t vi = ((size_t)(ci.y + r) * H + h) * dv + j0 + j;
+            Us[r * lds + j] = in ? U[vi] : 0.f;
+            Ds[r * lds + j] = in ? to_f32(dout[vi]) : 0.f;
+            Vs[r * lds + j] = in ? to_f32(v[vi]) : 0.f;
+        }
+        __syncthreads();
+        if (i < L) {
+            for (int j = 0; j < DVS; ++j) {
+                const float y = Ys[i * ldy + j0 + j], d = Ds[i * lds + j];
+#pragma unroll
+                for (int m = 0; m < CB / 4; ++m) {
+                    const float u = Us[(jl + 4 * m) * lds + j];
+                    accA[m] += y * u;
+                    accP[m] += d * u;
+                }
+            }
+            for (int j = jl; j < DVS; j += 4) yv += Ys[i * ldy + j0 + j] * Vs[i * lds + j];
+        }
+    }
+    const size_t cc = ((size_t)cidx * H + h) * CB * CB + (size_t)i * CB;
+    float part = yv;
+    if (i < L) {
+#pragma unroll
+        for (int m = 0; m < CB / 4; ++m) {
+            const int j = jl + 4 * m;
+            const float da = j < i ? -accA[m] : 0.f;
+            part += da * Ar[i * lda + j];
+            dAr[cc + j] = bs[i] * da;
+            dP[cc + j] = j <= i ? accP[m] : 0.f;
+        }
+    }
+    // the four threads of one row are adjacent lanes of one warp
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    if (i < L && jl == 0) dbB[(size_t)(ci.y + i) * H + h] = part;
+}
+
+size_t solve_smem(int dk, int dv) {
+    return sizeof(float) * ((size_t)2 * CB * (dk + 1) + (size_t)CB * (CB + 1) + CB +
+                            (size_t)CB * (dv + 1) + (size_t)3 * CB * (DVS + 1));
+}
+
+// ------------------------------------------------------------ b4: dense
+// One block per (chunk, head).  dQt = dO S^T, YS = Y S^T, dKb = U dS'^T over
+// the dv columns, and dGam = rowsum(S * dS').  Thread (rg = tid / 16, cl =
+// tid % 16) owns rows 4 rg .. 4 rg + 3 and channels cl + 16 m.  Shared:
+// S and dS' slices [DK][DVS+1], dO, Y, U slices [C][DVS+1].
+template <int DK, typename TIn>
+__global__ void __launch_bounds__(256) bwd_dense_kernel(
+    const TIn* __restrict__ k, const TIn* __restrict__ dout, const float* __restrict__ G,
+    const float* __restrict__ beta, const float* __restrict__ U, const float* __restrict__ Y,
+    const float* __restrict__ states, const float* __restrict__ dSx,
+    const float* __restrict__ dbB, const int4* __restrict__ info, int H, int dv,
+    const uint32_t* status, float* __restrict__ dQt, float* __restrict__ dKt,
+    float* __restrict__ dKb, float* __restrict__ dGam, float* __restrict__ dbeta) {
+    constexpr int NM = DK / 16;
+    constexpr int LD = DVS + 1;
+    if (status_bad(status)) return;
+    const int cidx = blockIdx.x, h = blockIdx.y;
+    const int4 ci = info[cidx];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int rg = tid >> 4, cl = tid & 15;
+    extern __shared__ float sm[];
+    float* Ss = sm;             // [DK][LD]
+    float* Xs = Ss + DK * LD;   // [DK][LD]
+    float* Ds = Xs + DK * LD;   // [C][LD]
+    float* Ysl = Ds + CB * LD;  // [C][LD]
+    float* Us = Ysl + CB * LD;  // [C][LD]
+    float aQ[4][NM], aY[4][NM], aK[4][NM];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int m = 0; m < NM; ++m) aQ[a][m] = aY[a][m] = aK[a][m] = 0.f;
+    float gam = 0.f;
+    const size_t cbase = ((size_t)cidx * H + h) * DK * dv;
+    for (int j0 = 0; j0 < dv; j0 += DVS) {
+        __syncthreads();
+        for (int idx = tid; idx < DK * DVS; idx += nt) {
+            const int c = idx / DVS, j = idx % DVS;
+            Ss[c * LD + j] = states[cbase + (size_t)c * dv + j0 + j];
+            Xs[c * LD + j] = dSx[cbase + (size_t)c * dv + j0 + j];
+        }
+        for (int idx = tid; idx < CB * DVS; idx += nt) {
+            const int r = idx / DVS, j = idx % DVS;
+            const bool in = r < L;
+            const size_t vi = ((size_t)(ci.y + r) * H + h) * dv + j0 + j;
+            Ds[r * LD + j] = in ? to_f32(dout[vi]) : 0.f;
+            Ysl[r * LD + j] = in ? Y[vi] : 0.f;
+            Us[r * LD + j] = in ? U[vi] : 0.f;
+        }
+        __syncthreads();
+        if (tid < DK)
+            for (int j = 0; j < DVS; ++j) gam += Ss[tid * LD + j] * Xs[tid * LD + j];
+        for (int j = 0; j < DVS; ++j) {
+            float d[4], y[4], u[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                d[a] = Ds[(4 * rg + a) * LD + j];
+                y[a] = Ysl[(4 * rg + a) * LD + j];
+                u[a] = Us[(4 * rg + a) * LD + j];
+            }
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const float sv = Ss[(cl + 16 * m) * LD + j], xv = Xs[(cl + 16 * m) * LD + j];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    aQ[a][m] += d[a] * sv;
+                    aY[a][m] += y[a] * sv;
+                    aK[a][m] += u[a] * xv;
+                }
+            }
+        }
+    }
+    if (tid < DK) dGam[((size_t)cidx * H + h) * DK + tid] = gam;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int r = 4 * rg + a;
+        float part = 0.f;
+        if (r < L) {
+            const size_t row = ((size_t)(ci.y + r) * H + h) * DK;
+            const float b = beta[(size_t)(ci.y + r) * H + h];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const int c = cl + 16 * m;
+                dQt[row + c] = aQ[a][m];
+                dKt[row + c] = -b * aY[a][m];
+                dKb[row + c] = aK[a][m];
+                part += to_f32(k[row + c]) * expf(G[row + c]) * aY[a][m];
+            }
+        }
+        // the sixteen threads of one row group are one half of a warp
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (cl == 0 && r < L) {
+            const size_t bi = (size_t)(ci.y + r) * H + h;
+            dbeta[bi] = dbB[bi] - part;
+        }
+    }
+}
+
+size_t dense_smem(int dk) { return sizeof(float) * (size_t)(2 * dk + 3 * CB) * (DVS + 1); }
+
+// ------------------------------------------------------------ b5: pairs
+// One block per (chunk, head, 32 channels).  Thread (grp = tid / 32, lane)
+// takes channel c0 + lane and the rows r = grp + 8 n: first as the later
+// token of each pair (sums over i <= r), then as the earlier one (sums over
+// r' >= r); then it adds the elementwise terms, and a reverse scan over the
+// chunk's rows turns dG into dg.  Shared: Q, K, G, dG [C][32], b dA and dP
+// [C][C+1], and the per-group sums for the last row [8][32].
+template <typename TIn>
+__global__ void __launch_bounds__(256) bwd_pair_kernel(
+    const TIn* __restrict__ q, const TIn* __restrict__ k, const float* __restrict__ G,
+    const float* __restrict__ dAr, const float* __restrict__ dP, const float* __restrict__ dQt,
+    const float* __restrict__ dKt, const float* __restrict__ dKb,
+    const float* __restrict__ dGam, const int4* __restrict__ info, int H, int dk,
+    const uint32_t* status, float* __restrict__ dq, float* __restrict__ dk_out,
+    float* __restrict__ dg) {
+    constexpr int NR = CB / 8;
+    constexpr int LA = CB + 1;
+    if (status_bad(status)) return;
+    const int cidx = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * 32;
+    const int4 ci = info[cidx];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
+    extern __shared__ float sm[];
+    float* Qs = sm;              // [C][32]
+    float* Ks = Qs + CB * 32;    // [C][32]
+    float* Gs = Ks + CB * 32;    // [C][32]
+    float* dGs = Gs + CB * 32;   // [C][32]
+    float* sA = dGs + CB * 32;   // [C][LA]
+    float* sP = sA + CB * LA;    // [C][LA]
+    float* lastred = sP + CB * LA;  // [8][32]
+    for (int idx = tid; idx < CB * 32; idx += 256) {
+        const int r = idx / 32, c = idx % 32;
+        const bool in = r < L;
+        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c0 + c;
+        Qs[idx] = in ? to_f32(q[gi]) : 0.f;
+        Ks[idx] = in ? to_f32(k[gi]) : 0.f;
+        Gs[idx] = in ? G[gi] : 0.f;
+    }
+    const size_t cc = ((size_t)cidx * H + h) * CB * CB;
+    for (int idx = tid; idx < CB * CB; idx += 256) {
+        const int r = idx / CB, i = idx % CB;
+        const bool in = r < L && i < L;
+        sA[r * LA + i] = in ? dAr[cc + idx] : 0.f;
+        sP[r * LA + i] = in ? dP[cc + idx] : 0.f;
+    }
+    __syncthreads();
+    float rowA[NR], dQp[NR], col[NR];
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+        const int r = grp + 8 * n;
+        float a = 0.f, p = 0.f, cs = 0.f;
+        if (r < L) {
+            const float gr = Gs[r * 32 + lane];
+            // r as the later token: i < r (A) and i <= r (P)
+            for (int i = 0; i < r; ++i) {
+                const float e = Ks[i * 32 + lane] * expf(gr - Gs[i * 32 + lane]);
+                a += sA[r * LA + i] * e;
+                p += sP[r * LA + i] * e;
+            }
+            p += sP[r * LA + r] * Ks[r * 32 + lane];
+            // r as the earlier token: r' > r (A and P) and r' = r (P)
+            for (int i = r + 1; i < L; ++i) {
+                const float e = expf(Gs[i * 32 + lane] - gr);
+                cs += (sA[i * LA + r] * Ks[i * 32 + lane] + sP[i * LA + r] * Qs[i * 32 + lane]) * e;
+            }
+            cs += sP[r * LA + r] * Qs[r * 32 + lane];
+        }
+        rowA[n] = a;
+        dQp[n] = p;
+        col[n] = cs;
+    }
+    const float glast = Gs[(L - 1) * 32 + lane];
+    float lastsum = 0.f;
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+        const int r = grp + 8 * n;
+        if (r < L) {
+            const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c0 + lane;
+            const float gr = Gs[r * 32 + lane], qr = Qs[r * 32 + lane], kr = Ks[r * 32 + lane];
+            const float eg = expf(gr), eb = expf(glast - gr);
+            const float a = dQt[gi], b = dKt[gi], d = dKb[gi];
+            dq[gi] = dQp[n] + a * eg;
+            dk_out[gi] = rowA[n] + col[n] + b * eg + d * eb;
+            dGs[r * 32 + lane] = kr * (rowA[n] - col[n]) + qr * dQp[n] + a * qr * eg +
+                                 b * kr * eg - d * kr * eb;
+            lastsum += d * kr * eb;
+        }
+    }
+    lastred[grp * 32 + lane] = lastsum;
+    __syncthreads();
+    if (grp == 0) {
+        float acc = expf(glast) * dGam[((size_t)cidx * H + h) * dk + c0 + lane];
+#pragma unroll
+        for (int g2 = 0; g2 < 8; ++g2) acc += lastred[g2 * 32 + lane];
+        for (int r = L - 1; r >= 0; --r) {
+            acc += dGs[r * 32 + lane];
+            dg[((size_t)(ci.y + r) * H + h) * dk + c0 + lane] = acc;
+        }
+    }
+}
+
+size_t pair_smem() {
+    return sizeof(float) * ((size_t)4 * CB * 32 + (size_t)2 * CB * (CB + 1) + 8 * 32);
+}
+
+template <typename Kern>
+cudaError_t set_smem(Kern* kern, size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 template <int DK, typename TIn>
-cudaError_t bwd_launch(const BwdParams& p, cudaStream_t st) {
-    const size_t smem = (size_t)SB * DK * DVS * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<DK, TIn>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t launch_dense(const BwdBufs& b, const TIn* K, const TIn* DO, const float* beta,
+                         int maxc, int H, int dv, float* db, cudaStream_t st) {
+    const size_t sm = dense_smem(DK);
+    cudaError_t e = set_smem(bwd_dense_kernel<DK, TIn>, sm);
     if (e != cudaSuccess) return e;
-    bwd_kernel<DK, TIn><<<dim3(p.N * p.H, p.DV / DVS), NTB, smem, st>>>(p);
+    bwd_dense_kernel<DK, TIn><<<dim3(maxc, H), 256, sm, st>>>(
+        K, DO, b.w.G, beta, b.w.U, b.Y, b.w.states, b.dSx, b.dbB, b.w.chunk_info, H, dv,
+        b.w.status, b.dQt, b.dKt, b.dKb, b.dGam, db);
+    return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* v,
+                    const float* beta, const void* dout, const float* dhT, const int32_t* cu,
+                    int T, int N, int H, int dk, int dv, int maxc, float* dq, float* dkk,
+                    float* dvv, float* dg, float* db, float* dh0, cudaStream_t st) {
+    const TIn* Q = static_cast<const TIn*>(q);
+    const TIn* K = static_cast<const TIn*>(k);
+    const TIn* V = static_cast<const TIn*>(v);
+    const TIn* DO = static_cast<const TIn*>(dout);
+    const Workspace& w = b.w;
+    cudaError_t e;
+    if (maxc > 0) {
+        const size_t sm = prep_smem(dk);
+        if ((e = set_smem(bwd_prep_kernel<TIn>, sm)) != cudaSuccess) return e;
+        bwd_prep_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(Q, K, DO, w.G, w.W, w.chunk_info, H,
+                                                            dk, dv, w.status, b.E, b.F);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        const size_t sm = chain_smem(dk);
+        if ((e = set_smem(bwd_chain_kernel<TIn>, sm)) != cudaSuccess) return e;
+        bwd_chain_kernel<TIn><<<dim3(N, H, dv / DVS), 256, sm, st>>>(
+            K, w.G, w.W, b.E, b.F, dhT, cu, T, w.chunk_start, H, dk, dv, w.status, b.dU, b.dSx,
+            dh0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (maxc == 0) return cudaSuccess;
+    {
+        const size_t sm = solve_smem(dk, dv);
+        if ((e = set_smem(bwd_solve_kernel<TIn>, sm)) != cudaSuccess) return e;
+        bwd_solve_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(K, V, DO, w.G, beta, w.U, b.dU,
+                                                             w.chunk_info, H, dk, dv, w.status,
+                                                             b.Y, dvv, b.dAr, b.dP, b.dbB);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    e = dk == 128 ? launch_dense<128, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
+        : dk == 64 ? launch_dense<64, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
+                   : launch_dense<32, TIn>(b, K, DO, beta, maxc, H, dv, db, st);
+    if (e != cudaSuccess) return e;
+    const size_t sm = pair_smem();
+    if ((e = set_smem(bwd_pair_kernel<TIn>, sm)) != cudaSuccess) return e;
+    bwd_pair_kernel<TIn><<<dim3(maxc, H, dk / 32), 256, sm, st>>>(
+        Q, K, w.G, b.dAr, b.dP, b.dQt, b.dKt, b.dKb, b.dGam, w.chunk_info, H, dk, w.status, dq,
+        dkk, dg);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t bwd_workspace_bytes(int total, int N, int H, int dk, int dv) {
-    const size_t ck = ((size_t)total / SB + N + 1) * H * dk * dv * sizeof(float);
-    const size_t slices = dv / DVS;
-    const size_t part = slices * (size_t)total * H * (3 * dk + 1) * sizeof(float);
-    return align_up(ck) + align_up(part);
+    return carve_bwd(nullptr, total, N, H, dk, dv).bytes;
 }
 
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* g,
@@ -348,33 +649,29 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float*
                        float* dq, float* dkk, float* dvv, float* dg, float* db, float* dh0,
                        void* workspace, cudaStream_t st) {
     const int total = cu ? T : N * T;
-    if (N * H == 0) return cudaSuccess;
-    char* ws = static_cast<char*>(workspace);
-    const size_t ck = align_up(((size_t)total / SB + N + 1) * H * dk * dv * sizeof(float));
-    const int slices = dv / DVS;
-    const size_t n = (size_t)total * H * dk;
-    float* part = reinterpret_cast<float*>(ws + ck);
-    BwdParams p{q, k, v, g, beta, h0, dout, dhT, cu, T, N, H, dv, total,
-                reinterpret_cast<float*>(ws), part, part + slices * n, part + 2 * slices * n,
-                part + 3 * slices * n, dvv, dh0};
-    cudaError_t e;
-    if (dt == KDA_DTYPE_BF16) {
-        e = dk == 128 ? bwd_launch<128, __nv_bfloat16>(p, st)
-            : dk == 64 ? bwd_launch<64, __nv_bfloat16>(p, st)
-                       : bwd_launch<32, __nv_bfloat16>(p, st);
-    } else {
-        e = dk == 128 ? bwd_launch<128, float>(p, st)
-            : dk == 64 ? bwd_launch<64, float>(p, st)
-                       : bwd_launch<32, float>(p, st);
-    }
-    if (e != cudaSuccess || total == 0) return e;
-    const long long rows = (long long)total * H;
-    const long long work = rows * dk;
-    const unsigned grid = static_cast<unsigned>(work / 256 + 1 < 148 * 16 ? work / 256 + 1
-                                                                          : 148 * 16);
-    bwd_reduce_kernel<<<grid, 256, 0, st>>>(p.dq_p, p.dk_p, p.dg_p, p.db_p, slices, rows, dk, dq,
-                                            dkk, dg, db);
-    return cudaGetLastError();
+    const int B = cu ? 1 : N;
+    const BwdBufs b = carve_bwd(workspace, total, N, H, dk, dv);
+    const Workspace& w = b.w;
+    const int maxc = max_chunks(total, N, CB);
+    // forward half: the CUDA-core prefill's chunk table, a1 (G), a2 (W, Ut)
+    // and a3 (U and every chunk's entry state)
+    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+    if (e == cudaSuccess)
+        e = launch_build_chunk_table(cu, B, T, N, CB, maxc, w.status, w.chunk_start,
+                                     w.chunk_info, st);
+    if (e == cudaSuccess) e = launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
+    if (e == cudaSuccess)
+        e = launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, CB, dt, w.status, w.W,
+                         w.U, st);
+    if (e == cudaSuccess)
+        e = launch_inter(k, w.G, w.W, w.U, h0, cu, B, T, N, w.chunk_start, H, dk, dv, CB, dt,
+                         w.status, w.states, nullptr, st);
+    if (e != cudaSuccess) return e;
+    return dt == KDA_DTYPE_BF16
+               ? run_bwd<__nv_bfloat16>(b, q, k, v, beta, dout, dhT, cu, T, N, H, dk, dv, maxc,
+                                        dq, dkk, dvv, dg, db, dh0, st)
+               : run_bwd<float>(b, q, k, v, beta, dout, dhT, cu, T, N, H, dk, dv, maxc, dq, dkk,
+                                dvv, dg, db, dh0, st);
 }
 
 }  // namespace kda

@@ -39,7 +39,25 @@ CASES = {
                                             dtype="f32", varlen=True),
     "bf16_batched_d32": lambda: wl.make_prefill(503, [25, 25], H=2, dk=32, dv=64, chunk=16,
                                                 dtype="bf16"),
+    # several 64-token chunks per sequence, ragged tails, an exact multiple
+    "bf16_d128_multichunk": lambda: wl.make_prefill(504, [150, 64, 129], H=2, dk=128, dv=128,
+                                                    chunk=64, dtype="bf16", varlen=True),
+    "f32_d128_dv64_batched": lambda: wl.make_prefill(505, [200, 200], H=1, dk=128, dv=64,
+                                                     chunk=64, dtype="f32"),
 }
+
+
+def _strong_decay():
+    """Gates twenty times stronger: the states forget within a few tokens and
+    exp(G) of a whole chunk underflows, while every pairwise factor stays
+    finite."""
+    case = wl.make_prefill(506, [130, 70], H=2, dk=64, dv=64, chunk=64, dtype="f32",
+                           varlen=True)
+    case.g = case.g * 20.0
+    return case
+
+
+CASES["f32_d64_strong_decay"] = _strong_decay
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
