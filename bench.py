@@ -266,6 +266,12 @@ def run_ours(args, rank, world, local_rank):
     # output gate after), on this workload's tensors, each timed alone
     layer = layer_times(kda, torch, P, dev, stream, reps=max(5, min(50, args.steps)))
 
+    # ---- the backward (gradients of o and the final state) on the same workload
+    bwd = None if args.no_backward else backward_times(
+        kda, torch, P, pc, dev, stream, reps=max(3, min(20, args.steps)),
+        sm_max_mhz=clk.get("sm_max_mhz") if isinstance(clk, dict) else None,
+        oracle_sample=(rank == 0 and world == 1 and not args.no_cpu_baseline))
+
     # ---- end to end through host buffers (pinned), copies inside the region
     e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=max(3, min(args.steps, 50)))
 
@@ -306,6 +312,7 @@ def run_ours(args, rank, world, local_rank):
                                 "algorithmic_bytes_per_launch": db}},
         "roofline": roof,
         "layer_steps": layer,
+        "backward": bwd,
         "e2e": e2e,
         "gpu_launches": args.steps * (kern["launches_per_call"] + 1),
         "clocks": clk,
@@ -450,6 +457,78 @@ def layer_times(kda, torch, P, dev, stream, reps=20):
         t = statistics.median(x.elapsed_time(z) for x, z in ts) / 1e3
         res[name] = {"us": t * 1e6, "bytes": nbytes, "gbs": nbytes / t / 1e9,
                      "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+    return res
+
+
+def backward_flops(head_tokens, dk, dv, C=64):
+    """Floating-point operations of the chunked backward per call: per chunk
+    of C tokens and one head, the multiply-adds of each step (the forward's
+    A, P, W, Ut and chain recomputed, then E, F, the reverse chain, the back
+    substitution, the products with U, S and dS', and the pair sums), two
+    flops each."""
+    tri, stri = C * (C + 1) // 2, C * (C - 1) // 2
+    fma = (2 * tri * dk + stri * (dk + dv) + 2 * C * dk * dv      # A, P; [W | Ut]; chain
+           + tri * dv + 2 * C * dk * dv + 2 * C * dk * dv        # E; F; reverse chain
+           + stri * dv + 2 * C * C * dv + 3 * C * dk * dv        # Y; Y U^T, dO U^T; dense
+           + 4 * tri * dk)                                        # pair sums
+    return 2 * fma * head_tokens / C
+
+
+def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None, oracle_sample=True):
+    """kda_chunk_bwd on the prefill workload (fp32 gradients of o and the final
+    state), timed with CUDA events on the launching stream, L2 flushed before
+    each call.  Bound by fp32 arithmetic on the CUDA cores: the roofline peak
+    is 148 SMs x 128 fp32 lanes x 2 flops x the SM clock."""
+    total, H, dk, dv = P.total, P.H, P.dk, P.dv
+    Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
+    g = torch.Generator(device=dev).manual_seed(9)
+    do = torch.randn(total, H, dv, device=dev, generator=g).to(torch.bfloat16)
+    dhT = torch.randn(P.N, H, dk, dv, device=dev, generator=g)
+    f32 = dict(dtype=torch.float32, device=dev)
+    outs = [torch.empty(total, H, dk, **f32), torch.empty(total, H, dk, **f32),
+            torch.empty(total, H, dv, **f32), torch.empty(total, H, dk, **f32),
+            torch.empty(total, H, **f32), torch.empty(P.N, H, dk, dv, **f32)]
+    ws = torch.empty(kda.kda_chunk_bwd_workspace_size(total, P.N, H, dk, dv), dtype=torch.uint8,
+                     device=dev)
+    call = lambda: kda.kda_chunk_bwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, do, dhT,
+                                     P.cu_seqlens, Bc, Tc, P.N, H, dk, dv, "bf16", *outs, ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    call()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    t = statistics.median(x.elapsed_time(z) for x, z in ts) / 1e3
+    fl = backward_flops(total * H, dk, dv)
+    mhz = sm_max_mhz or 1965.0
+    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 7,
+           "roofline": {"bound": "alu", "achieved": fl / t / 1e12, "peak": peak,
+                        "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak,
+                        "peak_kind": f"fp32 CUDA cores, 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",
+                        "algorithmic_flops_per_call": fl},
+           "workspace_bytes": int(ws.numel())}
+    if oracle_sample:
+        from oracle import backward as obwd
+        Ts = min(256, int(pc.cu_host()[1]))
+        hd = lambda x: x[:Ts, :1]
+        g0 = torch.Generator().manual_seed(9)
+        do0 = torch.randn(Ts, 1, dv, generator=g0).to(torch.bfloat16)
+        h0 = pc.initial_state[:1, :1] if pc.initial_state is not None else torch.zeros(1, 1, dk, dv)
+        t0 = time.perf_counter()
+        obwd.backward(hd(pc.q), hd(pc.k), hd(pc.v), hd(pc.g), pc.beta[:Ts, :1], h0, do0, None,
+                      [0, Ts])
+        el = time.perf_counter() - t0
+        res["cpu_oracle"] = {"value": Ts / el / H, "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"1 sequence x {Ts} tokens x 1 of {H} heads, fp64 token "
+                                       f"recurrence differentiated by autograd, {el:.2f} s"}
     return res
 
 
@@ -603,6 +682,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward timing beside the step")
     ap.add_argument("--prefill-config", type=int, default=1, choices=[1, 2, 3],
                     help="prefill workload: 1 = B=2 x T=2048 (default), 2 = B=1 x T=65536, "
                          "3 = 16 packed sequences of U[1024,16384] tokens")

@@ -10,7 +10,7 @@
 //   O = (Q * exp(G)) S + P U,    S' = Diag(Gam) S + (K * exp(G_last - G))^T U
 // Going backwards with dS' the gradient of the exit state and dO of the
 // chunk's outputs (Qt = Q * exp(G), Kt = K * exp(G), Kb = K * exp(G_last - G)):
-//   E  = P^T dO,  F = Qt^T dO - W^T E                              (b1 prep)
+//   E  = P^T dO,  F = Qt^T dO - W^T E                              (b1 intra)
 //   X  = Kb dS',  dU = E + X,  dS = Diag(Gam) dS' - W^T X + F      (b2 chain)
 //   Y  = T^T dU (back substitution),  dv = b Y,
 //   dA = -strict_lower(Y U^T),  dP = lower(dO U^T)                 (b3 solve)
@@ -19,10 +19,12 @@
 //   then the pair sums over (r, i, c) of A and P give dq, dk and dG, and
 //   dg is the reverse cumulative sum of dG inside the chunk          (b5 pairs)
 // The gradient of T = (I + A)^-1 never appears on its own: T^T dT T^T reduces
-// to Y U^T because the gradient reaching W is -dU S^T.  The forward half (G,
-// W, U and the entry state of every chunk) is the CUDA-core prefill's own
-// a1 .. a3.  Every exponent is a difference exp(G_r - G_i) with i <= r, so
-// never positive for g <= 0; all arithmetic is fp32.
+// to Y U^T because the gradient reaching W is -dU S^T.  The forward half is
+// recomputed: b1 forms G, A, P, W and Ut of each chunk (the forward's a1 and
+// a2, with A and P from one pass over the token pairs) and the CUDA-core
+// prefill's a3 chain gives U and the entry state of every chunk.  Every
+// exponent is a difference exp(G_r - G_i) with i <= r, so never positive for
+// g <= 0; all arithmetic is fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -41,6 +43,8 @@ struct BwdBufs {
     float* dU;    // [total, H, dv]
     float* Y;     // [total, H, dv]
     float* F;     // [maxc, H, dk, dv]
+    float* Ar;    // [maxc, H, C, C]     A without the b_r factor
+    float* Kb;    // [total, H, dk]      K * exp(G_last - G)
     float* dSx;   // [maxc, H, dk, dv]   gradient of each chunk's exit state
     float* dAr;   // [maxc, H, C, C]     b_r dA[r][i]
     float* dP;    // [maxc, H, C, C]
@@ -69,6 +73,8 @@ BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
     b.dU = take(tv);
     b.Y = take(tv);
     b.F = take(cs);
+    b.Ar = take(cc);
+    b.Kb = take(tk);
     b.dSx = take(cs);
     b.dAr = take(cc);
     b.dP = take(cc);
@@ -81,14 +87,21 @@ BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
     return b;
 }
 
-// ------------------------------------------------------------ b1: prep
-// One block per (chunk, head).  Shared: Qt, K, G, W [C][dk+1], P [C][C+1],
-// dO and E slices [C][DVS+1].
+// ------------------------------------------------------------ b1: intra
+// One block per (chunk, head).  Shared: Q (later Qt) [C][dk+4]; K, G
+// [C][dk+1]; A without b and P [C][C+1]; X = [b Kt | b V] solved in place
+// into [W | Ut] [C][dk+dv+4]; b [C]; dO and E slices [C][DVS+4] (rows of Q,
+// X, dO and E start on 16 bytes for the F tiles).  Rows past the chunk's end
+// are zero.
+constexpr int kPairTiles = (CB / 4) * (CB / 4 + 1) / 2;  // 4 x 4 tiles with i <= r
+
 template <typename TIn>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(
-    const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ dout,
-    const float* __restrict__ G, const float* __restrict__ W, const int4* __restrict__ info,
-    int H, int dk, int dv, const uint32_t* status, float* __restrict__ E,
+__global__ void __launch_bounds__(256) bwd_intra_kernel(
+    const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+    const TIn* __restrict__ dout, const float* __restrict__ g, const float* __restrict__ beta,
+    const int4* __restrict__ info, int H, int dk, int dv, const uint32_t* status,
+    float* __restrict__ G, float* __restrict__ W, float* __restrict__ Ut,
+    float* __restrict__ Ar_out, float* __restrict__ Kb, float* __restrict__ E,
     float* __restrict__ F) {
     if (status_bad(status)) return;
     const int cidx = blockIdx.x, h = blockIdx.y;
@@ -96,162 +109,364 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const int L = ci.z;
     if (L <= 0) return;
     const int tid = threadIdx.x, nt = blockDim.x;
-    extern __shared__ float sm[];
-    const int ldk = dk + 1, lda = CB + 1, lds = DVS + 1;
+    extern __shared__ __align__(16) float sm[];
+    const int ldq = dk + 4, ldk = dk + 1, lda = CB + 1, ldx = dk + dv + 4, lds = DVS + 4;
     float* Qs = sm;
-    float* Ks = Qs + CB * ldk;
+    float* Ks = Qs + CB * ldq;
     float* Gs = Ks + CB * ldk;
-    float* Ws = Gs + CB * ldk;
-    float* Ps = Ws + CB * ldk;
-    float* Ds = Ps + CB * lda;
+    float* As = Gs + CB * ldk;
+    float* Ps = As + CB * lda;
+    float* X = Ps + CB * lda;
+    float* bs = X + CB * ldx;
+    float* Ds = bs + CB;
     float* Es = Ds + CB * lds;
+    for (int idx = tid; idx < CB * dk; idx += nt) {
+        const int r = idx / dk, c = idx % dk;
+        const bool in = r < L;
+        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
+        Qs[r * ldq + c] = in ? to_f32(q[gi]) : 0.f;
+        Ks[r * ldk + c] = in ? to_f32(k[gi]) : 0.f;
+        Gs[r * ldk + c] = in ? g[gi] : 0.f;
+    }
+    for (int r = tid; r < CB; r += nt) bs[r] = r < L ? beta[(size_t)(ci.y + r) * H + h] : 0.f;
+    __syncthreads();
+    // a1: G = inclusive cumulative sum of g over the chunk's rows
+    for (int c = tid; c < dk; c += nt) {
+        float acc = 0.f;
+        for (int r = 0; r < L; ++r) {
+            acc += Gs[r * ldk + c];
+            Gs[r * ldk + c] = acc;
+            G[((size_t)(ci.y + r) * H + h) * dk + c] = acc;
+        }
+    }
+    __syncthreads();
+    // A[r][i] (i < r, without b) and P[r][i] (i <= r) from one exponent per
+    // (r, i, c): work item = (4 x 4 tile of pairs, channels c = q4 mod 4), the
+    // four items of a tile on adjacent lanes
+    for (int item = tid; item < kPairTiles * 4; item += nt) {
+        const int tile = item >> 2, q4 = item & 3;
+        int bi = 0;
+        while ((bi + 1) * (bi + 2) / 2 <= tile) ++bi;
+        const int bj = tile - bi * (bi + 1) / 2;
+        const int r0 = 4 * bi, i0 = 4 * bj;
+        float aA[4][4], aP[4][4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) aA[x][y] = aP[x][y] = 0.f;
+        for (int c = q4; c < dk; c += 4) {
+            float kr[4], qr[4], gr[4], ki[4], gi[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                kr[x] = Ks[(r0 + x) * ldk + c];
+                qr[x] = Qs[(r0 + x) * ldq + c];
+                gr[x] = Gs[(r0 + x) * ldk + c];
+                ki[x] = Ks[(i0 + x) * ldk + c];
+                gi[x] = Gs[(i0 + x) * ldk + c];
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    // pairs with i > r may overflow here; they are not kept
+                    const float ke = ki[y] * __expf(gr[x] - gi[y]);
+                    aA[x][y] += kr[x] * ke;
+                    aP[x][y] += qr[x] * ke;
+                }
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                aA[x][y] += __shfl_xor_sync(0xffffffffu, aA[x][y], 1);
+                aA[x][y] += __shfl_xor_sync(0xffffffffu, aA[x][y], 2);
+                aP[x][y] += __shfl_xor_sync(0xffffffffu, aP[x][y], 1);
+                aP[x][y] += __shfl_xor_sync(0xffffffffu, aP[x][y], 2);
+            }
+        if (q4 == 0) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const int r = r0 + x, i = i0 + y;
+                    As[r * lda + i] = (r < L && i < r) ? aA[x][y] : 0.f;
+                    Ps[r * lda + i] = (r < L && i <= r) ? aP[x][y] : 0.f;
+                }
+        }
+    }
+    // right-hand sides [b Kt | b V]
+    for (int idx = tid; idx < CB * dk; idx += nt) {
+        const int r = idx / dk, c = idx % dk;
+        X[r * ldx + c] = bs[r] * Ks[r * ldk + c] * __expf(Gs[r * ldk + c]);
+    }
+    for (int idx = tid; idx < CB * dv; idx += nt) {
+        const int r = idx / dv, j = idx % dv;
+        X[r * ldx + dk + j] = r < L ? bs[r] * to_f32(v[((size_t)(ci.y + r) * H + h) * dv + j]) : 0.f;
+    }
+    __syncthreads();
+    {
+        float* Ac = Ar_out + ((size_t)cidx * H + h) * CB * CB;
+        for (int idx = tid; idx < CB * CB; idx += nt) {
+            const int r = idx / CB, i = idx % CB;
+            Ac[idx] = i < r ? As[r * lda + i] : 0.f;
+        }
+    }
+    // a2: (I + A) [W | Ut] = X by forward substitution, one column per
+    // thread, four partial sums per row
+    for (int col = tid; col < dk + dv; col += nt) {
+        for (int r = 1; r < L; ++r) {
+            const float* ar = As + r * lda;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            int i = 0;
+            for (; i + 4 <= r; i += 4) {
+                a0 += ar[i] * X[i * ldx + col];
+                a1 += ar[i + 1] * X[(i + 1) * ldx + col];
+                a2 += ar[i + 2] * X[(i + 2) * ldx + col];
+                a3 += ar[i + 3] * X[(i + 3) * ldx + col];
+            }
+            for (; i < r; ++i) a0 += ar[i] * X[i * ldx + col];
+            X[r * ldx + col] -= bs[r] * ((a0 + a1) + (a2 + a3));
+        }
+    }
+    __syncthreads();
     for (int idx = tid; idx < L * dk; idx += nt) {
         const int r = idx / dk, c = idx % dk;
         const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
-        Qs[r * ldk + c] = to_f32(q[gi]);
-        Ks[r * ldk + c] = to_f32(k[gi]);
-        Gs[r * ldk + c] = G[gi];
-        Ws[r * ldk + c] = W[gi];
+        const float gr = Gs[r * ldk + c];
+        W[gi] = X[r * ldx + c];
+        Kb[gi] = Ks[r * ldk + c] * __expf(Gs[(L - 1) * ldk + c] - gr);
+        Qs[r * ldq + c] *= __expf(gr);
     }
-    __syncthreads();
-    for (int idx = tid; idx < L * L; idx += nt) {
-        const int r = idx / L, i = idx % L;
-        float acc = 0.f;
-        if (i <= r) {
-            const float* qr = Qs + r * ldk;
-            const float* ki = Ks + i * ldk;
-            const float* gr = Gs + r * ldk;
-            const float* gi = Gs + i * ldk;
-            for (int c = 0; c < dk; ++c) acc += qr[c] * ki[c] * expf(gr[c] - gi[c]);
-        }
-        Ps[r * lda + i] = acc;
+    for (int idx = tid; idx < L * dv; idx += nt) {
+        const int r = idx / dv, j = idx % dv;
+        Ut[((size_t)(ci.y + r) * H + h) * dv + j] = X[r * ldx + dk + j];
     }
-    __syncthreads();
-    for (int idx = tid; idx < L * dk; idx += nt) {
-        const int r = idx / dk, c = idx % dk;
-        Qs[r * ldk + c] *= expf(Gs[r * ldk + c]);
-    }
+    // E = P^T dO and F = Qt^T dO - W^T E, one slice of DVS columns at a time;
+    // F by 4 x 4 register tiles (channels 4 c4 + x, columns 4 j4 + y)
     float* Fc = F + ((size_t)cidx * H + h) * dk * dv;
     for (int j0 = 0; j0 < dv; j0 += DVS) {
         __syncthreads();
-        for (int idx = tid; idx < L * DVS; idx += nt) {
+        for (int idx = tid; idx < CB * DVS; idx += nt) {
             const int r = idx / DVS, j = idx % DVS;
-            Ds[r * lds + j] = to_f32(dout[((size_t)(ci.y + r) * H + h) * dv + j0 + j]);
+            Ds[r * lds + j] =
+                r < L ? to_f32(dout[((size_t)(ci.y + r) * H + h) * dv + j0 + j]) : 0.f;
         }
         __syncthreads();
-        // E[i][j] = sum_{r >= i} P[r][i] dO[r][j]
-        for (int idx = tid; idx < L * DVS; idx += nt) {
-            const int i = idx / DVS, j = idx % DVS;
-            float acc = 0.f;
-            for (int r = i; r < L; ++r) acc += Ps[r * lda + i] * Ds[r * lds + j];
-            Es[i * lds + j] = acc;
-            E[((size_t)(ci.y + i) * H + h) * dv + j0 + j] = acc;
+        // E rows 2 ip, 2 ip + 1, columns jq + 8 y (P[r][i] = 0 for i > r
+        // inside a diagonal 4 x 4 tile, so both rows start at r = 2 ip)
+        for (int t = tid; t < (CB / 2) * (DVS / 4); t += nt) {
+            const int jq = t % (DVS / 4), ip = t / (DVS / 4);
+            const int i = 2 * ip;
+            float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int r = i; r < L; ++r) {
+                const float p0 = Ps[r * lda + i], p1 = Ps[r * lda + i + 1];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const float d = Ds[r * lds + jq + 8 * y];
+                    e0[y] += p0 * d;
+                    e1[y] += p1 * d;
+                }
+            }
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                const int j = jq + 8 * y;
+                Es[i * lds + j] = e0[y];
+                Es[(i + 1) * lds + j] = e1[y];
+                if (i < L) E[((size_t)(ci.y + i) * H + h) * dv + j0 + j] = e0[y];
+                if (i + 1 < L) E[((size_t)(ci.y + i + 1) * H + h) * dv + j0 + j] = e1[y];
+            }
         }
         __syncthreads();
-        // F[c][j] = sum_r Qt[r][c] dO[r][j] - W[r][c] E[r][j]
-        for (int idx = tid; idx < dk * DVS; idx += nt) {
-            const int c = idx / DVS, j = idx % DVS;
-            float acc = 0.f;
-            for (int r = 0; r < L; ++r)
-                acc += Qs[r * ldk + c] * Ds[r * lds + j] - Ws[r * ldk + c] * Es[r * lds + j];
-            Fc[(size_t)c * dv + j0 + j] = acc;
+        for (int t = tid; t < (dk / 4) * (DVS / 4); t += nt) {
+            const int j4 = t % (DVS / 4), c4 = t / (DVS / 4);
+            float acc[4][4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 2
+            for (int r = 0; r < L; ++r) {
+                const float4 q4 = *reinterpret_cast<const float4*>(Qs + r * ldq + 4 * c4);
+                const float4 w4 = *reinterpret_cast<const float4*>(X + r * ldx + 4 * c4);
+                const float4 d4 = *reinterpret_cast<const float4*>(Ds + r * lds + 4 * j4);
+                const float4 e4 = *reinterpret_cast<const float4*>(Es + r * lds + 4 * j4);
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w}, wv[4] = {w4.x, w4.y, w4.z, w4.w};
+                const float dd[4] = {d4.x, d4.y, d4.z, d4.w}, ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) acc[x][y] += qv[x] * dd[y] - wv[x] * ev[y];
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                *reinterpret_cast<float4*>(Fc + (size_t)(4 * c4 + x) * dv + j0 + 4 * j4) =
+                    make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
         }
     }
 }
 
-size_t prep_smem(int dk) {
-    return sizeof(float) * ((size_t)4 * CB * (dk + 1) + (size_t)CB * (CB + 1) +
-                            (size_t)2 * CB * (DVS + 1));
+size_t intra_smem(int dk, int dv) {
+    return sizeof(float) * ((size_t)CB * (dk + 4) + (size_t)2 * CB * (dk + 1) +
+                            (size_t)2 * CB * (CB + 1) + (size_t)CB * (dk + dv + 4) + CB +
+                            (size_t)2 * CB * (DVS + 4));
 }
 
-// ------------------------------------------------------------ b2: chain
-// One block per (sequence, head, dv slice), serial over the chunks from the
-// last.  Shared: dS [dk][DVS], W and Kb [C][dk+1], X [C][DVS+1], Gam [dk].
-template <typename TIn>
-__global__ void __launch_bounds__(256) bwd_chain_kernel(
-    const TIn* __restrict__ k, const float* __restrict__ G, const float* __restrict__ W,
-    const float* __restrict__ E, const float* __restrict__ F, const float* __restrict__ dhT,
+// ------------------------------------------------------------ b2: chains
+// Both serial passes over a sequence's chunks, one block per (sequence, head,
+// slice of 32 value columns), the state slice in shared memory:
+//   forward  (first to last):  S_n -> states;  U = Ut - W S;
+//                              S <- Diag(Gam) S + Kb^T U
+//   backward (last to first):  dS' -> dSx;  X = Kb dS';  dU = E + X;
+//                              dS <- Diag(Gam) dS' - W^T X + F
+// Each chunk: W and Kb rows staged in shared memory with 16-byte loads, then
+// two small products on 4-column register tiles (M1: rows 2 rg, 2 rg + 1;
+// M2: channels 4 cg .. 4 cg + 3).  Shared: W, Kb [C][dk+4], state [dk][36],
+// M1 result [C][36], Gam [dk].
+constexpr int kChainDVS = 32;
+constexpr int kLdA = 128 + 4;  // row stride of the staged W and Kb (floats)
+constexpr int kLdS = kChainDVS + 4;
+
+template <bool kBack, typename TIn>
+__global__ void __launch_bounds__(256) chain_kernel(
+    const float* __restrict__ Wg, const float* __restrict__ Kbg, const float* __restrict__ G,
+    const float* __restrict__ S0, const float* EF_rows, const float* __restrict__ F,
     const int32_t* __restrict__ cu, int T, const int* __restrict__ chunk_start, int H, int dk,
-    int dv, const uint32_t* status, float* __restrict__ dU, float* __restrict__ dSx,
-    float* __restrict__ dh0) {
+    int dv, const uint32_t* status, float* rows_out, float* __restrict__ per_chunk,
+    float* __restrict__ S_end) {
+    // EF_rows and rows_out are the same buffer in the forward pass (Ut is
+    // replaced by U): each element is read and then written by one thread
     if (status_bad(status)) return;
-    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVS;
-    const int tid = threadIdx.x, nt = blockDim.x;
+    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kChainDVS;
+    const int tid = threadIdx.x;
     const int t_begin = cu ? cu[s] : s * T;
     const int t_end = cu ? cu[s + 1] : (s + 1) * T;
-    extern __shared__ float sm[];
-    const int ldk = dk + 1, ldx = DVS + 1;
-    float* dS = sm;                // [dk][DVS]
-    float* Ws = dS + dk * DVS;     // [C][ldk]
-    float* Kb = Ws + CB * ldk;     // [C][ldk]
-    float* Xs = Kb + CB * ldk;     // [C][ldx]
-    float* eGl = Xs + CB * ldx;    // [dk]
+    extern __shared__ __align__(16) float sm[];
+    float* Ws = sm;                 // [C][kLdA]
+    float* Kb = Ws + CB * kLdA;     // [C][kLdA]
+    float* Ss = Kb + CB * kLdA;     // [dk][kLdS]
+    float* Rs = Ss + 128 * kLdS;    // [C][kLdS]
+    float* Gam = Rs + CB * kLdS;    // [dk]
     const size_t st_base = ((size_t)s * H + h) * dk * dv;
-    for (int idx = tid; idx < dk * DVS; idx += nt) {
-        const int c = idx / DVS, j = idx % DVS;
-        dS[idx] = dhT ? dhT[st_base + (size_t)c * dv + j0 + j] : 0.f;
+    for (int idx = tid; idx < dk * kChainDVS; idx += 256) {
+        const int c = idx / kChainDVS, j = idx % kChainDVS;
+        Ss[c * kLdS + j] = S0 ? S0[st_base + (size_t)c * dv + j0 + j] : 0.f;
     }
+    const int jg = tid & 7, rg = tid >> 3;
     const int nch = (t_end - t_begin + CB - 1) / CB;
-    for (int n = nch - 1; n >= 0; --n) {
+    const int dk4 = dk / 4;
+    for (int step = 0; step < nch; ++step) {
+        const int n = kBack ? nch - 1 - step : step;
         const int t0 = t_begin + n * CB;
         const int L = min(CB, t_end - t0);
-        const size_t cs = (size_t)chunk_start[s] + n;
-        const size_t cbase = (cs * H + h) * dk * dv;
+        const size_t cbase = (((size_t)chunk_start[s] + n) * H + h) * dk * dv;
         __syncthreads();
-        for (int idx = tid; idx < dk * DVS; idx += nt) {
-            const int c = idx / DVS, j = idx % DVS;
-            dSx[cbase + (size_t)c * dv + j0 + j] = dS[idx];
+        // the state entering this step: the forward's S_n, the backward's dS'
+        for (int idx = tid; idx < dk * kChainDVS; idx += 256) {
+            const int c = idx / kChainDVS, j = idx % kChainDVS;
+            per_chunk[cbase + (size_t)c * dv + j0 + j] = Ss[c * kLdS + j];
         }
-        const float* Glast = G + ((size_t)(t0 + L - 1) * H + h) * dk;
-        for (int c = tid; c < dk; c += nt) eGl[c] = expf(Glast[c]);
-        for (int idx = tid; idx < L * dk; idx += nt) {
-            const int r = idx / dk, c = idx % dk;
-            const size_t gi = ((size_t)(t0 + r) * H + h) * dk + c;
-            Ws[r * ldk + c] = W[gi];
-            Kb[r * ldk + c] = to_f32(k[gi]) * expf(Glast[c] - G[gi]);
+        for (int idx = tid; idx < L * dk4; idx += 256) {
+            const int r = idx / dk4, c4 = idx % dk4;
+            const size_t gi = ((size_t)(t0 + r) * H + h) * dk + 4 * c4;
+            *reinterpret_cast<float4*>(Ws + r * kLdA + 4 * c4) =
+                *reinterpret_cast<const float4*>(Wg + gi);
+            *reinterpret_cast<float4*>(Kb + r * kLdA + 4 * c4) =
+                *reinterpret_cast<const float4*>(Kbg + gi);
+        }
+        for (int c = tid; c < dk; c += 256) Gam[c] = expf(G[((size_t)(t0 + L - 1) * H + h) * dk + c]);
+        __syncthreads();
+        // M1: rows 2 rg, 2 rg + 1, columns 4 jg .. 4 jg + 3
+        {
+            const float* A1 = kBack ? Kb : Ws;
+            float acc[2][4];
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+            for (int c = 0; c < dk; ++c) {
+                const float a0 = A1[(2 * rg) * kLdA + c], a1 = A1[(2 * rg + 1) * kLdA + c];
+                const float4 sv = *reinterpret_cast<const float4*>(Ss + c * kLdS + 4 * jg);
+                acc[0][0] += a0 * sv.x; acc[0][1] += a0 * sv.y;
+                acc[0][2] += a0 * sv.z; acc[0][3] += a0 * sv.w;
+                acc[1][0] += a1 * sv.x; acc[1][1] += a1 * sv.y;
+                acc[1][2] += a1 * sv.z; acc[1][3] += a1 * sv.w;
+            }
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int r = 2 * rg + x;
+                if (r < L) {
+                    const size_t vi = ((size_t)(t0 + r) * H + h) * dv + j0 + 4 * jg;
+                    const float4 base = *reinterpret_cast<const float4*>(EF_rows + vi);
+                    float4 m;  // forward: U = Ut - W S; backward: X = Kb dS'
+                    if (kBack) {
+                        m = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+                        *reinterpret_cast<float4*>(rows_out + vi) =
+                            make_float4(base.x + m.x, base.y + m.y, base.z + m.z, base.w + m.w);
+                    } else {
+                        m = make_float4(base.x - acc[x][0], base.y - acc[x][1],
+                                        base.z - acc[x][2], base.w - acc[x][3]);
+                        *reinterpret_cast<float4*>(rows_out + vi) = m;
+                    }
+                    *reinterpret_cast<float4*>(Rs + r * kLdS + 4 * jg) = m;
+                }
+            }
         }
         __syncthreads();
-        // X = Kb dS',  dU = E + X
-        for (int idx = tid; idx < L * DVS; idx += nt) {
-            const int r = idx / DVS, j = idx % DVS;
-            float acc = 0.f;
-            const float* kr = Kb + r * ldk;
-            for (int c = 0; c < dk; ++c) acc += kr[c] * dS[c * DVS + j];
-            Xs[r * ldx + j] = acc;
-            const size_t vi = ((size_t)(t0 + r) * H + h) * dv + j0 + j;
-            dU[vi] = E[vi] + acc;
-        }
-        __syncthreads();
-        // dS <- Diag(Gam) dS' - W^T X + F
-        for (int idx = tid; idx < dk * DVS; idx += nt) {
-            const int c = idx / DVS, j = idx % DVS;
-            float acc = eGl[c] * dS[idx] + F[cbase + (size_t)c * dv + j0 + j];
-            for (int r = 0; r < L; ++r) acc -= Ws[r * ldk + c] * Xs[r * ldx + j];
-            dS[idx] = acc;
+        // M2: channels 4 cg .. 4 cg + 3, columns 4 jg .. 4 jg + 3
+        for (int cg = rg; cg < dk4; cg += 32) {
+            const float* A2 = kBack ? Ws : Kb;
+            float acc[4][4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int c = 4 * cg + x;
+                const float4 sv = *reinterpret_cast<const float4*>(Ss + c * kLdS + 4 * jg);
+                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (kBack) f = *reinterpret_cast<const float4*>(F + cbase + (size_t)c * dv + j0 + 4 * jg);
+                acc[x][0] = Gam[c] * sv.x + f.x; acc[x][1] = Gam[c] * sv.y + f.y;
+                acc[x][2] = Gam[c] * sv.z + f.z; acc[x][3] = Gam[c] * sv.w + f.w;
+            }
+            const float sg = kBack ? -1.f : 1.f;
+#pragma unroll 4
+            for (int r = 0; r < L; ++r) {
+                const float4 a4 = *reinterpret_cast<const float4*>(A2 + r * kLdA + 4 * cg);
+                const float4 m4 = *reinterpret_cast<const float4*>(Rs + r * kLdS + 4 * jg);
+                const float av[4] = {sg * a4.x, sg * a4.y, sg * a4.z, sg * a4.w};
+                const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) acc[x][y] += av[x] * mv[y];
+            }
+            // every thread reads only its own tile of the state in M2
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                *reinterpret_cast<float4*>(Ss + (4 * cg + x) * kLdS + 4 * jg) =
+                    make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
         }
     }
     __syncthreads();
-    if (dh0) {
-        for (int idx = tid; idx < dk * DVS; idx += nt) {
-            const int c = idx / DVS, j = idx % DVS;
-            dh0[st_base + (size_t)c * dv + j0 + j] = dS[idx];
+    if (S_end) {
+        for (int idx = tid; idx < dk * kChainDVS; idx += 256) {
+            const int c = idx / kChainDVS, j = idx % kChainDVS;
+            S_end[st_base + (size_t)c * dv + j0 + j] = Ss[c * kLdS + j];
         }
     }
 }
 
-size_t chain_smem(int dk) {
-    return sizeof(float) * ((size_t)dk * DVS + (size_t)2 * CB * (dk + 1) +
-                            (size_t)CB * (DVS + 1) + dk);
+size_t chain_smem() {
+    return sizeof(float) * ((size_t)2 * CB * kLdA + (size_t)128 * kLdS + (size_t)CB * kLdS + 128);
 }
 
 // ------------------------------------------------------------ b3: solve
-// One block per (chunk, head).  Shared: K, G [C][dk+1], A without b [C][C+1],
-// b [C], Y [C][dv+1], then U, dO, V slices [C][DVS+1].
+// One block per (chunk, head).  Shared: A without b [C][C+1], b [C], Y
+// [C][dv+1], then U, dO, V slices [C][DVS+1].
 template <typename TIn>
 __global__ void __launch_bounds__(256) bwd_solve_kernel(
-    const TIn* __restrict__ k, const TIn* __restrict__ v, const TIn* __restrict__ dout,
-    const float* __restrict__ G, const float* __restrict__ beta, const float* __restrict__ U,
-    const float* __restrict__ dU, const int4* __restrict__ info, int H, int dk, int dv,
+    const TIn* __restrict__ v, const TIn* __restrict__ dout, const float* __restrict__ Ain,
+    const float* __restrict__ beta, const float* __restrict__ U,
+    const float* __restrict__ dU, const int4* __restrict__ info, int H, int dv,
     const uint32_t* status, float* __restrict__ Y, float* __restrict__ dv_out,
     float* __restrict__ dAr, float* __restrict__ dP, float* __restrict__ dbB) {
     if (status_bad(status)) return;
@@ -261,20 +476,16 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
     if (L <= 0) return;
     const int tid = threadIdx.x, nt = blockDim.x;
     extern __shared__ float sm[];
-    const int ldk = dk + 1, lda = CB + 1, ldy = dv + 1, lds = DVS + 1;
-    float* Ks = sm;
-    float* Gs = Ks + CB * ldk;
-    float* Ar = Gs + CB * ldk;
+    const int lda = CB + 1, ldy = dv + 1, lds = DVS + 1;
+    float* Ar = sm;
     float* bs = Ar + CB * lda;
     float* Ys = bs + CB;
     float* Us = Ys + CB * ldy;
     float* Ds = Us + CB * lds;
     float* Vs = Ds + CB * lds;
-    for (int idx = tid; idx < L * dk; idx += nt) {
-        const int r = idx / dk, c = idx % dk;
-        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
-        Ks[r * ldk + c] = to_f32(k[gi]);
-        Gs[r * ldk + c] = G[gi];
+    {
+        const float* Ac = Ain + ((size_t)cidx * H + h) * CB * CB;
+        for (int idx = tid; idx < CB * CB; idx += nt) Ar[(idx / CB) * lda + idx % CB] = Ac[idx];
     }
     for (int r = tid; r < L; r += nt) bs[r] = beta[(size_t)(ci.y + r) * H + h];
     for (int idx = tid; idx < L * dv; idx += nt) {
@@ -282,26 +493,20 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
         Ys[r * ldy + j] = dU[((size_t)(ci.y + r) * H + h) * dv + j];
     }
     __syncthreads();
-    for (int idx = tid; idx < L * L; idx += nt) {
-        const int r = idx / L, i = idx % L;
-        float acc = 0.f;
-        if (i < r) {
-            const float* kr = Ks + r * ldk;
-            const float* ki = Ks + i * ldk;
-            const float* gr = Gs + r * ldk;
-            const float* gi = Gs + i * ldk;
-            for (int c = 0; c < dk; ++c) acc += kr[c] * ki[c] * expf(gr[c] - gi[c]);
-        }
-        Ar[r * lda + i] = acc;
-    }
-    __syncthreads();
     // (I + A)^T Y = dU by back substitution, one column per thread:
     // Y_r = dU_r - sum_{i > r} b_i A[i][r] Y_i
     for (int col = tid; col < dv; col += nt) {
         for (int r = L - 2; r >= 0; --r) {
-            float acc = Ys[r * ldy + col];
-            for (int i = r + 1; i < L; ++i) acc -= bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
-            Ys[r * ldy + col] = acc;
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            int i = r + 1;
+            for (; i + 4 <= L; i += 4) {
+                a0 += bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
+                a1 += bs[i + 1] * Ar[(i + 1) * lda + r] * Ys[(i + 1) * ldy + col];
+                a2 += bs[i + 2] * Ar[(i + 2) * lda + r] * Ys[(i + 2) * ldy + col];
+                a3 += bs[i + 3] * Ar[(i + 3) * lda + r] * Ys[(i + 3) * ldy + col];
+            }
+            for (; i < L; ++i) a0 += bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
+            Ys[r * ldy + col] -= (a0 + a1) + (a2 + a3);
         }
     }
     __syncthreads();
@@ -360,8 +565,8 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
     if (i < L && jl == 0) dbB[(size_t)(ci.y + i) * H + h] = part;
 }
 
-size_t solve_smem(int dk, int dv) {
-    return sizeof(float) * ((size_t)2 * CB * (dk + 1) + (size_t)CB * (CB + 1) + CB +
+size_t solve_smem(int dv) {
+    return sizeof(float) * ((size_t)CB * (CB + 1) + CB +
                             (size_t)CB * (dv + 1) + (size_t)3 * CB * (DVS + 1));
 }
 
@@ -522,15 +727,17 @@ __global__ void __launch_bounds__(256) bwd_pair_kernel(
         if (r < L) {
             const float gr = Gs[r * 32 + lane];
             // r as the later token: i < r (A) and i <= r (P)
+#pragma unroll 4
             for (int i = 0; i < r; ++i) {
-                const float e = Ks[i * 32 + lane] * expf(gr - Gs[i * 32 + lane]);
+                const float e = Ks[i * 32 + lane] * __expf(gr - Gs[i * 32 + lane]);
                 a += sA[r * LA + i] * e;
                 p += sP[r * LA + i] * e;
             }
             p += sP[r * LA + r] * Ks[r * 32 + lane];
             // r as the earlier token: r' > r (A and P) and r' = r (P)
+#pragma unroll 4
             for (int i = r + 1; i < L; ++i) {
-                const float e = expf(Gs[i * 32 + lane] - gr);
+                const float e = __expf(Gs[i * 32 + lane] - gr);
                 cs += (sA[i * LA + r] * Ks[i * 32 + lane] + sP[i * LA + r] * Qs[i * 32 + lane]) * e;
             }
             cs += sP[r * LA + r] * Qs[r * 32 + lane];
@@ -592,9 +799,10 @@ cudaError_t launch_dense(const BwdBufs& b, const TIn* K, const TIn* DO, const fl
 
 template <typename TIn>
 cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* v,
-                    const float* beta, const void* dout, const float* dhT, const int32_t* cu,
-                    int T, int N, int H, int dk, int dv, int maxc, float* dq, float* dkk,
-                    float* dvv, float* dg, float* db, float* dh0, cudaStream_t st) {
+                    const float* g, const float* beta, const float* h0, const void* dout,
+                    const float* dhT, const int32_t* cu, int T, int N, int H, int dk, int dv,
+                    kda_dtype_t dt, int maxc, float* dq, float* dkk, float* dvv, float* dg,
+                    float* db, float* dh0, cudaStream_t st) {
     const TIn* Q = static_cast<const TIn*>(q);
     const TIn* K = static_cast<const TIn*>(k);
     const TIn* V = static_cast<const TIn*>(v);
@@ -602,27 +810,36 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
     const Workspace& w = b.w;
     cudaError_t e;
     if (maxc > 0) {
-        const size_t sm = prep_smem(dk);
-        if ((e = set_smem(bwd_prep_kernel<TIn>, sm)) != cudaSuccess) return e;
-        bwd_prep_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(Q, K, DO, w.G, w.W, w.chunk_info, H,
-                                                            dk, dv, w.status, b.E, b.F);
+        const size_t sm = intra_smem(dk, dv);
+        if ((e = set_smem(bwd_intra_kernel<TIn>, sm)) != cudaSuccess) return e;
+        bwd_intra_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(Q, K, V, DO, g, beta, w.chunk_info,
+                                                             H, dk, dv, w.status, w.G, w.W, w.U,
+                                                             b.Ar, b.Kb, b.E, b.F);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
-        const size_t sm = chain_smem(dk);
-        if ((e = set_smem(bwd_chain_kernel<TIn>, sm)) != cudaSuccess) return e;
-        bwd_chain_kernel<TIn><<<dim3(N, H, dv / DVS), 256, sm, st>>>(
-            K, w.G, w.W, b.E, b.F, dhT, cu, T, w.chunk_start, H, dk, dv, w.status, b.dU, b.dSx,
-            dh0);
+        const size_t sm = chain_smem();
+        const dim3 grid(N, H, dv / kChainDVS);
+        if ((e = set_smem(chain_kernel<false, TIn>, sm)) != cudaSuccess) return e;
+        if ((e = set_smem(chain_kernel<true, TIn>, sm)) != cudaSuccess) return e;
+        // forward: U = Ut - W S (in place) and every chunk's entry state
+        chain_kernel<false, TIn><<<grid, 256, sm, st>>>(w.W, b.Kb, w.G, h0, w.U, nullptr, cu, T,
+                                                       w.chunk_start, H, dk, dv, w.status, w.U,
+                                                       w.states, nullptr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        // backward: dU, the exit-state gradient of every chunk, dS_0
+        chain_kernel<true, TIn><<<grid, 256, sm, st>>>(w.W, b.Kb, w.G, dhT, b.E, b.F, cu, T,
+                                                      w.chunk_start, H, dk, dv, w.status, b.dU,
+                                                      b.dSx, dh0);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (maxc == 0) return cudaSuccess;
     {
-        const size_t sm = solve_smem(dk, dv);
+        const size_t sm = solve_smem(dv);
         if ((e = set_smem(bwd_solve_kernel<TIn>, sm)) != cudaSuccess) return e;
-        bwd_solve_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(K, V, DO, w.G, beta, w.U, b.dU,
-                                                             w.chunk_info, H, dk, dv, w.status,
-                                                             b.Y, dvv, b.dAr, b.dP, b.dbB);
+        bwd_solve_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(V, DO, b.Ar, beta, w.U, b.dU,
+                                                             w.chunk_info, H, dv, w.status, b.Y,
+                                                             dvv, b.dAr, b.dP, b.dbB);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     e = dk == 128 ? launch_dense<128, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
@@ -649,29 +866,19 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float*
                        float* dq, float* dkk, float* dvv, float* dg, float* db, float* dh0,
                        void* workspace, cudaStream_t st) {
     const int total = cu ? T : N * T;
-    const int B = cu ? 1 : N;
     const BwdBufs b = carve_bwd(workspace, total, N, H, dk, dv);
     const Workspace& w = b.w;
     const int maxc = max_chunks(total, N, CB);
-    // forward half: the CUDA-core prefill's chunk table, a1 (G), a2 (W, Ut)
-    // and a3 (U and every chunk's entry state)
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
     if (e == cudaSuccess)
-        e = launch_build_chunk_table(cu, B, T, N, CB, maxc, w.status, w.chunk_start,
+        e = launch_build_chunk_table(cu, cu ? 1 : N, T, N, CB, maxc, w.status, w.chunk_start,
                                      w.chunk_info, st);
-    if (e == cudaSuccess) e = launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
-    if (e == cudaSuccess)
-        e = launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, CB, dt, w.status, w.W,
-                         w.U, st);
-    if (e == cudaSuccess)
-        e = launch_inter(k, w.G, w.W, w.U, h0, cu, B, T, N, w.chunk_start, H, dk, dv, CB, dt,
-                         w.status, w.states, nullptr, st);
     if (e != cudaSuccess) return e;
     return dt == KDA_DTYPE_BF16
-               ? run_bwd<__nv_bfloat16>(b, q, k, v, beta, dout, dhT, cu, T, N, H, dk, dv, maxc,
-                                        dq, dkk, dvv, dg, db, dh0, st)
-               : run_bwd<float>(b, q, k, v, beta, dout, dhT, cu, T, N, H, dk, dv, maxc, dq, dkk,
-                                dvv, dg, db, dh0, st);
+               ? run_bwd<__nv_bfloat16>(b, q, k, v, g, beta, h0, dout, dhT, cu, T, N, H, dk, dv,
+                                        dt, maxc, dq, dkk, dvv, dg, db, dh0, st)
+               : run_bwd<float>(b, q, k, v, g, beta, h0, dout, dhT, cu, T, N, H, dk, dv, dt,
+                                maxc, dq, dkk, dvv, dg, db, dh0, st);
 }
 
 }  // namespace kda

@@ -337,10 +337,11 @@ cudaError_t launch_inter(const void* k, const float* G, const float* W, float* U
                          const float* h0, const int32_t* cu_seqlens, int B, int T, int N,
                          const int* chunk_start, int H, int dk, int dv, int chunk,
                          kda_dtype_t dt, const uint32_t* status, float* states, float* hN,
-                         cudaStream_t st) {
+                         cudaStream_t st, int dv_slice) {
     (void)B;
     if (N == 0) return cudaSuccess;
-    const int dvs = dv < kInterDVS ? dv : kInterDVS;
+    const int want = dv_slice > 0 ? dv_slice : kInterDVS;
+    const int dvs = dv < want ? dv : want;
     const size_t smem = sizeof(float) * ((size_t)dk * dvs + (size_t)2 * chunk * (dk + 1) +
                                          (size_t)chunk * (dvs + 1) + dk);
     dim3 grid(N, H, dv / dvs);

@@ -123,7 +123,7 @@ cudaError_t launch_inter(const void* k, const float* G, const float* W, float* U
                          const float* h0, const int32_t* cu_seqlens, int B, int T, int N,
                          const int* chunk_start, int H, int dk, int dv, int chunk,
                          kda_dtype_t dt, const uint32_t* status, float* states, float* hN,
-                         cudaStream_t st);
+                         cudaStream_t st, int dv_slice = 0);
 cudaError_t launch_output(const void* q, const void* k, const float* G, const float* U,
                           const float* states, const int4* info, int maxc, int H, int dk,
                           int dv, int chunk, kda_dtype_t dt, const uint32_t* status, void* o,

@@ -74,3 +74,29 @@ def test_backward_matches_autograd(name, with_dhT):
                        dhT, cu)
     for name_, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), got, ref):
         assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
+
+
+@pytest.mark.parametrize("unit", [(0, 0), (1, 31)])
+def test_backward_bench_workload_sampled_heads(unit):
+    """The bench's prefill workload (B=2, T=2048, H=32, d=128, bf16) in the
+    launch configuration the bench times; the oracle's gradients of one
+    (sequence, head) at a time -- heads are independent, so the slice is an
+    exact reference for that head's outputs."""
+    case = wl.prefill_config(1)
+    s, h = unit
+    g = torch.Generator().manual_seed(11)
+    do = torch.randn(case.total, case.H, case.dv, generator=g).to(torch.bfloat16)
+    dhT = torch.randn(case.N, case.H, case.dk, case.dv, generator=g)
+    got = _run(case, do, dhT)
+    rows = slice(s * case.T, (s + 1) * case.T)
+    one = lambda x: x[rows, h:h + 1]
+    h0 = case.initial_state[s:s + 1, h:h + 1] if case.initial_state is not None else None
+    if h0 is None:
+        h0 = torch.zeros(1, 1, case.dk, case.dv)
+    ref = bwd.backward(one(case.q), one(case.k), one(case.v), one(case.g),
+                       case.beta[rows, h:h + 1], h0, one(do), dhT[s:s + 1, h:h + 1],
+                       np.array([0, case.T]))
+    sel = (one(got[0]), one(got[1]), one(got[2]), one(got[3]), got[4][rows, h:h + 1],
+           got[5][s:s + 1, h:h + 1])
+    for name_, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), sel, ref):
+        assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
