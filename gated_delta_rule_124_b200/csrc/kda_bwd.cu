@@ -45,6 +45,7 @@ struct BwdBufs {
     float* F;     // [maxc, H, dk, dv]
     float* Ar;    // [maxc, H, C, C]     A without the b_r factor
     float* Kb;    // [total, H, dk]      K * exp(G_last - G)
+    float* Pm;    // [maxc, H, C, C]     P
     float* dSx;   // [maxc, H, dk, dv]   gradient of each chunk's exit state
     float* dAr;   // [maxc, H, C, C]     b_r dA[r][i]
     float* dP;    // [maxc, H, C, C]
@@ -75,6 +76,7 @@ BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
     b.F = take(cs);
     b.Ar = take(cc);
     b.Kb = take(tk);
+    b.Pm = take(cc);
     b.dSx = take(cs);
     b.dAr = take(cc);
     b.dP = take(cc);
@@ -88,62 +90,60 @@ BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
 }
 
 // ------------------------------------------------------------ b1: intra
-// One block per (chunk, head).  Shared: Q (later Qt) [C][dk+4]; K, G
-// [C][dk+1]; A without b and P [C][C+1]; X = [b Kt | b V] solved in place
-// into [W | Ut] [C][dk+dv+4]; b [C]; dO and E slices [C][DVS+4] (rows of Q,
-// X, dO and E start on 16 bytes for the F tiles).  Rows past the chunk's end
-// are zero.
+// Three kernels, one block per (chunk, head) each, small enough in shared
+// memory for two blocks per SM.  Rows past the chunk's end are zero.
+//   b1a: G (a1), A without b and P from one exponent per (r, i, c), Kb, and
+//        the right-hand sides b Kt (into the W buffer).  Shared: Q, K, G
+//        [C][dk+1].
+//   b1b: (I + A) [W | Ut] = [b Kt | b V] by forward substitution (a2).
+//        Shared: A [C][C+1], X [C][dk+dv+1], b [C].
+//   b1c: E = P^T dO and F = Qt^T dO - W^T E.  Shared: P [C][C+1], Qt and W
+//        [C][dk+4], dO and E slices [C][DVS+4] (16-byte rows for the F tiles).
 constexpr int kPairTiles = (CB / 4) * (CB / 4 + 1) / 2;  // 4 x 4 tiles with i <= r
 
-template <typename TIn>
-__global__ void __launch_bounds__(256) bwd_intra_kernel(
-    const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-    const TIn* __restrict__ dout, const float* __restrict__ g, const float* __restrict__ beta,
-    const int4* __restrict__ info, int H, int dk, int dv, const uint32_t* status,
-    float* __restrict__ G, float* __restrict__ W, float* __restrict__ Ut,
-    float* __restrict__ Ar_out, float* __restrict__ Kb, float* __restrict__ E,
-    float* __restrict__ F) {
+template <int DK, typename TIn>
+__global__ void __launch_bounds__(256) bwd_apkb_kernel(
+    const TIn* __restrict__ q, const TIn* __restrict__ k, const float* __restrict__ g,
+    const float* __restrict__ beta, const int4* __restrict__ info, int H,
+    const uint32_t* status, float* __restrict__ G, float* __restrict__ Ar_out,
+    float* __restrict__ P_out, float* __restrict__ Kb, float* __restrict__ Rk) {
+    constexpr int LDK = DK + 1;
     if (status_bad(status)) return;
     const int cidx = blockIdx.x, h = blockIdx.y;
     const int4 ci = info[cidx];
     const int L = ci.z;
     if (L <= 0) return;
-    const int tid = threadIdx.x, nt = blockDim.x;
+    const int tid = threadIdx.x;
     extern __shared__ __align__(16) float sm[];
-    const int ldq = dk + 4, ldk = dk + 1, lda = CB + 1, ldx = dk + dv + 4, lds = DVS + 4;
     float* Qs = sm;
-    float* Ks = Qs + CB * ldq;
-    float* Gs = Ks + CB * ldk;
-    float* As = Gs + CB * ldk;
-    float* Ps = As + CB * lda;
-    float* X = Ps + CB * lda;
-    float* bs = X + CB * ldx;
-    float* Ds = bs + CB;
-    float* Es = Ds + CB * lds;
-    for (int idx = tid; idx < CB * dk; idx += nt) {
-        const int r = idx / dk, c = idx % dk;
+    float* Ks = Qs + CB * LDK;
+    float* Gs = Ks + CB * LDK;
+    const size_t row0 = ((size_t)ci.y * H + h) * DK;  // element (r, c) at row0 + r H DK + c
+    const size_t rstride = (size_t)H * DK;
+    for (int idx = tid; idx < CB * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
         const bool in = r < L;
-        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
-        Qs[r * ldq + c] = in ? to_f32(q[gi]) : 0.f;
-        Ks[r * ldk + c] = in ? to_f32(k[gi]) : 0.f;
-        Gs[r * ldk + c] = in ? g[gi] : 0.f;
+        const size_t gi = row0 + r * rstride + c;
+        Qs[r * LDK + c] = in ? to_f32(q[gi]) : 0.f;
+        Ks[r * LDK + c] = in ? to_f32(k[gi]) : 0.f;
+        Gs[r * LDK + c] = in ? g[gi] : 0.f;
     }
-    for (int r = tid; r < CB; r += nt) bs[r] = r < L ? beta[(size_t)(ci.y + r) * H + h] : 0.f;
     __syncthreads();
     // a1: G = inclusive cumulative sum of g over the chunk's rows
-    for (int c = tid; c < dk; c += nt) {
+    for (int c = tid; c < DK; c += 256) {
         float acc = 0.f;
         for (int r = 0; r < L; ++r) {
-            acc += Gs[r * ldk + c];
-            Gs[r * ldk + c] = acc;
-            G[((size_t)(ci.y + r) * H + h) * dk + c] = acc;
+            acc += Gs[r * LDK + c];
+            Gs[r * LDK + c] = acc;
+            G[row0 + r * rstride + c] = acc;
         }
     }
     __syncthreads();
-    // A[r][i] (i < r, without b) and P[r][i] (i <= r) from one exponent per
-    // (r, i, c): work item = (4 x 4 tile of pairs, channels c = q4 mod 4), the
-    // four items of a tile on adjacent lanes
-    for (int item = tid; item < kPairTiles * 4; item += nt) {
+    float* Ac = Ar_out + ((size_t)cidx * H + h) * CB * CB;
+    float* Pc = P_out + ((size_t)cidx * H + h) * CB * CB;
+    // A[r][i] (i < r) and P[r][i] (i <= r): work item = (4 x 4 tile of
+    // pairs, channels c = q4 mod 4), the four items of a tile on adjacent lanes
+    for (int item = tid; item < kPairTiles * 4; item += 256) {
         const int tile = item >> 2, q4 = item & 3;
         int bi = 0;
         while ((bi + 1) * (bi + 2) / 2 <= tile) ++bi;
@@ -154,15 +154,16 @@ __global__ void __launch_bounds__(256) bwd_intra_kernel(
         for (int x = 0; x < 4; ++x)
 #pragma unroll
             for (int y = 0; y < 4; ++y) aA[x][y] = aP[x][y] = 0.f;
-        for (int c = q4; c < dk; c += 4) {
+#pragma unroll 2
+        for (int c = q4; c < DK; c += 4) {
             float kr[4], qr[4], gr[4], ki[4], gi[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
-                kr[x] = Ks[(r0 + x) * ldk + c];
-                qr[x] = Qs[(r0 + x) * ldq + c];
-                gr[x] = Gs[(r0 + x) * ldk + c];
-                ki[x] = Ks[(i0 + x) * ldk + c];
-                gi[x] = Gs[(i0 + x) * ldk + c];
+                kr[x] = Ks[(r0 + x) * LDK + c];
+                qr[x] = Qs[(r0 + x) * LDK + c];
+                gr[x] = Gs[(r0 + x) * LDK + c];
+                ki[x] = Ks[(i0 + x) * LDK + c];
+                gi[x] = Gs[(i0 + x) * LDK + c];
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -183,37 +184,73 @@ __global__ void __launch_bounds__(256) bwd_intra_kernel(
                 aP[x][y] += __shfl_xor_sync(0xffffffffu, aP[x][y], 1);
                 aP[x][y] += __shfl_xor_sync(0xffffffffu, aP[x][y], 2);
             }
-        if (q4 == 0) {
+        // lane q4 writes row r0 + q4 of the tile
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
+        for (int x = 0; x < 4; ++x) {
+            if (x != q4) continue;
+            const int r = r0 + x;
+            float4 va, vp;
+            float* pa = &va.x;
+            float* pp = &vp.x;
 #pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    const int r = r0 + x, i = i0 + y;
-                    As[r * lda + i] = (r < L && i < r) ? aA[x][y] : 0.f;
-                    Ps[r * lda + i] = (r < L && i <= r) ? aP[x][y] : 0.f;
-                }
+            for (int y = 0; y < 4; ++y) {
+                const int i = i0 + y;
+                pa[y] = (r < L && i < r) ? aA[x][y] : 0.f;
+                pp[y] = (r < L && i <= r) ? aP[x][y] : 0.f;
+            }
+            *reinterpret_cast<float4*>(Ac + r * CB + i0) = va;
+            *reinterpret_cast<float4*>(Pc + r * CB + i0) = vp;
         }
     }
-    // right-hand sides [b Kt | b V]
-    for (int idx = tid; idx < CB * dk; idx += nt) {
-        const int r = idx / dk, c = idx % dk;
-        X[r * ldx + c] = bs[r] * Ks[r * ldk + c] * __expf(Gs[r * ldk + c]);
+    // the tiles above the diagonal are zero
+    for (int idx = tid; idx < CB * CB / 4; idx += 256) {
+        const int r = idx / (CB / 4), i4 = idx % (CB / 4);
+        if (i4 > r / 4) {
+            *reinterpret_cast<float4*>(Ac + r * CB + 4 * i4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(Pc + r * CB + 4 * i4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
-    for (int idx = tid; idx < CB * dv; idx += nt) {
-        const int r = idx / dv, j = idx % dv;
-        X[r * ldx + dk + j] = r < L ? bs[r] * to_f32(v[((size_t)(ci.y + r) * H + h) * dv + j]) : 0.f;
+    // Kb = K exp(G_last - G) and the right-hand sides b K exp(G)
+    for (int idx = tid; idx < L * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        const size_t gi = row0 + r * rstride + c;
+        const float gr = Gs[r * LDK + c], kr = Ks[r * LDK + c];
+        Kb[gi] = kr * __expf(Gs[(L - 1) * LDK + c] - gr);
+        Rk[gi] = beta[(size_t)(ci.y + r) * H + h] * kr * __expf(gr);
+    }
+}
+
+template <int DK, typename TIn>
+__global__ void __launch_bounds__(256) bwd_subst_kernel(
+    const TIn* __restrict__ v, const float* __restrict__ beta, const float* __restrict__ Ain,
+    const int4* __restrict__ info, int H, int dv, const uint32_t* status,
+    float* __restrict__ W, float* __restrict__ Ut) {
+    if (status_bad(status)) return;
+    const int cidx = blockIdx.x, h = blockIdx.y;
+    const int4 ci = info[cidx];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int tid = threadIdx.x;
+    extern __shared__ __align__(16) float sm[];
+    const int lda = CB + 1, ldx = DK + dv + 1;
+    float* As = sm;
+    float* X = As + CB * lda;
+    float* bs = X + CB * ldx;
+    const float* Ac = Ain + ((size_t)cidx * H + h) * CB * CB;
+    for (int idx = tid; idx < CB * CB; idx += 256) As[(idx / CB) * lda + idx % CB] = Ac[idx];
+    for (int r = tid; r < L; r += 256) bs[r] = beta[(size_t)(ci.y + r) * H + h];
+    for (int idx = tid; idx < L * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        X[r * ldx + c] = W[((size_t)(ci.y + r) * H + h) * DK + c];
     }
     __syncthreads();
-    {
-        float* Ac = Ar_out + ((size_t)cidx * H + h) * CB * CB;
-        for (int idx = tid; idx < CB * CB; idx += nt) {
-            const int r = idx / CB, i = idx % CB;
-            Ac[idx] = i < r ? As[r * lda + i] : 0.f;
-        }
+    for (int idx = tid; idx < L * dv; idx += 256) {
+        const int r = idx / dv, j = idx % dv;
+        X[r * ldx + DK + j] = bs[r] * to_f32(v[((size_t)(ci.y + r) * H + h) * dv + j]);
     }
-    // a2: (I + A) [W | Ut] = X by forward substitution, one column per
-    // thread, four partial sums per row
-    for (int col = tid; col < dk + dv; col += nt) {
+    __syncthreads();
+    // one column per thread, four partial sums per row
+    for (int col = tid; col < DK + dv; col += 256) {
         for (int r = 1; r < L; ++r) {
             const float* ar = As + r * lda;
             float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
@@ -229,41 +266,63 @@ __global__ void __launch_bounds__(256) bwd_intra_kernel(
         }
     }
     __syncthreads();
-    for (int idx = tid; idx < L * dk; idx += nt) {
-        const int r = idx / dk, c = idx % dk;
-        const size_t gi = ((size_t)(ci.y + r) * H + h) * dk + c;
-        const float gr = Gs[r * ldk + c];
-        W[gi] = X[r * ldx + c];
-        Kb[gi] = Ks[r * ldk + c] * __expf(Gs[(L - 1) * ldk + c] - gr);
-        Qs[r * ldq + c] *= __expf(gr);
+    for (int idx = tid; idx < L * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        W[((size_t)(ci.y + r) * H + h) * DK + c] = X[r * ldx + c];
     }
-    for (int idx = tid; idx < L * dv; idx += nt) {
+    for (int idx = tid; idx < L * dv; idx += 256) {
         const int r = idx / dv, j = idx % dv;
-        Ut[((size_t)(ci.y + r) * H + h) * dv + j] = X[r * ldx + dk + j];
+        Ut[((size_t)(ci.y + r) * H + h) * dv + j] = X[r * ldx + DK + j];
     }
-    // E = P^T dO and F = Qt^T dO - W^T E, one slice of DVS columns at a time;
-    // F by 4 x 4 register tiles (channels 4 c4 + x, columns 4 j4 + y)
-    float* Fc = F + ((size_t)cidx * H + h) * dk * dv;
+}
+
+template <int DK, typename TIn>
+__global__ void __launch_bounds__(256) bwd_ef_kernel(
+    const TIn* __restrict__ q, const TIn* __restrict__ dout, const float* __restrict__ G,
+    const float* __restrict__ Pin, const float* __restrict__ W, const int4* __restrict__ info,
+    int H, int dv, const uint32_t* status, float* __restrict__ E, float* __restrict__ F) {
+    constexpr int LDQ = DK + 4, LDS = DVS + 4, LDA = CB + 1;
+    if (status_bad(status)) return;
+    const int cidx = blockIdx.x, h = blockIdx.y;
+    const int4 ci = info[cidx];
+    const int L = ci.z;
+    if (L <= 0) return;
+    const int tid = threadIdx.x;
+    extern __shared__ __align__(16) float sm[];
+    float* Qs = sm;                // Qt [C][LDQ]
+    float* Ws = Qs + CB * LDQ;     // [C][LDQ]
+    float* Ps = Ws + CB * LDQ;     // [C][LDA]
+    float* Ds = Ps + CB * LDA;     // [C][LDS]
+    float* Es = Ds + CB * LDS;     // [C][LDS]
+    const float* Pc = Pin + ((size_t)cidx * H + h) * CB * CB;
+    for (int idx = tid; idx < CB * CB; idx += 256) Ps[(idx / CB) * LDA + idx % CB] = Pc[idx];
+    for (int idx = tid; idx < L * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        const size_t gi = ((size_t)(ci.y + r) * H + h) * DK + c;
+        Qs[r * LDQ + c] = to_f32(q[gi]) * __expf(G[gi]);
+        Ws[r * LDQ + c] = W[gi];
+    }
+    float* Fc = F + ((size_t)cidx * H + h) * DK * dv;
     for (int j0 = 0; j0 < dv; j0 += DVS) {
         __syncthreads();
-        for (int idx = tid; idx < CB * DVS; idx += nt) {
+        for (int idx = tid; idx < CB * DVS; idx += 256) {
             const int r = idx / DVS, j = idx % DVS;
-            Ds[r * lds + j] =
+            Ds[r * LDS + j] =
                 r < L ? to_f32(dout[((size_t)(ci.y + r) * H + h) * dv + j0 + j]) : 0.f;
         }
         __syncthreads();
         // E rows 2 ip, 2 ip + 1, columns jq + 8 y (P[r][i] = 0 for i > r
         // inside a diagonal 4 x 4 tile, so both rows start at r = 2 ip)
-        for (int t = tid; t < (CB / 2) * (DVS / 4); t += nt) {
+        for (int t = tid; t < (CB / 2) * (DVS / 4); t += 256) {
             const int jq = t % (DVS / 4), ip = t / (DVS / 4);
             const int i = 2 * ip;
             float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
             for (int r = i; r < L; ++r) {
-                const float p0 = Ps[r * lda + i], p1 = Ps[r * lda + i + 1];
+                const float p0 = Ps[r * LDA + i], p1 = Ps[r * LDA + i + 1];
 #pragma unroll
                 for (int y = 0; y < 4; ++y) {
-                    const float d = Ds[r * lds + jq + 8 * y];
+                    const float d = Ds[r * LDS + jq + 8 * y];
                     e0[y] += p0 * d;
                     e1[y] += p1 * d;
                 }
@@ -271,26 +330,26 @@ __global__ void __launch_bounds__(256) bwd_intra_kernel(
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
                 const int j = jq + 8 * y;
-                Es[i * lds + j] = e0[y];
-                Es[(i + 1) * lds + j] = e1[y];
+                Es[i * LDS + j] = e0[y];
+                Es[(i + 1) * LDS + j] = e1[y];
                 if (i < L) E[((size_t)(ci.y + i) * H + h) * dv + j0 + j] = e0[y];
                 if (i + 1 < L) E[((size_t)(ci.y + i + 1) * H + h) * dv + j0 + j] = e1[y];
             }
         }
         __syncthreads();
-        for (int t = tid; t < (dk / 4) * (DVS / 4); t += nt) {
+        // F by 4 x 4 register tiles (channels 4 c4 + x, columns 4 j4 + y)
+        for (int t = tid; t < (DK / 4) * (DVS / 4); t += 256) {
             const int j4 = t % (DVS / 4), c4 = t / (DVS / 4);
             float acc[4][4];
 #pragma unroll
             for (int x = 0; x < 4; ++x)
 #pragma unroll
                 for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
-#pragma unroll 2
             for (int r = 0; r < L; ++r) {
-                const float4 q4 = *reinterpret_cast<const float4*>(Qs + r * ldq + 4 * c4);
-                const float4 w4 = *reinterpret_cast<const float4*>(X + r * ldx + 4 * c4);
-                const float4 d4 = *reinterpret_cast<const float4*>(Ds + r * lds + 4 * j4);
-                const float4 e4 = *reinterpret_cast<const float4*>(Es + r * lds + 4 * j4);
+                const float4 q4 = *reinterpret_cast<const float4*>(Qs + r * LDQ + 4 * c4);
+                const float4 w4 = *reinterpret_cast<const float4*>(Ws + r * LDQ + 4 * c4);
+                const float4 d4 = *reinterpret_cast<const float4*>(Ds + r * LDS + 4 * j4);
+                const float4 e4 = *reinterpret_cast<const float4*>(Es + r * LDS + 4 * j4);
                 const float qv[4] = {q4.x, q4.y, q4.z, q4.w}, wv[4] = {w4.x, w4.y, w4.z, w4.w};
                 const float dd[4] = {d4.x, d4.y, d4.z, d4.w}, ev[4] = {e4.x, e4.y, e4.z, e4.w};
 #pragma unroll
@@ -306,9 +365,12 @@ __global__ void __launch_bounds__(256) bwd_intra_kernel(
     }
 }
 
-size_t intra_smem(int dk, int dv) {
-    return sizeof(float) * ((size_t)CB * (dk + 4) + (size_t)2 * CB * (dk + 1) +
-                            (size_t)2 * CB * (CB + 1) + (size_t)CB * (dk + dv + 4) + CB +
+size_t apkb_smem(int dk) { return sizeof(float) * (size_t)3 * CB * (dk + 1); }
+size_t subst_smem(int dk, int dv) {
+    return sizeof(float) * ((size_t)CB * (CB + 1) + (size_t)CB * (dk + dv + 1) + CB);
+}
+size_t ef_smem(int dk) {
+    return sizeof(float) * ((size_t)2 * CB * (dk + 4) + (size_t)CB * (CB + 1) +
                             (size_t)2 * CB * (DVS + 4));
 }
 
@@ -797,6 +859,30 @@ cudaError_t launch_dense(const BwdBufs& b, const TIn* K, const TIn* DO, const fl
     return cudaGetLastError();
 }
 
+template <int DK, typename TIn>
+cudaError_t launch_intra3(const BwdBufs& b, const TIn* Q, const TIn* K, const TIn* V,
+                          const TIn* DO, const float* g, const float* beta, int maxc, int H,
+                          int dv, cudaStream_t st) {
+    const Workspace& w = b.w;
+    const dim3 grid(maxc, H);
+    cudaError_t e;
+    size_t sm = apkb_smem(DK);
+    if ((e = set_smem(bwd_apkb_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
+    bwd_apkb_kernel<DK, TIn><<<grid, 256, sm, st>>>(Q, K, g, beta, w.chunk_info, H, w.status,
+                                                    w.G, b.Ar, b.Pm, b.Kb, w.W);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    sm = subst_smem(DK, dv);
+    if ((e = set_smem(bwd_subst_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
+    bwd_subst_kernel<DK, TIn><<<grid, 256, sm, st>>>(V, beta, b.Ar, w.chunk_info, H, dv,
+                                                     w.status, w.W, w.U);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    sm = ef_smem(DK);
+    if ((e = set_smem(bwd_ef_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
+    bwd_ef_kernel<DK, TIn><<<grid, 256, sm, st>>>(Q, DO, w.G, b.Pm, w.W, w.chunk_info, H, dv,
+                                                  w.status, b.E, b.F);
+    return cudaGetLastError();
+}
+
 template <typename TIn>
 cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* v,
                     const float* g, const float* beta, const float* h0, const void* dout,
@@ -810,12 +896,10 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
     const Workspace& w = b.w;
     cudaError_t e;
     if (maxc > 0) {
-        const size_t sm = intra_smem(dk, dv);
-        if ((e = set_smem(bwd_intra_kernel<TIn>, sm)) != cudaSuccess) return e;
-        bwd_intra_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(Q, K, V, DO, g, beta, w.chunk_info,
-                                                             H, dk, dv, w.status, w.G, w.W, w.U,
-                                                             b.Ar, b.Kb, b.E, b.F);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = dk == 128 ? launch_intra3<128, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st)
+            : dk == 64 ? launch_intra3<64, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st)
+                       : launch_intra3<32, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st);
+        if (e != cudaSuccess) return e;
     }
     {
         const size_t sm = chain_smem();
