@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(256) bwd_subst_kernel(
     if (L <= 0) return;
     const int tid = threadIdx.x;
     extern __shared__ __align__(16) float sm[];
-    const int lda = CB + 1, ldx = DK + dv + 1;
+    const int lda = CB + 1, ldx = DK + dv + 4, nc = DK + dv;
     float* As = sm;
     float* X = As + CB * lda;
     float* bs = X + CB * ldx;
@@ -249,21 +249,52 @@ __global__ void __launch_bounds__(256) bwd_subst_kernel(
         X[r * ldx + DK + j] = bs[r] * to_f32(v[((size_t)(ci.y + r) * H + h) * dv + j]);
     }
     __syncthreads();
-    // one column per thread, four partial sums per row
-    for (int col = tid; col < DK + dv; col += 256) {
-        for (int r = 1; r < L; ++r) {
-            const float* ar = As + r * lda;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            int i = 0;
-            for (; i + 4 <= r; i += 4) {
-                a0 += ar[i] * X[i * ldx + col];
-                a1 += ar[i + 1] * X[(i + 1) * ldx + col];
-                a2 += ar[i + 2] * X[(i + 2) * ldx + col];
-                a3 += ar[i + 3] * X[(i + 3) * ldx + col];
+    // blocks of 16 rows: first the rows above the block (4 x 4 register
+    // tiles, one task per 4 rows and 4 columns), then the block itself, one
+    // column per thread
+    for (int r0 = 0; r0 < L; r0 += 16) {
+        if (r0 > 0) {
+            for (int t = tid; t < 4 * (nc / 4); t += 256) {
+                const int rq = t / (nc / 4), cq = t % (nc / 4);
+                const int ra = r0 + 4 * rq;
+                if (ra >= L) continue;
+                float acc[4][4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+                for (int i = 0; i < r0; ++i) {
+                    const float4 xv = *reinterpret_cast<const float4*>(X + i * ldx + 4 * cq);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const float a = As[(ra + x) * lda + i];
+                        acc[x][0] += a * xv.x; acc[x][1] += a * xv.y;
+                        acc[x][2] += a * xv.z; acc[x][3] += a * xv.w;
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    if (ra + x >= L) break;
+                    float4* dst = reinterpret_cast<float4*>(X + (ra + x) * ldx + 4 * cq);
+                    float4 cur = *dst;
+                    const float b = bs[ra + x];
+                    cur.x -= b * acc[x][0]; cur.y -= b * acc[x][1];
+                    cur.z -= b * acc[x][2]; cur.w -= b * acc[x][3];
+                    *dst = cur;
+                }
             }
-            for (; i < r; ++i) a0 += ar[i] * X[i * ldx + col];
-            X[r * ldx + col] -= bs[r] * ((a0 + a1) + (a2 + a3));
+            __syncthreads();
         }
+        const int r1 = min(r0 + 16, L);
+        for (int col = tid; col < nc; col += 256) {
+            for (int r = r0 + 1; r < r1; ++r) {
+                float acc = 0.f;
+                for (int i = r0; i < r; ++i) acc += As[r * lda + i] * X[i * ldx + col];
+                X[r * ldx + col] -= bs[r] * acc;
+            }
+        }
+        __syncthreads();
     }
     __syncthreads();
     for (int idx = tid; idx < L * DK; idx += 256) {
@@ -367,7 +398,7 @@ __global__ void __launch_bounds__(256) bwd_ef_kernel(
 
 size_t apkb_smem(int dk) { return sizeof(float) * (size_t)3 * CB * (dk + 1); }
 size_t subst_smem(int dk, int dv) {
-    return sizeof(float) * ((size_t)CB * (CB + 1) + (size_t)CB * (dk + dv + 1) + CB);
+    return sizeof(float) * ((size_t)CB * (CB + 1) + (size_t)CB * (dk + dv + 4) + CB);
 }
 size_t ef_smem(int dk) {
     return sizeof(float) * ((size_t)2 * CB * (dk + 4) + (size_t)CB * (CB + 1) +
@@ -538,7 +569,7 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
     if (L <= 0) return;
     const int tid = threadIdx.x, nt = blockDim.x;
     extern __shared__ float sm[];
-    const int lda = CB + 1, ldy = dv + 1, lds = DVS + 1;
+    const int lda = CB + 1, ldy = dv + 4, lds = DVS + 1;
     float* Ar = sm;
     float* bs = Ar + CB * lda;
     float* Ys = bs + CB;
@@ -555,23 +586,53 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
         Ys[r * ldy + j] = dU[((size_t)(ci.y + r) * H + h) * dv + j];
     }
     __syncthreads();
-    // (I + A)^T Y = dU by back substitution, one column per thread:
-    // Y_r = dU_r - sum_{i > r} b_i A[i][r] Y_i
-    for (int col = tid; col < dv; col += nt) {
-        for (int r = L - 2; r >= 0; --r) {
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-            int i = r + 1;
-            for (; i + 4 <= L; i += 4) {
-                a0 += bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
-                a1 += bs[i + 1] * Ar[(i + 1) * lda + r] * Ys[(i + 1) * ldy + col];
-                a2 += bs[i + 2] * Ar[(i + 2) * lda + r] * Ys[(i + 2) * ldy + col];
-                a3 += bs[i + 3] * Ar[(i + 3) * lda + r] * Ys[(i + 3) * ldy + col];
+    // (I + A)^T Y = dU by back substitution, Y_r = dU_r - sum_{i > r} b_i
+    // A[i][r] Y_i, in blocks of 16 rows from the last: first the rows below
+    // the block (4 x 4 register tiles), then the block, one column per thread
+    for (int r1 = L; r1 > 0; r1 -= 16) {
+        const int r0 = max(r1 - 16, 0);
+        if (r1 < L) {
+            for (int t = tid; t < 4 * (dv / 4); t += nt) {
+                const int rq = t / (dv / 4), cq = t % (dv / 4);
+                const int ra = r0 + 4 * rq;
+                if (ra >= r1) continue;
+                float acc[4][4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+                for (int i = r1; i < L; ++i) {
+                    const float4 yv = *reinterpret_cast<const float4*>(Ys + i * ldy + 4 * cq);
+                    const float bi = bs[i];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const float a = bi * Ar[i * lda + ra + x];
+                        acc[x][0] += a * yv.x; acc[x][1] += a * yv.y;
+                        acc[x][2] += a * yv.z; acc[x][3] += a * yv.w;
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    if (ra + x >= r1) break;
+                    float4* dst = reinterpret_cast<float4*>(Ys + (ra + x) * ldy + 4 * cq);
+                    float4 cur = *dst;
+                    cur.x -= acc[x][0]; cur.y -= acc[x][1];
+                    cur.z -= acc[x][2]; cur.w -= acc[x][3];
+                    *dst = cur;
+                }
             }
-            for (; i < L; ++i) a0 += bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
-            Ys[r * ldy + col] -= (a0 + a1) + (a2 + a3);
+            __syncthreads();
         }
+        for (int col = tid; col < dv; col += nt) {
+            for (int r = r1 - 2; r >= r0; --r) {
+                float acc = 0.f;
+                for (int i = r + 1; i < r1; ++i) acc += bs[i] * Ar[i * lda + r] * Ys[i * ldy + col];
+                Ys[r * ldy + col] -= acc;
+            }
+        }
+        __syncthreads();
     }
-    __syncthreads();
     for (int idx = tid; idx < L * dv; idx += nt) {
         const int r = idx / dv, j = idx % dv;
         const size_t vi = ((size_t)(ci.y + r) * H + h) * dv + j;
@@ -629,7 +690,7 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
 
 size_t solve_smem(int dv) {
     return sizeof(float) * ((size_t)CB * (CB + 1) + CB +
-                            (size_t)CB * (dv + 1) + (size_t)3 * CB * (DVS + 1));
+                            (size_t)CB * (dv + 4) + (size_t)3 * CB * (DVS + 1));
 }
 
 // ------------------------------------------------------------ b4: dense
