@@ -673,6 +673,24 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_backward_only(args):
+    """kda_chunk_bwd alone on the prefill workload (one GPU)."""
+    import torch
+
+    import gated_delta_rule_124_b200 as kda
+    from gated_delta_rule_124_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kda.load()
+    pc = prefill_case(wl, args)
+    P = pc.to(dev)
+    bwd = backward_times(kda, torch, P, pc, dev, torch.cuda.current_stream(),
+                         reps=max(3, min(20, args.steps)),
+                         oracle_sample=not args.no_cpu_baseline)
+    return {"backward": bwd, "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": pc.H,
+                                        "dk": pc.dk, "dv": pc.dv}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -684,6 +702,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward timing beside the step")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only kda_chunk_bwd on the prefill workload and print its "
+                         "entry (for profiling the backward kernels alone)")
     ap.add_argument("--prefill-config", type=int, default=1, choices=[1, 2, 3],
                     help="prefill workload: 1 = B=2 x T=2048 (default), 2 = B=1 x T=65536, "
                          "3 = 16 packed sequences of U[1024,16384] tokens")
@@ -700,6 +721,10 @@ def main():
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+    if args.backward_only:
+        if rank == 0:
+            print(json.dumps(run_backward_only(args)), flush=True)
         return
     if world > 1:
         import datetime
