@@ -508,7 +508,7 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None, ora
     fl = backward_flops(total * H, dk, dv)
     mhz = sm_max_mhz or 1965.0
     peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-    res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 7,
+    res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 9,
            "roofline": {"bound": "alu", "achieved": fl / t / 1e12, "peak": peak,
                         "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak,
                         "peak_kind": f"fp32 CUDA cores, 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",

@@ -276,10 +276,12 @@ kda_status_t kda_gdn_decode_step(const void* q, const void* k, const void* v, co
  * dfinal_state) for the forward kda_chunk_fwd computes (same inputs, shapes
  * and sequence description), with respect to q, k, v, g, beta and the
  * initial state.  The pages give no backward equations; they are derived from
- * the token recurrence (Kimi Linear (aiwiki.ai), "Kimi Delta Attention") and
- * evaluated recurrently, token by token, one CTA per (sequence, head, 32 value
- * columns), with the states rebuilt from checkpoints every 8 tokens kept in
- * the workspace: correct, and much slower than the forward.
+ * the chunk form (Kimi Linear (aiwiki.ai), "The constrained DPLR form and the
+ * chunkwise algorithm"; chunks of 64 tokens): the forward's per-chunk
+ * quantities and entry states are recomputed, a reverse pass over each
+ * sequence's chunks carries the state gradient, and per-chunk kernels form
+ * the token gradients.  Nine kernel launches on `stream`, fp32 arithmetic on
+ * the CUDA cores.
  * In:  q, k [total, H, dk], v [total, H, dv], dout [total, H, dv] (dtype);
  *      g [total, H, dk], beta [total, H] fp32; initial_state [num_seqs, H, dk,
  *      dv] fp32 or NULL (zeros); dfinal_state likewise or NULL (zeros).
@@ -287,9 +289,13 @@ kda_status_t kda_gdn_decode_step(const void* q, const void* k, const void* v, co
  *      [total, H] -- all fp32; dinitial_state [num_seqs, H, dk, dv] fp32 or
  *      NULL (not written).
  * Workspace: kda_chunk_bwd_workspace_size() bytes, 256-byte aligned (the
- *      checkpoints: about total * H * dk * dv / 2 bytes, plus per-slice
- *      partial sums).  Shapes: dk, dv in {32, 64, 128}.  cu_seqlens must be
- *      valid (0 .. T, non-decreasing): it is not checked on the device here.
+ *      forward's intermediates and per-chunk states, the backward's per-token
+ *      and per-chunk gradients: about 4 * (total * H * (6 dk + 4 dv + 1) +
+ *      chunks * H * (3 dk dv + 4 * 64 * 64 + dk)) bytes, chunks <= (total +
+ *      63 num_seqs) / 64).  It starts with the same status word as the
+ *      prefill workspace: invalid device cu_seqlens (not 0 .. T, or
+ *      decreasing) leave the outputs unwritten and are reported by
+ *      kda_get_device_status(workspace).  Shapes: dk, dv in {32, 64, 128}.
  */
 size_t kda_chunk_bwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv);
 

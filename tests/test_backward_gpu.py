@@ -100,3 +100,26 @@ def test_backward_bench_workload_sampled_heads(unit):
            got[5][s:s + 1, h:h + 1])
     for name_, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), sel, ref):
         assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
+
+
+def test_backward_bad_cu_seqlens_reported_on_device():
+    """Invalid device cu_seqlens: the chunk table flags them, every later kernel
+    returns before reading them, and the status word says so; a good call on
+    the same workspace clears it."""
+    case = wl.make_prefill(508, [40, 40], H=1, dk=32, dv=32, chunk=64, dtype="f32", varlen=True)
+    c = case.to("cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    outs = [torch.zeros(80, 1, 32, **f32) for _ in range(4)]
+    db, dh0 = torch.zeros(80, 1, **f32), torch.zeros(2, 1, 32, 32, **f32)
+    do = torch.randn(80, 1, 32, device="cuda")
+    ws = torch.empty(kda.kda_chunk_bwd_workspace_size(80, 2, 1, 32, 32), dtype=torch.uint8,
+                     device="cuda")
+    call = lambda cu: kda.kda_chunk_bwd(c.q, c.k, c.v, c.g, c.beta, None, do, None, cu, 1, 80, 2,
+                                        1, 32, 32, "f32", outs[0], outs[1], outs[2], outs[3],
+                                        db, dh0, ws)
+    call(torch.tensor([0, 50, 40], dtype=torch.int32, device="cuda"))  # not monotone
+    assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
+    call(torch.tensor([0, 30, 70], dtype=torch.int32, device="cuda"))  # wrong total
+    assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
+    call(c.cu_seqlens)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
