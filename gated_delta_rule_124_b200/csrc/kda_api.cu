@@ -497,6 +497,38 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
                                      static_cast<cudaStream_t>(stream)));
 }
 
+size_t kda_gdn_chunk_bwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv) {
+    if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv)) return 0;
+    return kda::bwd_head_gate_workspace_bytes(total_tokens, num_seqs, H, dk, dv);
+}
+
+kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* initial_state, const void* dout,
+                               const float* dfinal_state, const int32_t* cu_seqlens, int B, int T,
+                               int num_seqs, int H, int dk, int dv, kda_dtype_t dtype, float* dq,
+                               float* dk_out, float* dv_out, float* dg, float* dbeta,
+                               float* dinitial_state, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+    Prefill p;
+    kda_status_t s = check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, 64, dtype, &p);
+    if (s != KDA_OK) return s;
+    for (const void* ptr : std::initializer_list<const void*>{
+             q, k, v, (const void*)g, (const void*)beta, dout, (const void*)dq,
+             (const void*)dk_out, (const void*)dv_out, (const void*)dg, (const void*)dbeta})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : std::initializer_list<const void*>{
+             (const void*)initial_state, (const void*)dfinal_state, (const void*)dinitial_state})
+        if (ptr && !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return KDA_ERR_INVALID_ARG;
+    if (workspace_bytes < kda::bwd_head_gate_workspace_bytes(p.total, p.N, H, dk, dv))
+        return KDA_ERR_WORKSPACE;
+    return from_cuda(kda::launch_bwd_head_gate(
+        q, k, v, g, beta, initial_state, dout, dfinal_state, cu_seqlens, T, p.N, H, dk, dv, dtype,
+        dq, dk_out, dv_out, dg, dbeta, dinitial_state, workspace,
+        static_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------------ layer steps (NEXT-2)
 
 kda_status_t kda_qkv_conv_norm(const void* xq, const void* xk, const void* xv, const float* wq,

@@ -999,7 +999,49 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
     return cudaGetLastError();
 }
 
+// dg_head[row] = sum over the dk channels of dg[row, :] (one warp per row):
+// the gradient of a head-uniform gate spread over the channels
+__global__ void sum_channels_kernel(const float* __restrict__ x, long long rows, int dk,
+                                    float* __restrict__ out) {
+    const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float acc = 0.f;
+    for (int c = lane; c < dk; c += 32) acc += x[row * dk + c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) out[row] = acc;
+}
+
 }  // namespace
+
+size_t bwd_head_gate_workspace_bytes(int total, int N, int H, int dk, int dv) {
+    return align_up(bwd_workspace_bytes(total, N, H, dk, dv)) +
+           2 * align_up(sizeof(float) * (size_t)total * H * dk);
+}
+
+cudaError_t launch_bwd_head_gate(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, const float* h0, const void* dout,
+                                 const float* dhT, const int32_t* cu, int T, int N, int H, int dk,
+                                 int dv, kda_dtype_t dt, float* dq, float* dkk, float* dvv,
+                                 float* dg_head, float* db, float* dh0, void* workspace,
+                                 cudaStream_t st) {
+    const int total = cu ? T : N * T;
+    char* base = static_cast<char*>(workspace);
+    const size_t off = align_up(bwd_workspace_bytes(total, N, H, dk, dv));
+    float* g_full = reinterpret_cast<float*>(base + off);
+    float* dg_full =
+        reinterpret_cast<float*>(base + off + align_up(sizeof(float) * (size_t)total * H * dk));
+    cudaError_t e = launch_spread_gate(g, total, H, dk, g_full, st);
+    if (e == cudaSuccess)
+        e = launch_bwd(q, k, v, g_full, beta, h0, dout, dhT, cu, T, N, H, dk, dv, dt, dq, dkk,
+                       dvv, dg_full, db, dh0, workspace, st);
+    if (e != cudaSuccess || total == 0) return e;
+    const long long rows = (long long)total * H;
+    sum_channels_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(dg_full, rows, dk,
+                                                                              dg_head);
+    return cudaGetLastError();
+}
 
 size_t bwd_workspace_bytes(int total, int N, int H, int dk, int dv) {
     return carve_bwd(nullptr, total, N, H, dk, dv).bytes;

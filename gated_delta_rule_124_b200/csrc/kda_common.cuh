@@ -142,6 +142,15 @@ cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float*
                        const int32_t* cu, int T, int N, int H, int dk, int dv, kda_dtype_t dt,
                        float* dq, float* dkk, float* dvv, float* dg, float* db, float* dh0,
                        void* workspace, cudaStream_t st);
+// the backward with a head-uniform gate g [total, H]: spread over the channels,
+// the per-channel backward, the channel gradients summed into dg_head [total, H]
+size_t bwd_head_gate_workspace_bytes(int total, int N, int H, int dk, int dv);
+cudaError_t launch_bwd_head_gate(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, const float* h0, const void* dout,
+                                 const float* dhT, const int32_t* cu, int T, int N, int H, int dk,
+                                 int dv, kda_dtype_t dt, float* dq, float* dkk, float* dvv,
+                                 float* dg_head, float* db, float* dh0, void* workspace,
+                                 cudaStream_t st);
 // G_full[t, h, c] = g[t, h] (a head-uniform gate spread over dk channels)
 cudaError_t launch_spread_gate(const float* g, int total, int H, int dk, float* out,
                                cudaStream_t st);

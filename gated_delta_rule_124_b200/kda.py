@@ -42,6 +42,7 @@ EXPORTS = (
     "kda_chunk_split_chain", "kda_chunk_fwd_plan", "kda_qkv_conv_norm",
     "kda_output_norm_gate", "kda_gdn_chunk_fwd_workspace_size", "kda_gdn_chunk_fwd",
     "kda_gdn_decode_step", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
+    "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd",
 )
 
 
@@ -76,6 +77,8 @@ _SIGS = {
     "kda_gdn_decode_step": ([_vp] * 7 + [_i] * 5 + [_vp], _i),
     "kda_chunk_bwd_workspace_size": ([_i] * 5, _sz),
     "kda_chunk_bwd": ([_vp] * 9 + [_i] * 7 + [_vp] * 7 + [_sz, _vp], _i),
+    "kda_gdn_chunk_bwd_workspace_size": ([_i] * 5, _sz),
+    "kda_gdn_chunk_bwd": ([_vp] * 9 + [_i] * 7 + [_vp] * 7 + [_sz, _vp], _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
@@ -273,6 +276,22 @@ def kda_chunk_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_seqlen
                               _p(dbeta), _p(dinitial_state), _p(workspace), wb,
                               _stream(stream))
     return _ret(st, "kda_chunk_bwd", check)
+
+
+def kda_gdn_chunk_bwd_workspace_size(total_tokens, num_seqs, H, dk, dv) -> int:
+    return int(load().kda_gdn_chunk_bwd_workspace_size(total_tokens, num_seqs, H, dk, dv))
+
+
+def kda_gdn_chunk_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_seqlens, B, T,
+                      num_seqs, H, dk, dv, dtype, dq, dk_out, dv_out, dg, dbeta, dinitial_state,
+                      workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_gdn_chunk_bwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
+                                  _p(dout), _p(dfinal_state), _p(cu_seqlens), B, T, num_seqs, H,
+                                  dk, dv, dtype_code(dtype), _p(dq), _p(dk_out), _p(dv_out),
+                                  _p(dg), _p(dbeta), _p(dinitial_state), _p(workspace), wb,
+                                  _stream(stream))
+    return _ret(st, "kda_gdn_chunk_bwd", check)
 
 
 def kda_qkv_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens, B, T, num_seqs, H, dk, dv, dtype,

@@ -307,6 +307,25 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
                            float* dinitial_state, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/* kda_gdn_chunk_bwd: the same gradients for Gated DeltaNet (Kimi Linear
+ * (aiwiki.ai), "Kimi Delta Attention": one gate value per token and head).
+ * g and dg are [total, H] fp32; every other argument is as in kda_chunk_bwd.
+ * The gate is spread over the dk channels, the per-channel backward runs, and
+ * dg[t, h] is the sum of the channel gradients (the chain rule of the
+ * spread).  Workspace: kda_gdn_chunk_bwd_workspace_size() bytes (the
+ * kda_chunk_bwd workspace plus two [total, H, dk] fp32 arrays), 256-byte
+ * aligned; the status word is read the same way.
+ */
+size_t kda_gdn_chunk_bwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv);
+
+kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, const float* initial_state, const void* dout,
+                               const float* dfinal_state, const int32_t* cu_seqlens, int B, int T,
+                               int num_seqs, int H, int dk, int dv, kda_dtype_t dtype, float* dq,
+                               float* dk_out, float* dv_out, float* dg, float* dbeta,
+                               float* dinitial_state, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* ---------------------------------------- the steps around the operator
  * Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
  * algorithm" (the paragraph on what each KDA head applies): a short depthwise

@@ -205,3 +205,19 @@ def test_backward_call_rejects_bad_arguments(lib):
     assert kda.kda_chunk_bwd(**{**a, "dinitial_state": FAKE + 8}) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_chunk_bwd(**{**a, "dk": 48}) == kda.KDA_ERR_UNSUPPORTED
     assert kda.kda_chunk_bwd(**a) == kda.KDA_ERR_WORKSPACE
+
+
+def test_gdn_backward_call_rejects_bad_arguments(lib):
+    n = kda.kda_chunk_bwd_workspace_size(4096, 2, 32, 128, 128)
+    m = kda.kda_gdn_chunk_bwd_workspace_size(4096, 2, 32, 128, 128)
+    assert m >= n + 2 * 4096 * 32 * 128 * 4  # the spread gate and its gradient
+    assert kda.kda_gdn_chunk_bwd_workspace_size(4096, 2, 32, 128, 40) == 0
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, initial_state=None, dout=FAKE,
+             dfinal_state=None, cu_seqlens=None, B=1, T=64, num_seqs=1, H=1, dk=32, dv=32,
+             dtype="f32", dq=FAKE, dk_out=FAKE, dv_out=FAKE, dg=FAKE, dbeta=FAKE,
+             dinitial_state=None, workspace=FAKE * 2, workspace_bytes=16, stream=0, check=False)
+    assert kda.kda_gdn_chunk_bwd(**{**a, "g": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_gdn_chunk_bwd(**{**a, "dg": FAKE + 4}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_gdn_chunk_bwd(**{**a, "dv": 40}) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_gdn_chunk_bwd(**{**a, "num_seqs": 2}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_gdn_chunk_bwd(**a) == kda.KDA_ERR_WORKSPACE

@@ -123,3 +123,38 @@ def test_backward_bad_cu_seqlens_reported_on_device():
     assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
     call(c.cu_seqlens)
     assert kda.kda_get_device_status(ws) == kda.KDA_OK
+
+
+@pytest.mark.parametrize("with_dhT", [True, False])
+def test_gdn_backward_head_gate(with_dhT):
+    """Gated DeltaNet: one gate value per (token, head).  The oracle runs on the
+    gate spread over the dk channels; the gate's gradient is the sum of the
+    per-channel ones (the chain rule of the spread)."""
+    case = wl.make_prefill(509, [70, 0, 45], H=2, dk=64, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    gen = torch.Generator().manual_seed(13)
+    gh = -torch.nn.functional.softplus(torch.randn(case.total, case.H, generator=gen))
+    do = torch.randn(case.total, case.H, case.dv, generator=gen).to(torch.bfloat16)
+    dhT = torch.randn(case.N, case.H, case.dk, case.dv, generator=gen) if with_dhT else None
+    c = case.to("cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dq = torch.full((c.total, c.H, c.dk), float("nan"), **f32)
+    dk, dv = torch.full_like(dq, float("nan")), torch.full((c.total, c.H, c.dv), float("nan"), **f32)
+    dg = torch.full((c.total, c.H), float("nan"), **f32)
+    db = torch.full((c.total, c.H), float("nan"), **f32)
+    dh0 = torch.full((c.N, c.H, c.dk, c.dv), float("nan"), **f32)
+    ws = torch.empty(kda.kda_gdn_chunk_bwd_workspace_size(c.total, c.N, c.H, c.dk, c.dv),
+                     dtype=torch.uint8, device="cuda")
+    kda.kda_gdn_chunk_bwd(c.q, c.k, c.v, gh.cuda(), c.beta, c.initial_state, do.cuda(),
+                          None if dhT is None else dhT.cuda(), c.cu_seqlens, 1, c.total, c.N,
+                          c.H, c.dk, c.dv, "bf16", dq, dk, dv, dg, db, dh0, ws)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    g_full = gh[:, :, None].expand(-1, -1, case.dk).contiguous()
+    ref = bwd.backward(case.q, case.k, case.v, g_full, case.beta, case.initial_state, do, dhT,
+                       case.cu_host())
+    ref_dg = ref[3].sum(axis=2)
+    for name_, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"),
+                           (dq, dk, dv, dg, db, dh0),
+                           (ref[0], ref[1], ref[2], ref_dg, ref[4], ref[5])):
+        assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
