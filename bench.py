@@ -44,11 +44,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _SPLIT = "gated_delta_rule_124_b200/csrc/kda_chunk_split.cu"
 _CFG1 = "prefill: B=2 H=32 T=2048 d=128 C=64 bf16"
 _CFG2 = "long prefill: B=1 H=32 T=65536 d=128 C=64 bf16 slow decay"
+_DECODE = "gated_delta_rule_124_b200/csrc/kda_decode.cu"
+_DEC = "decode: N=256 H=32 d=128 bf16, fp32 state, 8 input sets cycled"
 MEASURED_TRAFFIC = {
     ("split_intra", _CFG1): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 222362880),
     ("split_chain", _CFG1): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 195830272),
     # captured on B=1 x T=16384 (a quarter of the tokens) and scaled by 4
     ("chunk_fwd_overlap", _CFG2): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 5597298688),
+    ("decode", _DEC): (_DECODE, "e97a0fa46338f7541982499a4e97d31ac9101889", 1027143936),
 }
 
 
