@@ -6,7 +6,8 @@ its ctypes binding and :mod:`.workloads` draws seeded synthetic inputs.
 from .kda import (  # noqa: F401
     EXPORTS, KDA_DTYPE_BF16, KDA_DTYPE_F32, KDA_NOALLOC_SCRATCH_BYTES, KDA_ERR_BAD_SEQLENS, KDA_ERR_CUDA,
     KDA_ERR_INVALID_ARG, KDA_ERR_TIMEOUT, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_OK,
-    KdaError, alloc_workspace, chunk_fwd, decode_step, kda_chunk_fwd,
+    KdaError, alloc_workspace, chunk_fwd, chunk_bwd, chunk_kda, ChunkKDA, decode_step,
+    kda_chunk_fwd,
     kda_chunk_fwd_workspace_size, kda_chunk_gate_cumsum, kda_chunk_inter, kda_chunk_intra,
     kda_chunk_output, kda_chunk_fwd_noalloc, kda_chunk_split_chain, kda_chunk_split_intra,
     kda_chunk_split_workspace_size, kda_chunk_fwd_plan, kda_qkv_conv_norm, kda_output_norm_gate, PLAN_NAMES,

@@ -369,6 +369,82 @@ def chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, chunk=64,
     return o, hN
 
 
+def chunk_bwd(q, k, v, g, beta, dout, initial_state=None, dfinal_state=None, cu_seqlens=None,
+              head_gate=False, workspace=None, stream=None):
+    """Gradients of sum(o * dout) + sum(final_state * dfinal_state) for
+    chunk_fwd's inputs: returns (dq, dk, dv, dg, dbeta, dinitial_state), fp32,
+    shaped like the inputs (dinitial_state [N, H, dk, dv]).  head_gate=True:
+    g and dg are [.., H] (Gated DeltaNet)."""
+    packed = q.dim() == 3
+    if packed:
+        total, H, dk = q.shape
+        B, T = 1, total
+        N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    else:
+        B, T, H, dk = q.shape
+        total, N = B * T, B
+        if cu_seqlens is not None:
+            raise ValueError("cu_seqlens needs packed [T_total, H, d] inputs")
+    dv = v.shape[-1]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(q.shape, **f32)
+    dk_ = torch.empty(k.shape, **f32)
+    dv_ = torch.empty(v.shape, **f32)
+    dg = torch.empty(g.shape, **f32)
+    db = torch.empty(beta.shape, **f32)
+    dh0 = torch.empty(N, H, dk, dv, **f32)
+    size = (kda_gdn_chunk_bwd_workspace_size if head_gate else kda_chunk_bwd_workspace_size)(
+        total, N, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(size, dtype=torch.uint8, device=q.device)
+    call = kda_gdn_chunk_bwd if head_gate else kda_chunk_bwd
+    call(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_seqlens, B, T, N, H, dk, dv,
+         q.dtype, dq, dk_, dv_, dg, db, dh0, workspace, stream=stream)
+    return dq, dk_, dv_, dg, db, dh0
+
+
+class ChunkKDA(torch.autograd.Function):
+    """Differentiable KDA prefill: forward = chunk_fwd, backward = chunk_bwd (which
+    recomputes the forward's per-chunk quantities, so only the inputs are
+    saved).  Gradients of q, k, v are returned in their dtype."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, beta, initial_state, cu_seqlens, head_gate):
+        if head_gate:
+            packed = q.dim() == 3
+            H, dk = q.shape[-2], q.shape[-1]
+            B, T = (1, q.shape[0]) if packed else (q.shape[0], q.shape[1])
+            total = B * T
+            N = (cu_seqlens.numel() - 1) if cu_seqlens is not None else B
+            dv = v.shape[-1]
+            o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+            hN = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+            ws = torch.empty(kda_gdn_chunk_fwd_workspace_size(total, N, H, dk, dv, 64, q.dtype),
+                             dtype=torch.uint8, device=q.device)
+            kda_gdn_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, N, H, dk, dv, 64,
+                              q.dtype, o, hN, ws)
+        else:
+            o, hN = chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens=cu_seqlens, chunk=64)
+        ctx.save_for_backward(q, k, v, g, beta, initial_state, cu_seqlens)
+        ctx.head_gate = head_gate
+        return o, hN
+
+    @staticmethod
+    def backward(ctx, do, dhN):
+        q, k, v, g, beta, h0, cu = ctx.saved_tensors
+        do = torch.zeros_like(v) if do is None else do.to(v.dtype).contiguous()
+        dhN = None if dhN is None else dhN.float().contiguous()
+        dq, dk, dv, dg, db, dh0 = chunk_bwd(q, k, v, g, beta, do, h0, dhN, cu,
+                                            head_gate=ctx.head_gate)
+        return (dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), dg, db,
+                dh0 if h0 is not None else None, None, None)
+
+
+def chunk_kda(q, k, v, g, beta, initial_state=None, cu_seqlens=None, head_gate=False):
+    """Differentiable prefill: (o, final_state); see ChunkKDA."""
+    return ChunkKDA.apply(q, k, v, g, beta, initial_state, cu_seqlens, head_gate)
+
+
 def decode_step(q, k, v, g, beta, state, o=None, stream=None):
     """One recurrent step.  q, k, g [N, H, dk]; v [N, H, dv]; beta [N, H];
     state [N, H, dk, dv] fp32, updated in place.  Returns o [N, H, dv]."""

@@ -158,3 +158,31 @@ def test_gdn_backward_head_gate(with_dhT):
                            (dq, dk, dv, dg, db, dh0),
                            (ref[0], ref[1], ref[2], ref_dg, ref[4], ref[5])):
         assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
+
+
+@pytest.mark.parametrize("head_gate", [False, True])
+def test_autograd_function_matches_oracle(head_gate):
+    """chunk_kda (forward + backward through autograd) against the oracle's
+    gradients: q, k, v gradients come back in bf16 (their inputs' dtype), the
+    rest in fp32."""
+    case = wl.make_prefill(510, [90, 40], H=2, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    gen = torch.Generator().manual_seed(17)
+    g_in = (-torch.nn.functional.softplus(torch.randn(case.total, case.H, generator=gen))
+            if head_gate else case.g)
+    do = torch.randn(case.total, case.H, case.dv, generator=gen).to(torch.bfloat16)
+    dhT = torch.randn(case.N, case.H, case.dk, case.dv, generator=gen)
+    leaves = [x.cuda().requires_grad_(True)
+              for x in (case.q, case.k, case.v, g_in, case.beta, case.initial_state)]
+    o, hN = kda.chunk_kda(*leaves, cu_seqlens=case.cu_seqlens.cuda(), head_gate=head_gate)
+    loss = (o.float() * do.cuda().float()).sum() + (hN * dhT.cuda()).sum()
+    loss.backward()
+    g_full = g_in[:, :, None].expand(-1, -1, case.dk).contiguous() if head_gate else g_in
+    ref = list(bwd.backward(case.q, case.k, case.v, g_full, case.beta, case.initial_state, do,
+                            dhT, case.cu_host()))
+    if head_gate:
+        ref[3] = ref[3].sum(axis=2)
+    tol = (1e-2, 1e-2, 1e-2, 1e-3, 1e-3, 1e-3)  # bf16-rounded q, k, v gradients
+    for name_, x, r, t in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), leaves, ref, tol):
+        assert x.grad is not None and x.grad.dtype == x.dtype, name_
+        assert rel_err(x.grad, r) <= t, (name_, rel_err(x.grad, r))
