@@ -186,3 +186,21 @@ def test_autograd_function_matches_oracle(head_gate):
     for name_, x, r, t in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), leaves, ref, tol):
         assert x.grad is not None and x.grad.dtype == x.dtype, name_
         assert rel_err(x.grad, r) <= t, (name_, rel_err(x.grad, r))
+
+
+def test_backward_no_tokens():
+    """No tokens at all: the state gradient passes through unchanged
+    (dS_0 = dS_T), for one sequence and for several empty ones."""
+    for N in (1, 3):
+        cu = torch.zeros(N + 1, dtype=torch.int32, device="cuda")
+        f32 = dict(dtype=torch.float32, device="cuda")
+        e = torch.zeros(64, **f32)  # token arrays: valid pointers, nothing read or written
+        dhT = torch.randn(N, 2, 32, 32, **f32)
+        dh0 = torch.full_like(dhT, float("nan"))
+        ws = torch.empty(max(kda.kda_chunk_bwd_workspace_size(0, N, 2, 32, 32), 256),
+                         dtype=torch.uint8, device="cuda")
+        kda.kda_chunk_bwd(e, e, e, e, e, None, e, dhT, cu, 1, 0, N, 2, 32, 32, "f32", e, e, e,
+                          e, e, dh0, ws)
+        torch.cuda.synchronize()
+        assert kda.kda_get_device_status(ws) == kda.KDA_OK
+        assert torch.equal(dh0, dhT)
