@@ -20,11 +20,12 @@
 //   dg is the reverse cumulative sum of dG inside the chunk          (b5 pairs)
 // The gradient of T = (I + A)^-1 never appears on its own: T^T dT T^T reduces
 // to Y U^T because the gradient reaching W is -dU S^T.  The forward half is
-// recomputed: b1 forms G, A, P, W and Ut of each chunk (the forward's a1 and
-// a2, with A and P from one pass over the token pairs) and the CUDA-core
-// prefill's a3 chain gives U and the entry state of every chunk.  Every
-// exponent is a difference exp(G_r - G_i) with i <= r, so never positive for
-// g <= 0; all arithmetic is fp32.
+// recomputed: b1 forms G, A, P, Kb, W and Ut of each chunk (the forward's a1
+// and a2, with A and P from one pass over the token pairs) and the forward
+// pass of the b2 chain kernel gives U and the entry state of every chunk.
+// Launches per call: chunk table, b1a/b1b/b1c, b2 forward and backward, b3,
+// b4, b5.  Every exponent is a difference exp(G_r - G_i) with i <= r, so
+// never positive for g <= 0; all arithmetic is fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
