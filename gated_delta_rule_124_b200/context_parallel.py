@@ -16,6 +16,14 @@ composition is associative.
 Cost: three prefills of the local segment per rank (two independent, one
 after the exchange) plus ``R`` small dk x dk products; the exchange carries
 ``2 x H x dk x max(dk, dv)`` floats per sequence and rank.
+
+The backward runs the same way in reverse.  The state gradient's recurrence
+does not involve the state, so over a segment ``dS_in = M^T dS_out + c`` with
+``c`` the entry-state gradient the segment's own outputs produce (the
+library's backward with a zero exit gradient); one exchange of ``(M, B, c)``
+gives every rank its entry state (forward fold) and its exit-state gradient
+(reverse fold), and a last backward of the segment with both gives its token
+gradients.
 """
 from __future__ import annotations
 
@@ -33,6 +41,15 @@ Prefill = Callable[..., tuple]
 def _library_prefill(q, k, v, g, beta, initial_state):
     return _kda.chunk_fwd(q, k, v, g, beta, initial_state=initial_state, chunk=64,
                           output_final_state=True)
+
+
+# backward(q, k, v, g, beta, initial_state, dout, dfinal_state) ->
+# (dq, dk, dv, dg, dbeta, dinitial_state); tensors [B, T, H, d] as above.
+Backward = Callable[..., tuple]
+
+
+def _library_backward(q, k, v, g, beta, initial_state, dout, dfinal_state):
+    return _kda.chunk_bwd(q, k, v, g, beta, dout, initial_state, dfinal_state)
 
 
 def segment_maps(q, k, v, g, beta, prefill: Prefill = _library_prefill):
@@ -80,3 +97,52 @@ def context_parallel_prefill(q, k, v, g, beta, initial_state=None, group=None,
     entries, final = entry_states(maps, initial_state)
     o, _ = prefill(q, k, v, g, beta, entries[rank].contiguous())
     return o, final
+
+
+def exit_gradients(maps: Sequence[tuple], offsets: Sequence, dfinal_state):
+    """Gradient of every segment's exit state and of the initial state:
+    dS_out of the last segment = dfinal_state, dS_out of segment r - 1 =
+    dS_in of segment r = M_r^T dS_out_r + c_r."""
+    g = dfinal_state
+    out = [None] * len(maps)
+    for r in range(len(maps) - 1, -1, -1):
+        out[r] = g
+        g = torch.matmul(maps[r][0].transpose(-1, -2), g) + offsets[r]
+    return out, g
+
+
+def context_parallel_backward(q, k, v, g, beta, dout, initial_state=None, dfinal_state=None,
+                              group=None, prefill: Prefill = _library_prefill,
+                              backward: Backward = _library_backward):
+    """Gradients for this rank's tokens of sum(o * dout) + sum(final_state *
+    dfinal_state) over the whole sequence, and of the initial state.
+
+    Arguments as in context_parallel_prefill, plus dout [B, T_r, H, dv] for this
+    rank's outputs and dfinal_state [B, H, dk, dv] (the same on every rank, or
+    None).  Returns (dq, dk, dv, dg, dbeta, dinitial_state); dinitial_state is
+    the whole sequence's and the same on every rank.  One all-gather."""
+    import torch.distributed as dist
+    B, _, H, dk = q.shape
+    dv = v.shape[-1]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    if initial_state is None:
+        initial_state = torch.zeros(B, H, dk, dv, **f32)
+    if dfinal_state is None:
+        dfinal_state = torch.zeros(B, H, dk, dv, **f32)
+    m, bm = segment_maps(q, k, v, g, beta, prefill)
+    c = backward(q, k, v, g, beta, None, dout, None)[5]
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    packed = torch.cat([m.reshape(B, H, -1), bm.reshape(B, H, -1),
+                        c.reshape(B, H, -1).to(torch.float32)], dim=-1).contiguous()
+    gathered = [torch.empty_like(packed) for _ in range(world)]
+    dist.all_gather(gathered, packed, group=group)
+    n1, n2 = dk * dk, dk * dk + dk * dv
+    maps = [(x[..., :n1].reshape(B, H, dk, dk), x[..., n1:n2].reshape(B, H, dk, dv))
+            for x in gathered]
+    offsets = [x[..., n2:].reshape(B, H, dk, dv) for x in gathered]
+    entries, _ = entry_states(maps, initial_state)
+    exits, dh0 = exit_gradients(maps, offsets, dfinal_state)
+    dq, dk_, dv_, dg, db, _ = backward(q, k, v, g, beta, entries[rank].contiguous(), dout,
+                                       exits[rank].contiguous())
+    return dq, dk_, dv_, dg, db, dh0

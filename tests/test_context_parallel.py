@@ -24,6 +24,19 @@ def _oracle_prefill(q, k, v, g, beta, initial_state):
     return torch.from_numpy(o).float(), torch.from_numpy(hN).float()
 
 
+def _oracle_backward(q, k, v, g, beta, initial_state, dout, dfinal_state):
+    """fp64 gradient oracle as the per-rank backward ([B, T, H, d] tensors)."""
+    from oracle import backward as obwd
+    B, T, H = q.shape[:3]
+    flat = lambda x: None if x is None else x.reshape(B * T, H, *x.shape[3:])  # noqa: E731
+    h0 = (torch.zeros(B, H, q.shape[-1], v.shape[-1]) if initial_state is None
+          else initial_state)
+    r = obwd.backward(flat(q), flat(k), flat(v), flat(g), flat(beta), h0, flat(dout),
+                      dfinal_state, np.arange(B + 1) * T)
+    shp = (q.shape, k.shape, v.shape, g.shape, beta.shape, h0.shape)
+    return tuple(torch.from_numpy(x).float().reshape(s) for x, s in zip(r, shp))
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -61,6 +74,43 @@ def test_two_ranks_gloo_match_the_whole_sequence():
     assert rel_err(o, ro) <= 1e-5
     for r in range(2):
         assert rel_err(out[r][1], rh) <= 1e-5
+
+
+def _bwd_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        c, q, k, v, g, beta, h0 = _case(T=48)
+        gen = torch.Generator().manual_seed(3)
+        do = torch.randn(q.shape[0], 48, q.shape[2], v.shape[-1], generator=gen)
+        dfin = torch.randn(h0.shape, generator=gen)
+        T = q.shape[1]
+        a, b = rank * T // world, (rank + 1) * T // world
+        grads = cp.context_parallel_backward(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b],
+                                             beta[:, a:b], do[:, a:b], h0, dfin,
+                                             prefill=_oracle_prefill, backward=_oracle_backward)
+        out[rank] = tuple(x.numpy() for x in grads)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_gloo_backward_matches_the_whole_sequence():
+    """Context-parallel backward over 2 gloo ranks (oracle as each rank's
+    prefill and backward) against the oracle's gradients of the whole
+    sequence."""
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_bwd_worker, args=(2, _free_port(), out), nprocs=2, join=True)
+    c, q, k, v, g, beta, h0 = _case(T=48)
+    gen = torch.Generator().manual_seed(3)
+    do = torch.randn(q.shape[0], 48, q.shape[2], v.shape[-1], generator=gen)
+    dfin = torch.randn(h0.shape, generator=gen)
+    ref = _oracle_backward(q, k, v, g, beta, h0, do, dfin)
+    for i, name in enumerate(("dq", "dk", "dv", "dg", "dbeta")):
+        x = np.concatenate([out[0][i], out[1][i]], axis=1)
+        assert rel_err(x, ref[i].numpy()) <= 1e-5, name
+    for r in range(2):
+        assert rel_err(out[r][5], ref[5].numpy()) <= 1e-5
 
 
 def test_fold_of_segment_maps_is_the_recurrence():
@@ -134,3 +184,40 @@ def test_chunked_prefill_then_decode_hands_the_state_over():
     assert rel_err(torch.cat(outs), ro[:T]) <= 2e-2
     assert rel_err(torch.stack(dec), ro[T:]) <= 2e-2
     assert rel_err(state[0], rh[0]) <= 2e-2
+
+
+@pytest.mark.gpu
+def test_simulated_ranks_backward_on_the_gpu():
+    """The context-parallel backward over three segments of two 600-token
+    sequences with the library's prefill and backward, against the oracle's
+    gradients of the whole sequences."""
+    c = wl.make_prefill(24, [600, 600], H=2, dk=64, dv=64, chunk=64, dtype="f32")
+    B, T, H, d = 2, 600, 2, 64
+    sh = lambda x, last: x.reshape(B, T, H, *last).cuda()  # noqa: E731
+    q, k, v, g = (sh(x, (d,)) for x in (c.q, c.k, c.v, c.g))
+    beta, h0 = sh(c.beta, ()), c.initial_state.cuda()
+    gen = torch.Generator().manual_seed(4)
+    do = torch.randn(B, T, H, d, generator=gen)
+    dfin = torch.randn(B, H, d, d, generator=gen)
+    cuts = [0, 200, 450, 600]
+    segs = list(zip(cuts, cuts[1:]))
+    part = lambda x, a, b: x[:, a:b].contiguous()  # noqa: E731
+    maps, offs = [], []
+    for a, b in segs:
+        args = [part(x, a, b) for x in (q, k, v, g, beta)]
+        maps.append(cp.segment_maps(*args))
+        offs.append(cp._library_backward(*args, None, part(do.cuda(), a, b), None)[5])
+    entries, _ = cp.entry_states(maps, h0)
+    exits, dh0 = cp.exit_gradients(maps, offs, dfin.cuda())
+    grads = []
+    for (a, b), s_in, d_out in zip(segs, entries, exits):
+        args = [part(x, a, b) for x in (q, k, v, g, beta)]
+        grads.append(cp._library_backward(*args, s_in.contiguous(), part(do.cuda(), a, b),
+                                          d_out.contiguous()))
+    ref = _oracle_backward(c.q.reshape(B, T, H, d), c.k.reshape(B, T, H, d),
+                           c.v.reshape(B, T, H, d), c.g.reshape(B, T, H, d),
+                           c.beta.reshape(B, T, H), c.initial_state, do, dfin)
+    for i, name in enumerate(("dq", "dk", "dv", "dg", "dbeta")):
+        x = torch.cat([gr[i] for gr in grads], dim=1)
+        assert rel_err(x, ref[i].numpy()) <= 1e-3, name
+    assert rel_err(dh0, ref[5].numpy()) <= 1e-3
