@@ -10,7 +10,8 @@ from .kda import (  # noqa: F401
     kda_chunk_fwd,
     kda_chunk_fwd_workspace_size, kda_chunk_gate_cumsum, kda_chunk_inter, kda_chunk_intra,
     kda_chunk_output, kda_chunk_fwd_noalloc, kda_chunk_split_chain, kda_chunk_split_intra,
-    kda_chunk_split_workspace_size, kda_chunk_fwd_plan, kda_qkv_conv_norm, kda_output_norm_gate, PLAN_NAMES,
+    kda_chunk_split_workspace_size, kda_chunk_fwd_plan, kda_qkv_conv_norm, kda_qkv_conv_norm_step, kda_output_norm_gate,
+    PLAN_NAMES,
     kda_gdn_chunk_fwd, kda_gdn_chunk_fwd_workspace_size, kda_gdn_decode_step,
     kda_chunk_bwd, kda_chunk_bwd_workspace_size, kda_gdn_chunk_bwd,
     kda_gdn_chunk_bwd_workspace_size, KDA_PLAN_SIMT, KDA_PLAN_FUSED,

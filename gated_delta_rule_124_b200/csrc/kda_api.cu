@@ -551,6 +551,28 @@ kda_status_t kda_qkv_conv_norm(const void* xq, const void* xk, const void* xv, c
                                           static_cast<cudaStream_t>(stream)));
 }
 
+kda_status_t kda_qkv_conv_norm_step(const void* xq, const void* xk, const void* xv,
+                                    const float* wq, const float* wk, const float* wv,
+                                    void* conv_q, void* conv_k, void* conv_v, int N, int H,
+                                    int dk, int dv, kda_dtype_t dtype, float eps, void* q,
+                                    void* k, void* v, void* stream) {
+    if (N < 0 || H < 1 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!(eps > 0.f) || !(eps < 1e30f)) return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    for (const void* ptr : std::initializer_list<const void*>{
+             xq, xk, xv, (const void*)wq, (const void*)wk, (const void*)wv, conv_q, conv_k,
+             conv_v, q, k, v})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    const void* const x[3] = {xq, xk, xv};
+    const float* const w[3] = {wq, wk, wv};
+    void* const state[3] = {conv_q, conv_k, conv_v};
+    void* const y[3] = {q, k, v};
+    return from_cuda(kda::launch_qkv_conv_step(x, w, state, y, dk, dv, N, H, eps, dtype,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* w,
                                   int total_tokens, int H, int dv, kda_dtype_t dtype, float eps,
                                   void* y, void* stream) {

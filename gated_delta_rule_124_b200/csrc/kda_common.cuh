@@ -131,6 +131,9 @@ cudaError_t launch_output(const void* q, const void* k, const float* G, const fl
 cudaError_t launch_qkv_conv(const void* const x[3], const float* const w[3], void* const y[3],
                             int dk, int dv, const int32_t* cu, int N, int T, int total, int H,
                             float eps, kda_dtype_t dt, cudaStream_t st);
+cudaError_t launch_qkv_conv_step(const void* const x[3], const float* const w[3],
+                                 void* const state[3], void* const y[3], int dk, int dv, int N,
+                                 int H, float eps, kda_dtype_t dt, cudaStream_t st);
 cudaError_t launch_norm_gate(const void* o, const void* gate, const float* w, int total, int H,
                              int d, float eps, kda_dtype_t dt, void* y, cudaStream_t st);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,

@@ -177,6 +177,76 @@ __device__ __forceinline__ void conv_run(const TIn* __restrict__ x, const float*
     }
 }
 
+// One decode token per (tensor, sequence, head), one warp: the filter's first
+// three taps read the sequence's last three inputs from its convolution state
+// [N, 3, H, D] (oldest first), the fourth the new input; the state then drops
+// its oldest row and appends the input.
+template <int CPL, typename TIn>
+__device__ __forceinline__ void conv_step(const TIn* __restrict__ x, const float* __restrict__ w,
+                                          TIn* __restrict__ state, TIn* __restrict__ y, int H,
+                                          int n, int h, bool l2, float eps) {
+    constexpr int D = 32 * CPL;
+    const int lane = threadIdx.x & 31, c0 = lane * CPL;
+    float wt[CPL][4];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(w + ((size_t)h * D + c0 + j) * 4);
+        wt[j][0] = v.x; wt[j][1] = v.y; wt[j][2] = v.z; wt[j][3] = v.w;
+    }
+    float win[3][CPL], cur[CPL];
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+        Vec<CPL, TIn>::load(state + (((size_t)n * 3 + i) * H + h) * D + c0, win[i]);
+    Vec<CPL, TIn>::load(x + ((size_t)n * H + h) * D + c0, cur);
+    float out[CPL], ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        float acc = wt[j][3] * cur[j];
+        acc = fmaf(wt[j][2], win[2][j], acc);
+        acc = fmaf(wt[j][1], win[1][j], acc);
+        acc = fmaf(wt[j][0], win[0][j], acc);
+        out[j] = __fdividef(acc, 1.f + __expf(-acc));
+        ss = fmaf(out[j], out[j], ss);
+    }
+    Vec<CPL, TIn>::store(state + (((size_t)n * 3 + 0) * H + h) * D + c0, win[1]);
+    Vec<CPL, TIn>::store(state + (((size_t)n * 3 + 1) * H + h) * D + c0, win[2]);
+    Vec<CPL, TIn>::store(state + (((size_t)n * 3 + 2) * H + h) * D + c0, cur);
+    if (l2) {
+        const float inv = rsqrtf(warp_sum(ss) + eps);
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) out[j] *= inv;
+    }
+    Vec<CPL, TIn>::store(y + ((size_t)n * H + h) * D + c0, out);
+}
+
+struct StepArgs {
+    const void* x[3];
+    const float* w[3];
+    void* state[3];
+    void* y[3];
+    int d[3];
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(32 * kWarps) conv_step_kernel(const StepArgs a, int N, int H,
+                                                                float eps) {
+    const int tensor = blockIdx.y;  // 0 q, 1 k, 2 v
+    const long long task = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (task >= (long long)N * H) return;
+    const int h = static_cast<int>(task % H), n = static_cast<int>(task / H);
+    const TIn* x = static_cast<const TIn*>(tensor == 0 ? a.x[0] : tensor == 1 ? a.x[1] : a.x[2]);
+    TIn* y = static_cast<TIn*>(tensor == 0 ? a.y[0] : tensor == 1 ? a.y[1] : a.y[2]);
+    TIn* st = static_cast<TIn*>(tensor == 0 ? a.state[0] : tensor == 1 ? a.state[1] : a.state[2]);
+    const float* w = tensor == 0 ? a.w[0] : tensor == 1 ? a.w[1] : a.w[2];
+    const int d = tensor == 0 ? a.d[0] : tensor == 1 ? a.d[1] : a.d[2];
+    const bool l2 = tensor < 2;
+    switch (d) {
+        case 128: conv_step<4, TIn>(x, w, st, y, H, n, h, l2, eps); break;
+        case 64: conv_step<2, TIn>(x, w, st, y, H, n, h, l2, eps); break;
+        default: conv_step<1, TIn>(x, w, st, y, H, n, h, l2, eps); break;
+    }
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(32 * kWarps) conv_swish_kernel(
     const ConvArgs a, const int32_t* __restrict__ cu, int N, int T, int total, int H, float eps) {
@@ -291,6 +361,26 @@ cudaError_t launch_qkv_conv(const void* const x[3], const float* const w[3], voi
         conv_swish_kernel<__nv_bfloat16><<<grid, 32 * kWarps, 0, st>>>(a, cu, N, T, total, H, eps);
     else
         conv_swish_kernel<float><<<grid, 32 * kWarps, 0, st>>>(a, cu, N, T, total, H, eps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qkv_conv_step(const void* const x[3], const float* const w[3],
+                                 void* const state[3], void* const y[3], int dk, int dv, int N,
+                                 int H, float eps, kda_dtype_t dt, cudaStream_t st) {
+    if ((long long)N * H == 0) return cudaSuccess;
+    StepArgs a;
+    for (int i = 0; i < 3; ++i) {
+        a.x[i] = x[i];
+        a.w[i] = w[i];
+        a.state[i] = state[i];
+        a.y[i] = y[i];
+        a.d[i] = i < 2 ? dk : dv;
+    }
+    const dim3 grid(static_cast<unsigned>(((long long)N * H + kWarps - 1) / kWarps), 3);
+    if (dt == KDA_DTYPE_BF16)
+        conv_step_kernel<__nv_bfloat16><<<grid, 32 * kWarps, 0, st>>>(a, N, H, eps);
+    else
+        conv_step_kernel<float><<<grid, 32 * kWarps, 0, st>>>(a, N, H, eps);
     return cudaGetLastError();
 }
 

@@ -42,7 +42,7 @@ EXPORTS = (
     "kda_chunk_split_chain", "kda_chunk_fwd_plan", "kda_qkv_conv_norm",
     "kda_output_norm_gate", "kda_gdn_chunk_fwd_workspace_size", "kda_gdn_chunk_fwd",
     "kda_gdn_decode_step", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
-    "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd",
+    "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd", "kda_qkv_conv_norm_step",
 )
 
 
@@ -79,6 +79,7 @@ _SIGS = {
     "kda_chunk_bwd": ([_vp] * 9 + [_i] * 7 + [_vp] * 7 + [_sz, _vp], _i),
     "kda_gdn_chunk_bwd_workspace_size": ([_i] * 5, _sz),
     "kda_gdn_chunk_bwd": ([_vp] * 9 + [_i] * 7 + [_vp] * 7 + [_sz, _vp], _i),
+    "kda_qkv_conv_norm_step": ([_vp] * 9 + [_i] * 5 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
@@ -292,6 +293,15 @@ def kda_gdn_chunk_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_se
                                   _p(dg), _p(dbeta), _p(dinitial_state), _p(workspace), wb,
                                   _stream(stream))
     return _ret(st, "kda_gdn_chunk_bwd", check)
+
+
+def kda_qkv_conv_norm_step(xq, xk, xv, wq, wk, wv, conv_q, conv_k, conv_v, N, H, dk, dv,
+                           dtype, eps, q, k, v, stream=None, check=True) -> int:
+    st = load().kda_qkv_conv_norm_step(_p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
+                                       _p(conv_q), _p(conv_k), _p(conv_v), N, H, dk, dv,
+                                       dtype_code(dtype), eps, _p(q), _p(k), _p(v),
+                                       _stream(stream))
+    return _ret(st, "kda_qkv_conv_norm_step", check)
 
 
 def kda_qkv_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens, B, T, num_seqs, H, dk, dv, dtype,

@@ -353,6 +353,23 @@ kda_status_t kda_qkv_conv_norm(const void* xq, const void* xk, const void* xv, c
                                kda_dtype_t dtype, float eps, void* q, void* k, void* v,
                                void* stream);
 
+/* kda_qkv_conv_norm_step: the same for one decode token per sequence, with a
+ * convolution state per tensor: conv_q, conv_k [N, 3, H, dk] and conv_v
+ * [N, 3, H, dv] (dtype) hold each sequence's last three inputs, oldest first
+ * (zeros: no history, as at the start of a prefill).  y = Swish(w0 c0 + w1 c1
+ * + w2 c2 + w3 x), q and k L2-normalised; then each state drops its oldest
+ * row and appends x (in place).  A prefill hands over by copying the last
+ * three input rows of each sequence (zero rows before its start).
+ * In:  xq, xk [N, H, dk], xv [N, H, dv] (dtype); weights as above; eps > 0.
+ * Out: q, k [N, H, dk], v [N, H, dv] (dtype), not aliasing the inputs or the
+ *      states.  Shapes: dk, dv in {32, 64, 128}; N == 0 does nothing.
+ */
+kda_status_t kda_qkv_conv_norm_step(const void* xq, const void* xk, const void* xv,
+                                    const float* wq, const float* wk, const float* wv,
+                                    void* conv_q, void* conv_k, void* conv_v, int N, int H,
+                                    int dk, int dv, kda_dtype_t dtype, float eps, void* q,
+                                    void* k, void* v, void* stream);
+
 /* kda_output_norm_gate: y[t, h, :] = o[t, h, :] / sqrt(mean_j o[t, h, j]^2 +
  * eps) * w * sigmoid(gate[t, h, :]).
  * In:  o, gate [total_tokens, H, dv] (dtype); w [dv] fp32 (shared by the

@@ -221,3 +221,15 @@ def test_gdn_backward_call_rejects_bad_arguments(lib):
     assert kda.kda_gdn_chunk_bwd(**{**a, "dv": 40}) == kda.KDA_ERR_UNSUPPORTED
     assert kda.kda_gdn_chunk_bwd(**{**a, "num_seqs": 2}) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_gdn_chunk_bwd(**a) == kda.KDA_ERR_WORKSPACE
+
+
+def test_conv_step_rejects_bad_arguments(lib):
+    a = dict(xq=FAKE, xk=FAKE, xv=FAKE, wq=FAKE, wk=FAKE, wv=FAKE, conv_q=FAKE, conv_k=FAKE,
+             conv_v=FAKE, N=4, H=2, dk=128, dv=128, dtype="bf16", eps=1e-6, q=FAKE, k=FAKE,
+             v=FAKE, stream=0, check=False)
+    assert kda.kda_qkv_conv_norm_step(**{**a, "conv_k": None}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm_step(**{**a, "xv": FAKE + 2}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm_step(**{**a, "dk": 96}) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_qkv_conv_norm_step(**{**a, "eps": 0.0}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm_step(**{**a, "N": -1}) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_qkv_conv_norm_step(**{**a, "N": 0}) == kda.KDA_OK

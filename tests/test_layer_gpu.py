@@ -107,3 +107,39 @@ def test_layer_steps_around_the_operator():
                            torch.zeros(1, H, d, d), None)
     ry = layer.output_norm_gate(ro, gate, wn, eps=EPS)
     assert rel_err(y, ry) <= 2e-2
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32)])
+def test_conv_step_continues_a_prefill(dtype, dk, dv):
+    """Decode-time convolution: a prefill over the first 5 tokens of each of 3
+    sequences, the state taken from their last three input rows, then two
+    steps; and steps from a zero state from the first token.  Both against the
+    prefill convolution of all 7 tokens and the oracle."""
+    B, T, H, T0 = 3, 7, 2, 5
+    x, w = _inputs(31, B * T, H, dk, dv, dtype)
+    full = _run_conv(x, w, None, B, T, B, H, dk, dv, dtype)
+    ref = layer.qkv_conv_norm(*x, *w, cu_seqlens=np.arange(B + 1) * T, eps=EPS)
+    wd = [t.cuda() for t in w]
+    xs = [t.cuda().reshape(B, T, H, -1) for t in x]
+    for start in (0, T0):
+        # state: the last three inputs before `start` (zeros before the sequence)
+        st = []
+        for xt in xs:
+            s = torch.zeros(B, 3, H, xt.shape[-1], dtype=xt.dtype, device="cuda")
+            for i in range(3):
+                t = start - 3 + i
+                if t >= 0:
+                    s[:, i] = xt[:, t]
+            st.append(s)
+        for t in range(start, T):
+            xt = [a[:, t].contiguous() for a in xs]
+            out = [torch.full_like(a, float("nan")) for a in xt]
+            kda.kda_qkv_conv_norm_step(*xt, *wd, *st, B, H, dk, dv, dtype, EPS, *out)
+            torch.cuda.synchronize()
+            for j in range(3):
+                f = full[j].reshape(B, T, H, -1)[:, t]
+                r = ref[j].reshape(B, T, H, -1)[:, t]
+                assert rel_err(out[j], r) <= TOL[dtype], (start, t, j)
+                same = 1e-6 if dtype == "f32" else TOL[dtype]  # bf16: one rounding apart
+                assert rel_err(out[j], f.float().cpu().numpy()) <= same, (start, t, j)
