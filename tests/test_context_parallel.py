@@ -221,3 +221,31 @@ def test_simulated_ranks_backward_on_the_gpu():
         x = torch.cat([gr[i] for gr in grads], dim=1)
         assert rel_err(x, ref[i].numpy()) <= 1e-3, name
     assert rel_err(dh0, ref[5].numpy()) <= 1e-3
+
+
+def test_reverse_fold_gives_the_boundary_state_gradients():
+    """exit_gradients over oracle maps and oracle state-gradient offsets
+    reproduces the gradient of the state at every segment boundary (the
+    oracle's initial-state gradient of the suffix after that boundary) and of
+    the initial state (pure host arithmetic)."""
+    c, q, k, v, g, beta, h0 = _case(T=50)
+    gen = torch.Generator().manual_seed(8)
+    do = torch.randn(q.shape[0], 50, q.shape[2], v.shape[-1], generator=gen)
+    dfin = torch.randn(h0.shape, generator=gen)
+    cuts = [0, 11, 30, 50]
+    segs = list(zip(cuts, cuts[1:]))
+    part = lambda x, a, b: x[:, a:b]  # noqa: E731
+    maps = [cp.segment_maps(*(part(x, a, b) for x in (q, k, v, g, beta)), _oracle_prefill)
+            for a, b in segs]
+    offs = [_oracle_backward(*(part(x, a, b) for x in (q, k, v, g, beta)), None,
+                             part(do, a, b), None)[5] for a, b in segs]
+    exits, dh0 = cp.exit_gradients(maps, offs, dfin)
+    entries, _ = cp.entry_states(maps, h0)
+    for i, (a, b) in enumerate(segs):
+        if b == 50:
+            ref = dfin.numpy()
+        else:
+            ref = _oracle_backward(*(part(x, b, 50) for x in (q, k, v, g, beta)),
+                                   entries[i + 1], part(do, b, 50), dfin)[5].numpy()
+        assert rel_err(exits[i], ref) <= 1e-5, i
+    assert rel_err(dh0, _oracle_backward(q, k, v, g, beta, h0, do, dfin)[5].numpy()) <= 1e-5
