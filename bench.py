@@ -279,8 +279,7 @@ def run_ours(args, rank, world, local_rank):
         try:
             bwd = backward_times(
                 kda, torch, P, pc, dev, stream, reps=max(3, min(20, args.steps)),
-                sm_max_mhz=clk.get("sm_max_mhz") if isinstance(clk, dict) else None,
-                oracle_sample=(rank == 0 and world == 1 and not args.no_cpu_baseline))
+                sm_max_mhz=clk.get("sm_max_mhz") if isinstance(clk, dict) else None)
         except (kda.KdaError, RuntimeError, AssertionError) as e:
             bwd = {"error": f"{type(e).__name__}: {e}"}
 
@@ -328,6 +327,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(pc, seconds=args.cpu_seconds)
+        if isinstance(bwd, dict) and "error" not in bwd:
+            bwd["cpu_oracle"] = cpu_baseline_backward(pc)
     return res
 
 
@@ -483,7 +484,7 @@ def backward_flops(head_tokens, dk, dv, C=64):
     return 2 * fma * head_tokens / C
 
 
-def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None, oracle_sample=True):
+def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
     """kda_chunk_bwd on the prefill workload (fp32 gradients of o and the final
     state), timed with CUDA events on the launching stream, L2 flushed before
     each call.  Bound by fp32 arithmetic on the CUDA cores: the roofline peak
@@ -523,21 +524,6 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None, ora
                         "peak_kind": f"fp32 CUDA cores, 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",
                         "algorithmic_flops_per_call": fl},
            "workspace_bytes": int(ws.numel())}
-    if oracle_sample:
-        from oracle import backward as obwd
-        Ts = min(256, int(pc.cu_host()[1]))
-        hd = lambda x: x[:Ts, :1]
-        g0 = torch.Generator().manual_seed(9)
-        do0 = torch.randn(Ts, 1, dv, generator=g0).to(torch.bfloat16)
-        h0 = pc.initial_state[:1, :1] if pc.initial_state is not None else torch.zeros(1, 1, dk, dv)
-        t0 = time.perf_counter()
-        obwd.backward(hd(pc.q), hd(pc.k), hd(pc.v), hd(pc.g), pc.beta[:Ts, :1], h0, do0, None,
-                      [0, Ts])
-        el = time.perf_counter() - t0
-        res["cpu_oracle"] = {"value": Ts / el / H, "unit": "tokens/s", "cores": 1,
-                             "kind": "oracle",
-                             "sample": f"1 sequence x {Ts} tokens x 1 of {H} heads, fp64 token "
-                                       f"recurrence differentiated by autograd, {el:.2f} s"}
     return res
 
 
@@ -656,6 +642,29 @@ def cpu_baseline(pc, seconds=15.0, heads=None):
                                         f"1 thread, {el1:.2f} s"}}
 
 
+def cpu_baseline_backward(pc, tokens=256):
+    """The gradient oracle (fp64 token recurrence differentiated by autograd, as
+    it stands) on a bounded sample of the prefill workload: the first `tokens`
+    tokens of the first sequence, one head, one thread.  Reported as tokens/s of
+    the full workload (head-tokens/s / H), beside the backward's GPU time."""
+    import torch
+
+    from oracle import backward as obwd
+    H, dk, dv = pc.H, pc.dk, pc.dv
+    Ts = min(tokens, int(pc.cu_host()[1]))
+    hd = lambda x: x[:Ts, :1]  # noqa: E731
+    g0 = torch.Generator().manual_seed(9)
+    do0 = torch.randn(Ts, 1, dv, generator=g0).to(torch.bfloat16)
+    h0 = pc.initial_state[:1, :1] if pc.initial_state is not None else torch.zeros(1, 1, dk, dv)
+    t0 = time.perf_counter()
+    obwd.backward(hd(pc.q), hd(pc.k), hd(pc.v), hd(pc.g), pc.beta[:Ts, :1], h0, do0, None,
+                  [0, Ts])
+    el = time.perf_counter() - t0
+    return {"value": Ts / el / H, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"1 sequence x {Ts} tokens x 1 of {H} heads, fp64 token recurrence "
+                      f"differentiated by autograd, {el:.2f} s"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -694,8 +703,9 @@ def run_backward_only(args):
     pc = prefill_case(wl, args)
     P = pc.to(dev)
     bwd = backward_times(kda, torch, P, pc, dev, torch.cuda.current_stream(),
-                         reps=max(3, min(20, args.steps)),
-                         oracle_sample=not args.no_cpu_baseline)
+                         reps=max(3, min(20, args.steps)))
+    if not args.no_cpu_baseline:
+        bwd["cpu_oracle"] = cpu_baseline_backward(pc)
     return {"backward": bwd, "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": pc.H,
                                         "dk": pc.dk, "dv": pc.dv}}
 
