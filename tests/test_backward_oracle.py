@@ -96,3 +96,25 @@ def test_recurrent_backward_matches_the_oracle(seed):
     order = [0, 1, 2, 3, 4, 5]  # q k v g beta h0 vs dq dk dv dg db dh0
     for i, j in zip(order, [0, 1, 2, 3, 4, 5]):
         np.testing.assert_allclose(got[j], ref[i], rtol=1e-10, atol=1e-12)
+
+
+def test_head_gate_gradient_is_the_channel_sum():
+    """Gated DeltaNet: with the gate spread over the channels, the gradient of
+    the per-(token, head) gate is the sum of the per-channel gradients --
+    checked against central finite differences of the C forward oracle in the
+    head gate itself."""
+    args, cu, do, dhT = _problem(9, lens=(6, 4), H=2, dk=5, dv=3)
+    r = np.random.default_rng(10)
+    T, H, dk = args[3].shape
+    gh = -np.log1p(np.exp(r.normal(size=(T, H))))
+    spread = lambda x: np.repeat(x[:, :, None], dk, axis=2)  # noqa: E731
+    args[3] = spread(gh)
+    dg_head = bwd.backward(*args, do, dhT, cu)[3].sum(axis=2)
+    eps = 1e-6
+    for _ in range(3):
+        d = r.normal(size=gh.shape)
+        plus, minus = list(args), list(args)
+        plus[3], minus[3] = spread(gh + eps * d), spread(gh - eps * d)
+        fd = (_loss(plus, cu, do, dhT) - _loss(minus, cu, do, dhT)) / (2 * eps)
+        an = float((dg_head * d).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (fd, an)
