@@ -11,10 +11,10 @@ from .kda import (  # noqa: F401
     kda_chunk_fwd_workspace_size, kda_chunk_gate_cumsum, kda_chunk_inter, kda_chunk_intra,
     kda_chunk_output, kda_chunk_fwd_noalloc, kda_chunk_split_chain, kda_chunk_split_intra,
     kda_chunk_split_workspace_size, kda_chunk_fwd_plan, kda_qkv_conv_norm, kda_qkv_conv_norm_step, kda_output_norm_gate,
-    PLAN_NAMES,
+    PLAN_NAMES, PLAN_CODES, plan_code, kda_chunk_fwd_with_plan, kda_chunk_fwd_plan_workspace_size,
     kda_gdn_chunk_fwd, kda_gdn_chunk_fwd_workspace_size, kda_gdn_decode_step,
     kda_chunk_bwd, kda_chunk_bwd_workspace_size, kda_gdn_chunk_bwd,
-    kda_gdn_chunk_bwd_workspace_size, KDA_PLAN_SIMT, KDA_PLAN_FUSED,
+    kda_gdn_chunk_bwd_workspace_size, KDA_PLAN_SIMT,
     KDA_PLAN_SPLIT, KDA_PLAN_OVERLAP, kda_decode_step, kda_get_device_status, kda_num_chunks_upper_bound,
     load, status_string,
 )

@@ -22,13 +22,12 @@ bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
 bool dtype_ok(kda_dtype_t t) { return t == KDA_DTYPE_F32 || t == KDA_DTYPE_BF16; }
 
-// Shapes and sequence description shared by every prefill entry point.
-struct Prefill {
-    int total, N;
-};
+}  // namespace
+
+namespace kda {
 
 kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, int H, int dk,
-                                  int dv, int chunk, kda_dtype_t dt, Prefill* out) {
+                                 int dv, int chunk, kda_dtype_t dt, Prefill* out) {
     if (B < 1 || T < 0 || num_seqs < 1 || H < 1) return KDA_ERR_INVALID_ARG;
     if (!dtype_ok(dt)) return KDA_ERR_INVALID_ARG;
     if (cu) {
@@ -46,8 +45,49 @@ kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, 
     return KDA_OK;
 }
 
-// Which kernels kda_chunk_fwd runs.
-enum class Path { Simt, Fused, Split, Overlap };
+kda_status_t begin_prefill(const Workspace& w, const int32_t* cu, int B, int T, int N, int chunk,
+                           int maxc, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    e = launch_build_chunk_table(cu, B, T, N, chunk, maxc, w.status, w.chunk_start,
+                                 w.chunk_info, st);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status_t run_simt(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                      int B, int T, const Prefill& p, int H, int dk, int dv, int chunk,
+                      kda_dtype_t dtype, void* o, float* final_state, const Workspace& w,
+                      int maxc, cudaStream_t st) {
+    cudaError_t e = launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
+    if (e == cudaSuccess)
+        e = launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, chunk, dtype, w.status,
+                         w.W, w.U, st);
+    if (e == cudaSuccess)
+        e = launch_inter(k, w.G, w.W, w.U, initial_state, cu_seqlens, B, T, p.N, w.chunk_start,
+                         H, dk, dv, chunk, dtype, w.status, w.states, final_state, st);
+    if (e == cudaSuccess)
+        e = launch_output(q, k, w.G, w.U, w.states, w.chunk_info, maxc, H, dk, dv, chunk, dtype,
+                          w.status, o, st);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace kda
+
+namespace {
+
+using kda::Prefill;
+using kda::begin_prefill;
+using kda::check_prefill_shape;
+using kda::run_simt;
+
+// Which kernels kda_chunk_fwd runs (the values of the KDA_PLAN_* constants).
+enum class Path { Simt = KDA_PLAN_SIMT, Split = KDA_PLAN_SPLIT, Overlap = KDA_PLAN_OVERLAP };
+
+bool tc_shape(int dk, int dv, int chunk, kda_dtype_t dt) {
+    return dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
+           kda::tc_path_available();
+}
 
 // Whether co-scheduling the two split kernels pays: the chains get one SM per
 // unit (2 N H SMs) and the intra-chunk items the rest, against the two kernels
@@ -63,29 +103,39 @@ bool overlap_pays(long long items, long long rounds, long long NH, int sms) {
     return (intra_ov > chain ? intra_ov : chain) <= 0.85 * (intra_split + chain);
 }
 
-// bf16, dk = dv = 128, chunk 64 runs on the tensor cores as the split plan:
-// the chunk-parallel intra-chunk kernel and the per-chain kernel, co-scheduled
-// in one launch on disjoint SMs where overlap_pays(), else as two launches.
-// The single fused kernel (one CTA per (sequence, head)) is slower on every
-// measured shape and runs only when forced.  KDA_CHUNK_PATH = fused | split |
-// overlap | simt forces a plan (testing); overlap falls back to split where
-// the launch does not apply.
+// Whether `path` can run a problem of these shapes on the current device.
+bool path_applies(Path path, int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
+    switch (path) {
+        case Path::Simt: return true;
+        case Path::Split: return tc_shape(dk, dv, chunk, dt);
+        case Path::Overlap: return tc_shape(dk, dv, chunk, dt) && kda::overlap_grid(N, H) > 0;
+    }
+    return false;
+}
+
+// The default plan, a function of the arguments and the device only: bf16,
+// dk = dv = 128, chunk 64 runs on the tensor cores as the split plan -- the
+// chunk-parallel intra-chunk kernel and the per-chain kernel -- co-scheduled
+// in one launch on disjoint SMs where overlap_pays(), else as two launches;
+// every other supported shape runs the CUDA-core plan.
 Path select_path(int total, int N, bool packed, int H, int dk, int dv, int chunk,
                  kda_dtype_t dt) {
-    const bool tc_shape = dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
-                          kda::tc_path_available();
-    const char* env = getenv("KDA_CHUNK_PATH");
-    if (env && !strcmp(env, "simt")) return Path::Simt;
-    if (!tc_shape) return Path::Simt;
-    if (env && !strcmp(env, "fused")) return Path::Fused;
-    if (env && !strcmp(env, "split")) return Path::Split;
+    if (!tc_shape(dk, dv, chunk, dt)) return Path::Simt;
     const int sms = kda::overlap_grid(N, H);
     if (sms == 0) return Path::Split;
-    if (env && !strcmp(env, "overlap")) return Path::Overlap;
     if (packed && N > 1) return Path::Split;
     const long long rounds = ((long long)total / N + chunk - 1) / chunk;
     const long long items = rounds * N * H;
     return overlap_pays(items, rounds, (long long)N * H, sms) ? Path::Overlap : Path::Split;
+}
+
+bool plan_from_int(int plan, Path* out) {
+    switch (plan) {
+        case KDA_PLAN_SIMT: *out = Path::Simt; return true;
+        case KDA_PLAN_SPLIT: *out = Path::Split; return true;
+        case KDA_PLAN_OVERLAP: *out = Path::Overlap; return true;
+    }
+    return false;
 }
 
 Workspace carve_for(void* base, const Prefill& p, int H, int dk, int dv, int chunk, Path path) {
@@ -94,12 +144,9 @@ Workspace carve_for(void* base, const Prefill& p, int H, int dk, int dv, int chu
                                                                      : 0);
 }
 
-size_t workspace_bytes_for(int total, int N, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
-    // the split and co-scheduled plans share one layout, so packing does not matter
+size_t workspace_bytes_for(int total, int N, int H, int dk, int dv, int chunk, Path path) {
     const Prefill p{total, N};
-    return carve_for(nullptr, p, H, dk, dv, chunk,
-                     select_path(total, N, false, H, dk, dv, chunk, dt))
-        .total_bytes;
+    return carve_for(nullptr, p, H, dk, dv, chunk, path).total_bytes;
 }
 
 kda_status_t check_ws(void* ws, size_t bytes, const Prefill& p, int H, int dk, int dv,
@@ -112,47 +159,25 @@ kda_status_t check_ws(void* ws, size_t bytes, const Prefill& p, int H, int dk, i
     return KDA_OK;
 }
 
+// The step calls keep only the status word and the chunk table in the
+// workspace (their intermediates are the caller's buffers).
+kda_status_t check_ws_header(void* ws, size_t bytes, const Prefill& p, int H, int dk, int dv,
+                             int chunk, Workspace* out) {
+    if (!ws) return KDA_ERR_WORKSPACE;
+    if (!aligned256(ws)) return KDA_ERR_INVALID_ARG;
+    Workspace w = kda::carve(ws, p.total, p.N, H, dk, dv, chunk, false);
+    if (bytes < w.total_bytes) return KDA_ERR_WORKSPACE;
+    *out = w;
+    return KDA_OK;
+}
+
 kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
-
-// Reset the status word and build the chunk table (two stream operations).
-kda_status_t begin_prefill(const Workspace& w, const int32_t* cu, int B, int T, int N, int chunk,
-                           int maxc, cudaStream_t st) {
-    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
-    if (e != cudaSuccess) return KDA_ERR_CUDA;
-    e = kda::launch_build_chunk_table(cu, B, T, N, chunk, maxc, w.status, w.chunk_start,
-                                      w.chunk_info, st);
-    return from_cuda(e);
-}
-
-// The CUDA-core plan after the chunk table: a1 .. a4 as four kernels.
-kda_status_t run_simt(const void* q, const void* k, const void* v, const float* g,
-                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
-                      int B, int T, const Prefill& p, int H, int dk, int dv, int chunk,
-                      kda_dtype_t dtype, void* o, float* final_state, const Workspace& w,
-                      int maxc, cudaStream_t st) {
-    cudaError_t e = kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
-    if (e == cudaSuccess)
-        e = kda::launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, chunk, dtype,
-                              w.status, w.W, w.U, st);
-    if (e == cudaSuccess)
-        e = kda::launch_inter(k, w.G, w.W, w.U, initial_state, cu_seqlens, B, T, p.N,
-                              w.chunk_start, H, dk, dv, chunk, dtype, w.status, w.states,
-                              final_state, st);
-    if (e == cudaSuccess)
-        e = kda::launch_output(q, k, w.G, w.U, w.states, w.chunk_info, maxc, H, dk, dv, chunk,
-                               dtype, w.status, o, st);
-    return from_cuda(e);
-}
 
 // Gated DeltaNet (head-uniform gate): the split plan reads the gate per
 // (token, head) directly; every other shape spreads it over the dk channels
 // into the workspace, after the CUDA-core plan's own part, and runs that plan.
 Path gdn_path(int dk, int dv, int chunk, kda_dtype_t dt) {
-    const bool tc_shape = dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && chunk == 64 &&
-                          kda::tc_path_available();
-    const char* env = getenv("KDA_CHUNK_PATH");
-    if (env && !strcmp(env, "simt")) return Path::Simt;
-    return tc_shape ? Path::Split : Path::Simt;
+    return tc_shape(dk, dv, chunk, dt) ? Path::Split : Path::Simt;
 }
 
 size_t gdn_workspace_bytes(const Prefill& p, int H, int dk, int dv, int chunk, Path path,
@@ -191,13 +216,8 @@ int kda_chunk_fwd_plan(int total_tokens, int num_seqs, int packed, int H, int dk
     if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
         !chunk_ok(chunk) || !dtype_ok(dtype))
         return -1;
-    switch (select_path(total_tokens, num_seqs, packed != 0, H, dk, dv, chunk, dtype)) {
-        case Path::Simt: return KDA_PLAN_SIMT;
-        case Path::Fused: return KDA_PLAN_FUSED;
-        case Path::Split: return KDA_PLAN_SPLIT;
-        case Path::Overlap: return KDA_PLAN_OVERLAP;
-    }
-    return -1;
+    return static_cast<int>(
+        select_path(total_tokens, num_seqs, packed != 0, H, dk, dv, chunk, dtype));
 }
 
 size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
@@ -205,38 +225,46 @@ size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int d
     if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
         !chunk_ok(chunk) || !dtype_ok(dtype))
         return 0;
-    return workspace_bytes_for(total_tokens, num_seqs, H, dk, dv, chunk, dtype);
+    // the split and co-scheduled plans share one layout, so packing does not matter
+    return workspace_bytes_for(total_tokens, num_seqs, H, dk, dv, chunk,
+                               select_path(total_tokens, num_seqs, false, H, dk, dv, chunk,
+                                           dtype));
 }
 
-kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
-                           const float* beta, const float* initial_state,
-                           const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
-                           int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
-                           float* final_state, void* workspace, size_t workspace_bytes,
-                           void* stream) {
-    Prefill p;
-    kda_status_t s =
-        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);
-    if (s != KDA_OK) return s;
+size_t kda_chunk_fwd_plan_workspace_size(int plan, int total_tokens, int num_seqs, int H, int dk,
+                                         int dv, int chunk, kda_dtype_t dtype) {
+    Path path;
+    if (!plan_from_int(plan, &path) || total_tokens < 0 || num_seqs < 1 || H < 1 ||
+        !dim_ok(dk) || !dim_ok(dv) || !chunk_ok(chunk) || !dtype_ok(dtype) ||
+        !path_applies(path, num_seqs, H, dk, dv, chunk, dtype))
+        return 0;
+    return workspace_bytes_for(total_tokens, num_seqs, H, dk, dv, chunk, path);
+}
+
+}  // extern "C"
+
+namespace {
+
+// kda_chunk_fwd's body on a given plan (checked to apply).
+kda_status_t chunk_fwd_on(Path path, const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* initial_state,
+                          const int32_t* cu_seqlens, int B, int T, const Prefill& p, int H,
+                          int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                          float* final_state, void* workspace, size_t workspace_bytes,
+                          void* stream) {
     if (!q || !k || !v || !g || !beta || !o) return KDA_ERR_INVALID_ARG;
     for (const void* ptr : {q, k, v, (const void*)g, (const void*)beta, (const void*)o})
         if (!aligned16(ptr)) return KDA_ERR_INVALID_ARG;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_INVALID_ARG;
-    const Path path = select_path(p.total, p.N, cu_seqlens != nullptr, H, dk, dv, chunk, dtype);
     Workspace w;
-    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, path, &w);
+    kda_status_t s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, path, &w);
     if (s != KDA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int maxc = kda::max_chunks(p.total, p.N, chunk);
     s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);
     if (s != KDA_OK) return s;
     if (p.total == 0 && !final_state) return KDA_OK;
-    if (path == Path::Fused) {
-        return from_cuda(kda::launch_chunk_fwd_tc(q, k, v, g, beta, initial_state, cu_seqlens,
-                                                  T, p.N, H, w.chunk_start, w.status, o,
-                                                  final_state, st));
-    }
     if (path == Path::Overlap) {
         return from_cuda(kda::launch_chunk_fwd_overlap(q, k, v, g, beta, initial_state,
                                                        cu_seqlens, T, p.N, H, w.chunk_info,
@@ -253,6 +281,42 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
                     dtype, o, final_state, w, maxc, st);
 }
 
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                           int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
+                           float* final_state, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    Prefill p;
+    kda_status_t s =
+        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);
+    if (s != KDA_OK) return s;
+    const Path path = select_path(p.total, p.N, cu_seqlens != nullptr, H, dk, dv, chunk, dtype);
+    return chunk_fwd_on(path, q, k, v, g, beta, initial_state, cu_seqlens, B, T, p, H, dk, dv,
+                        chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
+}
+
+kda_status_t kda_chunk_fwd_with_plan(int plan, const void* q, const void* k, const void* v,
+                                     const float* g, const float* beta,
+                                     const float* initial_state, const int32_t* cu_seqlens, int B,
+                                     int T, int num_seqs, int H, int dk, int dv, int chunk,
+                                     kda_dtype_t dtype, void* o, float* final_state,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    Path path;
+    if (!plan_from_int(plan, &path)) return KDA_ERR_INVALID_ARG;
+    Prefill p;
+    kda_status_t s =
+        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);
+    if (s != KDA_OK) return s;
+    if (!path_applies(path, p.N, H, dk, dv, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    return chunk_fwd_on(path, q, k, v, g, beta, initial_state, cu_seqlens, B, T, p, H, dk, dv,
+                        chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
+}
+
 // ------------------------------------------------- one step per call (a1-a4)
 
 #define KDA_PREFILL_PROLOGUE(...)                                                   \
@@ -263,7 +327,7 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
     for (const void* ptr : std::initializer_list<const void*>{__VA_ARGS__})              \
         if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;                          \
     Workspace w;                                                                          \
-    s = check_ws(workspace, workspace_bytes, p, H, dk, dv, chunk, Path::Fused, &w);       \
+    s = check_ws_header(workspace, workspace_bytes, p, H, dk, dv, chunk, &w);          \
     if (s != KDA_OK) return s;                                                            \
     cudaStream_t st = static_cast<cudaStream_t>(stream);                                  \
     const int maxc = kda::max_chunks(p.total, p.N, chunk);

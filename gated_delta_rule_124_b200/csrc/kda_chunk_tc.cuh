@@ -7,17 +7,13 @@
 
 namespace kda {
 
-// True when the tensor-core prefill kernel is compiled into this library.
+// True when the tensor-core prefill kernels can run (the driver entry point
+// that encodes TMA tensor maps is available).
 bool tc_path_available();
 
-cudaError_t launch_chunk_fwd_tc(const void* q, const void* k, const void* v, const float* g,
-                                const float* beta, const float* h0, const int32_t* cu_seqlens,
-                                int T, int N, int H, const int* chunk_start,
-                                uint32_t* status, void* o, float* hN, cudaStream_t st);
-
-// Two-kernel split of the same computation for problems with few (sequence,
-// head) chains: chunk-parallel intra-chunk kernel + per-chain kernel, handing
-// over through `blobs` (split_blob_bytes() per (chunk slot, head)).
+// The chunkwise prefill as two tensor-core kernels: chunk-parallel
+// intra-chunk kernel + per-chain kernel, handing over through `blobs`
+// (split_blob_bytes() per (chunk slot, head)).
 size_t split_blob_bytes();
 // gh != NULL: the gate is head-uniform, gh [total, H] (g is then unused).
 cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,

@@ -108,6 +108,28 @@ __device__ __forceinline__ bool status_bad(const uint32_t* status) {
 
 }  // namespace kda
 
+// Host-side prefill helpers shared by the entry points (kda_api.cu defines them).
+namespace kda {
+// Tokens and sequences of one prefill call.
+struct Prefill {
+    int total, N;
+};
+// The argument rules every prefill entry point shares (sizes, dtype, the
+// cu_seqlens / B / T / num_seqs combination, supported dk, dv and chunk).
+kda_status_t check_prefill_shape(const int32_t* cu, int B, int T, int num_seqs, int H, int dk,
+                                 int dv, int chunk, kda_dtype_t dt, Prefill* out);
+// Clear the status word and build the chunk table (two stream operations).
+kda_status_t begin_prefill(const Workspace& w, const int32_t* cu, int B, int T, int N, int chunk,
+                           int maxc, cudaStream_t st);
+// The CUDA-core plan after the chunk table: a1 .. a4 as four kernels on the
+// intermediates of `w` (carved with_intermediates).
+kda_status_t run_simt(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                      int B, int T, const Prefill& p, int H, int dk, int dv, int chunk,
+                      kda_dtype_t dtype, void* o, float* final_state, const Workspace& w,
+                      int maxc, cudaStream_t st);
+}  // namespace kda
+
 // Launchers implemented in the .cu files (host side, return cudaError_t).
 namespace kda {
 cudaError_t launch_build_chunk_table(const int32_t* cu_seqlens, int B, int T, int N, int chunk,

@@ -12,8 +12,15 @@
 // CUDA-core path's intermediates) in one statically sized device array.
 //
 // Costs and rules:
-//  * Every GPU on which this library's module is loaded holds the array
-//    (KDA_NOALLOC_SCRATCH_BYTES) until the process exits.
+//  * Every GPU on which this file's device module is loaded holds the array
+//    (KDA_NOALLOC_SCRATCH_BYTES) until the process exits.  When the driver
+//    loads that module is CUDA's choice: with lazy module loading (the
+//    default of CUDA 12, CUDA_MODULE_LOADING=LAZY) it is the first
+//    cudaGetSymbolAddress below, i.e. the first call of this entry point on
+//    the device, so the 64 MiB are committed by that call; with eager loading
+//    they are committed when the context is created.  A caller that reserves
+//    nearly all HBM up front should therefore make its first call (on a tiny
+//    problem, if need be) before taking that reservation.
 //  * The first call on a device looks up the array's device address (one
 //    cudaGetSymbolAddress with that device current) and caches it; make that
 //    first call before any stream capture begins.
@@ -67,8 +74,6 @@ cudaError_t scratch_address(void** out) {
 }
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
-bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
 
 }  // namespace
 
@@ -80,19 +85,11 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
                                               kda_dtype_t dtype, void* o, float* final_state,
                                               void* stream) {
     // --- the same argument rules as kda_chunk_fwd
-    if (B < 1 || T < 0 || num_seqs < 1 || H < 1) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
-    int total, N;
-    if (cu_seqlens) {
-        if (B != 1 || !al16(cu_seqlens)) return KDA_ERR_INVALID_ARG;
-        total = T;
-        N = num_seqs;
-    } else {
-        if (num_seqs != B || (long long)B * T > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
-        total = B * T;
-        N = B;
-    }
-    if (!dim_ok(dk) || !dim_ok(dv) || !chunk_ok(chunk)) return KDA_ERR_UNSUPPORTED;
+    kda::Prefill pf;
+    const kda_status_t chk =
+        kda::check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &pf);
+    if (chk != KDA_OK) return chk;
+    const int total = pf.total, N = pf.N;
     for (const void* p : {q, k, v, (const void*)g, (const void*)beta, (const void*)o})
         if (!p || !al16(p)) return KDA_ERR_INVALID_ARG;
     if ((initial_state && !al16(initial_state)) || (final_state && !al16(final_state)))
@@ -106,22 +103,9 @@ extern "C" kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, cons
     const kda::Workspace w = kda::carve(base, total, N, H, dk, dv, chunk, true);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int maxc = kda::max_chunks(total, N, chunk);
-    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
-    if (e == cudaSuccess)
-        e = kda::launch_build_chunk_table(cu_seqlens, B, T, N, chunk, maxc, w.status,
-                                          w.chunk_start, w.chunk_info, st);
-    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    kda_status_t r = kda::begin_prefill(w, cu_seqlens, B, T, N, chunk, maxc, st);
+    if (r != KDA_OK) return r;
     if (total == 0 && !final_state) return KDA_OK;
-    e = kda::launch_gate_cumsum(g, w.chunk_info, maxc, H, dk, w.status, w.G, st);
-    if (e == cudaSuccess)
-        e = kda::launch_intra(k, v, w.G, beta, w.chunk_info, maxc, H, dk, dv, chunk, dtype,
-                              w.status, w.W, w.U, st);
-    if (e == cudaSuccess)
-        e = kda::launch_inter(k, w.G, w.W, w.U, initial_state, cu_seqlens, B, T, N,
-                              w.chunk_start, H, dk, dv, chunk, dtype, w.status, w.states,
-                              final_state, st);
-    if (e == cudaSuccess)
-        e = kda::launch_output(q, k, w.G, w.U, w.states, w.chunk_info, maxc, H, dk, dv, chunk,
-                               dtype, w.status, o, st);
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::run_simt(q, k, v, g, beta, initial_state, cu_seqlens, B, T, pf, H, dk, dv, chunk,
+                         dtype, o, final_state, w, maxc, st);
 }

@@ -43,6 +43,7 @@ EXPORTS = (
     "kda_output_norm_gate", "kda_gdn_chunk_fwd_workspace_size", "kda_gdn_chunk_fwd",
     "kda_gdn_decode_step", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
     "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd", "kda_qkv_conv_norm_step",
+    "kda_chunk_fwd_with_plan", "kda_chunk_fwd_plan_workspace_size",
 )
 
 
@@ -70,6 +71,8 @@ _SIGS = {
     "kda_chunk_fwd_noalloc": ([_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp], _i),
     "kda_chunk_split_workspace_size": ([_i, _i, _i], _sz),
     "kda_chunk_fwd_plan": ([_i] * 8, _i),
+    "kda_chunk_fwd_with_plan": ([_i] + [_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_chunk_fwd_plan_workspace_size": ([_i] * 8, _sz),
     "kda_qkv_conv_norm": ([_vp] * 7 + [_i] * 7 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_output_norm_gate": ([_vp] * 3 + [_i] * 4 + [ctypes.c_float] + [_vp] * 2, _i),
     "kda_gdn_chunk_fwd_workspace_size": ([_i] * 7, _sz),
@@ -113,12 +116,41 @@ def status_string(status: int) -> str:
 
 
 def _p(t) -> int | None:
-    """Device pointer of a tensor (or None for NULL)."""
+    """Device pointer of a tensor (or None for NULL); a plain int is passed
+    through as a raw address."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
     return t.data_ptr()
+
+
+_TORCH_OF = {KDA_DTYPE_F32: torch.float32, KDA_DTYPE_BF16: torch.bfloat16}
+
+
+def _check(what, dtype=None, typed=(), f32=(), i32=(), raw=()):
+    """Reject tensors the C ABI would misread, before any pointer is passed:
+    every tensor must be contiguous and on one device; `typed` tensors (q, k,
+    v, o, dout ...) must have the call's dtype, `f32` ones (g, beta, states,
+    gradients) float32, `i32` ones (cu_seqlens) int32; `raw` ones (workspaces)
+    only contiguous.  Plain ints (raw addresses) and None are not checked."""
+    want = None if dtype is None else _TORCH_OF[dtype_code(dtype)]
+    dev = None
+    for group, need in ((typed, want), (f32, torch.float32), (i32, torch.int32), (raw, None)):
+        for t in group:
+            if t is None or isinstance(t, int):
+                continue
+            if not isinstance(t, torch.Tensor):
+                raise ValueError(f"{what}: expected a tensor, got {type(t).__name__}")
+            if not t.is_contiguous():
+                raise ValueError(f"{what}: every tensor must be contiguous (got strides "
+                                 f"{tuple(t.stride())} for shape {tuple(t.shape)})")
+            if need is not None and t.dtype != need:
+                raise ValueError(f"{what}: expected {need}, got {t.dtype}")
+            if dev is None:
+                dev = t.device
+            elif t.device != dev:
+                raise ValueError(f"{what}: tensors on {dev} and {t.device}")
 
 
 def _stream(stream) -> int | None:
@@ -156,9 +188,13 @@ def kda_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype
                                                    dtype_code(dtype)))
 
 
-KDA_PLAN_SIMT, KDA_PLAN_FUSED, KDA_PLAN_SPLIT, KDA_PLAN_OVERLAP = 0, 1, 2, 3
-PLAN_NAMES = {KDA_PLAN_SIMT: "simt", KDA_PLAN_FUSED: "fused", KDA_PLAN_SPLIT: "split",
-              KDA_PLAN_OVERLAP: "overlap"}
+KDA_PLAN_SIMT, KDA_PLAN_SPLIT, KDA_PLAN_OVERLAP = 0, 2, 3
+PLAN_NAMES = {KDA_PLAN_SIMT: "simt", KDA_PLAN_SPLIT: "split", KDA_PLAN_OVERLAP: "overlap"}
+PLAN_CODES = {v: k for k, v in PLAN_NAMES.items()}
+
+
+def plan_code(plan) -> int:
+    return PLAN_CODES[plan] if isinstance(plan, str) else int(plan)
 
 
 def kda_chunk_fwd_plan(total_tokens, num_seqs, H, dk, dv, chunk, dtype, packed=False) -> int:
@@ -173,6 +209,8 @@ def kda_num_chunks_upper_bound(total_tokens, num_seqs, chunk) -> int:
 def kda_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H, dk, dv,
                   chunk, dtype, o, final_state, workspace, workspace_bytes=None, stream=None,
                   check=True) -> int:
+    _check("kda_chunk_fwd", dtype, typed=(q, k, v, o), f32=(g, beta, initial_state, final_state),
+           i32=(cu_seqlens,), raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
                               _p(cu_seqlens), B, T, num_seqs, H, dk, dv, chunk,
@@ -181,8 +219,30 @@ def kda_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H
     return _ret(st, "kda_chunk_fwd", check)
 
 
+def kda_chunk_fwd_plan_workspace_size(plan, total_tokens, num_seqs, H, dk, dv, chunk,
+                                      dtype) -> int:
+    return int(load().kda_chunk_fwd_plan_workspace_size(plan_code(plan), total_tokens, num_seqs,
+                                                        H, dk, dv, chunk, dtype_code(dtype)))
+
+
+def kda_chunk_fwd_with_plan(plan, q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H,
+                            dk, dv, chunk, dtype, o, final_state, workspace, workspace_bytes=None,
+                            stream=None, check=True) -> int:
+    """kda_chunk_fwd on an explicitly chosen plan ('simt', 'split', 'overlap'
+    or its KDA_PLAN_* code); KDA_ERR_UNSUPPORTED where it cannot run."""
+    _check("kda_chunk_fwd_with_plan", dtype, typed=(q, k, v, o),
+           f32=(g, beta, initial_state, final_state), i32=(cu_seqlens,), raw=(workspace,))
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_fwd_with_plan(plan_code(plan), _p(q), _p(k), _p(v), _p(g), _p(beta),
+                                        _p(initial_state), _p(cu_seqlens), B, T, num_seqs, H,
+                                        dk, dv, chunk, dtype_code(dtype), _p(o),
+                                        _p(final_state), _p(workspace), wb, _stream(stream))
+    return _ret(st, "kda_chunk_fwd_with_plan", check)
+
+
 def kda_chunk_gate_cumsum(g, cu_seqlens, B, T, num_seqs, H, dk, chunk, G, workspace,
                           workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_chunk_gate_cumsum", None, f32=(g, G), i32=(cu_seqlens,), raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_gate_cumsum(_p(g), _p(cu_seqlens), B, T, num_seqs, H, dk, chunk,
                                       _p(G), _p(workspace), wb, _stream(stream))
@@ -191,6 +251,8 @@ def kda_chunk_gate_cumsum(g, cu_seqlens, B, T, num_seqs, H, dk, chunk, G, worksp
 
 def kda_chunk_intra(k, v, G, beta, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, W, Ut,
                     workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_chunk_intra", dtype, typed=(k, v), f32=(G, beta, W, Ut), i32=(cu_seqlens,),
+           raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_intra(_p(k), _p(v), _p(G), _p(beta), _p(cu_seqlens), B, T, num_seqs,
                                 H, dk, dv, chunk, dtype_code(dtype), _p(W), _p(Ut),
@@ -201,6 +263,8 @@ def kda_chunk_intra(k, v, G, beta, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk,
 def kda_chunk_inter(k, G, W, U, initial_state, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk,
                     dtype, chunk_states, final_state, workspace, workspace_bytes=None,
                     stream=None, check=True) -> int:
+    _check("kda_chunk_inter", dtype, typed=(k,), f32=(G, W, U, initial_state, chunk_states,
+           final_state), i32=(cu_seqlens,), raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_inter(_p(k), _p(G), _p(W), _p(U), _p(initial_state), _p(cu_seqlens),
                                 B, T, num_seqs, H, dk, dv, chunk, dtype_code(dtype),
@@ -212,6 +276,8 @@ def kda_chunk_inter(k, G, W, U, initial_state, cu_seqlens, B, T, num_seqs, H, dk
 def kda_chunk_output(q, k, G, U, chunk_states, cu_seqlens, B, T, num_seqs, H, dk, dv, chunk,
                      dtype, o, workspace, workspace_bytes=None, stream=None,
                      check=True) -> int:
+    _check("kda_chunk_output", dtype, typed=(q, k, o), f32=(G, U, chunk_states),
+           i32=(cu_seqlens,), raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_output(_p(q), _p(k), _p(G), _p(U), _p(chunk_states), _p(cu_seqlens),
                                  B, T, num_seqs, H, dk, dv, chunk, dtype_code(dtype), _p(o),
@@ -225,6 +291,8 @@ def kda_chunk_split_workspace_size(total_tokens, num_seqs, H) -> int:
 
 def kda_chunk_split_intra(q, k, g, beta, cu_seqlens, B, T, num_seqs, H, workspace,
                           workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_chunk_split_intra", "bf16", typed=(q, k), f32=(g, beta), i32=(cu_seqlens,),
+           raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_split_intra(_p(q), _p(k), _p(g), _p(beta), _p(cu_seqlens), B, T,
                                       num_seqs, H, _p(workspace), wb, _stream(stream))
@@ -233,6 +301,8 @@ def kda_chunk_split_intra(q, k, g, beta, cu_seqlens, B, T, num_seqs, H, workspac
 
 def kda_chunk_split_chain(v, initial_state, cu_seqlens, B, T, num_seqs, H, o, final_state,
                           workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_chunk_split_chain", "bf16", typed=(v, o), f32=(initial_state, final_state),
+           i32=(cu_seqlens,), raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_split_chain(_p(v), _p(initial_state), _p(cu_seqlens), B, T,
                                       num_seqs, H, _p(o), _p(final_state), _p(workspace), wb,
@@ -248,6 +318,8 @@ def kda_gdn_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, d
 def kda_gdn_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs, H, dk, dv,
                       chunk, dtype, o, final_state, workspace, workspace_bytes=None, stream=None,
                       check=True) -> int:
+    _check("kda_gdn_chunk_fwd", dtype, typed=(q, k, v, o), f32=(g, beta, initial_state,
+           final_state), i32=(cu_seqlens,), raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
                                   _p(cu_seqlens), B, T, num_seqs, H, dk, dv, chunk,
@@ -258,6 +330,7 @@ def kda_gdn_chunk_fwd(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seq
 
 def kda_gdn_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,
                         check=True) -> int:
+    _check("kda_gdn_decode_step", dtype, typed=(q, k, v, o), f32=(g, beta, state))
     st = load().kda_gdn_decode_step(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state), _p(o), N,
                                     H, dk, dv, dtype_code(dtype), _stream(stream))
     return _ret(st, "kda_gdn_decode_step", check)
@@ -270,6 +343,9 @@ def kda_chunk_bwd_workspace_size(total_tokens, num_seqs, H, dk, dv) -> int:
 def kda_chunk_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_seqlens, B, T,
                   num_seqs, H, dk, dv, dtype, dq, dk_out, dv_out, dg, dbeta, dinitial_state,
                   workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_chunk_bwd", dtype, typed=(q, k, v, dout), f32=(g, beta, initial_state,
+           dfinal_state, dq, dk_out, dv_out, dg, dbeta, dinitial_state), i32=(cu_seqlens,),
+           raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_chunk_bwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
                               _p(dout), _p(dfinal_state), _p(cu_seqlens), B, T, num_seqs, H, dk,
@@ -286,6 +362,9 @@ def kda_gdn_chunk_bwd_workspace_size(total_tokens, num_seqs, H, dk, dv) -> int:
 def kda_gdn_chunk_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_seqlens, B, T,
                       num_seqs, H, dk, dv, dtype, dq, dk_out, dv_out, dg, dbeta, dinitial_state,
                       workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_gdn_chunk_bwd", dtype, typed=(q, k, v, dout), f32=(g, beta, initial_state,
+           dfinal_state, dq, dk_out, dv_out, dg, dbeta, dinitial_state), i32=(cu_seqlens,),
+           raw=(workspace,))
     wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
     st = load().kda_gdn_chunk_bwd(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
                                   _p(dout), _p(dfinal_state), _p(cu_seqlens), B, T, num_seqs, H,
@@ -297,6 +376,8 @@ def kda_gdn_chunk_bwd(q, k, v, g, beta, initial_state, dout, dfinal_state, cu_se
 
 def kda_qkv_conv_norm_step(xq, xk, xv, wq, wk, wv, conv_q, conv_k, conv_v, N, H, dk, dv,
                            dtype, eps, q, k, v, stream=None, check=True) -> int:
+    _check("kda_qkv_conv_norm_step", dtype, typed=(xq, xk, xv, conv_q, conv_k, conv_v, q, k, v),
+           f32=(wq, wk, wv))
     st = load().kda_qkv_conv_norm_step(_p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
                                        _p(conv_q), _p(conv_k), _p(conv_v), N, H, dk, dv,
                                        dtype_code(dtype), eps, _p(q), _p(k), _p(v),
@@ -306,6 +387,8 @@ def kda_qkv_conv_norm_step(xq, xk, xv, wq, wk, wv, conv_q, conv_k, conv_v, N, H,
 
 def kda_qkv_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens, B, T, num_seqs, H, dk, dv, dtype,
                       eps, q, k, v, stream=None, check=True) -> int:
+    _check("kda_qkv_conv_norm", dtype, typed=(xq, xk, xv, q, k, v), f32=(wq, wk, wv),
+           i32=(cu_seqlens,))
     st = load().kda_qkv_conv_norm(_p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
                                   _p(cu_seqlens), B, T, num_seqs, H, dk, dv, dtype_code(dtype),
                                   float(eps), _p(q), _p(k), _p(v), _stream(stream))
@@ -314,6 +397,7 @@ def kda_qkv_conv_norm(xq, xk, xv, wq, wk, wv, cu_seqlens, B, T, num_seqs, H, dk,
 
 def kda_output_norm_gate(o, gate, w, total_tokens, H, dv, dtype, eps, y, stream=None,
                          check=True) -> int:
+    _check("kda_output_norm_gate", dtype, typed=(o, gate, y), f32=(w,))
     st = load().kda_output_norm_gate(_p(o), _p(gate), _p(w), total_tokens, H, dv,
                                      dtype_code(dtype), float(eps), _p(y), _stream(stream))
     return _ret(st, "kda_output_norm_gate", check)
@@ -321,6 +405,7 @@ def kda_output_norm_gate(o, gate, w, total_tokens, H, dv, dtype, eps, y, stream=
 
 def kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,
                     check=True) -> int:
+    _check("kda_decode_step", dtype, typed=(q, k, v, o), f32=(g, beta, state))
     st = load().kda_decode_step(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(state), _p(o), N, H,
                                 dk, dv, dtype_code(dtype), _stream(stream))
     return _ret(st, "kda_decode_step", check)
@@ -331,6 +416,8 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num
     """kda_chunk_fwd without a workspace: for callers that may not allocate
     device memory.  The library's own static scratch array is used instead;
     see include/kda.h for its size limit and sharing rules."""
+    _check("kda_chunk_fwd_noalloc", dtype, typed=(q, k, v, o), f32=(g, beta, initial_state,
+           final_state), i32=(cu_seqlens,))
     st = load().kda_chunk_fwd_noalloc(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(initial_state),
                                       _p(cu_seqlens), B, T, num_seqs, H, dk, dv, chunk,
                                       dtype_code(dtype), _p(o), _p(final_state),
@@ -339,6 +426,7 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num
 
 
 def kda_get_device_status(workspace, stream=None) -> int:
+    _check("kda_get_device_status", None, raw=(workspace,))
     return int(load().kda_get_device_status(_p(workspace), _stream(stream)))
 
 

@@ -94,29 +94,24 @@ size_t kda_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int d
 
 /* Plans of kda_chunk_fwd (which kernels one call runs):
  *   KDA_PLAN_SIMT     the CUDA-core kernels: gate cumsum, intra, inter, output;
- *   KDA_PLAN_FUSED    one tensor-core kernel, one CTA per (sequence, head)
- *                     walking its chunks (runs only when forced, see below);
  *   KDA_PLAN_SPLIT    kda_chunk_split_intra then kda_chunk_split_chain (below):
  *                     the chunk-parallel part on every SM, then the chains;
  *   KDA_PLAN_OVERLAP  the same two kernels co-scheduled in one cooperative
  *                     launch, chains and intra-chunk work on disjoint SMs,
  *                     each chain starting on a chunk as soon as that chunk's
- *                     operands are ready.  Taken when the chain length is known
- *                     on the host (no cu_seqlens, or a single packed sequence),
- *                     2 * num_seqs * H is below the number of SMs, and a cost
- *                     model says that the chains, not the intra-chunk work,
- *                     are the longer part (long sequences, few heads).
- * kda_chunk_fwd_plan returns the plan for these arguments on the current
- * device (`packed` != 0: the call passes cu_seqlens), or -1 for arguments
- * kda_chunk_fwd_workspace_size() rejects.  The split and overlap plans share
- * one workspace layout.  The environment variable KDA_CHUNK_PATH = fused |
- * split | overlap | simt forces a plan (testing; shapes without the
- * tensor-core plans always run SIMT, and overlap falls back to split where the
- * launch does not apply); it is read by every call, so set it before sizing
- * the workspace, not between the two calls. */
+ *                     operands are ready.  Runs only where 2 * num_seqs * H is
+ *                     below the number of SMs (one SM per chain half).
+ * The default plan depends only on the arguments and the device: SIMT for
+ * every shape other than bf16, dk = dv = 128, chunk = 64; for that shape
+ * OVERLAP when the chain length is known on the host (no cu_seqlens, or a
+ * single packed sequence), the launch applies, and a cost model says that the
+ * chains, not the intra-chunk work, are the longer part (long sequences, few
+ * heads); SPLIT otherwise.  kda_chunk_fwd_plan returns it (`packed` != 0: the
+ * call passes cu_seqlens), or -1 for arguments kda_chunk_fwd_workspace_size()
+ * rejects.  The split and overlap plans share one workspace layout.  (The
+ * value 1 is not a plan.) */
 enum {
     KDA_PLAN_SIMT = 0,
-    KDA_PLAN_FUSED = 1,
     KDA_PLAN_SPLIT = 2,
     KDA_PLAN_OVERLAP = 3
 };
@@ -129,6 +124,24 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
                            int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
                            float* final_state, void* workspace, size_t workspace_bytes,
                            void* stream);
+
+/* kda_chunk_fwd_with_plan: kda_chunk_fwd on an explicitly chosen plan (for
+ * testing one plan against another, and for measuring each), with the same
+ * arguments, results and error behaviour.  A plan that cannot run these
+ * shapes on this device (a tensor-core plan for another shape or dtype, the
+ * overlap plan where its launch does not apply) returns KDA_ERR_UNSUPPORTED;
+ * an unknown plan KDA_ERR_INVALID_ARG.  Its workspace is
+ * kda_chunk_fwd_plan_workspace_size(plan, ...) bytes, which is 0 exactly when
+ * the plan does not apply (or the arguments are invalid). */
+size_t kda_chunk_fwd_plan_workspace_size(int plan, int total_tokens, int num_seqs, int H, int dk,
+                                         int dv, int chunk, kda_dtype_t dtype);
+
+kda_status_t kda_chunk_fwd_with_plan(int plan, const void* q, const void* k, const void* v,
+                                     const float* g, const float* beta,
+                                     const float* initial_state, const int32_t* cu_seqlens, int B,
+                                     int T, int num_seqs, int H, int dk, int dv, int chunk,
+                                     kda_dtype_t dtype, void* o, float* final_state,
+                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* --------------------------------------------- prefill, one step per call
  * The four steps of the chunkwise form as separate calls, with the
@@ -255,7 +268,7 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
  * bf16, dk = dv = 128, chunk 64 runs the split tensor-core plan with the gate
  * read per (token, head) (one exponential per row instead of per element);
  * other shapes spread g over the dk channels in the workspace and run the
- * CUDA-core plan.  KDA_CHUNK_PATH=simt forces the latter.
+ * CUDA-core plan.
  */
 size_t kda_gdn_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
                                         int chunk, kda_dtype_t dtype);
@@ -389,11 +402,16 @@ kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* 
  * fragment that reservation or stall other streams.  The pages have no
  * counterpart to this call; it is a packaging choice of this library.
  * Scratch: one static device array of KDA_NOALLOC_SCRATCH_BYTES inside the
- *      library, held on every GPU that loads the library until the process
- *      exits.  The first call on a device looks up that array's address (with
- *      the device current) -- make it before any stream capture.  Calls share
- *      the array: results never depend on an earlier call, but calls whose
- *      work overlaps on the GPU race.
+ *      library, held on every GPU that loads it until the process exits.
+ *      When it is committed is the CUDA driver's module-loading choice: with
+ *      lazy loading (CUDA 12's default) it is the first call of this entry
+ *      point on the device, with eager loading the creation of the context.
+ *      So a caller that reserves nearly all HBM up front makes its first call
+ *      (a tiny problem will do) before taking that reservation; later calls
+ *      take no memory.  The first call on a device also looks up the array's
+ *      address (with the device current) -- make it before any stream
+ *      capture.  Calls share the array: results never depend on an earlier
+ *      call, but calls whose work overlaps on the GPU race.
  * Limit: a problem fits when kda_chunk_fwd_workspace_size(total_tokens,
  *      num_seqs, H, dk, dv, chunk, KDA_DTYPE_F32) <= KDA_NOALLOC_SCRATCH_BYTES;
  *      otherwise KDA_ERR_WORKSPACE and nothing is enqueued.

@@ -233,3 +233,60 @@ def test_conv_step_rejects_bad_arguments(lib):
     assert kda.kda_qkv_conv_norm_step(**{**a, "eps": 0.0}) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_qkv_conv_norm_step(**{**a, "N": -1}) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_qkv_conv_norm_step(**{**a, "N": 0}) == kda.KDA_OK
+
+
+def test_explicit_plan_rules(lib):
+    """kda_chunk_fwd_with_plan: an unknown plan is an invalid argument; a
+    plan's workspace size is 0 where it cannot run (a tensor-core plan for
+    fp32, or for another head dimension)."""
+    ws = kda.kda_chunk_fwd_plan_workspace_size
+    assert ws("simt", 4096, 2, 32, 128, 128, 64, "bf16") > 0
+    assert ws("split", 4096, 2, 32, 128, 128, 64, "f32") == 0
+    assert ws("split", 4096, 2, 32, 64, 64, 64, "bf16") == 0
+    assert ws(1, 4096, 2, 32, 128, 128, 64, "bf16") == 0  # 1 is not a plan
+    fake = 1 << 20
+    st = kda.kda_chunk_fwd_with_plan(1, fake, fake, fake, fake, fake, None, None, 1, 64, 1, 1,
+                                     32, 32, 16, "f32", fake, None, fake, 1 << 30, stream=0,
+                                     check=False)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    st = kda.kda_chunk_fwd_with_plan("split", fake, fake, fake, fake, fake, None, None, 1, 64, 1,
+                                     1, 32, 32, 16, "f32", fake, None, fake, 1 << 30, stream=0,
+                                     check=False)
+    assert st == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_default_plan_ignores_the_environment(lib, monkeypatch):
+    """The plan and the workspace size are functions of the arguments only."""
+    f = kda.kda_chunk_fwd_workspace_size
+    before = (f(4096, 2, 32, 128, 128, 64, "bf16"), kda.kda_chunk_fwd_plan(
+        4096, 2, 32, 128, 128, 64, "bf16"))
+    monkeypatch.setenv("KDA_CHUNK_PATH", "simt")
+    after = (f(4096, 2, 32, 128, 128, 64, "bf16"), kda.kda_chunk_fwd_plan(
+        4096, 2, 32, 128, 128, 64, "bf16"))
+    assert before == after
+
+
+def test_python_wrappers_reject_tensors_the_abi_would_misread(lib):
+    """Checked in Python before any pointer reaches the library: a transposed
+    (non-contiguous) view, a bf16 gate, q and v of different dtypes."""
+    import torch
+    T, H, d = 8, 2, 32
+    q = torch.zeros(T, H, d, dtype=torch.bfloat16)
+    g = torch.zeros(T, H, d)
+    beta = torch.zeros(T, H)
+    o = torch.zeros(T, H, d, dtype=torch.bfloat16)
+    ws = torch.zeros(1 << 16, dtype=torch.uint8)
+    args = dict(initial_state=None, cu_seqlens=None, B=1, T=T, num_seqs=1, H=H, dk=d, dv=d,
+                chunk=16, dtype="bf16", o=o, final_state=None, workspace=ws)
+    with pytest.raises(ValueError, match="contiguous"):
+        kda.kda_chunk_fwd(q.transpose(0, 1), q, q, g, beta, **args)
+    with pytest.raises(ValueError, match="float32"):
+        kda.kda_chunk_fwd(q, q, q, g.to(torch.bfloat16), beta, **args)
+    with pytest.raises(ValueError, match="bfloat16"):
+        kda.kda_chunk_fwd(q, q, q.float(), g, beta, **args)
+    with pytest.raises(ValueError, match="float32"):
+        kda.kda_decode_step(q[0], q[0], q[0], g[0], beta[0].to(torch.bfloat16),
+                            torch.zeros(1, H, d, d), o[0], 1, H, d, d, "bf16")
+    with pytest.raises(ValueError, match="contiguous"):
+        kda.kda_decode_step(q[0], q[0], q[0], g[0], beta[0],
+                            torch.zeros(1, H, d, d).transpose(2, 3), o[0], 1, H, d, d, "bf16")

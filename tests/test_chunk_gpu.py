@@ -12,21 +12,32 @@ from tests.helpers import oracle_prefill, rel_err, tol_for
 pytestmark = pytest.mark.gpu
 
 
-def run_fwd(case, final=True):
+def run_fwd(case, final=True, plan=None):
+    """kda_chunk_fwd on the case (its default plan), or kda_chunk_fwd_with_plan."""
     c = case.to("cuda")
     packed = c.cu_seqlens is not None
     B, T = (1, c.total) if packed else (c.B, c.T)
-    ws = kda.alloc_workspace(c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype)
+    if plan is None:
+        ws = kda.alloc_workspace(c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype)
+    else:
+        n = kda.kda_chunk_fwd_plan_workspace_size(plan, c.total, c.N, c.H, c.dk, c.dv, c.chunk,
+                                                  c.dtype)
+        assert n > 0, f"plan {plan} does not apply"
+        ws = torch.empty(n, dtype=torch.uint8, device="cuda")
     o = torch.full_like(c.v, float("nan"))
     hN = torch.full((c.N, c.H, c.dk, c.dv), float("nan"), device="cuda") if final else None
-    kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, B, T, c.N,
-                      c.H, c.dk, c.dv, c.chunk, c.dtype, o, hN, ws)
+    args = (c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, B, T, c.N, c.H, c.dk,
+            c.dv, c.chunk, c.dtype, o, hN, ws)
+    if plan is None:
+        kda.kda_chunk_fwd(*args)
+    else:
+        kda.kda_chunk_fwd_with_plan(plan, *args)
     assert kda.kda_get_device_status(ws) == kda.KDA_OK
     return o, hN
 
 
-def check_case(case, heads=None):
-    o, hN = run_fwd(case)
+def check_case(case, heads=None, plan=None):
+    o, hN = run_fwd(case, plan=plan)
     ro, rh = oracle_prefill(case, heads)
     sl = slice(None) if heads is None else list(heads)
     tol = tol_for(case.dtype)
@@ -232,10 +243,11 @@ def test_varlen_edge_lengths_bf16_d128(lens):
     check_case(case)
 
 
-# ----------------------------- every prefill path on the same problems
-# bf16, d = 128, chunk 64 can run as one tensor-core kernel per (sequence, head)
-# ("fused"), as the chunk-parallel + per-chain pair ("split"), or on the
-# CUDA-core kernels ("simt"); KDA_CHUNK_PATH forces the choice.
+# ----------------------------- every prefill plan on the same problems
+# bf16, d = 128, chunk 64 runs as the chunk-parallel + per-chain pair of
+# tensor-core kernels ("split"), the same pair co-scheduled in one launch
+# ("overlap"), or on the CUDA-core kernels ("simt"); kda_chunk_fwd_with_plan
+# chooses one explicitly.
 
 PATH_CASES = {
     "varlen": lambda: wl.make_prefill(301, [300, 77, 1, 128], H=4, dk=128, dv=128, chunk=64,
@@ -251,64 +263,60 @@ PATH_CASES = {
 }
 
 
-@pytest.fixture
-def chunk_path(request, monkeypatch):
-    monkeypatch.setenv("KDA_CHUNK_PATH", request.param)
-    return request.param
-
-
-def assert_plan(case, name):
-    """The forced plan is the one the library reports for this problem."""
-    plan = kda.kda_chunk_fwd_plan(case.total, case.N, case.H, case.dk, case.dv, case.chunk,
-                                  case.dtype, packed=case.cu_seqlens is not None)
-    assert kda.PLAN_NAMES[plan] == name, (kda.PLAN_NAMES[plan], name)
-
-
-@pytest.mark.parametrize("chunk_path", ["fused", "split", "overlap", "simt"], indirect=True)
+@pytest.mark.parametrize("plan", ["split", "overlap", "simt"])
 @pytest.mark.parametrize("name", sorted(PATH_CASES))
-def test_every_path_matches_oracle(chunk_path, name):
-    case = PATH_CASES[name]()
-    assert_plan(case, chunk_path)
-    check_case(case)
+def test_every_plan_matches_oracle(plan, name):
+    check_case(PATH_CASES[name](), plan=plan)
 
 
-@pytest.mark.parametrize("chunk_path", ["fused", "split", "overlap"], indirect=True)
-def test_tc_paths_mixed_fast_and_exact_chunks(chunk_path):
+@pytest.mark.parametrize("plan", ["split", "overlap"])
+def test_tc_plans_mixed_fast_and_exact_chunks(plan):
     case = wl.make_prefill(306, [64 * 4 + 10], H=2, dk=128, dv=128, chunk=64, dtype="bf16")
     case.g[64:128] *= 6.0
-    assert_plan(case, chunk_path)
-    check_case(case)
+    check_case(case, plan=plan)
+
+
+def test_plan_that_does_not_apply_is_unsupported():
+    """A tensor-core plan for an fp32 problem: KDA_ERR_UNSUPPORTED, and its
+    workspace size is 0."""
+    case = wl.make_prefill(312, [100], H=2, dk=64, dv=64, chunk=32, dtype="f32").to("cuda")
+    assert kda.kda_chunk_fwd_plan_workspace_size("split", case.total, 1, 2, 64, 64, 32,
+                                                 "f32") == 0
+    ws = kda.alloc_workspace(case.total, 1, 2, 64, 64, 32, "f32")
+    o = torch.empty_like(case.v)
+    st = kda.kda_chunk_fwd_with_plan("split", case.q, case.k, case.v, case.g, case.beta, None,
+                                     None, 1, case.total, 1, 2, 64, 64, 32, "f32", o, None, ws,
+                                     check=False)
+    assert st == kda.KDA_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("lengths", [[640, 333], [64 * 40, 1, 64 * 7 + 5, 0, 200]])
-def test_overlap_and_split_identical(monkeypatch, lengths):
+def test_overlap_and_split_identical(lengths):
     """The co-scheduled launch runs the same device code as the two-launch
     split, only interleaved: identical bits."""
     case = wl.make_prefill(310, lengths, H=3, dk=128, dv=128, chunk=64, dtype="bf16",
                            varlen=True)
-    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
-    o1, h1 = run_fwd(case)
-    monkeypatch.setenv("KDA_CHUNK_PATH", "overlap")
-    assert_plan(case, "overlap")
-    o2, h2 = run_fwd(case)
+    o1, h1 = run_fwd(case, plan="split")
+    o2, h2 = run_fwd(case, plan="overlap")
     assert torch.equal(o1, o2) and torch.equal(h1, h2)
 
 
-def test_overlap_repeated_calls_same_workspace(monkeypatch):
+def test_overlap_repeated_calls_same_workspace():
     """Ready flags are reset by every call: back-to-back calls on one
     workspace give identical results."""
-    monkeypatch.setenv("KDA_CHUNK_PATH", "overlap")
     case = wl.make_prefill(311, [500, 64 * 9], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
                            varlen=True)
-    assert_plan(case, "overlap")
     c = case.to("cuda")
-    ws = kda.alloc_workspace(c.total, c.N, c.H, 128, 128, 64, "bf16")
+    ws = torch.empty(kda.kda_chunk_fwd_plan_workspace_size("overlap", c.total, c.N, c.H, 128,
+                                                           128, 64, "bf16"),
+                     dtype=torch.uint8, device="cuda")
     outs = []
     for _ in range(3):
         o = torch.empty_like(c.v)
         hN = torch.empty(c.N, c.H, 128, 128, device="cuda")
-        kda.kda_chunk_fwd(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, 1,
-                          c.total, c.N, c.H, 128, 128, 64, "bf16", o, hN, ws)
+        kda.kda_chunk_fwd_with_plan("overlap", c.q, c.k, c.v, c.g, c.beta, c.initial_state,
+                                    c.cu_seqlens, 1, c.total, c.N, c.H, 128, 128, 64, "bf16", o,
+                                    hN, ws)
         outs.append((o, hN))
     assert kda.kda_get_device_status(ws) == kda.KDA_OK
     for o, hN in outs[1:]:
@@ -317,10 +325,9 @@ def test_overlap_repeated_calls_same_workspace(monkeypatch):
     assert rel_err(outs[0][0], ro) <= tol_for("bf16")
 
 
-def test_default_plans(monkeypatch):
-    """Without an override: long chains over few heads -> overlap; short
-    chains, many chains, or packed sequences of unknown length -> split."""
-    monkeypatch.delenv("KDA_CHUNK_PATH", raising=False)
+def test_default_plans():
+    """Long chains over few heads -> overlap; short chains, many chains, or
+    packed sequences of unknown length -> split; other shapes -> simt."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     f = kda.kda_chunk_fwd_plan
     assert f(65536, 1, 32, 128, 128, 64, "bf16") == kda.KDA_PLAN_OVERLAP
@@ -331,30 +338,12 @@ def test_default_plans(monkeypatch):
     assert f(4096, 2, 32, 128, 128, 64, "f32") == kda.KDA_PLAN_SIMT
 
 
-def test_split_and_fused_agree_closely(monkeypatch):
-    """The two tensor-core paths use the same factorisation and operand
-    layouts; only the in-chunk cumulative sum of g is taken in a different
-    order (sequential in the fused kernel, two-level in the split one), so an
-    operand can round to the neighbouring bf16 value.  Their results agree far
-    inside the oracle tolerance."""
-    case = wl.make_prefill(307, [640, 333], H=4, dk=128, dv=128, chunk=64, dtype="bf16",
-                           varlen=True)
-    monkeypatch.setenv("KDA_CHUNK_PATH", "fused")
-    o1, h1 = run_fwd(case)
-    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
-    o2, h2 = run_fwd(case)
-    torch.cuda.synchronize()
-    assert rel_err(o2, o1.double().cpu().numpy()) <= 1e-2
-    assert rel_err(h2, h1.double().cpu().numpy()) <= 2e-3
-
-
-def test_split_step_calls_compose(monkeypatch):
+def test_split_step_calls_compose():
     """kda_chunk_split_intra then kda_chunk_split_chain is the split plan of
     kda_chunk_fwd: identical bits, and within tolerance of the oracle."""
     case = wl.make_prefill(308, [333, 64, 0, 700], H=3, dk=128, dv=128, chunk=64,
                            dtype="bf16", varlen=True)
-    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
-    o1, h1 = run_fwd(case)
+    o1, h1 = run_fwd(case, plan="split")
     c = case.to("cuda")
     n = kda.kda_chunk_split_workspace_size(c.total, c.N, c.H)
     assert n == kda.kda_chunk_fwd_workspace_size(c.total, c.N, c.H, 128, 128, 64, "bf16")

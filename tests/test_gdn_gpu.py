@@ -45,13 +45,11 @@ def _check(case, gh, gfull):
     return o, hN
 
 
-@pytest.mark.parametrize("path", ["default", "simt"])
-def test_gdn_prefill_bf16_d128(monkeypatch, path):
-    if path == "simt":
-        monkeypatch.setenv("KDA_CHUNK_PATH", "simt")
-    else:
-        monkeypatch.delenv("KDA_CHUNK_PATH", raising=False)
-    case = wl.make_prefill(401, [300, 77, 1, 128], H=4, dk=128, dv=128, chunk=64,
+@pytest.mark.parametrize("d,C", [(128, 64), (64, 32)])
+def test_gdn_prefill_bf16(d, C):
+    """d = 128, chunk 64: the split tensor-core plan with the gate read per
+    (token, head); d = 64: the gate spread over the channels, CUDA-core plan."""
+    case = wl.make_prefill(401, [300, 77, 1, 128], H=4, dk=d, dv=d, chunk=C,
                            dtype="bf16", varlen=True)
     gh, gfull = _head_gate(case, 1)
     _check(case, gh, gfull)

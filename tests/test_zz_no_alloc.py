@@ -6,7 +6,10 @@ reserved nearly all HBM up front -- and cannot pass a workspace.  This entry
 point uses a static scratch array inside the library instead.  The GPU test
 calls it twice in a row, through the C ABI, on two different problems (so the
 second call runs on scratch the first one left behind) and compares each
-result with kda_chunk_fwd's.  This file is collected last on purpose.
+result with kda_chunk_fwd's, and reads the device's free memory around the
+calls: the static array is committed by the first call (lazy module loading)
+or before it (eager loading), never by a later one.  This file is collected
+last on purpose.
 """
 import pytest
 import torch
@@ -35,6 +38,33 @@ def _no_alloc(c):
     kda.kda_chunk_fwd_noalloc(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, 1,
                               c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype, o, hN)
     return o, hN
+
+
+@pytest.mark.gpu
+def test_no_alloc_commits_its_scratch_once():
+    """Free device memory around the calls (torch allocates nothing in
+    between): the first call takes either the whole static array (lazy module
+    loading: the driver loads the array's module on that call) or nothing
+    (eager loading, or an earlier call already did); a repeated call takes
+    nothing."""
+    c = _problem(503, [130, 7], H=2, d=64, C=32, dtype="f32").to("cuda")
+    _with_workspace(c)  # loads the CUDA-core kernels this problem runs
+    o = torch.empty_like(c.v)
+    hN = torch.empty(c.N, c.H, c.dk, c.dv, device="cuda")
+    torch.cuda.synchronize()
+    mib = 1 << 20
+    free0 = torch.cuda.mem_get_info()[0]
+    for i in range(2):
+        kda.kda_chunk_fwd_noalloc(c.q, c.k, c.v, c.g, c.beta, c.initial_state, c.cu_seqlens, 1,
+                                  c.total, c.N, c.H, c.dk, c.dv, c.chunk, c.dtype, o, hN)
+        torch.cuda.synchronize()
+        if i == 0:
+            free1 = torch.cuda.mem_get_info()[0]
+    free2 = torch.cuda.mem_get_info()[0]
+    first = free0 - free1
+    assert abs(first) <= 4 * mib or \
+        abs(first - kda.KDA_NOALLOC_SCRATCH_BYTES) <= 4 * mib, first / mib
+    assert free1 - free2 == 0, (free1 - free2) / mib
 
 
 @pytest.mark.gpu
