@@ -2,14 +2,20 @@
 """Benchmark: KDA prefill tokens/s and decode tokens/s on one B200 (replicas for N > 1).
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-  * prefill leg: kda_chunk_fwd over B=2 sequences x T=2048 tokens, H=32 heads,
-    dk = dv = 128, chunk 64, bf16 q/k/v/o, fp32 g/beta/state (steps a1-a4);
-  * decode leg: kda_decode_step for N=256 sequences x H=32 heads, 128 x 128 fp32
-    state updated in place (step a5); the 8 pre-drawn input sets are cycled.
+  * prefill leg: kda_chunk_fwd over the varlen workload -- 16 packed sequences
+    of U[1024, 16384] tokens (seeded), H=32 heads, dk = dv = 128, chunk 64,
+    bf16 q/k/v/o, fp32 g/beta/state (steps a1-a4), the largest configuration;
+  * decode leg: the decode workload, N=256 sequences x H=32 heads, 128 x 128
+    fp32 states updated in place, all 1000 steps of its schedule (8 pre-drawn
+    input sets cycled), one kda_decode_step launch per step (step a5).
 Each leg is timed with CUDA events on the stream it is launched on.  `value` is
 the prefill leg's tokens/s (sum of sequence lengths, not x heads); the decode
-leg's tokens/s (sequences x steps) is reported in `decode`.  L2 is flushed
-(a 256 MiB write) before each leg of each step, outside the leg's events.
+leg's tokens/s (sequences x steps) is reported in `decode`.  Both workloads are
+larger than L2 (≈6 GB of prefill inputs, a 512 MiB state); L2 is also flushed
+(a 256 MiB write) before each prefill leg.  The other prefill configurations
+(B=2 x T=2048 and B=1 x T=65536) are timed outside the step and reported under
+`configs`; `parity` holds the errors of the timed configurations against the
+fp64 oracle.
 
 Multi-GPU: every rank runs an independent replica (no data-path collective;
 the path shards by sequence and head).  value = sum over ranks of the tokens
@@ -43,6 +49,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture; null once it has changed, or for a workload never captured.
 _SPLIT = "gated_delta_rule_124_b200/csrc/kda_chunk_split.cu"
 _CFG1 = "prefill: B=2 H=32 T=2048 d=128 C=64 bf16"
+_CFG3 = "varlen prefill: 16 seqs U[1024,16384] H=32 d=128 C=64 bf16"
 _CFG2 = "long prefill: B=1 H=32 T=65536 d=128 C=64 bf16 slow decay"
 _DECODE = "gated_delta_rule_124_b200/csrc/kda_decode.cu"
 _DEC = "decode: N=256 H=32 d=128 bf16, fp32 state, 8 input sets cycled"
@@ -184,6 +191,51 @@ def prefill_case(wl, args):
     return wl.prefill_config(args.prefill_config)
 
 
+def _events(torch, n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def time_calls(torch, stream, flush, f, reps):
+    """Median device time (s) of f() over `reps` calls, CUDA events on the
+    launching stream, L2 flushed before each call outside its events."""
+    f()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = _events(torch, 2)
+        a.record(stream)
+        f()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(x.elapsed_time(y) for x, y in ts) / 1e3
+
+
+def prefill_roofline(kern, pc, peaks, peak_kind):
+    """Roofline of the dominant kernel of one prefill call: its algorithmic
+    bytes per launch over its CUDA-event time, against the measured HBM copy
+    bandwidth; `traffic` is its ncu DRAM bytes while the source matches."""
+    hbm = peaks["hbm_gbs"]
+    dom_name, dom_s = kern["dominant"]
+    dom_bytes = kern["bytes"][dom_name]
+    return {"kernel": dom_name, "bound": "hbm", "achieved": dom_bytes / dom_s / 1e9,
+            "peak": hbm, "unit": "GB/s", "frac": dom_bytes / dom_s / 1e9 / hbm,
+            "traffic": measured_traffic(dom_name, pc.name),
+            "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+            "per_launch_us": dom_s * 1e6, "algorithmic_bytes_per_launch": dom_bytes}
+
+
+def prefill_summary(P, t, peaks):
+    """tokens/s, HBM and tensor fractions of one prefill call of t seconds."""
+    tx = P.total * P.H
+    pb = prefill_bytes(tx, P.N * P.H)
+    pf = prefill_flops(tx)
+    return {"value": P.total / t, "unit": "tokens/s", "ms_per_call": t * 1e3,
+            "hbm_frac": pb / t / 1e9 / peaks["hbm_gbs"],
+            "tensor_frac": pf / t / 1e12 / peaks["bf16_tflops"],
+            "algorithmic_bytes": pb, "paper_flops": pf}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -195,50 +247,54 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     kda.load()
+    peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
 
     # ---- inputs (resident in HBM before timing)
     pc = prefill_case(wl, args)
     P = pc.to(dev)
     dcase = wl.decode_config()
     D = [{k: v.to(dev) for k, v in s.items()} for s in dcase.steps]
-    state = dcase.state0.to(dev)
+    state0 = dcase.state0.to(dev)
+    state = state0.clone()
     Np, H, dk, dv, C = P.N, P.H, P.dk, P.dv, P.chunk
     total = P.total
     ws = kda.alloc_workspace(total, Np, H, dk, dv, C, "bf16", dev)
     o = torch.empty_like(P.v)
     hN = torch.empty(Np, H, dk, dv, dtype=torch.float32, device=dev)
     Nd = dcase.N
+    dsteps = args.decode_steps
     od = torch.empty(Nd, H, dv, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
 
-    def prefill():
+    def prefill(out=o):
         kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc, Tc, Np,
-                          H, dk, dv, C, "bf16", o, hN, ws)
+                          H, dk, dv, C, "bf16", out, hN, ws)
 
-    def decode(i):
-        s = D[i % len(D)]
-        kda.kda_decode_step(s["q"], s["k"], s["v"], s["g"], s["beta"], state, od, Nd, H, dk,
-                            dv, "bf16")
+    def decode_pass(st, outs=None):
+        for i in range(dsteps):
+            s = D[i % len(D)]
+            kda.kda_decode_step(s["q"], s["k"], s["v"], s["g"], s["beta"], st,
+                                od if outs is None else outs[i], Nd, H, dk, dv, "bf16")
 
-    def step(i, ev=None):
+    def step(ev=None):
         flush.zero_()
         if ev: ev[0].record(stream)
         prefill()
         if ev: ev[1].record(stream)
-        flush.zero_()
         if ev: ev[2].record(stream)
-        decode(i)
+        decode_pass(state)
         if ev: ev[3].record(stream)
 
     for i in range(args.warmup):
-        step(i)
+        step()
     torch.cuda.synchronize()
     assert kda.kda_get_device_status(ws) == kda.KDA_OK
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [_events(torch, 4) for _ in range(args.steps)]
+    t0, t1 = _events(torch, 2)
     clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
     if world > 1:
         dist.barrier()
@@ -246,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     clocks.start()
     t0.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, evs[i])
+        step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -260,81 +316,204 @@ def run_ours(args, rank, world, local_rank):
     # ---- max over ranks (device time), whole-job throughput
     total_ms, pre_sum, dec_sum = max_over_ranks([total_ms, pre_sum, dec_sum], world, dev)
     value = job_throughput(total, world, args.steps, pre_sum)
-    dec_value = job_throughput(Nd, world, args.steps, dec_sum)
+    dec_value = job_throughput(Nd * dsteps, world, args.steps, dec_sum)
 
     # ---- per-kernel times of the prefill (dominant kernel) with the step calls
-    kern = prefill_kernel_times(kda, P, ws, dev, stream, reps=max(5, min(50, args.steps)))
+    reps = max(5, min(20, args.steps))
+    kern = prefill_kernel_times(kda, P, ws, dev, stream, reps=reps)
+    pre_avg = pre_sum / args.steps / 1e3  # s
+    prefill_entry = prefill_summary(P, pre_avg, peaks)
+    prefill_entry["kernels_us"] = {k: v * 1e6 for k, v in kern["times"].items()}
+    roof = prefill_roofline(kern, pc, peaks, peak_kind)
+
+    # ---- parity of the timed configurations against the fp64 oracle (one
+    # untimed call each), the oracle's time doubling as the CPU baseline
+    do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    parity, cpu = {}, None
+    if do_cpu:
+        o_chk = torch.full_like(P.v, float("nan"))
+        prefill(o_chk)
+        torch.cuda.synchronize()
+        cpu, parity[pc.name] = oracle_prefill_parity(pc, o_chk, hN)
+        del o_chk
+
+    # ---- the other prefill configurations, each timed outside the step
+    configs = {}
+    if not args.only_headline:
+        for idx in (1, 2):
+            pcx = wl.prefill_config(idx)
+            if pcx.name == pc.name:
+                continue
+            configs[str(idx)] = prefill_config_entry(kda, torch, pcx, dev, stream, flush, peaks,
+                                                     peak_kind, reps, do_cpu, parity)
+
+    # ---- decode: roofline and a parity pass from the initial state
+    dec_avg = dec_sum / args.steps / dsteps / 1e3  # s per decode step
+    db = decode_bytes(Nd * H)
+    decode_entry = {"value": dec_value, "unit": "tokens/s", "ms_per_step": dec_avg * 1e3,
+                    "steps_per_pass": dsteps,
+                    "roofline": {"bound": "hbm", "achieved": db / dec_avg / 1e9, "peak": hbm,
+                                 "unit": "GB/s", "frac": db / dec_avg / 1e9 / hbm,
+                                 "traffic": measured_traffic("decode", dcase.name),
+                                 "algorithmic_bytes_per_launch": db}}
+    if do_cpu:
+        outs = torch.empty(dsteps, Nd, H, dv, dtype=torch.bfloat16, device=dev)
+        st = state0.clone()
+        decode_pass(st, outs)
+        torch.cuda.synchronize()
+        decode_entry["cpu_baseline"], parity[dcase.name] = oracle_decode_parity(
+            dcase, dsteps, outs, st, seqs=args.decode_parity_seqs)
+        del outs, st
 
     # ---- the steps around the operator (conv/Swish/L2-norm before, RMSNorm and
     # output gate after), on this workload's tensors, each timed alone
-    layer = layer_times(kda, torch, P, dev, stream, reps=max(5, min(50, args.steps)))
+    layer = layer_times(kda, torch, P, dev, stream, reps=reps)
 
     # ---- end to end through host buffers (pinned), copies inside the region
-    e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=max(3, min(args.steps, 50)))
+    e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=3)
 
-    # ---- the backward (gradients of o and the final state) on the same workload,
-    # last: a failure there is reported in its entry and leaves the line intact
+    # ---- the backward (gradients of o and the final state) on the B=2 x
+    # T=2048 workload, last: a failure there is reported in its entry and
+    # leaves the line intact
     bwd = None
     if not args.no_backward:
         try:
+            pcb = wl.prefill_config(1)
             bwd = backward_times(
-                kda, torch, P, pc, dev, stream, reps=max(3, min(20, args.steps)),
+                kda, torch, pcb.to(dev), pcb, dev, stream, reps=max(3, min(20, args.steps)),
                 sm_max_mhz=clk.get("sm_max_mhz") if isinstance(clk, dict) else None)
+            bwd["workload"] = pcb.name
+            if do_cpu:
+                bwd["cpu_oracle"] = cpu_baseline_backward(pcb)
         except (kda.KdaError, RuntimeError, AssertionError) as e:
             bwd = {"error": f"{type(e).__name__}: {e}"}
 
-    peaks, peak_kind = load_peaks()
-    hbm = peaks["hbm_gbs"]
-    tx = total * H
-    pb = prefill_bytes(tx, Np * H)
-    pf = prefill_flops(tx)
-    pre_avg = pre_sum / args.steps / 1e3  # s
-    dom_name, dom_s = kern["dominant"]
-    # roofline of the dominant prefill kernel: its share of the algorithmic bytes
-    dom_bytes = kern["bytes"][dom_name]
-    roof = {"kernel": dom_name, "bound": "hbm", "achieved": dom_bytes / dom_s / 1e9,
-            "peak": hbm, "unit": "GB/s", "frac": dom_bytes / dom_s / 1e9 / hbm,
-            "traffic": measured_traffic(dom_name, pc.name),
-            "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
-            "per_launch_us": dom_s * 1e6, "algorithmic_bytes_per_launch": dom_bytes}
-    dec_avg = dec_sum / args.steps / 1e3
-    db = decode_bytes(Nd * H)
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; distributions of the pages' configurations)",
-        "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": H, "dk": dk, "dv": dv,
-                   "chunk": C, "prefill_path": kern["path"], "decode_workload": dcase.name,
-                   "l2": "flushed (256 MiB write) before each leg",
+        "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "N": Np, "tokens": total,
+                   "H": H, "dk": dk, "dv": dv, "chunk": C, "prefill_path": kern["path"],
+                   "decode_workload": dcase.name, "decode_steps_per_step": dsteps,
+                   "l2": "inputs larger than L2; L2 also flushed (256 MiB write) before each "
+                         "prefill leg",
                    "parallelism": f"replicas x{world}"},
-        "prefill": {"value": value, "unit": "tokens/s", "ms_per_call": pre_avg * 1e3,
-                    "hbm_frac": pb / pre_avg / 1e9 / hbm,
-                    "tensor_frac": pf / pre_avg / 1e12 / peaks["bf16_tflops"],
-                    "algorithmic_bytes": pb, "paper_flops": pf,
-                    "kernels_us": {k: v * 1e6 for k, v in kern["times"].items()}},
-        "decode": {"value": dec_value, "unit": "tokens/s", "ms_per_step": dec_avg * 1e3,
-                   "roofline": {"bound": "hbm", "achieved": db / dec_avg / 1e9, "peak": hbm,
-                                "unit": "GB/s", "frac": db / dec_avg / 1e9 / hbm,
-                                "traffic": measured_traffic("decode", dcase.name),
-                                "algorithmic_bytes_per_launch": db}},
+        "prefill": prefill_entry,
+        "decode": decode_entry,
         "roofline": roof,
+        "configs": configs,
+        "parity": parity,
         "layer_steps": layer,
         "backward": bwd,
         "e2e": e2e,
-        "gpu_launches": args.steps * (kern["launches_per_call"] + 1),
+        "gpu_launches": args.steps * (kern["launches_per_call"] + dsteps),
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(pc, seconds=args.cpu_seconds)
-        if isinstance(bwd, dict) and "error" not in bwd:
-            bwd["cpu_oracle"] = cpu_baseline_backward(pc)
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
     return res
+
+
+def prefill_config_entry(kda, torch, pc, dev, stream, flush, peaks, peak_kind, reps, do_cpu,
+                         parity):
+    """One other prefill configuration: the default call timed alone (median of
+    `reps`, L2 flushed before each), its plan, kernel times and dominant-kernel
+    roofline, and (rank 0, one GPU) its parity and CPU-oracle baseline."""
+    P = pc.to(dev)
+    Bc, Tc = (1, P.total) if P.cu_seqlens is not None else (P.B, P.T)
+    ws = kda.alloc_workspace(P.total, P.N, P.H, P.dk, P.dv, P.chunk, "bf16", dev)
+    o = torch.empty_like(P.v)
+    hN = torch.empty(P.N, P.H, P.dk, P.dv, device=dev)
+    call = lambda: kda.kda_chunk_fwd(P.q, P.k, P.v, P.g, P.beta, P.initial_state,  # noqa: E731
+                                     P.cu_seqlens, Bc, Tc, P.N, P.H, P.dk, P.dv, P.chunk, "bf16",
+                                     o, hN, ws)
+    t = time_calls(torch, stream, flush, call, reps)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    kern = prefill_kernel_times(kda, P, ws, dev, stream, reps=reps)
+    e = prefill_summary(P, t, peaks)
+    e.update({"workload": pc.name, "prefill_path": kern["path"],
+              "kernels_us": {k: v * 1e6 for k, v in kern["times"].items()},
+              "roofline": prefill_roofline(kern, pc, peaks, peak_kind)})
+    if do_cpu:
+        o.fill_(float("nan"))
+        call()
+        torch.cuda.synchronize()
+        e["cpu_baseline"], parity[pc.name] = oracle_prefill_parity(pc, o, hN)
+    del P, ws, o, hN
+    torch.cuda.empty_cache()
+    return e
+
+
+def _parity_entry(x, ref):
+    """max |x - ref| / max |ref| and max |x - ref| / (|ref| + 1e-3 max |ref|)."""
+    import numpy as np
+    x = x.detach().to("cpu", dtype=__import__("torch").float64).numpy() \
+        if hasattr(x, "detach") else np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    d = np.abs(x - ref)
+    m = float(np.abs(ref).max(initial=0.0))
+    return {"max_abs_over_max_ref": float(d.max(initial=0.0)) / max(m, 1e-30),
+            "elementwise": float((d / (np.abs(ref) + 1e-3 * m)).max(initial=0.0)),
+            "finite": bool(np.isfinite(x).all())}
+
+
+def oracle_prefill_parity(pc, o, hN):
+    """The fp64 oracle (as it stands) on the whole prefill workload, on all host
+    cores, once: its time is the CPU baseline and its result the parity
+    reference of the GPU call's o and final state."""
+    import oracle
+    cores = oracle.max_threads()
+    t = time.perf_counter()
+    ro, rh = oracle.forward(pc.q, pc.k, pc.v, pc.g, pc.beta, pc.initial_state,
+                            cu_seqlens=pc.cu_host(), num_threads=cores)
+    el = time.perf_counter() - t
+    tol = 2e-2 if pc.dtype == "bf16" else 1e-4
+    par = {"o": _parity_entry(o, ro), "final_state": _parity_entry(hN, rh), "tolerance": tol,
+           "sample": "every sequence, head and token"}
+    par["pass"] = all(par[k]["max_abs_over_max_ref"] <= tol and par[k]["finite"]
+                      for k in ("o", "final_state"))
+    cpu = {"value": pc.total / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"whole workload ({pc.N} sequences, {pc.total} tokens x {pc.H} heads) "
+                     f"once, fp64 token recurrence, {el:.1f} s"}
+    return cpu, par
+
+
+def oracle_decode_parity(dcase, steps, outs, state, seqs=32):
+    """The fp64 oracle replays the first `seqs` sequences' `steps` decode steps
+    (all heads) as one recurrence per sequence; its time is the decode CPU
+    baseline, its outputs (every step) and final states the parity reference."""
+    import numpy as np
+    import torch
+
+    import oracle
+    cores = oracle.max_threads()
+    sched = [t % len(dcase.steps) for t in range(steps)]
+    H, dv = dcase.H, dcase.dv
+    seqs = min(seqs, dcase.N)
+    seq = {k: torch.stack([dcase.steps[i][k][:seqs] for i in sched], 1)
+           for k in ("q", "k", "v", "g", "beta")}
+    flat = {k: v.reshape(-1, *v.shape[2:]) for k, v in seq.items()}
+    cu = np.arange(0, (seqs + 1) * steps, steps, dtype=np.int32)
+    t = time.perf_counter()
+    ro, rs = oracle.forward(flat["q"], flat["k"], flat["v"], flat["g"], flat["beta"],
+                            dcase.state0[:seqs], cu_seqlens=cu, num_threads=cores)
+    el = time.perf_counter() - t
+    ro = ro.reshape(seqs, steps, H, dv).transpose(1, 0, 2, 3)
+    par = {"o": _parity_entry(outs[:, :seqs], ro), "state": _parity_entry(state[:seqs], rs),
+           "tolerance": 2e-2,
+           "sample": f"{seqs} of {dcase.N} sequences x {H} heads, all {steps} steps"}
+    par["pass"] = all(par[k]["max_abs_over_max_ref"] <= 2e-2 and par[k]["finite"]
+                      for k in ("o", "state"))
+    cpu = {"value": seqs * steps / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{seqs} sequences x {H} heads x {steps} steps, fp64 recurrence, "
+                     f"{el:.1f} s"}
+    return cpu, par
 
 
 def prefill_path(kda, total, Np, H, dk, dv, C, packed, dtype="bf16"):
     """The plan kda_chunk_fwd runs for this problem (the library's own answer):
-    'simt', 'fused', 'split' or 'overlap' (see include/kda.h)."""
+    'simt', 'split' or 'overlap' (see include/kda.h)."""
     return kda.PLAN_NAMES[kda.kda_chunk_fwd_plan(total, Np, H, dk, dv, C, dtype, packed)]
 
 
@@ -342,7 +521,7 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     """Device times of the prefill kernels, each from CUDA events around its own
     call on the launching stream, L2 flushed before each.  CUDA-core path: the
     four step calls (a1..a4); split plan: kda_chunk_split_intra and
-    kda_chunk_split_chain; fused plan: the one kernel (the whole call).  Each
+    kda_chunk_split_chain; overlap plan: the one co-scheduled launch.  Each
     call's time includes the chunk-table kernel that starts it, where it has
     one.  Algorithmic bytes are the pages' inputs and outputs that each kernel
     must move; the split plan's hand-over through the workspace is overhead."""
@@ -377,8 +556,8 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
     if path != "simt":
         o = torch.empty_like(P.v)
         hN = torch.empty(Np, H, dk, dv, device=dev)
-        if path in ("fused", "overlap"):
-            name = "chunk_fwd_tc" if path == "fused" else "chunk_fwd_overlap"
+        if path == "overlap":
+            name = "chunk_fwd_overlap"
             calls = {name: lambda: kda.kda_chunk_fwd(
                 P.q, P.k, P.v, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc, Tc, Np, H, dk,
                 dv, C, "bf16", o, hN, ws)}
@@ -601,45 +780,25 @@ def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
 
 # ------------------------------------------------------------- cpu baseline
 
-def cpu_baseline(pc, seconds=15.0, heads=None):
+def cpu_baseline(pc, heads=1, tokens=None):
     """The fp64 oracle (as it stands) on the host cores, on a bounded sample of
-    the prefill workload.  With `heads` given: the first sequence, first
-    `heads` heads, once.  Otherwise the whole workload (all sequences and
-    heads), repeated until about `seconds` of CPU time have run.  Reported as
-    tokens/s of the full workload (head-tokens/s / H)."""
+    the prefill workload: the first sequence's first `tokens` tokens (all of
+    them when None) on its first `heads` heads, once.  Reported as tokens/s of
+    the full workload (head-tokens/s / H)."""
     import oracle
     cores = oracle.max_threads()
     H = pc.H
-    if heads is not None:
-        T = pc.T
-        t = time.perf_counter()
-        oracle.forward(pc.q[:T, :heads], pc.k[:T, :heads], pc.v[:T, :heads], pc.g[:T, :heads],
-                       pc.beta[:T, :heads], pc.initial_state[:1, :heads], num_threads=cores)
-        el = time.perf_counter() - t
-        return {"value": T * heads / el / H, "unit": "tokens/s", "cores": cores,
-                "kind": "oracle", "sample": f"1 sequence x {T} tokens x {heads} of {H} heads, "
-                                            f"fp64 token recurrence, {el:.1f} s"}
-    cu = pc.cu_host()
-    reps, el = 0, 0.0
-    while el < seconds:
-        t = time.perf_counter()
-        oracle.forward(pc.q, pc.k, pc.v, pc.g, pc.beta, pc.initial_state, cu_seqlens=cu,
-                       num_threads=cores)
-        el += time.perf_counter() - t
-        reps += 1
-    # one thread, on the first sequence's first two heads
-    T1, h1 = int(cu[1]) - int(cu[0]), min(2, H)
+    T = int(pc.cu_host()[1])
+    if tokens is not None:
+        T = min(T, tokens)
+    h0 = None if pc.initial_state is None else pc.initial_state[:1, :heads]
     t = time.perf_counter()
-    oracle.forward(pc.q[:T1, :h1], pc.k[:T1, :h1], pc.v[:T1, :h1], pc.g[:T1, :h1],
-                   pc.beta[:T1, :h1], pc.initial_state[:1, :h1], num_threads=1)
-    el1 = time.perf_counter() - t
-    return {"value": pc.total * reps / el, "unit": "tokens/s", "cores": cores,
-            "kind": "oracle",
-            "sample": f"whole prefill workload ({pc.N} x {pc.T} tokens x {H} heads) x {reps} "
-                      f"repetitions, fp64 token recurrence, {el:.1f} s",
-            "single_thread": {"value": T1 * h1 / el1 / H, "unit": "tokens/s",
-                              "sample": f"1 sequence x {T1} tokens x {h1} of {H} heads, "
-                                        f"1 thread, {el1:.2f} s"}}
+    oracle.forward(pc.q[:T, :heads], pc.k[:T, :heads], pc.v[:T, :heads], pc.g[:T, :heads],
+                   pc.beta[:T, :heads], h0, num_threads=cores)
+    el = time.perf_counter() - t
+    return {"value": T * heads / el / H, "unit": "tokens/s", "cores": min(cores, heads),
+            "kind": "oracle", "sample": f"1 sequence x {T} tokens x {heads} of {H} heads, "
+                                        f"fp64 token recurrence, {el:.2f} s"}
 
 
 def cpu_baseline_backward(pc, tokens=256):
@@ -666,16 +825,20 @@ def cpu_baseline_backward(pc, tokens=256):
 
 
 def run_reference(args, rank, world):
+    """The oracle as it stands on the host cores, on the headline prefill
+    workload's configuration: each step one bounded sample (the first
+    sequence's tokens on `--ref-heads` heads, one thread per head)."""
     if rank != 0:
         return None
     from gated_delta_rule_124_b200 import workloads as wl
-    pc = wl.prefill_config(1)
+    pc = prefill_case(wl, args)
+    heads = max(1, min(pc.H, args.ref_heads))
     for _ in range(args.warmup):
-        cpu_baseline(pc, heads=1)
+        cpu_baseline(pc, heads=1, tokens=256)
     vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        r = cpu_baseline(pc, heads=max(1, min(pc.H, args.ref_heads)))
+        r = cpu_baseline(pc, heads=heads)
         vals.append(r["value"])
     el = time.perf_counter() - t0
     v = statistics.median(vals)
@@ -683,8 +846,9 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "H": pc.H, "dk": pc.dk,
-                       "dv": pc.dv, "chunk": pc.chunk},
+            "config": {"workload": pc.name, "B": pc.B, "T": pc.T, "N": pc.N,
+                       "tokens": pc.total, "H": pc.H, "dk": pc.dk, "dv": pc.dv,
+                       "chunk": pc.chunk},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": r["cores"],
                              "kind": "oracle", "sample": r["sample"]},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -700,7 +864,7 @@ def run_backward_only(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     kda.load()
-    pc = prefill_case(wl, args)
+    pc = wl.prefill_config(args.backward_config)
     P = pc.to(dev)
     bwd = backward_times(kda, torch, P, pc, dev, torch.cuda.current_stream(),
                          reps=max(3, min(20, args.steps)))
@@ -713,20 +877,27 @@ def run_backward_only(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-heads", type=int, default=4)
+    ap.add_argument("--decode-steps", type=int, default=1000,
+                    help="decode steps per bench step (the decode workload's schedule)")
+    ap.add_argument("--decode-parity-seqs", type=int, default=32,
+                    help="decode sequences the oracle replays for the parity entry")
+    ap.add_argument("--only-headline", action="store_true",
+                    help="skip the other prefill configurations (for profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward timing beside the step")
+    ap.add_argument("--backward-config", type=int, default=1, choices=[1, 2, 3],
+                    help="workload of --backward-only (default: B=2 x T=2048)")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only kda_chunk_bwd on the prefill workload and print its "
                          "entry (for profiling the backward kernels alone)")
-    ap.add_argument("--prefill-config", type=int, default=1, choices=[1, 2, 3],
-                    help="prefill workload: 1 = B=2 x T=2048 (default), 2 = B=1 x T=65536, "
-                         "3 = 16 packed sequences of U[1024,16384] tokens")
+    ap.add_argument("--prefill-config", type=int, default=3, choices=[1, 2, 3],
+                    help="prefill workload: 3 = 16 packed sequences of U[1024,16384] tokens "
+                         "(default, the largest), 1 = B=2 x T=2048, 2 = B=1 x T=65536")
     ap.add_argument("--prefill-shape", default=None, metavar="B,T,H",
                     help="instead of --prefill-config: B sequences of T tokens, H heads "
                          "(d = 128, chunk 64, bf16, the default configuration's distributions)")

@@ -57,18 +57,48 @@ def _normal(seed: int, tid: int, n: int, mu: float = 0.0, sigma: float = 1.0) ->
     return out
 
 
+def _blockwise(f, x: np.ndarray, rows: int = 1) -> np.ndarray:
+    """f applied to x in blocks of whole rows (the last axis when rows > 1),
+    on a thread pool; the same values as f(x) in one piece."""
+    out = np.empty(x.shape, dtype=np.float32)
+    if rows > 1:
+        xf, of = x.reshape(-1, rows), out.reshape(-1, rows)
+    else:
+        xf, of = x.reshape(-1), out.reshape(-1)
+    n = xf.shape[0]
+    step = max(1, _BLOCK // max(1, rows))
+    nblk = (n + step - 1) // step
+
+    def blk(i):
+        lo, hi = i * step, min(n, (i + 1) * step)
+        of[lo:hi] = f(xf[lo:hi])
+
+    if nblk <= 1:
+        for i in range(nblk):
+            blk(i)
+    else:
+        with ThreadPoolExecutor(min(_THREADS, nblk)) as ex:
+            list(ex.map(blk, range(nblk)))
+    return out
+
+
 def _l2norm_rows(x: np.ndarray) -> np.ndarray:
-    n = np.sqrt((x.astype(np.float64) ** 2).sum(-1, keepdims=True))
-    return (x / np.maximum(n, 1e-30)).astype(np.float32)
+    def f(b):
+        n = np.sqrt((b.astype(np.float64) ** 2).sum(-1, keepdims=True))
+        return (b / np.maximum(n, 1e-30)).astype(np.float32)
+    return _blockwise(f, x, rows=x.shape[-1])
 
 
 def _neg_softplus(x: np.ndarray) -> np.ndarray:
-    x64 = x.astype(np.float64)
-    return (-(np.maximum(x64, 0.0) + np.log1p(np.exp(-np.abs(x64))))).astype(np.float32)
+    def f(b):
+        b64 = b.astype(np.float64)
+        return (-(np.maximum(b64, 0.0) + np.log1p(np.exp(-np.abs(b64))))).astype(np.float32)
+    return _blockwise(f, x)
 
 
 def _sigmoid(x: np.ndarray) -> np.ndarray:
-    return (1.0 / (1.0 + np.exp(-x.astype(np.float64)))).astype(np.float32)
+    return _blockwise(lambda b: (1.0 / (1.0 + np.exp(-b.astype(np.float64)))).astype(np.float32),
+                      x)
 
 
 _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}

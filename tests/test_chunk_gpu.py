@@ -7,7 +7,7 @@ import torch
 import gated_delta_rule_124_b200 as kda
 from gated_delta_rule_124_b200 import workloads as wl
 from oracle import chunkwise
-from tests.helpers import oracle_prefill, rel_err, tol_for
+from tests.helpers import oracle_prefill, record, rel_err, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -36,39 +36,46 @@ def run_fwd(case, final=True, plan=None):
     return o, hN
 
 
-def check_case(case, heads=None, plan=None):
+def check_case(case, heads=None, plan=None, report=False):
+    """The case against the fp64 oracle (all heads, or the given ones); with
+    `report`, the errors go to the parity report printed after the run."""
     o, hN = run_fwd(case, plan=plan)
     ro, rh = oracle_prefill(case, heads)
     sl = slice(None) if heads is None else list(heads)
     tol = tol_for(case.dtype)
-    eo = rel_err(o[:, sl], ro)
-    eh = rel_err(hN[:, sl], rh)
+    if report:
+        eo = record(case.name, "o", o[:, sl], ro)
+        eh = record(case.name, "final_state", hN[:, sl], rh)
+    else:
+        eo = rel_err(o[:, sl], ro)
+        eh = rel_err(hN[:, sl], rh)
     assert eo <= tol and eh <= tol, (case.name, eo, eh)
     return eo, eh
 
 
 # ---------------------------------------------------------------- configs
 
+# Every configuration at full extent: all sequences, heads and tokens against
+# the fp64 oracle (on all host cores), in the launch configuration the
+# benchmark times (the default plan of kda_chunk_fwd).
+
 def test_config0_tiny_fp32():
-    case = wl.prefill_config(0)
-    check_case(case)
+    check_case(wl.prefill_config(0), report=True)
 
 
 def test_config1_all_heads():
-    case = wl.prefill_config(1)
-    check_case(case)
+    check_case(wl.prefill_config(1), report=True)
 
 
-def test_config2_long_sampled_heads():
-    """T = 65536: all tokens of three heads (first, middle, last) against the
-    oracle; the chunk chain is 1024 chunks long."""
-    case = wl.prefill_config(2)
-    check_case(case, heads=[0, 17, 31])
+def test_config2_long_all_heads():
+    """T = 65536, all 32 heads: each chunk chain is 1024 chunks long, with the
+    S operand rounded to bf16 at every chunk."""
+    check_case(wl.prefill_config(2), report=True)
 
 
-def test_config3_varlen_sampled_heads():
-    case = wl.prefill_config(3)
-    check_case(case, heads=[0, 31])
+def test_config3_varlen_all_heads():
+    """16 packed sequences of U[1024, 16384] tokens, all 32 heads."""
+    check_case(wl.prefill_config(3), report=True)
 
 
 # ----------------------------------------------------- shapes and edge cases

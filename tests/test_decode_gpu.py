@@ -6,7 +6,7 @@ import torch
 import gated_delta_rule_124_b200 as kda
 import oracle
 from gated_delta_rule_124_b200 import workloads as wl
-from tests.helpers import rel_err, tol_for
+from tests.helpers import ErrAccum, record, rel_err, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -46,17 +46,42 @@ def test_decode_small_shapes(dtype, dk, dv):
     assert rel_err(state, r_state) <= tol
 
 
-def test_decode_full_size_config_few_steps():
-    """N=256, H=32, 128 x 128 fp32 state: every (sequence, head) checked over
-    16 steps of the 8-set schedule (the oracle replays the same schedule)."""
+def test_decode_full_config_all_steps():
+    """The decode configuration at full extent: N=256 sequences x H=32 heads,
+    128 x 128 fp32 states, all 1000 steps of the 8-set schedule; o of every
+    step and the final state of every (sequence, head) against the fp64
+    oracle.  The oracle replays each sequence's 1000 steps as one 1000-token
+    recurrence (a decode step is one step of that recurrence), eight
+    sequences at a time."""
     c = wl.DECODE_CONFIG
     case = wl.decode_config()
-    steps = 16
-    outs, state = _run(case, steps)
-    r_outs, r_state = _oracle(case, steps)
-    errs = [rel_err(o, ro) for o, ro in zip(outs, r_outs)]
-    assert max(errs) <= tol_for(c["dtype"]), errs
-    assert rel_err(state, r_state) <= 1e-4  # fp32 state, fp32 arithmetic
+    steps, N, H, d = c["steps"], case.N, case.H, case.dk
+    dev = "cuda"
+    state = case.state0.to(dev).contiguous()
+    dsets = [{k: v.to(dev).contiguous() for k, v in s.items()} for s in case.steps]
+    o_all = torch.empty(steps, N, H, d, dtype=torch.bfloat16, device=dev)
+    for t in range(steps):
+        s = dsets[t % len(dsets)]
+        kda.decode_step(s["q"], s["k"], s["v"], s["g"], s["beta"], state, o=o_all[t])
+    torch.cuda.synchronize()
+    acc_o, acc_s = ErrAccum(), ErrAccum()
+    sched = [t % len(case.steps) for t in range(steps)]
+    G = 8
+    for n0 in range(0, N, G):
+        n1 = min(N, n0 + G)
+        seq = {k: torch.stack([case.steps[i][k][n0:n1] for i in sched], 1)
+               for k in ("q", "k", "v", "g", "beta")}  # [n, steps, ...]
+        flat = {k: v.reshape(-1, *v.shape[2:]) for k, v in seq.items()}
+        cu = np.arange(0, (n1 - n0 + 1) * steps, steps, dtype=np.int32)
+        ro, rs = oracle.forward(flat["q"], flat["k"], flat["v"], flat["g"], flat["beta"],
+                                case.state0[n0:n1], cu_seqlens=cu)
+        ro = ro.reshape(n1 - n0, steps, H, d).transpose(1, 0, 2, 3)
+        acc_o.add(o_all[:, n0:n1], ro)
+        acc_s.add(state[n0:n1], rs)
+    eo = record(case.name, "o (all steps)", acc=acc_o)
+    es = record(case.name, "state", acc=acc_s)
+    assert eo <= tol_for(c["dtype"]), eo
+    assert es <= tol_for(c["dtype"]), es
 
 
 def test_decode_n_zero_is_noop():
