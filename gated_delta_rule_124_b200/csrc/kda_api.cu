@@ -317,6 +317,41 @@ kda_status_t kda_chunk_fwd_with_plan(int plan, const void* q, const void* k, con
                         chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
 }
 
+kda_status_t kda_test_overlap_flag_timeout(const void* q, const void* k, const void* v,
+                                           const float* g, const float* beta,
+                                           const float* initial_state,
+                                           const int32_t* cu_seqlens, int B, int T,
+                                           int num_seqs, int H, void* o, float* final_state,
+                                           void* workspace, size_t workspace_bytes,
+                                           int withheld_chunk, int withheld_head,
+                                           unsigned long long flag_wait_ns, void* stream) {
+    Prefill p;
+    kda_status_t s = check_prefill_shape(cu_seqlens, B, T, num_seqs, H, 128, 128, 64,
+                                         KDA_DTYPE_BF16, &p);
+    if (s != KDA_OK) return s;
+    if (!path_applies(Path::Overlap, p.N, H, 128, 128, 64, KDA_DTYPE_BF16))
+        return KDA_ERR_UNSUPPORTED;
+    const int maxc = kda::max_chunks(p.total, p.N, 64);
+    if (withheld_chunk < 0 || withheld_chunk >= maxc || withheld_head < 0 ||
+        withheld_head >= H || flag_wait_ns == 0 || flag_wait_ns > 2000000000ull)
+        return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : {q, k, v, (const void*)g, (const void*)beta, (const void*)o})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    Workspace w;
+    s = check_ws(workspace, workspace_bytes, p, H, 128, 128, 64, Path::Overlap, &w);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, 64, maxc, st);
+    if (s != KDA_OK) return s;
+    if (p.total == 0) return KDA_OK;
+    return from_cuda(kda::launch_chunk_fwd_overlap(
+        q, k, v, g, beta, initial_state, cu_seqlens, T, p.N, H, w.chunk_info, maxc,
+        w.chunk_start, w.status, w.blobs, w.flags, o, final_state, st,
+        (long long)withheld_chunk * H + withheld_head, flag_wait_ns));
+}
+
 // ------------------------------------------------- one step per call (a1-a4)
 
 #define KDA_PREFILL_PROLOGUE(...)                                                   \

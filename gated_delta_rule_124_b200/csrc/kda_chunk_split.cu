@@ -141,6 +141,9 @@ struct Params {
     const uint32_t* rounds;  // largest number of chunks of one sequence
     uint32_t* flags;         // [slot, head]: set once that blob is complete
     const float* gh;         // head-uniform gate [total, H] (kScalar)
+    // (testing the bounded-wait error path only) the flag index slot * H + h
+    // that is never released, or -1
+    long long withheld;
 };
 
 // One worker (CTA) of the intra-chunk kernel.  Items are (chunk slot, head)
@@ -615,7 +618,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             if (tid == NTI - 32) {  // idle in this phase
                 // the previous item's blob is complete (all of its writes came
                 // before this item's first barrier): release it to its chain
-                if (kOverlap && flag_pending >= 0) {
+                if (kOverlap && flag_pending >= 0 && flag_pending != p.withheld) {
                     fence_proxy_async_global();
                     flag_release(p.flags + flag_pending, 1u);
                 }
@@ -728,7 +731,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     }
     tc_fence_before();
     group_sync(bar, NTI);
-    if (kOverlap && flag_pending >= 0 && tid == NTI - 32) {
+    if (kOverlap && flag_pending >= 0 && flag_pending != p.withheld && tid == NTI - 32) {
         fence_proxy_async_global();
         flag_release(p.flags + flag_pending, 1u);
     }
@@ -805,6 +808,7 @@ struct Params {
     __nv_bfloat16* o;
     float* hN;
     const uint32_t* flags;  // co-scheduled with the intra kernel: blob ready flags
+    uint64_t flag_wait_ns;  // bound of the watcher's wait on one flag
 };
 
 // One chain CTA: (sequence, head) `chain_id`, value columns [64 half, +64).
@@ -1113,7 +1117,7 @@ __device__ __forceinline__ void watch(const Params& p, uint8_t* sm_chain, int ch
     for (int n = 0; n < nch; ++n) {
         const uint64_t t0 = global_timer_ns();
         while (flag_acquire(f + (size_t)n * p.H) == 0u) {
-            if (status_bad(p.status) || global_timer_ns() - t0 > kWaitNs) {
+            if (status_bad(p.status) || global_timer_ns() - t0 > p.flag_wait_ns) {
                 smem_release(s_rdy, -1);
                 return;
             }
@@ -1324,7 +1328,8 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
                                      const int32_t* cu_seqlens, int T, int N, int H,
                                      const int4* chunk_info, int maxc, const int* chunk_start,
                                      uint32_t* status, void* blobs, uint32_t* flags, void* o,
-                                     float* hN, cudaStream_t st) {
+                                     float* hN, cudaStream_t st, long long withheld_flag,
+                                     unsigned long long flag_wait_ns) {
     const int total = cu_seqlens ? T : N * T;
     if (total == 0)
         return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN,
@@ -1344,10 +1349,12 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
     cudaError_t e = cudaMemsetAsync(flags, 0, sizeof(uint32_t) * (size_t)maxc * H, st);
     if (e != cudaSuccess) return e;
     uint8_t* bl = static_cast<uint8_t*>(blobs);
-    const intra::Params pi{beta, chunk_info, maxc, H, status, status, bl,
-                           N, chunk_start, status + 1, flags};
-    const chain::Params pc{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
-                           (__nv_bfloat16*)o, hN, flags};
+    intra::Params pi{beta, chunk_info, maxc, H, status, status, bl,
+                     N, chunk_start, status + 1, flags};
+    pi.withheld = withheld_flag;
+    chain::Params pc{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
+                     (__nv_bfloat16*)o, hN, flags};
+    pc.flag_wait_ns = flag_wait_ns ? flag_wait_ns : kWaitNs;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(NTO);

@@ -33,6 +33,9 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
                                const void* blobs, void* o, float* hN, cudaStream_t st);
 // The two kernels co-scheduled in one cooperative launch (chains wait for the
 // blobs of their chunks through `flags`, one uint32 per (chunk slot, head)).
+// withheld_flag >= 0 (testing the bounded-wait error path only): the flag of
+// that (slot * H + head) is never released; flag_wait_ns != 0 bounds the
+// chains' wait on one flag (default 2 s).
 // overlap_grid() is its grid size, or 0 when the launch does not apply.
 int overlap_grid(int N, int H);
 cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v, const float* g,
@@ -40,6 +43,7 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
                                      const int32_t* cu_seqlens, int T, int N, int H,
                                      const int4* chunk_info, int maxc, const int* chunk_start,
                                      uint32_t* status, void* blobs, uint32_t* flags, void* o,
-                                     float* hN, cudaStream_t st);
+                                     float* hN, cudaStream_t st, long long withheld_flag = -1,
+                                     unsigned long long flag_wait_ns = 0);
 
 }  // namespace kda

@@ -44,6 +44,7 @@ EXPORTS = (
     "kda_gdn_decode_step", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
     "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd", "kda_qkv_conv_norm_step",
     "kda_chunk_fwd_with_plan", "kda_chunk_fwd_plan_workspace_size",
+    "kda_test_overlap_flag_timeout",
 )
 
 
@@ -73,6 +74,8 @@ _SIGS = {
     "kda_chunk_fwd_plan": ([_i] * 8, _i),
     "kda_chunk_fwd_with_plan": ([_i] + [_vp] * 7 + [_i] * 8 + [_vp, _vp, _vp, _sz, _vp], _i),
     "kda_chunk_fwd_plan_workspace_size": ([_i] * 8, _sz),
+    "kda_test_overlap_flag_timeout": ([_vp] * 7 + [_i] * 4 + [_vp] * 3 + [_sz, _i, _i,
+                                      ctypes.c_ulonglong, _vp], _i),
     "kda_qkv_conv_norm": ([_vp] * 7 + [_i] * 7 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_output_norm_gate": ([_vp] * 3 + [_i] * 4 + [ctypes.c_float] + [_vp] * 2, _i),
     "kda_gdn_chunk_fwd_workspace_size": ([_i] * 7, _sz),
@@ -238,6 +241,24 @@ def kda_chunk_fwd_with_plan(plan, q, k, v, g, beta, initial_state, cu_seqlens, B
                                         dk, dv, chunk, dtype_code(dtype), _p(o),
                                         _p(final_state), _p(workspace), wb, _stream(stream))
     return _ret(st, "kda_chunk_fwd_with_plan", check)
+
+
+def kda_test_overlap_flag_timeout(q, k, v, g, beta, initial_state, cu_seqlens, B, T, num_seqs,
+                                  H, o, final_state, workspace, withheld_chunk, withheld_head,
+                                  flag_wait_ns, workspace_bytes=None, stream=None,
+                                  check=True) -> int:
+    """The overlap plan with one chunk's ready flag withheld and the chains'
+    flag waits bounded by flag_wait_ns: exercises the bounded-wait error path
+    (kda_get_device_status then reports KDA_ERR_TIMEOUT).  Testing only."""
+    _check("kda_test_overlap_flag_timeout", "bf16", typed=(q, k, v, o),
+           f32=(g, beta, initial_state, final_state), i32=(cu_seqlens,), raw=(workspace,))
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_test_overlap_flag_timeout(_p(q), _p(k), _p(v), _p(g), _p(beta),
+                                              _p(initial_state), _p(cu_seqlens), B, T, num_seqs,
+                                              H, _p(o), _p(final_state), _p(workspace), wb,
+                                              withheld_chunk, withheld_head, flag_wait_ns,
+                                              _stream(stream))
+    return _ret(st, "kda_test_overlap_flag_timeout", check)
 
 
 def kda_chunk_gate_cumsum(g, cu_seqlens, B, T, num_seqs, H, dk, chunk, G, workspace,

@@ -428,6 +428,31 @@ kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
                                    int dk, int dv, int chunk, kda_dtype_t dtype, void* o,
                                    float* final_state, void* stream);
 
+/* ------------------------------------------------- testing the error path
+ * kda_test_overlap_flag_timeout: the overlap plan of kda_chunk_fwd (bf16,
+ * dk = dv = 128, chunk 64; KDA_ERR_UNSUPPORTED where that plan does not apply)
+ * with the ready flag of global chunk slot `withheld_chunk` of head
+ * `withheld_head` never set, and every chain's wait on one flag bounded by
+ * flag_wait_ns (1 ns .. 2 s) instead of 2 s.  It exists to exercise the
+ * device-side bounded-wait error path without any fault: the chain that needs
+ * the withheld chunk gives up after flag_wait_ns, waits for its own copies and
+ * products in flight, records KDA_ERR_TIMEOUT in the status word and returns;
+ * every other chain and every intra-chunk unit completes (none of them waits
+ * on that flag).  kda_get_device_status(workspace) then returns
+ * KDA_ERR_TIMEOUT; outputs are unspecified; the next prefill call on the same
+ * workspace starts clean.  Arguments otherwise as kda_chunk_fwd_with_plan with
+ * KDA_PLAN_OVERLAP (workspace: kda_chunk_fwd_plan_workspace_size of that plan).
+ * Not a computation: no caller outside the tests needs it.
+ */
+kda_status_t kda_test_overlap_flag_timeout(const void* q, const void* k, const void* v,
+                                           const float* g, const float* beta,
+                                           const float* initial_state,
+                                           const int32_t* cu_seqlens, int B, int T,
+                                           int num_seqs, int H, void* o, float* final_state,
+                                           void* workspace, size_t workspace_bytes,
+                                           int withheld_chunk, int withheld_head,
+                                           unsigned long long flag_wait_ns, void* stream);
+
 /* ------------------------------------------------------------------ status
  * Synchronises `stream`, then reads the device status word kept at the start
  * of `workspace`.  Every prefill call (kda_chunk_fwd and the step calls)

@@ -380,3 +380,39 @@ def test_split_chain_keeps_the_intra_status():
     kda.kda_chunk_split_intra(c.q, c.k, c.g, c.beta, *args, ws)
     kda.kda_chunk_split_chain(c.v, None, *args, o, None, ws)
     assert kda.kda_get_device_status(ws) == kda.KDA_ERR_BAD_SEQLENS
+
+
+def test_bounded_wait_reports_timeout_and_next_call_is_clean():
+    """The device-side error path, without any fault: the overlap plan with
+    one chunk's ready flag withheld and the chains' flag waits bounded by
+    10 ms.  The chain that needs that chunk gives up, drains its own copies
+    and products and records KDA_ERR_TIMEOUT; the next call on the same
+    workspace reports KDA_OK and matches the oracle."""
+    case = wl.make_prefill(313, [64 * 6 + 5], H=2, dk=128, dv=128, chunk=64, dtype="bf16")
+    c = case.to("cuda")
+    n = kda.kda_chunk_fwd_plan_workspace_size("overlap", c.total, 1, 2, 128, 128, 64, "bf16")
+    assert n > 0
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(c.v)
+    hN = torch.empty(1, 2, 128, 128, device="cuda")
+    kda.kda_test_overlap_flag_timeout(c.q, c.k, c.v, c.g, c.beta, c.initial_state, None, 1,
+                                      c.total, 1, 2, o, hN, ws, withheld_chunk=2,
+                                      withheld_head=1, flag_wait_ns=10_000_000)
+    assert kda.kda_get_device_status(ws) == kda.KDA_ERR_TIMEOUT
+    kda.kda_chunk_fwd_with_plan("overlap", c.q, c.k, c.v, c.g, c.beta, c.initial_state, None, 1,
+                                c.total, 1, 2, 128, 128, 64, "bf16", o, hN, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    ro, rh = oracle_prefill(case)
+    assert rel_err(o, ro) <= tol_for("bf16") and rel_err(hN, rh) <= tol_for("bf16")
+
+
+def test_timeout_hook_rejects_bad_arguments():
+    case = wl.make_prefill(314, [200], H=2, dk=128, dv=128, chunk=64, dtype="bf16").to("cuda")
+    n = kda.kda_chunk_fwd_plan_workspace_size("overlap", case.total, 1, 2, 128, 128, 64, "bf16")
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(case.v)
+    for chunk, head, wait in ((99, 0, 10_000), (0, 2, 10_000), (0, 0, 0), (0, 0, 3 * 10**9)):
+        st = kda.kda_test_overlap_flag_timeout(case.q, case.k, case.v, case.g, case.beta, None,
+                                               None, 1, case.total, 1, 2, o, None, ws, chunk,
+                                               head, wait, check=False)
+        assert st == kda.KDA_ERR_INVALID_ARG, (chunk, head, wait)
