@@ -685,6 +685,30 @@ kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* 
                                            static_cast<cudaStream_t>(stream)));
 }
 
+kda_status_t kda_layer_decode_step(const void* xq, const void* xk, const void* xv,
+                                  const float* wq, const float* wk, const float* wv,
+                                  void* conv_q, void* conv_k, void* conv_v, const float* g,
+                                  const float* beta, float* state, const void* gate,
+                                  const float* w_norm, int N, int H, int dk, int dv,
+                                  kda_dtype_t dtype, float l2_eps, float rms_eps, void* y,
+                                  void* stream) {
+    if (N < 0 || H < 1 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if ((long long)N * H > 0x3fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!(l2_eps > 0.f) || !(l2_eps < 1e30f) || !(rms_eps > 0.f) || !(rms_eps < 1e30f))
+        return KDA_ERR_INVALID_ARG;
+    if (N == 0) return KDA_OK;
+    for (const void* ptr : std::initializer_list<const void*>{
+             xq, xk, xv, (const void*)wq, (const void*)wk, (const void*)wv, conv_q, conv_k,
+             conv_v, (const void*)g, (const void*)beta, (const void*)state, gate,
+             (const void*)w_norm, y})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_layer_decode(xq, xk, xv, wq, wk, wv, conv_q, conv_k, conv_v, g,
+                                              beta, state, gate, w_norm, N, H, dk, dv, dtype,
+                                              l2_eps, rms_eps, y,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 // ----------------------------------------------------------------- status
 
 kda_status_t kda_get_device_status(void* workspace, void* stream) {

@@ -158,6 +158,12 @@ cudaError_t launch_qkv_conv_step(const void* const x[3], const float* const w[3]
                                  int H, float eps, kda_dtype_t dt, cudaStream_t st);
 cudaError_t launch_norm_gate(const void* o, const void* gate, const float* w, int total, int H,
                              int d, float eps, kda_dtype_t dt, void* y, cudaStream_t st);
+cudaError_t launch_layer_decode(const void* xq, const void* xk, const void* xv, const float* wq,
+                                const float* wk, const float* wv, void* conv_q, void* conv_k,
+                                void* conv_v, const float* g, const float* beta, float* state,
+                                const void* gate, const float* w_norm, int N, int H, int dk,
+                                int dv, kda_dtype_t dt, float l2_eps, float rms_eps, void* y,
+                                cudaStream_t st);
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, float* state, void* o, int N, int H, int dk,
                           int dv, kda_dtype_t dt, cudaStream_t st, bool head_gate = false);

@@ -1,6 +1,6 @@
 // Device helpers shared by the tensor-core prefill kernels (internal to libkda):
 // fp32 64 x 64 matrix indexing, bf16 packing, swizzled tile access, and the
-// warp-level TF32 products used by the blocked triangular inverse.
+// warp-level TF32 products and block steps of the triangular inverse.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -39,6 +39,18 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
         x[2 * i + 1] = f.y;
     }
 }
+__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
+    return make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+}
+__device__ __forceinline__ void unpack4(uint2 u, float (&x)[4]) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
 __device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
     *reinterpret_cast<float4*>(x) = *reinterpret_cast<const float4*>(p);
     *reinterpret_cast<float4*>(x + 4) = *reinterpret_cast<const float4*>(p + 4);
@@ -68,77 +80,104 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Off-diagonal blocks of T at distance DIST:
-//   T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ,   I = J + DIST,  J = 0 .. 3 - DIST,
-// one warp per block J.  Fragments (m16n8k8, tf32): lane = 4 g + t;
-// A: (g, t), (g+8, t), (g, t+4), (g+8, t+4); B: (t, g), (t+4, g);
-// C: (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
-// Ends with a barrier over the thread group: `bar_id` 0 = the whole CTA,
-// otherwise named barrier `bar_id` over `nthreads` threads.
-template <int DIST>
-__device__ __forceinline__ void offdiag_level(const float* Af, float* Tf, float* Ms, int warp,
-                                              int lane, uint32_t bar_id = 0,
-                                              uint32_t nthreads = 0) {
-    constexpr int NB = 4 - DIST;
-    if (warp < NB) {
-        const int J = warp, I = J + DIST, g = lane >> 2, t = lane & 3;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+// The off-diagonal blocks of T = (I + A)^{-1} (A strictly lower, 4 x 4 blocks
+// of 16 x 16, the diagonal blocks T_II already inverted), by the 2 x 2 block
+// inverse applied twice:
+//   inverse_pairs:      T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
+//                       (warps 0 and 1; M = A_IJ T_JJ through the warp's
+//                       16 x 16 scratch, then -T_II M)
+//   inverse_lower_left: the 32 x 32 block [T_20 T_21; T_30 T_31] =
+//                       -T_hi (A_ll T_lo), T_lo = [T_00 0; T_10 T_11],
+//                       T_hi = [T_22 0; T_32 T_33]: warp w (0-3) owns tile
+//                       (i, j) = (2 + w / 2, w % 2), first M_ij = sum_k A_ik T_kj
+//                       (k = j..1) into scratch tile w, then, after a named
+//                       barrier of the four warps, T_ij = -sum_k T_ik M_kj
+//                       (k = 2..i).
+// 16 x 16 tiles on the warp-level TF32 products above (fragments as there).
+// acc[nt] += X[16 xi.., 16 xk..] * Y[16 xk.., 16 yj..], X and Y in the a_idx
+// layout.
+__device__ __forceinline__ void blk_mma(float (&acc)[2][4], const float* X, int xi, int xk,
+                                        const float* Y, int yj, int g, int t) {
 #pragma unroll
-        for (int kk = 0; kk < DIST; ++kk) {
-            const int K = J + kk;
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                const int c0 = 16 * K + 8 * ks + t;
-                const uint32_t a[4] = {to_tf32(Af[a_idx(16 * I + g, c0)]),
-                                       to_tf32(Af[a_idx(16 * I + g + 8, c0)]),
-                                       to_tf32(Af[a_idx(16 * I + g, c0 + 4)]),
-                                       to_tf32(Af[a_idx(16 * I + g + 8, c0 + 4)])};
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int col = 16 * J + 8 * nt + g;
-                    const uint32_t b[2] = {to_tf32(Tf[t_idx(c0, col)]),
-                                           to_tf32(Tf[t_idx(c0 + 4, col)])};
-                    mma_tf32(acc[nt], a, b);
-                }
-            }
-        }
-        float* M = Ms + warp * 256;
+    for (int ks = 0; ks < 2; ++ks) {
+        const int c0 = 16 * xk + 8 * ks + t;
+        const uint32_t a[4] = {to_tf32(X[a_idx(16 * xi + g, c0)]),
+                               to_tf32(X[a_idx(16 * xi + g + 8, c0)]),
+                               to_tf32(X[a_idx(16 * xi + g, c0 + 4)]),
+                               to_tf32(X[a_idx(16 * xi + g + 8, c0 + 4)])};
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            M[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
-            M[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
-            M[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
-            M[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
-        }
-        __syncwarp();
-        float out[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const int c0 = 16 * I + 8 * ks + t;
-            const uint32_t a[4] = {to_tf32(Tf[t_idx(16 * I + g, c0)]),
-                                   to_tf32(Tf[t_idx(16 * I + g + 8, c0)]),
-                                   to_tf32(Tf[t_idx(16 * I + g, c0 + 4)]),
-                                   to_tf32(Tf[t_idx(16 * I + g + 8, c0 + 4)])};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t b[2] = {to_tf32(M[(8 * ks + t) * 16 + 8 * nt + g]),
-                                       to_tf32(M[(8 * ks + t + 4) * 16 + 8 * nt + g])};
-                mma_tf32(out[nt], a, b);
-            }
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int col = 16 * J + 8 * nt + 2 * t;
-            Tf[t_idx(16 * I + g, col)] = -out[nt][0];
-            Tf[t_idx(16 * I + g, col + 1)] = -out[nt][1];
-            Tf[t_idx(16 * I + g + 8, col)] = -out[nt][2];
-            Tf[t_idx(16 * I + g + 8, col + 1)] = -out[nt][3];
+            const int col = 16 * yj + 8 * nt + g;
+            const uint32_t b[2] = {to_tf32(Y[a_idx(c0, col)]), to_tf32(Y[a_idx(c0 + 4, col)])};
+            mma_tf32(acc[nt], a, b);
         }
     }
-    if (bar_id == 0)
-        __syncthreads();
-    else
-        sm100::group_sync(bar_id, nthreads);
+}
+// acc[nt] += X[16 xi.., 16 xk..] * M, M a row-major 16 x 16 scratch tile.
+__device__ __forceinline__ void blk_mma_scratch(float (&acc)[2][4], const float* X, int xi,
+                                                int xk, const float* M, int g, int t) {
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const int c0 = 16 * xk + 8 * ks + t;
+        const uint32_t a[4] = {to_tf32(X[a_idx(16 * xi + g, c0)]),
+                               to_tf32(X[a_idx(16 * xi + g + 8, c0)]),
+                               to_tf32(X[a_idx(16 * xi + g, c0 + 4)]),
+                               to_tf32(X[a_idx(16 * xi + g + 8, c0 + 4)])};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b[2] = {to_tf32(M[(8 * ks + t) * 16 + 8 * nt + g]),
+                                   to_tf32(M[(8 * ks + t + 4) * 16 + 8 * nt + g])};
+            mma_tf32(acc[nt], a, b);
+        }
+    }
+}
+__device__ __forceinline__ void acc_to_scratch(const float (&acc)[2][4], float* M, int g, int t) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        M[g * 16 + 8 * nt + 2 * t] = acc[nt][0];
+        M[g * 16 + 8 * nt + 2 * t + 1] = acc[nt][1];
+        M[(g + 8) * 16 + 8 * nt + 2 * t] = acc[nt][2];
+        M[(g + 8) * 16 + 8 * nt + 2 * t + 1] = acc[nt][3];
+    }
+}
+__device__ __forceinline__ void acc_to_T_neg(const float (&acc)[2][4], float* Tf, int I, int J,
+                                             int g, int t) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int col = 16 * J + 8 * nt + 2 * t;
+        Tf[a_idx(16 * I + g, col)] = -acc[nt][0];
+        Tf[a_idx(16 * I + g, col + 1)] = -acc[nt][1];
+        Tf[a_idx(16 * I + g + 8, col)] = -acc[nt][2];
+        Tf[a_idx(16 * I + g + 8, col + 1)] = -acc[nt][3];
+    }
+}
+
+__device__ __forceinline__ void inverse_pairs(const float* Af, float* Tf, float* Ms, int warp,
+                                              int lane) {
+    if (warp >= 2) return;
+    const int J = 2 * warp, I = J + 1, g = lane >> 2, t = lane & 3;
+    float* M = Ms + warp * 256;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    blk_mma(acc, Af, I, J, Tf, J, g, t);  // A_IJ T_JJ
+    acc_to_scratch(acc, M, g, t);
+    __syncwarp();
+    float out[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    blk_mma_scratch(out, Tf, I, I, M, g, t);  // T_II M
+    acc_to_T_neg(out, Tf, I, J, g, t);
+}
+
+__device__ __forceinline__ void inverse_lower_left(const float* Af, float* Tf, float* Ms,
+                                                   int warp, int lane, uint32_t bar4) {
+    if (warp >= 4) return;
+    const int i = 2 + (warp >> 1), j = warp & 1, g = lane >> 2, t = lane & 3;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int k = j; k < 2; ++k) blk_mma(acc, Af, i, k, Tf, j, g, t);  // M_ij
+    acc_to_scratch(acc, Ms + warp * 256, g, t);
+    sm100::group_sync(bar4, 128);
+    float out[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // T_ij = -(T_i2 M_2j [+ T_33 M_3j]); scratch tile of M_kj is 2 (k - 2) + j
+    for (int k = 2; k <= i; ++k) blk_mma_scratch(out, Tf, i, k, Ms + (2 * (k - 2) + j) * 256, g, t);
+    acc_to_T_neg(out, Tf, i, j, g, t);
 }
 
 }  // namespace tc

@@ -44,7 +44,7 @@ EXPORTS = (
     "kda_gdn_decode_step", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
     "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd", "kda_qkv_conv_norm_step",
     "kda_chunk_fwd_with_plan", "kda_chunk_fwd_plan_workspace_size",
-    "kda_test_overlap_flag_timeout",
+    "kda_test_overlap_flag_timeout", "kda_layer_decode_step",
 )
 
 
@@ -87,6 +87,7 @@ _SIGS = {
     "kda_gdn_chunk_bwd": ([_vp] * 9 + [_i] * 7 + [_vp] * 7 + [_sz, _vp], _i),
     "kda_qkv_conv_norm_step": ([_vp] * 9 + [_i] * 5 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
+    "kda_layer_decode_step": ([_vp] * 14 + [_i] * 5 + [ctypes.c_float] * 2 + [_vp, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
 
@@ -422,6 +423,19 @@ def kda_output_norm_gate(o, gate, w, total_tokens, H, dv, dtype, eps, y, stream=
     st = load().kda_output_norm_gate(_p(o), _p(gate), _p(w), total_tokens, H, dv,
                                      dtype_code(dtype), float(eps), _p(y), _stream(stream))
     return _ret(st, "kda_output_norm_gate", check)
+
+
+def kda_layer_decode_step(xq, xk, xv, wq, wk, wv, conv_q, conv_k, conv_v, g, beta, state, gate,
+                          w_norm, N, H, dk, dv, dtype, l2_eps, rms_eps, y, stream=None,
+                          check=True) -> int:
+    _check("kda_layer_decode_step", dtype, typed=(xq, xk, xv, conv_q, conv_k, conv_v, gate, y),
+           f32=(wq, wk, wv, g, beta, state, w_norm))
+    st = load().kda_layer_decode_step(_p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv),
+                                      _p(conv_q), _p(conv_k), _p(conv_v), _p(g), _p(beta),
+                                      _p(state), _p(gate), _p(w_norm), N, H, dk, dv,
+                                      dtype_code(dtype), float(l2_eps), float(rms_eps), _p(y),
+                                      _stream(stream))
+    return _ret(st, "kda_layer_decode_step", check)
 
 
 def kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, dtype, stream=None,

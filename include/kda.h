@@ -393,6 +393,34 @@ kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* 
                                   int total_tokens, int H, int dv, kda_dtype_t dtype, float eps,
                                   void* y, void* stream);
 
+/* kda_layer_decode_step: one decode token of a whole KDA layer core in one
+ * launch -- kda_qkv_conv_norm_step, kda_decode_step and kda_output_norm_gate
+ * fused, so q, k, v and o never leave the chip:
+ *   q, k = L2-normalised Swish(conv4) of xq, xk with the convolution states
+ *   (eps l2_eps), v = Swish(conv4) of xv; the states shift in place;
+ *   the decode step on (q, k, v, g, beta, state) -> o (fp32, not rounded);
+ *   y = o / sqrt(mean_j o_j^2 + rms_eps) * w_norm * sigmoid(gate).
+ * Defining passages: those of the three calls (Kimi Linear (aiwiki.ai), "The
+ * constrained DPLR form and the chunkwise algorithm": the steps each KDA head
+ * applies around the operator).
+ * In:  xq, xk [N, H, dk], xv [N, H, dv], gate [N, H, dv] (dtype); wq, wk
+ *      [H*dk, 4], wv [H*dv, 4], w_norm [dv], g [N, H, dk], beta [N, H] fp32.
+ * In/out: conv_q, conv_k [N, 3, H, dk], conv_v [N, 3, H, dv] (dtype) as for
+ *      kda_qkv_conv_norm_step; state [N, H, dk, dv] fp32 as for kda_decode_step.
+ * Out: y [N, H, dv] (dtype), not aliasing any input.
+ * The value columns of a (sequence, head) are split over two CTAs of one
+ * thread-block cluster when dv = 128 (they share the RMSNorm's sum over dv
+ * through distributed shared memory).  Shapes: dk, dv in {32, 64, 128};
+ * N == 0 does nothing.  No workspace.
+ */
+kda_status_t kda_layer_decode_step(const void* xq, const void* xk, const void* xv,
+                                  const float* wq, const float* wk, const float* wv,
+                                  void* conv_q, void* conv_k, void* conv_v, const float* g,
+                                  const float* beta, float* state, const void* gate,
+                                  const float* w_norm, int N, int H, int dk, int dv,
+                                  kda_dtype_t dtype, float l2_eps, float rms_eps, void* y,
+                                  void* stream);
+
 /* ------------------------------------------------ prefill, no allocation
  * kda_chunk_fwd_noalloc: the same computation as kda_chunk_fwd, with no
  * workspace argument, for callers that may not obtain device memory: an

@@ -290,3 +290,16 @@ def test_python_wrappers_reject_tensors_the_abi_would_misread(lib):
     with pytest.raises(ValueError, match="contiguous"):
         kda.kda_decode_step(q[0], q[0], q[0], g[0], beta[0],
                             torch.zeros(1, H, d, d).transpose(2, 3), o[0], 1, H, d, d, "bf16")
+
+
+def test_layer_decode_rejects_bad_arguments(lib):
+    f, F = kda.kda_layer_decode_step, 1 << 20
+    ptrs = [F] * 14
+    ok = dict(N=2, H=2, dk=128, dv=128, dtype="bf16", l2_eps=1e-6, rms_eps=1e-6, y=F, stream=0,
+              check=False)
+    assert f(*ptrs, **dict(ok, dk=48)) == kda.KDA_ERR_UNSUPPORTED
+    assert f(*ptrs, **dict(ok, rms_eps=0.0)) == kda.KDA_ERR_INVALID_ARG
+    assert f(*ptrs, **dict(ok, N=-1)) == kda.KDA_ERR_INVALID_ARG
+    assert f(*ptrs[:13], None, **ok) == kda.KDA_ERR_INVALID_ARG      # no w_norm
+    assert f(*ptrs[:13], F + 4, **ok) == kda.KDA_ERR_INVALID_ARG     # misaligned
+    assert f(*ptrs, **dict(ok, N=0)) == kda.KDA_OK
