@@ -50,7 +50,7 @@ kda_status_t begin_prefill(const Workspace& w, const int32_t* cu, int B, int T, 
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     e = launch_build_chunk_table(cu, B, T, N, chunk, maxc, w.status, w.chunk_start,
-                                 w.chunk_info, st);
+                                 w.chunk_info, st, w.seq_order);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -275,7 +275,7 @@ kda_status_t chunk_fwd_on(Path path, const void* q, const void* k, const void* v
         return from_cuda(kda::launch_chunk_fwd_split(q, k, v, g, beta, initial_state,
                                                      cu_seqlens, T, p.N, H, w.chunk_info, maxc,
                                                      w.chunk_start, w.status, w.blobs, o,
-                                                     final_state, st));
+                                                     final_state, st, nullptr, w.seq_order));
     }
     return run_simt(q, k, v, g, beta, initial_state, cu_seqlens, B, T, p, H, dk, dv, chunk,
                     dtype, o, final_state, w, maxc, st);
@@ -478,7 +478,7 @@ kda_status_t kda_chunk_split_chain(const void* v, const float* initial_state,
         return KDA_ERR_INVALID_ARG;
     return from_cuda(kda::launch_split_chain(v, initial_state, cu_seqlens, T, p.N, H,
                                              w.chunk_start, w.status, w.blobs, o, final_state,
-                                             static_cast<cudaStream_t>(stream)));
+                                             static_cast<cudaStream_t>(stream), w.seq_order));
 }
 
 // ----------------------------------------------------------------- decode
@@ -540,7 +540,7 @@ kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, cons
         return from_cuda(kda::launch_chunk_fwd_split(q, k, v, nullptr, beta, initial_state,
                                                      cu_seqlens, T, p.N, H, w.chunk_info, maxc,
                                                      w.chunk_start, w.status, w.blobs, o,
-                                                     final_state, st, g));
+                                                     final_state, st, g, w.seq_order));
     float* gfull = reinterpret_cast<float*>(static_cast<char*>(workspace) + spread_off);
     const cudaError_t e = kda::launch_spread_gate(g, p.total, H, dk, gfull, st);
     if (e != cudaSuccess) return KDA_ERR_CUDA;

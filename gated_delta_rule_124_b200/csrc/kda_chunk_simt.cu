@@ -23,12 +23,16 @@ namespace kda {
 
 // ------------------------------------------------------------- chunk table
 // One block.  Validates cu_seqlens (or synthesises B equal sequences of T),
-// writes chunk_start[N + 1] and fills chunk_info[maxc].
+// writes chunk_start[N + 1], fills chunk_info[maxc] and, when `order` is
+// given, the sequences by descending chunk count (ties by index) -- per-chain
+// work launched in that order starts with the longest chains, so that the
+// last one to start is short.
 __global__ void build_chunk_table_kernel(const int32_t* __restrict__ cu, int B, int T, int N,
                                          int chunk, int maxc, uint32_t* status,
                                          int* __restrict__ chunk_start,
-                                         int4* __restrict__ info) {
+                                         int4* __restrict__ info, int* __restrict__ order) {
     __shared__ int warp_sums[32];
+    __shared__ int s_nch[kMaxOrderedSeqs];
     __shared__ int bad, most;
     const int tid = threadIdx.x, nt = blockDim.x;
     if (tid == 0) bad = most = 0;
@@ -85,6 +89,24 @@ __global__ void build_chunk_table_kernel(const int32_t* __restrict__ cu, int B, 
         excl += (seq_lo(s + 1) - seq_lo(s) + chunk - 1) / chunk;
     }
     if (s1 == N && s0 < s1) chunk_start[N] = excl;
+    if (order) {
+        if (N <= kMaxOrderedSeqs) {
+            for (int s = tid; s < N; s += nt)
+                s_nch[s] = (seq_lo(s + 1) - seq_lo(s) + chunk - 1) / chunk;
+            __syncthreads();
+            for (int s = tid; s < N; s += nt) {
+                const int c = s_nch[s];
+                int rank = 0;
+                for (int u = 0; u < N; ++u) {
+                    const int cu2 = s_nch[u];
+                    rank += (cu2 > c) || (cu2 == c && u < s);
+                }
+                order[rank] = s;
+            }
+        } else {
+            for (int s = tid; s < N; s += nt) order[s] = s;
+        }
+    }
     if (N == 0 && tid == 0) chunk_start[0] = 0;
     __syncthreads();
     if (tid == 0 && per * nt >= N && s0 >= N) {
@@ -115,9 +137,9 @@ __global__ void build_chunk_table_kernel(const int32_t* __restrict__ cu, int B, 
 
 cudaError_t launch_build_chunk_table(const int32_t* cu_seqlens, int B, int T, int N, int chunk,
                                      int maxc, uint32_t* status, int* chunk_start,
-                                     int4* chunk_info, cudaStream_t st) {
+                                     int4* chunk_info, cudaStream_t st, int* seq_order) {
     build_chunk_table_kernel<<<1, 1024, 0, st>>>(cu_seqlens, B, T, N, chunk, maxc, status,
-                                                 chunk_start, chunk_info);
+                                                 chunk_start, chunk_info, seq_order);
     return cudaGetLastError();
 }
 

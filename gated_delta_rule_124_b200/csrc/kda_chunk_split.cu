@@ -267,15 +267,6 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         const int slot = cur.slot, h = cur.h, L = cur.L;
         const bool more = nxt.it < nitems;
         uint8_t* blob = p.blobs + ((size_t)slot * p.H + h) * BLOB;
-        // one thread (idle in the inverse phase, where the lookup is resolved)
-        // starts looking up the item after the next now, so that the global
-        // read of its chunk descriptor is in flight during E1 and E2
-        int ahead_cand = nitems;
-        int4 ahead_info = make_int4(0, 0, 0, 0);
-        if (tid == NTI - 32) {
-            ahead_cand = more ? nxt.it + nworkers : nitems;
-            if (!kOverlap && ahead_cand < nitems) ahead_info = p.info[slot_of(ahead_cand)];
-        }
         if (tid < C) sbeta[tid] = beta_next;
         if (kScalar && tid < C) sGs[tid] = gs_next;
         if (tid == 0) {
@@ -291,17 +282,15 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             failed = true;
             break;
         }
+        // ------------- E1: in-chunk cumulative log-gate, per channel.  Thread
+        // (row group grp = 8 rows, channels 4 c4 ..): scan of its 8 rows, then
+        // the totals of the groups above it added; per-channel max / min.
         bool slow_local = false;
-        // (per-channel gate) thread (c4, grp) owns rows 8 grp .. 8 grp + 7 and
-        // channels 4 c4 .. 4 c4 + 3 from the scan to the operand tiles: its G
-        // stays in registers, with its channels' reference Gm and exp(Gm)
-        const int c4 = tid & 31, grp = tid >> 5, r0 = 8 * grp;
-        float4 Gr[8], Gm4 = make_float4(0.f, 0.f, 0.f, 0.f), eGm4 = Gm4;
         if (kScalar) {
             // one warp: lane l holds rows 2l, 2l + 1; inclusive scan by shuffles
             if (warp == 0) {
-                const int rr = 2 * lane;
-                const float v0 = rr < L ? sGs[rr] : 0.f, v1 = rr + 1 < L ? sGs[rr + 1] : 0.f;
+                const int r0 = 2 * lane;
+                const float v0 = r0 < L ? sGs[r0] : 0.f, v1 = r0 + 1 < L ? sGs[r0 + 1] : 0.f;
                 float pre = v0 + v1;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -310,16 +299,16 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 }
                 const float G0 = pre - v1, G1 = pre;
                 float mx = -INFINITY, mn = INFINITY;
-                if (rr < L) { mx = G0; mn = G0; }
-                if (rr + 1 < L) { mx = fmaxf(mx, G1); mn = fminf(mn, G1); }
+                if (r0 < L) { mx = G0; mn = G0; }
+                if (r0 + 1 < L) { mx = fmaxf(mx, G1); mn = fminf(mn, G1); }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
                 }
                 __syncwarp();
-                sGs[rr] = G0;
-                sGs[rr + 1] = G1;
+                sGs[r0] = G0;
+                sGs[r0 + 1] = G1;
                 __syncwarp();
                 if (lane == 0) {
                     const float Gm = mx - kRef;
@@ -336,20 +325,19 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 sGL[tid] = sGsc[2];
             }
         } else {
-            // ------------- E1: in-chunk cumulative log-gate, per channel: scan
-            // of the thread's 8 rows, then the totals of the row groups above
-            // it added; per-channel max / min over the chunk's rows
-            const float* g = reinterpret_cast<const float*>(sm + OFF_G);
+            float* g = reinterpret_cast<float*>(sm + OFF_G);
             float4* tot = reinterpret_cast<float4*>(sm + OFF_TB);           // [8][32]
             float4* gmx = reinterpret_cast<float4*>(sm + OFF_TB + 4096);    // [8][32]
             float4* gmn = reinterpret_cast<float4*>(sm + OFF_TB + 8192);    // [8][32]
+            const int c4 = tid & 31, grp = tid >> 5, r0 = 8 * grp;
+            float4 x[8];
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float4 v = *reinterpret_cast<const float4*>(g + (r0 + i) * D + 4 * c4);
                 if (r0 + i >= L) v = make_float4(0.f, 0.f, 0.f, 0.f);
                 acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-                Gr[i] = acc;
+                x[i] = acc;
             }
             tot[grp * 32 + c4] = acc;
             group_sync(bar, NTI);
@@ -362,32 +350,36 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             float4 mn = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float4& v = Gr[i];
+                float4 v = x[i];
                 v.x += off.x; v.y += off.y; v.z += off.z; v.w += off.w;
+                *reinterpret_cast<float4*>(g + (r0 + i) * D + 4 * c4) = v;
                 if (r0 + i < L) {
                     mx.x = fmaxf(mx.x, v.x); mx.y = fmaxf(mx.y, v.y);
                     mx.z = fmaxf(mx.z, v.z); mx.w = fmaxf(mx.w, v.w);
                     mn.x = fminf(mn.x, v.x); mn.y = fminf(mn.y, v.y);
                     mn.z = fminf(mn.z, v.z); mn.w = fminf(mn.w, v.w);
                 }
-                if (r0 + i == L - 1) *reinterpret_cast<float4*>(sGL + 4 * c4) = v;
             }
             gmx[grp * 32 + c4] = mx;
             gmn[grp * 32 + c4] = mn;
             group_sync(bar, NTI);
-            float4 gx = gmx[c4], gn = gmn[c4];
+            if (tid < D) {
+                const int c = tid;
+                const float* fx = reinterpret_cast<const float*>(gmx);
+                const float* fn = reinterpret_cast<const float*>(gmn);
+                float gmax = -INFINITY, gmin = INFINITY;
 #pragma unroll
-            for (int j = 1; j < 8; ++j) {
-                const float4 a = gmx[j * 32 + c4], b = gmn[j * 32 + c4];
-                gx.x = fmaxf(gx.x, a.x); gx.y = fmaxf(gx.y, a.y);
-                gx.z = fmaxf(gx.z, a.z); gx.w = fmaxf(gx.w, a.w);
-                gn.x = fminf(gn.x, b.x); gn.y = fminf(gn.y, b.y);
-                gn.z = fminf(gn.z, b.z); gn.w = fminf(gn.w, b.w);
+                for (int j = 0; j < 8; ++j) {
+                    gmax = fmaxf(gmax, fx[j * D + c]);
+                    gmin = fminf(gmin, fn[j * D + c]);
+                }
+                const float Gm = gmax - kRef;
+                const float gl = g[(L - 1) * D + c];
+                sGm[c] = Gm;
+                seGm[c] = expf(Gm);
+                sGL[c] = gl;
+                slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
             }
-            Gm4 = make_float4(gx.x - kRef, gx.y - kRef, gx.z - kRef, gx.w - kRef);
-            eGm4 = make_float4(expf(Gm4.x), expf(Gm4.y), expf(Gm4.z), expf(Gm4.w));
-            auto bad = [](float hi, float lo) { return !(hi - lo <= 2.f * kRef) || !(hi <= 60.f); };
-            slow_local = bad(gx.x, gn.x) || bad(gx.y, gn.y) || bad(gx.z, gn.z) || bad(gx.w, gn.w);
         }
         ok = mbar_wait(bar_k, n & 1, kWaitNs) && mbar_wait(bar_q, n & 1, kWaitNs);
         if (group_sync_or(bar, NTI, !ok)) {
@@ -395,38 +387,16 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             break;
         }
         const bool slow = group_sync_or(bar, NTI, slow_local);
-        // row scales of the chain kernel; -W column scale
-        if (kScalar) {
-            if (tid < D) {
-                const float gl = sGL[tid];
-                sWsc[tid] = slow ? -1.f : -seGm[tid];
-                float* sc = reinterpret_cast<float*>(blob + BL_SC);
-                sc[tid] = expf(gl);
-                sc[D + tid] = slow ? 1.f : expf(gl - sGm[tid]);
-            }
-        } else if (grp == 0) {
-            const float4 gl = *reinterpret_cast<const float4*>(sGL + 4 * c4);
+        if (tid < D) {  // row scales of the chain kernel; -W column scale
+            const float gl = sGL[tid];
+            sWsc[tid] = slow ? -1.f : -seGm[tid];
             float* sc = reinterpret_cast<float*>(blob + BL_SC);
-            *reinterpret_cast<float4*>(sWsc + 4 * c4) =
-                slow ? make_float4(-1.f, -1.f, -1.f, -1.f)
-                     : make_float4(-eGm4.x, -eGm4.y, -eGm4.z, -eGm4.w);
-            *reinterpret_cast<float4*>(sc + 4 * c4) =
-                make_float4(expf(gl.x), expf(gl.y), expf(gl.z), expf(gl.w));
-            *reinterpret_cast<float4*>(sc + D + 4 * c4) =
-                slow ? make_float4(1.f, 1.f, 1.f, 1.f)
-                     : make_float4(expf(gl.x - Gm4.x), expf(gl.y - Gm4.y), expf(gl.z - Gm4.z),
-                                   expf(gl.w - Gm4.w));
+            sc[tid] = expf(gl);
+            sc[D + tid] = slow ? 1.f : expf(gl - sGm[tid]);
         }
         // -------- exact A (fp32, into the Tb region) and P (straight to the
         // blob) on CUDA cores (rare: extreme decay)
         if (slow) {
-            if (!kScalar) {  // the exact path reads G from shared memory
-                float* Gs = reinterpret_cast<float*>(sm + OFF_G);
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    *reinterpret_cast<float4*>(Gs + (r0 + i) * D + 4 * c4) = Gr[i];
-                group_sync(bar, NTI);
-            }
             const float* G = reinterpret_cast<const float*>(sm + OFF_G);
             float* Af = reinterpret_cast<float*>(sm + OFF_TB);
             for (int task = tid; task < C * 8; task += NTI) {
@@ -479,42 +449,69 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             }
             group_sync(bar, NTI);
         }
-        // ------------------------------ E2: operand tiles, in place over K and
-        // Q (K * E, Q * E; exact path: K * Gam, 0), K * E^-1 (exact path:
-        // K * exp(G_last - G)) and Q * Gam straight to the blob
-        if (kScalar) {
-            // each thread keeps one 8-channel group (j = tid & 15) for all its rows
-            const int j = tid & 15, kb = j >> 3, ch = j & 7;
-            const float m0 = slow ? sGL[0] : sGm[0], e0 = seGm[0];
+        // ------------------------------ E2: operand tiles, row-parallel; each
+        // thread keeps one 8-channel group (j = tid & 15) for all its rows
+        {
+            const float* G = reinterpret_cast<const float*>(sm + OFF_G);
+            const int j = tid & 15, kb = j >> 3, ch = j & 7, c0 = 8 * j;
+            float m8[8], e8[8];
+            load8(slow ? sGL + c0 : sGm + c0, m8);
+            load8(seGm + c0, e8);
 #pragma unroll
-            for (int s2 = 0; s2 < (C * 16) / NTI; ++s2) {
-                const int r = (tid + NTI * s2) >> 4;
+            for (int s = 0; s < (C * 16) / NTI; ++s) {
+                const int r = (tid + NTI * s) >> 4;
                 const uint32_t o64 = sw128_off(r, ch);
                 uint8_t* pk = sm + OFF_KQ + kb * 16384 + o64;
                 uint8_t* pq = pk + 8192;
                 float lk[8], lq[8], rk[8], qg[8];
-                if (r < L) {  // the row's factors, once
+                if (r < L && kScalar) {  // the row's factors, once
                     float k8[8], q8[8];
                     unpack8(*reinterpret_cast<const uint4*>(pk), k8);
                     unpack8(*reinterpret_cast<const uint4*>(pq), q8);
                     const float gr = sGs[r];
                     if (!slow) {
-                        const float x = gr - m0;
-                        const float E = __expf(x), Ei = __expf(-x);
+                        const float x = gr - m8[0];
+                        const float E = __expf(x), Ei = __expf(-x), eg = e8[0];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             lk[i] = k8[i] * E;
                             lq[i] = q8[i] * E;
                             rk[i] = k8[i] * Ei;
-                            qg[i] = lq[i] * e0;
+                            qg[i] = lq[i] * eg;
                         }
-                    } else {  // m0 holds G_last here
-                        const float gam = expf(gr), back = expf(m0 - gr);
+                    } else {  // m8 holds G_last here
+                        const float gam = expf(gr), back = expf(m8[0] - gr);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             lk[i] = k8[i] * gam;
                             lq[i] = 0.f;
                             rk[i] = k8[i] * back;
+                            qg[i] = q8[i] * gam;
+                        }
+                    }
+                } else if (r < L) {
+                    float k8[8], q8[8], g8[8];
+                    unpack8(*reinterpret_cast<const uint4*>(pk), k8);
+                    unpack8(*reinterpret_cast<const uint4*>(pq), q8);
+                    load8(G + r * D + c0, g8);
+                    if (!slow) {
+                        // factors within exp(+-80), rounded to bf16 right after
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float x = g8[i] - m8[i];
+                            const float E = __expf(x), Ei = __expf(-x);
+                            lk[i] = k8[i] * E;
+                            lq[i] = q8[i] * E;
+                            rk[i] = k8[i] * Ei;
+                            qg[i] = lq[i] * e8[i];
+                        }
+                    } else {  // m8 holds G_last here
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float gam = expf(g8[i]);
+                            lk[i] = k8[i] * gam;  // K * Gam, in place of K
+                            lq[i] = 0.f;
+                            rk[i] = k8[i] * expf(m8[i] - g8[i]);
                             qg[i] = q8[i] * gam;
                         }
                     }
@@ -526,56 +523,6 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 *reinterpret_cast<uint4*>(pq) = pack8(lq);
                 *reinterpret_cast<uint4*>(sm + OFF_RAP + kb * 8192 + o64) = pack8(rk);
                 *reinterpret_cast<uint4*>(blob + BL_WQ + kb * 16384 + 8192 + o64) = pack8(qg);
-            }
-        } else {
-            // channels 4 c4 .. 4 c4 + 3 are half of one 16-byte chunk of a row:
-            // 64-column block kb, chunk ch, byte offset hb inside the chunk
-            const int kb = c4 >> 4, ch = (c4 & 15) >> 1, hb = (c4 & 1) * 8;
-            const float4 gl = *reinterpret_cast<const float4*>(sGL + 4 * c4);
-            const float m[4] = {slow ? gl.x : Gm4.x, slow ? gl.y : Gm4.y, slow ? gl.z : Gm4.z,
-                                slow ? gl.w : Gm4.w};
-            const float e[4] = {eGm4.x, eGm4.y, eGm4.z, eGm4.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = r0 + i;
-                const uint32_t o64 = sw128_off(r, ch) + hb;
-                uint8_t* pk = sm + OFF_KQ + kb * 16384 + o64;
-                uint8_t* pq = pk + 8192;
-                float lk[4], lq[4], rk[4], qg[4];
-                if (r < L) {
-                    float k4[4], q4[4];
-                    unpack4(*reinterpret_cast<const uint2*>(pk), k4);
-                    unpack4(*reinterpret_cast<const uint2*>(pq), q4);
-                    const float g4[4] = {Gr[i].x, Gr[i].y, Gr[i].z, Gr[i].w};
-                    if (!slow) {
-                        // factors within exp(+-80), rounded to bf16 right after
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float x = g4[j] - m[j];
-                            const float E = __expf(x), Ei = __expf(-x);
-                            lk[j] = k4[j] * E;
-                            lq[j] = q4[j] * E;
-                            rk[j] = k4[j] * Ei;
-                            qg[j] = lq[j] * e[j];
-                        }
-                    } else {  // m holds G_last here
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float gam = expf(g4[j]);
-                            lk[j] = k4[j] * gam;  // K * Gam, in place of K
-                            lq[j] = 0.f;
-                            rk[j] = k4[j] * expf(m[j] - g4[j]);
-                            qg[j] = q4[j] * gam;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) lk[j] = lq[j] = rk[j] = qg[j] = 0.f;
-                }
-                *reinterpret_cast<uint2*>(pk) = pack4(lk);
-                *reinterpret_cast<uint2*>(pq) = pack4(lq);
-                *reinterpret_cast<uint2*>(sm + OFF_RAP + kb * 8192 + o64) = pack4(rk);
-                *reinterpret_cast<uint2*>(blob + BL_WQ + kb * 16384 + 8192 + o64) = pack4(qg);
             }
         }
         fence_async_smem();
@@ -675,13 +622,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                     fence_proxy_async_global();
                     flag_release(p.flags + flag_pending, 1u);
                 }
-                // the item after the next (no further read when the first
-                // candidate's descriptor, read at the top of the item, is valid)
-                const Item d =
-                    (!kOverlap && ahead_cand < nitems && ahead_info.z > 0)
-                        ? Item{ahead_cand, slot_of(ahead_cand), head_of(ahead_cand), ahead_info.z,
-                               ahead_info.y}
-                        : describe(ahead_cand < nitems ? advance(ahead_cand) : nitems);
+                // look up the item after the next
+                const Item d = describe(more ? advance(nxt.it + nworkers) : nitems);
                 s_ahead[0] = d.it;
                 s_ahead[1] = d.slot;
                 s_ahead[2] = d.h;
@@ -870,6 +812,7 @@ struct Params {
     float* hN;
     const uint32_t* flags;  // co-scheduled with the intra kernel: blob ready flags
     uint64_t flag_wait_ns;  // bound of the watcher's wait on one flag
+    const int* order;       // (split plan) sequences, longest first, or NULL
 };
 
 // One chain CTA: (sequence, head) `chain_id`, value columns [64 half, +64).
@@ -1200,7 +1143,10 @@ __global__ void __launch_bounds__(NTC, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    run<false>(&tmv, p, align1024(smem_raw), s_tmem, 1, blockIdx.x >> 1, blockIdx.x & 1);
+    // CTA pairs take the (sequence, head) chains longest sequence first
+    const int r = static_cast<int>(blockIdx.x >> 1);
+    const int chain_id = p.order ? p.order[r / p.H] * p.H + r % p.H : r;
+    run<false>(&tmv, p, align1024(smem_raw), s_tmem, 1, chain_id, blockIdx.x & 1);
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
@@ -1336,7 +1282,8 @@ cudaError_t launch_split_intra(const void* q, const void* k, const float* g, con
 
 cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
                                int N, int H, const int* chunk_start, uint32_t* status,
-                               const void* blobs, void* o, float* hN, cudaStream_t st) {
+                               const void* blobs, void* o, float* hN, cudaStream_t st,
+                               const int* seq_order) {
     const int total = cu_seqlens ? T : N * T;
     if (total == 0) {
         if (hN) {
@@ -1356,6 +1303,7 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
     if (e != cudaSuccess) return e;
     chain::Params pb{h0, cu_seqlens, T, H, chunk_start, status, status,
                      static_cast<const uint8_t*>(blobs), (__nv_bfloat16*)o, hN};
+    pb.order = seq_order;
     chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
     return cudaGetLastError();
 }
@@ -1434,12 +1382,13 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
                                    const int32_t* cu_seqlens, int T, int N, int H,
                                    const int4* chunk_info, int maxc, const int* chunk_start,
                                    uint32_t* status, void* blobs, void* o, float* hN,
-                                   cudaStream_t st, const float* gh) {
+                                   cudaStream_t st, const float* gh, const int* seq_order) {
     const int total = cu_seqlens ? T : N * T;
     cudaError_t e =
         launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs, st, gh);
     if (e != cudaSuccess) return e;
-    return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN, st);
+    return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN, st,
+                              seq_order);
 }
 
 }  // namespace kda

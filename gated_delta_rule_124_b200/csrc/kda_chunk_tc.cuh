@@ -21,16 +21,20 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
                                    const int32_t* cu_seqlens, int T, int N, int H,
                                    const int4* chunk_info, int maxc, const int* chunk_start,
                                    uint32_t* status, void* blobs, void* o, float* hN,
-                                   cudaStream_t st, const float* gh = nullptr);
+                                   cudaStream_t st, const float* gh = nullptr,
+                                   const int* seq_order = nullptr);
 // Its two kernels one at a time (the chain kernel reads what the intra kernel
 // wrote, on the same stream).
 cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
                                int total, int H, const int4* chunk_info, int maxc,
                                uint32_t* status, void* blobs, cudaStream_t st,
                                const float* gh = nullptr);
+// seq_order (the chunk table's longest-first order of the sequences, or NULL):
+// the order in which the chains are launched.
 cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
                                int N, int H, const int* chunk_start, uint32_t* status,
-                               const void* blobs, void* o, float* hN, cudaStream_t st);
+                               const void* blobs, void* o, float* hN, cudaStream_t st,
+                               const int* seq_order = nullptr);
 // The two kernels co-scheduled in one cooperative launch (chains wait for the
 // blobs of their chunks through `flags`, one uint32 per (chunk slot, head)).
 // withheld_flag >= 0 (testing the bounded-wait error path only): the flag of

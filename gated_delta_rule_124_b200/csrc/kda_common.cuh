@@ -15,6 +15,8 @@ namespace kda {
 //                         largest number of chunks of one sequence (written
 //                         by the chunk-table kernel); padding
 //   chunk_start[N + 1]    int32: global index of each sequence's first chunk
+//   seq_order[N]          int32: the sequences by descending chunk count (ties
+//                         by index; the identity beyond kMaxOrderedSeqs)
 //   chunk_info[maxc]      int4 {seq, first token, rows, chunk-in-sequence};
 //                         unused slots hold seq = -1, rows = 0
 //   then, for the CUDA-core path only: G, W, U (token-major fp32) and the
@@ -22,6 +24,9 @@ namespace kda {
 //   only: one operand blob per (chunk slot, head), then one uint32 ready flag
 //   per (chunk slot, head).
 constexpr size_t kAlign = 256;
+// Sequences the chunk-table kernel sorts by length (it ranks them in shared
+// memory); larger batches keep their order.
+constexpr int kMaxOrderedSeqs = 4096;
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a = kAlign) {
     return (x + a - 1) / a * a;
@@ -33,6 +38,7 @@ enum : uint32_t { STATUS_BAD_SEQLENS = 1u, STATUS_TIMEOUT = 2u };
 struct Workspace {
     uint32_t* status;
     int* chunk_start;
+    int* seq_order;
     int4* chunk_info;
     float* G;
     float* W;
@@ -59,6 +65,8 @@ inline Workspace carve(void* base, int total, int N, int H, int dk, int dv, int 
     off += kAlign;
     w.chunk_start = reinterpret_cast<int*>(p + off);
     off = align_up(off + sizeof(int) * (size_t)(N + 1));
+    w.seq_order = reinterpret_cast<int*>(p + off);
+    off = align_up(off + sizeof(int) * (size_t)N);
     w.chunk_info = reinterpret_cast<int4*>(p + off);
     off = align_up(off + sizeof(int4) * (size_t)maxc);
     w.header_bytes = off;
@@ -134,7 +142,8 @@ kda_status_t run_simt(const void* q, const void* k, const void* v, const float* 
 namespace kda {
 cudaError_t launch_build_chunk_table(const int32_t* cu_seqlens, int B, int T, int N, int chunk,
                                      int maxc, uint32_t* status, int* chunk_start,
-                                     int4* chunk_info, cudaStream_t st);
+                                     int4* chunk_info, cudaStream_t st,
+                                     int* seq_order = nullptr);
 cudaError_t launch_gate_cumsum(const float* g, const int4* info, int maxc, int H, int dk,
                                const uint32_t* status, float* G, cudaStream_t st);
 cudaError_t launch_intra(const void* k, const void* v, const float* G, const float* beta,

@@ -39,18 +39,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&x)[8]) {
         x[2 * i + 1] = f.y;
     }
 }
-__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
-    return make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
-}
-__device__ __forceinline__ void unpack4(uint2 u, float (&x)[4]) {
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        float2 f = __bfloat1622float2(p[i]);
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-    }
-}
 __device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
     *reinterpret_cast<float4*>(x) = *reinterpret_cast<const float4*>(p);
     *reinterpret_cast<float4*>(x + 4) = *reinterpret_cast<const float4*>(p + 4);
