@@ -317,6 +317,94 @@ kda_status_t kda_chunk_fwd_with_plan(int plan, const void* q, const void* k, con
                         chunk, dtype, o, final_state, workspace, workspace_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+// kda_layer_chunk_fwd's workspace: the plan's own, then (composed path only)
+// q, k, v and o in the input dtype.
+size_t layer_workspace_bytes(const Prefill& p, int H, int dk, int dv, int chunk,
+                             kda_dtype_t dt, Path path, size_t* extra_off) {
+    const size_t base = carve_for(nullptr, p, H, dk, dv, chunk, path).total_bytes;
+    *extra_off = kda::align_up(base);
+    if (path != Path::Simt) return base;
+    const size_t es = dt == KDA_DTYPE_BF16 ? 2 : 4;
+    return kda::align_up(*extra_off + es * (size_t)p.total * H * (2 * dk + 2 * dv));
+}
+}  // namespace
+
+extern "C" {
+
+size_t kda_layer_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
+                                          int chunk, kda_dtype_t dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || H < 1 || !dim_ok(dk) || !dim_ok(dv) ||
+        !chunk_ok(chunk) || !dtype_ok(dtype))
+        return 0;
+    const Prefill p{total_tokens, num_seqs};
+    size_t off;
+    return layer_workspace_bytes(p, H, dk, dv, chunk, dtype,
+                                 tc_shape(dk, dv, chunk, dtype) ? Path::Split : Path::Simt, &off);
+}
+
+kda_status_t kda_layer_chunk_fwd(const void* xq, const void* xk, const void* xv, const float* wq,
+                                 const float* wk, const float* wv, const float* g,
+                                 const float* beta, const float* initial_state,
+                                 const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                                 int dk, int dv, int chunk, kda_dtype_t dtype, const void* gate,
+                                 const float* w_norm, float l2_eps, float rms_eps, void* y,
+                                 float* final_state, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+    Prefill p;
+    kda_status_t s =
+        check_prefill_shape(cu_seqlens, B, T, num_seqs, H, dk, dv, chunk, dtype, &p);
+    if (s != KDA_OK) return s;
+    if (!(l2_eps > 0.f) || !(l2_eps < 1e30f) || !(rms_eps > 0.f) || !(rms_eps < 1e30f))
+        return KDA_ERR_INVALID_ARG;
+    for (const void* ptr : std::initializer_list<const void*>{
+             xq, xk, xv, (const void*)wq, (const void*)wk, (const void*)wv, (const void*)g,
+             (const void*)beta, gate, (const void*)w_norm, y})
+        if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_INVALID_ARG;
+    const Path path = tc_shape(dk, dv, chunk, dtype) ? Path::Split : Path::Simt;
+    size_t extra = 0;
+    const size_t need = layer_workspace_bytes(p, H, dk, dv, chunk, dtype, path, &extra);
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return KDA_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    const Workspace w = carve_for(workspace, p, H, dk, dv, chunk, path);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int maxc = kda::max_chunks(p.total, p.N, chunk);
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);
+    if (s != KDA_OK) return s;
+    if (p.total == 0 && !final_state) return KDA_OK;
+    if (path == Path::Split) {
+        const kda::LayerArgs la{xq, xk, xv, wq, wk, wv, l2_eps, gate, w_norm, rms_eps, y};
+        return from_cuda(kda::launch_chunk_fwd_split(nullptr, nullptr, nullptr, g, beta,
+                                                     initial_state, cu_seqlens, T, p.N, H,
+                                                     w.chunk_info, maxc, w.chunk_start, w.status,
+                                                     w.blobs, nullptr, final_state, st, nullptr,
+                                                     w.seq_order, &la));
+    }
+    // every other shape: the three steps one after another, q, k, v and o in
+    // the workspace
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    char* base = static_cast<char*>(workspace) + extra;
+    void* q = base;
+    void* k = base + es * (size_t)p.total * H * dk;
+    void* v = base + es * (size_t)p.total * H * 2 * dk;
+    void* o = base + es * (size_t)p.total * H * (2 * dk + dv);
+    const void* const x3[3] = {xq, xk, xv};
+    const float* const w3[3] = {wq, wk, wv};
+    void* const y3[3] = {q, k, v};
+    cudaError_t e = kda::launch_qkv_conv(x3, w3, y3, dk, dv, cu_seqlens, p.N, cu_seqlens ? 0 : T,
+                                         p.total, H, l2_eps, dtype, st);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    s = run_simt(q, k, v, g, beta, initial_state, cu_seqlens, B, T, p, H, dk, dv, chunk, dtype, o,
+                 final_state, w, maxc, st);
+    if (s != KDA_OK) return s;
+    return from_cuda(kda::launch_norm_gate(o, gate, w_norm, p.total, H, dv, rms_eps, dtype, y, st));
+}
+
 kda_status_t kda_test_overlap_flag_timeout(const void* q, const void* k, const void* v,
                                            const float* g, const float* beta,
                                            const float* initial_state,

@@ -121,8 +121,13 @@ constexpr uint32_t OFF_GS = OFF_WSC + 512;
 constexpr uint32_t OFF_GSC = OFF_GS + 256;
 constexpr uint32_t OFF_BAR = OFF_GSC + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+// (layer variant) the 3 raw rows before the chunk of xq, xk [2][3][128] bf16,
+// and the head's convolution filters of q, k [2][128][4] fp32
+constexpr uint32_t OFF_HALO = OFF_BAR + 64;
+constexpr uint32_t OFF_CW = OFF_HALO + 1536;
+constexpr uint32_t SMEM_BYTES_CONV = OFF_CW + 4096 + 1024;
 static_assert(OFF_MID == OFF_TB + 8192, "Tb garbage rows follow Tb");
-static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
+static_assert(2 * (SMEM_BYTES_CONV + 1024) <= 233472, "two CTAs per SM");
 constexpr uint32_t TM_X = 0;     // [A ; P] accumulator, 64 columns
 constexpr uint32_t TM_W = 128;   // W accumulator, 128 columns
 constexpr uint32_t TX_K = 16384, TX_Q = 16384, TX_G = 32768;
@@ -144,7 +149,74 @@ struct Params {
     // (testing the bounded-wait error path only) the flag index slot * H + h
     // that is never released, or -1
     long long withheld;
+    // (layer variant) raw xq, xk [total, H, 128] (the tensor maps read them
+    // too), their filters [H * 128, 4] and the L2-norm epsilon
+    const __nv_bfloat16* xq;
+    const __nv_bfloat16* xk;
+    const float* wq;
+    const float* wk;
+    float l2_eps;
 };
+
+// (layer variant) q and k of the chunk from the raw inputs in place: the
+// depthwise causal convolution of kernel 4 (the 3 rows before the chunk come
+// from the halo buffer: the previous chunk's rows, or zeros at a sequence
+// start), Swish, then each row divided by sqrt(sum of squares + eps) over its
+// 128 channels.  Thread (row block b = tid / 16, channel chunk j = tid % 16)
+// owns rows 4 b .. 4 b + 3, channels 8 j .. 8 j + 7: it reads its raw rows
+// (and the three above them), waits at the barrier until every thread has
+// read, then writes its rows.  The 16 threads of a row block are 16
+// consecutive lanes, so the row sums are shuffles.
+__device__ __forceinline__ void conv_qk_tile(uint8_t* sm, const Params& p, int tid, uint32_t bar,
+                                             int nthreads) {
+    const int j = tid & 15, kb = j >> 3, ch = j & 7, b = tid >> 4;
+    uint4 out[2][4];
+#pragma unroll
+    for (int tensor = 0; tensor < 2; ++tensor) {
+        const uint8_t* tile = sm + OFF_KQ + kb * 16384 + tensor * 8192;
+        const float4* w = reinterpret_cast<const float4*>(sm + OFF_CW) + tensor * 128 + 8 * j;
+        float x[7][8];
+#pragma unroll
+        for (int rr = 0; rr < 7; ++rr) {
+            const int row = 4 * b - 3 + rr;
+            const uint4 u = row >= 0 ? *reinterpret_cast<const uint4*>(tile + sw128_off(row, ch))
+                                     : *reinterpret_cast<const uint4*>(
+                                           sm + OFF_HALO + (tensor * 3 + row + 3) * 256 + 16 * j);
+            unpack8(u, x[rr]);
+        }
+        float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 wc = w[c];  // taps 0..3, tap 3 on the current row
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // x[i] is not read again after row i
+                const float a = wc.x * x[i][c] + wc.y * x[i + 1][c] + wc.z * x[i + 2][c] +
+                                wc.w * x[i + 3][c];
+                const float y = a / (1.f + __expf(-a));
+                x[i][c] = y;
+                ss[i] += y * y;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], o);
+            const float inv = rsqrtf(ss[i] + p.l2_eps);
+            float y[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) y[c] = x[i][c] * inv;
+            out[tensor][i] = pack8(y);
+        }
+    }
+    group_sync(bar, nthreads);
+#pragma unroll
+    for (int tensor = 0; tensor < 2; ++tensor) {
+        uint8_t* tile = sm + OFF_KQ + kb * 16384 + tensor * 8192;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(tile + sw128_off(4 * b + i, ch)) = out[tensor][i];
+    }
+}
 
 // One worker (CTA) of the intra-chunk kernel.  Items are (chunk slot, head)
 // pairs taken with a stride of `nworkers`: alone, in slot order; co-scheduled
@@ -156,7 +228,9 @@ struct Params {
 // Linear (aiwiki.ai), "Background: from the delta rule to gated DeltaNet"):
 // read from p.gh by plain loads, scanned by one warp, and every per-channel
 // factor of a row is that row's one factor.
-template <bool kOverlap, bool kScalar = false>
+// kConv (layer variant, not with kOverlap or kScalar): the tensor maps read
+// the raw inputs xq, xk, and conv_qk_tile makes q and k of them in place.
+template <bool kOverlap, bool kScalar = false, bool kConv = false>
 __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* tmk,
                                     const CUtensorMap* tmg, const Params& p, uint8_t* sm,
                                     uint32_t tbase, uint32_t bar, int worker, int nworkers) {
@@ -194,16 +268,17 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     // everything the loop needs of an item, fetched (global loads) one item
     // ahead of its use: {item, chunk slot, head, rows, first token}
     struct Item {
-        int it, slot, h, L, t0;
+        int it, slot, h, L, t0, cs;  // cs: the chunk's index in its sequence
     };
     auto describe = [&](int it) {
-        Item d{it, 0, 0, 0, 0};
+        Item d{it, 0, 0, 0, 0, 0};
         if (it < nitems) {
             d.slot = slot_of(it);
             d.h = head_of(it);
             const int4 c = p.info[d.slot];
             d.L = c.z;
             d.t0 = c.y;
+            d.cs = c.w;
         }
         return d;
     };
@@ -267,6 +342,26 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         const int slot = cur.slot, h = cur.h, L = cur.L;
         const bool more = nxt.it < nitems;
         uint8_t* blob = p.blobs + ((size_t)slot * p.H + h) * BLOB;
+        if (kConv) {
+            // the 3 raw rows of xq, xk before the chunk (zeros at a sequence
+            // start) and the head's filters, waited for before the convolution
+            for (int e = tid; e < 96 + 256; e += NTI) {
+                if (e < 96) {
+                    const int tensor = e / 48, row = (e % 48) / 16, j = e % 16;
+                    uint8_t* dst = sm + OFF_HALO + (tensor * 3 + row) * 256 + 16 * j;
+                    if (cur.cs > 0)
+                        cp_async16(dst, (tensor ? p.xk : p.xq) +
+                                            ((size_t)(cur.t0 - 3 + row) * p.H + h) * D + 8 * j);
+                    else
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+                } else {
+                    const int tensor = (e - 96) >> 7, c = (e - 96) & 127;
+                    cp_async16(sm + OFF_CW + (tensor * 128 + c) * 16,
+                               (tensor ? p.wk : p.wq) + ((size_t)h * D + c) * 4);
+                }
+            }
+            cp_async_commit();
+        }
         if (tid < C) sbeta[tid] = beta_next;
         if (kScalar && tid < C) sGs[tid] = gs_next;
         if (tid == 0) {
@@ -382,10 +477,12 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             }
         }
         ok = mbar_wait(bar_k, n & 1, kWaitNs) && mbar_wait(bar_q, n & 1, kWaitNs);
+        if (kConv) cp_async_wait_all();
         if (group_sync_or(bar, NTI, !ok)) {
             failed = true;
             break;
         }
+        if (kConv) conv_qk_tile(sm, p, tid, bar, NTI);  // its writes: visible after the next barrier
         const bool slow = group_sync_or(bar, NTI, slow_local);
         if (tid < D) {  // row scales of the chain kernel; -W column scale
             const float gl = sGL[tid];
@@ -629,6 +726,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 s_ahead[2] = d.h;
                 s_ahead[3] = d.L;
                 s_ahead[4] = d.t0;
+                s_ahead[5] = d.cs;
             }
             if (tid < C) {
                 // diagonal blocks, right-looking forward substitution in
@@ -720,7 +818,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
         }
         if (kOverlap) flag_pending = static_cast<long long>(slot) * p.H + h;
         cur = nxt;
-        nxt = Item{s_ahead[0], s_ahead[1], s_ahead[2], s_ahead[3], s_ahead[4]};
+        nxt = Item{s_ahead[0], s_ahead[1], s_ahead[2], s_ahead[3], s_ahead[4], s_ahead[5]};
     }
     if (tid == 0) bulk_wait_all();
     if (failed && tid == 0) {
@@ -740,7 +838,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
     }
 }
 
-template <bool kScalar>
+template <bool kScalar, bool kConv>
 __global__ void __launch_bounds__(NTI, 2)
     chunk_intra_kernel(const __grid_constant__ CUtensorMap tmq,
                        const __grid_constant__ CUtensorMap tmk,
@@ -755,8 +853,8 @@ __global__ void __launch_bounds__(NTI, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    run<false, kScalar>(&tmq, &tmk, &tmg, p, align1024(smem_raw), s_tmem, 1, blockIdx.x,
-                        gridDim.x);
+    run<false, kScalar, kConv>(&tmq, &tmk, &tmg, p, align1024(smem_raw), s_tmem, 1, blockIdx.x,
+                               gridDim.x);
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
@@ -785,6 +883,20 @@ constexpr uint32_t OFF_BAR = 108544;
 // wait for one gave up; written by the watcher thread, read by thread 0
 constexpr uint32_t OFF_RDY = OFF_BAR + 32;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+// (layer variant) raw V rows 61-63 of the previous chunk [3][64] bf16 (zeros
+// before a sequence's first chunk); this half's v filters [64][4] fp32 and
+// RMSNorm weights [64] fp32; the partner half's row sums of o^2 written into
+// this CTA by the partner [2 chunk parities][64]; this CTA's two column
+// pieces' row sums [2][64]; two mbarriers (one per parity) on which the
+// partner's 64 row threads arrive
+constexpr uint32_t OFF_VH = OFF_BAR + 64;
+constexpr uint32_t OFF_WV = OFF_VH + 384;
+constexpr uint32_t OFF_WN = OFF_WV + 1024;
+constexpr uint32_t OFF_SSX = OFF_WN + 256;
+constexpr uint32_t OFF_SSL = OFF_SSX + 512;
+constexpr uint32_t OFF_NBAR = OFF_SSL + 512;
+constexpr uint32_t SMEM_BYTES_LAYER = OFF_NBAR + 16 + 1024;
+static_assert(2 * (SMEM_BYTES_LAYER + 1024) <= 233472, "two CTAs per SM");
 static_assert(OFF_ZERO == OFF_TB + 8192, "Tb zero rows");
 static_assert(OFF_PM == OFF_RAP + 16384, "P garbage rows");
 static_assert(2 * SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
@@ -813,7 +925,60 @@ struct Params {
     const uint32_t* flags;  // co-scheduled with the intra kernel: blob ready flags
     uint64_t flag_wait_ns;  // bound of the watcher's wait on one flag
     const int* order;       // (split plan) sequences, longest first, or NULL
+    // (layer variant) the tensor map reads raw xv; its filters [H * 128, 4];
+    // y = RMSNorm(o) * w_norm * sigmoid(gate) is written instead of o
+    const float* wv;
+    const __nv_bfloat16* gate;
+    const float* w_norm;
+    float rms_eps;
+    __nv_bfloat16* y;
 };
+
+// (layer variant) V of the chunk from the raw inputs in place: the depthwise
+// causal convolution of kernel 4 and Swish.  Thread (row pair b = tid / 8,
+// column chunk j = tid % 8) owns rows 2 b, 2 b + 1 and columns 8 j .. 8 j + 7;
+// the 3 rows above the tile come from the halo (the previous chunk's raw rows
+// 61-63), which the owners of rows 61-63 then refill from this chunk.  Reads,
+// barrier, writes.
+__device__ __forceinline__ void conv_v_tile(uint8_t* sm, int tid, uint32_t bar, int nthreads) {
+    const int j = tid & 7, b = tid >> 3;
+    const float4* w = reinterpret_cast<const float4*>(sm + OFF_WV) + 8 * j;
+    float x[5][8];
+#pragma unroll
+    for (int rr = 0; rr < 5; ++rr) {
+        const int row = 2 * b - 3 + rr;
+        const uint4 u = row >= 0
+                            ? *reinterpret_cast<const uint4*>(sm + OFF_V + sw128_off(row, j))
+                            : *reinterpret_cast<const uint4*>(sm + OFF_VH + (row + 3) * 128 + 16 * j);
+        unpack8(u, x[rr]);
+    }
+    // raw rows 61, 62, 63 for the next chunk's halo: rows 2b+1 (b = 30) and 2b,
+    // 2b+1 (b = 31) are x[4] (b = 30), x[3], x[4] (b = 31)
+    const uint4 raw_a = pack8(x[3]), raw_b = pack8(x[4]);
+    uint4 out[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float y[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 wc = w[c];
+            const float a = wc.x * x[i][c] + wc.y * x[i + 1][c] + wc.z * x[i + 2][c] +
+                            wc.w * x[i + 3][c];
+            y[c] = a / (1.f + __expf(-a));
+        }
+        out[i] = pack8(y);
+    }
+    group_sync(bar, nthreads);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        *reinterpret_cast<uint4*>(sm + OFF_V + sw128_off(2 * b + i, j)) = out[i];
+    uint4* vh = reinterpret_cast<uint4*>(sm + OFF_VH);
+    if (b == 30) vh[0 * 8 + j] = raw_b;  // row 61
+    if (b == 31) {
+        vh[1 * 8 + j] = raw_a;  // row 62
+        vh[2 * 8 + j] = raw_b;  // row 63
+    }
+}
 
 // One chain CTA: (sequence, head) `chain_id`, value columns [64 half, +64).
 // Each chunk's loads come in three groups, issued as soon as their regions
@@ -824,7 +989,12 @@ struct Params {
 // is next.
 // The unit is a group of NTC threads synchronising on named barrier `bar`;
 // `tbase` is its 256 TMEM columns.
-template <bool kOverlap>
+// kLayer (layer variant, split plan only, a cluster of the two halves of a
+// chain): V is convolved in place (conv_v_tile) between the two parts of the
+// first product, and the O read-out writes y = RMSNorm(o) * w_norm *
+// sigmoid(gate), the row sums of o^2 over all 128 columns combined with the
+// partner CTA's through distributed shared memory.
+template <bool kOverlap, bool kLayer = false>
 __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uint8_t* sm,
                                     uint32_t tbase, uint32_t bar, int chain_id, int half) {
     const uint32_t sbase = smem_u32(sm);
@@ -944,27 +1114,78 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     }
     for (int i = tid; i < 8192 / 16; i += NTC)
         reinterpret_cast<uint4*>(sm + OFF_ZERO)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (kLayer) {  // this half's filters and norm weights; no rows before the sequence
+        for (int i = tid; i < DVS; i += NTC) {
+            reinterpret_cast<float4*>(sm + OFF_WV)[i] =
+                reinterpret_cast<const float4*>(p.wv)[(size_t)h * D + j0 + i];
+            reinterpret_cast<float*>(sm + OFF_WN)[i] = p.w_norm[j0 + i];
+        }
+        for (int i = tid; i < 24; i += NTC)
+            reinterpret_cast<uint4*>(sm + OFF_VH)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     fence_async_smem();
     tc_fence_before();
     group_sync(bar, NTC);
     tc_fence_after();
 
-    // O rows of chunk m (rows 64-127 of its X buffer; warps of lane quarters 2, 3)
-    auto o_out = [&](int m, int tt0, int LL) {
+    // O rows of chunk m (rows 64-127 of its X buffer; warps of lane quarters 2,
+    // 3); false if (layer variant) the wait for the partner's row sums gave up
+    uint64_t* nbar = reinterpret_cast<uint64_t*>(sm + OFF_NBAR);
+    auto o_out = [&](int m, int tt0, int LL) -> bool {
         const int r = trow - C;
         uint32_t v[32];
         tmem_ld32(tbase + tlane + tx(m) + cq * 32, v);
         tmem_wait_ld();
+        if (!kLayer) {
+            if (r < LL) {
+                __nv_bfloat16* dst = p.o + ((size_t)(tt0 + r) * p.H + h) * D + j0 + cq * 32;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float y[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]);
+                    *reinterpret_cast<uint4*>(dst + q4 * 8) = pack8(y);
+                }
+            }
+            return true;
+        }
+        // y = o / sqrt(mean o^2 + eps) * w_norm * sigmoid(gate): the row sum of
+        // o^2 is this thread's 32 columns + the other column piece's (shared
+        // memory) + the partner half's 64 (written into this CTA by the
+        // partner, with an arrival on nbar[m & 1] per row)
+        const size_t grow = ((size_t)(tt0 + min(r, LL - 1)) * p.H + h) * D + j0 + cq * 32;
+        uint4 gv[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) gv[q4] = *reinterpret_cast<const uint4*>(p.gate + grow + 8 * q4);
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss += __uint_as_float(v[i]) * __uint_as_float(v[i]);
+        float* ssl = reinterpret_cast<float*>(sm + OFF_SSL);
+        float* ssx = reinterpret_cast<float*>(sm + OFF_SSX) + (m & 1) * C;
+        ssl[cq * C + r] = ss;
+        group_sync(bar + 1, 128);  // the four read-out warps
+        if (cq == 0) {
+            const uint32_t partner = static_cast<uint32_t>(half ^ 1);
+            st_cluster_f32(cluster_map(ssx + r, partner), ssl[r] + ssl[C + r]);
+            mbar_arrive_remote(cluster_map(nbar + (m & 1), partner));
+        }
+        if (!mbar_wait_cluster(nbar + (m & 1), (m >> 1) & 1, kWaitNs)) return false;
+        const float inv = rsqrtf((ssl[r] + ssl[C + r] + ssx[r]) / D + p.rms_eps);
         if (r < LL) {
-            __nv_bfloat16* dst = p.o + ((size_t)(tt0 + r) * p.H + h) * D + j0 + cq * 32;
+            const float* wn = reinterpret_cast<const float*>(sm + OFF_WN) + cq * 32;
+            __nv_bfloat16* dst = p.y + grow;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                float y[8];
+                float gt[8], y[8];
+                unpack8(gv[q4], gt);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = __uint_as_float(v[q4 * 8 + i]);
-                *reinterpret_cast<uint4*>(dst + q4 * 8) = pack8(y);
+                for (int i = 0; i < 8; ++i)
+                    y[i] = __uint_as_float(v[q4 * 8 + i]) * inv * wn[q4 * 8 + i] /
+                           (1.f + __expf(-gt[i]));
+                *reinterpret_cast<uint4*>(dst + 8 * q4) = pack8(y);
             }
         }
+        return true;
     };
     int prev_t0 = 0, prev_L = 0;
     int n = 0;
@@ -987,23 +1208,47 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
             gate(n + 1, 1);
         }
         // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
-        if (tid == 0) {
-            constexpr uint32_t id = idesc_bf16_f32(128, DVS, false, true);
+        constexpr uint32_t id1 = idesc_bf16_f32(128, DVS, false, true);
+        if (!kLayer && tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
-                         sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id, ks > 0);
+                         sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id1, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int kb = ks >> 2, kk = ks & 3;
                 mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
-                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id, 1);
+                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id1, 1);
             }
             mma_commit(bar_mma);
         }
+        if (kLayer) {
+            // the S part first; V is convolved in place meanwhile, then its part
+            if (tid == 0) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int kb = ks >> 2, kk = ks & 3;
+                    mma_bf16(tbase + tx(n),
+                             sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id1, ks > 0);
+                }
+            }
+            conv_v_tile(sm, tid, bar, NTC);
+            fence_async_smem();
+            group_sync(bar, NTC);
+            if (tid == 0) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id1, 1);
+                mma_commit(bar_mma);
+            }
+        }
         // the previous chunk's O rows, read out while these products run
-        if (n > 0 && quarter >= 2) o_out(n - 1, prev_t0, prev_L);
+        bool ook = true;
+        if (n > 0 && quarter >= 2) ook = o_out(n - 1, prev_t0, prev_L);
         ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ok = ok && ook;
         ++mma_phase;
         if (group_sync_or(bar, NTC, !ok)) {
             failed = true;
@@ -1084,7 +1329,9 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         prev_t0 = t0;
         prev_L = L;
     }
-    if (!failed && n > 0 && quarter >= 2) o_out(n - 1, prev_t0, prev_L);
+    bool last_ok = true;
+    if (!failed && n > 0 && quarter >= 2) last_ok = o_out(n - 1, prev_t0, prev_L);
+    if (group_sync_or(bar, NTC, !last_ok)) failed = true;
 
     if (!failed && p.hN) {
         const int c = trow;
@@ -1131,24 +1378,39 @@ __device__ __forceinline__ void watch(const Params& p, uint8_t* sm_chain, int ch
     }
 }
 
+// kLayer: launched as clusters of two CTAs (the two halves of a chain), which
+// exchange the RMSNorm's row sums; each initialises its two row-sum mbarriers
+// before a cluster barrier (so no arrival precedes an initialisation) and
+// leaves only after a last cluster barrier (so no partner write reaches an
+// exited CTA).  Every wait between the two barriers is bounded.
+template <bool kLayer>
 __global__ void __launch_bounds__(NTC, 2)
     chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
     if (status_bad(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t s_tmem;
+    uint8_t* sm = align1024(smem_raw);
     if (threadIdx.x < 32) {
         tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
     }
+    if (kLayer && threadIdx.x == 0) {
+        uint64_t* nbar = reinterpret_cast<uint64_t*>(sm + OFF_NBAR);
+        mbar_init(nbar, C);
+        mbar_init(nbar + 1, C);
+        fence_mbar_init();
+    }
     tc_fence_before();
     __syncthreads();
+    if (kLayer) cluster_barrier();
     tc_fence_after();
     // CTA pairs take the (sequence, head) chains longest sequence first
     const int r = static_cast<int>(blockIdx.x >> 1);
     const int chain_id = p.order ? p.order[r / p.H] * p.H + r % p.H : r;
-    run<false>(&tmv, p, align1024(smem_raw), s_tmem, 1, chain_id, blockIdx.x & 1);
+    run<false, kLayer>(&tmv, p, sm, s_tmem, 1, chain_id, blockIdx.x & 1);
     tc_fence_before();
     __syncthreads();
+    if (kLayer) cluster_barrier();
     if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
 }
 }  // namespace chain
@@ -1199,7 +1461,7 @@ __global__ void __launch_bounds__(NTO, 1)
     const uint32_t tb = s_tmem + 256u * unit;
     if (b < nchain) {
         if (unit == 0)
-            chain::run<true>(&tmv, pc, sm, tb, 1, b >> 1, b & 1);
+            chain::run<true, false>(&tmv, pc, sm, tb, 1, b >> 1, b & 1);
         else if (threadIdx.x == 256)
             chain::watch(pc, align1024(smem_raw), b >> 1);
     } else
@@ -1242,12 +1504,14 @@ bool tc_path_available() { return split_encode_fn() != nullptr; }
 
 cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
                                int total, int H, const int4* chunk_info, int maxc,
-                               uint32_t* status, void* blobs, cudaStream_t st, const float* gh) {
+                               uint32_t* status, void* blobs, cudaStream_t st, const float* gh,
+                               const LayerArgs* layer) {
     if (total == 0 || maxc == 0) return cudaSuccess;
+    if (layer && gh) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mg;
-    if (!split_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+    if (!split_map(&mq, layer ? layer->xq : q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+        !split_map(&mk, layer ? layer->xk : k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (gh) {
@@ -1256,13 +1520,17 @@ cudaError_t launch_split_intra(const void* q, const void* k, const float* g, con
                           CU_TENSOR_MAP_SWIZZLE_NONE)) {
         return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel<false>,
+    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel<false, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)intra::SMEM_BYTES);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(intra::chunk_intra_kernel<true>,
+        e = cudaFuncSetAttribute(intra::chunk_intra_kernel<true, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)intra::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(intra::chunk_intra_kernel<false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)intra::SMEM_BYTES_CONV);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -1271,19 +1539,29 @@ cudaError_t launch_split_intra(const void* q, const void* k, const float* g, con
     const int grid = (int)(items < 2 * sms ? items : 2 * sms);
     intra::Params pa{beta, chunk_info, maxc, H, status, status, static_cast<uint8_t*>(blobs)};
     pa.gh = gh;
-    if (gh)
-        intra::chunk_intra_kernel<true><<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(mq, mk, mg,
-                                                                                    pa);
-    else
-        intra::chunk_intra_kernel<false><<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(mq, mk, mg,
-                                                                                     pa);
+    pa.withheld = -1;
+    if (layer) {
+        pa.xq = static_cast<const __nv_bfloat16*>(layer->xq);
+        pa.xk = static_cast<const __nv_bfloat16*>(layer->xk);
+        pa.wq = layer->wq;
+        pa.wk = layer->wk;
+        pa.l2_eps = layer->l2_eps;
+        intra::chunk_intra_kernel<false, true>
+            <<<grid, intra::NTI, intra::SMEM_BYTES_CONV, st>>>(mq, mk, mg, pa);
+    } else if (gh) {
+        intra::chunk_intra_kernel<true, false><<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(
+            mq, mk, mg, pa);
+    } else {
+        intra::chunk_intra_kernel<false, false><<<grid, intra::NTI, intra::SMEM_BYTES, st>>>(
+            mq, mk, mg, pa);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu_seqlens, int T,
                                int N, int H, const int* chunk_start, uint32_t* status,
                                const void* blobs, void* o, float* hN, cudaStream_t st,
-                               const int* seq_order) {
+                               const int* seq_order, const LayerArgs* layer) {
     const int total = cu_seqlens ? T : N * T;
     if (total == 0) {
         if (hN) {
@@ -1294,18 +1572,42 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
         return cudaSuccess;
     }
     CUtensorMap mv;
-    if (!split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+    if (!split_map(&mv, layer ? layer->xv : v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)chain::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
     chain::Params pb{h0, cu_seqlens, T, H, chunk_start, status, status,
                      static_cast<const uint8_t*>(blobs), (__nv_bfloat16*)o, hN};
     pb.order = seq_order;
-    chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
-    return cudaGetLastError();
+    if (!layer) {
+        cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)chain::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        chain::chunk_chain_kernel<false><<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
+        return cudaGetLastError();
+    }
+    cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)chain::SMEM_BYTES_LAYER);
+    if (e != cudaSuccess) return e;
+    pb.wv = layer->wv;
+    pb.gate = static_cast<const __nv_bfloat16*>(layer->gate);
+    pb.w_norm = layer->w_norm;
+    pb.rms_eps = layer->rms_eps;
+    pb.y = static_cast<__nv_bfloat16*>(layer->y);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * N * H);
+    cfg.blockDim = dim3(chain::NTC);
+    cfg.dynamicSmemBytes = chain::SMEM_BYTES_LAYER;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chain::chunk_chain_kernel<true>, mv, pb);
 }
 
 // Grid of the co-scheduled launch (one CTA per SM), or 0 when it does not
@@ -1382,13 +1684,14 @@ cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, 
                                    const int32_t* cu_seqlens, int T, int N, int H,
                                    const int4* chunk_info, int maxc, const int* chunk_start,
                                    uint32_t* status, void* blobs, void* o, float* hN,
-                                   cudaStream_t st, const float* gh, const int* seq_order) {
+                                   cudaStream_t st, const float* gh, const int* seq_order,
+                                   const LayerArgs* layer) {
     const int total = cu_seqlens ? T : N * T;
-    cudaError_t e =
-        launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs, st, gh);
+    cudaError_t e = launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs,
+                                       st, gh, layer);
     if (e != cudaSuccess) return e;
     return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN, st,
-                              seq_order);
+                              seq_order, layer);
 }
 
 }  // namespace kda

@@ -44,7 +44,8 @@ EXPORTS = (
     "kda_gdn_decode_step", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
     "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd", "kda_qkv_conv_norm_step",
     "kda_chunk_fwd_with_plan", "kda_chunk_fwd_plan_workspace_size",
-    "kda_test_overlap_flag_timeout", "kda_layer_decode_step",
+    "kda_test_overlap_flag_timeout", "kda_layer_decode_step", "kda_layer_chunk_fwd",
+    "kda_layer_chunk_fwd_workspace_size",
 )
 
 
@@ -88,6 +89,9 @@ _SIGS = {
     "kda_qkv_conv_norm_step": ([_vp] * 9 + [_i] * 5 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_layer_decode_step": ([_vp] * 14 + [_i] * 5 + [ctypes.c_float] * 2 + [_vp, _vp], _i),
+    "kda_layer_chunk_fwd": ([_vp] * 10 + [_i] * 9 + [_vp, _vp] + [ctypes.c_float] * 2 +
+                            [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_layer_chunk_fwd_workspace_size": ([_i] * 7, _sz),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
 
@@ -423,6 +427,27 @@ def kda_output_norm_gate(o, gate, w, total_tokens, H, dv, dtype, eps, y, stream=
     st = load().kda_output_norm_gate(_p(o), _p(gate), _p(w), total_tokens, H, dv,
                                      dtype_code(dtype), float(eps), _p(y), _stream(stream))
     return _ret(st, "kda_output_norm_gate", check)
+
+
+def kda_layer_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype) -> int:
+    return int(load().kda_layer_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk,
+                                                         dtype_code(dtype)))
+
+
+def kda_layer_chunk_fwd(xq, xk, xv, wq, wk, wv, g, beta, initial_state, cu_seqlens, B, T,
+                        num_seqs, H, dk, dv, chunk, dtype, gate, w_norm, l2_eps, rms_eps, y,
+                        final_state, workspace, workspace_bytes=None, stream=None,
+                        check=True) -> int:
+    _check("kda_layer_chunk_fwd", dtype, typed=(xq, xk, xv, gate, y),
+           f32=(wq, wk, wv, g, beta, initial_state, w_norm, final_state), i32=(cu_seqlens,),
+           raw=(workspace,))
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_layer_chunk_fwd(_p(xq), _p(xk), _p(xv), _p(wq), _p(wk), _p(wv), _p(g),
+                                    _p(beta), _p(initial_state), _p(cu_seqlens), B, T, num_seqs,
+                                    H, dk, dv, chunk, dtype_code(dtype), _p(gate), _p(w_norm),
+                                    float(l2_eps), float(rms_eps), _p(y), _p(final_state),
+                                    _p(workspace), wb, _stream(stream))
+    return _ret(st, "kda_layer_chunk_fwd", check)
 
 
 def kda_layer_decode_step(xq, xk, xv, wq, wk, wv, conv_q, conv_k, conv_v, g, beta, state, gate,

@@ -393,6 +393,42 @@ kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* 
                                   int total_tokens, int H, int dv, kda_dtype_t dtype, float eps,
                                   void* y, void* stream);
 
+/* kda_layer_chunk_fwd: the prefill of a whole KDA layer core --
+ * kda_qkv_conv_norm, kda_chunk_fwd and kda_output_norm_gate in one call:
+ *   q, k = L2-normalised Swish(conv4) of xq, xk (eps l2_eps), v = Swish(conv4)
+ *   of xv, per sequence (zero history at each sequence start);
+ *   the chunkwise prefill on (q, k, v, g, beta, initial_state) -> o, S_final;
+ *   y = o / sqrt(mean_j o_j^2 + rms_eps) * w_norm * sigmoid(gate).
+ * Defining passages: those of the three calls (Kimi Linear (aiwiki.ai), "The
+ * constrained DPLR form and the chunkwise algorithm").
+ * bf16, dk = dv = 128, chunk 64 runs the split tensor-core plan with the steps
+ * fused into its kernels: the intra-chunk kernel convolves and normalises the
+ * q and k tiles it loads (the 3 rows before a chunk read from the previous
+ * chunk), the chain kernel convolves its V tiles and writes y from the O
+ * read-out (the two value-column halves of a chain form a thread-block
+ * cluster and add their row sums of o^2 through distributed shared memory);
+ * q, k, v and o never reach HBM.  Every other supported shape runs the three
+ * steps one after another with q, k, v, o in the workspace.
+ * In:  xq, xk [total, H, dk], xv [total, H, dv], gate [total, H, dv] (dtype);
+ *      wq, wk [H*dk, 4], wv [H*dv, 4], w_norm [dv], g [total, H, dk], beta
+ *      [total, H] fp32; initial_state and cu_seqlens as for kda_chunk_fwd.
+ * Out: y [total, H, dv] (dtype), every token written; final_state as for
+ *      kda_chunk_fwd.
+ * Workspace: kda_layer_chunk_fwd_workspace_size() bytes, 256-byte aligned,
+ *      with the status word read by kda_get_device_status().
+ */
+size_t kda_layer_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
+                                          int chunk, kda_dtype_t dtype);
+
+kda_status_t kda_layer_chunk_fwd(const void* xq, const void* xk, const void* xv, const float* wq,
+                                 const float* wk, const float* wv, const float* g,
+                                 const float* beta, const float* initial_state,
+                                 const int32_t* cu_seqlens, int B, int T, int num_seqs, int H,
+                                 int dk, int dv, int chunk, kda_dtype_t dtype, const void* gate,
+                                 const float* w_norm, float l2_eps, float rms_eps, void* y,
+                                 float* final_state, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* kda_layer_decode_step: one decode token of a whole KDA layer core in one
  * launch -- kda_qkv_conv_norm_step, kda_decode_step and kda_output_norm_gate
  * fused, so q, k, v and o never leave the chip:

@@ -108,3 +108,81 @@ def test_layer_decode_full_size_matches_unfused_and_oracle():
     assert rel_err(st_f, rst) <= tol_for("bf16")
     for a, b in zip(conv_f, conv_u):
         assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ prefill
+
+def _prefill_problem(seed, lens, H, dk, dv, dtype):
+    g = torch.Generator().manual_seed(seed)
+    dt = DT[dtype]
+    total = sum(lens)
+    x = [torch.randn(total, H, d, generator=g).to(dt) for d in (dk, dk, dv)]
+    w = [torch.randn(H * d, 4, generator=g) * 0.5 for d in (dk, dk, dv)]
+    gk = -torch.nn.functional.softplus(torch.randn(total, H, dk, generator=g))
+    beta = torch.sigmoid(torch.randn(total, H, generator=g))
+    ogate = torch.randn(total, H, dv, generator=g).to(dt)
+    wn = torch.rand(dv, generator=g) + 0.5
+    h0 = torch.randn(len(lens), H, dk, dv, generator=g) * 0.02
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return x, w, gk, beta, ogate, wn, h0, cu
+
+
+def _oracle_prefill_layer(x, w, gk, beta, ogate, wn, h0, cu):
+    q, k, v = layer.qkv_conv_norm(*x, *w, cu_seqlens=cu, eps=EPS)
+    o, hN = oracle.forward(q, k, v, gk, beta, h0, cu_seqlens=cu)
+    return layer.output_norm_gate(o, ogate, wn, EPS), hN
+
+
+def _run_prefill_layer(x, w, gk, beta, ogate, wn, h0, cu, H, dk, dv, C, dtype):
+    d = lambda t: t.cuda().contiguous()  # noqa: E731
+    total, N = int(cu[-1]), len(cu) - 1
+    cud = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    y = torch.full_like(d(x[2]), float("nan"))
+    hN = torch.full((N, H, dk, dv), float("nan"), device="cuda")
+    ws = torch.empty(kda.kda_layer_chunk_fwd_workspace_size(total, N, H, dk, dv, C, dtype),
+                     dtype=torch.uint8, device="cuda")
+    kda.kda_layer_chunk_fwd(*[d(a) for a in x], *[d(a) for a in w], d(gk), d(beta), d(h0), cud,
+                            1, total, N, H, dk, dv, C, dtype, d(ogate), d(wn), EPS, EPS, y, hN, ws)
+    assert kda.kda_get_device_status(ws) == kda.KDA_OK
+    return y, hN
+
+
+@pytest.mark.parametrize("dtype,dk,dv,C", [("bf16", 128, 128, 64), ("f32", 64, 32, 32),
+                                           ("bf16", 64, 64, 16)])
+def test_layer_prefill_matches_oracle(dtype, dk, dv, C):
+    """Packed sequences with a 1-token one, one shorter than a chunk, and
+    several chunks (the rows before a chunk come from the previous chunk)."""
+    lens = [C * 3 + 5, 1, C - 3, 2 * C]
+    H = 3
+    args = _prefill_problem(41, lens, H, dk, dv, dtype)
+    ry, rh = _oracle_prefill_layer(*args)
+    y, hN = _run_prefill_layer(*args, H, dk, dv, C, dtype)
+    tol = tol_for(dtype)
+    assert rel_err(y, ry) <= tol, rel_err(y, ry)
+    assert rel_err(hN, rh) <= tol, rel_err(hN, rh)
+
+
+def test_layer_prefill_full_size_matches_unfused_and_oracle():
+    """B=2 x T=2048 tokens, H=32, d=128, bf16: the fused call against the fp64
+    composition (every output and final state) and against the three unfused
+    library calls on the same inputs."""
+    lens, H, d = [2048, 2048], 32, 128
+    x, w, gk, beta, ogate, wn, h0, cu = _prefill_problem(42, lens, H, d, d, "bf16")
+    ry, rh = _oracle_prefill_layer(x, w, gk, beta, ogate, wn, h0, cu)
+    y, hN = _run_prefill_layer(x, w, gk, beta, ogate, wn, h0, cu, H, d, d, 64, "bf16")
+    eo, eh = record("layer prefill (fused): B=2 T=2048 H=32 d=128 bf16", "y", y, ry), \
+        record("layer prefill (fused): B=2 T=2048 H=32 d=128 bf16", "final_state", hN, rh)
+    assert eo <= tol_for("bf16") and eh <= tol_for("bf16"), (eo, eh)
+    # the unfused path
+    dv_ = lambda t: t.cuda().contiguous()  # noqa: E731
+    cud = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    xs = [dv_(a) for a in x]
+    q, k, v = (torch.empty_like(a) for a in xs)
+    kda.kda_qkv_conv_norm(*xs, *[dv_(a) for a in w], cud, 1, 4096, 2, H, d, d, "bf16", EPS,
+                          q, k, v)
+    o, hu = kda.chunk_fwd(q, k, v, dv_(gk), dv_(beta), dv_(h0), cu_seqlens=cud, chunk=64)
+    yu = torch.empty_like(o)
+    kda.kda_output_norm_gate(o, dv_(ogate), dv_(wn), 4096, H, d, "bf16", EPS, yu)
+    torch.cuda.synchronize()
+    assert rel_err(y, yu.double().cpu().numpy()) <= tol_for("bf16")
+    assert rel_err(hN, hu.double().cpu().numpy()) <= tol_for("bf16")
