@@ -1386,7 +1386,14 @@ __device__ __forceinline__ void watch(const Params& p, uint8_t* sm_chain, int ch
 template <bool kLayer>
 __global__ void __launch_bounds__(NTC, 2)
     chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
-    if (status_bad(p.status)) return;
+    // Both CTAs of a cluster must take the same branch here, so the layer
+    // variant leaves only on invalid cu_seqlens (set before this kernel and
+    // never during it -- another chain's timeout can be recorded between the
+    // two CTAs' reads); after a timeout of the intra kernel its chains read
+    // in-bounds blobs and the status already reports the failure.
+    if (kLayer ? (*reinterpret_cast<const volatile uint32_t*>(p.status) & STATUS_BAD_SEQLENS) != 0u
+               : status_bad(p.status))
+        return;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t s_tmem;
     uint8_t* sm = align1024(smem_raw);

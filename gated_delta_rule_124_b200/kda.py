@@ -89,7 +89,7 @@ _SIGS = {
     "kda_qkv_conv_norm_step": ([_vp] * 9 + [_i] * 5 + [ctypes.c_float] + [_vp] * 4, _i),
     "kda_chunk_split_intra": ([_vp] * 5 + [_i] * 4 + [_vp, _sz, _vp], _i),
     "kda_layer_decode_step": ([_vp] * 14 + [_i] * 5 + [ctypes.c_float] * 2 + [_vp, _vp], _i),
-    "kda_layer_chunk_fwd": ([_vp] * 10 + [_i] * 9 + [_vp, _vp] + [ctypes.c_float] * 2 +
+    "kda_layer_chunk_fwd": ([_vp] * 10 + [_i] * 8 + [_vp, _vp] + [ctypes.c_float] * 2 +
                             [_vp, _vp, _vp, _sz, _vp], _i),
     "kda_layer_chunk_fwd_workspace_size": ([_i] * 7, _sz),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),

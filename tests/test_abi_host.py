@@ -303,3 +303,31 @@ def test_layer_decode_rejects_bad_arguments(lib):
     assert f(*ptrs[:13], None, **ok) == kda.KDA_ERR_INVALID_ARG      # no w_norm
     assert f(*ptrs[:13], F + 4, **ok) == kda.KDA_ERR_INVALID_ARG     # misaligned
     assert f(*ptrs, **dict(ok, N=0)) == kda.KDA_OK
+
+
+def test_layer_prefill_rejects_bad_arguments(lib):
+    f, F = kda.kda_layer_chunk_fwd, 1 << 20
+    ptrs = [F] * 10
+    ok = dict(B=1, T=64, num_seqs=1, H=2, dk=128, dv=128, chunk=64, dtype="bf16", gate=F,
+              w_norm=F, l2_eps=1e-6, rms_eps=1e-6, y=F, final_state=None, workspace=F,
+              workspace_bytes=1 << 30, stream=0, check=False)
+    assert f(*ptrs, **dict(ok, dk=48)) == kda.KDA_ERR_UNSUPPORTED
+    assert f(*ptrs, **dict(ok, l2_eps=0.0)) == kda.KDA_ERR_INVALID_ARG
+    assert f(*ptrs, **dict(ok, w_norm=None)) == kda.KDA_ERR_INVALID_ARG
+    assert f(*ptrs, **dict(ok, y=F + 8)) == kda.KDA_ERR_INVALID_ARG
+    assert f(*ptrs, **dict(ok, workspace=None)) == kda.KDA_ERR_WORKSPACE
+    assert f(*ptrs, **dict(ok, workspace_bytes=16)) == kda.KDA_ERR_WORKSPACE
+    assert kda.kda_layer_chunk_fwd_workspace_size(64, 1, 2, 128, 128, 64, "bf16") > 0
+    assert kda.kda_layer_chunk_fwd_workspace_size(64, 1, 2, 48, 128, 64, "bf16") == 0
+
+
+def test_binding_argument_counts_match_the_header(lib):
+    """Every ctypes signature in the binding has as many arguments as the
+    header's declaration of that function."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    from gated_delta_rule_124_b200 import kda as kmod
+    for name, (args, _res) in kmod._SIGS.items():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", src)
+        assert m, name
+        params = [x for x in m.group(1).split(",") if x.strip() and x.strip() != "void"]
+        assert len(params) == len(args), (name, len(params), len(args))
