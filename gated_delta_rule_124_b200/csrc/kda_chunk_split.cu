@@ -121,8 +121,9 @@ constexpr uint32_t OFF_GS = OFF_WSC + 512;
 constexpr uint32_t OFF_GSC = OFF_GS + 256;
 constexpr uint32_t OFF_BAR = OFF_GSC + 64;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
-// (layer variant) the 3 raw rows before the chunk of xq, xk [2][3][128] bf16,
-// and the head's convolution filters of q, k [2][128][4] fp32
+// (layer variant) the 3 raw rows before the chunk of xk, xq [2][3][128] bf16,
+// and the head's convolution filters of k, q [2][128][4] fp32 (slot 0: k,
+// slot 1: q, the order of the K and Q tiles)
 constexpr uint32_t OFF_HALO = OFF_BAR + 64;
 constexpr uint32_t OFF_CW = OFF_HALO + 1536;
 constexpr uint32_t SMEM_BYTES_CONV = OFF_CW + 4096 + 1024;
@@ -349,15 +350,15 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 if (e < 96) {
                     const int tensor = e / 48, row = (e % 48) / 16, j = e % 16;
                     uint8_t* dst = sm + OFF_HALO + (tensor * 3 + row) * 256 + 16 * j;
-                    if (cur.cs > 0)
-                        cp_async16(dst, (tensor ? p.xk : p.xq) +
+                    if (cur.cs > 0)  // slot 0: k, slot 1: q (the order of the tiles)
+                        cp_async16(dst, (tensor ? p.xq : p.xk) +
                                             ((size_t)(cur.t0 - 3 + row) * p.H + h) * D + 8 * j);
                     else
                         *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
                 } else {
                     const int tensor = (e - 96) >> 7, c = (e - 96) & 127;
                     cp_async16(sm + OFF_CW + (tensor * 128 + c) * 16,
-                               (tensor ? p.wk : p.wq) + ((size_t)h * D + c) * 4);
+                               (tensor ? p.wq : p.wk) + ((size_t)h * D + c) * 4);
                 }
             }
             cp_async_commit();
@@ -996,11 +997,13 @@ __device__ __forceinline__ void conv_v_tile(uint8_t* sm, int tid, uint32_t bar, 
 // partner CTA's through distributed shared memory.
 template <bool kOverlap, bool kLayer = false>
 __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uint8_t* sm,
-                                    uint32_t tbase, uint32_t bar, int chain_id, int half) {
+                                    uint32_t tbase, uint32_t bar, int chain_id, int half,
+                                    const CUtensorMap* tmgate = nullptr) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_ld + 1;
     uint64_t* bar_ld3 = bar_ld + 2;
+    uint64_t* bar_gt = bar_ld + 3;  // (layer variant) the output gate tile of a chunk
     const int tid = threadIdx.x & (NTC - 1), warp = tid >> 5;
     const int quarter = warp & 3, cq = warp >> 2;  // rows 32 quarter + lane, columns 32 cq ..
     const int trow = 32 * quarter + (tid & 31);
@@ -1015,6 +1018,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
+        if (kLayer) mbar_init(bar_gt, 1);
         mbar_init(bar_ld3, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
@@ -1028,6 +1032,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
     // transaction count is registered, whether its blob was seen ready
     int pend = 0, coming = 0;
     int ld3_chunk = -1;  // chunk whose group 3 is in flight and not yet waited for
+    int gt_issued = 0;   // (layer variant, thread 0) gate tiles requested
     bool armed = false, armed3 = false, rdy = false;
     const int* s_rdy = reinterpret_cast<const int*>(sm + OFF_RDY);
     auto issue = [&](int n, int groups) {
@@ -1154,9 +1159,6 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         // memory) + the partner half's 64 (written into this CTA by the
         // partner, with an arrival on nbar[m & 1] per row)
         const size_t grow = ((size_t)(tt0 + min(r, LL - 1)) * p.H + h) * D + j0 + cq * 32;
-        uint4 gv[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) gv[q4] = *reinterpret_cast<const uint4*>(p.gate + grow + 8 * q4);
         float ss = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) ss += __uint_as_float(v[i]) * __uint_as_float(v[i]);
@@ -1170,6 +1172,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
             mbar_arrive_remote(cluster_map(nbar + (m & 1), partner));
         }
         if (!mbar_wait_cluster(nbar + (m & 1), (m >> 1) & 1, kWaitNs)) return false;
+        // the chunk's gate tile, brought into the (then idle) U buffer by TMA
+        if (!mbar_wait(bar_gt, m & 1, kWaitNs)) return false;
         const float inv = rsqrtf((ssl[r] + ssl[C + r] + ssx[r]) / D + p.rms_eps);
         if (r < LL) {
             const float* wn = reinterpret_cast<const float*>(sm + OFF_WN) + cq * 32;
@@ -1177,7 +1181,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 float gt[8], y[8];
-                unpack8(gv[q4], gt);
+                unpack8(*reinterpret_cast<const uint4*>(sm + OFF_UB + sw128_off(r, cq * 4 + q4)),
+                        gt);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     y[i] = __uint_as_float(v[q4 * 8 + i]) * inv * wn[q4 * 8 + i] /
@@ -1209,7 +1214,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         }
         // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
         constexpr uint32_t id1 = idesc_bf16_f32(128, DVS, false, true);
-        if (!kLayer && tid == 0) {
+        if ((!kLayer || n > 0) && tid == 0) {  // (layer: V already convolved, below)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
@@ -1222,8 +1227,9 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
             }
             mma_commit(bar_mma);
         }
-        if (kLayer) {
+        if (kLayer && n == 0) {
             // the S part first; V is convolved in place meanwhile, then its part
+            // (later chunks' V is convolved during the previous chunk)
             if (tid == 0) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
@@ -1293,6 +1299,18 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
                          sdesc_sw128(sbase + OFF_UB + ks * 2048, 8192, 1024), idK, ks > 0);
             mma_commit(bar_mma);
         }
+        if (kLayer && has_next) {
+            // while these products run: the next chunk's V (loaded since the
+            // first products completed) convolved in place
+            const bool okv = mbar_wait(bar_ld, (n + 1) & 1, kWaitNs);
+            if (group_sync_or(bar, NTC, !okv)) {
+                ++mma_phase;  // the drain below then waits for these products too
+                failed = true;
+                break;
+            }
+            conv_v_tile(sm, tid, bar, NTC);
+            fence_async_smem();
+        }
         ok = ok3 && mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
         ++mma_phase;
         if (group_sync_or(bar, NTC, !ok)) {
@@ -1301,6 +1319,12 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         }
         tc_fence_after();
         if (has_next && tid == 0) gate(n + 1, 7);  // K E^-1 and P regions free
+        if (kLayer && tid == 0) {  // U is consumed: this chunk's gate tile into its buffer
+            fence_async_smem();
+            mbar_arrive_expect_tx(bar_gt, 8192);
+            tma_load_3d(sm + OFF_UB, tmgate, bar_gt, j0, h, t0);
+            ++gt_issued;
+        }
         // S <- Gam_last * S + ksc * (K E^-1)^T U   (lane = state row c)
         {
             const int c = trow;
@@ -1350,6 +1374,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
         if (armed) mbar_wait(bar_ld, coming & 1, kWaitNs);  // at once if complete
         if (ld3_chunk >= 0) mbar_wait(bar_ld3, ld3_chunk & 1, kWaitNs);
+        if (kLayer && gt_issued > 0) mbar_wait(bar_gt, (gt_issued - 1) & 1, kWaitNs);
         atomicOr(p.status_out, STATUS_TIMEOUT);
     }
     tc_fence_before();
@@ -1385,7 +1410,8 @@ __device__ __forceinline__ void watch(const Params& p, uint8_t* sm_chain, int ch
 // exited CTA).  Every wait between the two barriers is bounded.
 template <bool kLayer>
 __global__ void __launch_bounds__(NTC, 2)
-    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
+    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv,
+                       const __grid_constant__ CUtensorMap tmgate, const Params p) {
     // Both CTAs of a cluster must take the same branch here, so the layer
     // variant leaves only on invalid cu_seqlens (set before this kernel and
     // never during it -- another chain's timeout can be recorded between the
@@ -1414,7 +1440,7 @@ __global__ void __launch_bounds__(NTC, 2)
     // CTA pairs take the (sequence, head) chains longest sequence first
     const int r = static_cast<int>(blockIdx.x >> 1);
     const int chain_id = p.order ? p.order[r / p.H] * p.H + r % p.H : r;
-    run<false, kLayer>(&tmv, p, sm, s_tmem, 1, chain_id, blockIdx.x & 1);
+    run<false, kLayer>(&tmv, p, sm, s_tmem, 1, chain_id, blockIdx.x & 1, &tmgate);
     tc_fence_before();
     __syncthreads();
     if (kLayer) cluster_barrier();
@@ -1590,7 +1616,8 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)chain::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        chain::chunk_chain_kernel<false><<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
+        chain::chunk_chain_kernel<false><<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, mv,
+                                                                                          pb);
         return cudaGetLastError();
     }
     cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel<true>,
@@ -1614,7 +1641,11 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chain::chunk_chain_kernel<true>, mv, pb);
+    CUtensorMap mgt;
+    if (!split_map(&mgt, layer->gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    return cudaLaunchKernelEx(&cfg, chain::chunk_chain_kernel<true>, mv, mgt, pb);
 }
 
 // Grid of the co-scheduled launch (one CTA per SM), or 0 when it does not
