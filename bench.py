@@ -367,7 +367,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- the steps around the operator (conv/Swish/L2-norm before, RMSNorm and
     # output gate after), on this workload's tensors, each timed alone
-    layer = layer_times(kda, torch, P, dev, stream, reps=reps)
+    layer = layer_times(kda, torch, P, dcase, dev, stream, reps=reps)
 
     # ---- end to end through host buffers (pinned), copies inside the region
     e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=3)
@@ -607,45 +607,80 @@ def prefill_kernel_times(kda, P, ws, dev, stream, reps=20):
             "launches_per_call": 5, "path": path}
 
 
-def layer_times(kda, torch, P, dev, stream, reps=20):
-    """CUDA-event times of kda_qkv_conv_norm and kda_output_norm_gate on the
-    prefill workload's shapes (bf16), L2 flushed before each, with their HBM
-    fraction (bytes: every tensor read or written once; conv weights excluded)."""
+def layer_times(kda, torch, P, dcase, dev, stream, reps=20):
+    """The steps around the operator on this workload's shapes (bf16), each
+    timed with CUDA events, L2 flushed before each call: the three separate
+    calls (kda_qkv_conv_norm, kda_output_norm_gate, with their HBM fraction --
+    every tensor read or written once, filters excluded) and, for the whole
+    layer core, the fused call (kda_layer_chunk_fwd) against the three
+    separate launches around kda_chunk_fwd; the same for one decode step
+    (kda_layer_decode_step against kda_qkv_conv_norm_step + kda_decode_step +
+    kda_output_norm_gate) on the decode workload."""
     total, H, dk, dv = P.total, P.H, P.dk, P.dv
+    N = P.N
     Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
     g = torch.Generator(device=dev).manual_seed(7)
     xs = [torch.randn(total, H, d, device=dev, generator=g).to(torch.bfloat16)
           for d in (dk, dk, dv)]
-    ws = [torch.randn(H * d, 4, device=dev, generator=g) for d in (dk, dk, dv)]
+    ws = [torch.randn(H * d, 4, device=dev, generator=g) * 0.5 for d in (dk, dk, dv)]
     outs = [torch.empty_like(x) for x in xs]
     gate = torch.randn(total, H, dv, device=dev, generator=g).to(torch.bfloat16)
     wn = torch.ones(dv, device=dev)
     y = torch.empty_like(gate)
+    o = torch.empty_like(gate)
+    hN = torch.empty(N, H, dk, dv, device=dev)
+    wsp = kda.alloc_workspace(total, N, H, dk, dv, P.chunk, "bf16", dev)
+    wsl = torch.empty(kda.kda_layer_chunk_fwd_workspace_size(total, N, H, dk, dv, P.chunk, "bf16"),
+                      dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    calls = {
-        "qkv_conv_norm": (lambda: kda.kda_qkv_conv_norm(*xs, *ws, P.cu_seqlens, Bc, Tc, P.N, H,
-                                                        dk, dv, "bf16", 1e-6, *outs),
-                          2 * 2 * total * H * (2 * dk + dv)),
-        "output_norm_gate": (lambda: kda.kda_output_norm_gate(outs[2], gate, wn, total, H, dv,
-                                                              "bf16", 1e-6, y),
-                             2 * 3 * total * H * dv),
-    }
+    conv = lambda: kda.kda_qkv_conv_norm(*xs, *ws, P.cu_seqlens, Bc, Tc, N, H, dk, dv,  # noqa
+                                         "bf16", 1e-6, *outs)
+    norm = lambda: kda.kda_output_norm_gate(outs[2], gate, wn, total, H, dv, "bf16", 1e-6, y)  # noqa
+
+    def separate():
+        conv()
+        kda.kda_chunk_fwd(*outs, P.g, P.beta, P.initial_state, P.cu_seqlens, Bc, Tc, N, H, dk,
+                          dv, P.chunk, "bf16", o, hN, wsp)
+        kda.kda_output_norm_gate(o, gate, wn, total, H, dv, "bf16", 1e-6, y)
+
+    fused = lambda: kda.kda_layer_chunk_fwd(*xs, *ws, P.g, P.beta, P.initial_state,  # noqa
+                                            P.cu_seqlens, Bc, Tc, N, H, dk, dv, P.chunk, "bf16",
+                                            gate, wn, 1e-6, 1e-6, y, hN, wsl)
     peaks, _ = load_peaks()
     res = {}
-    for name, (f, nbytes) in calls.items():
-        f()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            f()
-            b.record(stream)
-            ts.append((a, b))
-        torch.cuda.synchronize()
-        t = statistics.median(x.elapsed_time(z) for x, z in ts) / 1e3
+    for name, f, nbytes in (("qkv_conv_norm", conv, 2 * 2 * total * H * (2 * dk + dv)),
+                            ("output_norm_gate", norm, 2 * 3 * total * H * dv)):
+        t = time_calls(torch, stream, flush, f, reps)
         res[name] = {"us": t * 1e6, "bytes": nbytes, "gbs": nbytes / t / 1e9,
                      "hbm_frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+    res["layer_prefill"] = {"workload": P.name if hasattr(P, "name") else None,
+                            "fused_us": time_calls(torch, stream, flush, fused, reps) * 1e6,
+                            "separate_launches_us": time_calls(torch, stream, flush, separate,
+                                                               reps) * 1e6}
+    assert kda.kda_get_device_status(wsl) == kda.KDA_OK
+    # one decode step of the layer core
+    Nd = dcase.N
+    s0 = {k: v.to(dev) for k, v in dcase.steps[0].items()}
+    st = dcase.state0.to(dev)
+    dxs = [torch.randn(Nd, H, d, device=dev, generator=g).to(torch.bfloat16)
+           for d in (dk, dk, dv)]
+    cst = [torch.zeros(Nd, 3, H, d, device=dev, dtype=torch.bfloat16) for d in (dk, dk, dv)]
+    dgate = torch.randn(Nd, H, dv, device=dev, generator=g).to(torch.bfloat16)
+    dy = torch.empty_like(dgate)
+    qkv = [torch.empty_like(x) for x in dxs]
+    od = torch.empty_like(dgate)
+    dfused = lambda: kda.kda_layer_decode_step(*dxs, *ws, *cst, s0["g"], s0["beta"], st,  # noqa
+                                               dgate, wn, Nd, H, dk, dv, "bf16", 1e-6, 1e-6, dy)
+
+    def dseparate():
+        kda.kda_qkv_conv_norm_step(*dxs, *ws, *cst, Nd, H, dk, dv, "bf16", 1e-6, *qkv)
+        kda.kda_decode_step(*qkv, s0["g"], s0["beta"], st, od, Nd, H, dk, dv, "bf16")
+        kda.kda_output_norm_gate(od, dgate, wn, Nd, H, dv, "bf16", 1e-6, dy)
+
+    res["layer_decode_step"] = {"workload": dcase.name,
+                                "fused_us": time_calls(torch, stream, flush, dfused, reps) * 1e6,
+                                "separate_launches_us": time_calls(torch, stream, flush,
+                                                                   dseparate, reps) * 1e6}
     return res
 
 

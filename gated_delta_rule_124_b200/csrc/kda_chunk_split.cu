@@ -193,7 +193,7 @@ __device__ __forceinline__ void conv_qk_tile(uint8_t* sm, const Params& p, int t
             for (int i = 0; i < 4; ++i) {  // x[i] is not read again after row i
                 const float a = wc.x * x[i][c] + wc.y * x[i + 1][c] + wc.z * x[i + 2][c] +
                                 wc.w * x[i + 3][c];
-                const float y = a / (1.f + __expf(-a));
+                const float y = fast_swish(a);
                 x[i][c] = y;
                 ss[i] += y * y;
             }
@@ -887,17 +887,15 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
 // (layer variant) raw V rows 61-63 of the previous chunk [3][64] bf16 (zeros
 // before a sequence's first chunk); this half's v filters [64][4] fp32 and
 // RMSNorm weights [64] fp32; the partner half's row sums of o^2 written into
-// this CTA by the partner [2 chunk parities][64]; this CTA's two column
-// pieces' row sums [2][64]; two mbarriers (one per parity) on which the
-// partner's 64 row threads arrive
+// this unit by the partner unit [2 chunk parities][64]; this unit's two
+// column pieces' row sums [2][64]; two mbarriers (one per parity) on which
+// the partner's 64 row threads arrive
 constexpr uint32_t OFF_VH = OFF_BAR + 64;
 constexpr uint32_t OFF_WV = OFF_VH + 384;
 constexpr uint32_t OFF_WN = OFF_WV + 1024;
 constexpr uint32_t OFF_SSX = OFF_WN + 256;
 constexpr uint32_t OFF_SSL = OFF_SSX + 512;
 constexpr uint32_t OFF_NBAR = OFF_SSL + 512;
-constexpr uint32_t SMEM_BYTES_LAYER = OFF_NBAR + 16 + 1024;
-static_assert(2 * (SMEM_BYTES_LAYER + 1024) <= 233472, "two CTAs per SM");
 static_assert(OFF_ZERO == OFF_TB + 8192, "Tb zero rows");
 static_assert(OFF_PM == OFF_RAP + 16384, "P garbage rows");
 static_assert(2 * SMEM_BYTES <= 228 * 1024, "two CTAs per SM");
@@ -965,7 +963,7 @@ __device__ __forceinline__ void conv_v_tile(uint8_t* sm, int tid, uint32_t bar, 
             const float4 wc = w[c];
             const float a = wc.x * x[i][c] + wc.y * x[i + 1][c] + wc.z * x[i + 2][c] +
                             wc.w * x[i + 3][c];
-            y[c] = a / (1.f + __expf(-a));
+            y[c] = fast_swish(a);
         }
         out[i] = pack8(y);
     }
@@ -990,15 +988,18 @@ __device__ __forceinline__ void conv_v_tile(uint8_t* sm, int tid, uint32_t bar, 
 // is next.
 // The unit is a group of NTC threads synchronising on named barrier `bar`;
 // `tbase` is its 256 TMEM columns.
-// kLayer (layer variant, split plan only, a cluster of the two halves of a
-// chain): V is convolved in place (conv_v_tile) between the two parts of the
-// first product, and the O read-out writes y = RMSNorm(o) * w_norm *
-// sigmoid(gate), the row sums of o^2 over all 128 columns combined with the
-// partner CTA's through distributed shared memory.
+// kLayer (layer variant, split plan only, the two halves of a chain as the two
+// units of one CTA): V is convolved in place (conv_v_tile) -- the first
+// chunk's between the two parts of its first product, later ones' during the
+// previous chunk's second products -- and the O read-out writes y =
+// RMSNorm(o) * w_norm * sigmoid(gate), the row sums of o^2 over all 128
+// columns combined with the partner unit's through shared memory
+// (sm_partner: the partner unit's region).
 template <bool kOverlap, bool kLayer = false>
 __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uint8_t* sm,
                                     uint32_t tbase, uint32_t bar, int chain_id, int half,
-                                    const CUtensorMap* tmgate = nullptr) {
+                                    const CUtensorMap* tmgate = nullptr,
+                                    uint8_t* sm_partner = nullptr) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_mma = bar_ld + 1;
@@ -1156,8 +1157,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         }
         // y = o / sqrt(mean o^2 + eps) * w_norm * sigmoid(gate): the row sum of
         // o^2 is this thread's 32 columns + the other column piece's (shared
-        // memory) + the partner half's 64 (written into this CTA by the
-        // partner, with an arrival on nbar[m & 1] per row)
+        // memory) + the partner half's 64 (written into this unit's buffer by
+        // the partner unit, with an arrival on nbar[m & 1] per row)
         const size_t grow = ((size_t)(tt0 + min(r, LL - 1)) * p.H + h) * D + j0 + cq * 32;
         float ss = 0.f;
 #pragma unroll
@@ -1165,13 +1166,13 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         float* ssl = reinterpret_cast<float*>(sm + OFF_SSL);
         float* ssx = reinterpret_cast<float*>(sm + OFF_SSX) + (m & 1) * C;
         ssl[cq * C + r] = ss;
-        group_sync(bar + 1, 128);  // the four read-out warps
-        if (cq == 0) {
-            const uint32_t partner = static_cast<uint32_t>(half ^ 1);
-            st_cluster_f32(cluster_map(ssx + r, partner), ssl[r] + ssl[C + r]);
-            mbar_arrive_remote(cluster_map(nbar + (m & 1), partner));
+        group_sync(bar + 2, 128);  // the four read-out warps of this unit
+        if (cq == 0) {  // into the partner unit's buffer, then arrive on its barrier
+            float* pssx = reinterpret_cast<float*>(sm_partner + OFF_SSX) + (m & 1) * C;
+            pssx[r] = ssl[r] + ssl[C + r];
+            mbar_arrive(reinterpret_cast<uint64_t*>(sm_partner + OFF_NBAR) + (m & 1));
         }
-        if (!mbar_wait_cluster(nbar + (m & 1), (m >> 1) & 1, kWaitNs)) return false;
+        if (!mbar_wait(nbar + (m & 1), (m >> 1) & 1, kWaitNs)) return false;
         // the chunk's gate tile, brought into the (then idle) U buffer by TMA
         if (!mbar_wait(bar_gt, m & 1, kWaitNs)) return false;
         const float inv = rsqrtf((ssl[r] + ssl[C + r] + ssx[r]) / D + p.rms_eps);
@@ -1185,8 +1186,8 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
                         gt);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    y[i] = __uint_as_float(v[q4 * 8 + i]) * inv * wn[q4 * 8 + i] /
-                           (1.f + __expf(-gt[i]));
+                    y[i] = __uint_as_float(v[q4 * 8 + i]) * inv * wn[q4 * 8 + i] *
+                           fast_sigmoid(gt[i]);
                 *reinterpret_cast<uint4*>(dst + 8 * q4) = pack8(y);
             }
         }
@@ -1403,48 +1404,66 @@ __device__ __forceinline__ void watch(const Params& p, uint8_t* sm_chain, int ch
     }
 }
 
-// kLayer: launched as clusters of two CTAs (the two halves of a chain), which
-// exchange the RMSNorm's row sums; each initialises its two row-sum mbarriers
-// before a cluster barrier (so no arrival precedes an initialisation) and
-// leaves only after a last cluster barrier (so no partner write reaches an
-// exited CTA).  Every wait between the two barriers is bounded.
-template <bool kLayer>
 __global__ void __launch_bounds__(NTC, 2)
-    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv,
-                       const __grid_constant__ CUtensorMap tmgate, const Params p) {
-    // Both CTAs of a cluster must take the same branch here, so the layer
-    // variant leaves only on invalid cu_seqlens (set before this kernel and
-    // never during it -- another chain's timeout can be recorded between the
-    // two CTAs' reads); after a timeout of the intra kernel its chains read
-    // in-bounds blobs and the status already reports the failure.
-    if (kLayer ? (*reinterpret_cast<const volatile uint32_t*>(p.status) & STATUS_BAD_SEQLENS) != 0u
-               : status_bad(p.status))
-        return;
+    chunk_chain_kernel(const __grid_constant__ CUtensorMap tmv, const Params p) {
+    if (status_bad(p.status)) return;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t s_tmem;
-    uint8_t* sm = align1024(smem_raw);
     if (threadIdx.x < 32) {
         tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
     }
-    if (kLayer && threadIdx.x == 0) {
-        uint64_t* nbar = reinterpret_cast<uint64_t*>(sm + OFF_NBAR);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // CTA pairs take the (sequence, head) chains longest sequence first
+    const int r = static_cast<int>(blockIdx.x >> 1);
+    const int chain_id = p.order ? p.order[r / p.H] * p.H + r % p.H : r;
+    run<false>(&tmv, p, align1024(smem_raw), s_tmem, 1, chain_id, blockIdx.x & 1);
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
+}
+
+// The layer variant: one CTA of two 256-thread units per (sequence, head),
+// unit u running the chain on value half u with named barriers 1 + u (and
+// 3 + u for its read-out warps), its own shared-memory region and 256 TMEM
+// columns.  The units add their row sums of o^2 through each other's shared
+// memory (the partner's buffer, then an arrival on the partner's mbarrier;
+// every wait bounded), so the RMSNorm over all 128 columns needs no cluster:
+// a cluster launch of kernels that allocate tensor memory is placed one CTA
+// per SM.
+constexpr uint32_t LAYER_UNIT = (OFF_NBAR + 16 + 1023) / 1024 * 1024;
+constexpr uint32_t LAYER_SMEM = 2 * LAYER_UNIT + 1024;
+static_assert(LAYER_SMEM + 1024 <= 232448, "one 512-thread CTA per SM");
+__global__ void __launch_bounds__(2 * NTC, 1)
+    chunk_chain_layer_kernel(const __grid_constant__ CUtensorMap tmv,
+                             const __grid_constant__ CUtensorMap tmgate, const Params p) {
+    if (status_bad(p.status)) return;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    uint8_t* base = align1024(smem_raw);
+    const int unit = static_cast<int>(threadIdx.x) >> 8;
+    if (threadIdx.x < 32) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+    }
+    if (threadIdx.x < 2) {  // the row-sum barriers of unit threadIdx.x
+        uint64_t* nbar = reinterpret_cast<uint64_t*>(base + threadIdx.x * LAYER_UNIT + OFF_NBAR);
         mbar_init(nbar, C);
         mbar_init(nbar + 1, C);
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
-    if (kLayer) cluster_barrier();
     tc_fence_after();
-    // CTA pairs take the (sequence, head) chains longest sequence first
-    const int r = static_cast<int>(blockIdx.x >> 1);
+    const int r = static_cast<int>(blockIdx.x);
     const int chain_id = p.order ? p.order[r / p.H] * p.H + r % p.H : r;
-    run<false, kLayer>(&tmv, p, sm, s_tmem, 1, chain_id, blockIdx.x & 1, &tmgate);
+    run<false, true>(&tmv, p, base + unit * LAYER_UNIT, s_tmem + 256u * unit, 1 + unit, chain_id,
+                     unit, &tmgate, base + (1 - unit) * LAYER_UNIT);
     tc_fence_before();
     __syncthreads();
-    if (kLayer) cluster_barrier();
-    if (threadIdx.x < 32) tmem_dealloc(s_tmem, 256);
+    if (threadIdx.x < 32) tmem_dealloc(s_tmem, 512);
 }
 }  // namespace chain
 
@@ -1535,6 +1554,20 @@ bool split_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
 
 bool tc_path_available() { return split_encode_fn() != nullptr; }
 
+namespace {
+// Dynamic shared memory of `smem` bytes and the largest shared-memory carveout
+// (two of these CTAs, about 100 KB each, share an SM).
+template <typename F>
+cudaError_t set_smem_max_carveout(F* fn, uint32_t smem) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    return e;
+}
+}  // namespace
+
 cudaError_t launch_split_intra(const void* q, const void* k, const float* g, const float* beta,
                                int total, int H, const int4* chunk_info, int maxc,
                                uint32_t* status, void* blobs, cudaStream_t st, const float* gh,
@@ -1553,17 +1586,12 @@ cudaError_t launch_split_intra(const void* q, const void* k, const float* g, con
                           CU_TENSOR_MAP_SWIZZLE_NONE)) {
         return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(intra::chunk_intra_kernel<false, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)intra::SMEM_BYTES);
+    cudaError_t e = set_smem_max_carveout(intra::chunk_intra_kernel<false, false>,
+                                          intra::SMEM_BYTES);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(intra::chunk_intra_kernel<true, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)intra::SMEM_BYTES);
+        e = set_smem_max_carveout(intra::chunk_intra_kernel<true, false>, intra::SMEM_BYTES);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(intra::chunk_intra_kernel<false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)intra::SMEM_BYTES_CONV);
+        e = set_smem_max_carveout(intra::chunk_intra_kernel<false, true>, intra::SMEM_BYTES_CONV);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -1612,40 +1640,25 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
                      static_cast<const uint8_t*>(blobs), (__nv_bfloat16*)o, hN};
     pb.order = seq_order;
     if (!layer) {
-        cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)chain::SMEM_BYTES);
+        cudaError_t e = set_smem_max_carveout(chain::chunk_chain_kernel, chain::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        chain::chunk_chain_kernel<false><<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, mv,
-                                                                                          pb);
+        chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
         return cudaGetLastError();
     }
-    cudaError_t e = cudaFuncSetAttribute(chain::chunk_chain_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)chain::SMEM_BYTES_LAYER);
+    cudaError_t e = set_smem_max_carveout(chain::chunk_chain_layer_kernel, chain::LAYER_SMEM);
     if (e != cudaSuccess) return e;
     pb.wv = layer->wv;
     pb.gate = static_cast<const __nv_bfloat16*>(layer->gate);
     pb.w_norm = layer->w_norm;
     pb.rms_eps = layer->rms_eps;
     pb.y = static_cast<__nv_bfloat16*>(layer->y);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * N * H);
-    cfg.blockDim = dim3(chain::NTC);
-    cfg.dynamicSmemBytes = chain::SMEM_BYTES_LAYER;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     CUtensorMap mgt;
     if (!split_map(&mgt, layer->gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    return cudaLaunchKernelEx(&cfg, chain::chunk_chain_kernel<true>, mv, mgt, pb);
+    chain::chunk_chain_layer_kernel<<<N * H, 2 * chain::NTC, chain::LAYER_SMEM, st>>>(mv, mgt,
+                                                                                      pb);
+    return cudaGetLastError();
 }
 
 // Grid of the co-scheduled launch (one CTA per SM), or 0 when it does not

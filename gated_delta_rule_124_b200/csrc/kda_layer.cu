@@ -162,7 +162,7 @@ __device__ __forceinline__ void conv_run(const TIn* __restrict__ x, const float*
             acc = fmaf(wt[j][2], win[2][j], acc);
             acc = fmaf(wt[j][1], win[1][j], acc);
             acc = fmaf(wt[j][0], win[0][j], acc);
-            out[j] = __fdividef(acc, 1.f + __expf(-acc));
+            out[j] = swish_for<TIn>(acc);
             ss = fmaf(out[j], out[j], ss);
             win[0][j] = win[1][j];
             win[1][j] = win[2][j];
@@ -205,7 +205,7 @@ __device__ __forceinline__ void conv_step(const TIn* __restrict__ x, const float
         acc = fmaf(wt[j][2], win[2][j], acc);
         acc = fmaf(wt[j][1], win[1][j], acc);
         acc = fmaf(wt[j][0], win[0][j], acc);
-        out[j] = __fdividef(acc, 1.f + __expf(-acc));
+        out[j] = swish_for<TIn>(acc);
         ss = fmaf(out[j], out[j], ss);
     }
     Vec<CPL, TIn>::store(state + (((size_t)n * 3 + 0) * H + h) * D + c0, win[1]);
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(32 * kWarps) norm_gate_kernel(
         float out[CPL];
 #pragma unroll
         for (int j = 0; j < CPL; ++j)
-            out[j] = __fdividef(ov[p][j] * r * wv[j], 1.f + __expf(-gv[p][j]));
+            out[j] = ov[p][j] * r * wv[j] * sigmoid_for<TIn>(gv[p][j]);
         Vec<CPL, TIn>::store(y + (size_t)(first + p) * D + lane * CPL, out);
     }
 }

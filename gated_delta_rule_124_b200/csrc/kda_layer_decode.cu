@@ -55,8 +55,6 @@ struct LayerDecodeArgs {
     float rms_eps;
 };
 
-__device__ __forceinline__ float swish(float x) { return x / (1.f + __expf(-x)); }
-
 // Block-wide sum over NW warps (every thread gets the total).
 template <int NW>
 __device__ __forceinline__ float block_sum(float x, float* red) {
@@ -124,8 +122,8 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
         const float k0 = to_f32(ck[srow(0, DK) + c]), k1 = to_f32(ck[srow(1, DK) + c]),
                     k2 = to_f32(ck[srow(2, DK) + c]);
         const float qx = to_f32(xq[(size_t)unit * DK + c]), kx = to_f32(xk[(size_t)unit * DK + c]);
-        yq = swish(wqv.x * q0 + wqv.y * q1 + wqv.z * q2 + wqv.w * qx);
-        yk = swish(wkv.x * k0 + wkv.y * k1 + wkv.z * k2 + wkv.w * kx);
+        yq = swish_for<TIn>(wqv.x * q0 + wqv.y * q1 + wqv.z * q2 + wqv.w * qx);
+        yk = swish_for<TIn>(wkv.x * k0 + wkv.y * k1 + wkv.z * k2 + wkv.w * kx);
         nq[0] = q1; nq[1] = q2; nq[2] = qx;
         nk[0] = k1; nk[1] = k2; nk[2] = kx;
         s_a[c] = expf(a.g[(size_t)unit * DK + c]);
@@ -136,7 +134,7 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
         const float v0 = to_f32(cv[srow(0, DV) + c]), v1 = to_f32(cv[srow(1, DV) + c]),
                     v2 = to_f32(cv[srow(2, DV) + c]);
         const float vx = to_f32(xv[(size_t)unit * DV + c]);
-        s_v[tid] = swish(wvv.x * v0 + wvv.y * v1 + wvv.z * v2 + wvv.w * vx);
+        s_v[tid] = swish_for<TIn>(wvv.x * v0 + wvv.y * v1 + wvv.z * v2 + wvv.w * vx);
         nv[0] = v1; nv[1] = v2; nv[2] = vx;
     }
     const float sq = block_sum<NW>(yq * yq, s_red);
@@ -238,7 +236,8 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float gt = to_f32(gate[vo + i]);
-            y[vo + i] = from_f32<TIn>(o4[i] * inv * a.w_norm[j0 + 4 * c4 + i] / (1.f + __expf(-gt)));
+            y[vo + i] = from_f32<TIn>(
+                o4[i] * inv * a.w_norm[j0 + 4 * c4 + i] * sigmoid_for<TIn>(gt));
         }
     }
     // keep this CTA's shared memory until the partner has read s_ss

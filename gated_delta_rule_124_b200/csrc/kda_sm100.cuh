@@ -111,49 +111,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-// ------------------------------------------------- distributed shared memory
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t cluster_map(const void* p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// Arrive on an mbarrier of another CTA of the cluster (release at cluster
-// scope: this thread's earlier writes, its DSMEM stores included, are visible
-// to a thread that observes the phase with an acquire wait).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr)
-                 : "memory");
-}
-// Bounded wait on a phase parity with acquire at cluster scope.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  uint64_t limit_ns) {
-    auto test = [&]() {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        return ok != 0;
-    };
-    if (test()) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (test()) return true;
-        if (global_timer_ns() - t0 > limit_ns) return false;
-        __nanosleep(64);
-    }
-}
-// All threads of all CTAs of the cluster (release / acquire at cluster scope).
-__device__ __forceinline__ void cluster_barrier() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                     : "memory");
+// Arrive once on an mbarrier of this CTA (release at CTA scope: this
+// thread's earlier shared-memory writes are visible to a thread that observes
+// the phase with mbar_wait).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Order this thread's generic-proxy shared-memory accesses before later
