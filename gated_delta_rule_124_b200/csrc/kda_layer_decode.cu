@@ -14,16 +14,12 @@
 //   y = o / sqrt(mean_j o_j^2 + rms_eps) * w_norm * sigmoid(gate)
 //
 // q, k, v and o never leave the chip.  As in the plain decode kernel, the
-// value columns of one (sequence, head) are split over NS = DV / DVS CTAs
-// (DVS = 64 for DV = 128); those CTAs form one thread-block cluster, because
-// three things cross the split: both CTAs read the whole q/k convolution
-// states (so the state is overwritten only after a cluster barrier, by rank 0),
-// and the RMSNorm needs the sum of o^2 over all DV columns (each CTA publishes
-// its slice's sum in shared memory and reads its partner's through
-// distributed shared memory).  Every CTA of a cluster reaches every barrier, so
-// none waits for long; a final barrier keeps each CTA's shared memory alive
-// until its partner has read it.
-#include <cooperative_groups.h>
+// value columns of one (sequence, head) are split into NS = DV / DVS slices
+// (DVS = 64 for DV = 128); here the slices are the NS 256-thread units of one
+// CTA, because three things cross the split: the q / k convolution (computed
+// once per CTA and shared), the convolution states (overwritten after a CTA
+// barrier, once every thread has read them) and the RMSNorm, which needs the
+// sum of o^2 over all DV columns (each unit's slice sum in shared memory).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -31,8 +27,6 @@
 
 namespace kda {
 namespace {
-
-namespace cg = cooperative_groups;
 
 struct LayerDecodeArgs {
     const void* xq;
@@ -70,27 +64,27 @@ __device__ __forceinline__ float block_sum(float x, float* red) {
 }
 
 template <int DK, int DV, int DVS, typename TIn>
-__global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
+__global__ void __launch_bounds__(256 * (DV / DVS), ((DK * DVS <= 8192) ? 4 : 2) / (DV / DVS))
     layer_decode_kernel(const LayerDecodeArgs a) {
-    constexpr int NS = DV / DVS;       // CTAs per (sequence, head) = cluster size
-    constexpr int NW = 8;
+    constexpr int NS = DV / DVS;       // value slices = 256-thread units per CTA
+    constexpr int NW = 8;              // warps per unit
     constexpr int LPR = DVS / 4;
     constexpr int RPW = 32 / LPR;
     constexpr int RP = NW * RPW;
     constexpr int NP = DK / RP;
     static_assert(DK % RP == 0 && DK <= 256 && DVS <= 256, "shape");
 
-    __shared__ float s_k[DK], s_q[DK], s_a[DK], s_v[DVS];
-    __shared__ float4 s_redk[NW][LPR], s_redq[NW][LPR];
-    __shared__ float s_red[NW];
-    __shared__ float s_kq, s_ss;
+    __shared__ float s_k[DK], s_q[DK], s_a[DK], s_v[NS][DVS];
+    __shared__ float4 s_redk[NS][NW][LPR], s_redq[NS][NW][LPR];
+    __shared__ float s_red[NS * NW];
+    __shared__ float s_kq, s_ss[NS];
 
-    cg::cluster_group cluster = cg::this_cluster();
-    const int rank = static_cast<int>(cluster.block_rank());
-    const int unit = static_cast<int>(blockIdx.x) / NS;  // (sequence, head)
+    const int unit = static_cast<int>(blockIdx.x);  // (sequence, head)
     const int n = unit / a.H, h = unit % a.H;
-    const int j0 = rank * DVS;
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int sl = static_cast<int>(threadIdx.x) >> 8;  // value slice of this thread's unit
+    const int j0 = sl * DVS;
+    const int t = threadIdx.x;
+    const int tid = t & 255, lane = tid & 31, w = tid >> 5;
     const int rw = lane / LPR, c4 = lane % LPR;
     float4* S = reinterpret_cast<float4*>(a.state + (size_t)unit * DK * DV + j0);
 
@@ -101,8 +95,8 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
         const int row = p * RP + w * RPW + rw;
         x[p] = __ldcs(S + row * (DV / 4) + c4);
     }
-    // 2. prologue: convolution + Swish of q, k (all DK channels, in every CTA
-    // of the cluster) and of this CTA's DVS value columns
+    // 2. prologue: convolution + Swish of q, k (threads t < DK, once per CTA)
+    // and of each unit's DVS value columns
     const TIn* xq = static_cast<const TIn*>(a.xq);
     const TIn* xk = static_cast<const TIn*>(a.xk);
     const TIn* xv = static_cast<const TIn*>(a.xv);
@@ -113,8 +107,8 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
     auto srow = [&](int i, int d) { return ((size_t)(n * 3 + i) * a.H + h) * d; };
     float nq[3] = {0.f, 0.f, 0.f}, nk[3] = {0.f, 0.f, 0.f}, nv[3] = {0.f, 0.f, 0.f};
     float yq = 0.f, yk = 0.f;
-    if (tid < DK) {
-        const int c = tid;
+    if (t < DK) {
+        const int c = t;
         const float4 wqv = *reinterpret_cast<const float4*>(a.wq + ((size_t)h * DK + c) * 4);
         const float4 wkv = *reinterpret_cast<const float4*>(a.wk + ((size_t)h * DK + c) * 4);
         const float q0 = to_f32(cq[srow(0, DK) + c]), q1 = to_f32(cq[srow(1, DK) + c]),
@@ -134,28 +128,25 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
         const float v0 = to_f32(cv[srow(0, DV) + c]), v1 = to_f32(cv[srow(1, DV) + c]),
                     v2 = to_f32(cv[srow(2, DV) + c]);
         const float vx = to_f32(xv[(size_t)unit * DV + c]);
-        s_v[tid] = swish_for<TIn>(wvv.x * v0 + wvv.y * v1 + wvv.z * v2 + wvv.w * vx);
+        s_v[sl][tid] = swish_for<TIn>(wvv.x * v0 + wvv.y * v1 + wvv.z * v2 + wvv.w * vx);
         nv[0] = v1; nv[1] = v2; nv[2] = vx;
     }
-    const float sq = block_sum<NW>(yq * yq, s_red);
-    const float sk = block_sum<NW>(yk * yk, s_red);
-    if (tid < DK) {
-        s_q[tid] = yq * rsqrtf(sq + a.l2_eps);
-        s_k[tid] = yk * rsqrtf(sk + a.l2_eps);
-    }
-    // every CTA of the cluster has read the old q / k states: rank 0 shifts them
-    cluster.sync();
-    if (tid < DK && rank == 0) {
+    const float sq = block_sum<NS * NW>(yq * yq, s_red);
+    const float sk = block_sum<NS * NW>(yk * yk, s_red);
+    // (block_sum ends with a barrier: every thread has read the old states)
+    if (t < DK) {
+        s_q[t] = yq * rsqrtf(sq + a.l2_eps);
+        s_k[t] = yk * rsqrtf(sk + a.l2_eps);
         for (int i = 0; i < 3; ++i) {
-            cq[srow(i, DK) + tid] = from_f32<TIn>(nq[i]);
-            ck[srow(i, DK) + tid] = from_f32<TIn>(nk[i]);
+            cq[srow(i, DK) + t] = from_f32<TIn>(nq[i]);
+            ck[srow(i, DK) + t] = from_f32<TIn>(nk[i]);
         }
     }
     if (tid < DVS) {
         for (int i = 0; i < 3; ++i) cv[srow(i, DV) + j0 + tid] = from_f32<TIn>(nv[i]);
     }
     __syncthreads();
-    if (w == 0) {
+    if (t < 32) {
         float kq = 0.f;
         for (int c = lane; c < DK; c += 32) kq += s_k[c] * s_q[c];
 #pragma unroll
@@ -184,23 +175,23 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
         pq.w += __shfl_xor_sync(0xffffffffu, pq.w, off);
     }
     if (rw == 0) {
-        s_redk[w][c4] = pk;
-        s_redq[w][c4] = pq;
+        s_redk[sl][w][c4] = pk;
+        s_redq[sl][w][c4] = pq;
     }
     __syncthreads();
     float4 rk = make_float4(0.f, 0.f, 0.f, 0.f), rq = rk;
 #pragma unroll
     for (int i = 0; i < NW; ++i) {
-        const float4 u = s_redk[i][c4], v = s_redq[i][c4];
+        const float4 u = s_redk[sl][i][c4], v = s_redq[sl][i][c4];
         rk.x += u.x; rk.y += u.y; rk.z += u.z; rk.w += u.w;
         rq.x += v.x; rq.y += v.y; rq.z += v.z; rq.w += v.w;
     }
     const float b = a.beta[unit];
     float4 u;
-    u.x = b * (s_v[4 * c4 + 0] - rk.x);
-    u.y = b * (s_v[4 * c4 + 1] - rk.y);
-    u.z = b * (s_v[4 * c4 + 2] - rk.z);
-    u.w = b * (s_v[4 * c4 + 3] - rk.w);
+    u.x = b * (s_v[sl][4 * c4 + 0] - rk.x);
+    u.y = b * (s_v[sl][4 * c4 + 1] - rk.y);
+    u.z = b * (s_v[sl][4 * c4 + 2] - rk.z);
+    u.w = b * (s_v[sl][4 * c4 + 3] - rk.w);
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const int row = p * RP + w * RPW + rw;
@@ -209,8 +200,8 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
         yv.x += kc * u.x; yv.y += kc * u.y; yv.z += kc * u.z; yv.w += kc * u.w;
         __stcs(S + row * (DV / 4) + c4, yv);
     }
-    // 4. epilogue: o of this slice (warp 0, lanes of row 0), its sum of squares
-    // published to the cluster, RMSNorm over all DV columns, weight and gate
+    // 4. epilogue: o of each slice (the unit's warp 0, lanes of row 0), the
+    // slices' sums of squares, RMSNorm over all DV columns, weight and gate
     float o4[4] = {0.f, 0.f, 0.f, 0.f};
     if (w == 0 && rw == 0) {
         const float kq = s_kq;
@@ -222,13 +213,13 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1)
             ss += __shfl_xor_sync((LPR == 32) ? 0xffffffffu : ((1u << LPR) - 1u), ss, off);
-        if (lane == 0) s_ss = ss;
+        if (lane == 0) s_ss[sl] = ss;
     }
-    cluster.sync();
+    __syncthreads();
     if (w == 0 && rw == 0) {
         float total = 0.f;
 #pragma unroll
-        for (int r = 0; r < NS; ++r) total += *cluster.map_shared_rank(&s_ss, r);
+        for (int r = 0; r < NS; ++r) total += s_ss[r];
         const float inv = rsqrtf(total / DV + a.rms_eps);
         const TIn* gate = static_cast<const TIn*>(a.gate);
         TIn* y = static_cast<TIn*>(a.y);
@@ -240,27 +231,13 @@ __global__ void __launch_bounds__(256, (DK * DVS <= 8192) ? 4 : 2)
                 o4[i] * inv * a.w_norm[j0 + 4 * c4 + i] * sigmoid_for<TIn>(gt));
         }
     }
-    // keep this CTA's shared memory until the partner has read s_ss
-    cluster.sync();
 }
 
 template <int DK, int DV, typename TIn>
 cudaError_t launch_layer_decode_t(const LayerDecodeArgs& a, int units, cudaStream_t st) {
     constexpr int DVS = (DV == 128) ? 64 : DV;
-    constexpr int NS = DV / DVS;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(units * NS);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = NS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, layer_decode_kernel<DK, DV, DVS, TIn>, a);
+    layer_decode_kernel<DK, DV, DVS, TIn><<<units, 256 * (DV / DVS), 0, st>>>(a);
+    return cudaGetLastError();
 }
 
 template <typename TIn>

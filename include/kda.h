@@ -405,8 +405,8 @@ kda_status_t kda_output_norm_gate(const void* o, const void* gate, const float* 
  * fused into its kernels: the intra-chunk kernel convolves and normalises the
  * q and k tiles it loads (the 3 rows before a chunk read from the previous
  * chunk), the chain kernel convolves its V tiles and writes y from the O
- * read-out (the two value-column halves of a chain form a thread-block
- * cluster and add their row sums of o^2 through distributed shared memory);
+ * read-out (the two value-column halves of a chain are the two units of one
+ * CTA and add their row sums of o^2 through its shared memory);
  * q, k, v and o never reach HBM.  Every other supported shape runs the three
  * steps one after another with q, k, v, o in the workspace.
  * In:  xq, xk [total, H, dk], xv [total, H, dv], gate [total, H, dv] (dtype);
@@ -444,9 +444,9 @@ kda_status_t kda_layer_chunk_fwd(const void* xq, const void* xk, const void* xv,
  * In/out: conv_q, conv_k [N, 3, H, dk], conv_v [N, 3, H, dv] (dtype) as for
  *      kda_qkv_conv_norm_step; state [N, H, dk, dv] fp32 as for kda_decode_step.
  * Out: y [N, H, dv] (dtype), not aliasing any input.
- * The value columns of a (sequence, head) are split over two CTAs of one
- * thread-block cluster when dv = 128 (they share the RMSNorm's sum over dv
- * through distributed shared memory).  Shapes: dk, dv in {32, 64, 128};
+ * The value columns of a (sequence, head) are split over the 256-thread units
+ * of one CTA when dv = 128 (they share the RMSNorm's sum over dv through its
+ * shared memory).  Shapes: dk, dv in {32, 64, 128};
  * N == 0 does nothing.  No workspace.
  */
 kda_status_t kda_layer_decode_step(const void* xq, const void* xk, const void* xv,
