@@ -17,5 +17,6 @@ from .kda import (  # noqa: F401
     kda_gdn_chunk_bwd_workspace_size, KDA_PLAN_SIMT,
     KDA_PLAN_SPLIT, KDA_PLAN_OVERLAP, kda_decode_step, kda_get_device_status, kda_num_chunks_upper_bound,
     load, status_string, kda_layer_decode_step, kda_test_overlap_flag_timeout,
-    kda_layer_chunk_fwd, kda_layer_chunk_fwd_workspace_size,
+    kda_layer_chunk_fwd, kda_layer_chunk_fwd_workspace_size, kda_chunk_state_maps,
+    kda_fold_segment_states,
 )

@@ -569,6 +569,42 @@ kda_status_t kda_chunk_split_chain(const void* v, const float* initial_state,
                                              static_cast<cudaStream_t>(stream), w.seq_order));
 }
 
+// ------------------------------------------- state maps of a prefill (CP)
+
+kda_status_t kda_chunk_state_maps(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* cu_seqlens, int B, int T,
+                                  int num_seqs, int H, float* M, float* Bm, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    Prefill p;
+    Workspace w;
+    kda_status_t s = split_prologue(cu_seqlens, B, T, num_seqs, H,
+                                    {q, k, v, (const void*)g, (const void*)beta, (const void*)M,
+                                     (const void*)Bm},
+                                    workspace, workspace_bytes, &p, &w);
+    if (s != KDA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int maxc = kda::max_chunks(p.total, p.N, kTcC);
+    s = begin_prefill(w, cu_seqlens, B, T, p.N, kTcC, maxc, st);
+    if (s != KDA_OK) return s;
+    return from_cuda(kda::launch_split_state_maps(q, k, v, g, beta, cu_seqlens, T, p.N, H,
+                                                  w.chunk_info, maxc, w.chunk_start, w.status,
+                                                  w.blobs, M, Bm, st, w.seq_order));
+}
+
+kda_status_t kda_fold_segment_states(const float* M, const float* Bm, const float* S0, int R,
+                                     int N, int H, int dk, int dv, int reverse, float* each,
+                                     float* final_state, void* stream) {
+    if (R < 0 || N < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_INVALID_ARG;
+    if (!final_state || !aligned16(final_state) || (S0 && !aligned16(S0))) return KDA_ERR_INVALID_ARG;
+    if (R > 0)
+        for (const void* ptr : {(const void*)M, (const void*)Bm, (const void*)each})
+            if (!ptr || !aligned16(ptr)) return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_fold_segments(M, Bm, S0, R, N * H, dk, dv, reverse != 0, each,
+                                               final_state, static_cast<cudaStream_t>(stream)));
+}
+
 // ----------------------------------------------------------------- decode
 
 kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const float* g,

@@ -963,7 +963,11 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
                        : launch_intra3<32, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st);
         if (e != cudaSuccess) return e;
     }
-    {
+    if (dk == 128 && dv == 128 && bwd_tc_available()) {
+        e = launch_bwd_chains_tc(w.W, b.Kb, w.G, h0, dhT, w.U, b.E, b.F, cu, T, N, H,
+                                 w.chunk_start, w.status, w.states, b.dU, b.dSx, dh0, st);
+        if (e != cudaSuccess) return e;
+    } else {
         const size_t sm = chain_smem();
         const dim3 grid(N, H, dv / kChainDVS);
         if ((e = set_smem(chain_kernel<false, TIn>, sm)) != cudaSuccess) return e;

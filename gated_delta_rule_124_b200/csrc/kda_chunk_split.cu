@@ -931,6 +931,10 @@ struct Params {
     const float* w_norm;
     float rms_eps;
     __nv_bfloat16* y;
+    // (state maps only) v taken as zero (V is not read, the Tb V product is
+    // not formed) and the entry state as the identity (h0 is not read)
+    bool zero_v;
+    bool identity_h0;
 };
 
 // (layer variant) V of the chunk from the raw inputs in place: the depthwise
@@ -1041,7 +1045,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         if (groups & 1) bulk_g2s(sm + ((n & 1) ? OFF_SC1 : OFF_SC0), b + BL_SC, 1024, bar_ld);
         if (groups & 2) {
             bulk_g2s(sm + OFF_TB, b + BL_TB, 8192, bar_ld);
-            tma_load_3d(sm + OFF_V, tmv, bar_ld, j0, h, t_begin + n * C);
+            if (!p.zero_v) tma_load_3d(sm + OFF_V, tmv, bar_ld, j0, h, t_begin + n * C);
             bulk_g2s(sm + OFF_WQ, b + BL_WQ, 32768, bar_ld);
         }
         if (groups & 4) {
@@ -1054,7 +1058,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         groups &= pend;
         if (!groups) return;
         if ((groups & 3) && !armed) {
-            mbar_arrive_expect_tx(bar_ld, TX_A);
+            mbar_arrive_expect_tx(bar_ld, p.zero_v ? TX_A - 8192 : TX_A);
             armed = true;
         }
         if ((groups & 4) && !armed3) {
@@ -1106,6 +1110,10 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
                            : make_float4(0.f, 0.f, 0.f, 0.f);
             x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
         }
+        if (p.identity_h0) {  // row c of the identity, this half's columns
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = (c == j0 + cq * 32 + i) ? 1.f : 0.f;
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
         tmem_st32(tbase + tlane + TM_S + cq * 32, r);
@@ -1143,7 +1151,7 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         tmem_ld32(tbase + tlane + tx(m) + cq * 32, v);
         tmem_wait_ld();
         if (!kLayer) {
-            if (r < LL) {
+            if (p.o && r < LL) {
                 __nv_bfloat16* dst = p.o + ((size_t)(tt0 + r) * p.H + h) * D + j0 + cq * 32;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
@@ -1216,15 +1224,18 @@ __device__ __forceinline__ void run(const CUtensorMap* tmv, const Params& p, uin
         // ---- [Ut ; 0] = [Tb ; 0] V, then += [-W ; Q*Gam] S  (one accumulator, N=64)
         constexpr uint32_t id1 = idesc_bf16_f32(128, DVS, false, true);
         if ((!kLayer || n > 0) && tid == 0) {  // (layer: V already convolved, below)
+            if (!p.zero_v) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
-                         sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id1, ks > 0);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_TB + ks * 32, 16, 1024),
+                             sdesc_sw128(sbase + OFF_V + ks * 2048, 8192, 1024), id1, ks > 0);
+            }
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int kb = ks >> 2, kk = ks & 3;
                 mma_bf16(tbase + tx(n), sdesc_sw128(sbase + OFF_WQ + kb * 16384 + kk * 32, 16, 1024),
-                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id1, 1);
+                         sdesc_sw128(sbase + OFF_SB + ks * 2048, 16384, 1024), id1,
+                         (p.zero_v && ks == 0) ? 0u : 1u);
             }
             mma_commit(bar_mma);
         }
@@ -1658,6 +1669,52 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
         return cudaErrorInvalidValue;
     chain::chunk_chain_layer_kernel<<<N * H, 2 * chain::NTC, chain::LAYER_SMEM, st>>>(mv, mgt,
                                                                                       pb);
+    return cudaGetLastError();
+}
+
+namespace {
+// dst[n, h] = I (dk = dv = 128): the state map of sequences without tokens.
+__global__ void identity_fill_kernel(float* dst, long long mats) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= mats * D * D) return;
+    const int e = static_cast<int>(i % (D * D));
+    dst[i] = (e / D == e % D) ? 1.f : 0.f;
+}
+}  // namespace
+
+cudaError_t launch_split_state_maps(const void* q, const void* k, const void* v, const float* g,
+                                    const float* beta, const int32_t* cu_seqlens, int T, int N,
+                                    int H, const int4* chunk_info, int maxc,
+                                    const int* chunk_start, uint32_t* status, void* blobs,
+                                    float* M, float* Bm, cudaStream_t st, const int* seq_order) {
+    const int total = cu_seqlens ? T : N * T;
+    if (total == 0) {
+        const long long mats = (long long)N * H;
+        cudaError_t e = cudaMemsetAsync(Bm, 0, sizeof(float) * (size_t)mats * D * D, st);
+        if (e != cudaSuccess) return e;
+        identity_fill_kernel<<<(unsigned)((mats * D * D + 255) / 256), 256, 0, st>>>(M, mats);
+        return cudaGetLastError();
+    }
+    cudaError_t e = launch_split_intra(q, k, g, beta, total, H, chunk_info, maxc, status, blobs,
+                                       st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mv;
+    if (!split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if ((e = set_smem_max_carveout(chain::chunk_chain_kernel, chain::SMEM_BYTES)) != cudaSuccess)
+        return e;
+    // B: from a zero state with the values; M: from the identity with zero values
+    chain::Params pb{nullptr, cu_seqlens, T, H, chunk_start, status, status,
+                     static_cast<const uint8_t*>(blobs), nullptr, Bm};
+    pb.order = seq_order;
+    chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    chain::Params pm = pb;
+    pm.hN = M;
+    pm.zero_v = true;
+    pm.identity_h0 = true;
+    chain::chunk_chain_kernel<<<2 * N * H, chain::NTC, chain::SMEM_BYTES, st>>>(mv, pm);
     return cudaGetLastError();
 }
 

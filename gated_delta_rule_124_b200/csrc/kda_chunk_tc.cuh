@@ -56,6 +56,17 @@ cudaError_t launch_split_chain(const void* v, const float* h0, const int32_t* cu
                                const void* blobs, void* o, float* hN, cudaStream_t st,
                                const int* seq_order = nullptr,
                                const LayerArgs* layer = nullptr);
+// The affine map of the prefill on the state, per (sequence, head): final
+// state = M S_0 + Bm (M = the product of the chunk transitions, dk x dk; Bm =
+// the final state from S_0 = 0): the intra-chunk kernel once, then the chain
+// kernel twice without outputs -- from a zero state with V (Bm) and from the
+// identity with V = 0 (M).
+cudaError_t launch_split_state_maps(const void* q, const void* k, const void* v, const float* g,
+                                    const float* beta, const int32_t* cu_seqlens, int T, int N,
+                                    int H, const int4* chunk_info, int maxc,
+                                    const int* chunk_start, uint32_t* status, void* blobs,
+                                    float* M, float* Bm, cudaStream_t st,
+                                    const int* seq_order = nullptr);
 // The two kernels co-scheduled in one cooperative launch (chains wait for the
 // blobs of their chunks through `flags`, one uint32 per (chunk slot, head)).
 // withheld_flag >= 0 (testing the bounded-wait error path only): the flag of

@@ -202,6 +202,20 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
                           const float* beta, float* state, void* o, int N, int H, int dk,
                           int dv, kda_dtype_t dt, cudaStream_t st, bool head_gate = false);
 size_t bwd_workspace_bytes(int total, int N, int H, int dk, int dv);
+// Composition of per-segment state maps (kda_segments.cu): forward entry
+// states, or (reverse) exit-state gradients; see kda_fold_segment_states.
+cudaError_t launch_fold_segments(const float* M, const float* Bm, const float* S0, int R, int NH,
+                                 int dk, int dv, bool reverse, float* each, float* fin,
+                                 cudaStream_t st);
+// The backward's two chains on the tensor cores (dk = dv = 128): the forward
+// pass (U in place of Ut, the entry state of every chunk) and the backward
+// pass (dU, the exit-state gradient of every chunk, dS_0); kda_bwd_tc.cu.
+bool bwd_tc_available();
+cudaError_t launch_bwd_chains_tc(const float* W, const float* Kb, const float* G, const float* S0,
+                                 const float* dS_end, float* U_in_out, const float* E,
+                                 const float* F, const int32_t* cu, int T, int N, int H,
+                                 const int* chunk_start, uint32_t* status, float* states,
+                                 float* dU, float* dSx, float* dS0, cudaStream_t st);
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* h0, const void* dout, const float* dhT,
                        const int32_t* cu, int T, int N, int H, int dk, int dv, kda_dtype_t dt,

@@ -268,6 +268,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major operand of 32-bit elements
+// (kind::tf32): the 128-byte swizzle with 32-byte granules (layout type 1),
+// whose atom is 4 rows of 128 bytes; LBO = byte stride between 128-byte
+// blocks along M/N, SBO = byte stride between groups of 4 rows along K.
+__device__ __forceinline__ uint64_t sdesc_sw128_32b(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100)
+    d |= static_cast<uint64_t>(1) << 61;  // SWIZZLE_128B_BASE32B
+    return d;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
                                                       bool b_mn_major) {
@@ -284,6 +299,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 // 128-byte-swizzled region whose base is 1024-byte aligned.
 __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// The same for the 128-byte swizzle with 32-byte granules (the layout TMA's
+// CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B writes): granule (chunk / 2) of row
+// `row` sits at granule (chunk / 2) ^ (row mod 4); base 512-byte aligned.
+__host__ __device__ __forceinline__ uint32_t sw128_32b_off(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((((chunk >> 1) ^ (row & 3u)) << 5) | ((chunk & 1u) << 4));
 }
 
 }  // namespace sm100

@@ -45,7 +45,7 @@ EXPORTS = (
     "kda_gdn_chunk_bwd_workspace_size", "kda_gdn_chunk_bwd", "kda_qkv_conv_norm_step",
     "kda_chunk_fwd_with_plan", "kda_chunk_fwd_plan_workspace_size",
     "kda_test_overlap_flag_timeout", "kda_layer_decode_step", "kda_layer_chunk_fwd",
-    "kda_layer_chunk_fwd_workspace_size",
+    "kda_layer_chunk_fwd_workspace_size", "kda_chunk_state_maps", "kda_fold_segment_states",
 )
 
 
@@ -92,6 +92,8 @@ _SIGS = {
     "kda_layer_chunk_fwd": ([_vp] * 10 + [_i] * 8 + [_vp, _vp] + [ctypes.c_float] * 2 +
                             [_vp, _vp, _vp, _sz, _vp], _i),
     "kda_layer_chunk_fwd_workspace_size": ([_i] * 7, _sz),
+    "kda_chunk_state_maps": ([_vp] * 6 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
+    "kda_fold_segment_states": ([_vp] * 3 + [_i] * 6 + [_vp, _vp, _vp], _i),
     "kda_chunk_split_chain": ([_vp] * 3 + [_i] * 4 + [_vp, _vp, _vp, _sz, _vp], _i),
 }
 
@@ -427,6 +429,25 @@ def kda_output_norm_gate(o, gate, w, total_tokens, H, dv, dtype, eps, y, stream=
     st = load().kda_output_norm_gate(_p(o), _p(gate), _p(w), total_tokens, H, dv,
                                      dtype_code(dtype), float(eps), _p(y), _stream(stream))
     return _ret(st, "kda_output_norm_gate", check)
+
+
+def kda_chunk_state_maps(q, k, v, g, beta, cu_seqlens, B, T, num_seqs, H, M, Bm, workspace,
+                         workspace_bytes=None, stream=None, check=True) -> int:
+    _check("kda_chunk_state_maps", "bf16", typed=(q, k, v), f32=(g, beta, M, Bm),
+           i32=(cu_seqlens,), raw=(workspace,))
+    wb = _nbytes(workspace) if workspace_bytes is None else workspace_bytes
+    st = load().kda_chunk_state_maps(_p(q), _p(k), _p(v), _p(g), _p(beta), _p(cu_seqlens), B, T,
+                                     num_seqs, H, _p(M), _p(Bm), _p(workspace), wb,
+                                     _stream(stream))
+    return _ret(st, "kda_chunk_state_maps", check)
+
+
+def kda_fold_segment_states(M, Bm, S0, R, N, H, dk, dv, reverse, each, final_state, stream=None,
+                            check=True) -> int:
+    _check("kda_fold_segment_states", None, f32=(M, Bm, S0, each, final_state))
+    st = load().kda_fold_segment_states(_p(M), _p(Bm), _p(S0), R, N, H, dk, dv, int(bool(reverse)),
+                                        _p(each), _p(final_state), _stream(stream))
+    return _ret(st, "kda_fold_segment_states", check)
 
 
 def kda_layer_chunk_fwd_workspace_size(total_tokens, num_seqs, H, dk, dv, chunk, dtype) -> int:

@@ -241,6 +241,45 @@ kda_status_t kda_chunk_split_chain(const void* v, const float* initial_state,
                                    void* o, float* final_state, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
+/* ------------------------------- affine state maps (context parallelism)
+ * Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
+ * algorithm": the state is carried recurrently between chunks, and over any
+ * span of tokens that carry is affine in the entry state, S_out = M S_in + B.
+ * A long sequence split over ranks by token ranges is therefore prefilled as:
+ * every rank computes its segment's (M, B), the ranks exchange them, every
+ * rank folds the maps before it into its entry state, and prefills its
+ * segment from that state.
+ *
+ * kda_chunk_state_maps: (M, B) of every (sequence, head) of a prefill, without
+ * its outputs: final_state = M initial_state + B, M [num_seqs, H, 128, 128]
+ * (the product of the transitions (I - beta k k^T) Diag(alpha), acting on the
+ * key side), B [num_seqs, H, 128, 128] (the final state from a zero initial
+ * state).  bf16 q, k, v, dk = dv = 128, chunk 64 (the split plan's shapes;
+ * otherwise KDA_ERR_UNSUPPORTED): the intra-chunk kernel once, then the chain
+ * kernel twice without outputs (from zero with v, from the identity with v
+ * taken as zero).  Other arguments and the workspace as kda_chunk_split_*.
+ */
+kda_status_t kda_chunk_state_maps(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const int32_t* cu_seqlens, int B, int T,
+                                  int num_seqs, int H, float* M, float* Bm, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* kda_fold_segment_states: composition of R segments' maps, per (sequence,
+ * head), on the CUDA cores in fp32.
+ *   reverse = 0: S_0 = S0 (NULL: zeros); each[r] = S_r (the entry state of
+ *     segment r); S_{r+1} = M_r S_r + Bm_r; final_state = S_R.
+ *   reverse != 0 (the backward): g_R = S0 (the final state's gradient; NULL:
+ *     zeros); each[r] = g_{r+1} (the gradient of segment r's exit state);
+ *     g_r = M_r^T g_{r+1} + Bm_r (Bm_r: the entry-state gradient segment r's
+ *     own outputs produce); final_state = g_0 (the initial state's gradient).
+ * In:  M [R, N, H, dk, dk], Bm [R, N, H, dk, dv], S0 [N, H, dk, dv] fp32.
+ * Out: each [R, N, H, dk, dv], final_state [N, H, dk, dv] fp32.
+ * Shapes: dk, dv in {32, 64, 128}; R >= 0 (R = 0: final_state = S0).
+ */
+kda_status_t kda_fold_segment_states(const float* M, const float* Bm, const float* S0, int R,
+                                     int N, int H, int dk, int dv, int reverse, float* each,
+                                     float* final_state, void* stream);
+
 /* ------------------------------------------------------------------- decode
  * kda_decode_step: one token per (sequence, head), state updated in place.
  *   Defining passages: Kimi Linear (aiwiki.ai), "Why linear attention exists"

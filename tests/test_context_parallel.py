@@ -37,6 +37,19 @@ def _oracle_backward(q, k, v, g, beta, initial_state, dout, dfinal_state):
     return tuple(torch.from_numpy(x).float().reshape(s) for x, s in zip(r, shp))
 
 
+def _host_fold(M, Bm, S0, reverse=False):
+    """The fold written out step by step on the host in fp64 (the test's own
+    composition of the maps; the product's fold is the library kernel)."""
+    M, Bm, S = M.double(), Bm.double(), S0.double()
+    R = M.shape[0]
+    each = [None] * R
+    for step in range(R):
+        r = R - 1 - step if reverse else step
+        each[r] = S.float()
+        S = (M[r].transpose(-1, -2) if reverse else M[r]) @ S + Bm[r]
+    return torch.stack(each), S.float()
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -58,7 +71,8 @@ def _worker(rank, world, port, out):
         T = q.shape[1]
         a, b = rank * T // world, (rank + 1) * T // world
         o, hN = cp.context_parallel_prefill(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b],
-                                            beta[:, a:b], h0, prefill=_oracle_prefill)
+                                            beta[:, a:b], h0, prefill=_oracle_prefill,
+                                            fold=_host_fold)
         out[rank] = (o.numpy(), hN.numpy())
     finally:
         dist.destroy_process_group()
@@ -88,7 +102,8 @@ def _bwd_worker(rank, world, port, out):
         a, b = rank * T // world, (rank + 1) * T // world
         grads = cp.context_parallel_backward(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b],
                                              beta[:, a:b], do[:, a:b], h0, dfin,
-                                             prefill=_oracle_prefill, backward=_oracle_backward)
+                                             prefill=_oracle_prefill, backward=_oracle_backward,
+                                             fold=_host_fold)
         out[rank] = tuple(x.numpy() for x in grads)
     finally:
         dist.destroy_process_group()
@@ -120,7 +135,7 @@ def test_fold_of_segment_maps_is_the_recurrence():
     cuts = [0, 13, 40, 60]
     maps = [cp.segment_maps(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b], beta[:, a:b],
                             _oracle_prefill) for a, b in zip(cuts, cuts[1:])]
-    entries, final = cp.entry_states(maps, h0)
+    entries, final = cp.entry_states(maps, h0, _host_fold)
     for i, a in enumerate(cuts[:-1]):
         if a == 0:
             ref = h0.numpy()
@@ -239,8 +254,8 @@ def test_reverse_fold_gives_the_boundary_state_gradients():
             for a, b in segs]
     offs = [_oracle_backward(*(part(x, a, b) for x in (q, k, v, g, beta)), None,
                              part(do, a, b), None)[5] for a, b in segs]
-    exits, dh0 = cp.exit_gradients(maps, offs, dfin)
-    entries, _ = cp.entry_states(maps, h0)
+    exits, dh0 = cp.exit_gradients(maps, offs, dfin, _host_fold)
+    entries, _ = cp.entry_states(maps, h0, _host_fold)
     for i, (a, b) in enumerate(segs):
         if b == 50:
             ref = dfin.numpy()
@@ -249,3 +264,80 @@ def test_reverse_fold_gives_the_boundary_state_gradients():
                                    entries[i + 1], part(do, b, 50), dfin)[5].numpy()
         assert rel_err(exits[i], ref) <= 1e-5, i
     assert rel_err(dh0, _oracle_backward(q, k, v, g, beta, h0, do, dfin)[5].numpy()) <= 1e-5
+
+
+@pytest.mark.gpu
+def test_state_maps_from_the_library_match_the_oracle_maps():
+    """kda_chunk_state_maps (one intra pass, two chain passes without outputs)
+    against the maps the fp64 oracle's two prefills give, on two 200-token
+    sequences (three full chunks and a ragged tail)."""
+    B, T, H, d = 2, 200, 2, 128
+    c = wl.make_prefill(25, [T] * B, H=H, dk=d, dv=d, chunk=64, dtype="bf16")
+    sh = lambda x, last: x.reshape(B, T, H, *last)  # noqa: E731
+    host = [sh(c.q, (d,)), sh(c.k, (d,)), sh(c.v, (d,)), sh(c.g, (d,)), sh(c.beta, ())]
+    m, bm = cp.segment_maps(*(x.cuda() for x in host))
+    rm, rb = cp.segment_maps(*host, _oracle_prefill)
+    assert rel_err(m.cpu(), rm.numpy()) <= 2e-2
+    assert rel_err(bm.cpu(), rb.numpy()) <= 2e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (32, 64)])
+@pytest.mark.parametrize("reverse", [False, True])
+def test_fold_kernel_matches_the_host_fold(dk, dv, reverse):
+    """kda_fold_segment_states against the fold written out in fp64, five
+    segments of random maps (contractive M, so the states stay bounded)."""
+    gen = torch.Generator().manual_seed(31 + dk + dv + reverse)
+    R, N, H = 5, 2, 3
+    M = torch.randn(R, N, H, dk, dk, generator=gen) / dk ** 0.5
+    Bm = torch.randn(R, N, H, dk, dv, generator=gen)
+    S0 = torch.randn(N, H, dk, dv, generator=gen)
+    each, fin = cp.library_fold(M.cuda(), Bm.cuda(), S0.cuda(), reverse)
+    re, rf = _host_fold(M, Bm, S0, reverse)
+    assert rel_err(each.cpu(), re.numpy()) <= 1e-5
+    assert rel_err(fin.cpu(), rf.numpy()) <= 1e-5
+
+
+@pytest.mark.gpu
+def test_fold_of_no_segments_returns_the_initial_state():
+    S0 = torch.randn(2, 2, 64, 64).cuda()
+    M = torch.zeros(0, 2, 2, 64, 64).cuda()
+    each, fin = cp.library_fold(M, torch.zeros(0, 2, 2, 64, 64).cuda(), S0, False)
+    assert each.shape[0] == 0 and torch.equal(fin, S0)
+
+
+def _gpu_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, T, H, d = 2, 512, 2, 128
+        c = wl.make_prefill(26, [T] * B, H=H, dk=d, dv=d, chunk=64, dtype="bf16")
+        a, b = rank * T // world, (rank + 1) * T // world
+        part = lambda x, last: x.reshape(B, T, H, *last)[:, a:b].contiguous().cuda()  # noqa: E731
+        o, hN = cp.context_parallel_prefill(part(c.q, (d,)), part(c.k, (d,)), part(c.v, (d,)),
+                                            part(c.g, (d,)), part(c.beta, ()),
+                                            c.initial_state.cuda())
+        torch.cuda.synchronize()
+        out[rank] = (o.float().cpu().numpy(), hN.cpu().numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_two_ranks_gloo_with_the_library_on_the_gpu():
+    """context_parallel_prefill with its defaults (the library's maps, fold
+    and prefill on cuda:0) in two processes exchanging over gloo, against the
+    oracle over the whole 512-token sequences.  The ranks' kernels never wait
+    on each other: the exchange is a host all-gather between them."""
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.spawn(_gpu_worker, args=(2, _free_port(), out), nprocs=2, join=True)
+    B, T, H, d = 2, 512, 2, 128
+    c = wl.make_prefill(26, [T] * B, H=H, dk=d, dv=d, chunk=64, dtype="bf16")
+    sh = lambda x, last: x.reshape(B, T, H, *last)  # noqa: E731
+    ro, rh = oracle.forward(sh(c.q, (d,)), sh(c.k, (d,)), sh(c.v, (d,)), sh(c.g, (d,)),
+                            sh(c.beta, ()), c.initial_state)
+    o = np.concatenate([out[0][0], out[1][0]], axis=1)
+    assert rel_err(o, ro) <= 2e-2
+    for r in range(2):
+        assert rel_err(out[r][1], rh) <= 2e-2
