@@ -107,7 +107,8 @@ __global__ void __launch_bounds__(256) bwd_apkb_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const float* __restrict__ g,
     const float* __restrict__ beta, const int4* __restrict__ info, int H,
     const uint32_t* status, float* __restrict__ G, float* __restrict__ Ar_out,
-    float* __restrict__ P_out, float* __restrict__ Kb, float* __restrict__ Rk) {
+    float* __restrict__ P_out, float* __restrict__ Kb, float* __restrict__ Rk, bool rt) {
+    // rt: P and Kb are tf32 operands of the tensor-core kernels after this one
     constexpr int LDK = DK + 1;
     if (status_bad(status)) return;
     const int cidx = blockIdx.x, h = blockIdx.y;
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(256) bwd_apkb_kernel(
             for (int y = 0; y < 4; ++y) {
                 const int i = i0 + y;
                 pa[y] = (r < L && i < r) ? aA[x][y] : 0.f;
-                pp[y] = (r < L && i <= r) ? aP[x][y] : 0.f;
+                pp[y] = (r < L && i <= r) ? (rt ? round_tf32(aP[x][y]) : aP[x][y]) : 0.f;
             }
             *reinterpret_cast<float4*>(Ac + r * CB + i0) = va;
             *reinterpret_cast<float4*>(Pc + r * CB + i0) = vp;
@@ -216,7 +217,8 @@ __global__ void __launch_bounds__(256) bwd_apkb_kernel(
         const int r = idx / DK, c = idx % DK;
         const size_t gi = row0 + r * rstride + c;
         const float gr = Gs[r * LDK + c], kr = Ks[r * LDK + c];
-        Kb[gi] = kr * __expf(Gs[(L - 1) * LDK + c] - gr);
+        const float kb = kr * __expf(Gs[(L - 1) * LDK + c] - gr);
+        Kb[gi] = rt ? round_tf32(kb) : kb;
         Rk[gi] = beta[(size_t)(ci.y + r) * H + h] * kr * __expf(gr);
     }
 }
@@ -225,7 +227,7 @@ template <int DK, typename TIn>
 __global__ void __launch_bounds__(256) bwd_subst_kernel(
     const TIn* __restrict__ v, const float* __restrict__ beta, const float* __restrict__ Ain,
     const int4* __restrict__ info, int H, int dv, const uint32_t* status,
-    float* __restrict__ W, float* __restrict__ Ut) {
+    float* __restrict__ W, float* __restrict__ Ut, bool rt) {  // rt: W rounded to tf32
     if (status_bad(status)) return;
     const int cidx = blockIdx.x, h = blockIdx.y;
     const int4 ci = info[cidx];
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(256) bwd_subst_kernel(
     __syncthreads();
     for (int idx = tid; idx < L * DK; idx += 256) {
         const int r = idx / DK, c = idx % DK;
-        W[((size_t)(ci.y + r) * H + h) * DK + c] = X[r * ldx + c];
+        W[((size_t)(ci.y + r) * H + h) * DK + c] = rt ? round_tf32(X[r * ldx + c]) : X[r * ldx + c];
     }
     for (int idx = tid; idx < L * dv; idx += 256) {
         const int r = idx / dv, j = idx % dv;
@@ -562,7 +564,8 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
     const float* __restrict__ beta, const float* __restrict__ U,
     const float* __restrict__ dU, const int4* __restrict__ info, int H, int dv,
     const uint32_t* status, float* __restrict__ Y, float* __restrict__ dv_out,
-    float* __restrict__ dAr, float* __restrict__ dP, float* __restrict__ dbB) {
+    float* __restrict__ dAr, float* __restrict__ dP, float* __restrict__ dbB, bool rt) {
+    // rt: Y is written rounded to tf32 (an operand of the tensor-core dense kernel)
     if (status_bad(status)) return;
     const int cidx = blockIdx.x, h = blockIdx.y;
     const int4 ci = info[cidx];
@@ -637,7 +640,7 @@ __global__ void __launch_bounds__(256) bwd_solve_kernel(
     for (int idx = tid; idx < L * dv; idx += nt) {
         const int r = idx / dv, j = idx % dv;
         const size_t vi = ((size_t)(ci.y + r) * H + h) * dv + j;
-        Y[vi] = Ys[r * ldy + j];
+        Y[vi] = rt ? round_tf32(Ys[r * ldy + j]) : Ys[r * ldy + j];
         dv_out[vi] = bs[r] * Ys[r * ldy + j];
     }
     // dA[i][j] = -(Y U^T)[i][j] (j < i), dP[i][j] = (dO U^T)[i][j] (j <= i):
@@ -924,20 +927,23 @@ cudaError_t launch_dense(const BwdBufs& b, const TIn* K, const TIn* DO, const fl
 template <int DK, typename TIn>
 cudaError_t launch_intra3(const BwdBufs& b, const TIn* Q, const TIn* K, const TIn* V,
                           const TIn* DO, const float* g, const float* beta, int maxc, int H,
-                          int dv, cudaStream_t st) {
+                          int dv, int total, bool tc, cudaStream_t st) {
     const Workspace& w = b.w;
     const dim3 grid(maxc, H);
     cudaError_t e;
     size_t sm = apkb_smem(DK);
     if ((e = set_smem(bwd_apkb_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
     bwd_apkb_kernel<DK, TIn><<<grid, 256, sm, st>>>(Q, K, g, beta, w.chunk_info, H, w.status,
-                                                    w.G, b.Ar, b.Pm, b.Kb, w.W);
+                                                    w.G, b.Ar, b.Pm, b.Kb, w.W, tc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     sm = subst_smem(DK, dv);
     if ((e = set_smem(bwd_subst_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
     bwd_subst_kernel<DK, TIn><<<grid, 256, sm, st>>>(V, beta, b.Ar, w.chunk_info, H, dv,
-                                                     w.status, w.W, w.U);
+                                                     w.status, w.W, w.U, tc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (tc)
+        return launch_bwd_ef_tc<TIn>(Q, DO, w.G, b.Pm, w.W, w.chunk_info, total, maxc, H,
+                                     w.status, b.E, b.F, st);
     sm = ef_smem(DK);
     if ((e = set_smem(bwd_ef_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
     bwd_ef_kernel<DK, TIn><<<grid, 256, sm, st>>>(Q, DO, w.G, b.Pm, w.W, w.chunk_info, H, dv,
@@ -956,14 +962,17 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
     const TIn* V = static_cast<const TIn*>(v);
     const TIn* DO = static_cast<const TIn*>(dout);
     const Workspace& w = b.w;
+    const int total = cu ? T : N * T;
+    // dk = dv = 128: the chains, E/F and the dense products on the tensor cores
+    const bool tc = dk == 128 && dv == 128 && bwd_tc_available();
     cudaError_t e;
     if (maxc > 0) {
-        e = dk == 128 ? launch_intra3<128, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st)
-            : dk == 64 ? launch_intra3<64, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st)
-                       : launch_intra3<32, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, st);
+        e = dk == 128 ? launch_intra3<128, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, total, tc, st)
+            : dk == 64 ? launch_intra3<64, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, total, tc, st)
+                       : launch_intra3<32, TIn>(b, Q, K, V, DO, g, beta, maxc, H, dv, total, tc, st);
         if (e != cudaSuccess) return e;
     }
-    if (dk == 128 && dv == 128 && bwd_tc_available()) {
+    if (tc) {
         e = launch_bwd_chains_tc(w.W, b.Kb, w.G, h0, dhT, w.U, b.E, b.F, cu, T, N, H,
                                  w.chunk_start, w.status, w.states, b.dU, b.dSx, dh0, st);
         if (e != cudaSuccess) return e;
@@ -989,10 +998,13 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
         if ((e = set_smem(bwd_solve_kernel<TIn>, sm)) != cudaSuccess) return e;
         bwd_solve_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(V, DO, b.Ar, beta, w.U, b.dU,
                                                              w.chunk_info, H, dv, w.status, b.Y,
-                                                             dvv, b.dAr, b.dP, b.dbB);
+                                                             dvv, b.dAr, b.dP, b.dbB, tc);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    e = dk == 128 ? launch_dense<128, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
+    e = tc ? launch_bwd_dense_tc<TIn>(K, DO, w.G, beta, w.U, b.Y, w.states, b.dSx, b.dbB,
+                                      w.chunk_info, total, maxc, H, w.status, b.dQt, b.dKt,
+                                      b.dKb, b.dGam, db, st)
+        : dk == 128 ? launch_dense<128, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
         : dk == 64 ? launch_dense<64, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
                    : launch_dense<32, TIn>(b, K, DO, beta, maxc, H, dv, db, st);
     if (e != cudaSuccess) return e;

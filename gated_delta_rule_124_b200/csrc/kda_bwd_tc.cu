@@ -1,6 +1,7 @@
-// The two serial chains of the chunked KDA backward on the 5th-generation
-// tensor cores (tcgen05, kind::tf32, accumulators in tensor memory), for
-// dk = dv = 128 and chunks of 64 tokens.  See kda_bwd.cu for the derivation
+// The contractions of the chunked KDA backward on the 5th-generation tensor
+// cores (tcgen05, kind::tf32, accumulators in tensor memory), for dk = dv =
+// 128 and chunks of 64 tokens: the two serial chains, E and F, and the dense
+// products after the back substitution.  See kda_bwd.cu for the derivation
 // (Kimi Linear (aiwiki.ai), "The constrained DPLR form and the chunkwise
 // algorithm", differentiated).  Per (sequence, head) and half of the value
 // columns, over the chunks of the sequence:
@@ -94,11 +95,13 @@ struct ChainArgs {
     float* S_end;          // forward: NULL; backward: dS_0 (or NULL)
 };
 
+// One 32-value row of an MN-major tf32 operand block, rounded to tf32.
 __device__ __forceinline__ void store_row32(uint8_t* blk, int row, const float (&x)[32]) {
 #pragma unroll
     for (int q = 0; q < 8; ++q)
         *reinterpret_cast<float4*>(blk + sw128_32b_off(row, q)) =
-            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            make_float4(round_tf32(x[4 * q]), round_tf32(x[4 * q + 1]), round_tf32(x[4 * q + 2]),
+                        round_tf32(x[4 * q + 3]));
 }
 
 template <bool kBack>
@@ -201,12 +204,13 @@ __global__ void __launch_bounds__(NTB, 1)
             }
         }
         const float gam = expf(a.G[((size_t)(t0 + L - 1) * a.H + h) * DD + trow]);
-        {  // the state entering this step
+        {  // the state entering this step (a tf32 operand of the dense kernel)
             float* dst = a.per_chunk + cbase + (size_t)trow * DD + j0 + 32 * cq;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4*>(dst + i) =
-                    make_float4(st[i], st[i + 1], st[i + 2], st[i + 3]);
+                    make_float4(round_tf32(st[i]), round_tf32(st[i + 1]), round_tf32(st[i + 2]),
+                                round_tf32(st[i + 3]));
         }
         bool ok = mbar_wait(bar_ld + s, (step >> 1) & 1, kWaitNs);
         if (__syncthreads_or(!ok)) {
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const float x = __uint_as_float(v[i]);
-                m[i] = row_ok ? (kBack ? x : base[i] - x) : 0.f;
+                m[i] = row_ok ? (kBack ? x : round_tf32(base[i] - x)) : 0.f;
             }
             if (row_ok) {
                 float* dst = a.rows_out + ((size_t)(t0 + trow) * a.H + h) * DD + j0 + 32 * cq;
@@ -311,6 +315,457 @@ __global__ void __launch_bounds__(NTB, 1)
     if (warp == 0) tmem_dealloc(tbase, 128);
 }
 
+// ------------------------------------------------------------ E and F
+// Per (chunk, head): E = P^T dO [64 tokens][128] and F = Qt^T dO - W^T E
+// [128 channels][128], the value columns in two halves of 64.  Every operand
+// is MN-major (the token index is K): P [r][i] (M = i, padded to 128 rows,
+// whose results are never read), Qt and W [r][c] (M = c), dO and -E [r][j]
+// (N = j), all in the 32-byte-granule swizzle.  Per half: E and the Qt^T dO
+// part of F in one commit; -E replaces dO in shared memory; then W^T (-E)
+// accumulates into F.  P and W come by TMA, Qt = q exp(G) and dO (widened
+// to fp32) are written by the threads.
+namespace ef {
+constexpr uint32_t OFF_P = 0;          // P: 2 blocks [64 r][32 i]
+constexpr uint32_t OFF_D = 16384;      // dO, then -E, of the half: 2 blocks [64 r][32 j]
+constexpr uint32_t OFF_Q = 32768;      // Qt: 4 blocks [64 r][32 c]
+constexpr uint32_t OFF_W = 65536;      // W: 4 blocks [64 r][32 c]
+constexpr uint32_t OFF_BAR = 98304;
+constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+constexpr uint32_t TM_E = 0, TM_F = 128;  // half jh at +64 jh
+}  // namespace ef
+
+// Store 16 consecutive fp32 values of row `row` (16-byte chunks q0 .. q0 + 3)
+// into a [rows][32] block in the 32-byte-granule swizzle.
+// (rounded to tf32)
+__device__ __forceinline__ void store16_32b(uint8_t* blk, int row, int q0, const float (&x)[16]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<float4*>(blk + sw128_32b_off(row, q0 + q)) =
+            make_float4(round_tf32(x[4 * q]), round_tf32(x[4 * q + 1]), round_tf32(x[4 * q + 2]),
+                        round_tf32(x[4 * q + 3]));
+}
+
+template <typename TIn>
+__device__ __forceinline__ void load16_f32(const TIn* src, float (&x)[16]);
+template <>
+__device__ __forceinline__ void load16_f32<float>(const float* src, float (&x)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src + i);
+        x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+    }
+}
+template <>
+__device__ __forceinline__ void load16_f32<__nv_bfloat16>(const __nv_bfloat16* src,
+                                                          float (&x)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            x[i + 2 * p] = __uint_as_float(w[p] << 16);
+            x[i + 2 * p + 1] = __uint_as_float(w[p] & 0xFFFF0000u);
+        }
+    }
+}
+
+struct EfArgs {
+    const void* q;
+    const void* dout;
+    const float* G;
+    const int4* info;  // per chunk slot: (sequence, first token, rows, -)
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    float* E;  // [total, H, 128]
+    float* F;  // [chunks, H, 128, 128]
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(NTB, 1)
+    ef_tc_kernel(const __grid_constant__ CUtensorMap tmp, const __grid_constant__ CUtensorMap tmw,
+                 const EfArgs a) {
+    using namespace ef;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_skip;
+    const int cidx = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int4 ci = a.info[cidx];
+    const int t0 = ci.y, L = ci.z;
+    if (tid == 0) s_skip = status_bad(a.status) || L <= 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + ef::OFF_BAR);
+    uint64_t* bar_mma = bar_ld + 1;
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cw = warp >> 2;
+    const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
+    const TIn* Qg = static_cast<const TIn*>(a.q);
+    const TIn* Dg = static_cast<const TIn*>(a.dout);
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_ld, 16384 + 32768);
+        tma_load_3d(sm + OFF_P, &tmp, bar_ld, 0, 0, cidx * a.H + h);
+        tma_load_3d(sm + OFF_P + 8192, &tmp, bar_ld, 32, 0, cidx * a.H + h);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb)
+            tma_load_3d(sm + OFF_W + kb * 8192, &tmw, bar_ld, 32 * kb, h, t0);
+    }
+    // Qt = q exp(G): row r = tid / 4, channels 32 (tid % 4) .. + 31 (block tid % 4)
+    {
+        const int r = tid >> 2, kb = tid & 3;
+        const bool ok = r < L;
+        const size_t gi = ((size_t)(t0 + r) * a.H + h) * DD + 32 * kb;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float x[16], gv[16];
+            if (ok) {
+                load16_f32<TIn>(Qg + gi + 16 * half, x);
+                load16_f32<float>(a.G + gi + 16 * half, gv);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] *= __expf(gv[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = 0.f;
+            }
+            store16_32b(sm + OFF_Q + kb * 8192, r, 4 * half, x);
+        }
+    }
+    const uint32_t tbase = s_tmem;
+    bool failed = false;
+    uint32_t mma_phase = 0;
+    constexpr uint32_t idn = idesc_tf32(128, 64, true, true);
+    for (int jh = 0; jh < 2 && !failed; ++jh) {
+        // dO of this half: row r = tid / 4, columns 64 jh + 16 (tid % 4) .. + 15
+        {
+            const int r = tid >> 2, part = tid & 3;
+            float x[16];
+            if (r < L) {
+                load16_f32<TIn>(Dg + ((size_t)(t0 + r) * a.H + h) * DD + 64 * jh + 16 * part, x);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = 0.f;
+            }
+            store16_32b(sm + OFF_D + (part >> 1) * 8192, r, 4 * (part & 1), x);
+        }
+        fence_async_smem();
+        bool ok = jh > 0 || mbar_wait(bar_ld, 0, kWaitNs);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_tf32_tc(tbase + TM_E + 64 * jh, sdesc_sw128_32b(sbase + OFF_P + ks * 1024, 8192, 512),
+                            sdesc_sw128_32b(sbase + OFF_D + ks * 1024, 8192, 512), idn, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_tf32_tc(tbase + TM_F + 64 * jh, sdesc_sw128_32b(sbase + OFF_Q + ks * 1024, 8192, 512),
+                            sdesc_sw128_32b(sbase + OFF_D + ks * 1024, 8192, 512), idn, ks > 0);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ++mma_phase;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+        // E rows (token i = lane of quarters 0, 1), 32 columns per warp: to
+        // global, and -E over dO in shared memory
+        if (quarter < 2) {
+            const int i = 32 * quarter + lane;
+            uint32_t v[32];
+            tmem_ld32(tbase + tlane + TM_E + 64 * jh + 32 * cw, v);
+            tmem_wait_ld();
+            float e[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) e[x] = i < L ? __uint_as_float(v[x]) : 0.f;
+            if (i < L) {
+                float* dst = a.E + ((size_t)(t0 + i) * a.H + h) * DD + 64 * jh + 32 * cw;
+#pragma unroll
+                for (int x = 0; x < 32; x += 4)
+                    *reinterpret_cast<float4*>(dst + x) = make_float4(e[x], e[x + 1], e[x + 2], e[x + 3]);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<float4*>(sm + OFF_D + cw * 8192 + sw128_32b_off(i, q)) =
+                    make_float4(-round_tf32(e[4 * q]), -round_tf32(e[4 * q + 1]),
+                                -round_tf32(e[4 * q + 2]), -round_tf32(e[4 * q + 3]));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_tf32_tc(tbase + TM_F + 64 * jh, sdesc_sw128_32b(sbase + OFF_W + ks * 1024, 8192, 512),
+                            sdesc_sw128_32b(sbase + OFF_D + ks * 1024, 8192, 512), idn, 1);
+            mma_commit(bar_mma);
+        }
+        ok = mbar_wait(bar_mma, mma_phase & 1, kWaitNs);
+        ++mma_phase;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        tc_fence_after();
+    }
+    if (!failed) {  // F: channel c = lane of the warp's quarter, 64 columns per warp
+        const int c = 32 * quarter + lane;
+        float* dst = a.F + (((size_t)cidx * a.H + h) * DD + c) * DD + 64 * cw;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            uint32_t v[32];
+            tmem_ld32(tbase + tlane + TM_F + 64 * cw + 32 * x, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int y = 0; y < 32; y += 4)
+                *reinterpret_cast<float4*>(dst + 32 * x + y) =
+                    make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+        }
+    } else if (tid == 0) {
+        if (mma_phase > 0) mbar_wait(bar_mma, (mma_phase - 1) & 1, kWaitNs);
+        mbar_wait(bar_ld, 0, kWaitNs);
+        atomicOr(a.status_out, STATUS_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
+// ------------------------------------------------------------ dense
+// Per (chunk, head), after the back substitution: [dO ; Y] S^T (one M = 128
+// product: rows 0-63 dQt = dO S^T, rows 64-127 Y S^T) and U dS'^T (M = 64
+// padded to 128), over the value columns in four quarters of 32 (K).  All
+// operands K-major in the 16-byte-granule swizzle: dO widened to fp32 by the
+// threads; Y, U, S and dS' by TMA.  Epilogue: dQt, dKt = -b (Y S^T), dKb =
+// U dS'^T, dbeta = dbB - sum_c Kt (Y S^T), and dGam = rowsum(S * dS') from
+// the staged quarters.
+namespace dn {
+constexpr uint32_t OFF_A = 0;       // [dO ; Y] quarter [128][32]
+constexpr uint32_t OFF_U = 16384;   // U quarter [64][32]; padding rows read OFF_S
+constexpr uint32_t OFF_S = 24576;   // S quarter [128 c][32 j]
+constexpr uint32_t OFF_X = 40960;   // dS' quarter [128 c][32 j]
+constexpr uint32_t OFF_RED = 57344; // dbeta partials [2][64]
+constexpr uint32_t OFF_BAR = OFF_RED + 512;
+constexpr uint32_t SMEM_USED = OFF_BAR + 64 + 1024;
+// requested size: at most two CTAs per SM (each holds 256 tensor-memory columns)
+constexpr uint32_t SMEM = 96 * 1024;
+static_assert(SMEM_USED <= SMEM, "dense tile");
+constexpr uint32_t TM_1 = 0, TM_2 = 128;
+}  // namespace dn
+
+struct DenseArgs {
+    const void* k;
+    const void* dout;
+    const float* G;
+    const float* beta;
+    const float* dbB;
+    const int4* info;
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    float* dQt;
+    float* dKt;
+    float* dKb;
+    float* dGam;
+    float* dbeta;
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(NTB, 1)
+    dense_tc_kernel(const __grid_constant__ CUtensorMap tmy, const __grid_constant__ CUtensorMap tmu,
+                    const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmx,
+                    const DenseArgs a) {
+    using namespace dn;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_skip;
+    const int cidx = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int4 ci = a.info[cidx];
+    const int t0 = ci.y, L = ci.z;
+    if (tid == 0) s_skip = status_bad(a.status) || L <= 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + dn::OFF_BAR);
+    uint64_t* bar_mma = bar_ld + 1;
+    float* s_red = reinterpret_cast<float*>(sm + OFF_RED);
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cw = warp >> 2;
+    const uint32_t tlane = static_cast<uint32_t>(32 * quarter) << 16;
+    const TIn* Dg = static_cast<const TIn*>(a.dout);
+    const TIn* Kg = static_cast<const TIn*>(a.k);
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const uint32_t tbase = s_tmem;
+    const int mat = cidx * a.H + h;
+    bool failed = false;
+    int fail_ld = -1, fail_mma = -1;  // the quarter whose copies / products were in flight
+    float gam = 0.f;
+    constexpr uint32_t idk = idesc_tf32(128, 128, false, false);
+    for (int qk = 0; qk < 4; ++qk) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar_ld, 8192 + 8192 + 16384 + 16384);
+            tma_load_3d(sm + OFF_A + 8192, &tmy, bar_ld, 32 * qk, h, t0);
+            tma_load_3d(sm + OFF_U, &tmu, bar_ld, 32 * qk, h, t0);
+            tma_load_3d(sm + OFF_S, &tms, bar_ld, 32 * qk, 0, mat);
+            tma_load_3d(sm + OFF_X, &tmx, bar_ld, 32 * qk, 0, mat);
+        }
+        {  // dO quarter: row r = tid / 4, columns 32 qk + 8 (tid % 4) .. + 7
+            const int r = tid >> 2, part = tid & 3;
+            float x[16];
+            if (r < L) {
+                const TIn* src = Dg + ((size_t)(t0 + r) * a.H + h) * DD + 32 * qk + 8 * part;
+                if constexpr (sizeof(TIn) == 2) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(src);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        x[2 * p] = __uint_as_float(w[p] << 16);
+                        x[2 * p + 1] = __uint_as_float(w[p] & 0xFFFF0000u);
+                    }
+                } else {
+                    const float4 v0 = *reinterpret_cast<const float4*>(src);
+                    const float4 v1 = *reinterpret_cast<const float4*>(src + 4);
+                    x[0] = v0.x; x[1] = v0.y; x[2] = v0.z; x[3] = v0.w;
+                    x[4] = v1.x; x[5] = v1.y; x[6] = v1.z; x[7] = v1.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] = 0.f;
+            }
+            *reinterpret_cast<float4*>(sm + OFF_A + sw128_off(r, 2 * part)) =
+                make_float4(round_tf32(x[0]), round_tf32(x[1]), round_tf32(x[2]), round_tf32(x[3]));
+            *reinterpret_cast<float4*>(sm + OFF_A + sw128_off(r, 2 * part + 1)) =
+                make_float4(round_tf32(x[4]), round_tf32(x[5]), round_tf32(x[6]), round_tf32(x[7]));
+        }
+        fence_async_smem();
+        bool ok = mbar_wait(bar_ld, qk & 1, kWaitNs);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            fail_ld = qk;
+            break;
+        }
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (qk | kk) > 0;
+                mma_tf32_tc(tbase + TM_1, sdesc_sw128(sbase + OFF_A + kk * 32, 16, 1024),
+                            sdesc_sw128(sbase + OFF_S + kk * 32, 16, 1024), idk, acc);
+                mma_tf32_tc(tbase + TM_2, sdesc_sw128(sbase + OFF_U + kk * 32, 16, 1024),
+                            sdesc_sw128(sbase + OFF_X + kk * 32, 16, 1024), idk, acc);
+            }
+            mma_commit(bar_mma);
+        }
+        if (tid < DD) {  // dGam: channel tid, this quarter's 32 columns
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 sv = *reinterpret_cast<const float4*>(sm + OFF_S + sw128_off(tid, q));
+                const float4 xv = *reinterpret_cast<const float4*>(sm + OFF_X + sw128_off(tid, q));
+                gam += sv.x * xv.x + sv.y * xv.y + sv.z * xv.z + sv.w * xv.w;
+            }
+        }
+        ok = mbar_wait(bar_mma, qk & 1, kWaitNs);
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            fail_mma = qk;
+            break;
+        }
+        tc_fence_after();
+    }
+    if (!failed) {
+        if (tid < DD) a.dGam[(size_t)mat * DD + tid] = gam;
+        const int r = 32 * (quarter & 1) + lane;  // token row of this thread
+        const bool row_ok = r < L;
+        const size_t row = ((size_t)(t0 + r) * a.H + h) * DD + 64 * cw;
+        float part = 0.f;
+        float b = 0.f;
+        if (quarter >= 2 && row_ok) b = a.beta[(size_t)(t0 + r) * a.H + h];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            uint32_t v[32];
+            tmem_ld32(tbase + tlane + TM_1 + 64 * cw + 32 * x, v);
+            tmem_wait_ld();
+            if (quarter < 2) {  // dQt = dO S^T
+                if (row_ok) {
+#pragma unroll
+                    for (int y = 0; y < 32; y += 4)
+                        *reinterpret_cast<float4*>(a.dQt + row + 32 * x + y) =
+                            make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                        __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+                }
+            } else if (row_ok) {  // Y S^T: dKt and the Kt . (Y S^T) part of dbeta
+                float kv[16], gv[16];
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    load16_f32<TIn>(Kg + row + 32 * x + 16 * hf, kv);
+                    load16_f32<float>(a.G + row + 32 * x + 16 * hf, gv);
+#pragma unroll
+                    for (int y = 0; y < 16; ++y)
+                        part += kv[y] * expf(gv[y]) * __uint_as_float(v[16 * hf + y]);
+                }
+#pragma unroll
+                for (int y = 0; y < 32; y += 4)
+                    *reinterpret_cast<float4*>(a.dKt + row + 32 * x + y) =
+                        make_float4(-b * __uint_as_float(v[y]), -b * __uint_as_float(v[y + 1]),
+                                    -b * __uint_as_float(v[y + 2]), -b * __uint_as_float(v[y + 3]));
+            }
+            if (quarter < 2) {  // dKb = U dS'^T
+                tmem_ld32(tbase + tlane + TM_2 + 64 * cw + 32 * x, v);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int y = 0; y < 32; y += 4)
+                        *reinterpret_cast<float4*>(a.dKb + row + 32 * x + y) =
+                            make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                        __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+                }
+            }
+        }
+        if (quarter >= 2) s_red[cw * 64 + r] = part;
+        __syncthreads();
+        if (quarter >= 2 && cw == 0 && row_ok) {
+            const size_t bi = (size_t)(t0 + r) * a.H + h;
+            a.dbeta[bi] = a.dbB[bi] - (s_red[r] + s_red[64 + r]);
+        }
+    } else if (tid == 0) {  // wait (bounded) for what is still in flight
+        if (fail_ld >= 0) mbar_wait(bar_ld, fail_ld & 1, kWaitNs);
+        if (fail_mma >= 0) mbar_wait(bar_mma, fail_mma & 1, kWaitNs);
+        atomicOr(a.status_out, STATUS_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void* ptr = nullptr;
@@ -332,6 +787,23 @@ bool map_f32_rows(CUtensorMap* m, const float* base, int total, int H, bool mn_m
     cuuint64_t dims[3] = {(cuuint64_t)DD, (cuuint64_t)H, (cuuint64_t)total};
     cuuint64_t strides[2] = {(cuuint64_t)DD * 4, (cuuint64_t)DD * 4 * H};
     cuuint32_t box[3] = {32, 1, (cuuint32_t)CB};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 [count][rows][cols] per-chunk matrices read as boxes of 32 columns x
+// all rows of one matrix, in either swizzle.
+bool map_f32_mats(CUtensorMap* m, const float* base, int count, int rows, int cols,
+                  bool mn_major) {
+    auto fn = bwd_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)count};
+    cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)cols * rows * 4};
+    cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -378,5 +850,62 @@ cudaError_t launch_bwd_chains_tc(const float* W, const float* Kb, const float* G
     chain_tc_kernel<true><<<grid, NTB, SMEM, st>>>(mw_mn, mkb_k, ba);
     return cudaGetLastError();
 }
+
+}  // namespace kda
+
+namespace kda {
+
+template <typename TIn>
+cudaError_t launch_bwd_ef_tc(const TIn* q, const TIn* dout, const float* G, const float* P,
+                             const float* W, const int4* info, int total, int maxc, int H,
+                             uint32_t* status, float* E, float* F, cudaStream_t st) {
+    if (maxc == 0 || total == 0) return cudaSuccess;
+    CUtensorMap mp, mw;
+    if (!map_f32_mats(&mp, P, maxc * H, 64, 64, true) || !map_f32_rows(&mw, W, total, H, true))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(ef_tc_kernel<TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ef::SMEM);
+    if (e != cudaSuccess) return e;
+    const EfArgs a{q, dout, G, info, H, status, status, E, F};
+    ef_tc_kernel<TIn><<<dim3(maxc, H), NTB, ef::SMEM, st>>>(mp, mw, a);
+    return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t launch_bwd_dense_tc(const TIn* k, const TIn* dout, const float* G, const float* beta,
+                                const float* U, const float* Y, const float* states,
+                                const float* dSx, const float* dbB, const int4* info, int total,
+                                int maxc, int H, uint32_t* status, float* dQt, float* dKt,
+                                float* dKb, float* dGam, float* dbeta, cudaStream_t st) {
+    if (maxc == 0 || total == 0) return cudaSuccess;
+    CUtensorMap my, mu, ms, mx;
+    if (!map_f32_rows(&my, Y, total, H, false) || !map_f32_rows(&mu, U, total, H, false) ||
+        !map_f32_mats(&ms, states, maxc * H, 128, 128, false) ||
+        !map_f32_mats(&mx, dSx, maxc * H, 128, 128, false))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(dense_tc_kernel<TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn::SMEM);
+    if (e != cudaSuccess) return e;
+    const DenseArgs a{k, dout, G, beta, dbB, info, H, status, status, dQt, dKt, dKb, dGam, dbeta};
+    dense_tc_kernel<TIn><<<dim3(maxc, H), NTB, dn::SMEM, st>>>(my, mu, ms, mx, a);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_bwd_ef_tc<float>(const float*, const float*, const float*,
+                                             const float*, const float*, const int4*, int, int,
+                                             int, uint32_t*, float*, float*, cudaStream_t);
+template cudaError_t launch_bwd_ef_tc<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                     const float*, const float*, const float*,
+                                                     const int4*, int, int, int, uint32_t*,
+                                                     float*, float*, cudaStream_t);
+template cudaError_t launch_bwd_dense_tc<float>(const float*, const float*, const float*,
+                                                const float*, const float*, const float*,
+                                                const float*, const float*, const float*,
+                                                const int4*, int, int, int, uint32_t*, float*,
+                                                float*, float*, float*, float*, cudaStream_t);
+template cudaError_t launch_bwd_dense_tc<__nv_bfloat16>(
+    const __nv_bfloat16*, const __nv_bfloat16*, const float*, const float*, const float*,
+    const float*, const float*, const float*, const float*, const int4*, int, int, int,
+    uint32_t*, float*, float*, float*, float*, float*, cudaStream_t);
 
 }  // namespace kda

@@ -92,6 +92,15 @@ inline Workspace carve(void* base, int total, int N, int H, int dk, int dv, int 
 }
 
 // ------------------------------------------------------------- conversions
+// x rounded to the nearest tf32 value (10-bit mantissa, ties away from zero;
+// the low 13 bits zero): operands of kind::tf32 products are written rounded,
+// since the tensor cores drop those bits, a bias that adds up over a sum.
+__device__ __forceinline__ float round_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);
 template <>
@@ -216,6 +225,19 @@ cudaError_t launch_bwd_chains_tc(const float* W, const float* Kb, const float* G
                                  const float* F, const int32_t* cu, int T, int N, int H,
                                  const int* chunk_start, uint32_t* status, float* states,
                                  float* dU, float* dSx, float* dS0, cudaStream_t st);
+// E = P^T dO and F = Qt^T dO - W^T E, and the dense products after the back
+// substitution (dQt, dKt, dKb, dGam, dbeta) on the tensor cores (dk = dv =
+// 128); kda_bwd_tc.cu.
+template <typename TIn>
+cudaError_t launch_bwd_ef_tc(const TIn* q, const TIn* dout, const float* G, const float* P,
+                             const float* W, const int4* info, int total, int maxc, int H,
+                             uint32_t* status, float* E, float* F, cudaStream_t st);
+template <typename TIn>
+cudaError_t launch_bwd_dense_tc(const TIn* k, const TIn* dout, const float* G, const float* beta,
+                                const float* U, const float* Y, const float* states,
+                                const float* dSx, const float* dbB, const int4* info, int total,
+                                int maxc, int H, uint32_t* status, float* dQt, float* dKt,
+                                float* dKb, float* dGam, float* dbeta, cudaStream_t st);
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* h0, const void* dout, const float* dhT,
                        const int32_t* cu, int T, int N, int H, int dk, int dv, kda_dtype_t dt,
