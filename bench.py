@@ -689,20 +689,28 @@ def backward_flops(head_tokens, dk, dv, C=64):
     of C tokens and one head, the multiply-adds of each step (the forward's
     A, P, W, Ut and chain recomputed, then E, F, the reverse chain, the back
     substitution, the products with U, S and dS', and the pair sums), two
-    flops each."""
+    flops each.  Returns (on the tensor cores, on the CUDA cores) for dk = dv
+    = 128, where the chains, E, F and the dense products run as tcgen05
+    products; other shapes run everything on the CUDA cores."""
     tri, stri = C * (C + 1) // 2, C * (C - 1) // 2
-    fma = (2 * tri * dk + stri * (dk + dv) + 2 * C * dk * dv      # A, P; [W | Ut]; chain
-           + tri * dv + 2 * C * dk * dv + 2 * C * dk * dv        # E; F; reverse chain
-           + stri * dv + 2 * C * C * dv + 3 * C * dk * dv        # Y; Y U^T, dO U^T; dense
-           + 4 * tri * dk)                                        # pair sums
-    return 2 * fma * head_tokens / C
+    tensor = (2 * C * dk * dv + 2 * C * dk * dv                    # the two chains
+              + tri * dv + 2 * C * dk * dv + 3 * C * dk * dv)      # E; F; dense
+    alu = (2 * tri * dk + stri * (dk + dv)                         # A, P; [W | Ut]
+           + stri * dv + 2 * C * C * dv                            # Y; Y U^T, dO U^T
+           + 4 * tri * dk)                                         # pair sums
+    if not (dk == 128 and dv == 128):
+        tensor, alu = 0, tensor + alu
+    return 2 * tensor * head_tokens / C, 2 * alu * head_tokens / C
 
 
 def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
     """kda_chunk_bwd on the prefill workload (fp32 gradients of o and the final
     state), timed with CUDA events on the launching stream, L2 flushed before
-    each call.  Bound by fp32 arithmetic on the CUDA cores: the roofline peak
-    is 148 SMs x 128 fp32 lanes x 2 flops x the SM clock."""
+    each call.  Roofline: the kernels run one after another, so the bound is
+    the tensor-core flops at the tf32 peak (the measured bf16 peak x the
+    nominal tf32 / bf16 ratio 1.1 / 2.25) plus the CUDA-core flops at 148
+    SMs x 128 fp32 lanes x 2 flops x the SM clock; `peak` is the total flops
+    over that time."""
     total, H, dk, dv = P.total, P.H, P.dk, P.dv
     Bc, Tc = (1, total) if P.cu_seqlens is not None else (P.B, P.T)
     g = torch.Generator(device=dev).manual_seed(9)
@@ -729,13 +737,23 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
     torch.cuda.synchronize()
     assert kda.kda_get_device_status(ws) == kda.KDA_OK
     t = statistics.median(x.elapsed_time(z) for x, z in ts) / 1e3
-    fl = backward_flops(total * H, dk, dv)
+    fl_tc, fl_alu = backward_flops(total * H, dk, dv)
+    fl = fl_tc + fl_alu
     mhz = sm_max_mhz or 1965.0
-    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    alu_peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    peaks, kind = load_peaks()
+    tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
+    t_bound = fl_tc / tf32_peak / 1e12 + fl_alu / alu_peak / 1e12
+    peak = fl / t_bound / 1e12
     res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 9,
            "roofline": {"bound": "alu", "achieved": fl / t / 1e12, "peak": peak,
                         "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak,
-                        "peak_kind": f"fp32 CUDA cores, 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",
+                        "peak_kind": (f"mixed: {fl_tc / 1e9:.1f} GFLOP at the tf32 tensor peak "
+                                      f"{tf32_peak:.0f} TFLOP/s ({kind} bf16 x 1.1/2.25) + "
+                                      f"{fl_alu / 1e9:.1f} GFLOP at the fp32 CUDA-core peak "
+                                      f"{alu_peak:.1f} TFLOP/s (148 SMs x 128 lanes x 2 x "
+                                      f"{mhz:.0f} MHz)"),
+                        "bound_ms": t_bound * 1e3,
                         "algorithmic_flops_per_call": fl},
            "workspace_bytes": int(ws.numel())}
     return res

@@ -80,7 +80,7 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-constexpr int kRun = 16;  // consecutive tokens per warp in the convolution
+constexpr int kRun = 32;  // consecutive tokens per warp in the convolution
 
 // The sequence holding token t: its index s (the last s with cu[s] <= t) --
 // clamped to [0, N - 1] so that a malformed cu_seqlens cannot send a read out
@@ -93,6 +93,25 @@ __device__ __forceinline__ int seq_of(const int32_t* cu, int N, int T, int t) {
         if (cu[mid] <= t) lo = mid; else hi = mid - 1;
     }
     return lo;
+}
+// The same for a whole warp (every lane gets the answer): a 32-ary search, one
+// load per lane and level, so one round trip per level instead of one per
+// halving (at most 32 sequences: one level).  cu is non-decreasing with cu[0]
+// = 0 <= t, so lane 0's entry always qualifies and the answer is the last
+// entry <= t, as in seq_of.
+__device__ __forceinline__ int warp_seq_of(const int32_t* cu, int N, int T, int t, int lane) {
+    if (!cu) return T > 0 ? t / T : 0;
+    int lo = 0, span = N;  // s lies in [lo, lo + span)
+    while (true) {
+        const int step = span <= 32 ? 1 : (span + 31) / 32;
+        const int idx = lo + lane * step;
+        const bool le = idx < lo + span && cu[idx] <= t;
+        const unsigned m = __ballot_sync(0xffffffffu, le);
+        const int k = m ? 31 - __clz(static_cast<int>(m)) : 0;
+        if (step == 1) return lo + k;
+        lo += k * step;
+        span = min(step, N - lo);
+    }
 }
 __device__ __forceinline__ int seq_begin(const int32_t* cu, int T, int s) {
     return cu ? max(0, cu[s]) : s * T;
@@ -125,13 +144,13 @@ __device__ __forceinline__ void conv_run(const TIn* __restrict__ x, const float*
         const float4 v = *reinterpret_cast<const float4*>(w + ((size_t)h * D + c0 + j) * 4);
         wt[j][0] = v.x; wt[j][1] = v.y; wt[j][2] = v.z; wt[j][3] = v.w;
     }
-    int s = seq_of(cu, N, T, t0);
-    int begin = seq_begin(cu, T, s), end = seq_end(cu, T, s);
+    // the halo rows and the first row are requested before the sequence
+    // lookup (which only decides whether the halo belongs to t0's sequence)
     float win[3][CPL];  // inputs of tokens t - 3, t - 2, t - 1
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
         const int src = t0 - 3 + i;
-        if (src >= begin && src >= 0) {
+        if (src >= 0) {
             Vec<CPL, TIn>::load(x + ((size_t)src * H + h) * D + c0, win[i]);
         } else {
 #pragma unroll
@@ -141,6 +160,13 @@ __device__ __forceinline__ void conv_run(const TIn* __restrict__ x, const float*
     const int t1 = min(total, t0 + kRun);
     float nxt[CPL];  // the next token's row, requested one token ahead
     Vec<CPL, TIn>::load(x + ((size_t)t0 * H + h) * D + c0, nxt);
+    int s = warp_seq_of(cu, N, T, t0, lane);
+    int begin = seq_begin(cu, T, s), end = seq_end(cu, T, s);
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+        if (t0 - 3 + i < begin)
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) win[i][j] = 0.f;
     for (int t = t0; t < t1; ++t) {
         float cur[CPL];
 #pragma unroll

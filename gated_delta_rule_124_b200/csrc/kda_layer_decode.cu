@@ -13,13 +13,13 @@
 //   the decode step of kda_decode.cu on (q, k, v, g, beta, S)
 //   y = o / sqrt(mean_j o_j^2 + rms_eps) * w_norm * sigmoid(gate)
 //
-// q, k, v and o never leave the chip.  As in the plain decode kernel, the
-// value columns of one (sequence, head) are split into NS = DV / DVS slices
-// (DVS = 64 for DV = 128); here the slices are the NS 256-thread units of one
-// CTA, because three things cross the split: the q / k convolution (computed
-// once per CTA and shared), the convolution states (overwritten after a CTA
-// barrier, once every thread has read them) and the RMSNorm, which needs the
-// sum of o^2 over all DV columns (each unit's slice sum in shared memory).
+// q, k, v and o never leave the chip.  One 256-thread CTA takes all DV value
+// columns of one (sequence, head), so the q / k convolution, the convolution
+// states (overwritten after a CTA barrier, once every thread has read them)
+// and the RMSNorm's sum of o^2 over the DV columns stay inside the CTA.  The
+// kernel is written for NS = DV / DVS 256-thread units per CTA (each unit a
+// slice of DVS value columns, the slices' sums of squares combined in shared
+// memory); the launch uses NS = 1.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -235,7 +235,10 @@ __global__ void __launch_bounds__(256 * (DV / DVS), ((DK * DVS <= 8192) ? 4 : 2)
 
 template <int DK, int DV, typename TIn>
 cudaError_t launch_layer_decode_t(const LayerDecodeArgs& a, int units, cudaStream_t st) {
-    constexpr int DVS = (DV == 128) ? 64 : DV;
+    // one 256-thread CTA per (sequence, head) over all DV columns: measured
+    // 209 us against 237 us for two 256-thread units of DV / 2 columns in one
+    // CTA (N = 256, H = 32, d = 128, bf16)
+    constexpr int DVS = DV;
     layer_decode_kernel<DK, DV, DVS, TIn><<<units, 256 * (DV / DVS), 0, st>>>(a);
     return cudaGetLastError();
 }

@@ -483,9 +483,9 @@ kda_status_t kda_layer_chunk_fwd(const void* xq, const void* xk, const void* xv,
  * In/out: conv_q, conv_k [N, 3, H, dk], conv_v [N, 3, H, dv] (dtype) as for
  *      kda_qkv_conv_norm_step; state [N, H, dk, dv] fp32 as for kda_decode_step.
  * Out: y [N, H, dv] (dtype), not aliasing any input.
- * The value columns of a (sequence, head) are split over the 256-thread units
- * of one CTA when dv = 128 (they share the RMSNorm's sum over dv through its
- * shared memory).  Shapes: dk, dv in {32, 64, 128};
+ * One 256-thread CTA per (sequence, head) takes all dv value columns, so the
+ * RMSNorm's sum over dv stays in its shared memory.  Shapes: dk, dv in
+ * {32, 64, 128};
  * N == 0 does nothing.  No workspace.
  */
 kda_status_t kda_layer_decode_step(const void* xq, const void* xk, const void* xv,
