@@ -54,11 +54,19 @@ _CFG2 = "long prefill: B=1 H=32 T=65536 d=128 C=64 bf16 slow decay"
 _DECODE = "gated_delta_rule_124_b200/csrc/kda_decode.cu"
 _DEC = "decode: N=256 H=32 d=128 bf16, fp32 state, 8 input sets cycled"
 MEASURED_TRAFFIC = {
-    ("split_intra", _CFG1): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 222362880),
-    ("split_chain", _CFG1): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 195830272),
-    # captured on B=1 x T=16384 (a quarter of the tokens) and scaled by 4
-    ("chunk_fwd_overlap", _CFG2): (_SPLIT, "0b693b66fe9f5011f077ea95ae6503d88abc4208", 5597298688),
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch, captured on
+    # B=8 x T=2048, H=32 (8192 (chunk, head) items, inputs larger than L2)
+    # and scaled by the items of the varlen workload (62560): per item
+    # 127.7 KB (intra) and 100.9 KB (chain)
+    ("split_intra", _CFG3): (_SPLIT, "7a72c2ac396efe749f7b84bf1575a2b6266215d8", 7988038115),
+    ("split_chain", _CFG3): (_SPLIT, "7a72c2ac396efe749f7b84bf1575a2b6266215d8", 6312896365),
     ("decode", _DEC): (_DECODE, "e97a0fa46338f7541982499a4e97d31ac9101889", 1027143936),
+}
+
+
+TRAFFIC_NOTE = {
+    ("split_intra", _CFG3): "ncu DRAM bytes of B=8 x T=2048, H=32 scaled by (chunk, head) items",
+    ("split_chain", _CFG3): "ncu DRAM bytes of B=8 x T=2048, H=32 scaled by (chunk, head) items",
 }
 
 
@@ -221,6 +229,8 @@ def prefill_roofline(kern, pc, peaks, peak_kind):
     return {"kernel": dom_name, "bound": "hbm", "achieved": dom_bytes / dom_s / 1e9,
             "peak": hbm, "unit": "GB/s", "frac": dom_bytes / dom_s / 1e9 / hbm,
             "traffic": measured_traffic(dom_name, pc.name),
+            "traffic_note": (TRAFFIC_NOTE.get((dom_name, pc.name))
+                             if measured_traffic(dom_name, pc.name) else None),
             "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
             "per_launch_us": dom_s * 1e6, "algorithmic_bytes_per_launch": dom_bytes}
 

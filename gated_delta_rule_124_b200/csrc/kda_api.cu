@@ -176,8 +176,10 @@ kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_E
 // Gated DeltaNet (head-uniform gate): the split plan reads the gate per
 // (token, head) directly; every other shape spreads it over the dk channels
 // into the workspace, after the CUDA-core plan's own part, and runs that plan.
-Path gdn_path(int dk, int dv, int chunk, kda_dtype_t dt) {
-    return tc_shape(dk, dv, chunk, dt) ? Path::Split : Path::Simt;
+// Gated DeltaNet takes the plans of KDA by the same rule (its intra-chunk
+// kernel is the head-gate variant of the same kernel).
+Path gdn_path(int total, int N, bool packed, int H, int dk, int dv, int chunk, kda_dtype_t dt) {
+    return select_path(total, N, packed, H, dk, dv, chunk, dt);
 }
 
 size_t gdn_workspace_bytes(const Prefill& p, int H, int dk, int dv, int chunk, Path path,
@@ -630,7 +632,8 @@ size_t kda_gdn_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, i
         return 0;
     const Prefill p{total_tokens, num_seqs};
     size_t off;
-    return gdn_workspace_bytes(p, H, dk, dv, chunk, gdn_path(dk, dv, chunk, dtype), &off);
+    return gdn_workspace_bytes(p, H, dk, dv, chunk,
+                               gdn_path(p.total, p.N, false, H, dk, dv, chunk, dtype), &off);
 }
 
 kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
@@ -648,7 +651,7 @@ kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, cons
         if (!aligned16(ptr)) return KDA_ERR_INVALID_ARG;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_INVALID_ARG;
-    const Path path = gdn_path(dk, dv, chunk, dtype);
+    const Path path = gdn_path(p.total, p.N, cu_seqlens != nullptr, H, dk, dv, chunk, dtype);
     size_t spread_off = 0;
     const size_t need = gdn_workspace_bytes(p, H, dk, dv, chunk, path, &spread_off);
     if (!workspace) return KDA_ERR_WORKSPACE;
@@ -660,6 +663,11 @@ kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, cons
     s = begin_prefill(w, cu_seqlens, B, T, p.N, chunk, maxc, st);
     if (s != KDA_OK) return s;
     if (p.total == 0 && !final_state) return KDA_OK;
+    if (path == Path::Overlap)
+        return from_cuda(kda::launch_chunk_fwd_overlap(q, k, v, nullptr, beta, initial_state,
+                                                       cu_seqlens, T, p.N, H, w.chunk_info,
+                                                       maxc, w.chunk_start, w.status, w.blobs,
+                                                       w.flags, o, final_state, st, -1, 0, g));
     if (path == Path::Split)
         return from_cuda(kda::launch_chunk_fwd_split(q, k, v, nullptr, beta, initial_state,
                                                      cu_seqlens, T, p.N, H, w.chunk_info, maxc,

@@ -1500,6 +1500,7 @@ constexpr uint32_t UNIT_BYTES = unit_bytes();
 constexpr uint32_t OVERLAP_SMEM = 2 * UNIT_BYTES + 1024;
 static_assert(OVERLAP_SMEM + 1024 <= 232448, "one CTA per SM");
 
+template <bool kScalar>
 __global__ void __launch_bounds__(NTO, 1)
     chunk_overlap_kernel(const __grid_constant__ CUtensorMap tmq,
                          const __grid_constant__ CUtensorMap tmk,
@@ -1528,8 +1529,9 @@ __global__ void __launch_bounds__(NTO, 1)
         else if (threadIdx.x == 256)
             chain::watch(pc, align1024(smem_raw), b >> 1);
     } else
-        intra::run<true>(&tmq, &tmk, &tmg, pi, sm, tb, 1 + unit, 2 * (b - nchain) + unit,
-                         2 * (static_cast<int>(gridDim.x) - nchain));
+        intra::run<true, kScalar>(&tmq, &tmk, &tmg, pi, sm, tb, 1 + unit,
+                                  2 * (b - nchain) + unit,
+                                  2 * (static_cast<int>(gridDim.x) - nchain));
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) tmem_dealloc(s_tmem, 512);
@@ -1724,20 +1726,20 @@ cudaError_t launch_split_state_maps(const void* q, const void* k, const void* v,
 // after one SM per chain unit.
 int overlap_grid(int N, int H) {
     int dev = 0, sms = 0, nb = 0, coop = 0;
+    int nb_scalar = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
-        cudaFuncSetAttribute(chunk_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)OVERLAP_SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(chunk_overlap_kernel,
-                             cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, chunk_overlap_kernel, NTO,
-                                                      OVERLAP_SMEM) != cudaSuccess) {
+        set_smem_max_carveout(chunk_overlap_kernel<false>, OVERLAP_SMEM) != cudaSuccess ||
+        set_smem_max_carveout(chunk_overlap_kernel<true>, OVERLAP_SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, chunk_overlap_kernel<false>, NTO,
+                                                      OVERLAP_SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb_scalar, chunk_overlap_kernel<true>,
+                                                      NTO, OVERLAP_SMEM) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
-    if (!coop || nb < 1 || sms <= 0) return 0;
+    if (!coop || nb < 1 || nb_scalar < 1 || sms <= 0) return 0;
     if (2LL * N * H >= sms) return 0;
     return sms;
 }
@@ -1748,7 +1750,7 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
                                      const int4* chunk_info, int maxc, const int* chunk_start,
                                      uint32_t* status, void* blobs, uint32_t* flags, void* o,
                                      float* hN, cudaStream_t st, long long withheld_flag,
-                                     unsigned long long flag_wait_ns) {
+                                     unsigned long long flag_wait_ns, const float* gh) {
     const int total = cu_seqlens ? T : N * T;
     if (total == 0)
         return launch_split_chain(v, h0, cu_seqlens, T, N, H, chunk_start, status, blobs, o, hN,
@@ -1760,17 +1762,22 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !split_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !split_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, total, H, 64,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    if (gh) {
+        mg = mq;  // not read: the head-uniform gate comes by plain loads
+    } else if (!split_map(&mg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, total, H, 128,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        return cudaErrorInvalidValue;
+    }
     cudaError_t e = cudaMemsetAsync(flags, 0, sizeof(uint32_t) * (size_t)maxc * H, st);
     if (e != cudaSuccess) return e;
     uint8_t* bl = static_cast<uint8_t*>(blobs);
     intra::Params pi{beta, chunk_info, maxc, H, status, status, bl,
                      N, chunk_start, status + 1, flags};
     pi.withheld = withheld_flag;
+    pi.gh = gh;
     chain::Params pc{h0, cu_seqlens, T, H, chunk_start, status, status, bl,
                      (__nv_bfloat16*)o, hN, flags};
     pc.flag_wait_ns = flag_wait_ns ? flag_wait_ns : kWaitNs;
@@ -1784,7 +1791,11 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chunk_overlap_kernel, mq, mk, mg, mv, pi, pc, 2 * N * H);
+    if (gh)
+        return cudaLaunchKernelEx(&cfg, chunk_overlap_kernel<true>, mq, mk, mg, mv, pi, pc,
+                                  2 * N * H);
+    return cudaLaunchKernelEx(&cfg, chunk_overlap_kernel<false>, mq, mk, mg, mv, pi, pc,
+                              2 * N * H);
 }
 
 cudaError_t launch_chunk_fwd_split(const void* q, const void* k, const void* v, const float* g,

@@ -72,6 +72,7 @@ cudaError_t launch_split_state_maps(const void* q, const void* k, const void* v,
 // withheld_flag >= 0 (testing the bounded-wait error path only): the flag of
 // that (slot * H + head) is never released; flag_wait_ns != 0 bounds the
 // chains' wait on one flag (default 2 s).
+// gh != nullptr: the head-uniform gate [total, H] of Gated DeltaNet (g unused).
 // overlap_grid() is its grid size, or 0 when the launch does not apply.
 int overlap_grid(int N, int H);
 cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v, const float* g,
@@ -80,6 +81,7 @@ cudaError_t launch_chunk_fwd_overlap(const void* q, const void* k, const void* v
                                      const int4* chunk_info, int maxc, const int* chunk_start,
                                      uint32_t* status, void* blobs, uint32_t* flags, void* o,
                                      float* hN, cudaStream_t st, long long withheld_flag = -1,
-                                     unsigned long long flag_wait_ns = 0);
+                                     unsigned long long flag_wait_ns = 0,
+                                     const float* gh = nullptr);
 
 }  // namespace kda

@@ -304,10 +304,11 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
  * kda_chunk_fwd / kda_decode_step, except:
  *   g [total, H] fp32 (prefill), [N, H] fp32 (decode) -- log alpha per (token,
  *   head); the workspace is kda_gdn_chunk_fwd_workspace_size() bytes.
- * bf16, dk = dv = 128, chunk 64 runs the split tensor-core plan with the gate
- * read per (token, head) (one exponential per row instead of per element);
- * other shapes spread g over the dk channels in the workspace and run the
- * CUDA-core plan.
+ * bf16, dk = dv = 128, chunk 64 runs the tensor-core plan kda_chunk_fwd would
+ * choose for the same shape (split, or co-scheduled for few long chains) with
+ * the gate read per (token, head) (one exponential per row instead of per
+ * element); other shapes spread g over the dk channels in the workspace and
+ * run the CUDA-core plan.
  */
 size_t kda_gdn_chunk_fwd_workspace_size(int total_tokens, int num_seqs, int H, int dk, int dv,
                                         int chunk, kda_dtype_t dtype);

@@ -76,6 +76,17 @@ def test_deltanet_is_gdn_with_zero_gate():
     _check(case, gh, torch.zeros(case.total, case.H, case.dk))
 
 
+def test_gdn_long_sequence_takes_the_co_scheduled_plan():
+    """One 16384-token sequence over 16 heads: few long chains, so the plan
+    rule picks the co-scheduled launch (intra units of the head-gate variant
+    beside the chain units); against the oracle on the spread gate."""
+    case = wl.make_prefill(406, [16384], H=16, dk=128, dv=128, chunk=64, dtype="bf16")
+    assert kda.PLAN_NAMES[kda.kda_chunk_fwd_plan(case.total, case.N, case.H, 128, 128, 64,
+                                                 "bf16")] == "overlap"
+    gh, gfull = _head_gate(case, 6)
+    _check(case, gh, gfull)
+
+
 def test_gdn_agrees_with_kda_on_a_spread_gate():
     case = wl.make_prefill(405, [256, 130], H=3, dk=128, dv=128, chunk=64, dtype="bf16",
                            varlen=True)
