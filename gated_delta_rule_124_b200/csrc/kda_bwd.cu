@@ -55,6 +55,7 @@ struct BwdBufs {
     float* dKb;   // [total, H, dk]
     float* dGam;  // [maxc, H, dk]
     float* dbB;   // [total, H]
+    int* slow;    // [maxc, H]  (tensor-core pair sums) 1: the chunk is left to the exact kernel
     size_t bytes;
 };
 
@@ -86,6 +87,7 @@ BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
     b.dKb = take(tk);
     b.dGam = take(maxc * H * dk);
     b.dbB = take((size_t)total * H);
+    b.slow = reinterpret_cast<int*>(take(maxc * H));
     b.bytes = off;
     return b;
 }
@@ -813,7 +815,8 @@ __global__ void __launch_bounds__(256) bwd_pair_kernel(
     const float* __restrict__ dKt, const float* __restrict__ dKb,
     const float* __restrict__ dGam, const int4* __restrict__ info, int H, int dk,
     const uint32_t* status, float* __restrict__ dq, float* __restrict__ dk_out,
-    float* __restrict__ dg) {
+    float* __restrict__ dg, const int* __restrict__ slow) {
+    // slow != NULL: only the chunks the tensor-core pair kernel left (flag 1)
     constexpr int NR = CB / 8;
     constexpr int LA = CB + 1;
     if (status_bad(status)) return;
@@ -821,6 +824,7 @@ __global__ void __launch_bounds__(256) bwd_pair_kernel(
     const int4 ci = info[cidx];
     const int L = ci.z;
     if (L <= 0) return;
+    if (slow && !slow[(size_t)cidx * H + h]) return;
     const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
     extern __shared__ float sm[];
     float* Qs = sm;              // [C][32]
@@ -1008,11 +1012,17 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
         : dk == 64 ? launch_dense<64, TIn>(b, K, DO, beta, maxc, H, dv, db, st)
                    : launch_dense<32, TIn>(b, K, DO, beta, maxc, H, dv, db, st);
     if (e != cudaSuccess) return e;
+    if (tc) {  // the pair sums as products; chunks outside the exponent range stay exact
+        e = launch_bwd_pair_tc<TIn>(Q, K, w.G, b.dAr, b.dP, b.dQt, b.dKt, b.dKb, b.dGam,
+                                    w.chunk_info, total, maxc, H, w.status, b.slow, dq, dkk, dg,
+                                    st);
+        if (e != cudaSuccess) return e;
+    }
     const size_t sm = pair_smem();
     if ((e = set_smem(bwd_pair_kernel<TIn>, sm)) != cudaSuccess) return e;
     bwd_pair_kernel<TIn><<<dim3(maxc, H, dk / 32), 256, sm, st>>>(
         Q, K, w.G, b.dAr, b.dP, b.dQt, b.dKt, b.dKb, b.dGam, w.chunk_info, H, dk, w.status, dq,
-        dkk, dg);
+        dkk, dg, tc ? b.slow : nullptr);
     return cudaGetLastError();
 }
 

@@ -766,6 +766,284 @@ __global__ void __launch_bounds__(NTB, 1)
     if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
+// ------------------------------------------------------------ pair sums
+// Per (chunk, head), with E = exp(G - Gm) under a per-channel reference Gm =
+// max_r G_r - 80 (every factor within exp(+-80) when the chunk's per-channel
+// log-decay range is at most 160 and max G <= 60, as in the forward's A/P):
+//   [rowA ; dQp] = ([bdA ; dP] (K * E^-1)) * [E ; E]     (one M = 128 product)
+//   col          = ([bdA ; dP]^T [K * E ; Q * E]) * E^-1  (M = 64 padded to 128)
+// i.e. rowA[r] = sum_{i<r} bdA[r][i] k_i e^{G_r - G_i}, dQp[r] = sum_{i<=r}
+// dP[r][i] k_i e^{G_r - G_i}, col[r] = sum_{i'>=r} (bdA[i'][r] k_i' + dP[i'][r]
+// q_i') e^{G_i' - G_r} (the masks are the zeros of bdA and dP), then the same
+// epilogue as the exact kernel: dq, dk, dG and the reverse cumulative sum dg.
+// X = [bdA ; dP] [128 rows][64 columns] is the K-major A operand of the first
+// product and the MN-major A operand of the second, so it is staged twice (the
+// 16-byte- and the 32-byte-granule swizzle).  A chunk outside the range sets
+// slow = 1 and is left to the exact kernel.
+namespace pr {
+constexpr uint32_t OFF_X1 = 0;        // X, 2 blocks [128][32] (16-byte granules)
+constexpr uint32_t OFF_X2 = 32768;    // X, 2 blocks [128][32] (32-byte granules)
+constexpr uint32_t OFF_B1 = 65536;    // K * E^-1 [64 i][128 c]: 4 blocks [64][32]
+constexpr uint32_t OFF_B2 = 98304;    // [K * E ; Q * E] [128][128 c]: 4 blocks [128][32]
+constexpr uint32_t OFF_GM = 163840;   // Gm [128]
+constexpr uint32_t OFF_RED = OFF_GM + 512;   // max, min [2][128] each; later the epilogue's exchange
+constexpr uint32_t OFF_BAR = OFF_RED + 2048;
+constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+// after the products, the accumulators as fp32 [rows][LDD] over the operands
+constexpr int LDD = 132;
+constexpr uint32_t OFF_D1 = 0;                       // rows 0-63 rowA, 64-127 dQp
+constexpr uint32_t OFF_D2 = 128 * LDD * 4;           // rows 0-63 col
+static_assert(OFF_D2 + 64 * LDD * 4 <= OFF_GM, "accumulator dump");
+constexpr uint32_t TM_1 = 0, TM_2 = 128;
+constexpr float kRefPair = 80.f;
+}  // namespace pr
+
+struct PairArgs {
+    const void* q;
+    const void* k;
+    const float* G;
+    const float* dAr;
+    const float* dP;
+    const float* dQt;
+    const float* dKt;
+    const float* dKb;
+    const float* dGam;
+    const int4* info;
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    int* slow;
+    float* dq;
+    float* dk;
+    float* dg;
+};
+
+template <typename TIn>
+__device__ __forceinline__ float4 load4_f32(const TIn* p);
+template <>
+__device__ __forceinline__ float4 load4_f32<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4_f32<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                       __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ float4 round4_tf32(float4 v) {
+    return make_float4(round_tf32(v.x), round_tf32(v.y), round_tf32(v.z), round_tf32(v.w));
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(NTB, 1) pair_tc_kernel(const PairArgs a) {
+    using namespace pr;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_skip;
+    const int cidx = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int4 ci = a.info[cidx];
+    const int t0 = ci.y, L = ci.z;
+    if (tid == 0) s_skip = status_bad(a.status) || L <= 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* sGm = reinterpret_cast<float*>(sm + OFF_GM);
+    float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
+    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + pr::OFF_BAR);
+    const TIn* Qg = static_cast<const TIn*>(a.q);
+    const TIn* Kg = static_cast<const TIn*>(a.k);
+    const int c = tid & 127, half = tid >> 7;
+    const size_t rowH = (size_t)a.H * DD;  // stride between tokens
+    const size_t base = ((size_t)t0 * a.H + h) * DD;
+    // 1. per-channel max / min of G over the chunk's rows, the reference and
+    // the range test (the exact kernel makes the same test from the flag)
+    {
+        float mx = -INFINITY, mn = INFINITY;
+        for (int r = 32 * half; r < min(L, 32 * half + 32); ++r) {
+            const float gv = a.G[base + r * rowH + c];
+            mx = fmaxf(mx, gv);
+            mn = fminf(mn, gv);
+        }
+        sRed[half * 128 + c] = mx;
+        sRed[256 + half * 128 + c] = mn;
+    }
+    __syncthreads();
+    bool bad = false;
+    if (tid < 128) {
+        const float mx = fmaxf(sRed[c], sRed[128 + c]), mn = fminf(sRed[256 + c], sRed[384 + c]);
+        sGm[c] = mx - kRefPair;
+        bad = !(mx - mn <= 2.f * kRefPair) || !(mx <= 60.f);
+    }
+    const bool slow = __syncthreads_or(bad);
+    if (tid == 0) a.slow[(size_t)cidx * a.H + h] = slow ? 1 : 0;
+    if (slow) return;
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cw = warp >> 2;
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    // 2. operands.  X rows m (< 64: bdA row m; >= 64: dP row m - 64), four
+    // columns per float4: both swizzles
+    {
+        const size_t cc = ((size_t)cidx * a.H + h) * 64 * 64;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int idx = tid + NTB * it;  // 0 .. 2047
+            const int m = idx >> 4, c4 = idx & 15;
+            const int r = m & 63;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < L) v = *reinterpret_cast<const float4*>((m < 64 ? a.dAr : a.dP) + cc + r * 64 + 4 * c4);
+            v = round4_tf32(v);
+            const int blk = c4 >> 3, q16 = c4 & 7;
+            *reinterpret_cast<float4*>(sm + OFF_X1 + blk * 16384 + sw128_off(m, q16)) = v;
+            *reinterpret_cast<float4*>(sm + OFF_X2 + blk * 16384 + sw128_32b_off(m, q16)) = v;
+        }
+    }
+    __syncthreads();  // Gm visible
+    // K * E^-1, K * E, Q * E: row r, channels 4 c4 .. 4 c4 + 3
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int idx = tid + NTB * it;  // 0 .. 2047
+        const int r = idx >> 5, c4 = idx & 31;
+        float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv, ke = kv, ki = kv;
+        if (r < L) {
+            const size_t gi = base + r * rowH + 4 * c4;
+            kv = load4_f32<TIn>(Kg + gi);
+            qv = load4_f32<TIn>(Qg + gi);
+            const float4 gv = *reinterpret_cast<const float4*>(a.G + gi);
+            const float4 gm = *reinterpret_cast<const float4*>(sGm + 4 * c4);
+            const float x0 = gv.x - gm.x, x1 = gv.y - gm.y, x2 = gv.z - gm.z, x3 = gv.w - gm.w;
+            const float e0 = __expf(x0), e1 = __expf(x1), e2 = __expf(x2), e3 = __expf(x3);
+            ke = make_float4(kv.x * e0, kv.y * e1, kv.z * e2, kv.w * e3);
+            qv = make_float4(qv.x * e0, qv.y * e1, qv.z * e2, qv.w * e3);
+            ki = make_float4(kv.x * __expf(-x0), kv.y * __expf(-x1), kv.z * __expf(-x2),
+                             kv.w * __expf(-x3));
+        }
+        const int blk = c4 >> 3, q16 = c4 & 7;
+        *reinterpret_cast<float4*>(sm + OFF_B1 + blk * 8192 + sw128_32b_off(r, q16)) =
+            round4_tf32(ki);
+        *reinterpret_cast<float4*>(sm + OFF_B2 + blk * 16384 + sw128_32b_off(r, q16)) =
+            round4_tf32(ke);
+        *reinterpret_cast<float4*>(sm + OFF_B2 + blk * 16384 + sw128_32b_off(64 + r, q16)) =
+            round4_tf32(qv);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s_tmem;
+    // 3. the two products, one commit
+    if (tid == 0) {
+        constexpr uint32_t id1 = idesc_tf32(128, 128, false, true);
+        constexpr uint32_t id2 = idesc_tf32(128, 128, true, true);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const int kb = ks >> 2, kk = ks & 3;
+            mma_tf32_tc(tbase + TM_1, sdesc_sw128(sbase + OFF_X1 + kb * 16384 + kk * 32, 16, 1024),
+                        sdesc_sw128_32b(sbase + OFF_B1 + ks * 1024, 8192, 512), id1, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks)
+            mma_tf32_tc(tbase + TM_2, sdesc_sw128_32b(sbase + OFF_X2 + ks * 1024, 16384, 512),
+                        sdesc_sw128_32b(sbase + OFF_B2 + ks * 1024, 16384, 512), id2, ks > 0);
+        mma_commit(bar_mma);
+    }
+    const bool ok = mbar_wait(bar_mma, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            mbar_wait(bar_mma, 0, kWaitNs);  // bounded: the products still in flight
+            atomicOr(a.status_out, STATUS_TIMEOUT);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tbase, 256);
+        return;
+    }
+    tc_fence_after();
+    // 4. the accumulators to shared memory (over the operands, all read)
+    {
+        float* D1 = reinterpret_cast<float*>(sm + OFF_D1);
+        float* D2 = reinterpret_cast<float*>(sm + OFF_D2);
+        const int row = 32 * quarter + lane;
+        const uint32_t tl = static_cast<uint32_t>(32 * quarter) << 16;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            uint32_t v[32];
+            tmem_ld32(tbase + tl + TM_1 + 64 * cw + 32 * x, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int y = 0; y < 32; y += 4)
+                *reinterpret_cast<float4*>(D1 + row * LDD + 64 * cw + 32 * x + y) =
+                    make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+            if (quarter < 2) {
+                tmem_ld32(tbase + tl + TM_2 + 64 * cw + 32 * x, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int y = 0; y < 32; y += 4)
+                    *reinterpret_cast<float4*>(D2 + row * LDD + 64 * cw + 32 * x + y) =
+                        make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                    __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+    // 5. the epilogue of the exact kernel, channel c, rows 32 half .. + 31
+    {
+        const float* D1 = reinterpret_cast<const float*>(sm + OFF_D1);
+        const float* D2 = reinterpret_cast<const float*>(sm + OFF_D2);
+        const float gm = sGm[c];
+        const float glast = a.G[base + (L - 1) * rowH + c];
+        float dG[32];
+        float tot = 0.f, last = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int r = 32 * half + j;
+            dG[j] = 0.f;
+            if (r < L) {
+                const size_t gi = base + r * rowH + c;
+                const float gr = a.G[gi], qr = to_f32(Qg[gi]), kr = to_f32(Kg[gi]);
+                const float e = __expf(gr - gm), ei = __expf(gm - gr);
+                const float rowA = D1[r * LDD + c] * e, dQp = D1[(64 + r) * LDD + c] * e;
+                const float col = D2[r * LDD + c] * ei;
+                const float eg = expf(gr), eb = expf(glast - gr);
+                const float x = a.dQt[gi], y = a.dKt[gi], z = a.dKb[gi];
+                a.dq[gi] = dQp + x * eg;
+                a.dk[gi] = rowA + col + y * eg + z * eb;
+                dG[j] = kr * (rowA - col) + qr * dQp + x * qr * eg + y * kr * eg - z * kr * eb;
+                tot += dG[j];
+                last += z * kr * eb;
+            }
+        }
+        // [2][128] row-sum totals, [2][128] last-row terms, over the max / min
+        // partials of step 1 (read before the range test's barrier)
+        float* xch = sRed;
+        xch[half * 128 + c] = tot;
+        xch[256 + half * 128 + c] = last;
+        __syncthreads();
+        float acc = expf(glast) * a.dGam[((size_t)cidx * a.H + h) * DD + c] + xch[256 + c] +
+                    xch[384 + c];
+        if (half == 0) acc += xch[128 + c];
+#pragma unroll
+        for (int j = 31; j >= 0; --j) {
+            const int r = 32 * half + j;
+            if (r < L) {
+                acc += dG[j];
+                a.dg[base + r * rowH + c] = acc;
+            }
+        }
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void* ptr = nullptr;
@@ -907,5 +1185,35 @@ template cudaError_t launch_bwd_dense_tc<__nv_bfloat16>(
     const __nv_bfloat16*, const __nv_bfloat16*, const float*, const float*, const float*,
     const float*, const float*, const float*, const float*, const int4*, int, int, int,
     uint32_t*, float*, float*, float*, float*, float*, cudaStream_t);
+
+}  // namespace kda
+
+namespace kda {
+
+template <typename TIn>
+cudaError_t launch_bwd_pair_tc(const TIn* q, const TIn* k, const float* G, const float* dAr,
+                               const float* dP, const float* dQt, const float* dKt,
+                               const float* dKb, const float* dGam, const int4* info, int total,
+                               int maxc, int H, uint32_t* status, int* slow, float* dq,
+                               float* dk, float* dg, cudaStream_t st) {
+    if (maxc == 0 || total == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(pair_tc_kernel<TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pr::SMEM);
+    if (e != cudaSuccess) return e;
+    const PairArgs a{q, k, G, dAr, dP, dQt, dKt, dKb, dGam, info, H, status, status, slow, dq, dk,
+                     dg};
+    pair_tc_kernel<TIn><<<dim3(maxc, H), NTB, pr::SMEM, st>>>(a);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_bwd_pair_tc<float>(const float*, const float*, const float*,
+                                               const float*, const float*, const float*,
+                                               const float*, const float*, const float*,
+                                               const int4*, int, int, int, uint32_t*, int*,
+                                               float*, float*, float*, cudaStream_t);
+template cudaError_t launch_bwd_pair_tc<__nv_bfloat16>(
+    const __nv_bfloat16*, const __nv_bfloat16*, const float*, const float*, const float*,
+    const float*, const float*, const float*, const float*, const int4*, int, int, int,
+    uint32_t*, int*, float*, float*, float*, cudaStream_t);
 
 }  // namespace kda

@@ -238,6 +238,15 @@ cudaError_t launch_bwd_dense_tc(const TIn* k, const TIn* dout, const float* G, c
                                 const float* dSx, const float* dbB, const int4* info, int total,
                                 int maxc, int H, uint32_t* status, float* dQt, float* dKt,
                                 float* dKb, float* dGam, float* dbeta, cudaStream_t st);
+// The pair sums (dq, dk, dg) as tensor-core products under a per-channel
+// exponent reference; a chunk whose gate range exceeds it gets slow[] = 1 and
+// is left to the exact CUDA-core kernel; kda_bwd_tc.cu.
+template <typename TIn>
+cudaError_t launch_bwd_pair_tc(const TIn* q, const TIn* k, const float* G, const float* dAr,
+                               const float* dP, const float* dQt, const float* dKt,
+                               const float* dKb, const float* dGam, const int4* info, int total,
+                               int maxc, int H, uint32_t* status, int* slow, float* dq,
+                               float* dk, float* dg, cudaStream_t st);
 cudaError_t launch_bwd(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* h0, const void* dout, const float* dhT,
                        const int32_t* cu, int T, int N, int H, int dk, int dv, kda_dtype_t dt,
