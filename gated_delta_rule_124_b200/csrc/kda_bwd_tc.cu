@@ -786,8 +786,8 @@ constexpr uint32_t OFF_X2 = 32768;    // X, 2 blocks [128][32] (32-byte granules
 constexpr uint32_t OFF_B1 = 65536;    // K * E^-1 [64 i][128 c]: 4 blocks [64][32]
 constexpr uint32_t OFF_B2 = 98304;    // [K * E ; Q * E] [128][128 c]: 4 blocks [128][32]
 constexpr uint32_t OFF_GM = 163840;   // Gm [128]
-constexpr uint32_t OFF_RED = OFF_GM + 512;   // max, min [2][128] each; later the epilogue's exchange
-constexpr uint32_t OFF_BAR = OFF_RED + 2048;
+constexpr uint32_t OFF_RED = OFF_GM + 512;   // max, min [4][128] each; later the epilogue's exchange
+constexpr uint32_t OFF_BAR = OFF_RED + 4096;
 constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
 // after the products, the accumulators as fp32 [rows][LDD] over the operands
 constexpr int LDD = 132;
@@ -796,6 +796,7 @@ constexpr uint32_t OFF_D2 = 128 * LDD * 4;           // rows 0-63 col
 static_assert(OFF_D2 + 64 * LDD * 4 <= OFF_GM, "accumulator dump");
 constexpr uint32_t TM_1 = 0, TM_2 = 128;
 constexpr float kRefPair = 80.f;
+constexpr int NTP = 512;  // threads: one CTA per SM (shared memory), so 16 warps
 }  // namespace pr
 
 struct PairArgs {
@@ -836,7 +837,7 @@ __device__ __forceinline__ float4 round4_tf32(float4 v) {
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(NTB, 1) pair_tc_kernel(const PairArgs a) {
+__global__ void __launch_bounds__(pr::NTP, 1) pair_tc_kernel(const PairArgs a) {
     using namespace pr;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t s_tmem;
@@ -855,32 +856,42 @@ __global__ void __launch_bounds__(NTB, 1) pair_tc_kernel(const PairArgs a) {
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + pr::OFF_BAR);
     const TIn* Qg = static_cast<const TIn*>(a.q);
     const TIn* Kg = static_cast<const TIn*>(a.k);
-    const int c = tid & 127, half = tid >> 7;
+    // channel c, a quarter `part` of the chunk's rows (16 each)
+    const int c = tid & 127, part = tid >> 7;
     const size_t rowH = (size_t)a.H * DD;  // stride between tokens
     const size_t base = ((size_t)t0 * a.H + h) * DD;
     // 1. per-channel max / min of G over the chunk's rows, the reference and
-    // the range test (the exact kernel makes the same test from the flag)
+    // the range test (the exact kernel reads the flag this writes)
     {
-        float mx = -INFINITY, mn = INFINITY;
-        for (int r = 32 * half; r < min(L, 32 * half + 32); ++r) {
-            const float gv = a.G[base + r * rowH + c];
-            mx = fmaxf(mx, gv);
-            mn = fminf(mn, gv);
+        float gv[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {  // all 16 loads in flight at once
+            const int r = 16 * part + j;
+            gv[j] = r < L ? __ldg(a.G + base + r * rowH + c) : 0.f;
         }
-        sRed[half * 128 + c] = mx;
-        sRed[256 + half * 128 + c] = mn;
+        float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (16 * part + j < L) {
+                mx = fmaxf(mx, gv[j]);
+                mn = fminf(mn, gv[j]);
+            }
+        }
+        sRed[part * 128 + c] = mx;
+        sRed[512 + part * 128 + c] = mn;
     }
     __syncthreads();
     bool bad = false;
     if (tid < 128) {
-        const float mx = fmaxf(sRed[c], sRed[128 + c]), mn = fminf(sRed[256 + c], sRed[384 + c]);
+        const float mx = fmaxf(fmaxf(sRed[c], sRed[128 + c]), fmaxf(sRed[256 + c], sRed[384 + c]));
+        const float mn = fminf(fminf(sRed[512 + c], sRed[640 + c]), fminf(sRed[768 + c], sRed[896 + c]));
         sGm[c] = mx - kRefPair;
         bad = !(mx - mn <= 2.f * kRefPair) || !(mx <= 60.f);
     }
     const bool slow = __syncthreads_or(bad);
     if (tid == 0) a.slow[(size_t)cidx * a.H + h] = slow ? 1 : 0;
     if (slow) return;
-    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cw = warp >> 2;
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cg = warp >> 2;
     if (warp == 0) {
         tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
@@ -894,12 +905,13 @@ __global__ void __launch_bounds__(NTB, 1) pair_tc_kernel(const PairArgs a) {
     {
         const size_t cc = ((size_t)cidx * a.H + h) * 64 * 64;
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int idx = tid + NTB * it;  // 0 .. 2047
+        for (int it = 0; it < 2048 / NTP; ++it) {
+            const int idx = tid + NTP * it;  // 0 .. 2047
             const int m = idx >> 4, c4 = idx & 15;
             const int r = m & 63;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < L) v = *reinterpret_cast<const float4*>((m < 64 ? a.dAr : a.dP) + cc + r * 64 + 4 * c4);
+            if (r < L)
+                v = __ldg(reinterpret_cast<const float4*>((m < 64 ? a.dAr : a.dP) + cc + r * 64 + 4 * c4));
             v = round4_tf32(v);
             const int blk = c4 >> 3, q16 = c4 & 7;
             *reinterpret_cast<float4*>(sm + OFF_X1 + blk * 16384 + sw128_off(m, q16)) = v;
@@ -909,15 +921,15 @@ __global__ void __launch_bounds__(NTB, 1) pair_tc_kernel(const PairArgs a) {
     __syncthreads();  // Gm visible
     // K * E^-1, K * E, Q * E: row r, channels 4 c4 .. 4 c4 + 3
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-        const int idx = tid + NTB * it;  // 0 .. 2047
+    for (int it = 0; it < 2048 / NTP; ++it) {
+        const int idx = tid + NTP * it;  // 0 .. 2047
         const int r = idx >> 5, c4 = idx & 31;
         float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv, ke = kv, ki = kv;
         if (r < L) {
             const size_t gi = base + r * rowH + 4 * c4;
             kv = load4_f32<TIn>(Kg + gi);
             qv = load4_f32<TIn>(Qg + gi);
-            const float4 gv = *reinterpret_cast<const float4*>(a.G + gi);
+            const float4 gv = __ldg(reinterpret_cast<const float4*>(a.G + gi));
             const float4 gm = *reinterpret_cast<const float4*>(sGm + 4 * c4);
             const float x0 = gv.x - gm.x, x1 = gv.y - gm.y, x2 = gv.z - gm.z, x3 = gv.w - gm.w;
             const float e0 = __expf(x0), e1 = __expf(x1), e2 = __expf(x2), e3 = __expf(x3);
@@ -967,75 +979,94 @@ __global__ void __launch_bounds__(NTB, 1) pair_tc_kernel(const PairArgs a) {
         return;
     }
     tc_fence_after();
-    // 4. the accumulators to shared memory (over the operands, all read)
+    // 4. the accumulators to shared memory (over the operands, all read):
+    // warp (lane quarter, 32-column group cg)
     {
         float* D1 = reinterpret_cast<float*>(sm + OFF_D1);
         float* D2 = reinterpret_cast<float*>(sm + OFF_D2);
         const int row = 32 * quarter + lane;
         const uint32_t tl = static_cast<uint32_t>(32 * quarter) << 16;
+        uint32_t v[32];
+        tmem_ld32(tbase + tl + TM_1 + 32 * cg, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            uint32_t v[32];
-            tmem_ld32(tbase + tl + TM_1 + 64 * cw + 32 * x, v);
+        for (int y = 0; y < 32; y += 4)
+            *reinterpret_cast<float4*>(D1 + row * LDD + 32 * cg + y) =
+                make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                            __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+        if (quarter < 2) {
+            tmem_ld32(tbase + tl + TM_2 + 32 * cg, v);
             tmem_wait_ld();
 #pragma unroll
             for (int y = 0; y < 32; y += 4)
-                *reinterpret_cast<float4*>(D1 + row * LDD + 64 * cw + 32 * x + y) =
+                *reinterpret_cast<float4*>(D2 + row * LDD + 32 * cg + y) =
                     make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
                                 __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
-            if (quarter < 2) {
-                tmem_ld32(tbase + tl + TM_2 + 64 * cw + 32 * x, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int y = 0; y < 32; y += 4)
-                    *reinterpret_cast<float4*>(D2 + row * LDD + 64 * cw + 32 * x + y) =
-                        make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
-                                    __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
-            }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 256);
-    // 5. the epilogue of the exact kernel, channel c, rows 32 half .. + 31
+    // 5. the epilogue of the exact kernel, channel c, rows 16 part .. + 15
     {
         const float* D1 = reinterpret_cast<const float*>(sm + OFF_D1);
         const float* D2 = reinterpret_cast<const float*>(sm + OFF_D2);
         const float gm = sGm[c];
-        const float glast = a.G[base + (L - 1) * rowH + c];
-        float dG[32];
+        const float glast = __ldg(a.G + base + (L - 1) * rowH + c);
+        float dG[16];
         float tot = 0.f, last = 0.f;
+        // eight rows at a time: their loads (read-only path) issued together,
+        // then their arithmetic and stores
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int r = 32 * half + j;
-            dG[j] = 0.f;
-            if (r < L) {
-                const size_t gi = base + r * rowH + c;
-                const float gr = a.G[gi], qr = to_f32(Qg[gi]), kr = to_f32(Kg[gi]);
-                const float e = __expf(gr - gm), ei = __expf(gm - gr);
-                const float rowA = D1[r * LDD + c] * e, dQp = D1[(64 + r) * LDD + c] * e;
-                const float col = D2[r * LDD + c] * ei;
-                const float eg = expf(gr), eb = expf(glast - gr);
-                const float x = a.dQt[gi], y = a.dKt[gi], z = a.dKb[gi];
-                a.dq[gi] = dQp + x * eg;
-                a.dk[gi] = rowA + col + y * eg + z * eb;
-                dG[j] = kr * (rowA - col) + qr * dQp + x * qr * eg + y * kr * eg - z * kr * eb;
-                tot += dG[j];
-                last += z * kr * eb;
+        for (int b8 = 0; b8 < 2; ++b8) {
+            float gr[8], qr[8], kr[8], x[8], y[8], z[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = 16 * part + 8 * b8 + j;
+                if (r < L) {
+                    const size_t gi = base + r * rowH + c;
+                    gr[j] = __ldg(a.G + gi);
+                    qr[j] = to_f32(__ldg(Qg + gi));
+                    kr[j] = to_f32(__ldg(Kg + gi));
+                    x[j] = __ldg(a.dQt + gi);
+                    y[j] = __ldg(a.dKt + gi);
+                    z[j] = __ldg(a.dKb + gi);
+                } else {
+                    gr[j] = qr[j] = kr[j] = x[j] = y[j] = z[j] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = 16 * part + 8 * b8 + j;
+                dG[8 * b8 + j] = 0.f;
+                if (r < L) {
+                    const size_t gi = base + r * rowH + c;
+                    const float e = __expf(gr[j] - gm), ei = __expf(gm - gr[j]);
+                    const float rowA = D1[r * LDD + c] * e, dQp = D1[(64 + r) * LDD + c] * e;
+                    const float col = D2[r * LDD + c] * ei;
+                    const float eg = expf(gr[j]), eb = expf(glast - gr[j]);
+                    a.dq[gi] = dQp + x[j] * eg;
+                    a.dk[gi] = rowA + col + y[j] * eg + z[j] * eb;
+                    const float d = kr[j] * (rowA - col) + qr[j] * dQp + x[j] * qr[j] * eg +
+                                    y[j] * kr[j] * eg - z[j] * kr[j] * eb;
+                    dG[8 * b8 + j] = d;
+                    tot += d;
+                    last += z[j] * kr[j] * eb;
+                }
             }
         }
-        // [2][128] row-sum totals, [2][128] last-row terms, over the max / min
+        // [4][128] row-sum totals, [4][128] last-row terms, over the max / min
         // partials of step 1 (read before the range test's barrier)
         float* xch = sRed;
-        xch[half * 128 + c] = tot;
-        xch[256 + half * 128 + c] = last;
+        xch[part * 128 + c] = tot;
+        xch[512 + part * 128 + c] = last;
         __syncthreads();
-        float acc = expf(glast) * a.dGam[((size_t)cidx * a.H + h) * DD + c] + xch[256 + c] +
-                    xch[384 + c];
-        if (half == 0) acc += xch[128 + c];
+        float acc = expf(glast) * a.dGam[((size_t)cidx * a.H + h) * DD + c] + xch[512 + c] +
+                    xch[640 + c] + xch[768 + c] + xch[896 + c];
+        for (int p2 = part + 1; p2 < 4; ++p2) acc += xch[p2 * 128 + c];  // rows after this part
 #pragma unroll
-        for (int j = 31; j >= 0; --j) {
-            const int r = 32 * half + j;
+        for (int j = 15; j >= 0; --j) {
+            const int r = 16 * part + j;
             if (r < L) {
                 acc += dG[j];
                 a.dg[base + r * rowH + c] = acc;
@@ -1202,7 +1233,7 @@ cudaError_t launch_bwd_pair_tc(const TIn* q, const TIn* k, const float* G, const
     if (e != cudaSuccess) return e;
     const PairArgs a{q, k, G, dAr, dP, dQt, dKt, dKb, dGam, info, H, status, status, slow, dq, dk,
                      dg};
-    pair_tc_kernel<TIn><<<dim3(maxc, H), NTB, pr::SMEM, st>>>(a);
+    pair_tc_kernel<TIn><<<dim3(maxc, H), pr::NTP, pr::SMEM, st>>>(a);
     return cudaGetLastError();
 }
 
