@@ -109,14 +109,17 @@ __global__ void __launch_bounds__(256) bwd_apkb_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const float* __restrict__ g,
     const float* __restrict__ beta, const int4* __restrict__ info, int H,
     const uint32_t* status, float* __restrict__ G, float* __restrict__ Ar_out,
-    float* __restrict__ P_out, float* __restrict__ Kb, float* __restrict__ Rk, bool rt) {
-    // rt: P and Kb are tf32 operands of the tensor-core kernels after this one
+    float* __restrict__ P_out, float* __restrict__ Kb, float* __restrict__ Rk, bool rt,
+    const int* __restrict__ slow) {
+    // rt: P and Kb are tf32 operands of the tensor-core kernels after this one;
+    // slow != NULL: only the chunks the tensor-core kernel left (flag 1)
     constexpr int LDK = DK + 1;
     if (status_bad(status)) return;
     const int cidx = blockIdx.x, h = blockIdx.y;
     const int4 ci = info[cidx];
     const int L = ci.z;
     if (L <= 0) return;
+    if (slow && !slow[(size_t)cidx * H + h]) return;
     const int tid = threadIdx.x;
     extern __shared__ __align__(16) float sm[];
     float* Qs = sm;
@@ -935,10 +938,16 @@ cudaError_t launch_intra3(const BwdBufs& b, const TIn* Q, const TIn* K, const TI
     const Workspace& w = b.w;
     const dim3 grid(maxc, H);
     cudaError_t e;
+    if (tc) {  // A and P as products; chunks outside the exponent range stay exact
+        e = launch_bwd_apkb_tc<TIn>(Q, K, g, beta, w.chunk_info, total, maxc, H, w.status, b.slow,
+                                    w.G, b.Ar, b.Pm, b.Kb, w.W, st);
+        if (e != cudaSuccess) return e;
+    }
     size_t sm = apkb_smem(DK);
     if ((e = set_smem(bwd_apkb_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
     bwd_apkb_kernel<DK, TIn><<<grid, 256, sm, st>>>(Q, K, g, beta, w.chunk_info, H, w.status,
-                                                    w.G, b.Ar, b.Pm, b.Kb, w.W, tc);
+                                                    w.G, b.Ar, b.Pm, b.Kb, w.W, tc,
+                                                    tc ? b.slow : nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     sm = subst_smem(DK, dv);
     if ((e = set_smem(bwd_subst_kernel<DK, TIn>, sm)) != cudaSuccess) return e;

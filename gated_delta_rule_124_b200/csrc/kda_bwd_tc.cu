@@ -1075,6 +1075,220 @@ __global__ void __launch_bounds__(pr::NTP, 1) pair_tc_kernel(const PairArgs a) {
     }
 }
 
+// ------------------------------------------------------------ A and P
+// The recompute's first step per (chunk, head): G (the in-chunk inclusive sum
+// of g), Kb = K exp(G_last - G), the right-hand sides b K exp(G), and
+//   A[r][i] = sum_c k_rc k_ic exp(G_rc - G_ic)  (i < r; without b),
+//   P[r][i] = sum_c q_rc k_ic exp(G_rc - G_ic)  (i <= r)
+// as one M = 128 product [K * E ; Q * E] (K * E^-1)^T under the per-channel
+// reference of the pair kernel.  A feeds the triangular solves, so the
+// product is taken in three tf32 passes (each operand split into a rounded
+// high part and the rounded remainder: hi hi + hi lo + lo hi), which keeps it
+// close to fp32.  A chunk outside the reference's range sets slow = 1; the
+// exact kernel then recomputes that chunk.
+namespace ap {
+constexpr uint32_t OFF_AH = 0;        // [K*E ; Q*E] high: 4 blocks [128][32] (K-major)
+constexpr uint32_t OFF_AL = 65536;    // low
+constexpr uint32_t OFF_BH = 131072;   // K*E^-1 [64 i][128 c] high: 4 blocks [64][32]
+constexpr uint32_t OFF_BL = 163840;   // low
+constexpr uint32_t OFF_RED = 196608;  // [4][128] totals, max, min
+constexpr uint32_t OFF_BAR = OFF_RED + 6144;
+constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+constexpr int NT = 512;
+}  // namespace ap
+
+struct ApArgs {
+    const void* q;
+    const void* k;
+    const float* g;
+    const float* beta;
+    const int4* info;
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    int* slow;
+    float* G;
+    float* Ar;
+    float* P;
+    float* Kb;
+    float* Rk;
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(ap::NT, 1) apkb_tc_kernel(const ApArgs a) {
+    using namespace ap;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_skip;
+    const int cidx = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int4 ci = a.info[cidx];
+    const int t0 = ci.y, L = ci.z;
+    if (tid == 0) s_skip = status_bad(a.status) || L <= 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* sRed = reinterpret_cast<float*>(sm + OFF_RED);  // tot [4][128], mx [4][128], mn [4][128]
+    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + ap::OFF_BAR);
+    const TIn* Qg = static_cast<const TIn*>(a.q);
+    const TIn* Kg = static_cast<const TIn*>(a.k);
+    const int c = tid & 127, part = tid >> 7;  // channel, rows 16 part .. + 15
+    const size_t rowH = (size_t)a.H * DD;
+    const size_t base = ((size_t)t0 * a.H + h) * DD;
+    // 1. G: each part's inclusive prefix over its 16 rows, then the totals of
+    // the parts above it; per-channel max / min
+    float gv[16], kv[16], qv[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int r = 16 * part + j;
+        const bool in = r < L;
+        gv[j] = in ? __ldg(a.g + base + r * rowH + c) : 0.f;
+        kv[j] = in ? to_f32(__ldg(Kg + base + r * rowH + c)) : 0.f;
+        qv[j] = in ? to_f32(__ldg(Qg + base + r * rowH + c)) : 0.f;
+    }
+    float run = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        run += gv[j];
+        gv[j] = run;
+    }
+    sRed[part * 128 + c] = run;
+    __syncthreads();
+    float off = 0.f, glast = 0.f;
+#pragma unroll
+    for (int p2 = 0; p2 < 4; ++p2) {
+        const float t = sRed[p2 * 128 + c];
+        if (p2 < part) off += t;
+        glast += t;  // the sum of every row < L
+    }
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        gv[j] += off;
+        if (16 * part + j < L) {
+            mx = fmaxf(mx, gv[j]);
+            mn = fminf(mn, gv[j]);
+        }
+    }
+    sRed[512 + part * 128 + c] = mx;
+    sRed[1024 + part * 128 + c] = mn;
+    // G, Kb and the right-hand sides: exact, whatever the range
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int r = 16 * part + j;
+        if (r < L) {
+            const size_t gi = base + r * rowH + c;
+            a.G[gi] = gv[j];
+            const float kb = kv[j] * __expf(glast - gv[j]);
+            a.Kb[gi] = round_tf32(kb);
+            a.Rk[gi] = __ldg(a.beta + (size_t)(t0 + r) * a.H + h) * kv[j] * __expf(gv[j]);
+        }
+    }
+    __syncthreads();
+    const float gmx = fmaxf(fmaxf(sRed[512 + c], sRed[640 + c]), fmaxf(sRed[768 + c], sRed[896 + c]));
+    const float gmn = fminf(fminf(sRed[1024 + c], sRed[1152 + c]), fminf(sRed[1280 + c], sRed[1408 + c]));
+    const bool bad = !(gmx - gmn <= 160.f) || !(gmx <= 60.f);
+    const bool slow = __syncthreads_or(bad);
+    if (tid == 0) a.slow[(size_t)cidx * a.H + h] = slow ? 1 : 0;
+    if (slow) return;
+    const float gm = gmx - 80.f;
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cg = warp >> 2;
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 64);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    // 2. the operands, split into tf32 high and low parts; element (r, c) of
+    // a K-major [rows][128] tile: block c / 32, 16-byte chunk (c % 32) / 4
+    {
+        const int blk = c >> 5, q16 = (c & 31) >> 2, w4 = (c & 3) * 4;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int r = 16 * part + j;
+            float ke = 0.f, qe = 0.f, ki = 0.f;
+            if (r < L) {
+                const float x = gv[j] - gm;
+                const float e = __expf(x), ei = __expf(-x);
+                ke = kv[j] * e;
+                qe = qv[j] * e;
+                ki = kv[j] * ei;
+            }
+            const float keh = round_tf32(ke), qeh = round_tf32(qe), kih = round_tf32(ki);
+            const uint32_t oa = blk * 16384 + sw128_off(r, q16) + w4;
+            const uint32_t oq = blk * 16384 + sw128_off(64 + r, q16) + w4;
+            const uint32_t ob = blk * 8192 + sw128_off(r, q16) + w4;
+            *reinterpret_cast<float*>(sm + OFF_AH + oa) = keh;
+            *reinterpret_cast<float*>(sm + OFF_AL + oa) = round_tf32(ke - keh);
+            *reinterpret_cast<float*>(sm + OFF_AH + oq) = qeh;
+            *reinterpret_cast<float*>(sm + OFF_AL + oq) = round_tf32(qe - qeh);
+            *reinterpret_cast<float*>(sm + OFF_BH + ob) = kih;
+            *reinterpret_cast<float*>(sm + OFF_BL + ob) = round_tf32(ki - kih);
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s_tmem;
+    // 3. D = Ah Bh^T + Ah Bl^T + Al Bh^T (M = 128, N = 64, K = 128)
+    if (tid == 0) {
+        constexpr uint32_t id = idesc_tf32(128, 64, false, false);
+        const uint32_t As[3] = {OFF_AH, OFF_AH, OFF_AL}, Bs[3] = {OFF_BH, OFF_BL, OFF_BH};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {
+                const int kb = ks >> 2, kk = ks & 3;
+                mma_tf32_tc(tbase, sdesc_sw128(sbase + As[pass] + kb * 16384 + kk * 32, 16, 1024),
+                            sdesc_sw128(sbase + Bs[pass] + kb * 8192 + kk * 32, 16, 1024), id,
+                            (pass | ks) > 0);
+            }
+        mma_commit(bar_mma);
+    }
+    const bool ok = mbar_wait(bar_mma, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            mbar_wait(bar_mma, 0, kWaitNs);
+            atomicOr(a.status_out, STATUS_TIMEOUT);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tbase, 64);
+        return;
+    }
+    tc_fence_after();
+    // 4. masked rows out: lane m of quarter (m < 64: A row m; else P row m - 64),
+    // 32 columns per warp (cg 0, 1)
+    if (cg < 2) {
+        const int m = 32 * quarter + lane;
+        const int r = m & 63, i0 = 32 * cg;
+        uint32_t v[32];
+        tmem_ld32(tbase + (static_cast<uint32_t>(32 * quarter) << 16) + i0, v);
+        tmem_wait_ld();
+        const bool isP = m >= 64;
+        float* dst = (isP ? a.P : a.Ar) + ((size_t)cidx * a.H + h) * 64 * 64 + r * 64 + i0;
+#pragma unroll
+        for (int y = 0; y < 32; y += 4) {
+            float o[4];
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const int i = i0 + y + z;
+                const bool keep = r < L && (isP ? i <= r : i < r);
+                const float x = __uint_as_float(v[y + z]);
+                o[z] = keep ? (isP ? round_tf32(x) : x) : 0.f;
+            }
+            *reinterpret_cast<float4*>(dst + y) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 64);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void* ptr = nullptr;
@@ -1246,5 +1460,33 @@ template cudaError_t launch_bwd_pair_tc<__nv_bfloat16>(
     const __nv_bfloat16*, const __nv_bfloat16*, const float*, const float*, const float*,
     const float*, const float*, const float*, const float*, const int4*, int, int, int,
     uint32_t*, int*, float*, float*, float*, cudaStream_t);
+
+}  // namespace kda
+
+namespace kda {
+
+template <typename TIn>
+cudaError_t launch_bwd_apkb_tc(const TIn* q, const TIn* k, const float* g, const float* beta,
+                               const int4* info, int total, int maxc, int H, uint32_t* status,
+                               int* slow, float* G, float* Ar, float* P, float* Kb, float* Rk,
+                               cudaStream_t st) {
+    if (maxc == 0 || total == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(apkb_tc_kernel<TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ap::SMEM);
+    if (e != cudaSuccess) return e;
+    const ApArgs a{q, k, g, beta, info, H, status, status, slow, G, Ar, P, Kb, Rk};
+    apkb_tc_kernel<TIn><<<dim3(maxc, H), ap::NT, ap::SMEM, st>>>(a);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_bwd_apkb_tc<float>(const float*, const float*, const float*,
+                                               const float*, const int4*, int, int, int,
+                                               uint32_t*, int*, float*, float*, float*, float*,
+                                               float*, cudaStream_t);
+template cudaError_t launch_bwd_apkb_tc<__nv_bfloat16>(const __nv_bfloat16*,
+                                                       const __nv_bfloat16*, const float*,
+                                                       const float*, const int4*, int, int, int,
+                                                       uint32_t*, int*, float*, float*, float*,
+                                                       float*, float*, cudaStream_t);
 
 }  // namespace kda

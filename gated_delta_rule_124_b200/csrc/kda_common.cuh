@@ -238,6 +238,14 @@ cudaError_t launch_bwd_dense_tc(const TIn* k, const TIn* dout, const float* G, c
                                 const float* dSx, const float* dbB, const int4* info, int total,
                                 int maxc, int H, uint32_t* status, float* dQt, float* dKt,
                                 float* dKb, float* dGam, float* dbeta, cudaStream_t st);
+// G, Kb, the right-hand sides b K exp(G), and A, P as a three-pass tf32
+// product under a per-channel exponent reference (slow[] = 1: the chunk is
+// left to the exact kernel); kda_bwd_tc.cu.
+template <typename TIn>
+cudaError_t launch_bwd_apkb_tc(const TIn* q, const TIn* k, const float* g, const float* beta,
+                               const int4* info, int total, int maxc, int H, uint32_t* status,
+                               int* slow, float* G, float* Ar, float* P, float* Kb, float* Rk,
+                               cudaStream_t st);
 // The pair sums (dq, dk, dg) as tensor-core products under a per-channel
 // exponent reference; a chunk whose gate range exceeds it gets slow[] = 1 and
 // is left to the exact CUDA-core kernel; kda_bwd_tc.cu.
