@@ -701,14 +701,15 @@ def backward_flops(head_tokens, dk, dv, C=64):
     A, P, W, Ut and chain recomputed, then E, F, the reverse chain, the back
     substitution, the products with U, S and dS', and the pair sums), two
     flops each.  Returns (on the tensor cores, on the CUDA cores) for dk = dv
-    = 128, where the chains, E, F and the dense products run as tcgen05
-    products; other shapes run everything on the CUDA cores."""
+    = 128, where A/P, the chains, E, F, the dense products and the pair sums
+    run as tcgen05 products; other shapes run everything on the CUDA cores."""
     tri, stri = C * (C + 1) // 2, C * (C - 1) // 2
-    tensor = (2 * C * dk * dv + 2 * C * dk * dv                    # the two chains
-              + tri * dv + 2 * C * dk * dv + 3 * C * dk * dv)      # E; F; dense
-    alu = (2 * tri * dk + stri * (dk + dv)                         # A, P; [W | Ut]
-           + stri * dv + 2 * C * C * dv                            # Y; Y U^T, dO U^T
-           + 4 * tri * dk)                                         # pair sums
+    tensor = (2 * tri * dk                                         # A, P
+              + 2 * C * dk * dv + 2 * C * dk * dv                  # the two chains
+              + tri * dv + 2 * C * dk * dv + 3 * C * dk * dv       # E; F; dense
+              + 4 * tri * dk)                                      # pair sums
+    alu = (stri * (dk + dv)                                        # [W | Ut]
+           + stri * dv + 2 * C * C * dv)                           # Y; Y U^T, dO U^T
     if not (dk == 128 and dv == 128):
         tensor, alu = 0, tensor + alu
     return 2 * tensor * head_tokens / C, 2 * alu * head_tokens / C

@@ -7,7 +7,7 @@ import torch
 import gated_delta_rule_124_b200 as kda
 from gated_delta_rule_124_b200 import workloads as wl
 from oracle import backward as bwd
-from tests.helpers import rel_err
+from tests.helpers import record, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -73,7 +73,8 @@ def test_backward_matches_autograd(name, with_dhT):
     ref = bwd.backward(case.q, case.k, case.v, case.g, case.beta, case.initial_state, do,
                        dhT, cu)
     for name_, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), got, ref):
-        assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
+        e = record(f"backward {name} {'with' if with_dhT else 'no'} dS_T", name_, x, r)
+        assert e <= 1e-3, (name_, e)
 
 
 @pytest.mark.parametrize("unit", [(0, 0), (1, 31)])
@@ -99,7 +100,8 @@ def test_backward_bench_workload_sampled_heads(unit):
     sel = (one(got[0]), one(got[1]), one(got[2]), one(got[3]), got[4][rows, h:h + 1],
            got[5][s:s + 1, h:h + 1])
     for name_, x, r in zip(("dq", "dk", "dv", "dg", "dbeta", "dh0"), sel, ref):
-        assert rel_err(x, r) <= 1e-3, (name_, rel_err(x, r))
+        e = record(f"backward B=2 T=2048 H=32 d=128 bf16 (seq {s}, head {h})", name_, x, r)
+        assert e <= 1e-3, (name_, e)
 
 
 def test_backward_bad_cu_seqlens_reported_on_device():
