@@ -56,6 +56,7 @@ struct BwdBufs {
     float* dGam;  // [maxc, H, dk]
     float* dbB;   // [total, H]
     int* slow;    // [maxc, H]  (tensor-core pair sums) 1: the chunk is left to the exact kernel
+    float* Tm;    // [maxc, H, C, C]     (tensor-core solves) T = (I + A)^-1
     size_t bytes;
 };
 
@@ -88,6 +89,7 @@ BwdBufs carve_bwd(void* base, int total, int N, int H, int dk, int dv) {
     b.dGam = take(maxc * H * dk);
     b.dbB = take((size_t)total * H);
     b.slow = reinterpret_cast<int*>(take(maxc * H));
+    b.Tm = take(cc);
     b.bytes = off;
     return b;
 }
@@ -949,11 +951,17 @@ cudaError_t launch_intra3(const BwdBufs& b, const TIn* Q, const TIn* K, const TI
                                                     w.G, b.Ar, b.Pm, b.Kb, w.W, tc,
                                                     tc ? b.slow : nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    sm = subst_smem(DK, dv);
-    if ((e = set_smem(bwd_subst_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
-    bwd_subst_kernel<DK, TIn><<<grid, 256, sm, st>>>(V, beta, b.Ar, w.chunk_info, H, dv,
-                                                     w.status, w.W, w.U, tc);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (tc) {
+        e = launch_bwd_subst_tc<TIn>(V, beta, b.Ar, w.chunk_info, total, maxc, H, w.status, w.W,
+                                     w.U, b.Tm, st);
+    } else {
+        sm = subst_smem(DK, dv);
+        if ((e = set_smem(bwd_subst_kernel<DK, TIn>, sm)) != cudaSuccess) return e;
+        bwd_subst_kernel<DK, TIn><<<grid, 256, sm, st>>>(V, beta, b.Ar, w.chunk_info, H, dv,
+                                                         w.status, w.W, w.U, tc);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
     if (tc)
         return launch_bwd_ef_tc<TIn>(Q, DO, w.G, b.Pm, w.W, w.chunk_info, total, maxc, H,
                                      w.status, b.E, b.F, st);
@@ -1006,7 +1014,11 @@ cudaError_t run_bwd(const BwdBufs& b, const void* q, const void* k, const void* 
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (maxc == 0) return cudaSuccess;
-    {
+    if (tc) {
+        e = launch_bwd_solve_tc<TIn>(V, DO, b.Ar, beta, w.U, b.dU, b.Tm, w.chunk_info, total, maxc,
+                                     H, w.status, b.Y, dvv, b.dAr, b.dP, b.dbB, st);
+        if (e != cudaSuccess) return e;
+    } else {
         const size_t sm = solve_smem(dv);
         if ((e = set_smem(bwd_solve_kernel<TIn>, sm)) != cudaSuccess) return e;
         bwd_solve_kernel<TIn><<<dim3(maxc, H), 256, sm, st>>>(V, DO, b.Ar, beta, w.U, b.dU,

@@ -1289,6 +1289,494 @@ __global__ void __launch_bounds__(ap::NT, 1) apkb_tc_kernel(const ApArgs a) {
     if (warp == 0) tmem_dealloc(tbase, 64);
 }
 
+// ------------------------------------------------------------ T = (I + A)^-1
+// T = (I + diag(b) Ar)^-1 of one chunk in fp32, in shared memory ([64][LDT]):
+// the four 16 x 16 diagonal blocks by forward substitution (one column per
+// thread), then the blocks below them a diagonal at a time, T_IJ = -T_II
+// sum_{K=J}^{I-1} A_IK T_KJ (the lower-triangular block inverse).  Ar rows
+// past the chunk are zero and b there is zero, so T is the identity there.
+constexpr int LDT = 65;
+__device__ void tri_inverse(const float* Ar, const float* bs, float* Tm, float* Msc, int tid,
+                            int nt) {
+    for (int e = tid; e < 64 * LDT; e += nt) Tm[e] = 0.f;
+    __syncthreads();
+    if (tid < 64) {  // diagonal block I, column j
+        const int I = tid >> 4, j = tid & 15, o = 16 * I;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) t[r] = r == j ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+            if (r > j) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < r; ++i)
+                    if (i >= j) acc += Ar[(o + r) * LDT + o + i] * t[i];
+                t[r] = -bs[o + r] * acc;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tm[(o + r) * LDT + o + j] = t[r];
+    }
+    __syncthreads();
+    for (int d = 1; d < 4; ++d) {
+        const int nb = 4 - d;  // blocks (J + d, J), J = 0 .. nb - 1
+        for (int e = tid; e < nb * 256; e += nt) {  // M_IJ = sum_K A_IK T_KJ
+            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15, I = J + d;
+            float acc = 0.f;
+            for (int K = J; K < I; ++K)
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc += Ar[(16 * I + r) * LDT + 16 * K + i] * Tm[(16 * K + i) * LDT + 16 * J + c];
+            Msc[e] = bs[16 * I + r] * acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nb * 256; e += nt) {  // T_IJ = -T_II M_IJ
+            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15, I = J + d;
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (k <= r) acc += Tm[(16 * I + r) * LDT + 16 * I + k] * Msc[J * 256 + k * 16 + c];
+            Tm[(16 * I + r) * LDT + 16 * J + c] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
+// x and its tf32 split
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+    hi = round_tf32(x);
+    lo = round_tf32(x - hi);
+}
+
+// ------------------------------------------------------------ [W | Ut]
+// (I + A) [W | Ut] = [b Kt | b V] as [W | Ut] = T [b Kt | b V]: T in fp32 by
+// tri_inverse (also written out for the back substitution), the product in
+// three tf32 passes (M = 64 padded to 128, N = 256, K = 64).
+namespace sb {
+constexpr int NT = 512;
+constexpr uint32_t OFF_AH = 0;        // T high: 2 blocks [128][32], K-major (rows 64-127 zero)
+constexpr uint32_t OFF_AL = 32768;    // T low
+constexpr uint32_t OFF_BH = 65536;    // [b Kt | b V] high: 8 blocks [64 i][32 n], MN-major
+constexpr uint32_t OFF_BL = 131072;   // low; before it is built: Ar, T, the block scratch
+constexpr uint32_t OFF_BS = 196608;   // b [64]
+constexpr uint32_t OFF_BAR = OFF_BS + 256;
+constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+}  // namespace sb
+
+struct SubstArgs {
+    const void* v;
+    const float* beta;
+    const float* Ar;
+    const int4* info;
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    float* W;   // in: b Kt; out: W (rounded to tf32)
+    float* Ut;  // out
+    float* Tout;  // [chunks, H, 64, 64]
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(sb::NT, 1) subst_tc_kernel(const SubstArgs a) {
+    using namespace sb;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_skip;
+    const int cidx = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int4 ci = a.info[cidx];
+    const int t0 = ci.y, L = ci.z;
+    if (tid == 0) s_skip = status_bad(a.status) || L <= 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* Ar = reinterpret_cast<float*>(sm + OFF_BL);
+    float* Tm = Ar + 64 * LDT;
+    float* Msc = Tm + 64 * LDT;
+    float* bs = reinterpret_cast<float*>(sm + OFF_BS);
+    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + sb::OFF_BAR);
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cg = warp >> 2;
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    const size_t cc = ((size_t)cidx * a.H + h) * 64 * 64;
+    for (int e = tid; e < 64 * 64; e += NT) Ar[(e >> 6) * LDT + (e & 63)] = __ldg(a.Ar + cc + e);
+    if (tid < 64) bs[tid] = tid < L ? __ldg(a.beta + (size_t)(t0 + tid) * a.H + h) : 0.f;
+    __syncthreads();
+    tri_inverse(Ar, bs, Tm, Msc, tid, NT);
+    // T out (fp32) and T's tf32 split as the K-major A operand
+    for (int e = tid; e < 128 * 64; e += NT) {
+        const int r = e >> 6, i = e & 63;
+        const float x = r < 64 ? Tm[r * LDT + i] : 0.f;
+        if (r < 64) a.Tout[cc + e] = x;
+        float hi, lo;
+        split_tf32(x, hi, lo);
+        const uint32_t o = (i >> 5) * 16384 + sw128_off(r, (i & 31) >> 2) + 4 * (i & 3);
+        *reinterpret_cast<float*>(sm + OFF_AH + o) = hi;
+        *reinterpret_cast<float*>(sm + OFF_AL + o) = lo;
+    }
+    __syncthreads();  // T, Ar read: the low half of B may overwrite them
+    // [b Kt | b V] rows i < L (zeros after), four columns per float4
+    {
+        const size_t base = ((size_t)t0 * a.H + h) * DD;
+        const size_t rowH = (size_t)a.H * DD;
+        const TIn* Vg = static_cast<const TIn*>(a.v);
+#pragma unroll
+        for (int it = 0; it < 4096 / NT; ++it) {
+            const int idx = tid + NT * it;
+            const int i = idx >> 6, n4 = idx & 63;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < L) {
+                if (n4 < 32) {
+                    x = __ldg(reinterpret_cast<const float4*>(a.W + base + i * rowH + 4 * n4));
+                } else {
+                    const float b = bs[i];
+                    const float4 vv = load4_f32<TIn>(Vg + base + i * rowH + 4 * (n4 - 32));
+                    x = make_float4(b * vv.x, b * vv.y, b * vv.z, b * vv.w);
+                }
+            }
+            float4 hi, lo;
+            split_tf32(x.x, hi.x, lo.x);
+            split_tf32(x.y, hi.y, lo.y);
+            split_tf32(x.z, hi.z, lo.z);
+            split_tf32(x.w, hi.w, lo.w);
+            const uint32_t o = (n4 >> 3) * 8192 + sw128_32b_off(i, n4 & 7);
+            *reinterpret_cast<float4*>(sm + OFF_BH + o) = hi;
+            *reinterpret_cast<float4*>(sm + OFF_BL + o) = lo;
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s_tmem;
+    if (tid == 0) {
+        constexpr uint32_t id = idesc_tf32(128, 256, false, true);
+        const uint32_t As[3] = {OFF_AH, OFF_AH, OFF_AL}, Bs[3] = {OFF_BH, OFF_BL, OFF_BH};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int kb = ks >> 2, kk = ks & 3;
+                mma_tf32_tc(tbase, sdesc_sw128(sbase + As[pass] + kb * 16384 + kk * 32, 16, 1024),
+                            sdesc_sw128_32b(sbase + Bs[pass] + ks * 1024, 8192, 512), id,
+                            (pass | ks) > 0);
+            }
+        mma_commit(bar_mma);
+    }
+    const bool ok = mbar_wait(bar_mma, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            mbar_wait(bar_mma, 0, kWaitNs);
+            atomicOr(a.status_out, STATUS_TIMEOUT);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tbase, 256);
+        return;
+    }
+    tc_fence_after();
+    // rows r < L (lanes 0-63): columns 64 cg .. + 63 (cg 0, 1: W; 2, 3: Ut)
+    if (quarter < 2) {
+        const int r = 32 * quarter + lane;
+        const size_t row = ((size_t)(t0 + r) * a.H + h) * DD;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            uint32_t v[32];
+            tmem_ld32(tbase + (static_cast<uint32_t>(32 * quarter) << 16) + 64 * cg + 32 * x, v);
+            tmem_wait_ld();
+            if (r < L) {
+                const int col = 64 * cg + 32 * x;
+                float* dst = col < 128 ? a.W + row + col : a.Ut + row + col - 128;
+#pragma unroll
+                for (int y = 0; y < 32; y += 4) {
+                    float4 o4 = make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                            __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+                    if (col < 128) o4 = round4_tf32(o4);
+                    *reinterpret_cast<float4*>(dst + y) = o4;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
+// ------------------------------------------------------------ the solve
+// (I + A)^T Y = dU as Y = T^T dU (T from the substitution kernel), then
+// dA = -strict_lower(Y U^T) and dP = lower(dO U^T) as one M = 128 product
+// [Y ; dO] U^T, both in three tf32 passes; dv = b Y, and the partial
+// gradient of b, Y.V + sum_i dA[r][i] Ar[r][i].
+namespace sv {
+constexpr int NT = 512;
+constexpr uint32_t OFF_TH = 0;        // T high: 2 blocks [64 i][32 r] (MN-major A; M padded)
+constexpr uint32_t OFF_TL = 16384;    // T low
+constexpr uint32_t OFF_DH = 32768;    // dU high: 4 blocks [64 i][32 j] (MN-major B)
+constexpr uint32_t OFF_DL = 65536;    // dU low
+constexpr uint32_t OFF_YH = 0;        // (second product) [Y ; dO] high: 4 blocks [128][32] (K-major)
+constexpr uint32_t OFF_YL = 65536;    // low
+constexpr uint32_t OFF_UH = 131072;   // U high: 4 blocks [64][32] (K-major B)
+constexpr uint32_t OFF_UL = 163840;   // low
+constexpr uint32_t OFF_RED = 196608;  // Y.V partials [4][64], dA.Ar partials [2][64]
+constexpr uint32_t OFF_BS = OFF_RED + 1536;
+constexpr uint32_t OFF_BAR = OFF_BS + 256;
+constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+constexpr uint32_t TM_Y = 0, TM_2 = 128;
+}  // namespace sv
+
+struct SolveArgs {
+    const void* v;
+    const void* dout;
+    const float* Ar;
+    const float* beta;
+    const float* U;
+    const float* dU;
+    const float* Tm;
+    const int4* info;
+    int H;
+    const uint32_t* status;
+    uint32_t* status_out;
+    float* Y;
+    float* dv;
+    float* dAr;
+    float* dP;
+    float* dbB;
+};
+
+template <typename TIn>
+__global__ void __launch_bounds__(sv::NT, 1) solve_tc_kernel(const SolveArgs a) {
+    using namespace sv;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_skip;
+    const int cidx = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int4 ci = a.info[cidx];
+    const int t0 = ci.y, L = ci.z;
+    if (tid == 0) s_skip = status_bad(a.status) || L <= 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float* sRed = reinterpret_cast<float*>(sm + OFF_RED);
+    float* bs = reinterpret_cast<float*>(sm + OFF_BS);
+    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + sv::OFF_BAR);
+    const int warp = tid >> 5, lane = tid & 31, quarter = warp & 3, cg = warp >> 2;
+    const TIn* Vg = static_cast<const TIn*>(a.v);
+    const TIn* Dg = static_cast<const TIn*>(a.dout);
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    const size_t cc = ((size_t)cidx * a.H + h) * 64 * 64;
+    const size_t base = ((size_t)t0 * a.H + h) * DD;
+    const size_t rowH = (size_t)a.H * DD;
+    if (tid < 64) bs[tid] = tid < L ? __ldg(a.beta + (size_t)(t0 + tid) * a.H + h) : 0.f;
+    // T (rows i, columns r contiguous: the MN-major A of T^T) and dU (rows i)
+#pragma unroll
+    for (int it = 0; it < 1024 / NT; ++it) {
+        const int idx = tid + NT * it;  // 0 .. 1023: (i, r4)
+        const int i = idx >> 4, r4 = idx & 15;
+        const float4 x = __ldg(reinterpret_cast<const float4*>(a.Tm + cc + i * 64 + 4 * r4));
+        float4 hi, lo;
+        split_tf32(x.x, hi.x, lo.x);
+        split_tf32(x.y, hi.y, lo.y);
+        split_tf32(x.z, hi.z, lo.z);
+        split_tf32(x.w, hi.w, lo.w);
+        const uint32_t o = (r4 >> 3) * 8192 + sw128_32b_off(i, r4 & 7);
+        *reinterpret_cast<float4*>(sm + OFF_TH + o) = hi;
+        *reinterpret_cast<float4*>(sm + OFF_TL + o) = lo;
+    }
+#pragma unroll
+    for (int it = 0; it < 2048 / NT; ++it) {
+        const int idx = tid + NT * it;  // 0 .. 2047: (i, j4)
+        const int i = idx >> 5, j4 = idx & 31;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < L) x = __ldg(reinterpret_cast<const float4*>(a.dU + base + i * rowH + 4 * j4));
+        float4 hi, lo;
+        split_tf32(x.x, hi.x, lo.x);
+        split_tf32(x.y, hi.y, lo.y);
+        split_tf32(x.z, hi.z, lo.z);
+        split_tf32(x.w, hi.w, lo.w);
+        const uint32_t o = (j4 >> 3) * 8192 + sw128_32b_off(i, j4 & 7);
+        *reinterpret_cast<float4*>(sm + OFF_DH + o) = hi;
+        *reinterpret_cast<float4*>(sm + OFF_DL + o) = lo;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s_tmem;
+    if (tid == 0) {  // Y = T^T dU: M = 64 padded to 128, N = 128, K = 64
+        constexpr uint32_t id = idesc_tf32(128, 128, true, true);
+        const uint32_t As[3] = {OFF_TH, OFF_TH, OFF_TL}, Bs[3] = {OFF_DH, OFF_DL, OFF_DH};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_tf32_tc(tbase + TM_Y, sdesc_sw128_32b(sbase + As[pass] + ks * 1024, 8192, 512),
+                            sdesc_sw128_32b(sbase + Bs[pass] + ks * 1024, 8192, 512), id,
+                            (pass | ks) > 0);
+        mma_commit(bar_mma);
+    }
+    bool ok = mbar_wait(bar_mma, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            mbar_wait(bar_mma, 0, kWaitNs);
+            atomicOr(a.status_out, STATUS_TIMEOUT);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tbase, 256);
+        return;
+    }
+    tc_fence_after();
+    // Y rows (lanes 0-63), 32 columns per warp: Y, dv out, Y.V, and the split
+    // of Y as rows 0-63 of the second product's A
+    if (quarter < 2) {
+        const int r = 32 * quarter + lane;
+        uint32_t v[32];
+        tmem_ld32(tbase + TM_Y + (static_cast<uint32_t>(32 * quarter) << 16) + 32 * cg, v);
+        tmem_wait_ld();
+        float yv = 0.f;
+        const size_t row = base + r * rowH + 32 * cg;
+        const bool in = r < L;
+#pragma unroll
+        for (int y = 0; y < 32; y += 4) {
+            float4 y4 = make_float4(__uint_as_float(v[y]), __uint_as_float(v[y + 1]),
+                                    __uint_as_float(v[y + 2]), __uint_as_float(v[y + 3]));
+            if (!in) y4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (in) {
+                const float b = bs[r];
+                *reinterpret_cast<float4*>(a.Y + row + y) = round4_tf32(y4);
+                *reinterpret_cast<float4*>(a.dv + row + y) =
+                    make_float4(b * y4.x, b * y4.y, b * y4.z, b * y4.w);
+                const float4 vv = load4_f32<TIn>(Vg + row + y);
+                yv += y4.x * vv.x + y4.y * vv.y + y4.z * vv.z + y4.w * vv.w;
+            }
+            float4 hi, lo;
+            split_tf32(y4.x, hi.x, lo.x);
+            split_tf32(y4.y, hi.y, lo.y);
+            split_tf32(y4.z, hi.z, lo.z);
+            split_tf32(y4.w, hi.w, lo.w);
+            const uint32_t o = cg * 16384 + sw128_off(r, y >> 2);
+            // the first product's operands are all read: the A region is free
+            *reinterpret_cast<float4*>(sm + OFF_YH + o) = hi;
+            *reinterpret_cast<float4*>(sm + OFF_YL + o) = lo;
+        }
+        sRed[cg * 64 + r] = yv;
+    }
+    // dO (rows 64-127 of the A operand) and U (the B operand), rows < L
+#pragma unroll
+    for (int it = 0; it < 2048 / NT; ++it) {
+        const int idx = tid + NT * it;  // (r, j4)
+        const int r = idx >> 5, j4 = idx & 31;
+        float4 dd = make_float4(0.f, 0.f, 0.f, 0.f), uu = dd;
+        if (r < L) {
+            dd = load4_f32<TIn>(Dg + base + r * rowH + 4 * j4);
+            uu = __ldg(reinterpret_cast<const float4*>(a.U + base + r * rowH + 4 * j4));
+        }
+        float4 hi, lo;
+        const uint32_t oa = (j4 >> 3) * 16384 + sw128_off(64 + r, j4 & 7);
+        split_tf32(dd.x, hi.x, lo.x);
+        split_tf32(dd.y, hi.y, lo.y);
+        split_tf32(dd.z, hi.z, lo.z);
+        split_tf32(dd.w, hi.w, lo.w);
+        *reinterpret_cast<float4*>(sm + OFF_YH + oa) = hi;
+        *reinterpret_cast<float4*>(sm + OFF_YL + oa) = lo;
+        const uint32_t ob = (j4 >> 3) * 8192 + sw128_off(r, j4 & 7);
+        split_tf32(uu.x, hi.x, lo.x);
+        split_tf32(uu.y, hi.y, lo.y);
+        split_tf32(uu.z, hi.z, lo.z);
+        split_tf32(uu.w, hi.w, lo.w);
+        *reinterpret_cast<float4*>(sm + OFF_UH + ob) = hi;
+        *reinterpret_cast<float4*>(sm + OFF_UL + ob) = lo;
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {  // [Y ; dO] U^T: M = 128, N = 64, K = 128
+        constexpr uint32_t id = idesc_tf32(128, 64, false, false);
+        const uint32_t As[3] = {OFF_YH, OFF_YH, OFF_YL}, Bs[3] = {OFF_UH, OFF_UL, OFF_UH};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks) {
+                const int kb = ks >> 2, kk = ks & 3;
+                mma_tf32_tc(tbase + TM_2, sdesc_sw128(sbase + As[pass] + kb * 16384 + kk * 32, 16, 1024),
+                            sdesc_sw128(sbase + Bs[pass] + kb * 8192 + kk * 32, 16, 1024), id,
+                            (pass | ks) > 0);
+            }
+        mma_commit(bar_mma);
+    }
+    ok = mbar_wait(bar_mma, 1, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            mbar_wait(bar_mma, 1, kWaitNs);
+            atomicOr(a.status_out, STATUS_TIMEOUT);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tbase, 256);
+        return;
+    }
+    tc_fence_after();
+    // lanes 0-63: Y U^T row r -> dA; lanes 64-127: dO U^T row r -> dP; 32
+    // columns per warp (cg 0, 1)
+    if (cg < 2) {
+        const int m = 32 * quarter + lane, r = m & 63, i0 = 32 * cg;
+        uint32_t v[32];
+        tmem_ld32(tbase + TM_2 + (static_cast<uint32_t>(32 * quarter) << 16) + i0, v);
+        tmem_wait_ld();
+        if (m < 64) {
+            float part = 0.f;
+            if (r < L) {
+                const float b = bs[r];
+                const float* arow = a.Ar + cc + r * 64 + i0;
+#pragma unroll
+                for (int y = 0; y < 32; y += 4) {
+                    const float4 ar = __ldg(reinterpret_cast<const float4*>(arow + y));
+                    float da[4];
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) da[z] = i0 + y + z < r ? -__uint_as_float(v[y + z]) : 0.f;
+                    part += da[0] * ar.x + da[1] * ar.y + da[2] * ar.z + da[3] * ar.w;
+                    *reinterpret_cast<float4*>(a.dAr + cc + r * 64 + i0 + y) =
+                        make_float4(b * da[0], b * da[1], b * da[2], b * da[3]);
+                }
+            }
+            sRed[256 + cg * 64 + r] = part;
+        } else if (r < L) {
+#pragma unroll
+            for (int y = 0; y < 32; y += 4) {
+                float p4[4];
+#pragma unroll
+                for (int z = 0; z < 4; ++z) p4[z] = i0 + y + z <= r ? __uint_as_float(v[y + z]) : 0.f;
+                *reinterpret_cast<float4*>(a.dP + cc + r * 64 + i0 + y) =
+                    make_float4(p4[0], p4[1], p4[2], p4[3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
+    if (tid < 64 && tid < L)
+        a.dbB[(size_t)(t0 + tid) * a.H + h] = sRed[tid] + sRed[64 + tid] + sRed[128 + tid] +
+                                              sRed[192 + tid] + sRed[256 + tid] + sRed[320 + tid];
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void* ptr = nullptr;
@@ -1488,5 +1976,49 @@ template cudaError_t launch_bwd_apkb_tc<__nv_bfloat16>(const __nv_bfloat16*,
                                                        const float*, const int4*, int, int, int,
                                                        uint32_t*, int*, float*, float*, float*,
                                                        float*, float*, cudaStream_t);
+
+}  // namespace kda
+
+namespace kda {
+
+template <typename TIn>
+cudaError_t launch_bwd_subst_tc(const TIn* v, const float* beta, const float* Ar,
+                                const int4* info, int total, int maxc, int H, uint32_t* status,
+                                float* W, float* Ut, float* Tm, cudaStream_t st) {
+    if (maxc == 0 || total == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(subst_tc_kernel<TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb::SMEM);
+    if (e != cudaSuccess) return e;
+    const SubstArgs a{v, beta, Ar, info, H, status, status, W, Ut, Tm};
+    subst_tc_kernel<TIn><<<dim3(maxc, H), sb::NT, sb::SMEM, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t launch_bwd_solve_tc(const TIn* v, const TIn* dout, const float* Ar,
+                                const float* beta, const float* U, const float* dU,
+                                const float* Tm, const int4* info, int total, int maxc, int H,
+                                uint32_t* status, float* Y, float* dv, float* dAr, float* dP,
+                                float* dbB, cudaStream_t st) {
+    if (maxc == 0 || total == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(solve_tc_kernel<TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sv::SMEM);
+    if (e != cudaSuccess) return e;
+    const SolveArgs a{v, dout, Ar, beta, U, dU, Tm, info, H, status, status, Y, dv, dAr, dP, dbB};
+    solve_tc_kernel<TIn><<<dim3(maxc, H), sv::NT, sv::SMEM, st>>>(a);
+    return cudaGetLastError();
+}
+
+#define KDA_BWD_ST_INST(TIn)                                                                  \
+    template cudaError_t launch_bwd_subst_tc<TIn>(const TIn*, const float*, const float*,      \
+                                                  const int4*, int, int, int, uint32_t*,       \
+                                                  float*, float*, float*, cudaStream_t);       \
+    template cudaError_t launch_bwd_solve_tc<TIn>(                                             \
+        const TIn*, const TIn*, const float*, const float*, const float*, const float*,        \
+        const float*, const int4*, int, int, int, uint32_t*, float*, float*, float*, float*,   \
+        float*, cudaStream_t);
+KDA_BWD_ST_INST(float)
+KDA_BWD_ST_INST(__nv_bfloat16)
+#undef KDA_BWD_ST_INST
 
 }  // namespace kda

@@ -246,6 +246,20 @@ cudaError_t launch_bwd_apkb_tc(const TIn* q, const TIn* k, const float* g, const
                                const int4* info, int total, int maxc, int H, uint32_t* status,
                                int* slow, float* G, float* Ar, float* P, float* Kb, float* Rk,
                                cudaStream_t st);
+// The two triangular solves through T = (I + A)^-1 (fp32, per chunk):
+// [W | Ut] = T [b Kt | b V] (W holds b Kt on entry), then Y = T^T dU, dv,
+// dA, dP and the partial dbeta, with the products in three tf32 passes;
+// kda_bwd_tc.cu.
+template <typename TIn>
+cudaError_t launch_bwd_subst_tc(const TIn* v, const float* beta, const float* Ar,
+                                const int4* info, int total, int maxc, int H, uint32_t* status,
+                                float* W, float* Ut, float* Tm, cudaStream_t st);
+template <typename TIn>
+cudaError_t launch_bwd_solve_tc(const TIn* v, const TIn* dout, const float* Ar,
+                                const float* beta, const float* U, const float* dU,
+                                const float* Tm, const int4* info, int total, int maxc, int H,
+                                uint32_t* status, float* Y, float* dv, float* dAr, float* dP,
+                                float* dbB, cudaStream_t st);
 // The pair sums (dq, dk, dg) as tensor-core products under a per-channel
 // exponent reference; a chunk whose gate range exceeds it gets slow[] = 1 and
 // is left to the exact CUDA-core kernel; kda_bwd_tc.cu.
