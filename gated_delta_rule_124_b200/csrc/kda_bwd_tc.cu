@@ -95,6 +95,14 @@ struct ChainArgs {
     float* S_end;          // forward: NULL; backward: dS_0 (or NULL)
 };
 
+// x as the sum of two tf32 values: hi = x rounded, lo = the remainder rounded
+// (operands of three-pass products: hi hi + hi lo + lo hi is within a few
+// fp32 ulps of the exact product).
+__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
+    hi = round_tf32(x);
+    lo = round_tf32(x - hi);
+}
+
 // One 32-value row of an MN-major tf32 operand block, rounded to tf32.
 __device__ __forceinline__ void store_row32(uint8_t* blk, int row, const float (&x)[32]) {
 #pragma unroll
@@ -777,15 +785,26 @@ __global__ void __launch_bounds__(NTB, 1)
 // q_i') e^{G_i' - G_r} (the masks are the zeros of bdA and dP), then the same
 // epilogue as the exact kernel: dq, dk, dG and the reverse cumulative sum dg.
 // X = [bdA ; dP] [128 rows][64 columns] is the K-major A operand of the first
-// product and the MN-major A operand of the second, so it is staged twice (the
-// 16-byte- and the 32-byte-granule swizzle).  A chunk outside the range sets
+// product and the MN-major A operand of the second (the 16-byte- and the
+// 32-byte-granule swizzle).  Both products are taken in three tf32 passes
+// (each operand split into a rounded high part and the rounded remainder:
+// hi hi + hi lo + lo hi): in one pass the pair sums carried most of the
+// gradients' error (dg is their reverse cumulative sum).  The two products
+// are staged one after the other in the same shared memory (the values of
+// the second kept in registers meanwhile).  A chunk outside the range sets
 // slow = 1 and is left to the exact kernel.
 namespace pr {
-constexpr uint32_t OFF_X1 = 0;        // X, 2 blocks [128][32] (16-byte granules)
-constexpr uint32_t OFF_X2 = 32768;    // X, 2 blocks [128][32] (32-byte granules)
-constexpr uint32_t OFF_B1 = 65536;    // K * E^-1 [64 i][128 c]: 4 blocks [64][32]
-constexpr uint32_t OFF_B2 = 98304;    // [K * E ; Q * E] [128][128 c]: 4 blocks [128][32]
-constexpr uint32_t OFF_GM = 163840;   // Gm [128]
+// first product
+constexpr uint32_t OFF_X1H = 0;       // X high, 2 blocks [128][32] (16-byte granules)
+constexpr uint32_t OFF_X1L = 32768;   // X low
+constexpr uint32_t OFF_B1H = 65536;   // K * E^-1 high [64 i][128 c]: 4 blocks [64][32]
+constexpr uint32_t OFF_B1L = 98304;   // low
+// second product (over the first's operands)
+constexpr uint32_t OFF_X2H = 0;       // X high, 2 blocks [128][32] (32-byte granules)
+constexpr uint32_t OFF_X2L = 32768;   // X low
+constexpr uint32_t OFF_B2H = 65536;   // [K * E ; Q * E] high: 4 blocks [128][32]
+constexpr uint32_t OFF_B2L = 131072;  // low
+constexpr uint32_t OFF_GM = 196608;   // Gm [128]
 constexpr uint32_t OFF_RED = OFF_GM + 512;   // max, min [4][128] each; later the epilogue's exchange
 constexpr uint32_t OFF_BAR = OFF_RED + 4096;
 constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
@@ -900,77 +919,147 @@ __global__ void __launch_bounds__(pr::NTP, 1) pair_tc_kernel(const PairArgs a) {
         mbar_init(bar_mma, 1);
         fence_mbar_init();
     }
-    // 2. operands.  X rows m (< 64: bdA row m; >= 64: dP row m - 64), four
-    // columns per float4: both swizzles
+    // 2. the first product's operands.  X rows m (< 64: bdA row m; >= 64: dP
+    // row m - 64), four columns per float4; K * E^-1 rows r, channels 4 c4 ..;
+    // X and K * E, Q * E stay in registers for the second product
+    constexpr int NX = 2048 / NTP;
+    float4 xv[NX], kev[NX], qev[NX];
     {
         const size_t cc = ((size_t)cidx * a.H + h) * 64 * 64;
 #pragma unroll
-        for (int it = 0; it < 2048 / NTP; ++it) {
+        for (int it = 0; it < NX; ++it) {
             const int idx = tid + NTP * it;  // 0 .. 2047
             const int m = idx >> 4, c4 = idx & 15;
             const int r = m & 63;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            xv[it] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < L)
-                v = __ldg(reinterpret_cast<const float4*>((m < 64 ? a.dAr : a.dP) + cc + r * 64 + 4 * c4));
-            v = round4_tf32(v);
-            const int blk = c4 >> 3, q16 = c4 & 7;
-            *reinterpret_cast<float4*>(sm + OFF_X1 + blk * 16384 + sw128_off(m, q16)) = v;
-            *reinterpret_cast<float4*>(sm + OFF_X2 + blk * 16384 + sw128_32b_off(m, q16)) = v;
+                xv[it] = __ldg(reinterpret_cast<const float4*>((m < 64 ? a.dAr : a.dP) + cc + r * 64 + 4 * c4));
+            float4 hi, lo;
+            split_tf32(xv[it].x, hi.x, lo.x);
+            split_tf32(xv[it].y, hi.y, lo.y);
+            split_tf32(xv[it].z, hi.z, lo.z);
+            split_tf32(xv[it].w, hi.w, lo.w);
+            const uint32_t o = (c4 >> 3) * 16384 + sw128_off(m, c4 & 7);
+            *reinterpret_cast<float4*>(sm + OFF_X1H + o) = hi;
+            *reinterpret_cast<float4*>(sm + OFF_X1L + o) = lo;
         }
     }
     __syncthreads();  // Gm visible
-    // K * E^-1, K * E, Q * E: row r, channels 4 c4 .. 4 c4 + 3
 #pragma unroll
-    for (int it = 0; it < 2048 / NTP; ++it) {
+    for (int it = 0; it < NX; ++it) {
         const int idx = tid + NTP * it;  // 0 .. 2047
         const int r = idx >> 5, c4 = idx & 31;
-        float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv, ke = kv, ki = kv;
+        float4 ki = make_float4(0.f, 0.f, 0.f, 0.f);
+        kev[it] = qev[it] = ki;
         if (r < L) {
             const size_t gi = base + r * rowH + 4 * c4;
-            kv = load4_f32<TIn>(Kg + gi);
-            qv = load4_f32<TIn>(Qg + gi);
+            const float4 kv = load4_f32<TIn>(Kg + gi);
+            const float4 qv = load4_f32<TIn>(Qg + gi);
             const float4 gv = __ldg(reinterpret_cast<const float4*>(a.G + gi));
             const float4 gm = *reinterpret_cast<const float4*>(sGm + 4 * c4);
             const float x0 = gv.x - gm.x, x1 = gv.y - gm.y, x2 = gv.z - gm.z, x3 = gv.w - gm.w;
             const float e0 = __expf(x0), e1 = __expf(x1), e2 = __expf(x2), e3 = __expf(x3);
-            ke = make_float4(kv.x * e0, kv.y * e1, kv.z * e2, kv.w * e3);
-            qv = make_float4(qv.x * e0, qv.y * e1, qv.z * e2, qv.w * e3);
+            kev[it] = make_float4(kv.x * e0, kv.y * e1, kv.z * e2, kv.w * e3);
+            qev[it] = make_float4(qv.x * e0, qv.y * e1, qv.z * e2, qv.w * e3);
             ki = make_float4(kv.x * __expf(-x0), kv.y * __expf(-x1), kv.z * __expf(-x2),
                              kv.w * __expf(-x3));
         }
-        const int blk = c4 >> 3, q16 = c4 & 7;
-        *reinterpret_cast<float4*>(sm + OFF_B1 + blk * 8192 + sw128_32b_off(r, q16)) =
-            round4_tf32(ki);
-        *reinterpret_cast<float4*>(sm + OFF_B2 + blk * 16384 + sw128_32b_off(r, q16)) =
-            round4_tf32(ke);
-        *reinterpret_cast<float4*>(sm + OFF_B2 + blk * 16384 + sw128_32b_off(64 + r, q16)) =
-            round4_tf32(qv);
+        float4 hi, lo;
+        split_tf32(ki.x, hi.x, lo.x);
+        split_tf32(ki.y, hi.y, lo.y);
+        split_tf32(ki.z, hi.z, lo.z);
+        split_tf32(ki.w, hi.w, lo.w);
+        const uint32_t o = (c4 >> 3) * 8192 + sw128_32b_off(r, c4 & 7);
+        *reinterpret_cast<float4*>(sm + OFF_B1H + o) = hi;
+        *reinterpret_cast<float4*>(sm + OFF_B1L + o) = lo;
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = s_tmem;
-    // 3. the two products, one commit
+    // 3. the first product: [rowA ; dQp] before scaling (M = 128, N = 128, K = 64)
     if (tid == 0) {
         constexpr uint32_t id1 = idesc_tf32(128, 128, false, true);
-        constexpr uint32_t id2 = idesc_tf32(128, 128, true, true);
+        const uint32_t As[3] = {OFF_X1H, OFF_X1H, OFF_X1L}, Bs[3] = {OFF_B1H, OFF_B1L, OFF_B1H};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const int kb = ks >> 2, kk = ks & 3;
-            mma_tf32_tc(tbase + TM_1, sdesc_sw128(sbase + OFF_X1 + kb * 16384 + kk * 32, 16, 1024),
-                        sdesc_sw128_32b(sbase + OFF_B1 + ks * 1024, 8192, 512), id1, ks > 0);
-        }
+        for (int pass = 0; pass < 3; ++pass)
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks)
-            mma_tf32_tc(tbase + TM_2, sdesc_sw128_32b(sbase + OFF_X2 + ks * 1024, 16384, 512),
-                        sdesc_sw128_32b(sbase + OFF_B2 + ks * 1024, 16384, 512), id2, ks > 0);
+            for (int ks = 0; ks < 8; ++ks) {
+                const int kb = ks >> 2, kk = ks & 3;
+                mma_tf32_tc(tbase + TM_1, sdesc_sw128(sbase + As[pass] + kb * 16384 + kk * 32, 16, 1024),
+                            sdesc_sw128_32b(sbase + Bs[pass] + ks * 1024, 8192, 512), id1,
+                            (pass | ks) > 0);
+            }
         mma_commit(bar_mma);
     }
-    const bool ok = mbar_wait(bar_mma, 0, kWaitNs);
+    bool ok = mbar_wait(bar_mma, 0, kWaitNs);
     if (__syncthreads_or(!ok)) {
         if (tid == 0) {
             mbar_wait(bar_mma, 0, kWaitNs);  // bounded: the products still in flight
+            atomicOr(a.status_out, STATUS_TIMEOUT);
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tbase, 256);
+        return;
+    }
+    tc_fence_after();
+    // 4. the second product's operands over the first's (all read)
+#pragma unroll
+    for (int it = 0; it < NX; ++it) {
+        const int idx = tid + NTP * it;
+        {
+            const int m = idx >> 4, c4 = idx & 15;
+            float4 hi, lo;
+            split_tf32(xv[it].x, hi.x, lo.x);
+            split_tf32(xv[it].y, hi.y, lo.y);
+            split_tf32(xv[it].z, hi.z, lo.z);
+            split_tf32(xv[it].w, hi.w, lo.w);
+            const uint32_t o = (c4 >> 3) * 16384 + sw128_32b_off(m, c4 & 7);
+            *reinterpret_cast<float4*>(sm + OFF_X2H + o) = hi;
+            *reinterpret_cast<float4*>(sm + OFF_X2L + o) = lo;
+        }
+        {
+            const int r = idx >> 5, c4 = idx & 31;
+            const uint32_t o = (c4 >> 3) * 16384 + sw128_32b_off(r, c4 & 7);
+            const uint32_t oq = (c4 >> 3) * 16384 + sw128_32b_off(64 + r, c4 & 7);
+            float4 hi, lo;
+            split_tf32(kev[it].x, hi.x, lo.x);
+            split_tf32(kev[it].y, hi.y, lo.y);
+            split_tf32(kev[it].z, hi.z, lo.z);
+            split_tf32(kev[it].w, hi.w, lo.w);
+            *reinterpret_cast<float4*>(sm + OFF_B2H + o) = hi;
+            *reinterpret_cast<float4*>(sm + OFF_B2L + o) = lo;
+            split_tf32(qev[it].x, hi.x, lo.x);
+            split_tf32(qev[it].y, hi.y, lo.y);
+            split_tf32(qev[it].z, hi.z, lo.z);
+            split_tf32(qev[it].w, hi.w, lo.w);
+            *reinterpret_cast<float4*>(sm + OFF_B2H + oq) = hi;
+            *reinterpret_cast<float4*>(sm + OFF_B2L + oq) = lo;
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // 5. the second product: col before scaling (M = 64 padded to 128, N = 128, K = 128)
+    if (tid == 0) {
+        constexpr uint32_t id2 = idesc_tf32(128, 128, true, true);
+        const uint32_t As[3] = {OFF_X2H, OFF_X2H, OFF_X2L}, Bs[3] = {OFF_B2H, OFF_B2L, OFF_B2H};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+            for (int ks = 0; ks < 16; ++ks)
+                mma_tf32_tc(tbase + TM_2, sdesc_sw128_32b(sbase + As[pass] + ks * 1024, 16384, 512),
+                            sdesc_sw128_32b(sbase + Bs[pass] + ks * 1024, 16384, 512), id2,
+                            (pass | ks) > 0);
+        mma_commit(bar_mma);
+    }
+    ok = mbar_wait(bar_mma, 1, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            mbar_wait(bar_mma, 1, kWaitNs);
             atomicOr(a.status_out, STATUS_TIMEOUT);
         }
         tc_fence_before();
@@ -1343,12 +1432,6 @@ __device__ void tri_inverse(const float* Ar, const float* bs, float* Tm, float* 
     }
 }
 
-// x and its tf32 split
-__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
-    hi = round_tf32(x);
-    lo = round_tf32(x - hi);
-}
-
 // ------------------------------------------------------------ [W | Ut]
 // (I + A) [W | Ut] = [b Kt | b V] as [W | Ut] = T [b Kt | b V]: T in fp32 by
 // tri_inverse (also written out for the back substitution), the product in
@@ -1409,6 +1492,25 @@ __global__ void __launch_bounds__(sb::NT, 1) subst_tc_kernel(const SubstArgs a) 
     const size_t cc = ((size_t)cidx * a.H + h) * 64 * 64;
     for (int e = tid; e < 64 * 64; e += NT) Ar[(e >> 6) * LDT + (e & 63)] = __ldg(a.Ar + cc + e);
     if (tid < 64) bs[tid] = tid < L ? __ldg(a.beta + (size_t)(t0 + tid) * a.H + h) : 0.f;
+    // the right-hand sides' rows i < L, requested now so that their latency
+    // overlaps the inverse: b Kt (W on entry) and v (b applied later)
+    constexpr int NB = 4096 / NT;
+    float4 rhs[NB];
+    {
+        const size_t base = ((size_t)t0 * a.H + h) * DD;
+        const size_t rowH = (size_t)a.H * DD;
+        const TIn* Vg = static_cast<const TIn*>(a.v);
+#pragma unroll
+        for (int it = 0; it < NB; ++it) {
+            const int idx = tid + NT * it;
+            const int i = idx >> 6, n4 = idx & 63;
+            rhs[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < L)
+                rhs[it] = n4 < 32
+                              ? __ldg(reinterpret_cast<const float4*>(a.W + base + i * rowH + 4 * n4))
+                              : load4_f32<TIn>(Vg + base + i * rowH + 4 * (n4 - 32));
+        }
+    }
     __syncthreads();
     tri_inverse(Ar, bs, Tm, Msc, tid, NT);
     // T out (fp32) and T's tf32 split as the K-major A operand
@@ -1425,22 +1527,14 @@ __global__ void __launch_bounds__(sb::NT, 1) subst_tc_kernel(const SubstArgs a) 
     __syncthreads();  // T, Ar read: the low half of B may overwrite them
     // [b Kt | b V] rows i < L (zeros after), four columns per float4
     {
-        const size_t base = ((size_t)t0 * a.H + h) * DD;
-        const size_t rowH = (size_t)a.H * DD;
-        const TIn* Vg = static_cast<const TIn*>(a.v);
 #pragma unroll
-        for (int it = 0; it < 4096 / NT; ++it) {
+        for (int it = 0; it < NB; ++it) {
             const int idx = tid + NT * it;
             const int i = idx >> 6, n4 = idx & 63;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < L) {
-                if (n4 < 32) {
-                    x = __ldg(reinterpret_cast<const float4*>(a.W + base + i * rowH + 4 * n4));
-                } else {
-                    const float b = bs[i];
-                    const float4 vv = load4_f32<TIn>(Vg + base + i * rowH + 4 * (n4 - 32));
-                    x = make_float4(b * vv.x, b * vv.y, b * vv.z, b * vv.w);
-                }
+            float4 x = rhs[it];
+            if (n4 >= 32) {
+                const float b = bs[i];
+                x = make_float4(b * x.x, b * x.y, b * x.z, b * x.w);
             }
             float4 hi, lo;
             split_tf32(x.x, hi.x, lo.x);
@@ -1584,6 +1678,20 @@ __global__ void __launch_bounds__(sv::NT, 1) solve_tc_kernel(const SolveArgs a) 
     const size_t base = ((size_t)t0 * a.H + h) * DD;
     const size_t rowH = (size_t)a.H * DD;
     if (tid < 64) bs[tid] = tid < L ? __ldg(a.beta + (size_t)(t0 + tid) * a.H + h) : 0.f;
+    // dO and U of the second product, requested now (their latency overlaps
+    // the first product)
+    constexpr int NP2 = 2048 / NT;
+    float4 dpre[NP2], upre[NP2];
+#pragma unroll
+    for (int it = 0; it < NP2; ++it) {
+        const int idx = tid + NT * it;
+        const int r = idx >> 5, j4 = idx & 31;
+        dpre[it] = upre[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < L) {
+            dpre[it] = load4_f32<TIn>(Dg + base + r * rowH + 4 * j4);
+            upre[it] = __ldg(reinterpret_cast<const float4*>(a.U + base + r * rowH + 4 * j4));
+        }
+    }
     // T (rows i, columns r contiguous: the MN-major A of T^T) and dU (rows i)
 #pragma unroll
     for (int it = 0; it < 1024 / NT; ++it) {
@@ -1680,14 +1788,10 @@ __global__ void __launch_bounds__(sv::NT, 1) solve_tc_kernel(const SolveArgs a) 
     }
     // dO (rows 64-127 of the A operand) and U (the B operand), rows < L
 #pragma unroll
-    for (int it = 0; it < 2048 / NT; ++it) {
+    for (int it = 0; it < NP2; ++it) {
         const int idx = tid + NT * it;  // (r, j4)
         const int r = idx >> 5, j4 = idx & 31;
-        float4 dd = make_float4(0.f, 0.f, 0.f, 0.f), uu = dd;
-        if (r < L) {
-            dd = load4_f32<TIn>(Dg + base + r * rowH + 4 * j4);
-            uu = __ldg(reinterpret_cast<const float4*>(a.U + base + r * rowH + 4 * j4));
-        }
+        const float4 dd = dpre[it], uu = upre[it];
         float4 hi, lo;
         const uint32_t oa = (j4 >> 3) * 16384 + sw128_off(64 + r, j4 & 7);
         split_tf32(dd.x, hi.x, lo.x);

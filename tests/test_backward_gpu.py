@@ -44,6 +44,9 @@ CASES = {
                                                     chunk=64, dtype="bf16", varlen=True),
     "f32_d128_dv64_batched": lambda: wl.make_prefill(505, [200, 200], H=1, dk=128, dv=64,
                                                      chunk=64, dtype="f32"),
+    # fp32 inputs through the tensor-core kernels (dk = dv = 128)
+    "f32_d128_varlen": lambda: wl.make_prefill(507, [90, 0, 130], H=2, dk=128, dv=128,
+                                               chunk=64, dtype="f32", varlen=True),
 }
 
 
@@ -58,6 +61,20 @@ def _strong_decay():
 
 
 CASES["f32_d64_strong_decay"] = _strong_decay
+
+
+def _mixed_decay_d128():
+    """dk = dv = 128 with the second sequence's gates twenty times stronger:
+    its chunks exceed the exponent reference's range and are recomputed by
+    the exact kernels, the first sequence's chunks are not — both kinds in
+    one call."""
+    case = wl.make_prefill(511, [130, 70], H=2, dk=128, dv=128, chunk=64, dtype="bf16",
+                           varlen=True)
+    case.g[130:] = case.g[130:] * 20.0
+    return case
+
+
+CASES["bf16_d128_mixed_decay"] = _mixed_decay_d128
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
