@@ -700,16 +700,19 @@ def backward_flops(head_tokens, dk, dv, C=64):
     of C tokens and one head, the multiply-adds of each step (the forward's
     A, P, W, Ut and chain recomputed, then E, F, the reverse chain, the back
     substitution, the products with U, S and dS', and the pair sums), two
-    flops each.  Returns (on the tensor cores, on the CUDA cores) for dk = dv
-    = 128, where A/P, the chains, E, F, the dense products and the pair sums
-    run as tcgen05 products; other shapes run everything on the CUDA cores."""
+    flops each.  Returns (on the tensor cores, on the CUDA cores): for dk = dv
+    = 128 every contraction runs as a tcgen05 product (the substitutions as
+    products with T = (I + A)^-1); other shapes run everything on the CUDA
+    cores."""
     tri, stri = C * (C + 1) // 2, C * (C - 1) // 2
     tensor = (2 * tri * dk                                         # A, P
+              + stri * (dk + dv)                                   # [W | Ut]
               + 2 * C * dk * dv + 2 * C * dk * dv                  # the two chains
-              + tri * dv + 2 * C * dk * dv + 3 * C * dk * dv       # E; F; dense
+              + tri * dv + 2 * C * dk * dv                         # E; F
+              + stri * dv + 2 * C * C * dv                         # Y; Y U^T, dO U^T
+              + 3 * C * dk * dv                                    # dense
               + 4 * tri * dk)                                      # pair sums
-    alu = (stri * (dk + dv)                                        # [W | Ut]
-           + stri * dv + 2 * C * C * dv)                           # Y; Y U^T, dO U^T
+    alu = 0
     if not (dk == 128 and dv == 128):
         tensor, alu = 0, tensor + alu
     return 2 * tensor * head_tokens / C, 2 * alu * head_tokens / C
@@ -720,7 +723,7 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
     state), timed with CUDA events on the launching stream, L2 flushed before
     each call.  Roofline: the kernels run one after another, so the bound is
     the tensor-core flops at the tf32 peak (the measured bf16 peak x the
-    nominal tf32 / bf16 ratio 1.1 / 2.25) plus the CUDA-core flops at 148
+    nominal tf32 / bf16 ratio 1.1 / 2.25) plus any CUDA-core flops at 148
     SMs x 128 fp32 lanes x 2 flops x the SM clock; `peak` is the total flops
     over that time."""
     total, H, dk, dv = P.total, P.H, P.dk, P.dv
@@ -758,13 +761,15 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
     t_bound = fl_tc / tf32_peak / 1e12 + fl_alu / alu_peak / 1e12
     peak = fl / t_bound / 1e12
     res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 9,
-           "roofline": {"bound": "alu", "achieved": fl / t / 1e12, "peak": peak,
+           "roofline": {"bound": "tensor" if fl_alu == 0 else "alu",
+                        "achieved": fl / t / 1e12, "peak": peak,
                         "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak,
-                        "peak_kind": (f"mixed: {fl_tc / 1e9:.1f} GFLOP at the tf32 tensor peak "
+                        "peak_kind": (f"{fl_tc / 1e9:.1f} GFLOP at the tf32 tensor peak "
                                       f"{tf32_peak:.0f} TFLOP/s ({kind} bf16 x 1.1/2.25) + "
                                       f"{fl_alu / 1e9:.1f} GFLOP at the fp32 CUDA-core peak "
                                       f"{alu_peak:.1f} TFLOP/s (148 SMs x 128 lanes x 2 x "
-                                      f"{mhz:.0f} MHz)"),
+                                      f"{mhz:.0f} MHz); the algorithm's count, not the three "
+                                      f"tf32 passes of the products that use them"),
                         "bound_ms": t_bound * 1e3,
                         "algorithmic_flops_per_call": fl},
            "workspace_bytes": int(ws.numel())}
