@@ -57,10 +57,9 @@ MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch, captured on
     # B=8 x T=2048, H=32 (8192 (chunk, head) items, inputs larger than L2)
     # and scaled by the items of the varlen workload (62560): per item
-    # 127.7 KB (intra) and 100.9 KB (chain); the source changed since only in
-    # the co-scheduled kernel's head-gate template and its launcher
-    ("split_intra", _CFG3): (_SPLIT, "581c0c3ce0132b875334ed49893da3c6f70a4281", 7988038115),
-    ("split_chain", _CFG3): (_SPLIT, "581c0c3ce0132b875334ed49893da3c6f70a4281", 6312896365),
+    # 127.7 KB (intra) and 100.9 KB (chain)
+    ("split_intra", _CFG3): (_SPLIT, "9df21f075afbbf808e885b6c9ed38680a6bbcf15", 7987911040),
+    ("split_chain", _CFG3): (_SPLIT, "9df21f075afbbf808e885b6c9ed38680a6bbcf15", 6312438895),
     ("decode", _DEC): (_DECODE, "e97a0fa46338f7541982499a4e97d31ac9101889", 1027143936),
 }
 
@@ -760,7 +759,7 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
     tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
     t_bound = fl_tc / tf32_peak / 1e12 + fl_alu / alu_peak / 1e12
     peak = fl / t_bound / 1e12
-    res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 9,
+    res = {"ms_per_call": t * 1e3, "tokens_per_s": total / t, "kernels_per_call": 11,
            "roofline": {"bound": "tensor" if fl_alu == 0 else "alu",
                         "achieved": fl / t / 1e12, "peak": peak,
                         "unit": "TFLOP/s", "frac": fl / t / 1e12 / peak,
