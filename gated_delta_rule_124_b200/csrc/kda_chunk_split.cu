@@ -106,7 +106,8 @@ constexpr uint32_t OFF_KQ = 0;
 constexpr uint32_t OFF_G = 32768;      // g (TMA) -> G -> A fp32 | T fp32
 constexpr uint32_t OFF_RAP = 65536;    // K * E^-1 (exact path: K * exp(G_last - G))
 // T diag(b) rows 0-63, then the garbage rows of its 128-row operand (also the
-// inverse's scratch); before that, on the exact path: A in fp32 (16 KB).
+// inverse's scratch); before that: the scan's partial results (E1) and, on
+// the exact path, A in fp32 (16 KB).
 constexpr uint32_t OFF_TB = 81920;
 constexpr uint32_t OFF_MID = 90112;
 constexpr uint32_t OFF_BETA = 98304;
@@ -377,8 +378,9 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
             failed = true;
             break;
         }
-        // ------------- E1: in-chunk cumulative log-gate G, per channel, its
-        // per-channel max / min over the chunk's rows, and G_last.
+        // ------------- E1: in-chunk cumulative log-gate, per channel.  Thread
+        // (row group grp = 8 rows, channels 4 c4 ..): scan of its 8 rows, then
+        // the totals of the groups above it added; per-channel max / min.
         bool slow_local = false;
         if (kScalar) {
             // one warp: lane l holds rows 2l, 2l + 1; inclusive scan by shuffles
@@ -419,80 +421,61 @@ __device__ __forceinline__ void run(const CUtensorMap* tmq, const CUtensorMap* t
                 sGL[tid] = sGsc[2];
             }
         } else {
-            // warp w scans channels 16 w .. 16 w + 15 without CTA barriers:
-            // lane 4 rb + q holds rows 8 rb .. 8 rb + 7 of channels
-            // c0 .. c0 + 3 (c0 = 16 w + 4 q), scans them in registers, adds
-            // the totals of the row blocks above it (inclusive scan over the
-            // lanes 4 apart), and reduces the per-channel max / min of the
-            // chunk's rows the same way; G_last comes from the lane of row
-            // L - 1.
-            static_assert(NTI == 256, "8 warps of 16 channels");
             float* g = reinterpret_cast<float*>(sm + OFF_G);
-            const int rb = lane >> 2, c0 = 16 * warp + 4 * (lane & 3), r0 = 8 * rb;
+            float4* tot = reinterpret_cast<float4*>(sm + OFF_TB);           // [8][32]
+            float4* gmx = reinterpret_cast<float4*>(sm + OFF_TB + 4096);    // [8][32]
+            float4* gmn = reinterpret_cast<float4*>(sm + OFF_TB + 8192);    // [8][32]
+            const int c4 = tid & 31, grp = tid >> 5, r0 = 8 * grp;
             float4 x[8];
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float4 v = *reinterpret_cast<const float4*>(g + (r0 + i) * D + c0);
+                float4 v = *reinterpret_cast<const float4*>(g + (r0 + i) * D + 4 * c4);
                 if (r0 + i >= L) v = make_float4(0.f, 0.f, 0.f, 0.f);
                 acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
                 x[i] = acc;
             }
-            float4 pre = acc;
-#pragma unroll
-            for (int o = 4; o < 32; o <<= 1) {
-                const float yx = __shfl_up_sync(0xffffffffu, pre.x, o);
-                const float yy = __shfl_up_sync(0xffffffffu, pre.y, o);
-                const float yz = __shfl_up_sync(0xffffffffu, pre.z, o);
-                const float yw = __shfl_up_sync(0xffffffffu, pre.w, o);
-                if (lane >= o) { pre.x += yx; pre.y += yy; pre.z += yz; pre.w += yw; }
+            tot[grp * 32 + c4] = acc;
+            group_sync(bar, NTI);
+            float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < grp; ++j) {
+                const float4 t = tot[j * 32 + c4];
+                off.x += t.x; off.y += t.y; off.z += t.z; off.w += t.w;
             }
-            const float4 off = make_float4(pre.x - acc.x, pre.y - acc.y, pre.z - acc.z,
-                                           pre.w - acc.w);
             float4 mx = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
             float4 mn = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
-            const int il = (L - 1) & 7;
-            float4 gsel = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 float4 v = x[i];
                 v.x += off.x; v.y += off.y; v.z += off.z; v.w += off.w;
-                *reinterpret_cast<float4*>(g + (r0 + i) * D + c0) = v;
+                *reinterpret_cast<float4*>(g + (r0 + i) * D + 4 * c4) = v;
                 if (r0 + i < L) {
                     mx.x = fmaxf(mx.x, v.x); mx.y = fmaxf(mx.y, v.y);
                     mx.z = fmaxf(mx.z, v.z); mx.w = fmaxf(mx.w, v.w);
                     mn.x = fminf(mn.x, v.x); mn.y = fminf(mn.y, v.y);
                     mn.z = fminf(mn.z, v.z); mn.w = fminf(mn.w, v.w);
                 }
-                if (i == il) gsel = v;
             }
+            gmx[grp * 32 + c4] = mx;
+            gmn[grp * 32 + c4] = mn;
+            group_sync(bar, NTI);
+            if (tid < D) {
+                const int c = tid;
+                const float* fx = reinterpret_cast<const float*>(gmx);
+                const float* fn = reinterpret_cast<const float*>(gmn);
+                float gmax = -INFINITY, gmin = INFINITY;
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) {
-                mx.x = fmaxf(mx.x, __shfl_xor_sync(0xffffffffu, mx.x, o));
-                mx.y = fmaxf(mx.y, __shfl_xor_sync(0xffffffffu, mx.y, o));
-                mx.z = fmaxf(mx.z, __shfl_xor_sync(0xffffffffu, mx.z, o));
-                mx.w = fmaxf(mx.w, __shfl_xor_sync(0xffffffffu, mx.w, o));
-                mn.x = fminf(mn.x, __shfl_xor_sync(0xffffffffu, mn.x, o));
-                mn.y = fminf(mn.y, __shfl_xor_sync(0xffffffffu, mn.y, o));
-                mn.z = fminf(mn.z, __shfl_xor_sync(0xffffffffu, mn.z, o));
-                mn.w = fminf(mn.w, __shfl_xor_sync(0xffffffffu, mn.w, o));
+                for (int j = 0; j < 8; ++j) {
+                    gmax = fmaxf(gmax, fx[j * D + c]);
+                    gmin = fminf(gmin, fn[j * D + c]);
+                }
+                const float Gm = gmax - kRef;
+                const float gl = g[(L - 1) * D + c];
+                sGm[c] = Gm;
+                seGm[c] = expf(Gm);
+                sGL[c] = gl;
+                slow_local = !(gmax - gmin <= 2.f * kRef) || !(gmax <= 60.f);
             }
-            const int src = 4 * ((L - 1) >> 3) + (lane & 3);
-            const float4 gl = make_float4(__shfl_sync(0xffffffffu, gsel.x, src),
-                                          __shfl_sync(0xffffffffu, gsel.y, src),
-                                          __shfl_sync(0xffffffffu, gsel.z, src),
-                                          __shfl_sync(0xffffffffu, gsel.w, src));
-            if (rb == 0) {
-                const float4 gm = make_float4(mx.x - kRef, mx.y - kRef, mx.z - kRef, mx.w - kRef);
-                *reinterpret_cast<float4*>(sGm + c0) = gm;
-                *reinterpret_cast<float4*>(seGm + c0) =
-                    make_float4(expf(gm.x), expf(gm.y), expf(gm.z), expf(gm.w));
-                *reinterpret_cast<float4*>(sGL + c0) = gl;
-            }
-            slow_local = !(mx.x - mn.x <= 2.f * kRef) || !(mx.x <= 60.f) ||
-                         !(mx.y - mn.y <= 2.f * kRef) || !(mx.y <= 60.f) ||
-                         !(mx.z - mn.z <= 2.f * kRef) || !(mx.z <= 60.f) ||
-                         !(mx.w - mn.w <= 2.f * kRef) || !(mx.w <= 60.f);
         }
         ok = mbar_wait(bar_k, n & 1, kWaitNs) && mbar_wait(bar_q, n & 1, kWaitNs);
         if (kConv) cp_async_wait_all();
