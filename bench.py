@@ -58,8 +58,8 @@ MEASURED_TRAFFIC = {
     # B=8 x T=2048, H=32 (8192 (chunk, head) items, inputs larger than L2)
     # and scaled by the items of the varlen workload (62560): per item
     # 127.7 KB (intra) and 100.9 KB (chain)
-    ("split_intra", _CFG3): (_SPLIT, "9df21f075afbbf808e885b6c9ed38680a6bbcf15", 7987911040),
-    ("split_chain", _CFG3): (_SPLIT, "9df21f075afbbf808e885b6c9ed38680a6bbcf15", 6312438895),
+    ("split_intra", _CFG3): (_SPLIT, "1dd5be2a9803eb0eceec8f921e9102c6fdb8dedc", 7986931585),
+    ("split_chain", _CFG3): (_SPLIT, "1dd5be2a9803eb0eceec8f921e9102c6fdb8dedc", 6309916945),
     ("decode", _DEC): (_DECODE, "e97a0fa46338f7541982499a4e97d31ac9101889", 1027143936),
 }
 
