@@ -380,7 +380,7 @@ def run_ours(args, rank, world, local_rank):
     layer = layer_times(kda, torch, P, dcase, dev, stream, reps=reps)
 
     # ---- end to end through host buffers (pinned), copies inside the region
-    e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=3)
+    e2e = run_e2e(kda, torch, pc, dcase, dev, stream, steps=6)
 
     # ---- the backward (gradients of o and the final state) on the B=2 x
     # T=2048 workload, last: a failure there is reported in its entry and
@@ -776,45 +776,80 @@ def backward_times(kda, torch, P, pc, dev, stream, reps=10, sm_max_mhz=None):
 
 
 def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
-    """Prefill through the public call with pinned host buffers: H2D of the
-    inputs, kda_chunk_fwd, D2H of o and the final state -- all inside the
-    events; the same for one decode step (state resident on the device)."""
+    """Prefill through the public call with pinned host buffers: every step
+    copies its inputs host -> device, runs kda_chunk_fwd and copies o and the
+    final state back, all inside the events.  Consecutive prefill batches are
+    independent, so the steps are pipelined as a server would run them: two
+    device buffer sets, the uploads on one stream, the calls on the launching
+    stream, the downloads on a third, so that one step's download and call
+    overlap the next step's upload (separate copy engines).  One decode step
+    (state resident on the device) the same way but serially, since a decode
+    step's inputs follow from the previous step's output."""
     pin = lambda t: None if t is None else t.pin_memory()
     hq, hk, hv, hg, hb, h0 = map(pin, (pc.q, pc.k, pc.v, pc.g, pc.beta, pc.initial_state))
-    dq, dk_, dv_, dg, db, d0 = (torch.empty_like(x, device=dev) for x in (hq, hk, hv, hg, hb, h0))
-    H, dk, dv, C, N, total = pc.H, pc.dk, pc.dv, pc.chunk, pc.N, pc.total
-    o = torch.empty_like(dv_)
-    hN = torch.empty(N, H, dk, dv, device=dev)
-    ho = torch.empty_like(hv).pin_memory()
-    hhN = torch.empty(N, H, dk, dv).pin_memory()
-    ws = kda.alloc_workspace(total, N, H, dk, dv, C, "bf16", dev)
-
     hcu = None if pc.cu_seqlens is None else pc.cu_seqlens.pin_memory()
-    dcu = None if hcu is None else torch.empty_like(hcu, device=dev)
+    host_in = (hq, hk, hv, hg, hb, h0, hcu)
+    H, dk, dv, C, N, total = pc.H, pc.dk, pc.dv, pc.chunk, pc.N, pc.total
     Bc, Tc = (1, total) if hcu is not None else (pc.B, pc.T)
 
-    def one():
-        for d, h in ((dq, hq), (dk_, hk), (dv_, hv), (dg, hg), (db, hb), (d0, h0), (dcu, hcu)):
-            if d is not None:
-                d.copy_(h, non_blocking=True)
-        kda.kda_chunk_fwd(dq, dk_, dv_, dg, db, d0, dcu, Bc, Tc, N, H, dk, dv, C, "bf16",
-                          o, hN, ws)
-        ho.copy_(o, non_blocking=True)
-        hhN.copy_(hN, non_blocking=True)
+    def buffers():
+        d_in = tuple(None if h is None else torch.empty_like(h, device=dev) for h in host_in)
+        return {"in": d_in, "o": torch.empty_like(d_in[2]),
+                "hN": torch.empty(N, H, dk, dv, device=dev),
+                "ho": torch.empty_like(hv).pin_memory(),
+                "hhN": torch.empty(N, H, dk, dv).pin_memory()}
 
-    for _ in range(2):
-        one()
+    sets = [buffers(), buffers()]
+    ws = kda.alloc_workspace(total, N, H, dk, dv, C, "bf16", dev)
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    free_in = [ev(), ev()]    # the call that read set b has run
+    up_done = [ev(), ev()]    # set b's inputs are on the device
+    called = [ev(), ev()]     # set b's outputs are written
+    down_done = [ev(), ev()]  # set b's outputs are on the host
+    for b in range(2):  # nothing pending on either set at the start
+        free_in[b].record(stream)
+        down_done[b].record(stream)
+
+    def one(i):
+        bset = sets[i % 2]
+        b = i % 2
+        s_up.wait_event(free_in[b])
+        with torch.cuda.stream(s_up):
+            for d, h in zip(bset["in"], host_in):
+                if d is not None:
+                    d.copy_(h, non_blocking=True)
+        up_done[b].record(s_up)
+        stream.wait_event(up_done[b])
+        stream.wait_event(down_done[b])  # o, hN of set b have been read back
+        dq, dk_, dv_, dg, db, d0, dcu = bset["in"]
+        kda.kda_chunk_fwd(dq, dk_, dv_, dg, db, d0, dcu, Bc, Tc, N, H, dk, dv, C, "bf16",
+                          bset["o"], bset["hN"], ws)
+        free_in[b].record(stream)
+        called[b].record(stream)
+        s_down.wait_event(called[b])
+        with torch.cuda.stream(s_down):
+            bset["ho"].copy_(bset["o"], non_blocking=True)
+            bset["hhN"].copy_(bset["hN"], non_blocking=True)
+        down_done[b].record(s_down)
+
+    for i in range(2):
+        one(i)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    s_up.wait_event(a)
+    for i in range(steps):
+        one(i)
+    stream.wait_event(down_done[(steps - 1) % 2])
+    stream.wait_event(down_done[steps % 2])
+    b_.record(stream)
     torch.cuda.synchronize()
-    t = a.elapsed_time(b) / 1e3 / steps
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg, hb, h0, hcu)
-              if x is not None)
-    d2h = ho.numel() * ho.element_size() + hhN.numel() * hhN.element_size()
+    t = a.elapsed_time(b_) / 1e3 / steps
+    h2d = sum(x.numel() * x.element_size() for x in host_in if x is not None)
+    d2h = sets[0]["ho"].numel() * sets[0]["ho"].element_size() + \
+        sets[0]["hhN"].numel() * sets[0]["hhN"].element_size()
+    del sets
 
     # decode: per step the token's inputs go up and o comes back
     s0 = dcase.steps[0]
@@ -837,9 +872,9 @@ def run_e2e(kda, torch, pc, dcase, dev, stream, steps=10):
     a.record(stream)
     for _ in range(steps):
         dec()
-    b.record(stream)
+    b_.record(stream)
     torch.cuda.synchronize()
-    td = a.elapsed_time(b) / 1e3 / steps
+    td = a.elapsed_time(b_) / 1e3 / steps
     dh2d = sum(x.numel() * x.element_size() for x in hs.values())
     return {"value": total / t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
