@@ -6,17 +6,18 @@ reserved nearly all HBM up front -- and cannot pass a workspace.  This entry
 point uses a static scratch array inside the library instead.  The GPU test
 calls it twice in a row, through the C ABI, on two different problems (so the
 second call runs on scratch the first one left behind) and compares each
-result with kda_chunk_fwd's, and reads the device's free memory around the
+result with kda_chunk_fwd's and with the fp64 oracle's, and reads the device's free memory around the
 calls: the static array is committed by the first call (lazy module loading)
 or before it (eager loading), never by a later one.  This file is collected
 last on purpose.
 """
+import numpy as np
 import pytest
 import torch
 
 import gated_delta_rule_124_b200 as kda
 from gated_delta_rule_124_b200 import workloads as wl
-from tests.helpers import rel_err, tol_for
+from tests.helpers import oracle_prefill, record, rel_err, tol_for
 
 
 def _problem(seed, lens, H, d, C, dtype):
@@ -68,16 +69,24 @@ def test_no_alloc_commits_its_scratch_once():
 
 
 @pytest.mark.gpu
-def test_no_alloc_matches_workspace_entry_point_twice():
-    first = _problem(501, [300, 64, 17], H=4, d=128, C=64, dtype="bf16").to("cuda")
-    second = _problem(502, [90, 1, 200], H=3, d=64, C=32, dtype="f32").to("cuda")
-    for c in (first, second):
+def test_no_alloc_matches_workspace_entry_point_and_oracle_twice():
+    """Each result against kda_chunk_fwd's and, directly, against the fp64
+    oracle on the same inputs."""
+    first = _problem(501, [300, 64, 17], H=4, d=128, C=64, dtype="bf16")
+    second = _problem(502, [90, 1, 200], H=3, d=64, C=32, dtype="f32")
+    for host in (first, second):
+        c = host.to("cuda")
         ref_o, ref_h = _with_workspace(c)
         o, h = _no_alloc(c)
         torch.cuda.synchronize()
         tol = tol_for(c.dtype)
         assert rel_err(o, ref_o.double().cpu().numpy()) <= tol
         assert rel_err(h, ref_h.double().cpu().numpy()) <= tol
+        oo, oh = oracle_prefill(host)
+        lens = [int(x) for x in np.diff(host.cu_host())]
+        name = f"no-alloc prefill: lengths {lens} H={c.H} d={c.dk} C={c.chunk} {c.dtype}"
+        assert record(name, "o", o, oo) <= tol
+        assert record(name, "final_state", h, oh) <= tol
 
 
 def test_no_alloc_rejects_problems_beyond_the_scratch():
