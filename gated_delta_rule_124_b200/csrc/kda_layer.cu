@@ -16,6 +16,7 @@
 #include <stdint.h>
 
 #include "kda_common.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 namespace {
@@ -295,6 +296,92 @@ __global__ void __launch_bounds__(32 * kWarps) conv_swish_kernel(
     }
 }
 
+// bf16, d = 128 (q, k and v): the same warp per (tensor, head, run of kRun
+// tokens), but the run's rows and the three before it are first copied into
+// the warp's part of shared memory at once (16-byte cp.async, 35 rows of 256 B;
+// zeros outside [0, total)), so that every warp has its whole run in flight
+// instead of one row ahead; the sliding window then reads the rows there.
+constexpr int kStageRows = kRun + 3;
+constexpr int kStageBytes = kWarps * kStageRows * 128 * 2;
+
+__global__ void __launch_bounds__(32 * kWarps) conv_staged_kernel(
+    const ConvArgs a, const int32_t* __restrict__ cu, int N, int T, int total, int H, float eps) {
+    constexpr int D = 128, CPL = 4;
+    extern __shared__ __align__(16) uint8_t conv_smem[];
+    const int tensor = blockIdx.y;  // 0 q, 1 k, 2 v
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c0 = lane * CPL;
+    const long long task = (long long)blockIdx.x * kWarps + warp;
+    const long long runs = (total + kRun - 1) / kRun;
+    if (task >= runs * H) return;  // (per warp; no block-wide barrier below)
+    const int h = static_cast<int>(task % H), t0 = static_cast<int>(task / H) * kRun;
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(
+        tensor == 0 ? a.x[0] : tensor == 1 ? a.x[1] : a.x[2]);
+    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(tensor == 0 ? a.y[0] : tensor == 1 ? a.y[1] : a.y[2]);
+    const float* w = tensor == 0 ? a.w[0] : tensor == 1 ? a.w[1] : a.w[2];
+    const bool l2 = tensor < 2;
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(conv_smem) + warp * kStageRows * D;
+    for (int e = lane; e < kStageRows * (D / 8); e += 32) {  // rows t0 - 3 .. t0 + kRun - 1
+        const int row = e >> 4, ch = e & 15, t = t0 - 3 + row;
+        __nv_bfloat16* dst = xs + row * D + ch * 8;
+        if (t >= 0 && t < total)
+            sm100::cp_async16(dst, x + ((size_t)t * H + h) * D + ch * 8);
+        else
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    sm100::cp_async_commit();
+    float wt[CPL][4];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        const float4 v = *reinterpret_cast<const float4*>(w + ((size_t)h * D + c0 + j) * 4);
+        wt[j][0] = v.x; wt[j][1] = v.y; wt[j][2] = v.z; wt[j][3] = v.w;
+    }
+    int s = warp_seq_of(cu, N, T, t0, lane);
+    int begin = seq_begin(cu, T, s), end = seq_end(cu, T, s);
+    sm100::cp_async_wait_all();
+    __syncwarp();
+    float win[3][CPL];  // inputs of tokens t - 3, t - 2, t - 1
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        Vec<CPL, __nv_bfloat16>::load(xs + i * D + c0, win[i]);
+        if (t0 - 3 + i < begin)
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) win[i][j] = 0.f;
+    }
+    const int t1 = min(total, t0 + kRun);
+    for (int t = t0; t < t1; ++t) {
+        float cur[CPL];
+        Vec<CPL, __nv_bfloat16>::load(xs + (t - t0 + 3) * D + c0, cur);
+        while (t >= end && s < N - 1) {  // t starts a new sequence: no history
+            ++s;
+            begin = seq_begin(cu, T, s);
+            end = seq_end(cu, T, s);
+#pragma unroll
+            for (int i = 0; i < 3; ++i)
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) win[i][j] = 0.f;
+        }
+        float out[CPL], ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            float acc = wt[j][3] * cur[j];
+            acc = fmaf(wt[j][2], win[2][j], acc);
+            acc = fmaf(wt[j][1], win[1][j], acc);
+            acc = fmaf(wt[j][0], win[0][j], acc);
+            out[j] = swish_for<__nv_bfloat16>(acc);
+            ss = fmaf(out[j], out[j], ss);
+            win[0][j] = win[1][j];
+            win[1][j] = win[2][j];
+            win[2][j] = cur[j];
+        }
+        if (l2) {
+            const float inv = rsqrtf(warp_sum(ss) + eps);
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) out[j] *= inv;
+        }
+        Vec<CPL, __nv_bfloat16>::store(y + ((size_t)t * H + h) * D + c0, out);
+    }
+}
+
 // y = o / sqrt(mean o^2 + eps) * w * sigmoid(gate), per (token, head); a warp
 // takes kPairs consecutive (token, head) rows, all loads issued first.
 constexpr int kPairs = 4;
@@ -383,7 +470,12 @@ cudaError_t launch_qkv_conv(const void* const x[3], const float* const w[3], voi
     }
     const long long runs = (total + kRun - 1) / kRun;
     const dim3 grid(static_cast<unsigned>((runs * H + kWarps - 1) / kWarps), 3);
-    if (dt == KDA_DTYPE_BF16)
+    if (dt == KDA_DTYPE_BF16 && dk == 128 && dv == 128) {
+        const cudaError_t attr = cudaFuncSetAttribute(
+            conv_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBytes);
+        if (attr != cudaSuccess) return attr;
+        conv_staged_kernel<<<grid, 32 * kWarps, kStageBytes, st>>>(a, cu, N, T, total, H, eps);
+    } else if (dt == KDA_DTYPE_BF16)
         conv_swish_kernel<__nv_bfloat16><<<grid, 32 * kWarps, 0, st>>>(a, cu, N, T, total, H, eps);
     else
         conv_swish_kernel<float><<<grid, 32 * kWarps, 0, st>>>(a, cu, N, T, total, H, eps);
